@@ -1,0 +1,233 @@
+"""CPU oracle for the MoonEP hot path -- TEST INFRASTRUCTURE ONLY.
+
+A plain, slow, single-threaded C implementation (``moonep_oracle.c``) of the
+plan, dispatch, combine, combine-backward and replica-gradient reduction,
+wrapped here with ctypes and numpy.  Only the test suite, the smoke check
+and the benchmark's CPU-baseline / reference legs may import this package;
+the product (``load_balancing_moonep_b200``) never does, and this package
+never imports the product.
+
+The pages the oracle follows (cited by title and section) are listed in the
+header of ``moonep_oracle.c``; each function below names the passage it
+implements.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moonep_oracle.c")
+_LIB = os.path.join(_HERE, "libmoonep_oracle.so")
+
+FLAG_STRICT_BUDGET = 1
+FLAG_TRAIN_B_RULE = 2
+FLAG_BWD_UNSCALED = 4
+
+ST_EXPERT_ID_RANGE = 1
+ST_OVERFLOW = 2
+ST_STRICT_VIOLATION = 4
+
+INFO_FIELDS = (
+    "status", "n_rep", "n_overflow", "n_pieces", "n_receivers",
+    "max_rep_per_rank", "n_rep_experts", "n_remote_pairs",
+)
+INFO_LEN = 16
+
+ERRORS = {0: "ok", 1: "bad argument", 2: "E not divisible by R",
+          3: "training budget rule B == E/R violated", 4: "B out of range",
+          6: "out of host memory"}
+
+
+class OracleError(RuntimeError):
+    pass
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (plain C11, -O2, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-std=c11", "-O2", "-fno-fast-math", "-ffp-contract=off",
+               "-fPIC", "-shared", "-o", _LIB, _SRC, "-lm"]
+        subprocess.check_call(cmd)
+    return _LIB
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        lib.or_plan.argtypes = [ctypes.c_void_p] + [ctypes.c_void_p] * 18
+        lib.or_plan.restype = ctypes.c_int
+        lib.or_check_config.argtypes = [ctypes.c_void_p]
+        lib.or_check_config.restype = ctypes.c_int
+        lib.or_dispatch.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int64] * 2
+        lib.or_dispatch.restype = ctypes.c_int
+        lib.or_combine.argtypes = [ctypes.c_void_p] * 6 + [ctypes.c_int64] * 2
+        lib.or_combine.restype = ctypes.c_int
+        lib.or_combine_backward.argtypes = [ctypes.c_void_p] * 8 + [ctypes.c_int64] * 2
+        lib.or_combine_backward.restype = ctypes.c_int
+        lib.or_reduce_replica_grads.argtypes = [ctypes.c_void_p] * 7 + [ctypes.c_int64] * 3
+        lib.or_reduce_replica_grads.restype = ctypes.c_int
+        lib.or_f32_to_bf16.argtypes = [ctypes.c_float]
+        lib.or_f32_to_bf16.restype = ctypes.c_uint16
+        _lib = lib
+    return _lib
+
+
+class _Cfg(ctypes.Structure):
+    _fields_ = [("R", ctypes.c_int32), ("E", ctypes.c_int32), ("K", ctypes.c_int32),
+                ("S", ctypes.c_int32), ("H", ctypes.c_int32), ("B", ctypes.c_int32),
+                ("flags", ctypes.c_uint32)]
+
+
+@dataclass(frozen=True)
+class Config:
+    R: int
+    E: int
+    K: int
+    S: int
+    H: int
+    B: int
+    flags: int = 0
+
+    @property
+    def L(self) -> int:
+        return self.E // self.R
+
+    @property
+    def C(self) -> int:
+        return self.S * self.K
+
+    def _c(self) -> _Cfg:
+        return _Cfg(self.R, self.E, self.K, self.S, self.H, self.B, self.flags)
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _check(rc: int):
+    if rc != 0:
+        raise OracleError(f"oracle error {rc}: {ERRORS.get(rc, '?')}")
+
+
+def check_config(cfg: Config) -> int:
+    c = cfg._c()
+    return _load().or_check_config(ctypes.byref(c))
+
+
+def f32_to_bf16(x: float) -> int:
+    """Round-to-nearest-even fp32 -> bf16 bit pattern (oracle's own routine)."""
+    return int(_load().or_f32_to_bf16(ctypes.c_float(x)))
+
+
+def plan(cfg: Config, topk_idx: np.ndarray) -> dict:
+    """Steps O1-O8 of the plan (redundant experts planned online from the
+    router output so every rank receives exactly S*K slots; MoonEP article,
+    'The core idea: dynamic redundant experts').  Returns a dict of numpy
+    int32 arrays with the same fields and shapes as the CUDA library's plan."""
+    lib = _load()
+    R, E, K, S = cfg.R, cfg.E, cfg.K, cfg.S
+    topk = np.ascontiguousarray(topk_idx, dtype=np.int32).reshape(R * S, K)
+    out = {
+        "expert_count": np.zeros(E, np.int32),
+        "slot_expert": np.zeros((R, E), np.int32),
+        "slot_count": np.zeros((R, E), np.int32),
+        "slot_offset": np.zeros((R, E + 1), np.int32),
+        "rep_expert": np.zeros(E + R, np.int32),
+        "rep_rank": np.zeros(E + R, np.int32),
+        "rep_slot": np.zeros(E + R, np.int32),
+        "rep_quota": np.zeros(E + R, np.int32),
+        "host_ptr": np.zeros(E + 1, np.int32),
+        "host_rank": np.zeros(2 * E + R, np.int32),
+        "host_slot": np.zeros(2 * E + R, np.int32),
+        "host_start": np.zeros(2 * E + R, np.int32),
+        "host_quota": np.zeros(2 * E + R, np.int32),
+        "rep_home_list": np.zeros(E, np.int32),
+        "dst_pos": np.zeros((R * S, K), np.int32),
+        "row_src": np.zeros(R * S * K, np.int32),
+        "info": np.zeros(INFO_LEN, np.int32),
+    }
+    c = cfg._c()
+    rc = lib.or_plan(ctypes.byref(c), _p(topk),
+                     _p(out["expert_count"]), _p(out["slot_expert"]), _p(out["slot_count"]),
+                     _p(out["slot_offset"]), _p(out["rep_expert"]), _p(out["rep_rank"]),
+                     _p(out["rep_slot"]), _p(out["rep_quota"]), _p(out["host_ptr"]),
+                     _p(out["host_rank"]), _p(out["host_slot"]), _p(out["host_start"]),
+                     _p(out["host_quota"]), _p(out["rep_home_list"]), _p(out["dst_pos"]),
+                     _p(out["row_src"]), _p(out["info"]))
+    _check(rc)
+    return out
+
+
+def info_dict(p: dict) -> dict:
+    return {k: int(p["info"][i]) for i, k in enumerate(INFO_FIELDS)}
+
+
+def dispatch(cfg: Config, p: dict, hidden_bits: np.ndarray, buf_bits: np.ndarray,
+             t0: int = 0, t1: int | None = None) -> np.ndarray:
+    """Zero-copy permute: hidden row t lands in buffer row dst_pos[t, k] for
+    every k (MoonEP article, 'The core idea', zero copy and static shapes).
+    hidden_bits: uint16 [R*S, H]; buf_bits: uint16 [R, S*K, H] (written in place)."""
+    lib = _load()
+    t1 = cfg.R * cfg.S if t1 is None else t1
+    assert hidden_bits.dtype == np.uint16 and hidden_bits.flags.c_contiguous
+    assert buf_bits.dtype == np.uint16 and buf_bits.flags.c_contiguous
+    c = cfg._c()
+    _check(lib.or_dispatch(ctypes.byref(c), _p(p["dst_pos"]), _p(p["info"]),
+                           _p(hidden_bits), _p(buf_bits), t0, t1))
+    return buf_bits
+
+
+def combine(cfg: Config, p: dict, y_bits: np.ndarray, w: np.ndarray,
+            out_bits: np.ndarray | None = None, t0: int = 0, t1: int | None = None) -> np.ndarray:
+    """Weighted unpermute with fp32 fused multiply-add accumulation in k order
+    and one bf16 rounding.  y_bits: uint16 [R, S*K, H]; w: float32 [R*S, K]."""
+    lib = _load()
+    t1 = cfg.R * cfg.S if t1 is None else t1
+    if out_bits is None:
+        out_bits = np.zeros((cfg.R * cfg.S, cfg.H), np.uint16)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    c = cfg._c()
+    _check(lib.or_combine(ctypes.byref(c), _p(p["dst_pos"]), _p(p["info"]), _p(y_bits),
+                          _p(w), _p(out_bits), t0, t1))
+    return out_bits
+
+
+def combine_backward(cfg: Config, p: dict, dy_bits: np.ndarray, w: np.ndarray,
+                     y_bits: np.ndarray, dy_buf_bits: np.ndarray, dw: np.ndarray,
+                     t0: int = 0, t1: int | None = None):
+    """Backward of the combine: scaled dispatch of dy, and dw[t,k] = <dy[t], y[dst_pos[t,k]]>."""
+    lib = _load()
+    t1 = cfg.R * cfg.S if t1 is None else t1
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    assert dw.dtype == np.float32 and dw.flags.c_contiguous
+    c = cfg._c()
+    _check(lib.or_combine_backward(ctypes.byref(c), _p(p["dst_pos"]), _p(p["info"]),
+                                   _p(dy_bits), _p(w), _p(y_bits), _p(dy_buf_bits), _p(dw),
+                                   t0, t1))
+    return dy_buf_bits, dw
+
+
+def reduce_replica_grads(cfg: Config, p: dict, reduce_buf: np.ndarray, home_grad: np.ndarray,
+                         P: int, i0: int = 0, i1: int | None = None):
+    """Sum prefetched replicas' fp32 grads into their home expert, ascending
+    host rank order, then zero the replica rows (MoonEP article explainer,
+    memory tab, training branch).  reduce_buf: f32 [R, B, P]; home_grad: f32 [E, P]."""
+    lib = _load()
+    i1 = P if i1 is None else i1
+    assert reduce_buf.dtype == np.float32 and reduce_buf.flags.c_contiguous
+    assert home_grad.dtype == np.float32 and home_grad.flags.c_contiguous
+    c = cfg._c()
+    _check(lib.or_reduce_replica_grads(ctypes.byref(c), _p(p["host_ptr"]), _p(p["host_rank"]),
+                                       _p(p["host_slot"]), _p(p["info"]), _p(reduce_buf),
+                                       _p(home_grad), P, i0, i1))
+    return reduce_buf, home_grad

@@ -1,0 +1,430 @@
+"""Pins for the CPU oracle: it is checked against things other than itself.
+
+* hand-worked plans (tests/golden/plan_example_*.json);
+* the constraints the pages fix (exact S*K slots per rank, pairs only on
+  ranks hosting their expert, replica budget) on many random routings;
+* closed forms: balanced routing needs no replica and places pairs in
+  home-grouped order; all tokens on one expert with K=1 gives R-1 replicas
+  of quota S and the identity placement;
+* brute-force optimum on micro routings: max(P, N) <= OPT <= greedy <= P+N-1;
+* library routines for the floating-point steps (torch's bf16 rounding,
+  numpy's fp64 dot, numpy fp32 products) and exact integer-valued cases.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bruteforce import min_cover_count, min_replicas
+from load_balancing_moonep_b200 import workloads as W
+from plan_checks import check_invariants, check_water_filling
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _cfg(wl, flags=0, **kw):
+    d = dict(R=wl.R, E=wl.E, K=wl.K, S=wl.S, H=wl.H, B=wl.B, flags=flags)
+    d.update(kw)
+    return oracle.Config(**d)
+
+
+# ------------------------------------------------------------- golden plans
+
+@pytest.mark.parametrize("name", ["plan_example_a", "plan_example_b"])
+def test_golden_plan(oracle_lib, name):
+    g = json.load(open(os.path.join(GOLDEN, name + ".json")))
+    cfg = oracle.Config(**g["config"])
+    topk = np.array(g["topk_idx"], np.int32)
+    p = oracle.plan(cfg, topk)
+    exp = g["expect"]
+    for k, v in exp.items():
+        if k == "info":
+            assert oracle.info_dict(p) == v
+        else:
+            assert p[k].tolist() == v, k
+    check_invariants(cfg, topk, p)
+    check_water_filling(cfg, topk, p)
+
+
+def test_golden_b_strict_flag(oracle_lib):
+    g = json.load(open(os.path.join(GOLDEN, "plan_example_b.json")))
+    cfg = oracle.Config(**{**g["config"], "flags": oracle.FLAG_STRICT_BUDGET})
+    p = oracle.plan(cfg, np.array(g["topk_idx"], np.int32))
+    assert p["info"][0] == oracle.ST_OVERFLOW | oracle.ST_STRICT_VIOLATION
+    # the plan itself does not change under strict mode
+    p0 = oracle.plan(oracle.Config(**g["config"]), np.array(g["topk_idx"], np.int32))
+    for k in p:
+        if k != "info":
+            assert np.array_equal(p[k], p0[k])
+
+
+# --------------------------------------------------------- config checking
+
+def test_config_errors(oracle_lib):
+    ok = oracle.Config(R=4, E=16, K=2, S=8, H=8, B=2)
+    assert oracle.check_config(ok) == 0
+    assert oracle.check_config(oracle.Config(R=3, E=16, K=2, S=8, H=8, B=2)) == 2
+    assert oracle.check_config(oracle.Config(R=4, E=16, K=2, S=8, H=8, B=3,
+                                             flags=oracle.FLAG_TRAIN_B_RULE)) == 3
+    assert oracle.check_config(oracle.Config(R=4, E=16, K=2, S=8, H=8, B=4,
+                                             flags=oracle.FLAG_TRAIN_B_RULE)) == 0
+    assert oracle.check_config(oracle.Config(R=4, E=16, K=2, S=8, H=8, B=13)) == 4
+    assert oracle.check_config(oracle.Config(R=4, E=16, K=17, S=8, H=8, B=2)) == 1
+    assert oracle.check_config(oracle.Config(R=0, E=16, K=2, S=8, H=8, B=2)) == 1
+
+
+def test_bad_expert_id(oracle_lib):
+    cfg = oracle.Config(R=2, E=4, K=2, S=4, H=8, B=1)
+    topk = np.zeros((8, 2), np.int32)
+    topk[3, 1] = 4
+    p = oracle.plan(cfg, topk)
+    assert p["info"][0] == oracle.ST_EXPERT_ID_RANGE
+    assert (p["dst_pos"] == -1).all() and (p["row_src"] == -1).all()
+    assert (p["slot_count"] == 0).all() and p["info"][1] == 0
+    assert p["expert_count"].tolist() == [15, 0, 0, 0]
+    topk[3, 1] = -1
+    assert oracle.plan(cfg, topk)["info"][0] == oracle.ST_EXPERT_ID_RANGE
+
+
+# ------------------------------------------------------ invariants, random
+
+def _random_topk(rng, R, E, K, S, skew):
+    # distinct experts per token drawn with Zipf-like weights
+    w = np.arange(1, E + 1, dtype=np.float64) ** (-skew)
+    w = w[rng.permutation(E)]
+    w /= w.sum()
+    out = np.empty((R * S, K), np.int32)
+    for t in range(R * S):
+        out[t] = rng.choice(E, size=K, replace=False, p=w)
+    return out
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_invariants_random(oracle_lib, seed):
+    rng = np.random.default_rng(seed)
+    R = int(rng.choice([2, 3, 4, 8]))
+    L = int(rng.choice([1, 2, 3, 4]))
+    E = R * L
+    K = int(rng.integers(1, min(E, 4) + 1))
+    S = int(rng.integers(1, 40))
+    B = int(rng.integers(0, E - L + 1))
+    cfg = oracle.Config(R=R, E=E, K=K, S=S, H=8, B=B)
+    topk = _random_topk(rng, R, E, K, S, skew=float(rng.uniform(0, 2.5)))
+    p = oracle.plan(cfg, topk)
+    check_invariants(cfg, topk, p)
+    check_water_filling(cfg, topk, p)
+
+
+@pytest.mark.parametrize("mv", [0.0, 0.5, 1.0, 2.0, 3.0])
+def test_invariants_mid(oracle_lib, mv):
+    wl = W.WORKLOADS["mid"]
+    r = W.routing(wl, mv)
+    cfg = _cfg(wl)
+    topk = r.topk_idx.numpy()
+    p = oracle.plan(cfg, topk)
+    check_invariants(cfg, topk, p)
+    check_water_filling(cfg, topk, p)
+    if mv == 0.0:
+        assert p["info"][1] == 0
+
+
+def test_invariants_tiny_and_adversarial(oracle_lib):
+    wl = W.WORKLOADS["tiny"]
+    for adv in (False, True):
+        r = W.routing(wl, 1.0, adversarial=adv)
+        cfg = _cfg(wl)
+        p = oracle.plan(cfg, r.topk_idx.numpy())
+        check_invariants(cfg, r.topk_idx.numpy(), p)
+        check_water_filling(cfg, r.topk_idx.numpy(), p)
+
+
+# ------------------------------------------------------------ closed forms
+
+def test_balanced_no_replicas_and_home_order(oracle_lib):
+    # T[e] = C/L for all e: no replica; each expert's pairs fill its home slot
+    # in (t, k) order, so dst = home*C + (e mod L)*(C/L) + rank-within-expert.
+    R, L, K, S = 4, 3, 3, 16
+    E = R * L
+    cfg = oracle.Config(R=R, E=E, K=K, S=S, H=8, B=2)
+    p_idx = np.arange(R * S * K)
+    topk = (p_idx % E).astype(np.int32).reshape(R * S, K)
+    p = oracle.plan(cfg, topk)
+    assert p["info"][1] == 0 and p["info"][0] == 0
+    flat = topk.ravel()
+    order = np.argsort(flat, kind="stable")
+    g = np.empty_like(order)
+    for e in range(E):
+        m = flat[order] == e
+        g[order[m]] = np.arange(m.sum())
+    C = S * K
+    expect = (flat // L) * C + (flat % L) * (C // L) + g
+    assert np.array_equal(p["dst_pos"].ravel(), expect)
+
+
+def test_rank_balanced_skewed_experts_no_replicas(oracle_lib):
+    # maxvio > 0 but every rank's home load is exactly C: no replica needed
+    R, L, K, S = 4, 2, 1, 6
+    E = R * L
+    cfg = oracle.Config(R=R, E=E, K=K, S=S, H=8, B=1)
+    topk = np.array([[2 * (t // S) + (0 if t % S < 5 else 1)] for t in range(R * S)], np.int32)
+    T = np.bincount(topk.ravel(), minlength=E)
+    assert W.maxvio_of_counts(T, R, S, K, E) > 0.5
+    p = oracle.plan(cfg, topk)
+    assert p["info"][1] == 0
+    check_invariants(cfg, topk, p)
+
+
+@pytest.mark.parametrize("R,L,S", [(2, 1, 3), (4, 2, 5), (8, 3, 7)])
+def test_all_on_one_expert(oracle_lib, R, L, S):
+    # K=1, every token picks expert 0: R-1 replicas of quota S, one per
+    # non-home rank in ascending rank order, and dst_pos is the identity.
+    E = R * L
+    cfg = oracle.Config(R=R, E=E, K=1, S=S, H=8, B=1)
+    topk = np.zeros((R * S, 1), np.int32)
+    p = oracle.plan(cfg, topk)
+    n = p["info"][1]
+    assert n == R - 1
+    assert p["rep_expert"][:n].tolist() == [0] * (R - 1)
+    assert p["rep_rank"][:n].tolist() == list(range(1, R))
+    assert p["rep_quota"][:n].tolist() == [S] * (R - 1)
+    assert np.array_equal(p["dst_pos"].ravel(), np.arange(R * S))
+    assert np.array_equal(p["row_src"], np.arange(R * S))
+
+
+# ------------------------------------------------------------- brute force
+
+def test_bruteforce_optimality_bounds(oracle_lib):
+    rng = np.random.default_rng(7)
+    gaps = []
+    for trial in range(300):
+        R = int(rng.choice([2, 3]))
+        L = int(rng.choice([1, 2]))
+        E = R * L
+        S = int(rng.integers(1, 7))
+        C = S  # K = 1
+        cfg = oracle.Config(R=R, E=E, K=1, S=S, H=8, B=E - L)
+        topk = rng.integers(0, E, size=(R * S, 1)).astype(np.int32)
+        p = oracle.plan(cfg, topk)
+        T = np.bincount(topk.ravel(), minlength=E).tolist()
+        opt = min_replicas(T, R, L, C)
+        P, N = int(p["info"][3]), int(p["info"][4])
+        greedy = int(p["info"][1])
+        assert max(P, N) <= opt <= greedy <= max(P + N - 1, 0)
+        gaps.append(greedy - opt)
+        # largest-first shedding: each donor sheds the fewest possible experts
+        Hl = np.array(T).reshape(R, L).sum(axis=1)
+        for r in range(R):
+            X = Hl[r] - C
+            if X > 0:
+                vals = T[r * L:(r + 1) * L]
+                n_shed = sum(1 for e in range(r * L, (r + 1) * L)
+                             if any(p["rep_expert"][q] == e for q in range(greedy)))
+                assert n_shed == min_cover_count(vals, X)
+    assert max(gaps) <= 2
+
+
+# ------------------------------------------------------------ data steps
+
+def test_bf16_rounding_matches_torch(oracle_lib):
+    rng = np.random.default_rng(3)
+    vals = np.concatenate([
+        rng.standard_normal(4000).astype(np.float32),
+        (rng.standard_normal(2000) * 1e30).astype(np.float32),
+        (rng.standard_normal(2000) * 1e-39).astype(np.float32),   # subnormals
+        np.array([0.0, -0.0, np.inf, -np.inf, 3.3895314e38, 1.0, -1.0], np.float32),
+    ])
+    # exact ties: bf16 value + half an ulp (even and odd last kept bit)
+    base = rng.integers(0, 0x7f00, size=2000).astype(np.uint32) << 16
+    ties = (base | 0x8000).view(np.float32)
+    vals = np.concatenate([vals, ties, (base | 0x18000).view(np.float32)])
+    ref = torch.from_numpy(vals).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = np.array([oracle.f32_to_bf16(float(v)) for v in vals], np.uint16)
+    assert np.array_equal(got, ref)
+    nan = oracle.f32_to_bf16(float("nan"))
+    assert (nan & 0x7f80) == 0x7f80 and (nan & 0x7f) != 0
+
+
+def _tiny_plan(seed=0, mv=1.0):
+    wl = W.WORKLOADS["tiny"]
+    cfg = _cfg(wl)
+    r = W.routing(wl, mv, seed=seed)
+    p = oracle.plan(cfg, r.topk_idx.numpy())
+    return wl, cfg, r, p
+
+
+def test_dispatch_rows(oracle_lib):
+    wl, cfg, r, p = _tiny_plan()
+    x = W.bits(W.hidden_states(wl, seed=5))
+    buf = np.full((wl.R, wl.C, wl.H), 0xFFFF, np.uint16)
+    oracle.dispatch(cfg, p, x, buf)
+    rows = buf.reshape(-1, wl.H)
+    # every row written exactly once, with the hidden row of the token that owns it
+    tok = p["row_src"] // wl.K
+    assert np.array_equal(rows, x[tok])
+    # and each rank's slot holds exactly the tokens routed to the slot's expert
+    check_invariants(cfg, r.topk_idx.numpy(), p)
+
+
+def test_combine_closed_forms(oracle_lib):
+    wl, cfg, r, p = _tiny_plan()
+    x = W.bits(W.hidden_states(wl, seed=5))
+    buf = np.zeros((wl.R, wl.C, wl.H), np.uint16)
+    oracle.dispatch(cfg, p, x, buf)
+    K = wl.K
+    # one-hot weights select one copy exactly
+    for k0 in range(K):
+        w = np.zeros((wl.tokens, K), np.float32)
+        w[:, k0] = 1.0
+        assert np.array_equal(oracle.combine(cfg, p, buf, w), x)
+    # unit weights: K copies of x summed; K = 2 so the sum is exact in fp32 and bf16
+    w = np.ones((wl.tokens, K), np.float32)
+    out = oracle.combine(cfg, p, buf, w)
+    ref = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).float() * K
+    assert np.array_equal(out, ref.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16))
+
+
+def test_combine_error_bound(oracle_lib):
+    # random y and weights: the result is within half a bf16 ulp plus the fp32
+    # accumulation bound of the exact (fp64) weighted sum
+    wl, cfg, r, p = _tiny_plan(seed=1)
+    y = W.bits(W.bf16_normal((wl.R, wl.C, wl.H), seed=9))
+    w = r.weights.numpy()
+    out = oracle.combine(cfg, p, y, w)
+    yf = torch.from_numpy(y.view(np.int16)).view(torch.bfloat16).double().numpy().reshape(-1, wl.H)
+    exact = np.einsum("tk,tkh->th", w.astype(np.float64), yf[p["dst_pos"]])
+    mag = np.einsum("tk,tkh->th", np.abs(w.astype(np.float64)), np.abs(yf[p["dst_pos"]]))
+    of = torch.from_numpy(out.view(np.int16)).view(torch.bfloat16).double().numpy()
+    ulp_half = np.maximum(np.abs(of), np.abs(exact)) * 2.0 ** -8
+    bound = ulp_half + wl.K * 2.0 ** -24 * mag + 1e-38
+    assert (np.abs(of - exact) <= bound).all()
+    # softmax weights sum to one: combine(dispatch(x)) is x up to rounding
+    x = W.bits(W.hidden_states(wl, seed=5))
+    buf = np.zeros((wl.R, wl.C, wl.H), np.uint16)
+    oracle.dispatch(cfg, p, x, buf)
+    o2 = torch.from_numpy(oracle.combine(cfg, p, buf, w).view(np.int16)).view(torch.bfloat16).double()
+    xf = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).double()
+    assert torch.all(torch.abs(o2 - xf) <= torch.abs(xf) * 2.0 ** -7 + 1e-30)
+
+
+def test_combine_backward_library(oracle_lib):
+    wl, cfg, r, p = _tiny_plan(seed=2)
+    dy = W.bits(W.bf16_normal((wl.tokens, wl.H), seed=11))
+    y = W.bits(W.bf16_normal((wl.R, wl.C, wl.H), seed=12))
+    w = r.weights.numpy()
+    dy_buf = np.zeros((wl.R, wl.C, wl.H), np.uint16)
+    dw = np.zeros((wl.tokens, wl.K), np.float32)
+    oracle.combine_backward(cfg, p, dy, w, y, dy_buf, dw)
+    dyf = torch.from_numpy(dy.view(np.int16)).view(torch.bfloat16).float().numpy()
+    yf = torch.from_numpy(y.view(np.int16)).view(torch.bfloat16).float().numpy().reshape(-1, wl.H)
+    # dy_buf row of (t, k) = bf16(fp32 product w * dy) via numpy and torch rounding
+    prod = (w[:, :, None] * dyf[:, None, :]).astype(np.float32)
+    ref = torch.from_numpy(prod).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    rows = dy_buf.reshape(-1, wl.H)
+    assert np.array_equal(rows[p["dst_pos"]], ref)
+    # dw against numpy's fp64 dot
+    ref_dw = np.einsum("th,tkh->tk", dyf.astype(np.float64), yf[p["dst_pos"]].astype(np.float64))
+    assert np.allclose(dw, ref_dw.astype(np.float32), rtol=0, atol=0) or \
+        np.all(np.abs(dw - ref_dw) <= 1e-6 * np.abs(ref_dw) + 1e-30)
+    # unscaled variant dispatches dy itself
+    cfg_u = oracle.Config(**{**cfg.__dict__, "flags": oracle.FLAG_BWD_UNSCALED})
+    dy_buf2 = np.zeros_like(dy_buf)
+    oracle.combine_backward(cfg_u, p, dy, w, y, dy_buf2, dw)
+    assert np.array_equal(dy_buf2.reshape(-1, wl.H)[p["dst_pos"]],
+                          np.repeat(dy[:, None, :], wl.K, axis=1))
+
+
+def test_reduce_exact_integers(oracle_lib):
+    g = json.load(open(os.path.join(GOLDEN, "plan_example_b.json")))
+    cfg = oracle.Config(**{**g["config"], "B": 3})  # all four replicas prefetched
+    p = oracle.plan(cfg, np.array(g["topk_idx"], np.int32))
+    R, E, B, P = cfg.R, cfg.E, cfg.B, 37
+    L = E // R
+    rb = np.zeros((R, B, P), np.float32)
+    for r in range(R):
+        for b in range(B):
+            rb[r, b] = 1000 * r + 100 * b + np.arange(P)
+    home = np.tile(np.arange(E, dtype=np.float32)[:, None] * 1e4, (1, P))
+    rb0, home0 = rb.copy(), home.copy()
+    oracle.reduce_replica_grads(cfg, p, rb, home, P)
+    # replicas: (e6, r0, slot 2 -> b0), (e6, r1, b0), (e4, r1, b1), (e7, r1, b2)
+    exp = home0.copy()
+    exp[6] += rb0[0, 0] + rb0[1, 0]
+    exp[4] += rb0[1, 1]
+    exp[7] += rb0[1, 2]
+    assert np.array_equal(home, exp)
+    used = {(0, 0), (1, 0), (1, 1), (1, 2)}
+    for r in range(R):
+        for b in range(B):
+            if (r, b) in used:
+                assert (rb[r, b] == 0).all()
+            else:
+                assert np.array_equal(rb[r, b], rb0[r, b])
+    # with B = 1 the overflow replicas have no reduce rows and are skipped
+    cfg1 = oracle.Config(**g["config"])
+    p1 = oracle.plan(cfg1, np.array(g["topk_idx"], np.int32))
+    rb1 = rb0[:, :1].copy()
+    h1 = home0.copy()
+    oracle.reduce_replica_grads(cfg1, p1, rb1, h1, P)
+    exp1 = home0.copy()
+    exp1[6] += rb0[0, 0] + rb0[1, 0]
+    assert np.array_equal(h1, exp1)
+    del L
+
+
+def test_reduce_order_is_rank_ascending(oracle_lib):
+    # values chosen so that fp32 addition is not associative: the result must
+    # equal ((home + rep_rank0) + rep_rank1), in ascending host rank order
+    g = json.load(open(os.path.join(GOLDEN, "plan_example_b.json")))
+    cfg = oracle.Config(**g["config"])
+    p = oracle.plan(cfg, np.array(g["topk_idx"], np.int32))
+    R, B, E, P = cfg.R, cfg.B, cfg.E, 4
+    rb = np.zeros((R, B, P), np.float32)
+    rb[0, 0] = np.float32(1.0)
+    rb[1, 0] = np.float32(-1e8)
+    home = np.zeros((E, P), np.float32)
+    home[6] = np.float32(1e8)
+    oracle.reduce_replica_grads(cfg, p, rb, home, P)
+    expect = (np.float32(1e8) + np.float32(1.0)) + np.float32(-1e8)
+    assert (home[6] == expect).all()
+
+
+# ------------------------------------------------------- generator metric
+
+def test_maxvio_definition_and_hottest_table():
+    # maxvio = max_e T_e / T_bar - 1, T_bar = S*K*R/E (explainer, maxvio tab)
+    R, S, K, E = 8, 4096, 8, 256
+    t_bar = S * K * R / E
+    T = np.full(E, t_bar)
+    assert W.maxvio_of_counts(T, R, S, K, E) == 0.0
+    for mv in (0.2, 1.0, 10.0, 20.0):
+        hot = W.hottest_expert_count(mv, S, K, R, E)
+        assert hot == round((1 + mv) * t_bar)
+        T2 = T.copy()
+        T2[3] = hot
+        assert abs(W.maxvio_of_counts(T2, R, S, K, E) - mv) <= 0.5 / t_bar
+
+
+def test_combine_uses_fused_multiply_add(oracle_lib):
+    # One token, two experts, no replicas (R = 1).  y0 = -1 and w0 = fp32(w1*y1),
+    # so after k = 0 the accumulator is exactly -fp32(w1*y1); a fused
+    # multiply-add at k = 1 leaves the (nonzero) rounding error of w1*y1,
+    # a separate multiply then add leaves exactly 0.  The expected value is
+    # the exact real w1*y1 - w0 (fits in fp64) rounded once to bf16.
+    cfg = oracle.Config(R=1, E=2, K=2, S=1, H=8, B=0)
+    p = oracle.plan(cfg, np.array([[0, 1]], np.int32))
+    assert p["dst_pos"].tolist() == [[0, 1]]
+    y1 = np.float32(1.0 + 2.0 ** -7)
+    w1 = np.float32(1.0 + 2.0 ** -17 + 2.0 ** -23)
+    w0 = np.float32(w1 * y1)
+    exact = float(w1) * float(y1) - float(w0)
+    assert exact != 0.0
+    y = np.zeros((1, 2, 8), np.uint16)
+    y[0, 0, :] = 0xBF80                      # bf16 -1.0
+    y[0, 1, :] = np.array([y1], np.float32).view(np.uint32)[0] >> 16
+    w = np.array([[w0, w1]], np.float32)
+    out = oracle.combine(cfg, p, y, w)
+    ref = torch.tensor([exact], dtype=torch.float64).to(torch.bfloat16).view(torch.int16)
+    assert (out == np.uint16(ref.numpy().view(np.uint16)[0])).all()

@@ -1,0 +1,554 @@
+"""Benchmark of the MoonEP hot path on B200.
+
+One step = one pass of the whole path over one batch of the large training
+shape (R=32 simulated ranks, E=384, K=8, S=4096, H=7168, B=12, Zipf-biased
+routing at maxvio 1): plan -> dispatch -> combine -> combine backward ->
+replica-gradient reduce (gate+up+down, 3*7168*2048 fp32 per expert).
+
+Printed value (rank 0, one JSON line): dispatch+combine HBM GB/s, i.e. the
+algorithmic bytes of the dispatch and combine launches of all ranks divided
+by their CUDA-event time (max over ranks).  The planner's microseconds, every
+kernel's roofline fraction, the maxvio sweep, an end-to-end number through
+the public API with host buffers, and the CPU oracle's number on a bounded
+sample are reported beside it.
+
+--impl reference times the CPU oracle on the host cores instead (bounded
+sample of the same workload per step), rank 0 only.
+
+Multi-GPU: the simulated ranks already live on one GPU, so N GPUs run N
+independent replicas of the step (weak scaling, no data-path collective);
+NCCL is used only for the barrier and the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import glob
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from load_balancing_moonep_b200 import workloads as W  # noqa: E402
+
+METRIC = "dispatch+combine HBM GB/s (% of ~8 TB/s) vs maxvio; planner µs/layer"
+UNIT = "GB/s"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+# ------------------------------------------------------------ byte models
+
+def bytes_dispatch(wl) -> int:
+    """read each token row once, write it K times, read dst_pos"""
+    return wl.tokens * wl.H * 2 * (1 + wl.K) + wl.pairs * 4
+
+
+def bytes_combine(wl) -> int:
+    """read K rows per token, write one row, read dst_pos and w"""
+    return wl.tokens * wl.H * 2 * (wl.K + 1) + wl.pairs * 8
+
+
+def bytes_combine_bwd(wl) -> int:
+    """read dy and K y rows, write K dy_buf rows; read dst_pos, w; write dw"""
+    return wl.tokens * wl.H * 2 * (1 + 2 * wl.K) + wl.pairs * 12
+
+
+def bytes_reduce(n_rep_prefetched: int, n_rep_experts: int, P: int) -> int:
+    """each replica row read + zeroed, each home row read + written"""
+    return (n_rep_prefetched + n_rep_experts) * P * 4 * 2
+
+
+def bytes_plan(wl) -> int:
+    """two passes over the ids, dst_pos and row_src written"""
+    return wl.pairs * 4 * 2 + wl.pairs * 4 * 2
+
+
+# ------------------------------------------------------------------ peaks
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_sources_hash() -> str:
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "load_balancing_moonep_b200", "csrc", "*"))):
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return {}
+    d = json.load(open(p))
+    if d.get("csrc_sha") != kernel_sources_hash():
+        return {}
+    return d.get("per_launch_bytes", {})
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self._t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self._t.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def smi_index(local: int) -> str:
+    """nvidia-smi's id for this process's GPU (CUDA_VISIBLE_DEVICES aware)."""
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local < len(ids):
+            return ids[local]
+    return str(local)
+
+
+# ------------------------------------------------------------ distributed
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        log(f"warning: --gpus {n_gpus} but WORLD_SIZE={world}; using WORLD_SIZE")
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group("nccl" if torch.cuda.is_available() else "gloo",
+                                timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        if torch.cuda.is_available():
+            dist.barrier(device_ids=[torch.cuda.current_device()])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(world, x: float) -> float:
+    if world <= 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(world, x: float) -> float:
+    if world <= 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ------------------------------------------------------------ CPU oracle
+
+def oracle_sample(wl, topk_np, w_np, hidden_sample_bits, tokens, y_rows_bits):
+    """Time the CPU oracle on a bounded sample: the plan over the whole
+    routing, dispatch and combine over the sampled tokens.  Returns
+    (plan_s, data_s, data_bytes)."""
+    import oracle
+    ocfg = oracle.Config(R=wl.R, E=wl.E, K=wl.K, S=wl.S, H=wl.H, B=wl.B)
+    t0 = time.perf_counter()
+    op = oracle.plan(ocfg, topk_np)
+    t1 = time.perf_counter()
+    n = len(tokens)
+    sub = {"dst_pos": np.arange(n * wl.K, dtype=np.int32).reshape(n, wl.K), "info": op["info"]}
+    scfg = oracle.Config(R=1, E=wl.E, K=wl.K, S=n, H=wl.H, B=0)
+    buf = np.zeros((n * wl.K, wl.H), np.uint16)
+    t2 = time.perf_counter()
+    oracle.dispatch(scfg, sub, hidden_sample_bits, buf)
+    oracle.combine(scfg, sub, y_rows_bits, np.ascontiguousarray(w_np[tokens]))
+    t3 = time.perf_counter()
+    frac = n / wl.tokens
+    data_bytes = (bytes_dispatch(wl) + bytes_combine(wl)) * frac
+    return t1 - t0, t3 - t2, data_bytes
+
+
+def sample_tokens(wl, n):
+    return np.arange(min(n, wl.tokens), dtype=np.int64)
+
+
+def cpu_inputs(wl, maxvio, n_tokens, device):
+    r = W.routing(wl, maxvio, seed=0, device=device)
+    topk = r.topk_idx.cpu().numpy()
+    w = r.weights.cpu().numpy()
+    tokens = sample_tokens(wl, n_tokens)
+    hid = W.bits(W.bf16_normal((len(tokens), wl.H), seed=1, device="cpu"))
+    y = W.bits(W.bf16_normal((len(tokens) * wl.K, wl.H), seed=2, device="cpu"))
+    return r, topk, w, tokens, hid, y
+
+
+def run_reference(args, world, rank):
+    """--impl reference: the CPU oracle as it stands, on the host cores."""
+    if rank != 0:
+        return
+    wl = W.WORKLOADS[args.workload]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    r, topk, w, tokens, hid, y = cpu_inputs(wl, args.maxvio, args.ref_tokens, dev)
+    times, plan_s = [], []
+    for i in range(args.warmup + args.steps):
+        ps, ds, db = oracle_sample(wl, topk, w, hid, tokens, y)
+        if i >= args.warmup:
+            times.append(ds)
+            plan_s.append(ps)
+    data_s = sum(times)
+    value = db * len(times) / data_s / 1e9
+    ms_step = (sum(times) + sum(plan_s)) / len(times) * 1e3
+    sample = (f"per step: plan over all {wl.pairs} pairs + dispatch and combine of the first "
+              f"{len(tokens)} of {wl.tokens} tokens, single-threaded C oracle")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": workload_config(wl, r, args),
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "planner_us": round(statistics.median(plan_s) * 1e6, 1),
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(wl, r, args):
+    return {"workload": f"{wl.name}: R={wl.R} E={wl.E} K={wl.K} S={wl.S} H={wl.H} B={wl.B}",
+            "R": wl.R, "E": wl.E, "K": wl.K, "S": wl.S, "H": wl.H, "B": wl.B,
+            "maxvio_target": args.maxvio, "maxvio": round(r.maxvio, 4),
+            "routing": f"gaussian logits + Zipf(s={wl.zipf_s}) expert bias, top-{wl.K}, seed 0",
+            "l2": "inputs larger than L2 (hidden 1.9 GB, buffers 15 GB, 126 MB L2); no flush",
+            "parallelism": "replicas (R ranks simulated in one GPU's HBM)"}
+
+
+# ------------------------------------------------------------- our arm
+
+class Timer:
+    """CUDA events on the current stream around each call of a step."""
+
+    def __init__(self):
+        self.pairs = {}
+
+    def mark(self, name):
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        self.pairs.setdefault(name, []).append((s, e))
+        s.record()
+        return e
+
+    def total_ms(self, name):
+        return sum(s.elapsed_time(e) for s, e in self.pairs.get(name, []))
+
+    def count(self, name):
+        return len(self.pairs.get(name, []))
+
+
+def run_ours(args, world, rank, local):
+    from load_balancing_moonep_b200 import moonep as mp
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wl = W.WORKLOADS[args.workload]
+    cfg = mp.Config(R=wl.R, E=wl.E, K=wl.K, S=wl.S, H=wl.H, B=wl.B)
+    peak, peak_kind = measured_peaks()
+
+    r = W.routing(wl, args.maxvio, seed=rank, device=dev)
+    hidden = W.hidden_states(wl, seed=1 + rank, device=dev)
+    dy = W.bf16_normal((wl.tokens, wl.H), seed=3 + rank, device=dev)
+    buf = torch.empty((wl.R, wl.C, wl.H), dtype=torch.bfloat16, device=dev)
+    dy_buf = torch.empty_like(buf)
+    out = torch.empty((wl.tokens, wl.H), dtype=torch.bfloat16, device=dev)
+    dw = torch.empty((wl.tokens, wl.K), dtype=torch.float32, device=dev)
+    plan = mp.Plan(cfg, dev)
+
+    # replica gradients: the full gate+up+down size if it fits, else one projection
+    P = wl.grad_elems if wl.H_ffn else 0
+    reduce_note = "gate+up+down per expert"
+    if P:
+        free, _ = torch.cuda.mem_get_info(dev)
+        need = 4 * P * (wl.R * wl.B + wl.E)
+        if need > free - (6 << 30):
+            P = wl.H * wl.H_ffn
+            reduce_note = "one projection per expert (device memory)"
+        rb = W.f32_normal((wl.R, wl.B, P), seed=4 + rank, device=dev, std=1e-3)
+        hg = W.f32_normal((wl.E, P), seed=5 + rank, device=dev, std=1e-3)
+
+    def step(tm: Timer | None):
+        ev = tm.mark("plan") if tm else None
+        mp.plan(cfg, r.topk_idx, out=plan)
+        if tm:
+            ev.record()
+            ev = tm.mark("dispatch")
+        mp.dispatch(cfg, plan, hidden, buf)
+        if tm:
+            ev.record()
+            ev = tm.mark("combine")
+        mp.combine(cfg, plan, buf, r.weights, out)
+        if tm:
+            ev.record()
+            ev = tm.mark("combine_bwd")
+        mp.combine_backward(cfg, plan, dy, r.weights, buf, dy_buf, dw)
+        if tm:
+            ev.record()
+        if P:
+            if tm:
+                ev = tm.mark("reduce")
+            mp.reduce_replica_grads(cfg, plan, rb, hg)
+            if tm:
+                ev.record()
+
+    for _ in range(args.warmup):
+        step(None)
+    torch.cuda.synchronize()
+    info = plan.info()
+    sampler = ClockSampler(smi_index(local))
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.start()
+    tm = Timer()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record()
+    for _ in range(args.steps):
+        step(tm)
+    t_end.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    barrier(world)
+    step_ms_local = t_start.elapsed_time(t_end) / args.steps
+    ms_per_step = max_over_ranks(world, step_ms_local)
+
+    k = args.steps
+    t = {n: tm.total_ms(n) / k for n in ("plan", "dispatch", "combine", "combine_bwd", "reduce")
+         if tm.count(n)}
+    dc_ms = max_over_ranks(world, t["dispatch"] + t["combine"])
+    dc_bytes = (bytes_dispatch(wl) + bytes_combine(wl)) * world
+    value = dc_bytes / (dc_ms * 1e-3) / 1e9
+
+    n_pref = info["n_rep"] - info["n_overflow"]
+    kb = {"plan": bytes_plan(wl), "dispatch": bytes_dispatch(wl), "combine": bytes_combine(wl),
+          "combine_bwd": bytes_combine_bwd(wl)}
+    if P:
+        kb["reduce"] = bytes_reduce(n_pref, info["n_rep_experts"], P)
+    traffic = ncu_traffic()
+    kernels = {}
+    for n, ms in t.items():
+        gbs = kb[n] / (ms * 1e-3) / 1e9
+        kernels[n] = {"ms": round(ms, 4), "bytes": kb[n], "GB/s": round(gbs, 1),
+                      "frac": round(gbs / peak, 4), "traffic": traffic.get(n)}
+    kernels["plan"]["us"] = round(t["plan"] * 1e3, 2)
+    dom = max((n for n in t if n != "plan"), key=lambda n: t[n])
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["GB/s"], "peak": peak,
+                "peak_kind": peak_kind + " (MEASURED_PEAKS.json hbm_gbs, copy read+write)",
+                "unit": "GB/s", "frac": kernels[dom]["frac"], "traffic": traffic.get(dom)}
+
+    # maxvio sweep: dispatch / combine GB/s and planner us per point
+    sweep = []
+    if not args.no_sweep:
+        for mv in wl.sweep:
+            rs = W.routing(wl, mv, seed=rank, device=dev)
+            ps = mp.Plan(cfg, dev)
+            for _ in range(3):
+                mp.plan(cfg, rs.topk_idx, out=ps)
+                mp.dispatch(cfg, ps, hidden, buf)
+                mp.combine(cfg, ps, buf, rs.weights, out)
+            torch.cuda.synchronize()
+            st = Timer()
+            for _ in range(args.sweep_iters):
+                e = st.mark("plan"); mp.plan(cfg, rs.topk_idx, out=ps); e.record()
+                e = st.mark("dispatch"); mp.dispatch(cfg, ps, hidden, buf); e.record()
+                e = st.mark("combine"); mp.combine(cfg, ps, buf, rs.weights, out); e.record()
+            torch.cuda.synchronize()
+            it = args.sweep_iters
+            pd, pc, pp = st.total_ms("dispatch") / it, st.total_ms("combine") / it, st.total_ms("plan") / it
+            inf = ps.info()
+            gd = bytes_dispatch(wl) / (pd * 1e-3) / 1e9
+            gc = bytes_combine(wl) / (pc * 1e-3) / 1e9
+            sweep.append({"maxvio": round(rs.maxvio, 3), "dispatch_GB/s": round(gd, 1),
+                          "combine_GB/s": round(gc, 1), "dispatch_frac": round(gd / peak, 4),
+                          "combine_frac": round(gc / peak, 4), "planner_us": round(pp * 1e3, 2),
+                          "dispatch_tok/s": round(wl.tokens / (pd * 1e-3)),
+                          "n_rep": inf["n_rep"], "n_overflow": inf["n_overflow"],
+                          "max_rep_per_rank": inf["max_rep_per_rank"],
+                          "remote_pair_frac": round(inf["n_remote_pairs"] / wl.pairs, 4)})
+            del ps
+
+    # end to end through the public API with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        h_topk = r.topk_idx.cpu().pin_memory()
+        h_w = r.weights.cpu().pin_memory()
+        h_hidden = hidden.cpu().pin_memory()
+        h_out = torch.empty((wl.tokens, wl.H), dtype=torch.bfloat16).pin_memory()
+        d_topk = torch.empty_like(r.topk_idx)
+        d_w = torch.empty_like(r.weights)
+        d_hidden = torch.empty_like(hidden)
+
+        def e2e_step():
+            d_topk.copy_(h_topk, non_blocking=True)
+            d_w.copy_(h_w, non_blocking=True)
+            d_hidden.copy_(h_hidden, non_blocking=True)
+            mp.plan(cfg, d_topk, out=plan)
+            mp.dispatch(cfg, plan, d_hidden, buf)
+            mp.combine(cfg, plan, buf, d_w, out)
+            h_out.copy_(out, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        n_e2e = max(3, min(args.steps, 10))
+        for _ in range(n_e2e):
+            e2e_step()
+        b.record()
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(world, a.elapsed_time(b) / n_e2e)
+        e2e = {"value": round(dc_bytes / (e_ms * 1e-3) / 1e9, 2), "unit": UNIT,
+               "ms_per_step": round(e_ms, 3),
+               "h2d_bytes_per_step": int(h_topk.numel() * 4 + h_w.numel() * 4 + h_hidden.numel() * 2),
+               "d2h_bytes_per_step": int(h_out.numel() * 2),
+               "what": "pinned host topk/weights/hidden -> plan -> dispatch -> combine -> host out"}
+
+    # the CPU oracle on a bounded sample (rank 0, one GPU only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        topk_np = r.topk_idx.cpu().numpy()
+        w_np = r.weights.cpu().numpy()
+        tokens = sample_tokens(wl, args.ref_tokens)
+        hid = W.bits(hidden[: len(tokens)])
+        y = W.bits(W.bf16_normal((len(tokens) * wl.K, wl.H), seed=2, device="cpu"))
+        ps_, ds_, db_ = oracle_sample(wl, topk_np, w_np, hid, tokens, y)
+        cpu = {"value": round(db_ / ds_ / 1e9, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": (f"dispatch+combine of the first {len(tokens)} of {wl.tokens} tokens "
+                          f"({ds_:.1f} s); plan over all {wl.pairs} pairs took {ps_ * 1e3:.0f} ms; "
+                          "single-threaded C")}
+
+    launches_per_step = 2 + 1 + 1 + 1 + (1 if P else 0)
+    cfgd = workload_config(wl, r, args)
+    cfgd["reduce"] = f"P={P} fp32 ({reduce_note}), {n_pref} prefetched replicas over {info['n_rep_experts']} experts"
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": cfgd,
+        "frac_of_peak": round(value / world / peak, 4),
+        "planner_us": kernels["plan"]["us"],
+        "roofline": roofline, "kernels": kernels, "sweep": sweep,
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks, "plan_info": info,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="large", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--maxvio", type=float, default=1.0)
+    ap.add_argument("--sweep-iters", type=int, default=10)
+    ap.add_argument("--ref-tokens", type=int, default=8192)
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        log("warmup raised to 3 (timing rule)")
+        args.warmup = 3
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,218 @@
+/*
+ * moonep.h -- C ABI of the MoonEP redundant-expert planner and fused
+ * permute/unpermute for NVIDIA B200 (sm_100a).
+ *
+ * The operation (cited by page title and section):
+ *   "Moonshot AI Open-Sources MoonEP: A Perfectly Balanced Expert
+ *   Parallelism Library for MoE Training" (MoonEP article below):
+ *     - "The problem MoonEP targets": top-K routing is skewed; skew is
+ *       measured by maxvio = max_e T_e / T_bar - 1.
+ *     - "The core idea: dynamic redundant experts": every rank receives
+ *       exactly S*K token slots however skewed the routing is; a small
+ *       number of redundant experts is planned online from the current
+ *       router output; tokens are written directly into expert-grouped
+ *       positions of a fixed S*K buffer and views of it are handed to the
+ *       computation; duplicated experts' gradients go back to their home.
+ *     - interactive explainer, memory tab: at most B prefetched replica
+ *       slots per rank (B = E/R in training), replica gradients in an fp32
+ *       reduce buffer [R, B, ...] that is summed home and zeroed; in
+ *       inference a rank needing more than B foreign experts reads the
+ *       overflow from the home rank (correctness unaffected).
+ *     - explainer, invariant tab: no host synchronisation per MoE layer.
+ *
+ * Scope: R expert-parallel ranks are simulated as R partitions of ONE
+ * GPU's memory; no collective is issued.  Rank r owns tokens
+ * [r*S, (r+1)*S) and rows [r*S*K, (r+1)*S*K) of the dispatch buffer.
+ * Expert e's home rank is e / L with L = E / R (contiguous homes).
+ *
+ * Conventions for every call below:
+ *   - All array pointers are DEVICE pointers unless stated otherwise and
+ *     are caller-allocated; the library never allocates and never frees.
+ *   - bf16 data are passed as uint16_t bit patterns.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every
+ *     call only enqueues kernels on it and returns; nothing synchronises
+ *     the host.  Data-dependent problems are reported in the device-side
+ *     status word plan->info[MOONEP_INFO_STATUS], which the caller may read
+ *     back whenever it likes.
+ *   - Return value: MOONEP_OK or a MOONEP_ERR_* code from the host-side
+ *     argument checks (nothing is launched then) or MOONEP_ERR_CUDA if a
+ *     launch failed.
+ *   - Calls are stream-ordered; two plans or workspaces must not be shared
+ *     by calls that can run concurrently.
+ */
+#ifndef MOONEP_H
+#define MOONEP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOONEP_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define MOONEP_API __attribute__((visibility("default")))
+#else
+#define MOONEP_API
+#endif
+
+/* ---- configuration flags ---------------------------------------------- */
+/* Overflow (a rank needs more than B replica slots) also sets
+ * MOONEP_ST_STRICT_VIOLATION: training has no reduce rows for overflow. */
+#define MOONEP_FLAG_STRICT_BUDGET 1u
+/* Require B == E/R, the training rule of the explainer's memory tab. */
+#define MOONEP_FLAG_TRAIN_B_RULE 2u
+/* combine_backward dispatches dy unscaled instead of w * dy. */
+#define MOONEP_FLAG_BWD_UNSCALED 4u
+
+/* ---- host return codes ------------------------------------------------- */
+#define MOONEP_OK 0
+#define MOONEP_ERR_ARG 1            /* null pointer, non-positive size, K > E, R*S*K >= 2^31 */
+#define MOONEP_ERR_E_NOT_DIVISIBLE 2 /* E % R != 0 (the explainer flags it) */
+#define MOONEP_ERR_BUDGET_RULE 3    /* TRAIN_B_RULE set and B != E/R */
+#define MOONEP_ERR_B_RANGE 4        /* B < 0 or B > E - L */
+#define MOONEP_ERR_CUDA 5           /* a kernel launch failed */
+#define MOONEP_ERR_LIMIT 7          /* E > MOONEP_MAX_E */
+#define MOONEP_ERR_ALIGN 8          /* H % 8 != 0 or a data pointer not 16-byte aligned */
+
+#define MOONEP_MAX_E 1024
+
+/* ---- device status bits (plan->info[MOONEP_INFO_STATUS]) -------------- */
+/* An id outside [0, E): the plan is empty, dst_pos/row_src are -1, and
+ * dispatch / combine / combine_backward / reduce become no-ops. */
+#define MOONEP_ST_EXPERT_ID_RANGE 1
+/* Some rank holds more than B replicas; the extra ones (ordinal >= B) are
+ * still planned, so every rank still gets exactly S*K slots, but they have
+ * no prefetch slot / reduce rows (read-through in inference). */
+#define MOONEP_ST_OVERFLOW 2
+#define MOONEP_ST_STRICT_VIOLATION 4
+/* A buffer row taken from the plan was outside [0, R*S*K) (a corrupted or
+ * mismatched plan); that row access was skipped. */
+#define MOONEP_ST_ROW_RANGE 8
+
+/* ---- plan->info[] fields (int32, device) ------------------------------ */
+#define MOONEP_INFO_STATUS 0
+#define MOONEP_INFO_N_REP 1            /* replicas created */
+#define MOONEP_INFO_N_OVERFLOW 2       /* replicas with ordinal >= B */
+#define MOONEP_INFO_N_PIECES 3         /* experts that shed load */
+#define MOONEP_INFO_N_RECEIVERS 4      /* ranks with a deficit */
+#define MOONEP_INFO_MAX_REP_PER_RANK 5
+#define MOONEP_INFO_N_REP_EXPERTS 6    /* experts with >= 1 prefetched replica */
+#define MOONEP_INFO_N_REMOTE_PAIRS 7   /* pairs whose buffer rank != source rank */
+#define MOONEP_INFO_LEN 16
+
+typedef struct moonep_config {
+    int32_t R;      /* simulated expert-parallel ranks */
+    int32_t E;      /* experts; E % R == 0, L = E / R home experts per rank */
+    int32_t K;      /* routed experts per token (top-K) */
+    int32_t S;      /* tokens per rank */
+    int32_t H;      /* hidden size (bf16 elements per row), H % 8 == 0 */
+    int32_t B;      /* replica (prefetch) slots per rank, 0 <= B <= E - L */
+    uint32_t flags; /* MOONEP_FLAG_* */
+} moonep_config;
+
+/* The plan: device arrays, all int32, laid out by moonep_plan_layout().
+ * Slot s of rank r: s < L is home expert r*L + s; s >= L is the rank's
+ * (s-L)-th replica in creation order; unused slots hold expert -1, count 0.
+ * Rows of rank r's buffer are grouped by slot: slot s occupies rows
+ * [slot_offset[r][s], slot_offset[r][s+1]) and slot_offset[r][E] == S*K. */
+typedef struct moonep_plan_s {
+    int32_t *expert_count;  /* [E] T_e = pairs routed to e */
+    int32_t *slot_expert;   /* [R][E] */
+    int32_t *slot_count;    /* [R][E] rows per slot */
+    int32_t *slot_offset;   /* [R][E+1] exclusive prefix of slot_count */
+    int32_t *rep_expert;    /* [E+R] replica list in creation order ... */
+    int32_t *rep_rank;      /* [E+R] ... rank holding the replica */
+    int32_t *rep_slot;      /* [E+R] ... its slot (L + ordinal) */
+    int32_t *rep_quota;     /* [E+R] ... rows it receives; entries >= n_rep: -1 / 0 */
+    int32_t *host_ptr;      /* [E+1] CSR: hosts of expert e are [host_ptr[e], host_ptr[e+1]) */
+    int32_t *host_rank;     /* [2E+R] hosts in ascending rank order (home copy included) */
+    int32_t *host_slot;     /* [2E+R] */
+    int32_t *host_start;    /* [2E+R] first within-expert rank g served by the host */
+    int32_t *host_quota;    /* [2E+R] number of g served by the host */
+    int32_t *rep_home_list; /* [E] experts with >= 1 prefetched replica, ascending, then -1 */
+    int32_t *dst_pos;       /* [R*S*K] buffer row of pair (t, k), index t*K + k */
+    int32_t *row_src;       /* [R*S*K] inverse: pair t*K + k held by a buffer row */
+    int32_t *info;          /* [MOONEP_INFO_LEN] status and statistics */
+} moonep_plan_t;
+
+/* Host-side validation of a configuration.  Returns MOONEP_OK or an error. */
+MOONEP_API int moonep_check_config(const moonep_config *cfg);
+
+/* Bytes of the plan block and of the planner workspace for `cfg`.
+ * The workspace must be zero-filled once after allocation (for example
+ * cudaMemset); every moonep_plan() call leaves it zero-filled again. */
+MOONEP_API int moonep_plan_sizes(const moonep_config *cfg, size_t *plan_bytes, size_t *workspace_bytes);
+
+/* Fills `out` with pointers into the device block `plan_base` of
+ * plan_bytes bytes (256-byte aligned sub-arrays).  Host-only arithmetic. */
+MOONEP_API int moonep_plan_layout(const moonep_config *cfg, void *plan_base, moonep_plan_t *out);
+
+/* Online planning (MoonEP article, "The core idea: dynamic redundant
+ * experts"; planner described as "near-optimal" with no algorithm given).
+ * topk_idx: device int32 [R*S, K], row t = token t (rank t / S), k order as
+ * produced by the router.  Computes, with no host synchronisation:
+ *   histogram T_e; home loads and excess/deficit per rank; largest-first
+ *   shedding by each overloaded rank (ties: lower expert id first);
+ *   pieces ordered by (shed desc, e asc) and receivers by (deficit desc,
+ *   rank asc); water-filling of pieces into deficits (every positive
+ *   overlap of the two prefix-sum partitions is one replica, created in
+ *   (piece, receiver) order; a rank's replicas take slots L, L+1, ...);
+ *   slot tables; per-expert host intervals in ascending rank order; and for
+ *   every pair in (t, k) order the buffer row
+ *     dst_pos = rank*S*K + slot_offset[rank][slot] + (g - host_start)
+ *   where g is the pair's rank among earlier pairs of the same expert.
+ * plan: laid out by moonep_plan_layout; workspace: workspace_bytes bytes,
+ * zero-filled before the first call.  Two kernel launches. */
+MOONEP_API int moonep_plan(const moonep_config *cfg, const int32_t *topk_idx, const moonep_plan_t *plan,
+                void *workspace, void *stream);
+
+/* Zero-copy permute (MoonEP article, "The core idea", zero copy and static
+ * shapes): buf[dst_pos[t*K+k], :] = hidden[t, :] for every pair.
+ * hidden: bf16 [R*S, H]; buf: bf16 [R, S*K, H] = R*S*K rows of H.  Every
+ * buffer row is written exactly once; values are copied bit for bit. */
+MOONEP_API int moonep_dispatch(const moonep_config *cfg, const moonep_plan_t *plan, const uint16_t *hidden,
+                    uint16_t *buf, void *stream);
+
+/* Weighted unpermute: out[t, h] = bf16_rne(sum_k w[t,k] * y[dst_pos[t*K+k], h])
+ * accumulated in fp32 as acc = fmaf(w, y, acc) from 0.0f in k order.
+ * y: bf16 [R, S*K, H] (expert outputs in buffer layout); w: fp32 [R*S, K];
+ * out: bf16 [R*S, H]. */
+MOONEP_API int moonep_combine(const moonep_config *cfg, const moonep_plan_t *plan, const uint16_t *y,
+                   const float *w, uint16_t *out, void *stream);
+
+/* Backward of combine:
+ *   dy_buf[dst_pos[t*K+k], h] = bf16_rne(w[t,k] * dy[t,h])   (one fp32 product;
+ *                                dy itself with MOONEP_FLAG_BWD_UNSCALED)
+ *   dw[t, k] = sum_h dy[t,h] * y[dst_pos[t*K+k], h]          (fp32 accumulation)
+ * dy: bf16 [R*S, H]; w: fp32 [R*S, K]; y: bf16 [R, S*K, H];
+ * dy_buf: bf16 [R, S*K, H]; dw: fp32 [R*S, K]. */
+MOONEP_API int moonep_combine_backward(const moonep_config *cfg, const moonep_plan_t *plan, const uint16_t *dy,
+                            const float *w, const uint16_t *y, uint16_t *dy_buf, float *dw,
+                            void *stream);
+
+/* Replica-gradient reduction (MoonEP explainer, memory tab, training
+ * branch: replica grads land in an fp32 reduce buffer mapped as
+ * [R, B, ...]; they are pulled back to the home expert and zeroed for the
+ * next microbatch).  For every expert with prefetched replicas, in
+ * ascending host rank order:
+ *   home_grad[e, i] = home_grad[e, i] + reduce_buf[r, slot - L, i]
+ * (separate fp32 adds), then those reduce_buf rows are set to 0.
+ * reduce_buf: fp32 [R, B, P]; home_grad: fp32 [E, P]; P > 0 elements per
+ * expert gradient.  Overflow replicas have no rows and are skipped. */
+MOONEP_API int moonep_reduce_replica_grads(const moonep_config *cfg, const moonep_plan_t *plan,
+                                float *reduce_buf, float *home_grad, int64_t P, void *stream);
+
+/* Human-readable text for a MOONEP_* return code. */
+MOONEP_API const char *moonep_error_string(int code);
+
+/* MOONEP_ABI_VERSION of the loaded library. */
+MOONEP_API int moonep_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOONEP_H */

@@ -1,0 +1,208 @@
+// C ABI entry points (declared in include/moonep.h): host-side argument
+// checks, plan layout and kernel launches.  No call allocates memory or
+// synchronises the host.
+#include <cstdint>
+#include <cstring>
+
+#include "common.cuh"
+
+namespace moonep {
+int launch_plan(const Dims &d, const int32_t *topk, const moonep_plan_t &p, void *ws, cudaStream_t st);
+size_t plan_smem_bytes_max(const Dims &d);
+int launch_dispatch(const Dims &d, const int *dst_pos, int *info, const uint16_t *hidden, uint16_t *buf,
+                    cudaStream_t st);
+int launch_combine(const Dims &d, const int *dst_pos, int *info, const uint16_t *y, const float *w,
+                   uint16_t *out, cudaStream_t st);
+int launch_combine_backward(const Dims &d, const int *dst_pos, int *info, const uint16_t *dy, const float *w,
+                            const uint16_t *y, uint16_t *dy_buf, float *dw, cudaStream_t st);
+int launch_reduce(const Dims &d, const moonep_plan_t &p, float *reduce_buf, float *home_grad, long long P,
+                  cudaStream_t st);
+
+constexpr size_t MAX_DYN_SMEM = 227 * 1024;
+constexpr int MAX_COMBINE_BWD_K = 16;
+
+static int make_dims(const moonep_config *c, Dims *d)
+{
+    const int rc = moonep_check_config(c);
+    if (rc != MOONEP_OK) return rc;
+    d->R = c->R;
+    d->E = c->E;
+    d->K = c->K;
+    d->S = c->S;
+    d->H = c->H;
+    d->B = c->B;
+    d->L = c->E / c->R;
+    d->flags = c->flags;
+    d->C = c->S * c->K;
+    d->tokens = c->R * c->S;
+    d->pairs = c->R * c->S * c->K;
+    int ct = (d->tokens + 255) / 256;
+    if (ct < 8) ct = 8;
+    int cap = 4096 / d->K;
+    if (cap < 1) cap = 1;
+    if (ct > cap) ct = cap;
+    if (ct > d->tokens) ct = d->tokens;
+    d->chunk_tokens = ct;
+    d->nchunk = (d->tokens + ct - 1) / ct;
+    if (plan_smem_bytes_max(*d) > MAX_DYN_SMEM) return MOONEP_ERR_LIMIT;
+    return MOONEP_OK;
+}
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static bool plan_ok(const moonep_plan_t *p)
+{
+    return p && p->expert_count && p->slot_expert && p->slot_count && p->slot_offset && p->rep_expert &&
+           p->rep_rank && p->rep_slot && p->rep_quota && p->host_ptr && p->host_rank && p->host_slot &&
+           p->host_start && p->host_quota && p->rep_home_list && p->dst_pos && p->row_src && p->info;
+}
+
+struct PlanLayout {
+    size_t off[17];
+    size_t total;
+};
+
+static PlanLayout plan_layout(const Dims &d)
+{
+    const size_t E = d.E, R = d.R, NP = (size_t)d.pairs;
+    const size_t n[17] = {E,         R * E,     R * E,     R * (E + 1), E + R,      E + R,
+                          E + R,     E + R,     E + 1,     2 * E + R,   2 * E + R,  2 * E + R,
+                          2 * E + R, E,         NP,        NP,          MOONEP_INFO_LEN};
+    PlanLayout l;
+    size_t o = 0;
+    for (int i = 0; i < 17; ++i) {
+        l.off[i] = o;
+        o = align256(o + n[i] * sizeof(int32_t));
+    }
+    l.total = o;
+    return l;
+}
+
+}  // namespace moonep
+
+using namespace moonep;
+
+extern "C" {
+
+int moonep_abi_version(void) { return MOONEP_ABI_VERSION; }
+
+const char *moonep_error_string(int code)
+{
+    switch (code) {
+    case MOONEP_OK: return "ok";
+    case MOONEP_ERR_ARG: return "invalid argument (null pointer, non-positive size, K > E or R*S*K >= 2^31)";
+    case MOONEP_ERR_E_NOT_DIVISIBLE: return "E is not divisible by R";
+    case MOONEP_ERR_BUDGET_RULE: return "training budget rule violated: B must equal E/R";
+    case MOONEP_ERR_B_RANGE: return "replica budget B out of range [0, E - E/R]";
+    case MOONEP_ERR_CUDA: return "CUDA launch failed";
+    case MOONEP_ERR_LIMIT: return "size beyond a library limit (E > 1024, shared memory, or K > 16 in combine_backward)";
+    case MOONEP_ERR_ALIGN: return "H must be a multiple of 8 and bf16 data pointers 16-byte aligned";
+    default: return "unknown error";
+    }
+}
+
+int moonep_check_config(const moonep_config *c)
+{
+    if (!c) return MOONEP_ERR_ARG;
+    if (c->R <= 0 || c->E <= 0 || c->K <= 0 || c->S <= 0 || c->H <= 0) return MOONEP_ERR_ARG;
+    if (c->K > c->E) return MOONEP_ERR_ARG;
+    if ((int64_t)c->R * c->S * c->K > INT32_MAX) return MOONEP_ERR_ARG;
+    if (c->E % c->R != 0) return MOONEP_ERR_E_NOT_DIVISIBLE;
+    const int L = c->E / c->R;
+    if ((c->flags & MOONEP_FLAG_TRAIN_B_RULE) && c->B != L) return MOONEP_ERR_BUDGET_RULE;
+    if (c->B < 0 || c->B > c->E - L) return MOONEP_ERR_B_RANGE;
+    if (c->E > MOONEP_MAX_E) return MOONEP_ERR_LIMIT;
+    if (c->H % 8 != 0) return MOONEP_ERR_ALIGN;
+    return MOONEP_OK;
+}
+
+int moonep_plan_sizes(const moonep_config *cfg, size_t *plan_bytes, size_t *workspace_bytes)
+{
+    Dims d;
+    const int rc = make_dims(cfg, &d);
+    if (rc != MOONEP_OK) return rc;
+    if (plan_bytes) *plan_bytes = plan_layout(d).total;
+    if (workspace_bytes) *workspace_bytes = ws_layout(d).total;
+    return MOONEP_OK;
+}
+
+int moonep_plan_layout(const moonep_config *cfg, void *plan_base, moonep_plan_t *out)
+{
+    if (!plan_base || !out) return MOONEP_ERR_ARG;
+    Dims d;
+    const int rc = make_dims(cfg, &d);
+    if (rc != MOONEP_OK) return rc;
+    if (reinterpret_cast<uintptr_t>(plan_base) & 255u) return MOONEP_ERR_ALIGN;
+    const PlanLayout l = plan_layout(d);
+    char *b = static_cast<char *>(plan_base);
+    int32_t **f[17] = {&out->expert_count, &out->slot_expert, &out->slot_count, &out->slot_offset,
+                       &out->rep_expert,   &out->rep_rank,    &out->rep_slot,   &out->rep_quota,
+                       &out->host_ptr,     &out->host_rank,   &out->host_slot,  &out->host_start,
+                       &out->host_quota,   &out->rep_home_list, &out->dst_pos,  &out->row_src,
+                       &out->info};
+    for (int i = 0; i < 17; ++i) *f[i] = reinterpret_cast<int32_t *>(b + l.off[i]);
+    return MOONEP_OK;
+}
+
+int moonep_plan(const moonep_config *cfg, const int32_t *topk_idx, const moonep_plan_t *plan, void *workspace,
+                void *stream)
+{
+    Dims d;
+    const int rc = make_dims(cfg, &d);
+    if (rc != MOONEP_OK) return rc;
+    if (!topk_idx || !plan_ok(plan) || !workspace) return MOONEP_ERR_ARG;
+    return launch_plan(d, topk_idx, *plan, workspace, static_cast<cudaStream_t>(stream));
+}
+
+int moonep_dispatch(const moonep_config *cfg, const moonep_plan_t *plan, const uint16_t *hidden, uint16_t *buf,
+                    void *stream)
+{
+    Dims d;
+    const int rc = make_dims(cfg, &d);
+    if (rc != MOONEP_OK) return rc;
+    if (!plan_ok(plan) || !hidden || !buf) return MOONEP_ERR_ARG;
+    if (!aligned16(hidden) || !aligned16(buf)) return MOONEP_ERR_ALIGN;
+    return launch_dispatch(d, plan->dst_pos, plan->info, hidden, buf, static_cast<cudaStream_t>(stream));
+}
+
+int moonep_combine(const moonep_config *cfg, const moonep_plan_t *plan, const uint16_t *y, const float *w,
+                   uint16_t *out, void *stream)
+{
+    Dims d;
+    const int rc = make_dims(cfg, &d);
+    if (rc != MOONEP_OK) return rc;
+    if (!plan_ok(plan) || !y || !w || !out) return MOONEP_ERR_ARG;
+    if (!aligned16(y) || !aligned16(out) || (reinterpret_cast<uintptr_t>(w) & 3u)) return MOONEP_ERR_ALIGN;
+    return launch_combine(d, plan->dst_pos, plan->info, y, w, out, static_cast<cudaStream_t>(stream));
+}
+
+int moonep_combine_backward(const moonep_config *cfg, const moonep_plan_t *plan, const uint16_t *dy,
+                            const float *w, const uint16_t *y, uint16_t *dy_buf, float *dw, void *stream)
+{
+    Dims d;
+    const int rc = make_dims(cfg, &d);
+    if (rc != MOONEP_OK) return rc;
+    if (!plan_ok(plan) || !dy || !w || !y || !dy_buf || !dw) return MOONEP_ERR_ARG;
+    if (d.K > MAX_COMBINE_BWD_K) return MOONEP_ERR_LIMIT;
+    if (!aligned16(dy) || !aligned16(y) || !aligned16(dy_buf) || (reinterpret_cast<uintptr_t>(w) & 3u) ||
+        (reinterpret_cast<uintptr_t>(dw) & 3u))
+        return MOONEP_ERR_ALIGN;
+    return launch_combine_backward(d, plan->dst_pos, plan->info, dy, w, y, dy_buf, dw,
+                                   static_cast<cudaStream_t>(stream));
+}
+
+int moonep_reduce_replica_grads(const moonep_config *cfg, const moonep_plan_t *plan, float *reduce_buf,
+                                float *home_grad, int64_t P, void *stream)
+{
+    Dims d;
+    const int rc = make_dims(cfg, &d);
+    if (rc != MOONEP_OK) return rc;
+    if (!plan_ok(plan) || !home_grad || P <= 0) return MOONEP_ERR_ARG;
+    if (d.B > 0 && !reduce_buf) return MOONEP_ERR_ARG;
+    if (d.B == 0) return MOONEP_OK;  // no prefetched replica can exist
+    if ((reinterpret_cast<uintptr_t>(reduce_buf) & 3u) || (reinterpret_cast<uintptr_t>(home_grad) & 3u))
+        return MOONEP_ERR_ALIGN;
+    return launch_reduce(d, *plan, reduce_buf, home_grad, (long long)P, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,347 @@
+// Fused permute / unpermute and their backward (sm_100a).
+//
+// MoonEP article ("Moonshot AI Open-Sources MoonEP: A Perfectly Balanced
+// Expert Parallelism Library for MoE Training", "The core idea: dynamic
+// redundant experts", zero copy and static shapes): tokens are written
+// straight into their expert-grouped rows of a fixed [R, S*K, H] buffer, and
+// the unpermute reads them back from there, with no intermediate copy.
+//
+// All three kernels are HBM-bound streams of 16-byte vectors.  One warp owns
+// one token at a time (grid sized to fill every SM): its K destination rows
+// are fetched once by lanes 0..K-1 and broadcast with shuffles, then the
+// token's row is walked in 16-byte vectors, U vectors per lane in flight.
+//   dispatch     read the row once, store it K times;
+//   combine      read K rows, fp32 fused multiply-add in k order, store once;
+//   combine_bwd  read dy once and K expert-output rows, store K scaled rows
+//                and K dot products (fp32, fixed reduction tree).
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+
+namespace moonep {
+
+constexpr int DATA_THREADS = 256;
+
+__device__ __forceinline__ uint4 ld_stream(const uint4 *p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ void st_vec(uint4 *p, const uint4 &v)
+{
+    asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
+                 "r"(v.w)
+                 : "memory");
+}
+
+__device__ __forceinline__ float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+
+// two fp32 -> packed bf16x2, round to nearest even (lo in the low half)
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+__device__ __forceinline__ void unpack8(const uint4 &v, float f[8])
+{
+    f[0] = bf_lo(v.x); f[1] = bf_hi(v.x);
+    f[2] = bf_lo(v.y); f[3] = bf_hi(v.y);
+    f[4] = bf_lo(v.z); f[5] = bf_hi(v.z);
+    f[6] = bf_lo(v.w); f[7] = bf_hi(v.w);
+}
+
+__device__ __forceinline__ uint4 pack8(const float f[8])
+{
+    uint4 v;
+    v.x = pack_bf16x2(f[0], f[1]);
+    v.y = pack_bf16x2(f[2], f[3]);
+    v.z = pack_bf16x2(f[4], f[5]);
+    v.w = pack_bf16x2(f[6], f[7]);
+    return v;
+}
+
+__device__ __forceinline__ bool plan_invalid(const int *info)
+{
+    return (*(volatile const int *)(info + MOONEP_INFO_STATUS) & MOONEP_ST_EXPERT_ID_RANGE) != 0;
+}
+
+// A row index from the plan outside [0, rows) is never dereferenced: the
+// access is skipped and MOONEP_ST_ROW_RANGE is raised.
+__device__ __forceinline__ bool row_ok(int row, int rows, int *info)
+{
+    if ((unsigned)row < (unsigned)rows) return true;
+    atomicOr(info + MOONEP_INFO_STATUS, MOONEP_ST_ROW_RANGE);
+    return false;
+}
+
+// --------------------------------------------------------------- dispatch
+
+template <int U>
+__global__ void __launch_bounds__(DATA_THREADS) dispatch_kernel(const uint4 *__restrict__ hidden,
+                                                               uint4 *__restrict__ buf,
+                                                               const int *__restrict__ dst_pos,
+                                                               int *info, int tokens, int K, int vpr, int rows)
+{
+    if (plan_invalid(info)) return;
+    const int lane = threadIdx.x & 31;
+    const int wpb = blockDim.x >> 5;
+    const int nw = gridDim.x * wpb;
+    for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < tokens; t += nw) {
+        const int *dp = dst_pos + (size_t)t * K;
+        const int dl = lane < K ? __ldg(dp + lane) : 0;
+        const uint4 *src = hidden + (size_t)t * vpr;
+        for (int c0 = 0; c0 < vpr; c0 += 32 * U) {
+            uint4 v[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int c = c0 + u * 32 + lane;
+                if (c < vpr) v[u] = ld_stream(src + c);
+            }
+            for (int k = 0; k < K; ++k) {
+                const int dk = k < 32 ? __shfl_sync(FULL_MASK, dl, k) : __ldg(dp + k);
+                if (!row_ok(dk, rows, info)) continue;
+                uint4 *dst = buf + (size_t)dk * vpr;
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int c = c0 + u * 32 + lane;
+                    if (c < vpr) st_vec(dst + c, v[u]);
+                }
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------- combine
+
+// KT > 0: compile-time K (all K loads of a vector issued together);
+// KT == 0: any K, one expert row at a time.
+template <int KT, int U>
+__global__ void __launch_bounds__(DATA_THREADS) combine_kernel(const uint4 *__restrict__ y,
+                                                              const float *__restrict__ w,
+                                                              uint4 *__restrict__ out,
+                                                              const int *__restrict__ dst_pos, int *info,
+                                                              int tokens, int K_rt, int vpr, int rows)
+{
+    if (plan_invalid(info)) return;
+    const int K = KT > 0 ? KT : K_rt;
+    const int lane = threadIdx.x & 31;
+    const int wpb = blockDim.x >> 5;
+    const int nw = gridDim.x * wpb;
+    for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < tokens; t += nw) {
+        const int *dp = dst_pos + (size_t)t * K;
+        const float *wp = w + (size_t)t * K;
+        const int dl = lane < K ? __ldg(dp + lane) : 0;
+        const float wl = lane < K ? __ldg(wp + lane) : 0.0f;
+        for (int c0 = 0; c0 < vpr; c0 += 32 * U) {
+            float acc[U][8];
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[u][j] = 0.0f;
+            if constexpr (KT > 0) {
+                uint4 v[KT][U];
+#pragma unroll
+                for (int k = 0; k < KT; ++k) {
+                    int dk = __shfl_sync(FULL_MASK, dl, k);
+                    const bool ok = row_ok(dk, rows, info);
+                    const uint4 *row = y + (size_t)(ok ? dk : 0) * vpr;
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        const int c = c0 + u * 32 + lane;
+                        v[k][u] = make_uint4(0u, 0u, 0u, 0u);
+                        if (ok && c < vpr) v[k][u] = ld_stream(row + c);
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < KT; ++k) {
+                    const float wk = __shfl_sync(FULL_MASK, wl, k);
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        float f[8];
+                        unpack8(v[k][u], f);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) acc[u][j] = fmaf(wk, f[j], acc[u][j]);
+                    }
+                }
+            } else {
+                for (int k = 0; k < K; ++k) {
+                    const int dk = k < 32 ? __shfl_sync(FULL_MASK, dl, k) : __ldg(dp + k);
+                    const float wk = k < 32 ? __shfl_sync(FULL_MASK, wl, k) : __ldg(wp + k);
+                    if (!row_ok(dk, rows, info)) continue;
+                    const uint4 *row = y + (size_t)dk * vpr;
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        const int c = c0 + u * 32 + lane;
+                        if (c < vpr) {
+                            float f[8];
+                            unpack8(ld_stream(row + c), f);
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) acc[u][j] = fmaf(wk, f[j], acc[u][j]);
+                        }
+                    }
+                }
+            }
+            uint4 *o = out + (size_t)t * vpr;
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int c = c0 + u * 32 + lane;
+                if (c < vpr) st_vec(o + c, pack8(acc[u]));
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------- combine backward
+
+__device__ __forceinline__ float dot8(const float a[8], const float b[8])
+{
+    // products of two bf16 values are exact in fp32; fixed pairwise tree
+    const float p0 = a[0] * b[0], p1 = a[1] * b[1], p2 = a[2] * b[2], p3 = a[3] * b[3];
+    const float p4 = a[4] * b[4], p5 = a[5] * b[5], p6 = a[6] * b[6], p7 = a[7] * b[7];
+    return ((p0 + p1) + (p2 + p3)) + ((p4 + p5) + (p6 + p7));
+}
+
+template <int KT, int U>
+__global__ void __launch_bounds__(DATA_THREADS) combine_bwd_kernel(
+    const uint4 *__restrict__ dy, const float *__restrict__ w, const uint4 *__restrict__ y,
+    uint4 *__restrict__ dy_buf, float *__restrict__ dw, const int *__restrict__ dst_pos, int *info,
+    int tokens, int vpr, int unscaled, int rows)
+{
+    if (plan_invalid(info)) return;
+    constexpr int K = KT;
+    const int lane = threadIdx.x & 31;
+    const int wpb = blockDim.x >> 5;
+    const int nw = gridDim.x * wpb;
+    for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < tokens; t += nw) {
+        const int *dp = dst_pos + (size_t)t * K;
+        const float *wp = w + (size_t)t * K;
+        const int dl = lane < K ? __ldg(dp + lane) : 0;
+        const float wl = lane < K ? __ldg(wp + lane) : 0.0f;
+        float dacc[K];
+#pragma unroll
+        for (int k = 0; k < K; ++k) dacc[k] = 0.0f;
+        const uint4 *g = dy + (size_t)t * vpr;
+        for (int c0 = 0; c0 < vpr; c0 += 32 * U) {
+            float gf[U][8];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int c = c0 + u * 32 + lane;
+                if (c < vpr) unpack8(ld_stream(g + c), gf[u]);
+            }
+#pragma unroll
+            for (int k = 0; k < K; ++k) {
+                const int dk = __shfl_sync(FULL_MASK, dl, k);
+                const float wk = __shfl_sync(FULL_MASK, wl, k);
+                if (!row_ok(dk, rows, info)) continue;
+                const uint4 *yr = y + (size_t)dk * vpr;
+                uint4 *br = dy_buf + (size_t)dk * vpr;
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int c = c0 + u * 32 + lane;
+                    if (c < vpr) {
+                        float yf[8];
+                        unpack8(ld_stream(yr + c), yf);
+                        dacc[k] += dot8(gf[u], yf);
+                        float s[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) s[j] = unscaled ? gf[u][j] : __fmul_rn(wk, gf[u][j]);
+                        st_vec(br + c, pack8(s));
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
+            float v = dacc[k];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(FULL_MASK, v, o);
+            if (lane == k) dw[(size_t)t * K + k] = v;
+        }
+    }
+}
+
+// ----------------------------------------------------------------- launch
+
+static int data_grid(int tokens)
+{
+    static int sms[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    if (!sms[dev]) {
+        int v = 0;
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+        sms[dev] = v > 0 ? v : 148;
+    }
+    const int wpb = DATA_THREADS / 32;
+    const int want = (tokens + wpb - 1) / wpb;
+    const int full = sms[dev] * (2048 / DATA_THREADS);
+    return want < full ? (want > 0 ? want : 1) : full;
+}
+
+int launch_dispatch(const Dims &d, const int *dst_pos, int *info, const uint16_t *hidden, uint16_t *buf,
+                    cudaStream_t st)
+{
+    const int vpr = d.H / 8;
+    const int grid = data_grid(d.tokens);
+    dispatch_kernel<4><<<grid, DATA_THREADS, 0, st>>>(reinterpret_cast<const uint4 *>(hidden),
+                                                     reinterpret_cast<uint4 *>(buf), dst_pos, info,
+                                                     d.tokens, d.K, vpr, d.pairs);
+    return cudaGetLastError() == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
+}
+
+int launch_combine(const Dims &d, const int *dst_pos, int *info, const uint16_t *y, const float *w,
+                   uint16_t *out, cudaStream_t st)
+{
+    const int vpr = d.H / 8;
+    const int grid = data_grid(d.tokens);
+    const uint4 *yv = reinterpret_cast<const uint4 *>(y);
+    uint4 *ov = reinterpret_cast<uint4 *>(out);
+    const int T = d.tokens, K = d.K, rows = d.pairs;
+    switch (K) {
+    case 1: combine_kernel<1, 4><<<grid, DATA_THREADS, 0, st>>>(yv, w, ov, dst_pos, info, T, K, vpr, rows); break;
+    case 2: combine_kernel<2, 4><<<grid, DATA_THREADS, 0, st>>>(yv, w, ov, dst_pos, info, T, K, vpr, rows); break;
+    case 4: combine_kernel<4, 2><<<grid, DATA_THREADS, 0, st>>>(yv, w, ov, dst_pos, info, T, K, vpr, rows); break;
+    case 6: combine_kernel<6, 2><<<grid, DATA_THREADS, 0, st>>>(yv, w, ov, dst_pos, info, T, K, vpr, rows); break;
+    case 8: combine_kernel<8, 2><<<grid, DATA_THREADS, 0, st>>>(yv, w, ov, dst_pos, info, T, K, vpr, rows); break;
+    default: combine_kernel<0, 2><<<grid, DATA_THREADS, 0, st>>>(yv, w, ov, dst_pos, info, T, K, vpr, rows); break;
+    }
+    return cudaGetLastError() == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
+}
+
+template <int KT>
+static void launch_bwd_k(const Dims &d, int grid, const uint4 *dy, const float *w, const uint4 *y, uint4 *dyb,
+                         float *dw, const int *dst_pos, int *info, int unscaled, cudaStream_t st)
+{
+    combine_bwd_kernel<KT, 2><<<grid, DATA_THREADS, 0, st>>>(dy, w, y, dyb, dw, dst_pos, info, d.tokens,
+                                                            d.H / 8, unscaled, d.pairs);
+}
+
+int launch_combine_backward(const Dims &d, const int *dst_pos, int *info, const uint16_t *dy, const float *w,
+                            const uint16_t *y, uint16_t *dy_buf, float *dw, cudaStream_t st)
+{
+    const int grid = data_grid(d.tokens);
+    const uint4 *dyv = reinterpret_cast<const uint4 *>(dy);
+    const uint4 *yv = reinterpret_cast<const uint4 *>(y);
+    uint4 *bv = reinterpret_cast<uint4 *>(dy_buf);
+    const int uns = (d.flags & MOONEP_FLAG_BWD_UNSCALED) ? 1 : 0;
+    switch (d.K) {
+#define MOONEP_BWD_CASE(k) \
+    case k: launch_bwd_k<k>(d, grid, dyv, w, yv, bv, dw, dst_pos, info, uns, st); break;
+    MOONEP_BWD_CASE(1) MOONEP_BWD_CASE(2) MOONEP_BWD_CASE(3) MOONEP_BWD_CASE(4)
+    MOONEP_BWD_CASE(5) MOONEP_BWD_CASE(6) MOONEP_BWD_CASE(7) MOONEP_BWD_CASE(8)
+    MOONEP_BWD_CASE(9) MOONEP_BWD_CASE(10) MOONEP_BWD_CASE(11) MOONEP_BWD_CASE(12)
+    MOONEP_BWD_CASE(13) MOONEP_BWD_CASE(14) MOONEP_BWD_CASE(15) MOONEP_BWD_CASE(16)
+#undef MOONEP_BWD_CASE
+    default: return MOONEP_ERR_LIMIT;
+    }
+    return cudaGetLastError() == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
+}
+
+}  // namespace moonep

@@ -1,0 +1,159 @@
+// Replica-gradient reduction (sm_100a).
+//
+// MoonEP article ("Moonshot AI Open-Sources MoonEP: A Perfectly Balanced
+// Expert Parallelism Library for MoE Training"), explainer memory tab,
+// training branch: duplicated experts' gradients land in an fp32 reduce
+// buffer mapped as [R, B, ...]; they are pulled back to the home expert and
+// the buffer rows are zeroed for the next microbatch.
+//
+// Work items are (expert with prefetched replicas, element chunk); the
+// expert list and its hosts come from the plan on the device, so the launch
+// needs no host synchronisation.  Each element is read from home_grad and
+// every replica once, summed with separate fp32 adds in ascending host rank
+// order, written once, and the replica elements are overwritten with zeros.
+#include "common.cuh"
+
+namespace moonep {
+
+constexpr int REDUCE_THREADS = 256;
+constexpr int REDUCE_UNROLL = 4;
+constexpr int REDUCE_MAX_LIST = 1024;
+
+struct ReduceParams {
+    float *reduce_buf;
+    float *home_grad;
+    const int *host_ptr, *host_rank, *host_slot, *rep_home_list, *info;
+    int L, B, E, R, n_hosts;
+    long long P;        // elements per gradient row
+    long long chunk;    // vectors per work item
+};
+
+template <typename V>
+__device__ __forceinline__ V vadd(const V &a, const V &b);
+template <>
+__device__ __forceinline__ float4 vadd<float4>(const float4 &a, const float4 &b)
+{
+    return make_float4(__fadd_rn(a.x, b.x), __fadd_rn(a.y, b.y), __fadd_rn(a.z, b.z), __fadd_rn(a.w, b.w));
+}
+template <>
+__device__ __forceinline__ float vadd<float>(const float &a, const float &b)
+{
+    return __fadd_rn(a, b);
+}
+template <typename V>
+__device__ __forceinline__ V vzero();
+template <>
+__device__ __forceinline__ float4 vzero<float4>() { return make_float4(0.f, 0.f, 0.f, 0.f); }
+template <>
+__device__ __forceinline__ float vzero<float>() { return 0.f; }
+
+template <typename V>
+__global__ void __launch_bounds__(REDUCE_THREADS) reduce_kernel(ReduceParams a)
+{
+    __shared__ long long s_row[REDUCE_MAX_LIST];
+    __shared__ int s_n;
+    const int status = __ldg(a.info + MOONEP_INFO_STATUS);
+    if (status & MOONEP_ST_EXPERT_ID_RANGE) return;
+    const int n_exp = min(max(__ldg(a.info + MOONEP_INFO_N_REP_EXPERTS), 0), a.E);
+    constexpr int W = sizeof(V) / sizeof(float);
+    const long long PV = a.P / W;  // vectors per row
+    const long long nchunks = (PV + a.chunk - 1) / a.chunk;
+    const long long n_items = (long long)n_exp * nchunks;
+    V *rb = reinterpret_cast<V *>(a.reduce_buf);
+    V *hg = reinterpret_cast<V *>(a.home_grad);
+
+    for (long long item = blockIdx.x; item < n_items; item += gridDim.x) {
+        const int e = __ldg(a.rep_home_list + item / nchunks);
+        const long long ci = item % nchunks;
+        if (e < 0 || e >= a.E) continue;  // uniform across the block
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int n = 0;
+            const int home = e / a.L;
+            const int h0 = max(0, __ldg(a.host_ptr + e));
+            const int h1 = min(a.n_hosts, __ldg(a.host_ptr + e + 1));
+            for (int h = h0; h < h1; ++h) {
+                const int r = __ldg(a.host_rank + h), b = __ldg(a.host_slot + h) - a.L;
+                if (r == home || r < 0 || r >= a.R || b < 0 || b >= a.B) continue;
+                if (n < REDUCE_MAX_LIST) s_row[n++] = (long long)r * a.B + b;
+            }
+            s_n = n;
+        }
+        __syncthreads();
+        const int n = s_n;
+        V *home_row = hg + (long long)e * PV;
+        const long long v0 = ci * a.chunk;
+        const long long v1 = min(PV, v0 + a.chunk);
+        for (long long v = v0 + threadIdx.x; v < v1; v += (long long)REDUCE_THREADS * REDUCE_UNROLL) {
+            V acc[REDUCE_UNROLL];
+#pragma unroll
+            for (int u = 0; u < REDUCE_UNROLL; ++u) {
+                const long long x = v + (long long)u * REDUCE_THREADS;
+                if (x < v1) acc[u] = home_row[x];
+            }
+            for (int m = 0; m < n; ++m) {
+                V *rrow = rb + s_row[m] * PV;
+                V r[REDUCE_UNROLL];
+#pragma unroll
+                for (int u = 0; u < REDUCE_UNROLL; ++u) {
+                    const long long x = v + (long long)u * REDUCE_THREADS;
+                    if (x < v1) r[u] = rrow[x];
+                }
+#pragma unroll
+                for (int u = 0; u < REDUCE_UNROLL; ++u) {
+                    const long long x = v + (long long)u * REDUCE_THREADS;
+                    if (x < v1) {
+                        acc[u] = vadd(acc[u], r[u]);
+                        rrow[x] = vzero<V>();
+                    }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < REDUCE_UNROLL; ++u) {
+                const long long x = v + (long long)u * REDUCE_THREADS;
+                if (x < v1) home_row[x] = acc[u];
+            }
+        }
+    }
+}
+
+int launch_reduce(const Dims &d, const moonep_plan_t &p, float *reduce_buf, float *home_grad, long long P,
+                  cudaStream_t st)
+{
+    static int sms[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    if (!sms[dev]) {
+        int v = 0;
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+        sms[dev] = v > 0 ? v : 148;
+    }
+    ReduceParams a;
+    a.reduce_buf = reduce_buf;
+    a.home_grad = home_grad;
+    a.host_ptr = p.host_ptr;
+    a.host_rank = p.host_rank;
+    a.host_slot = p.host_slot;
+    a.rep_home_list = p.rep_home_list;
+    a.info = p.info;
+    a.L = d.L;
+    a.B = d.B;
+    a.E = d.E;
+    a.R = d.R;
+    a.n_hosts = 2 * d.E + d.R;
+    a.P = P;
+    const bool vec = (P % 4 == 0) && (reinterpret_cast<uintptr_t>(reduce_buf) % 16 == 0) &&
+                     (reinterpret_cast<uintptr_t>(home_grad) % 16 == 0);
+    const int grid = sms[dev] * (2048 / REDUCE_THREADS);
+    if (vec) {
+        a.chunk = (long long)REDUCE_THREADS * REDUCE_UNROLL * 8;
+        reduce_kernel<float4><<<grid, REDUCE_THREADS, 0, st>>>(a);
+    } else {
+        a.chunk = (long long)REDUCE_THREADS * REDUCE_UNROLL * 32;
+        reduce_kernel<float><<<grid, REDUCE_THREADS, 0, st>>>(a);
+    }
+    return cudaGetLastError() == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
+}
+
+}  // namespace moonep

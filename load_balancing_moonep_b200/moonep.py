@@ -1,0 +1,296 @@
+"""Thin Python binding of the MoonEP C ABI (include/moonep.h).
+
+Argument marshalling only: every step of the plan, permute, unpermute and
+reduction runs in the CUDA library ``_lib/libmoonep.so``.  PyTorch supplies
+device memory and the current stream.  Importing this module loads the
+library and raises ``ImportError`` if it has not been built -- there is no
+CPU fallback.
+
+Semantics (MoonEP article, "Moonshot AI Open-Sources MoonEP: A Perfectly
+Balanced Expert Parallelism Library for MoE Training", "The core idea:
+dynamic redundant experts"): ``plan`` places a few replicas of overloaded
+experts so that each of the R simulated ranks receives exactly S*K token
+slots; ``dispatch`` writes every (token, k) row straight into its
+expert-grouped slot of a static [R, S*K, H] buffer; ``combine`` is the
+weighted top-K unpermute; ``reduce_replica_grads`` sums replica gradients
+back into their home experts.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "libmoonep.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(
+        f"MoonEP CUDA library not built ({_LIB_PATH} missing): run "
+        "`python -m load_balancing_moonep_b200.build`")
+_lib = ctypes.CDLL(_LIB_PATH)
+
+FLAG_STRICT_BUDGET = 1
+FLAG_TRAIN_B_RULE = 2
+FLAG_BWD_UNSCALED = 4
+
+ST_EXPERT_ID_RANGE = 1
+ST_OVERFLOW = 2
+ST_STRICT_VIOLATION = 4
+ST_ROW_RANGE = 8
+
+INFO_FIELDS = ("status", "n_rep", "n_overflow", "n_pieces", "n_receivers",
+               "max_rep_per_rank", "n_rep_experts", "n_remote_pairs")
+INFO_LEN = 16
+
+PLAN_FIELDS = ("expert_count", "slot_expert", "slot_count", "slot_offset", "rep_expert", "rep_rank",
+               "rep_slot", "rep_quota", "host_ptr", "host_rank", "host_slot", "host_start",
+               "host_quota", "rep_home_list", "dst_pos", "row_src", "info")
+
+EXPORTED = ("moonep_check_config", "moonep_plan_sizes", "moonep_plan_layout", "moonep_plan",
+            "moonep_dispatch", "moonep_combine", "moonep_combine_backward",
+            "moonep_reduce_replica_grads", "moonep_error_string", "moonep_abi_version")
+
+
+class _CConfig(ctypes.Structure):
+    _fields_ = [("R", ctypes.c_int32), ("E", ctypes.c_int32), ("K", ctypes.c_int32),
+                ("S", ctypes.c_int32), ("H", ctypes.c_int32), ("B", ctypes.c_int32),
+                ("flags", ctypes.c_uint32)]
+
+
+class _CPlan(ctypes.Structure):
+    _fields_ = [(f, ctypes.c_void_p) for f in PLAN_FIELDS]
+
+
+_vp = ctypes.c_void_p
+_cfgp = ctypes.POINTER(_CConfig)
+_planp = ctypes.POINTER(_CPlan)
+_lib.moonep_check_config.argtypes = [_cfgp]
+_lib.moonep_plan_sizes.argtypes = [_cfgp, ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)]
+_lib.moonep_plan_layout.argtypes = [_cfgp, _vp, _planp]
+_lib.moonep_plan.argtypes = [_cfgp, _vp, _planp, _vp, _vp]
+_lib.moonep_dispatch.argtypes = [_cfgp, _planp, _vp, _vp, _vp]
+_lib.moonep_combine.argtypes = [_cfgp, _planp, _vp, _vp, _vp, _vp]
+_lib.moonep_combine_backward.argtypes = [_cfgp, _planp, _vp, _vp, _vp, _vp, _vp, _vp]
+_lib.moonep_reduce_replica_grads.argtypes = [_cfgp, _planp, _vp, _vp, ctypes.c_int64, _vp]
+_lib.moonep_error_string.argtypes = [ctypes.c_int]
+_lib.moonep_error_string.restype = ctypes.c_char_p
+_lib.moonep_abi_version.argtypes = []
+for _f in EXPORTED:
+    if _f not in ("moonep_error_string",):
+        getattr(_lib, _f).restype = ctypes.c_int
+
+LIB_PATH = _LIB_PATH
+
+
+class MoonepError(RuntimeError):
+    def __init__(self, code: int):
+        self.code = code
+        super().__init__(f"moonep error {code}: {_lib.moonep_error_string(code).decode()}")
+
+
+def _check(rc: int):
+    if rc != 0:
+        raise MoonepError(rc)
+
+
+@dataclass(frozen=True)
+class Config:
+    R: int
+    E: int
+    K: int
+    S: int
+    H: int
+    B: int
+    flags: int = 0
+
+    @property
+    def L(self) -> int:
+        return self.E // self.R
+
+    @property
+    def C(self) -> int:
+        return self.S * self.K
+
+    @property
+    def tokens(self) -> int:
+        return self.R * self.S
+
+    @property
+    def pairs(self) -> int:
+        return self.R * self.S * self.K
+
+    def c(self) -> _CConfig:
+        return _CConfig(self.R, self.E, self.K, self.S, self.H, self.B, self.flags)
+
+
+def check_config(cfg: Config) -> int:
+    c = cfg.c()
+    return _lib.moonep_check_config(ctypes.byref(c))
+
+
+def plan_sizes(cfg: Config):
+    c = cfg.c()
+    pb, wb = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    _check(_lib.moonep_plan_sizes(ctypes.byref(c), ctypes.byref(pb), ctypes.byref(wb)))
+    return pb.value, wb.value
+
+
+class Plan:
+    """Device plan block plus the planner workspace, with int32 views of
+    every field (shapes as in moonep.h)."""
+
+    def __init__(self, cfg: Config, device=None):
+        device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        self.cfg = cfg
+        pb, wb = plan_sizes(cfg)
+        self.block = torch.zeros(pb, dtype=torch.uint8, device=device)
+        # zero-filled once; every plan call leaves it zero-filled again
+        self.workspace = torch.zeros(max(wb, 256), dtype=torch.uint8, device=device)
+        self.c_plan = _CPlan()
+        c = cfg.c()
+        _check(_lib.moonep_plan_layout(ctypes.byref(c), self.block.data_ptr(), ctypes.byref(self.c_plan)))
+        R, E, K, S = cfg.R, cfg.E, cfg.K, cfg.S
+        shapes = {
+            "expert_count": (E,), "slot_expert": (R, E), "slot_count": (R, E),
+            "slot_offset": (R, E + 1), "rep_expert": (E + R,), "rep_rank": (E + R,),
+            "rep_slot": (E + R,), "rep_quota": (E + R,), "host_ptr": (E + 1,),
+            "host_rank": (2 * E + R,), "host_slot": (2 * E + R,), "host_start": (2 * E + R,),
+            "host_quota": (2 * E + R,), "rep_home_list": (E,), "dst_pos": (R * S, K),
+            "row_src": (R * S * K,), "info": (INFO_LEN,),
+        }
+        base = self.block.data_ptr()
+        i32 = self.block.view(torch.int32) if pb % 4 == 0 else None
+        self.fields = {}
+        for f in PLAN_FIELDS:
+            off = (getattr(self.c_plan, f) - base) // 4
+            n = 1
+            for s in shapes[f]:
+                n *= s
+            self.fields[f] = i32[off:off + n].view(shapes[f])
+
+    def __getattr__(self, name):
+        f = self.__dict__.get("fields")
+        if f is not None and name in f:
+            return f[name]
+        raise AttributeError(name)
+
+    def info(self) -> dict:
+        """Status and statistics (synchronises with the device)."""
+        v = self.fields["info"].cpu().tolist()
+        return {k: v[i] for i, k in enumerate(INFO_FIELDS)}
+
+    def to_numpy(self) -> dict:
+        return {k: v.cpu().numpy() for k, v in self.fields.items()}
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _need(t: torch.Tensor, dtype, shape, name):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def plan(cfg: Config, topk_idx: torch.Tensor, out: Plan | None = None, stream=None) -> Plan:
+    """Plan replicas and buffer rows for int32 top-K ids [R*S, K] (two
+    kernels, no host synchronisation)."""
+    _need(topk_idx, torch.int32, (cfg.tokens, cfg.K), "topk_idx")
+    p = Plan(cfg, topk_idx.device) if out is None else out
+    c = cfg.c()
+    _check(_lib.moonep_plan(ctypes.byref(c), topk_idx.data_ptr(), ctypes.byref(p.c_plan),
+                            p.workspace.data_ptr(), _stream(stream)))
+    return p
+
+
+def dispatch(cfg: Config, p: Plan, hidden: torch.Tensor, buf: torch.Tensor | None = None,
+             stream=None) -> torch.Tensor:
+    """buf[dst_pos[t, k]] = hidden[t]; returns the static [R, S*K, H] bf16 buffer."""
+    _need(hidden, torch.bfloat16, (cfg.tokens, cfg.H), "hidden")
+    if buf is None:
+        buf = torch.empty((cfg.R, cfg.C, cfg.H), dtype=torch.bfloat16, device=hidden.device)
+    _need(buf, torch.bfloat16, (cfg.R, cfg.C, cfg.H), "buf")
+    c = cfg.c()
+    _check(_lib.moonep_dispatch(ctypes.byref(c), ctypes.byref(p.c_plan), hidden.data_ptr(),
+                                buf.data_ptr(), _stream(stream)))
+    return buf
+
+
+def combine(cfg: Config, p: Plan, y: torch.Tensor, w: torch.Tensor, out: torch.Tensor | None = None,
+            stream=None) -> torch.Tensor:
+    """out[t] = bf16(sum_k w[t,k] * y[dst_pos[t,k]]), fp32 FMA in k order."""
+    _need(y, torch.bfloat16, (cfg.R, cfg.C, cfg.H), "y")
+    _need(w, torch.float32, (cfg.tokens, cfg.K), "w")
+    if out is None:
+        out = torch.empty((cfg.tokens, cfg.H), dtype=torch.bfloat16, device=y.device)
+    _need(out, torch.bfloat16, (cfg.tokens, cfg.H), "out")
+    c = cfg.c()
+    _check(_lib.moonep_combine(ctypes.byref(c), ctypes.byref(p.c_plan), y.data_ptr(), w.data_ptr(),
+                               out.data_ptr(), _stream(stream)))
+    return out
+
+
+def combine_backward(cfg: Config, p: Plan, dy: torch.Tensor, w: torch.Tensor, y: torch.Tensor,
+                     dy_buf: torch.Tensor | None = None, dw: torch.Tensor | None = None, stream=None):
+    """Returns (dy_buf [R, S*K, H] bf16, dw [R*S, K] fp32)."""
+    _need(dy, torch.bfloat16, (cfg.tokens, cfg.H), "dy")
+    _need(w, torch.float32, (cfg.tokens, cfg.K), "w")
+    _need(y, torch.bfloat16, (cfg.R, cfg.C, cfg.H), "y")
+    if dy_buf is None:
+        dy_buf = torch.empty((cfg.R, cfg.C, cfg.H), dtype=torch.bfloat16, device=dy.device)
+    if dw is None:
+        dw = torch.empty((cfg.tokens, cfg.K), dtype=torch.float32, device=dy.device)
+    _need(dy_buf, torch.bfloat16, (cfg.R, cfg.C, cfg.H), "dy_buf")
+    _need(dw, torch.float32, (cfg.tokens, cfg.K), "dw")
+    c = cfg.c()
+    _check(_lib.moonep_combine_backward(ctypes.byref(c), ctypes.byref(p.c_plan), dy.data_ptr(),
+                                        w.data_ptr(), y.data_ptr(), dy_buf.data_ptr(), dw.data_ptr(),
+                                        _stream(stream)))
+    return dy_buf, dw
+
+
+def reduce_replica_grads(cfg: Config, p: Plan, reduce_buf: torch.Tensor, home_grad: torch.Tensor,
+                         stream=None):
+    """home_grad[e] += replica grads of e (ascending rank), then zero them.
+    reduce_buf: fp32 [R, B, P]; home_grad: fp32 [E, P]."""
+    P = home_grad.shape[-1]
+    _need(home_grad, torch.float32, (cfg.E, P), "home_grad")
+    _need(reduce_buf, torch.float32, (cfg.R, cfg.B, P), "reduce_buf")
+    c = cfg.c()
+    _check(_lib.moonep_reduce_replica_grads(ctypes.byref(c), ctypes.byref(p.c_plan),
+                                            reduce_buf.data_ptr() if reduce_buf.numel() else None,
+                                            home_grad.data_ptr(), P, _stream(stream)))
+    return home_grad
+
+
+def views(cfg: Config, p: Plan, buf: torch.Tensor):
+    """Debug convenience: per-(rank, slot) (expert, view) lists of the
+    buffer.  Synchronises the host (slicing needs host offsets); the hot path
+    hands the device-side slot_offset/slot_count to a grouped GEMM instead."""
+    so = p.slot_offset.cpu()
+    se = p.slot_expert.cpu()
+    out = []
+    for r in range(cfg.R):
+        row = []
+        for s in range(cfg.E):
+            e = int(se[r, s])
+            if e < 0:
+                break
+            row.append((e, buf[r, int(so[r, s]):int(so[r, s + 1])]))
+        out.append(row)
+    return out
+
+
+def abi_version() -> int:
+    return _lib.moonep_abi_version()

@@ -1,0 +1,80 @@
+"""The C ABI library loads, exports every symbol its header declares, and its
+host-side checks agree with the oracle's configuration rules.  No GPU needed:
+none of these calls launches a kernel."""
+import re
+import os
+
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "moonep.h")).read()
+    return re.findall(r"MOONEP_API\s+[\w\s\*]+?\b(moonep_\w+)\s*\(", src)
+
+
+def test_header_declares_entry_points():
+    names = _declared()
+    for n in ("moonep_plan", "moonep_dispatch", "moonep_combine", "moonep_combine_backward",
+              "moonep_reduce_replica_grads", "moonep_plan_sizes", "moonep_plan_layout"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(cuda_lib_path):
+    import ctypes
+    lib = ctypes.CDLL(cuda_lib_path)
+    for n in _declared():
+        assert hasattr(lib, n), n
+
+
+def test_binding_loads(cuda_lib_path):
+    from load_balancing_moonep_b200 import moonep
+    assert moonep.abi_version() == 1
+    for n in _declared():
+        assert n in moonep.EXPORTED
+
+
+def test_config_checks_match_oracle(cuda_lib_path):
+    from load_balancing_moonep_b200 import moonep
+    cases = [
+        dict(R=4, E=16, K=2, S=8, H=8, B=2),
+        dict(R=3, E=16, K=2, S=8, H=8, B=2),
+        dict(R=4, E=16, K=2, S=8, H=8, B=3, flags=2),
+        dict(R=4, E=16, K=2, S=8, H=8, B=4, flags=2),
+        dict(R=4, E=16, K=2, S=8, H=8, B=13),
+        dict(R=4, E=16, K=17, S=8, H=8, B=2),
+        dict(R=0, E=16, K=2, S=8, H=8, B=2),
+        dict(R=4, E=16, K=2, S=0, H=8, B=2),
+        dict(R=32, E=384, K=8, S=4096, H=7168, B=12, flags=2),
+        dict(R=64, E=384, K=8, S=128, H=7168, B=4),
+    ]
+    for c in cases:
+        assert moonep.check_config(moonep.Config(**c)) == oracle.check_config(oracle.Config(**c)), c
+    # CUDA-only limits
+    assert moonep.check_config(moonep.Config(R=4, E=16, K=2, S=8, H=12, B=2)) == 8
+    assert moonep.check_config(moonep.Config(R=2, E=2048, K=2, S=8, H=8, B=2)) == 7
+    with pytest.raises(moonep.MoonepError):
+        moonep.plan_sizes(moonep.Config(R=3, E=16, K=2, S=8, H=8, B=2))
+
+
+def test_plan_sizes_and_layout(cuda_lib_path):
+    import ctypes
+    from load_balancing_moonep_b200 import moonep
+    cfg = moonep.Config(R=32, E=384, K=8, S=4096, H=7168, B=12)
+    pb, wb = moonep.plan_sizes(cfg)
+    n_pairs = cfg.pairs
+    assert pb >= 4 * (2 * n_pairs + 384 + 3 * 32 * 385) and pb % 256 == 0
+    assert wb >= 4 * 384 and wb % 256 == 0
+    # layout of a fake, 256-aligned base address: host arithmetic only
+    base = 1 << 40
+    cp = moonep._CPlan()
+    c = cfg.c()
+    assert moonep._lib.moonep_plan_layout(ctypes.byref(c), base, ctypes.byref(cp)) == 0
+    offs = [getattr(cp, f) - base for f in moonep.PLAN_FIELDS]
+    assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+    assert offs[-1] < pb
+    # misaligned base is rejected
+    assert moonep._lib.moonep_plan_layout(ctypes.byref(c), base + 16, ctypes.byref(cp)) == 8

@@ -1,0 +1,343 @@
+"""GPU parity: the CUDA library (through its C ABI) against the CPU oracle on
+identical seeded inputs.
+
+Bars: plan, counts, offsets, dst_pos, row_src and dispatched rows bit-exact;
+combine and dy_buf bit-exact (same fp32 fused multiply-add order and one
+round-to-nearest-even); replica-gradient reduce bit-exact (same fp32 add
+order); dw within |dw - ref| <= 1e-5 * sum_h |dy*y| + 1e-30 (GPU reduction
+tree in fp32 vs the oracle's fp64 sum; the tree's worst-case bound is
+(8 + H/256 + 5) * 2^-24 relative to sum |dy*y|, under 1e-5 for H <= 37k).
+
+Small cases compare every element; the full-size configurations (large
+training shape, decode) compare the whole plan and sampled tokens / rows /
+element ranges of the data steps, run in the launch configuration the
+benchmark times.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from load_balancing_moonep_b200 import workloads as W
+from plan_checks import check_invariants, check_water_filling
+
+pytestmark = pytest.mark.gpu
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module")
+def mp(oracle_lib, cuda_lib_path):
+    if not torch.cuda.is_available():
+        pytest.fail("CUDA device required for -m gpu tests")
+    from load_balancing_moonep_b200 import moonep
+    return moonep
+
+
+def _cfgs(c: dict, mp):
+    return mp.Config(**c), oracle.Config(**c)
+
+
+def _plan_both(mp, c: dict, topk: np.ndarray):
+    gcfg, ocfg = _cfgs(c, mp)
+    t = torch.from_numpy(np.ascontiguousarray(topk, np.int32)).to(DEV)
+    gp = mp.plan(gcfg, t)
+    torch.cuda.synchronize()
+    return gcfg, ocfg, gp, oracle.plan(ocfg, topk)
+
+
+def _assert_plan_equal(gp, op):
+    g = gp.to_numpy()
+    for k, v in op.items():
+        assert np.array_equal(g[k], v), f"plan field {k} differs"
+
+
+def _wl_cfg(wl, **kw):
+    d = dict(R=wl.R, E=wl.E, K=wl.K, S=wl.S, H=wl.H, B=wl.B, flags=0)
+    d.update(kw)
+    return d
+
+
+# ------------------------------------------------------------------ plan
+
+@pytest.mark.parametrize("name", ["plan_example_a", "plan_example_b"])
+@pytest.mark.parametrize("flags", [0, 1])
+def test_plan_golden(mp, name, flags):
+    g = json.load(open(os.path.join(GOLDEN, name + ".json")))
+    c = {**g["config"], "flags": flags}
+    topk = np.array(g["topk_idx"], np.int32)
+    gcfg, ocfg, gp, op = _plan_both(mp, c, topk)
+    _assert_plan_equal(gp, op)
+    for k, v in g["expect"].items():
+        if k != "info":
+            assert gp.fields[k].cpu().numpy().tolist() == v
+
+
+@pytest.mark.parametrize("wname,mv,adv", [
+    ("tiny", 0.0, False), ("tiny", 1.0, False), ("tiny", 1.0, True), ("tiny", 3.0, False),
+    ("mid", 0.0, False), ("mid", 0.5, False), ("mid", 1.0, False), ("mid", 2.0, False),
+    ("mid", 3.0, False), ("mid", 3.0, True),
+    ("decode", 5.0, False), ("decode", 13.4, False), ("decode", 20.0, False),
+])
+def test_plan_workloads(mp, wname, mv, adv):
+    wl = W.WORKLOADS[wname]
+    r = W.routing(wl, mv, seed=0, adversarial=adv, device=DEV)
+    topk = r.topk_idx.cpu().numpy()
+    gcfg, ocfg, gp, op = _plan_both(mp, _wl_cfg(wl), topk)
+    _assert_plan_equal(gp, op)
+    check_invariants(ocfg, topk, gp.to_numpy())
+
+
+@pytest.mark.parametrize("mv,adv", [(0.0, False), (1.0, False), (3.0, False), (3.0, True)])
+def test_plan_large_full_size(mp, mv, adv):
+    wl = W.WORKLOADS["large"]
+    r = W.routing(wl, mv, seed=0, adversarial=adv, device=DEV)
+    topk = r.topk_idx.cpu().numpy()
+    gcfg, ocfg, gp, op = _plan_both(mp, _wl_cfg(wl), topk)
+    _assert_plan_equal(gp, op)
+    check_invariants(ocfg, topk, gp.to_numpy())
+    check_water_filling(ocfg, topk, gp.to_numpy())
+
+
+@pytest.mark.parametrize("seed", range(16))
+def test_plan_random_shapes(mp, seed):
+    # ragged shapes: token counts that are not multiples of the chunk size,
+    # every L, B from 0 to E-L, heavy and light skew
+    rng = np.random.default_rng(100 + seed)
+    R = int(rng.choice([1, 2, 3, 5, 8, 16, 64]))
+    L = int(rng.choice([1, 2, 3, 7, 12]))
+    E = R * L
+    if E > 1024:
+        L = max(1, 1024 // R)
+        E = R * L
+    K = int(rng.integers(1, min(E, 9) + 1))
+    S = int(rng.integers(1, 300))
+    B = int(rng.integers(0, E - L + 1))
+    skew = float(rng.uniform(0, 3))
+    w = np.arange(1, E + 1, dtype=np.float64) ** (-skew)
+    w = w[rng.permutation(E)]
+    w /= w.sum()
+    topk = np.stack([rng.choice(E, size=K, replace=False, p=w) for _ in range(R * S)]).astype(np.int32)
+    c = dict(R=R, E=E, K=K, S=S, H=8, B=B, flags=int(rng.integers(0, 2)))
+    gcfg, ocfg, gp, op = _plan_both(mp, c, topk)
+    _assert_plan_equal(gp, op)
+    check_invariants(ocfg, topk, gp.to_numpy())
+
+
+def test_plan_duplicates_within_token(mp):
+    # the pages are silent on repeated ids in one token's top-K: they are
+    # independent pairs; both sides must agree
+    rng = np.random.default_rng(5)
+    topk = rng.integers(0, 8, size=(4 * 20, 3)).astype(np.int32)
+    _, ocfg, gp, op = _plan_both(mp, dict(R=4, E=8, K=3, S=20, H=8, B=2), topk)
+    _assert_plan_equal(gp, op)
+
+
+def test_plan_all_on_one_expert_and_max_E(mp):
+    topk = np.zeros((64 * 5, 1), np.int32)
+    _, _, gp, op = _plan_both(mp, dict(R=64, E=128, K=1, S=5, H=8, B=2), topk)
+    _assert_plan_equal(gp, op)
+    assert gp.info()["n_rep"] == 63
+    rng = np.random.default_rng(9)
+    topk = rng.integers(0, 1024, size=(1024 * 4, 4)).astype(np.int32)
+    topk[: 1024, :] = 0  # one very hot expert
+    _, ocfg, gp, op = _plan_both(mp, dict(R=1024, E=1024, K=4, S=4, H=8, B=1), topk)
+    _assert_plan_equal(gp, op)
+    check_invariants(ocfg, topk, gp.to_numpy())
+
+
+def test_plan_bad_ids_status_and_noop(mp):
+    c = dict(R=4, E=16, K=2, S=64, H=64, B=2)
+    rng = np.random.default_rng(1)
+    topk = rng.integers(0, 16, size=(256, 2)).astype(np.int32)
+    topk[77, 1] = 16
+    gcfg, ocfg, gp, op = _plan_both(mp, c, topk)
+    _assert_plan_equal(gp, op)
+    assert gp.info()["status"] & mp.ST_EXPERT_ID_RANGE
+    hidden = W.hidden_states(W.Workload("x", 4, 16, 2, 64, 64, 2), seed=3, device=DEV)
+    buf = torch.full((4, 128, 64), 7.0, dtype=torch.bfloat16, device=DEV)
+    mp.dispatch(gcfg, gp, hidden, buf)
+    out = torch.full((256, 64), 5.0, dtype=torch.bfloat16, device=DEV)
+    mp.combine(gcfg, gp, buf, torch.ones(256, 2, device=DEV), out)
+    torch.cuda.synchronize()
+    assert (buf == 7.0).all() and (out == 5.0).all()
+    # a following valid plan with the same workspace is unaffected
+    topk[77, 1] = 3
+    t = torch.from_numpy(topk).to(DEV)
+    gp2 = mp.plan(gcfg, t, out=gp)
+    _assert_plan_equal(gp2, oracle.plan(ocfg, topk))
+
+
+def test_plan_repeat_deterministic(mp):
+    wl = W.WORKLOADS["mid"]
+    r = W.routing(wl, 2.0, device=DEV)
+    cfg = mp.Config(**_wl_cfg(wl))
+    p1 = mp.plan(cfg, r.topk_idx).to_numpy()
+    p = mp.Plan(cfg)
+    for _ in range(3):
+        p2 = mp.plan(cfg, r.topk_idx, out=p).to_numpy()
+        for k in p1:
+            assert np.array_equal(p1[k], p2[k])
+
+
+def test_host_errors(mp):
+    with pytest.raises(mp.MoonepError):
+        mp.plan(mp.Config(R=3, E=16, K=2, S=8, H=8, B=2), torch.zeros(24, 2, dtype=torch.int32, device=DEV))
+    with pytest.raises(ValueError):
+        mp.plan(mp.Config(R=4, E=16, K=2, S=8, H=8, B=2), torch.zeros(32, 3, dtype=torch.int32, device=DEV))
+    cfg = mp.Config(R=4, E=16, K=2, S=8, H=8, B=2)
+    p = mp.plan(cfg, torch.zeros(32, 2, dtype=torch.int32, device=DEV))
+    h = torch.zeros(32 * 8 + 1, dtype=torch.bfloat16, device=DEV)[1:].view(32, 8)  # misaligned
+    with pytest.raises(mp.MoonepError):
+        mp.dispatch(cfg, p, h)
+    big = mp.Config(R=4, E=64, K=17, S=8, H=8, B=2)
+    pb = mp.plan(big, torch.zeros(32, 17, dtype=torch.int32, device=DEV))
+    z = torch.zeros(32, 8, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(mp.MoonepError):
+        mp.combine_backward(big, pb, z, torch.zeros(32, 17, device=DEV),
+                            torch.zeros(4, 8 * 17, 8, dtype=torch.bfloat16, device=DEV))
+
+
+# ------------------------------------------------------------- data steps
+
+def _sub_plan(op, tokens, K):
+    """Index plumbing for sampled parity: the sampled tokens' rows, renumbered
+    0..n*K-1, so the oracle reads exactly the rows the GPU read."""
+    dp = op["dst_pos"][tokens]                        # [n, K] original rows
+    compact = np.arange(dp.size, dtype=np.int32).reshape(dp.shape)
+    return {"dst_pos": compact, "info": op["info"]}, dp.ravel()
+
+
+@pytest.mark.parametrize("wname,mv", [("tiny", 1.0), ("tiny", 0.0), ("mid", 0.0), ("mid", 1.0),
+                                      ("mid", 3.0)])
+def test_data_steps_full(mp, wname, mv):
+    wl = W.WORKLOADS[wname]
+    r = W.routing(wl, mv, device=DEV)
+    topk = r.topk_idx.cpu().numpy()
+    c = _wl_cfg(wl)
+    gcfg, ocfg, gp, op = _plan_both(mp, c, topk)
+    _assert_plan_equal(gp, op)
+    hidden = W.hidden_states(wl, seed=1, device=DEV)
+    # dispatch: every buffer row
+    buf = torch.full((wl.R, wl.C, wl.H), float("nan"), dtype=torch.bfloat16, device=DEV)
+    mp.dispatch(gcfg, gp, hidden, buf)
+    ob = np.zeros((wl.R, wl.C, wl.H), np.uint16)
+    oracle.dispatch(ocfg, op, W.bits(hidden), ob)
+    assert np.array_equal(W.bits(buf), ob)
+    # combine on independent expert outputs y
+    y = W.bf16_normal((wl.R, wl.C, wl.H), seed=2, device=DEV)
+    w = r.weights
+    out = mp.combine(gcfg, gp, y, w)
+    oo = oracle.combine(ocfg, op, W.bits(y), w.cpu().numpy())
+    assert np.array_equal(W.bits(out), oo)
+    # combine backward
+    dy = W.bf16_normal((wl.tokens, wl.H), seed=3, device=DEV)
+    dyb, dw = mp.combine_backward(gcfg, gp, dy, w, y)
+    odyb = np.zeros_like(ob)
+    odw = np.zeros((wl.tokens, wl.K), np.float32)
+    oracle.combine_backward(ocfg, op, W.bits(dy), w.cpu().numpy(), W.bits(y), odyb, odw)
+    assert np.array_equal(W.bits(dyb), odyb)
+    dyf = dy.float().cpu().numpy().astype(np.float64)
+    yf = y.float().cpu().numpy().reshape(-1, wl.H).astype(np.float64)
+    mag = np.einsum("th,tkh->tk", np.abs(dyf), np.abs(yf[op["dst_pos"]]))
+    assert (np.abs(dw.cpu().numpy().astype(np.float64) - odw) <= 1e-5 * mag + 1e-30).all()
+    assert gp.info()["status"] == op["info"][0]  # no row-range fault raised by the data kernels
+
+
+@pytest.mark.parametrize("wname,mv", [("large", 1.0), ("large", 3.0), ("decode", 5.0)])
+def test_data_steps_full_size_sampled(mp, wname, mv):
+    wl = W.WORKLOADS[wname]
+    r = W.routing(wl, mv, device=DEV)
+    topk = r.topk_idx.cpu().numpy()
+    gcfg, ocfg, gp, op = _plan_both(mp, _wl_cfg(wl), topk)
+    _assert_plan_equal(gp, op)
+    rng = np.random.default_rng(0)
+    tokens = np.unique(np.concatenate([rng.choice(wl.tokens, 192, replace=False),
+                                       [0, wl.S - 1, wl.tokens - 1]]))
+    n = len(tokens)
+    sub, rows = _sub_plan(op, tokens, wl.K)
+    scfg = oracle.Config(R=1, E=wl.E, K=wl.K, S=n, H=wl.H, B=0)
+    hidden = W.hidden_states(wl, seed=1, device=DEV)
+    buf = torch.empty((wl.R, wl.C, wl.H), dtype=torch.bfloat16, device=DEV)
+    mp.dispatch(gcfg, gp, hidden, buf)
+    # dispatch: the sampled tokens' K rows, and every row owner check via row_src
+    hb = W.bits(hidden[torch.from_numpy(tokens).to(DEV)])
+    ob = np.zeros((n * wl.K, wl.H), np.uint16)
+    oracle.dispatch(scfg, sub, hb, ob)
+    got = W.bits(buf.view(-1, wl.H)[torch.from_numpy(rows.astype(np.int64)).to(DEV)])
+    assert np.array_equal(got, ob)
+    # every buffer row holds the token that row_src says it holds
+    rs = torch.from_numpy(op["row_src"].astype(np.int64)).to(DEV)
+    sample_rows = torch.from_numpy(rng.choice(wl.pairs, 4096, replace=False)).to(DEV)
+    assert torch.equal(buf.view(-1, wl.H)[sample_rows], hidden[rs[sample_rows] // wl.K])
+    # combine and backward on independent y / dy, sampled tokens
+    del buf
+    y = W.bf16_normal((wl.R, wl.C, wl.H), seed=2, device=DEV)  # independent expert outputs
+    w = r.weights
+    out = mp.combine(gcfg, gp, y, w)
+    tt = torch.from_numpy(tokens).to(DEV)
+    yrows = W.bits(y.view(-1, wl.H)[torch.from_numpy(rows.astype(np.int64)).to(DEV)])
+    ws = w[tt].cpu().numpy()
+    oo = oracle.combine(scfg, sub, yrows, ws)
+    assert np.array_equal(W.bits(out[tt]), oo)
+    dy = W.bf16_normal((wl.tokens, wl.H), seed=3, device=DEV)
+    dyb, dw = mp.combine_backward(gcfg, gp, dy, w, y)
+    odyb = np.zeros((n * wl.K, wl.H), np.uint16)
+    odw = np.zeros((n, wl.K), np.float32)
+    oracle.combine_backward(scfg, sub, W.bits(dy[tt]), ws, yrows, odyb, odw)
+    assert np.array_equal(W.bits(dyb.view(-1, wl.H)[torch.from_numpy(rows.astype(np.int64)).to(DEV)]), odyb)
+    dyf = dy[tt].float().cpu().numpy().astype(np.float64)
+    yf = y.view(-1, wl.H)[torch.from_numpy(rows.astype(np.int64)).to(DEV)].float().cpu().numpy()
+    mag = np.einsum("th,tkh->tk", np.abs(dyf), np.abs(yf.astype(np.float64).reshape(n, wl.K, wl.H)))
+    assert (np.abs(dw[tt].cpu().numpy().astype(np.float64) - odw) <= 1e-5 * mag + 1e-30).all()
+
+
+# ---------------------------------------------------------------- reduce
+
+@pytest.mark.parametrize("wname,mv,P", [("tiny", 1.0, 1000), ("tiny", 1.0, 1003), ("mid", 3.0, 4096),
+                                        ("large", 3.0, 2048), ("decode", 13.4, 517)])
+def test_reduce_full(mp, wname, mv, P):
+    wl = W.WORKLOADS[wname]
+    r = W.routing(wl, mv, device=DEV)
+    topk = r.topk_idx.cpu().numpy()
+    gcfg, ocfg, gp, op = _plan_both(mp, _wl_cfg(wl), topk)
+    rb = W.f32_normal((wl.R, wl.B, P), seed=4, device=DEV, std=1e-3)
+    hg = W.f32_normal((wl.E, P), seed=5, device=DEV, std=1e-3)
+    orb, ohg = rb.cpu().numpy(), hg.cpu().numpy()
+    mp.reduce_replica_grads(gcfg, gp, rb, hg)
+    oracle.reduce_replica_grads(ocfg, op, orb, ohg, P)
+    assert np.array_equal(hg.cpu().numpy(), ohg)
+    assert np.array_equal(rb.cpu().numpy(), orb)
+    assert gp.info()["n_rep_experts"] == op["info"][6]
+
+
+def test_reduce_full_size_sampled(mp):
+    # the large training shape's real gradient size (gate + up + down,
+    # 3 * 7168 * 2048 fp32 per expert), compared on sampled element ranges
+    wl = W.WORKLOADS["large"]
+    P = wl.grad_elems
+    need = 4 * P * (wl.R * wl.B + wl.E) * 1.1
+    torch.cuda.empty_cache()
+    free, _ = torch.cuda.mem_get_info()
+    if need > free:
+        pytest.skip(f"needs {need / 1e9:.0f} GB of device memory, {free / 1e9:.0f} GB free")
+    r = W.routing(wl, 1.0, device=DEV)
+    topk = r.topk_idx.cpu().numpy()
+    gcfg, ocfg, gp, op = _plan_both(mp, _wl_cfg(wl), topk)
+    rb = W.f32_normal((wl.R, wl.B, P), seed=4, device=DEV, std=1e-3)
+    hg = W.f32_normal((wl.E, P), seed=5, device=DEV, std=1e-3)
+    ranges = [(0, 4096), (P // 2 - 1000, P // 2 + 3001), (P - 5003, P)]
+    before = [(rb[:, :, a:b].cpu().numpy().copy(), hg[:, a:b].cpu().numpy().copy()) for a, b in ranges]
+    mp.reduce_replica_grads(gcfg, gp, rb, hg)
+    for (a, b), (orb, ohg) in zip(ranges, before):
+        orb = np.ascontiguousarray(orb)
+        ohg = np.ascontiguousarray(ohg)
+        oracle.reduce_replica_grads(ocfg, op, orb, ohg, b - a)
+        assert np.array_equal(hg[:, a:b].cpu().numpy(), ohg)
+        assert np.array_equal(rb[:, :, a:b].cpu().numpy(), orb)
+    del rb, hg
+    torch.cuda.empty_cache()

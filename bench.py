@@ -521,6 +521,39 @@ def run_ours(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+def run_profile_case(args):
+    """--profile: two passes of the whole step on a reduced-size copy of the
+    workload (S tokens per rank, P gradient elements), a few GB on the
+    device, for ncu captures; prints a one-line summary, no timing."""
+    from load_balancing_moonep_b200 import moonep as mp
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    wl = W.WORKLOADS[args.workload].with_(S=args.profile_S)
+    cfg = mp.Config(R=wl.R, E=wl.E, K=wl.K, S=wl.S, H=wl.H, B=wl.B)
+    r = W.routing(wl, args.maxvio, seed=0, device=dev)
+    hidden = W.hidden_states(wl, seed=1, device=dev)
+    dy = W.bf16_normal((wl.tokens, wl.H), seed=3, device=dev)
+    buf = torch.empty((wl.R, wl.C, wl.H), dtype=torch.bfloat16, device=dev)
+    dy_buf = torch.empty_like(buf)
+    out = torch.empty((wl.tokens, wl.H), dtype=torch.bfloat16, device=dev)
+    P = args.profile_P
+    rb = W.f32_normal((wl.R, wl.B, P), seed=4, device=dev, std=1e-3)
+    hg = W.f32_normal((wl.E, P), seed=5, device=dev, std=1e-3)
+    plan = mp.Plan(cfg, dev)
+    for _ in range(2):
+        mp.plan(cfg, r.topk_idx, out=plan)
+        mp.dispatch(cfg, plan, hidden, buf)
+        mp.combine(cfg, plan, buf, r.weights, out)
+        mp.combine_backward(cfg, plan, dy, r.weights, buf, dy_buf)
+        mp.reduce_replica_grads(cfg, plan, rb, hg)
+    torch.cuda.synchronize()
+    info = plan.info()
+    print(json.dumps({"profile_case": f"{wl.name} S={wl.S} P={P}", "tokens": wl.tokens, "P": P,
+                      "n_rep": info["n_rep"], "n_overflow": info["n_overflow"],
+                      "n_rep_experts": info["n_rep_experts"],
+                      "device_GB": round(torch.cuda.max_memory_allocated() / 1e9, 2)}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -534,7 +567,14 @@ def main():
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="run two untimed steps of a reduced-size case (for ncu)")
+    ap.add_argument("--profile-S", type=int, default=512)
+    ap.add_argument("--profile-P", type=int, default=1 << 20)
     args = ap.parse_args()
+    if args.profile:
+        run_profile_case(args)
+        return
     if args.warmup < 3:
         log("warmup raised to 3 (timing rule)")
         args.warmup = 3

@@ -44,6 +44,7 @@ static int make_dims(const moonep_config *c, Dims *d)
     if (ct > d->tokens) ct = d->tokens;
     d->chunk_tokens = ct;
     d->nchunk = (d->tokens + ct - 1) / ct;
+    d->ngroups = (d->nchunk + CHUNK_GROUP - 1) / CHUNK_GROUP;
     if (plan_smem_bytes_max(*d) > MAX_DYN_SMEM) return MOONEP_ERR_LIMIT;
     return MOONEP_OK;
 }

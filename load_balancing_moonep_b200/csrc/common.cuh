@@ -19,13 +19,19 @@ struct Dims {
     int pairs;    // R*S*K
     int nchunk;   // planner token chunks
     int chunk_tokens;
+    int ngroups;  // groups of CHUNK_GROUP consecutive chunks
 };
+
+// Chunks per group: the assignment pass sums at most CHUNK_GROUP - 1
+// per-chunk counts on top of a group prefix.
+constexpr int CHUNK_GROUP = 16;
 
 // Workspace layout (bytes from the workspace base; 256-byte aligned parts).
 struct WsLayout {
     size_t ticket;     // int32: CTAs of the histogram kernel that finished
     size_t status;     // int32: status bits collected by the histogram kernel
-    size_t t_acc;      // int32 [E]: global expert counts being accumulated
+    size_t gs;         // int32 [ngroups][E]: per-group expert counts (atomic sums)
+    size_t gp;         // int32 [ngroups][E]: exclusive prefix of gs over groups
     size_t cc;         // int32 [nchunk][E]: per-chunk expert counts
     size_t host_dst0;  // int32 [2E+R]: rank*C + slot_offset - host_start per host
     size_t total;
@@ -40,7 +46,8 @@ __host__ inline WsLayout ws_layout(const Dims &d)
     w.ticket = o; o += 4;
     w.status = o; o += 4;
     o = align256(o);
-    w.t_acc = o; o = align256(o + sizeof(int32_t) * d.E);
+    w.gs = o; o = align256(o + sizeof(int32_t) * (size_t)d.ngroups * d.E);
+    w.gp = o; o = align256(o + sizeof(int32_t) * (size_t)d.ngroups * d.E);
     w.cc = o; o = align256(o + sizeof(int32_t) * (size_t)d.nchunk * d.E);
     w.host_dst0 = o; o = align256(o + sizeof(int32_t) * (size_t)(2 * d.E + d.R));
     w.total = o;

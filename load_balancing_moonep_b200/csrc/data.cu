@@ -234,24 +234,39 @@ __global__ void __launch_bounds__(DATA_THREADS) combine_bwd_kernel(
                 const int c = c0 + u * 32 + lane;
                 if (c < vpr) unpack8(ld_stream(g + c), gf[u]);
             }
+            // all K expert-output rows of this vector slice in flight first
+            uint4 yv[K][U];
+            unsigned okm = 0;
+#pragma unroll
+            for (int k = 0; k < K; ++k) {
+                const int dk = __shfl_sync(FULL_MASK, dl, k);
+                const bool ok = row_ok(dk, rows, info);
+                okm |= ok ? (1u << k) : 0u;
+                const uint4 *yr = y + (size_t)(ok ? dk : 0) * vpr;
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int c = c0 + u * 32 + lane;
+                    yv[k][u] = make_uint4(0u, 0u, 0u, 0u);
+                    if (ok && c < vpr) yv[k][u] = ld_stream(yr + c);
+                }
+            }
 #pragma unroll
             for (int k = 0; k < K; ++k) {
                 const int dk = __shfl_sync(FULL_MASK, dl, k);
                 const float wk = __shfl_sync(FULL_MASK, wl, k);
-                if (!row_ok(dk, rows, info)) continue;
-                const uint4 *yr = y + (size_t)dk * vpr;
+                if (!(okm & (1u << k))) continue;
                 uint4 *br = dy_buf + (size_t)dk * vpr;
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
                     const int c = c0 + u * 32 + lane;
                     if (c < vpr) {
                         float yf[8];
-                        unpack8(ld_stream(yr + c), yf);
+                        unpack8(yv[k][u], yf);
                         dacc[k] += dot8(gf[u], yf);
-                        float s[8];
+                        float sc[8];
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) s[j] = unscaled ? gf[u][j] : __fmul_rn(wk, gf[u][j]);
-                        st_vec(br + c, pack8(s));
+                        for (int j = 0; j < 8; ++j) sc[j] = unscaled ? gf[u][j] : __fmul_rn(wk, gf[u][j]);
+                        st_vec(br + c, pack8(sc));
                     }
                 }
             }
@@ -319,7 +334,8 @@ template <int KT>
 static void launch_bwd_k(const Dims &d, int grid, const uint4 *dy, const float *w, const uint4 *y, uint4 *dyb,
                          float *dw, const int *dst_pos, int *info, int unscaled, cudaStream_t st)
 {
-    combine_bwd_kernel<KT, 2><<<grid, DATA_THREADS, 0, st>>>(dy, w, y, dyb, dw, dst_pos, info, d.tokens,
+    constexpr int U = KT <= 8 ? 2 : 1;
+    combine_bwd_kernel<KT, U><<<grid, DATA_THREADS, 0, st>>>(dy, w, y, dyb, dw, dst_pos, info, d.tokens,
                                                             d.H / 8, unscaled, d.pairs);
 }
 

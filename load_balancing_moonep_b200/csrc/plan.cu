@@ -32,7 +32,8 @@ struct PlanParams {
     moonep_plan_t p;
     int *ticket;
     int *status;
-    int *t_acc;
+    int *gs;
+    int *gp;
     int *cc;
     int *host_dst0;
 };
@@ -122,12 +123,19 @@ __device__ void plan_block(const PlanParams &a, int *sm)
     for (int i = tid; i < 16; i += nt) misc[i] = 0;
     __syncthreads();
 
-    // ---- totals from the histogram pass; leave the workspace zeroed
+    // ---- totals from the histogram pass: exclusive prefix of the group
+    // counts for the assignment pass; leave the group counts zeroed
+    const int ng = d.ngroups;
     for (int e = tid; e < E; e += nt) {
-        int v = ld_cg(a.t_acc + e);
-        T[e] = v;
-        a.t_acc[e] = 0;
-        a.p.expert_count[e] = v;
+        int run = 0;
+        for (int g = 0; g < ng; ++g) {
+            const int v = ld_cg(a.gs + (size_t)g * E + e);
+            a.gs[(size_t)g * E + e] = 0;
+            a.gp[(size_t)g * E + e] = run;
+            run += v;
+        }
+        T[e] = run;
+        a.p.expert_count[e] = run;
     }
     if (tid == 0) {
         misc[0] = ld_cg(a.status);
@@ -421,10 +429,11 @@ __global__ void __launch_bounds__(PLAN_THREADS, 1) hist_plan_kernel(PlanParams a
         if (ok && lane == __ffs(peers) - 1) atomicAdd(&hist[e], __popc(peers));
     }
     bad = __syncthreads_or(bad);
+    const int grp = chunk / CHUNK_GROUP;
     for (int e = tid; e < E; e += nt) {
         const int c = hist[e];
         a.cc[(size_t)chunk * E + e] = c;
-        if (c) atomicAdd(a.t_acc + e, c);
+        if (c) atomicAdd(a.gs + (size_t)grp * E + e, c);  // commutative: order-free
     }
     if (bad && tid == 0) atomicOr(a.status, MOONEP_ST_EXPERT_ID_RANGE);
     __threadfence();
@@ -441,6 +450,7 @@ struct AssignParams {
     const int32_t *topk;
     moonep_plan_t p;
     const int *cc;
+    const int *gp;
     const int *host_dst0;
 };
 
@@ -480,17 +490,20 @@ __global__ void __launch_bounds__(ASSIGN_THREADS) assign_kernel(AssignParams a)
         hstart[h] = a.p.host_start[h];
         hdst[h] = a.host_dst0[h];
     }
-    for (int e = tid; e < E; e += nt) {
-        int s0 = 0, s1 = 0, s2 = 0, s3 = 0;
-        int c = 0;
-        for (; c + 4 <= chunk; c += 4) {
-            s0 += __ldg(a.cc + (size_t)(c + 0) * E + e);
-            s1 += __ldg(a.cc + (size_t)(c + 1) * E + e);
-            s2 += __ldg(a.cc + (size_t)(c + 2) * E + e);
-            s3 += __ldg(a.cc + (size_t)(c + 3) * E + e);
+    // pairs of each expert in earlier chunks: group prefix + earlier chunks
+    // of this chunk's group (at most CHUNK_GROUP - 1 independent loads)
+    {
+        const int grp = chunk / CHUNK_GROUP, c0 = grp * CHUNK_GROUP;
+        for (int e = tid; e < E; e += nt) {
+            int s = __ldg(a.gp + (size_t)grp * E + e);
+            int v[CHUNK_GROUP - 1];
+#pragma unroll
+            for (int j = 0; j < CHUNK_GROUP - 1; ++j)
+                v[j] = (c0 + j < chunk) ? __ldg(a.cc + (size_t)(c0 + j) * E + e) : 0;
+#pragma unroll
+            for (int j = 0; j < CHUNK_GROUP - 1; ++j) s += v[j];
+            base[e] = s;
         }
-        for (; c < chunk; ++c) s0 += __ldg(a.cc + (size_t)c * E + e);
-        base[e] = s0 + s1 + s2 + s3;
     }
     for (int i = tid; i < ASSIGN_WARPS * E; i += nt) cnt[i] = 0;
     for (int i = tid; i < n; i += nt) ids[i] = __ldg(a.topk + p0 + i);
@@ -574,7 +587,8 @@ int launch_plan(const Dims &d, const int32_t *topk, const moonep_plan_t &p, void
     a.p = p;
     a.ticket = reinterpret_cast<int *>(w + wl.ticket);
     a.status = reinterpret_cast<int *>(w + wl.status);
-    a.t_acc = reinterpret_cast<int *>(w + wl.t_acc);
+    a.gs = reinterpret_cast<int *>(w + wl.gs);
+    a.gp = reinterpret_cast<int *>(w + wl.gp);
     a.cc = reinterpret_cast<int *>(w + wl.cc);
     a.host_dst0 = reinterpret_cast<int *>(w + wl.host_dst0);
 
@@ -590,6 +604,7 @@ int launch_plan(const Dims &d, const int32_t *topk, const moonep_plan_t &p, void
     b.topk = topk;
     b.p = p;
     b.cc = a.cc;
+    b.gp = a.gp;
     b.host_dst0 = a.host_dst0;
     const size_t smem2 = sizeof(int) * (size_t)assign_smem_ints(d.E, d.R, d.chunk_tokens * d.K);
     if (cudaFuncSetAttribute(assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2) !=

@@ -17,7 +17,7 @@ namespace moonep {
 
 constexpr int REDUCE_THREADS = 256;
 constexpr int REDUCE_UNROLL = 4;
-constexpr int REDUCE_MAX_LIST = 1024;
+constexpr int REDUCE_MAX_LIST = 2048;  // >= E + R - 1 >= prefetched replicas
 
 struct ReduceParams {
     float *reduce_buf;
@@ -50,11 +50,49 @@ __device__ __forceinline__ float vzero<float>() { return 0.f; }
 template <typename V>
 __global__ void __launch_bounds__(REDUCE_THREADS) reduce_kernel(ReduceParams a)
 {
-    __shared__ long long s_row[REDUCE_MAX_LIST];
-    __shared__ int s_n;
+    // Per block, once: for every expert with prefetched replicas, the list
+    // of its reduce_buf rows (r*B + b) in ascending host rank order.
+    __shared__ int s_e[MOONEP_MAX_E];
+    __shared__ int s_off[MOONEP_MAX_E + 1];
+    __shared__ int s_row[REDUCE_MAX_LIST];
+    __shared__ int s_wsum[32];
     const int status = __ldg(a.info + MOONEP_INFO_STATUS);
     if (status & MOONEP_ST_EXPERT_ID_RANGE) return;
     const int n_exp = min(max(__ldg(a.info + MOONEP_INFO_N_REP_EXPERTS), 0), a.E);
+    if (n_exp == 0) return;
+    const int tid = threadIdx.x;
+    for (int i = tid; i <= n_exp; i += blockDim.x) {
+        int c = 0, e = -1;
+        if (i < n_exp) {
+            e = __ldg(a.rep_home_list + i);
+            if (e >= 0 && e < a.E) {
+                const int home = e / a.L;
+                const int h0 = max(0, __ldg(a.host_ptr + e)), h1 = min(a.n_hosts, __ldg(a.host_ptr + e + 1));
+                for (int h = h0; h < h1; ++h) {
+                    const int r = __ldg(a.host_rank + h), b = __ldg(a.host_slot + h) - a.L;
+                    c += (r != home && r >= 0 && r < a.R && b >= 0 && b < a.B);
+                }
+            }
+        }
+        if (i < n_exp) s_e[i] = e;
+        s_off[i] = c;
+    }
+    __syncthreads();
+    block_exscan(s_off, n_exp + 1, s_wsum);
+    for (int i = tid; i < n_exp; i += blockDim.x) {
+        const int e = s_e[i];
+        if (e < 0 || e >= a.E) continue;
+        const int home = e / a.L;
+        int o = s_off[i];
+        const int h0 = max(0, __ldg(a.host_ptr + e)), h1 = min(a.n_hosts, __ldg(a.host_ptr + e + 1));
+        for (int h = h0; h < h1; ++h) {
+            const int r = __ldg(a.host_rank + h), b = __ldg(a.host_slot + h) - a.L;
+            if (r != home && r >= 0 && r < a.R && b >= 0 && b < a.B && o < REDUCE_MAX_LIST)
+                s_row[o++] = r * a.B + b;
+        }
+    }
+    __syncthreads();
+
     constexpr int W = sizeof(V) / sizeof(float);
     const long long PV = a.P / W;  // vectors per row
     const long long nchunks = (PV + a.chunk - 1) / a.chunk;
@@ -63,28 +101,15 @@ __global__ void __launch_bounds__(REDUCE_THREADS) reduce_kernel(ReduceParams a)
     V *hg = reinterpret_cast<V *>(a.home_grad);
 
     for (long long item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const int e = __ldg(a.rep_home_list + item / nchunks);
-        const long long ci = item % nchunks;
-        if (e < 0 || e >= a.E) continue;  // uniform across the block
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            int n = 0;
-            const int home = e / a.L;
-            const int h0 = max(0, __ldg(a.host_ptr + e));
-            const int h1 = min(a.n_hosts, __ldg(a.host_ptr + e + 1));
-            for (int h = h0; h < h1; ++h) {
-                const int r = __ldg(a.host_rank + h), b = __ldg(a.host_slot + h) - a.L;
-                if (r == home || r < 0 || r >= a.R || b < 0 || b >= a.B) continue;
-                if (n < REDUCE_MAX_LIST) s_row[n++] = (long long)r * a.B + b;
-            }
-            s_n = n;
-        }
-        __syncthreads();
-        const int n = s_n;
+        const int ei = (int)(item / nchunks);
+        const long long ci = item - (long long)ei * nchunks;
+        const int e = s_e[ei];
+        if (e < 0 || e >= a.E) continue;
+        const int r0 = s_off[ei], n = min(s_off[ei + 1], REDUCE_MAX_LIST) - r0;
         V *home_row = hg + (long long)e * PV;
         const long long v0 = ci * a.chunk;
         const long long v1 = min(PV, v0 + a.chunk);
-        for (long long v = v0 + threadIdx.x; v < v1; v += (long long)REDUCE_THREADS * REDUCE_UNROLL) {
+        for (long long v = v0 + tid; v < v1; v += (long long)REDUCE_THREADS * REDUCE_UNROLL) {
             V acc[REDUCE_UNROLL];
 #pragma unroll
             for (int u = 0; u < REDUCE_UNROLL; ++u) {
@@ -92,7 +117,7 @@ __global__ void __launch_bounds__(REDUCE_THREADS) reduce_kernel(ReduceParams a)
                 if (x < v1) acc[u] = home_row[x];
             }
             for (int m = 0; m < n; ++m) {
-                V *rrow = rb + s_row[m] * PV;
+                V *rrow = rb + (long long)s_row[r0 + m] * PV;
                 V r[REDUCE_UNROLL];
 #pragma unroll
                 for (int u = 0; u < REDUCE_UNROLL; ++u) {

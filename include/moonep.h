@@ -91,6 +91,9 @@ extern "C" {
 /* A buffer row taken from the plan was outside [0, R*S*K) (a corrupted or
  * mismatched plan); that row access was skipped. */
 #define MOONEP_ST_ROW_RANGE 8
+/* A bounded wait inside a kernel (an mbarrier for a bulk copy) ran out of
+ * iterations; the kernel stopped early and its output is incomplete. */
+#define MOONEP_ST_WAIT_TIMEOUT 16
 
 /* ---- plan->info[] fields (int32, device) ------------------------------ */
 #define MOONEP_INFO_STATUS 0

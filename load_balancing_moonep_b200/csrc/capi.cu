@@ -45,6 +45,8 @@ static int make_dims(const moonep_config *c, Dims *d)
     d->chunk_tokens = ct;
     d->nchunk = (d->tokens + ct - 1) / ct;
     d->ngroups = (d->nchunk + CHUNK_GROUP - 1) / CHUNK_GROUP;
+    d->ebits = 0;
+    while ((1 << d->ebits) < d->E) ++d->ebits;
     if (plan_smem_bytes_max(*d) > MAX_DYN_SMEM) return MOONEP_ERR_LIMIT;
     return MOONEP_OK;
 }

@@ -5,50 +5,59 @@
 // redundant experts") fixes what the plan must achieve -- every rank gets
 // exactly S*K token slots, by replicating a few experts online from the
 // router output -- and calls the planner near-optimal without giving it.
-// This file implements the water-filling plan described in moonep.h:
+// This file implements the water-filling plan described in moonep.h in two
+// launches, with no host synchronisation and no inter-CTA waiting:
 //
-//   hist_plan_kernel  one CTA per token chunk: shared-memory histogram of the
-//                     chunk (per-chunk counts kept for the assignment pass,
-//                     totals accumulated with global atomics).  The CTA that
-//                     finishes last (atomic ticket, no waiting) runs the whole
-//                     planner as one 1024-thread block: loads, largest-first
-//                     shedding, (value desc, index asc) orders by counting
-//                     rank, prefix sums, water-filling as a parallel merge of
-//                     the two prefix-sum partitions, slot tables and
-//                     rank-ordered host intervals.
+//   hist_plan_kernel  one CTA per token chunk builds the chunk's expert
+//                     histogram in shared memory (ballot-matched lanes add
+//                     once per distinct expert), stores it for the second
+//                     pass and adds it to per-group and total counts with
+//                     atomics (sums: order-free, so deterministic).  The CTA
+//                     that finishes last (atomic ticket) runs the planner:
+//                     loads, largest-first shedding, (value desc, index asc)
+//                     orders by counting rank, prefix sums, water-filling as a
+//                     parallel merge of the two prefix-sum partitions,
+//                     compact per-rank slot lists, rank-ordered host
+//                     intervals.  It writes compact results only.
 //   assign_kernel     one CTA per token chunk: the stable within-expert rank g
-//                     of every (t, k) pair from the chunk prefix of the
-//                     per-chunk counts, per-warp counters and warp match/popc,
-//                     then the host interval holding g gives the buffer row.
-//
-// Nothing waits on another CTA, so no launch can hang.
+//                     of every (t, k) pair from the counts of earlier groups
+//                     and chunks, per-warp counters and ballot matching; the
+//                     host interval holding g gives the buffer row.  The CTAs
+//                     also expand the compact slot lists into the padded
+//                     [R][E] tables.  Launched with programmatic dependent
+//                     launch: its input-only prologue overlaps the planner.
 #include "common.cuh"
 
 namespace moonep {
+
+constexpr int PLAN_THREADS = 512;
+constexpr int ASSIGN_THREADS = 512;
+constexpr int ASSIGN_WARPS = ASSIGN_THREADS / 32;
 
 struct PlanParams {
     Dims d;
     const int32_t *topk;
     moonep_plan_t p;
-    int *ticket;
-    int *status;
-    int *gs;
-    int *gp;
-    int *cc;
-    int *host_dst0;
+    int *hdr;        // ticket, status, parity
+    int *t_acc;      // [E]
+    int *gs;         // [2][ngroups][E]
+    int *cc;         // [nchunk][E]
+    int *host_dst0;  // [2E+R]
+    int *sc_base;    // [R+1]
+    int *sc_exp;     // [2E+R]
+    int *sc_cnt;     // [2E+R]
+    int *sc_off;     // [2E+R]
+    FastDiv fK, fS, fC;
 };
-
-constexpr int PLAN_THREADS = 1024;
-constexpr int ASSIGN_THREADS = 512;
-constexpr int ASSIGN_WARPS = ASSIGN_THREADS / 32;
 
 // ints of dynamic shared memory used by the planner block
 __host__ __device__ inline int plan_smem_ints(int E, int R)
 {
-    const int mx = E > R ? E : R;
-    return 3 * E /*T, shed, flag2*/ + 2 * R /*X, D*/ + (mx + 1) /*scr*/ + 2 * E + (E + 1) /*pe pv PS*/ +
-           2 * R + (R + 1) /*qr qv QS*/ + E + (E + 1) /*pilo segb*/ + 3 * R /*jlo nrr ridx*/ +
-           E /*pof*/ + (R + 1) /*rbase*/ + (2 * E + R) /*offc*/ + (E + 1) /*hcnt*/ + 32 + 16;
+    const int nh = 2 * E + R;
+    return 3 * E /*T shed keep*/ + 2 * R /*X D*/ + (E + R + 2) /*scr*/ + 2 * E /*pe pv*/ + 2 * R /*qr qv*/ +
+           (E + R + 4) /*A: PS | QS*/ + E /*pilo*/ + (E + R + 4) /*Bs: segments | per rank*/ + R /*jlo*/ +
+           2 * R /*nrr ridx*/ + E /*pof*/ + 4 * nh /*cexp ccnt coff cspare*/ + (E + 1) /*hcnt*/ +
+           3 * nh /*hr hs hq*/ + E /*flag*/ + 32 + 16;
 }
 
 __host__ __device__ inline int assign_smem_ints(int E, int R, int max_pairs)
@@ -56,97 +65,84 @@ __host__ __device__ inline int assign_smem_ints(int E, int R, int max_pairs)
     return E + ASSIGN_WARPS * E + 2 * max_pairs + (E + 1) + 2 * (2 * E + R) + 32;
 }
 
-// quota of the overlap of piece j with receiver i
 __device__ __forceinline__ int seg_quota(const int *PS, const int *QS, int j, int i)
 {
     return min(PS[j + 1], QS[i + 1]) - max(PS[j], QS[i]);
 }
 
-__device__ void write_empty_plan(const PlanParams &a, int status)
+__device__ __forceinline__ void pdl_launch_dependents()
 {
-    const Dims &d = a.d;
-    const int E = d.E, R = d.R, tid = threadIdx.x, nt = blockDim.x;
-    for (int i = tid; i < R * E; i += nt) {
-        a.p.slot_expert[i] = -1;
-        a.p.slot_count[i] = 0;
-    }
-    for (int i = tid; i < R * (E + 1); i += nt) a.p.slot_offset[i] = 0;
-    for (int i = tid; i < E + R; i += nt) {
-        a.p.rep_expert[i] = -1;
-        a.p.rep_rank[i] = -1;
-        a.p.rep_slot[i] = -1;
-        a.p.rep_quota[i] = 0;
-    }
-    for (int i = tid; i <= E; i += nt) a.p.host_ptr[i] = 0;
-    for (int i = tid; i < 2 * E + R; i += nt) {
-        a.p.host_rank[i] = -1;
-        a.p.host_slot[i] = -1;
-        a.p.host_start[i] = 0;
-        a.p.host_quota[i] = 0;
-    }
-    for (int i = tid; i < E; i += nt) a.p.rep_home_list[i] = -1;
-    for (int i = tid; i < MOONEP_INFO_LEN; i += nt) a.p.info[i] = (i == MOONEP_INFO_STATUS) ? status : 0;
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// The planner, run by the last CTA of hist_plan_kernel (blockDim = 1024).
-__device__ void plan_block(const PlanParams &a, int *sm)
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// ------------------------------------------------------------- planner CTA
+
+__device__ void plan_block(const PlanParams &a, int *sm, int parity)
 {
     const Dims &d = a.d;
     const int E = d.E, R = d.R, L = d.L, C = d.C, B = d.B;
     const int tid = threadIdx.x, nt = blockDim.x;
-    const int mx = E > R ? E : R;
+    const int nh = 2 * E + R;
 
     int *T = sm;
     int *shed = T + E;
-    int *flag2 = shed + E;
-    int *X = flag2 + E;
+    int *keep = shed + E;
+    int *X = keep + E;
     int *D = X + R;
-    int *scr = D + R;          // mx + 1
-    int *pe = scr + mx + 1;    // E  pieces: expert, sorted
-    int *pv = pe + E;          // E  pieces: shed, sorted
-    int *PS = pv + E;          // E + 1
-    int *qr = PS + E + 1;      // R  receivers: rank, sorted
-    int *qv = qr + R;          // R  receivers: deficit, sorted
-    int *QS = qv + R;          // R + 1
-    int *pilo = QS + R + 1;    // E  first receiver of piece j
-    int *segb = pilo + E;      // E + 1 first replica index of piece j
-    int *jlo = segb + E + 1;   // R  first piece of receiver i
-    int *nrr = jlo + R;        // R  replicas on rank r
-    int *ridx = nrr + R;       // R  receiver index of rank r, -1 if none
-    int *pof = ridx + R;       // E  piece index of expert e, -1 if none
-    int *rbase = pof + E;      // R + 1 compact base of rank r's used slots
-    int *offc = rbase + R + 1; // 2E + R slot offsets of used slots
-    int *hcnt = offc + 2 * E + R;  // E + 1
-    int *wsum = hcnt + E + 1;      // 32
-    int *misc = wsum + 32;         // 16: 0 status 1 n_rep 2 n_over 3 max_rep 4 nP 5 nN 6 n_rep_experts
+    int *scr = D + R;              // E + R + 2
+    int *pe = scr + E + R + 2;     // E   pieces: expert, sorted
+    int *pv = pe + E;              // E   pieces: shed, sorted
+    int *qr = pv + E;              // R   receivers: rank, sorted
+    int *qv = qr + R;              // R   receivers: deficit, sorted
+    int *A = qv + R;               // E + R + 4: PS (nP+1) then QS (nN+1)
+    int *pilo = A + E + R + 4;     // E   first receiver of piece j
+    int *Bs = pilo + E;            // E + R + 4: segments per piece (nP+1) | replicas per rank (R+1)
+    int *jlo = Bs + E + R + 4;     // R   first piece of receiver i
+    int *nrr = jlo + R;            // R   replicas on rank r
+    int *ridx = nrr + R;           // R   receiver index of rank r, -1 if none
+    int *pof = ridx + R;           // E   piece index of expert e, -1 if none
+    int *cexp = pof + E;           // nh  compact used slots: expert
+    int *ccnt = cexp + nh;         // nh  rows
+    int *coff = ccnt + nh;         // nh  slot offset
+    int *cspare = coff + nh;       // nh  temporary
+    int *hcnt = cspare + nh;       // E + 1
+    int *hr = hcnt + E + 1;        // nh  host rank
+    int *hs = hr + nh;             // nh  host slot
+    int *hq = hs + nh;             // nh  host quota
+    int *flag = hq + nh;           // E
+    int *wsum = flag + E;          // 32
+    int *misc = wsum + 32;         // 16: 0 status in, 2 n_over, 3 max replicas per rank
 
     for (int i = tid; i < 16; i += nt) misc[i] = 0;
-    __syncthreads();
-
-    // ---- totals from the histogram pass: exclusive prefix of the group
-    // counts for the assignment pass; leave the group counts zeroed
-    const int ng = d.ngroups;
+    // ---- totals; leave the accumulators zeroed for the next call
     for (int e = tid; e < E; e += nt) {
-        int run = 0;
-        for (int g = 0; g < ng; ++g) {
-            const int v = ld_cg(a.gs + (size_t)g * E + e);
-            a.gs[(size_t)g * E + e] = 0;
-            a.gp[(size_t)g * E + e] = run;
-            run += v;
-        }
-        T[e] = run;
-        a.p.expert_count[e] = run;
+        const int v = ld_cg(a.t_acc + e);
+        T[e] = v;
+        a.t_acc[e] = 0;
+        a.p.expert_count[e] = v;
     }
+    // the previous call's group buffer is no longer read: zero it
+    {
+        int *old = a.gs + (size_t)(parity ^ 1) * d.ngroups * E;
+        for (int i = tid; i < d.ngroups * E; i += nt) old[i] = 0;
+    }
+    __syncthreads();
     if (tid == 0) {
-        misc[0] = ld_cg(a.status);
-        *a.status = 0;
-        *a.ticket = 0;
+        misc[0] = ld_cg(a.hdr + WS_STATUS);
+        a.hdr[WS_STATUS] = 0;
+        a.hdr[WS_TICKET] = 0;
+        a.hdr[WS_PARITY] = parity ^ 1;  // the next call accumulates into the other buffer
     }
     __syncthreads();
     const int status_in = misc[0];
     if (status_in & MOONEP_ST_EXPERT_ID_RANGE) {
-        write_empty_plan(a, status_in);
-        return;
+        if (tid == 0) {
+            a.p.info[MOONEP_INFO_STATUS] = status_in;
+            for (int i = 1; i < MOONEP_INFO_LEN; ++i) a.p.info[i] = 0;
+        }
+        return;  // the assignment pass writes the empty tables
     }
 
     // ---- home loads, excess X and deficit D per rank
@@ -158,8 +154,8 @@ __device__ void plan_block(const PlanParams &a, int *sm)
     }
     __syncthreads();
 
-    // ---- largest-first shedding: expert e's share of its rank's excess is
-    // what remains after all larger (T desc, e asc) experts of the rank
+    // ---- largest-first shedding: expert e sheds what remains of its rank's
+    // excess after all larger (T desc, e asc) experts of the rank
     for (int e = tid; e < E; e += nt) {
         const int r = e / L, v = T[e];
         int s = 0;
@@ -173,63 +169,70 @@ __device__ void plan_block(const PlanParams &a, int *sm)
             s = rem > 0 ? min(v, rem) : 0;
         }
         shed[e] = s;
+        keep[e] = v - s;
+        scr[e] = s > 0;
+        pof[e] = -1;
     }
-    __syncthreads();
-
-    // ---- pieces, compacted then ordered by (shed desc, e asc)
-    for (int e = tid; e < E; e += nt) scr[e] = shed[e] > 0;
-    __syncthreads();
-    const int nP = block_exscan(scr, E, wsum);
-    int *tv = pilo, *ti = segb;  // temporaries
-    for (int e = tid; e < E; e += nt)
-        if (shed[e] > 0) {
-            tv[scr[e]] = shed[e];
-            ti[scr[e]] = e;
-        }
-    __syncthreads();
-    for (int i = tid; i < nP; i += nt) {
-        const int v = tv[i], id = ti[i];
-        int pos = 0;
-        for (int j = 0; j < nP; ++j) pos += (tv[j] > v) || (tv[j] == v && ti[j] < id);
-        pe[pos] = id;
-        pv[pos] = v;
-    }
-    __syncthreads();
-
-    // ---- receivers, compacted then ordered by (deficit desc, r asc)
-    for (int r = tid; r < R; r += nt) scr[r] = D[r] > 0;
-    __syncthreads();
-    const int nN = block_exscan(scr, R, wsum);
-    int *uv = jlo, *ui = nrr;  // temporaries
-    for (int r = tid; r < R; r += nt)
-        if (D[r] > 0) {
-            uv[scr[r]] = D[r];
-            ui[scr[r]] = r;
-        }
-    __syncthreads();
-    for (int i = tid; i < nN; i += nt) {
-        const int v = uv[i], id = ui[i];
-        int pos = 0;
-        for (int j = 0; j < nN; ++j) pos += (uv[j] > v) || (uv[j] == v && ui[j] < id);
-        qr[pos] = id;
-        qv[pos] = v;
-    }
-    __syncthreads();
-
-    // ---- prefix sums PS over pieces, QS over receivers
-    for (int j = tid; j <= nP; j += nt) PS[j] = j < nP ? pv[j] : 0;
-    for (int i = tid; i <= nN; i += nt) QS[i] = i < nN ? qv[i] : 0;
-    for (int e = tid; e < E; e += nt) pof[e] = -1;
     for (int r = tid; r < R; r += nt) {
+        scr[E + r] = D[r] > 0;
         nrr[r] = 0;
         ridx[r] = -1;
     }
     __syncthreads();
-    block_exscan(PS, nP + 1, wsum);
-    block_exscan(QS, nN + 1, wsum);
 
-    // ---- water-filling: piece j overlaps receivers pilo[j] .. last; receiver
-    // i overlaps pieces jlo[i] .. last.  Replicas are numbered in (j, i) order.
+    // ---- compact pieces and receivers with one scan over [E experts | R ranks]
+    const int nPN = block_exscan(scr, E + R, wsum);
+    const int nP = scr[E];
+    const int nN = nPN - nP;
+    for (int e = tid; e < E; e += nt)
+        if (shed[e] > 0) {
+            hr[scr[e]] = shed[e];
+            hs[scr[e]] = e;
+        }
+    for (int r = tid; r < R; r += nt)
+        if (D[r] > 0) {
+            hq[scr[E + r] - nP] = D[r];
+            cspare[scr[E + r] - nP] = r;
+        }
+    __syncthreads();
+    // counting-rank sorts: pieces by (shed desc, e asc), receivers by (D desc, r asc)
+    for (int x = tid; x < nP + nN; x += nt) {
+        if (x < nP) {
+            const int v = hr[x], id = hs[x];
+            int pos = 0;
+            for (int j = 0; j < nP; ++j) pos += (hr[j] > v) || (hr[j] == v && hs[j] < id);
+            pe[pos] = id;
+            pv[pos] = v;
+        } else {
+            const int i0 = x - nP, v = hq[i0], id = cspare[i0];
+            int pos = 0;
+            for (int j = 0; j < nN; ++j) pos += (hq[j] > v) || (hq[j] == v && cspare[j] < id);
+            qr[pos] = id;
+            qv[pos] = v;
+        }
+    }
+    __syncthreads();
+
+    // ---- prefix sums: A = [pv..., 0, qv..., 0] scanned gives PS and QS
+    for (int x = tid; x < nP + nN + 2; x += nt) {
+        int v = 0;
+        if (x < nP) v = pv[x];
+        else if (x > nP && x < nP + 1 + nN) v = qv[x - nP - 1];
+        A[x] = v;
+    }
+    __syncthreads();
+    block_exscan(A, nP + nN + 2, wsum);
+    const int *PS = A;            // PS[0..nP]
+    int *QS = A + nP + 1;         // QS[0..nN] after removing the pieces' total
+    const int qbase = QS[0];
+    __syncthreads();
+    for (int x = tid; x <= nN; x += nt) QS[x] -= qbase;
+    __syncthreads();
+
+    // ---- water-filling: piece j meets receivers pilo[j].. ; receiver i meets
+    // pieces jlo[i].. ; replicas are numbered in (j, i) order
+    int *segb = Bs;           // nP + 1
+    int *rpre = Bs + nP + 1;  // R + 1
     for (int j = tid; j < nP; j += nt) {
         const int ilo = last_le(QS, nN, PS[j]);
         const int ihi = last_le(QS, nN, PS[j + 1] - 1);
@@ -237,7 +240,6 @@ __device__ void plan_block(const PlanParams &a, int *sm)
         segb[j] = ihi - ilo + 1;
         pof[pe[j]] = j;
     }
-    if (tid == 0) segb[nP] = 0;
     for (int i = tid; i < nN; i += nt) {
         const int jl = last_le(PS, nP, QS[i]);
         const int jh = last_le(PS, nP, QS[i + 1] - 1);
@@ -245,66 +247,57 @@ __device__ void plan_block(const PlanParams &a, int *sm)
         nrr[qr[i]] = jh - jl + 1;
         ridx[qr[i]] = i;
     }
+    if (tid == 0) segb[nP] = 0;
     __syncthreads();
-    const int n_rep = block_exscan(segb, nP + 1, wsum);
+    for (int r = tid; r <= R; r += nt) rpre[r] = r < R ? nrr[r] : 0;
+    __syncthreads();
+    // one scan over [segments per piece | replicas per rank]
+    block_exscan(Bs, nP + 1 + R + 1, wsum);
+    const int n_rep = Bs[nP];
+    __syncthreads();
+    for (int x = tid; x <= R; x += nt) rpre[x] -= n_rep;
+    __syncthreads();
 
-    // ---- replica list
-    for (int q = tid; q < E + R; q += nt) {
-        if (q < n_rep) {
-            const int j = last_le(segb, nP, q);
-            const int i = pilo[j] + (q - segb[j]);
-            const int ord = j - jlo[i];
-            a.p.rep_expert[q] = pe[j];
-            a.p.rep_rank[q] = qr[i];
-            a.p.rep_slot[q] = L + ord;
-            a.p.rep_quota[q] = seg_quota(PS, QS, j, i);
-            if (ord >= B) atomicAdd(&misc[2], 1);
-        } else {
-            a.p.rep_expert[q] = -1;
-            a.p.rep_rank[q] = -1;
-            a.p.rep_slot[q] = -1;
-            a.p.rep_quota[q] = 0;
-        }
+    // ---- replica list (creation order) and the compact used-slot lists:
+    // rank r's used slots sit at r*L + rpre[r] .. (home slots, then replicas)
+    for (int q = tid; q < n_rep; q += nt) {
+        const int j = last_le(segb, nP, q);
+        const int i = pilo[j] + (q - segb[j]);
+        const int ord = j - jlo[i];
+        const int r = qr[i];
+        const int quota = seg_quota(PS, QS, j, i);
+        a.p.rep_expert[q] = pe[j];
+        a.p.rep_rank[q] = r;
+        a.p.rep_slot[q] = L + ord;
+        a.p.rep_quota[q] = quota;
+        const int cs = r * L + rpre[r] + L + ord;
+        cexp[cs] = pe[j];
+        ccnt[cs] = quota;
+        if (ord >= B) atomicAdd(&misc[2], 1);
     }
-
-    // ---- slot tables: compact per-rank offsets of the used slots first
-    for (int r = tid; r <= R; r += nt) rbase[r] = r < R ? L + nrr[r] : 0;
+    for (int e = tid; e < E; e += nt) {
+        const int r = e / L;
+        const int cs = r * L + rpre[r] + (e - r * L);
+        cexp[cs] = e;
+        ccnt[cs] = keep[e];
+    }
     __syncthreads();
-    block_exscan(rbase, R + 1, wsum);
     for (int r = tid; r < R; r += nt) {
-        const int used = L + nrr[r];
+        const int b0 = r * L + rpre[r], used = L + nrr[r];
         int off = 0;
         for (int s = 0; s < used; ++s) {
-            offc[rbase[r] + s] = off;
-            int cnt;
-            if (s < L) {
-                cnt = T[r * L + s] - shed[r * L + s];
-            } else {
-                const int i = ridx[r];
-                cnt = seg_quota(PS, QS, jlo[i] + (s - L), i);
-            }
-            off += cnt;
+            coff[b0 + s] = off;
+            off += ccnt[b0 + s];
         }
+        a.sc_base[r] = b0;
         atomicMax(&misc[3], nrr[r]);
     }
+    if (tid == 0) a.sc_base[R] = E + n_rep;
     __syncthreads();
-    for (int idx = tid; idx < R * E; idx += nt) {
-        const int r = idx / E, s = idx - r * E, used = L + nrr[r];
-        int ex = -1, cnt = 0;
-        if (s < L) {
-            ex = r * L + s;
-            cnt = T[ex] - shed[ex];
-        } else if (s < used) {
-            const int i = ridx[r], j = jlo[i] + (s - L);
-            ex = pe[j];
-            cnt = seg_quota(PS, QS, j, i);
-        }
-        a.p.slot_expert[idx] = ex;
-        a.p.slot_count[idx] = cnt;
-    }
-    for (int idx = tid; idx < R * (E + 1); idx += nt) {
-        const int r = idx / (E + 1), s = idx - r * (E + 1), used = L + nrr[r];
-        a.p.slot_offset[idx] = s < used ? offc[rbase[r] + s] : C;
+    for (int x = tid; x < E + n_rep; x += nt) {
+        a.sc_exp[x] = cexp[x];
+        a.sc_cnt[x] = ccnt[x];
+        a.sc_off[x] = coff[x];
     }
 
     // ---- host intervals: home + replicas of e, ascending rank
@@ -319,20 +312,13 @@ __device__ void plan_block(const PlanParams &a, int *sm)
     __syncthreads();
     block_exscan(hcnt, E + 1, wsum);
     for (int e = tid; e <= E; e += nt) a.p.host_ptr[e] = hcnt[e];
-    for (int x = tid; x < 2 * E + R; x += nt) {
-        if (x >= E + n_rep) {
-            a.p.host_rank[x] = -1;
-            a.p.host_slot[x] = -1;
-            a.p.host_start[x] = 0;
-            a.p.host_quota[x] = 0;
-            continue;
-        }
+    for (int x = tid; x < E + n_rep; x += nt) {
         int e, r0, slot, quota, j, pos;
         if (x < E) {
             e = x;
             r0 = e / L;
             slot = e - r0 * L;
-            quota = T[e] - shed[e];
+            quota = keep[e];
             j = pof[e];
             pos = 0;
         } else {
@@ -350,18 +336,21 @@ __device__ void plan_block(const PlanParams &a, int *sm)
             for (int s = 0; s < ns; ++s) pos += qr[pilo[j] + s] < r0;
         }
         const int h = hcnt[e] + pos;
-        a.p.host_rank[h] = r0;
-        a.p.host_slot[h] = slot;
-        a.p.host_quota[h] = quota;
+        hr[h] = r0;
+        hs[h] = slot;
+        hq[h] = quota;
     }
     __syncthreads();
     for (int e = tid; e < E; e += nt) {
         int st = 0;
         for (int h = hcnt[e]; h < hcnt[e + 1]; ++h) {
-            const int r = a.p.host_rank[h], slot = a.p.host_slot[h];
+            const int r = hr[h], slot = hs[h];
+            a.p.host_rank[h] = r;
+            a.p.host_slot[h] = slot;
+            a.p.host_quota[h] = hq[h];
             a.p.host_start[h] = st;
-            a.host_dst0[h] = r * C + offc[rbase[r] + slot] - st;
-            st += a.p.host_quota[h];
+            a.host_dst0[h] = r * C + coff[r * L + rpre[r] + slot] - st;
+            st += hq[h];
         }
     }
 
@@ -374,13 +363,13 @@ __device__ void plan_block(const PlanParams &a, int *sm)
             for (int s = 0; s < ns; ++s)
                 if (j - jlo[pilo[j] + s] < B) f = 1;
         }
-        flag2[e] = f;
+        flag[e] = f;
         scr[e] = f;
     }
     __syncthreads();
     const int n_rep_experts = block_exscan(scr, E, wsum);
     for (int e = tid; e < E; e += nt) {
-        if (flag2[e]) a.p.rep_home_list[scr[e]] = e;
+        if (flag[e]) a.p.rep_home_list[scr[e]] = e;
         if (e >= n_rep_experts) a.p.rep_home_list[e] = -1;
     }
 
@@ -402,17 +391,22 @@ __device__ void plan_block(const PlanParams &a, int *sm)
     }
 }
 
-__global__ void __launch_bounds__(PLAN_THREADS, 1) hist_plan_kernel(PlanParams a)
+__global__ void __launch_bounds__(PLAN_THREADS) hist_plan_kernel(PlanParams a)
 {
     extern __shared__ int sm[];
-    __shared__ int s_last;
+    __shared__ int s_last, s_parity;
     const Dims &d = a.d;
     const int E = d.E, K = d.K, tid = threadIdx.x, nt = blockDim.x;
     const int lane = tid & 31, warp = tid >> 5;
+    // the assignment kernel may be scheduled now; it waits for this whole
+    // grid before it reads anything this grid writes
+    pdl_launch_dependents();
 
     int *hist = sm;
     for (int e = tid; e < E; e += nt) hist[e] = 0;
+    if (tid == 0) s_parity = ld_cg(a.hdr + WS_PARITY) & 1;
     __syncthreads();
+    const int parity = s_parity;
 
     const int chunk = blockIdx.x;
     const int t0 = chunk * d.chunk_tokens;
@@ -425,40 +419,36 @@ __global__ void __launch_bounds__(PLAN_THREADS, 1) hist_plan_kernel(PlanParams a
         const int e = valid ? __ldg(a.topk + p) : -1;
         const bool ok = valid && e >= 0 && e < E;
         if (valid && !ok) bad = 1;
-        const unsigned peers = __match_any_sync(FULL_MASK, ok ? e : E + lane);
+        const unsigned peers = peers_of(ok ? e : 0, ok, d.ebits);
         if (ok && lane == __ffs(peers) - 1) atomicAdd(&hist[e], __popc(peers));
     }
     bad = __syncthreads_or(bad);
-    const int grp = chunk / CHUNK_GROUP;
+    int *gsb = a.gs + ((size_t)parity * d.ngroups + chunk / CHUNK_GROUP) * E;
     for (int e = tid; e < E; e += nt) {
         const int c = hist[e];
         a.cc[(size_t)chunk * E + e] = c;
-        if (c) atomicAdd(a.gs + (size_t)grp * E + e, c);  // commutative: order-free
+        if (c) {
+            atomicAdd(a.t_acc + e, c);  // sums: order-free
+            atomicAdd(gsb + e, c);
+        }
     }
-    if (bad && tid == 0) atomicOr(a.status, MOONEP_ST_EXPERT_ID_RANGE);
+    if (bad && tid == 0) atomicOr(a.hdr + WS_STATUS, MOONEP_ST_EXPERT_ID_RANGE);
     __threadfence();
     __syncthreads();
-    if (tid == 0) s_last = (atomicAdd(a.ticket, 1) == (int)gridDim.x - 1);
+    if (tid == 0) s_last = (atomicAdd(a.hdr + WS_TICKET, 1) == (int)gridDim.x - 1);
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    plan_block(a, sm);
+    plan_block(a, sm, parity);
 }
 
-struct AssignParams {
-    Dims d;
-    const int32_t *topk;
-    moonep_plan_t p;
-    const int *cc;
-    const int *gp;
-    const int *host_dst0;
-};
+// ---------------------------------------------------------- assignment
 
-__global__ void __launch_bounds__(ASSIGN_THREADS) assign_kernel(AssignParams a)
+__global__ void __launch_bounds__(ASSIGN_THREADS) assign_kernel(PlanParams a)
 {
     extern __shared__ int sm[];
     const Dims &d = a.d;
-    const int E = d.E, K = d.K, R = d.R, C = d.C, S = d.S;
+    const int E = d.E, K = d.K, R = d.R, C = d.C;
     const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5;
     const int chunk = blockIdx.x;
     const int t0 = chunk * d.chunk_tokens;
@@ -466,15 +456,6 @@ __global__ void __launch_bounds__(ASSIGN_THREADS) assign_kernel(AssignParams a)
     const int p0 = t0 * K, n = (t1 - t0) * K;
     const int max_pairs = d.chunk_tokens * K;
     const int nh = 2 * E + R;
-
-    const int status = a.p.info[MOONEP_INFO_STATUS];
-    if (status & MOONEP_ST_EXPERT_ID_RANGE) {
-        for (int i = tid; i < n; i += nt) {
-            a.p.dst_pos[p0 + i] = -1;
-            a.p.row_src[p0 + i] = -1;
-        }
-        return;
-    }
 
     int *base = sm;                        // E
     int *cnt = base + E;                   // ASSIGN_WARPS * E
@@ -485,42 +466,112 @@ __global__ void __launch_bounds__(ASSIGN_THREADS) assign_kernel(AssignParams a)
     int *hdst = hstart + nh;               // nh
     int *red = hdst + nh;                  // 32
 
-    for (int e = tid; e <= E; e += nt) hptr[e] = a.p.host_ptr[e];
-    for (int h = tid; h < nh; h += nt) {
-        hstart[h] = a.p.host_start[h];
-        hdst[h] = a.host_dst0[h];
+    // prologue on inputs only, overlapping the histogram/planner grid
+    for (int i = tid; i < ASSIGN_WARPS * E; i += nt) cnt[i] = 0;
+    for (int i = tid; i < n; i += nt) ids[i] = __ldg(a.topk + p0 + i);
+    pdl_wait();  // the histogram/planner grid has completed; its writes are visible
+
+    const int status = ld_cg(a.p.info + MOONEP_INFO_STATUS);
+    const bool empty = (status & MOONEP_ST_EXPERT_ID_RANGE) != 0;
+    const int n_rep = empty ? 0 : ld_cg(a.p.info + MOONEP_INFO_N_REP);
+
+    // ---- padded tables from the compact slot lists, spread over the CTAs
+    {
+        const long long g = (long long)gridDim.x * nt, x0 = (long long)blockIdx.x * nt + tid;
+        for (long long x = x0; x < (long long)R * E; x += g) {
+            const int r = (int)(x / E), s = (int)(x - (long long)r * E);
+            int ex = -1, ct = 0;
+            if (!empty) {
+                const int b0 = ld_cg(a.sc_base + r), b1 = ld_cg(a.sc_base + r + 1);
+                if (s < b1 - b0) {
+                    ex = ld_cg(a.sc_exp + b0 + s);
+                    ct = ld_cg(a.sc_cnt + b0 + s);
+                }
+            }
+            a.p.slot_expert[x] = ex;
+            a.p.slot_count[x] = ct;
+        }
+        for (long long x = x0; x < (long long)R * (E + 1); x += g) {
+            const int r = (int)(x / (E + 1)), s = (int)(x - (long long)r * (E + 1));
+            int v = 0;
+            if (!empty) {
+                const int b0 = ld_cg(a.sc_base + r), b1 = ld_cg(a.sc_base + r + 1);
+                v = s < b1 - b0 ? ld_cg(a.sc_off + b0 + s) : C;
+            }
+            a.p.slot_offset[x] = v;
+        }
+        for (long long x = x0; x < E + R; x += g)
+            if (x >= n_rep) {
+                a.p.rep_expert[x] = -1;
+                a.p.rep_rank[x] = -1;
+                a.p.rep_slot[x] = -1;
+                a.p.rep_quota[x] = 0;
+            }
+        const int hused = empty ? 0 : E + n_rep;
+        for (long long x = x0; x < nh; x += g)
+            if (x >= hused) {
+                a.p.host_rank[x] = -1;
+                a.p.host_slot[x] = -1;
+                a.p.host_start[x] = 0;
+                a.p.host_quota[x] = 0;
+            }
+        if (empty) {
+            for (long long x = x0; x <= E; x += g) a.p.host_ptr[x] = 0;
+            for (long long x = x0; x < E; x += g) a.p.rep_home_list[x] = -1;
+        }
     }
-    // pairs of each expert in earlier chunks: group prefix + earlier chunks
-    // of this chunk's group (at most CHUNK_GROUP - 1 independent loads)
+
+    if (empty) {
+        for (int i = tid; i < n; i += nt) {
+            a.p.dst_pos[p0 + i] = -1;
+            a.p.row_src[p0 + i] = -1;
+        }
+        return;
+    }
+
+    for (int e = tid; e <= E; e += nt) hptr[e] = ld_cg(a.p.host_ptr + e);
+    for (int h = tid; h < E + n_rep; h += nt) {
+        hstart[h] = ld_cg(a.p.host_start + h);
+        hdst[h] = ld_cg(a.host_dst0 + h);
+    }
+    // pairs of each expert in earlier chunks: earlier groups + earlier chunks
+    // of this chunk's group (independent loads)
     {
         const int grp = chunk / CHUNK_GROUP, c0 = grp * CHUNK_GROUP;
+        const int parity = ld_cg(a.hdr + WS_PARITY) ^ 1;  // the buffer this call filled
+        const int *gsb = a.gs + (size_t)parity * d.ngroups * E;
         for (int e = tid; e < E; e += nt) {
-            int s = __ldg(a.gp + (size_t)grp * E + e);
+            int s = 0;
+            for (int g0 = 0; g0 < grp; g0 += 8) {
+                int v[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[j] = (g0 + j < grp) ? ld_cg(gsb + (size_t)(g0 + j) * E + e) : 0;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) s += v[j];
+            }
             int v[CHUNK_GROUP - 1];
 #pragma unroll
             for (int j = 0; j < CHUNK_GROUP - 1; ++j)
-                v[j] = (c0 + j < chunk) ? __ldg(a.cc + (size_t)(c0 + j) * E + e) : 0;
+                v[j] = (c0 + j < chunk) ? ld_cg(a.cc + (size_t)(c0 + j) * E + e) : 0;
 #pragma unroll
             for (int j = 0; j < CHUNK_GROUP - 1; ++j) s += v[j];
             base[e] = s;
         }
     }
-    for (int i = tid; i < ASSIGN_WARPS * E; i += nt) cnt[i] = 0;
-    for (int i = tid; i < n; i += nt) ids[i] = __ldg(a.topk + p0 + i);
     __syncthreads();
 
     // pass 1: rank of each pair among earlier pairs of its expert inside the
-    // warp's contiguous sub-range
+    // warp's contiguous sub-range (ballot-matched lanes)
     const int per = (n + ASSIGN_WARPS - 1) / ASSIGN_WARPS;
+    const int wbeg = min(warp * per, n), wend = min(wbeg + per, n);
     {
-        const int beg = min(warp * per, n), end = min(beg + per, n);
         int *wc = cnt + warp * E;
-        for (int b = beg; b < end; b += 32) {
+        for (int b = wbeg; b < wend; b += 32) {
             const int i = b + lane;
-            const bool valid = i < end;
-            const int e = valid ? ids[i] : -1;
+            const bool valid = i < wend;
+            const int e = valid ? ids[i] : 0;
             const bool ok = valid && e >= 0 && e < E;
-            const unsigned peers = __match_any_sync(FULL_MASK, ok ? e : E + lane);
+            const unsigned peers = peers_of(ok ? e : 0, ok, d.ebits);
             int r0 = 0;
             if (ok) {
                 r0 = wc[e];
@@ -543,26 +594,28 @@ __global__ void __launch_bounds__(ASSIGN_THREADS) assign_kernel(AssignParams a)
     }
     __syncthreads();
 
-    // pass 2: host interval holding g gives the buffer row
+    // pass 2: the host interval holding g gives the buffer row
     int remote = 0;
-    for (int i = tid; i < n; i += nt) {
-        const int e = ids[i];
-        if (e < 0 || e >= E) continue;
-        const int w = i / per;
-        const int g = cnt[w * E + e] + lr[i];
-        int h = hptr[e];
-        const int hend = hptr[e + 1];
-        while (h + 1 < hend && hstart[h + 1] <= g) ++h;
-        const int dst = hdst[h] + g;
-        const int p = p0 + i;
-        if (dst < 0 || dst >= R * C) {  // cannot happen for a consistent plan
-            atomicOr(a.p.info + MOONEP_INFO_STATUS, MOONEP_ST_ROW_RANGE);
-            a.p.dst_pos[p] = -1;
-            continue;
+    {
+        const int *wc = cnt + warp * E;
+        for (int i = wbeg + lane; i < wend; i += 32) {
+            const int e = ids[i];
+            if (e < 0 || e >= E) continue;
+            const int g = wc[e] + lr[i];
+            int h = hptr[e];
+            const int hend = hptr[e + 1];
+            while (h + 1 < hend && hstart[h + 1] <= g) ++h;
+            const int dst = hdst[h] + g;
+            const int p = p0 + i;
+            if (dst < 0 || dst >= R * C) {  // cannot happen for a consistent plan
+                atomicOr(a.p.info + MOONEP_INFO_STATUS, MOONEP_ST_ROW_RANGE);
+                a.p.dst_pos[p] = -1;
+                continue;
+            }
+            a.p.dst_pos[p] = dst;
+            a.p.row_src[dst] = p;
+            remote += fdiv((uint32_t)dst, a.fC) != fdiv(fdiv((uint32_t)p, a.fK), a.fS);
         }
-        a.p.dst_pos[p] = dst;
-        a.p.row_src[dst] = p;
-        remote += (dst / C) != ((p / K) / S);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) remote += __shfl_xor_sync(FULL_MASK, remote, o);
@@ -577,6 +630,11 @@ __global__ void __launch_bounds__(ASSIGN_THREADS) assign_kernel(AssignParams a)
 
 // ---------------------------------------------------------------- launch
 
+static bool set_smem(const void *fn, size_t bytes)
+{
+    return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess;
+}
+
 int launch_plan(const Dims &d, const int32_t *topk, const moonep_plan_t &p, void *ws, cudaStream_t st)
 {
     const WsLayout wl = ws_layout(d);
@@ -585,33 +643,37 @@ int launch_plan(const Dims &d, const int32_t *topk, const moonep_plan_t &p, void
     a.d = d;
     a.topk = topk;
     a.p = p;
-    a.ticket = reinterpret_cast<int *>(w + wl.ticket);
-    a.status = reinterpret_cast<int *>(w + wl.status);
+    a.hdr = reinterpret_cast<int *>(w + wl.hdr);
+    a.t_acc = reinterpret_cast<int *>(w + wl.t_acc);
     a.gs = reinterpret_cast<int *>(w + wl.gs);
-    a.gp = reinterpret_cast<int *>(w + wl.gp);
     a.cc = reinterpret_cast<int *>(w + wl.cc);
     a.host_dst0 = reinterpret_cast<int *>(w + wl.host_dst0);
+    a.sc_base = reinterpret_cast<int *>(w + wl.sc_base);
+    a.sc_exp = reinterpret_cast<int *>(w + wl.sc_exp);
+    a.sc_cnt = reinterpret_cast<int *>(w + wl.sc_cnt);
+    a.sc_off = reinterpret_cast<int *>(w + wl.sc_off);
+    a.fK = make_fastdiv((uint32_t)d.K);
+    a.fS = make_fastdiv((uint32_t)d.S);
+    a.fC = make_fastdiv((uint32_t)d.C);
 
     const size_t smem1 = sizeof(int) * (size_t)plan_smem_ints(d.E, d.R);
-    if (cudaFuncSetAttribute(hist_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1) !=
-        cudaSuccess)
-        return MOONEP_ERR_CUDA;
+    if (!set_smem((const void *)hist_plan_kernel, smem1)) return MOONEP_ERR_CUDA;
     hist_plan_kernel<<<d.nchunk, PLAN_THREADS, smem1, st>>>(a);
     if (cudaGetLastError() != cudaSuccess) return MOONEP_ERR_CUDA;
 
-    AssignParams b;
-    b.d = d;
-    b.topk = topk;
-    b.p = p;
-    b.cc = a.cc;
-    b.gp = a.gp;
-    b.host_dst0 = a.host_dst0;
     const size_t smem2 = sizeof(int) * (size_t)assign_smem_ints(d.E, d.R, d.chunk_tokens * d.K);
-    if (cudaFuncSetAttribute(assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2) !=
-        cudaSuccess)
-        return MOONEP_ERR_CUDA;
-    assign_kernel<<<d.nchunk, ASSIGN_THREADS, smem2, st>>>(b);
-    if (cudaGetLastError() != cudaSuccess) return MOONEP_ERR_CUDA;
+    if (!set_smem((const void *)assign_kernel, smem2)) return MOONEP_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(d.nchunk);
+    cfg.blockDim = dim3(ASSIGN_THREADS);
+    cfg.dynamicSmemBytes = smem2;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, assign_kernel, a) != cudaSuccess) return MOONEP_ERR_CUDA;
     return MOONEP_OK;
 }
 

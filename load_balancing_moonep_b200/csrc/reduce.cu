@@ -17,6 +17,7 @@ namespace moonep {
 
 constexpr int REDUCE_THREADS = 256;
 constexpr int REDUCE_UNROLL = 4;
+constexpr int REDUCE_GROUP = 4;
 constexpr int REDUCE_MAX_LIST = 2048;  // >= E + R - 1 >= prefetched replicas
 
 struct ReduceParams {
@@ -116,22 +117,30 @@ __global__ void __launch_bounds__(REDUCE_THREADS) reduce_kernel(ReduceParams a)
                 const long long x = v + (long long)u * REDUCE_THREADS;
                 if (x < v1) acc[u] = home_row[x];
             }
-            for (int m = 0; m < n; ++m) {
-                V *rrow = rb + (long long)s_row[r0 + m] * PV;
-                V r[REDUCE_UNROLL];
+            // replicas in groups of REDUCE_GROUP: every load of a group is in
+            // flight before the adds, which keep ascending host rank order
+            for (int m0 = 0; m0 < n; m0 += REDUCE_GROUP) {
+                V r[REDUCE_GROUP][REDUCE_UNROLL];
+                V *rrow[REDUCE_GROUP];
 #pragma unroll
-                for (int u = 0; u < REDUCE_UNROLL; ++u) {
-                    const long long x = v + (long long)u * REDUCE_THREADS;
-                    if (x < v1) r[u] = rrow[x];
-                }
+                for (int m = 0; m < REDUCE_GROUP; ++m) {
+                    rrow[m] = rb + (long long)s_row[r0 + min(m0 + m, n - 1)] * PV;
 #pragma unroll
-                for (int u = 0; u < REDUCE_UNROLL; ++u) {
-                    const long long x = v + (long long)u * REDUCE_THREADS;
-                    if (x < v1) {
-                        acc[u] = vadd(acc[u], r[u]);
-                        rrow[x] = vzero<V>();
+                    for (int u = 0; u < REDUCE_UNROLL; ++u) {
+                        const long long x = v + (long long)u * REDUCE_THREADS;
+                        if (m0 + m < n && x < v1) r[m][u] = rrow[m][x];
                     }
                 }
+#pragma unroll
+                for (int m = 0; m < REDUCE_GROUP; ++m)
+#pragma unroll
+                    for (int u = 0; u < REDUCE_UNROLL; ++u) {
+                        const long long x = v + (long long)u * REDUCE_THREADS;
+                        if (m0 + m < n && x < v1) {
+                            acc[u] = vadd(acc[u], r[m][u]);
+                            rrow[m][x] = vzero<V>();
+                        }
+                    }
             }
 #pragma unroll
             for (int u = 0; u < REDUCE_UNROLL; ++u) {

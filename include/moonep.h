@@ -76,6 +76,7 @@ extern "C" {
 #define MOONEP_ERR_CUDA 5           /* a kernel launch failed */
 #define MOONEP_ERR_LIMIT 7          /* E > MOONEP_MAX_E */
 #define MOONEP_ERR_ALIGN 8          /* H % 8 != 0 or a data pointer not 16-byte aligned */
+#define MOONEP_ERR_NOALLOC_SIZE 9   /* moonep_plan_noalloc: workspace above MOONEP_NOALLOC_WORKSPACE_BYTES */
 
 #define MOONEP_MAX_E 1024
 
@@ -207,6 +208,34 @@ MOONEP_API int moonep_combine_backward(const moonep_config *cfg, const moonep_pl
  * expert gradient.  Overflow replicas have no rows and are skipped. */
 MOONEP_API int moonep_reduce_replica_grads(const moonep_config *cfg, const moonep_plan_t *plan,
                                 float *reduce_buf, float *home_grad, int64_t P, void *stream);
+
+/* Size of the fixed device array behind moonep_plan_noalloc (4 MiB).  The
+ * large training shape (R=32, E=384, K=8, S=4096) needs about 0.5 MiB. */
+#define MOONEP_NOALLOC_WORKSPACE_BYTES (4u << 20)
+
+/* moonep_plan without a caller-supplied workspace -- the pages have no
+ * counterpart; this is a convenience of this library.  It is for callers
+ * that cannot allocate device memory themselves: code running inside a
+ * runtime or framework that owns every device allocation (a preallocated
+ * pool, a server that reserves all memory at start-up), or code that must
+ * not call cudaMalloc on its hot path because it can synchronise the device.
+ * The planner's scratch space is then a file-scope device array of
+ * MOONEP_NOALLOC_WORKSPACE_BYTES that every GPU loading this library holds
+ * until the process exits; this call allocates nothing.
+ *  - Same inputs, outputs and results as moonep_plan (plan laid out by
+ *    moonep_plan_layout); configurations whose workspace (moonep_plan_sizes)
+ *    exceeds the array are rejected with MOONEP_ERR_NOALLOC_SIZE before any
+ *    launch.
+ *  - The first call on a device looks up the array's device address with
+ *    cudaGetSymbolAddress (once per device, the device current); make that
+ *    first call before any stream capture.
+ *  - Each call first clears the part of the array it uses (an async memset
+ *    on `stream`), because the array keeps the previous call's contents.
+ *  - All calls on a device share the one array: calls that can overlap on
+ *    the GPU (different streams without ordering) race and give wrong plans.
+ */
+MOONEP_API int moonep_plan_noalloc(const moonep_config *cfg, const int32_t *topk_idx,
+                                   const moonep_plan_t *plan, void *stream);
 
 /* Human-readable text for a MOONEP_* return code. */
 MOONEP_API const char *moonep_error_string(int code);

@@ -100,6 +100,8 @@ const char *moonep_error_string(int code)
     case MOONEP_ERR_CUDA: return "CUDA launch failed";
     case MOONEP_ERR_LIMIT: return "size beyond a library limit (E > 1024, shared memory, or K > 16 in combine_backward)";
     case MOONEP_ERR_ALIGN: return "H must be a multiple of 8 and bf16 data pointers 16-byte aligned";
+    case MOONEP_ERR_NOALLOC_SIZE:
+        return "workspace larger than the fixed no-allocation array (MOONEP_NOALLOC_WORKSPACE_BYTES)";
     default: return "unknown error";
     }
 }

@@ -49,7 +49,8 @@ PLAN_FIELDS = ("expert_count", "slot_expert", "slot_count", "slot_offset", "rep_
 
 EXPORTED = ("moonep_check_config", "moonep_plan_sizes", "moonep_plan_layout", "moonep_plan",
             "moonep_dispatch", "moonep_combine", "moonep_combine_backward",
-            "moonep_reduce_replica_grads", "moonep_error_string", "moonep_abi_version")
+            "moonep_reduce_replica_grads", "moonep_error_string", "moonep_abi_version",
+            "moonep_plan_noalloc")
 
 
 class _CConfig(ctypes.Structure):
@@ -73,6 +74,7 @@ _lib.moonep_dispatch.argtypes = [_cfgp, _planp, _vp, _vp, _vp]
 _lib.moonep_combine.argtypes = [_cfgp, _planp, _vp, _vp, _vp, _vp]
 _lib.moonep_combine_backward.argtypes = [_cfgp, _planp, _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.moonep_reduce_replica_grads.argtypes = [_cfgp, _planp, _vp, _vp, ctypes.c_int64, _vp]
+_lib.moonep_plan_noalloc.argtypes = [_cfgp, _vp, _planp, _vp]
 _lib.moonep_error_string.argtypes = [ctypes.c_int]
 _lib.moonep_error_string.restype = ctypes.c_char_p
 _lib.moonep_abi_version.argtypes = []
@@ -212,6 +214,24 @@ def plan(cfg: Config, topk_idx: torch.Tensor, out: Plan | None = None, stream=No
     _check(_lib.moonep_plan(ctypes.byref(c), topk_idx.data_ptr(), ctypes.byref(p.c_plan),
                             p.workspace.data_ptr(), _stream(stream)))
     return p
+
+
+NOALLOC_WORKSPACE_BYTES = 4 << 20
+
+
+def plan_noalloc(cfg: Config, topk_idx: torch.Tensor, out: Plan, stream=None) -> Plan:
+    """Same plan as ``plan`` without using the workspace of ``out``: the
+    library's fixed device array serves as scratch space instead.  For
+    callers that cannot allocate device memory (a runtime that owns every
+    allocation, a hot path that must not call cudaMalloc).  ``out`` still
+    provides the plan arrays.  Calls share one array per device, so calls
+    that overlap on the GPU race; the first call on a device should come
+    before any stream capture."""
+    _need(topk_idx, torch.int32, (cfg.tokens, cfg.K), "topk_idx")
+    c = cfg.c()
+    _check(_lib.moonep_plan_noalloc(ctypes.byref(c), topk_idx.data_ptr(), ctypes.byref(out.c_plan),
+                                    _stream(stream)))
+    return out
 
 
 def dispatch(cfg: Config, p: Plan, hidden: torch.Tensor, buf: torch.Tensor | None = None,

@@ -36,7 +36,9 @@ static int make_dims(const moonep_config *c, Dims *d)
     d->C = c->S * c->K;
     d->tokens = c->R * c->S;
     d->pairs = c->R * c->S * c->K;
-    int ct = (d->tokens + 255) / 256;
+    // about two planner CTAs per SM of a B200 (148 SMs); the chunking only
+    // affects speed, never the plan
+    int ct = (d->tokens + 295) / 296;
     if (ct < 8) ct = 8;
     int cap = 4096 / d->K;
     if (cap < 1) cap = 1;

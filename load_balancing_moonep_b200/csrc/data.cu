@@ -118,165 +118,6 @@ __global__ void __launch_bounds__(DATA_THREADS) dispatch_kernel(const uint4 *__r
 }
 
 
-// ------------------------------------------------- dispatch, TMA bulk path
-//
-// One warp per CTA.  Token rows are staged in shared memory by 1-D bulk
-// copies (cp.async.bulk global -> shared, completion on an mbarrier; no
-// tensor map, no multicast), then written K times by bulk stores (shared ->
-// global, bulk async-groups).  NS stages: D = NS - LAG loads run ahead, and a
-// stage is refilled once the stores issued LAG tokens earlier have finished
-// reading it.  Rows longer than the stage size are split into pieces.
-
-constexpr int TMA_LAG = 3;
-constexpr long long WAIT_LIMIT = 1ll << 26;
-
-__device__ __forceinline__ uint32_t smem_u32(const void *p)
-{
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-__device__ __forceinline__ void bulk_load(void *sdst, const void *gsrc, uint32_t bytes, uint64_t *bar)
-{
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                     smem_u32(sdst)),
-                 "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
-                 : "memory");
-}
-
-__device__ __forceinline__ void bulk_store(void *gdst, const void *ssrc, uint32_t bytes)
-{
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(smem_u32(ssrc)),
-                 "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-
-template <int N>
-__device__ __forceinline__ void bulk_wait_read()
-{
-    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
-}
-
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-
-struct TmaDispatchArgs {
-    const uint8_t *hidden;
-    uint8_t *buf;
-    const int *dst_pos;
-    int *info;
-    int tokens, K, rows;
-    int row_bytes;    // H * 2
-    int piece_bytes;  // stage size, multiple of 16
-    int pieces;       // pieces per row
-    int NS;           // stages
-};
-
-__global__ void __launch_bounds__(32) dispatch_tma_kernel(TmaDispatchArgs a)
-{
-    extern __shared__ __align__(128) uint8_t sm[];
-    if (plan_invalid(a.info)) return;
-    const int lane = threadIdx.x;
-    uint64_t *full = reinterpret_cast<uint64_t *>(sm);
-    uint8_t *stages = sm + 128 * ((a.NS * 8 + 127) / 128);
-    const int NS = a.NS, D = a.NS - TMA_LAG;
-    if (lane == 0) {
-        for (int s = 0; s < NS; ++s) mbar_init(full + s, 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    __syncwarp();
-
-    const long long units = (long long)a.tokens * a.pieces;
-    const long long n = units > blockIdx.x ? (units - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
-    auto unit_src = [&](long long i, uint32_t &bytes) -> const uint8_t * {
-        const long long u = blockIdx.x + i * gridDim.x;
-        const long long t = u / a.pieces;
-        const int c = (int)(u - t * a.pieces);
-        const int off = c * a.piece_bytes;
-        bytes = (uint32_t)min(a.piece_bytes, a.row_bytes - off);
-        return a.hidden + t * a.row_bytes + off;
-    };
-    if (lane == 0) {
-        for (long long j = 0; j < (D < n ? (long long)D : n); ++j) {
-            uint32_t bytes;
-            const uint8_t *src = unit_src(j, bytes);
-            mbar_expect_tx(full + j, bytes);
-            bulk_load(stages + (size_t)j * a.piece_bytes, src, bytes, full + j);
-        }
-    }
-    bool timed_out = false;
-    for (long long i = 0; i < n; ++i) {
-        const int s = (int)(i % NS);
-        const uint32_t parity = (uint32_t)((i / NS) & 1);
-        const long long u = blockIdx.x + i * gridDim.x;
-        const long long t = u / a.pieces;
-        const int c = (int)(u - t * a.pieces);
-        const int off = c * a.piece_bytes;
-        const uint32_t bytes = (uint32_t)min(a.piece_bytes, a.row_bytes - off);
-        // destination rows of this token (lanes 0..K-1), fetched while the load lands
-        int d[2] = {-1, -1};
-#pragma unroll
-        for (int q = 0; q < 2; ++q)
-            if (lane + 32 * q < a.K) d[q] = __ldg(a.dst_pos + t * a.K + lane + 32 * q);
-        long long spins = 0;
-        while (!mbar_try_wait(full + s, parity)) {
-            if (++spins > WAIT_LIMIT) {
-                timed_out = true;
-                break;
-            }
-        }
-        if (__any_sync(FULL_MASK, timed_out)) {
-            timed_out = true;
-            break;
-        }
-#pragma unroll
-        for (int q = 0; q < 2; ++q)
-            if (lane + 32 * q < a.K && row_ok(d[q], a.rows, a.info))
-                bulk_store(a.buf + (long long)d[q] * a.row_bytes + off, stages + (size_t)s * a.piece_bytes, bytes);
-        bulk_commit();
-        const long long nxt = i + D;
-        if (nxt < n) {
-            // stage of unit nxt was last used by unit i - LAG: wait until its
-            // stores (and every older group of this lane) have read the stage
-            bulk_wait_read<TMA_LAG>();
-            __syncwarp();
-            if (lane == 0) {
-                const int sn = (int)(nxt % NS);
-                uint32_t nb;
-                const uint8_t *src = unit_src(nxt, nb);
-                mbar_expect_tx(full + sn, nb);
-                bulk_load(stages + (size_t)sn * a.piece_bytes, src, nb, full + sn);
-            }
-        }
-    }
-    bulk_wait_all();
-    if (timed_out && lane == 0) atomicOr(a.info + MOONEP_INFO_STATUS, MOONEP_ST_WAIT_TIMEOUT);
-}
-
 // ---------------------------------------------------------------- combine
 
 // KT > 0: compile-time K (all K loads of a vector issued together);
@@ -460,63 +301,9 @@ static int data_grid(int tokens)
     return want < full ? (want > 0 ? want : 1) : full;
 }
 
-// Dispatch path: TMA bulk copies for rows of at least 2 KB, otherwise the
-// vector kernel (tiny rows make per-copy overheads dominate).
-constexpr int TMA_MIN_ROW_BYTES = 2048;
-constexpr int TMA_MAX_PIECE = 32768;
-constexpr int TMA_CTAS_PER_SM = 1;
-
-static int sm_count()
-{
-    static int sms[64] = {0};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64) dev = 0;
-    if (!sms[dev]) {
-        int v = 0;
-        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-        sms[dev] = v > 0 ? v : 148;
-    }
-    return sms[dev];
-}
-
-static int launch_dispatch_tma(const Dims &d, const int *dst_pos, int *info, const uint16_t *hidden,
-                               uint16_t *buf, cudaStream_t st)
-{
-    TmaDispatchArgs a;
-    a.hidden = reinterpret_cast<const uint8_t *>(hidden);
-    a.buf = reinterpret_cast<uint8_t *>(buf);
-    a.dst_pos = dst_pos;
-    a.info = info;
-    a.tokens = d.tokens;
-    a.K = d.K;
-    a.rows = d.pairs;
-    a.row_bytes = d.H * 2;
-    a.piece_bytes = a.row_bytes < TMA_MAX_PIECE ? a.row_bytes : TMA_MAX_PIECE;
-    a.pieces = (a.row_bytes + a.piece_bytes - 1) / a.piece_bytes;
-    const int budget = (227 * 1024) / TMA_CTAS_PER_SM - 1024;
-    int ns = budget / a.piece_bytes;
-    if (ns > 16) ns = 16;
-    if (ns < TMA_LAG + 2) return -1;
-    a.NS = ns;
-    const size_t smem = 128 * ((ns * 8 + 127) / 128) + (size_t)ns * a.piece_bytes;
-    if (cudaFuncSetAttribute(dispatch_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
-        return MOONEP_ERR_CUDA;
-    const long long units = (long long)d.tokens * a.pieces;
-    long long grid = (long long)sm_count() * TMA_CTAS_PER_SM;
-    if (grid > units) grid = units;
-    dispatch_tma_kernel<<<(int)grid, 32, smem, st>>>(a);
-    return cudaGetLastError() == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
-}
-
 int launch_dispatch(const Dims &d, const int *dst_pos, int *info, const uint16_t *hidden, uint16_t *buf,
                     cudaStream_t st)
 {
-    if (d.H * 2 >= TMA_MIN_ROW_BYTES && d.K <= 64) {
-        const int rc = launch_dispatch_tma(d, dst_pos, info, hidden, buf, st);
-        if (rc >= 0) return rc;
-    }
     const int vpr = d.H / 8;
     const int grid = data_grid(d.tokens);
     dispatch_kernel<4><<<grid, DATA_THREADS, 0, st>>>(reinterpret_cast<const uint4 *>(hidden),

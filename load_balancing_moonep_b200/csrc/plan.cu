@@ -8,24 +8,28 @@
 // This file implements the water-filling plan described in moonep.h in two
 // launches, with no host synchronisation and no inter-CTA waiting:
 //
-//   hist_plan_kernel  one CTA per token chunk builds the chunk's expert
-//                     histogram in shared memory (ballot-matched lanes add
-//                     once per distinct expert), stores it for the second
-//                     pass and adds it to per-group and total counts with
-//                     atomics (sums: order-free, so deterministic).  The CTA
-//                     that finishes last (atomic ticket) runs the planner:
-//                     loads, largest-first shedding, (value desc, index asc)
-//                     orders by counting rank, prefix sums, water-filling as a
-//                     parallel merge of the two prefix-sum partitions,
-//                     compact per-rank slot lists, rank-ordered host
-//                     intervals.  It writes compact results only.
-//   assign_kernel     one CTA per token chunk: the stable within-expert rank g
-//                     of every (t, k) pair from the counts of earlier groups
-//                     and chunks, per-warp counters and ballot matching; the
-//                     host interval holding g gives the buffer row.  The CTAs
-//                     also expand the compact slot lists into the padded
-//                     [R][E] tables.  Launched with programmatic dependent
-//                     launch: its input-only prologue overlaps the planner.
+//   hist_plan_kernel  one CTA per token chunk stages the chunk's ids in
+//                     shared memory and counts them with shared-memory
+//                     atomics (a token's K experts are distinct, so few lanes
+//                     of a warp collide), stores the counts for the second
+//                     pass and adds them to per-group and total counts with
+//                     global atomics (sums: order-free, so deterministic).
+//                     The CTA that finishes last (atomic ticket) runs the
+//                     planner: loads, largest-first shedding, (value desc,
+//                     index asc) orders by counting rank, prefix sums,
+//                     water-filling as a parallel merge of the two prefix-sum
+//                     partitions, compact per-rank slot lists, rank-ordered
+//                     host intervals.  It writes compact results only.
+//   assign_kernel     one CTA per token chunk: each warp counts its
+//                     contiguous sub-range, a prefix over earlier groups,
+//                     chunks and warps gives every warp its base, then the
+//                     warp walks its sub-range in (t, k) order ranking equal
+//                     experts with ballots, so g is the pair's rank among all
+//                     earlier pairs of its expert; the host interval holding
+//                     g gives the buffer row.  The CTAs also expand the
+//                     compact slot lists into the padded [R][E] tables.
+//                     Launched with programmatic dependent launch: its
+//                     input-only prologue overlaps the planner.
 #include "common.cuh"
 
 namespace moonep {
@@ -47,7 +51,7 @@ struct PlanParams {
     int *sc_exp;     // [2E+R]
     int *sc_cnt;     // [2E+R]
     int *sc_off;     // [2E+R]
-    FastDiv fK, fS, fC;
+    FastDiv fC;
 };
 
 // ints of dynamic shared memory used by the planner block
@@ -62,7 +66,13 @@ __host__ __device__ inline int plan_smem_ints(int E, int R)
 
 __host__ __device__ inline int assign_smem_ints(int E, int R, int max_pairs)
 {
-    return E + ASSIGN_WARPS * E + 2 * max_pairs + (E + 1) + 2 * (2 * E + R) + 32;
+    return E + ASSIGN_WARPS * E + max_pairs + (E + 1) + 2 * (2 * E + R) + 32;
+}
+
+__host__ __device__ inline int hist_smem_ints(int E, int R, int max_pairs)
+{
+    const int a = plan_smem_ints(E, R), b = E + max_pairs;
+    return a > b ? a : b;
 }
 
 __device__ __forceinline__ int seg_quota(const int *PS, const int *QS, int j, int i)
@@ -397,30 +407,27 @@ __global__ void __launch_bounds__(PLAN_THREADS) hist_plan_kernel(PlanParams a)
     __shared__ int s_last, s_parity;
     const Dims &d = a.d;
     const int E = d.E, K = d.K, tid = threadIdx.x, nt = blockDim.x;
-    const int lane = tid & 31, warp = tid >> 5;
     // the assignment kernel may be scheduled now; it waits for this whole
     // grid before it reads anything this grid writes
     pdl_launch_dependents();
 
-    int *hist = sm;
-    for (int e = tid; e < E; e += nt) hist[e] = 0;
-    if (tid == 0) s_parity = ld_cg(a.hdr + WS_PARITY) & 1;
-    __syncthreads();
-    const int parity = s_parity;
-
     const int chunk = blockIdx.x;
     const int t0 = chunk * d.chunk_tokens;
     const int t1 = min(t0 + d.chunk_tokens, d.tokens);
-    const int p0 = t0 * K, p1 = t1 * K;
+    const int p0 = t0 * K, n = (t1 - t0) * K;
+    int *hist = sm;       // E
+    int *ids = sm + E;    // chunk_tokens * K
+    for (int e = tid; e < E; e += nt) hist[e] = 0;
+    for (int i = tid; i < n; i += nt) ids[i] = __ldg(a.topk + p0 + i);  // all loads in flight
+    if (tid == 0) s_parity = ld_cg(a.hdr + WS_PARITY) & 1;
+    __syncthreads();
+    const int parity = s_parity;
+    // distinct experts within a token: at most 32/K lanes of a warp collide
     int bad = 0;
-    for (int base = p0 + warp * 32; base < p1; base += nt) {
-        const int p = base + lane;
-        const bool valid = p < p1;
-        const int e = valid ? __ldg(a.topk + p) : -1;
-        const bool ok = valid && e >= 0 && e < E;
-        if (valid && !ok) bad = 1;
-        const unsigned peers = peers_of(ok ? e : 0, ok, d.ebits);
-        if (ok && lane == __ffs(peers) - 1) atomicAdd(&hist[e], __popc(peers));
+    for (int i = tid; i < n; i += nt) {
+        const int e = ids[i];
+        if (e < 0 || e >= E) bad = 1;
+        else atomicAdd(&hist[e], 1);
     }
     bad = __syncthreads_or(bad);
     int *gsb = a.gs + ((size_t)parity * d.ngroups + chunk / CHUNK_GROUP) * E;
@@ -444,7 +451,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) hist_plan_kernel(PlanParams a)
 
 // ---------------------------------------------------------- assignment
 
-__global__ void __launch_bounds__(ASSIGN_THREADS) assign_kernel(PlanParams a)
+__global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
 {
     extern __shared__ int sm[];
     const Dims &d = a.d;
@@ -460,8 +467,7 @@ __global__ void __launch_bounds__(ASSIGN_THREADS) assign_kernel(PlanParams a)
     int *base = sm;                        // E
     int *cnt = base + E;                   // ASSIGN_WARPS * E
     int *ids = cnt + ASSIGN_WARPS * E;     // max_pairs
-    int *lr = ids + max_pairs;             // max_pairs
-    int *hptr = lr + max_pairs;            // E + 1
+    int *hptr = ids + max_pairs;           // E + 1
     int *hstart = hptr + E + 1;            // nh
     int *hdst = hstart + nh;               // nh
     int *red = hdst + nh;                  // 32
@@ -535,51 +541,50 @@ __global__ void __launch_bounds__(ASSIGN_THREADS) assign_kernel(PlanParams a)
         hdst[h] = ld_cg(a.host_dst0 + h);
     }
     // pairs of each expert in earlier chunks: earlier groups + earlier chunks
-    // of this chunk's group (independent loads)
+    // of this chunk's group, all loads of a batch in flight together
     {
         const int grp = chunk / CHUNK_GROUP, c0 = grp * CHUNK_GROUP;
         const int parity = ld_cg(a.hdr + WS_PARITY) ^ 1;  // the buffer this call filled
         const int *gsb = a.gs + (size_t)parity * d.ngroups * E;
         for (int e = tid; e < E; e += nt) {
             int s = 0;
-            for (int g0 = 0; g0 < grp; g0 += 8) {
-                int v[8];
+            for (int g0 = 0; g0 < grp; g0 += 16) {
+                int v[16];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) v[j] = (g0 + j < grp) ? ld_cg(gsb + (size_t)(g0 + j) * E + e) : 0;
+                for (int j = 0; j < 16; ++j) v[j] = (g0 + j < grp) ? ld_cg(gsb + (size_t)(g0 + j) * E + e) : 0;
+                int w[CHUNK_GROUP - 1];
+                if (g0 == 0) {
 #pragma unroll
-                for (int j = 0; j < 8; ++j) s += v[j];
+                    for (int j = 0; j < CHUNK_GROUP - 1; ++j)
+                        w[j] = (c0 + j < chunk) ? ld_cg(a.cc + (size_t)(c0 + j) * E + e) : 0;
+#pragma unroll
+                    for (int j = 0; j < CHUNK_GROUP - 1; ++j) s += w[j];
+                }
+#pragma unroll
+                for (int j = 0; j < 16; ++j) s += v[j];
             }
-            int v[CHUNK_GROUP - 1];
+            if (grp == 0) {
+                int w[CHUNK_GROUP - 1];
 #pragma unroll
-            for (int j = 0; j < CHUNK_GROUP - 1; ++j)
-                v[j] = (c0 + j < chunk) ? ld_cg(a.cc + (size_t)(c0 + j) * E + e) : 0;
+                for (int j = 0; j < CHUNK_GROUP - 1; ++j)
+                    w[j] = (c0 + j < chunk) ? ld_cg(a.cc + (size_t)(c0 + j) * E + e) : 0;
 #pragma unroll
-            for (int j = 0; j < CHUNK_GROUP - 1; ++j) s += v[j];
+                for (int j = 0; j < CHUNK_GROUP - 1; ++j) s += w[j];
+            }
             base[e] = s;
         }
     }
     __syncthreads();
 
-    // pass 1: rank of each pair among earlier pairs of its expert inside the
-    // warp's contiguous sub-range (ballot-matched lanes)
+    // pass 1: count each expert's pairs in every warp's contiguous sub-range
+    // (distinct experts within a token: at most 32/K lanes collide)
     const int per = (n + ASSIGN_WARPS - 1) / ASSIGN_WARPS;
     const int wbeg = min(warp * per, n), wend = min(wbeg + per, n);
     {
         int *wc = cnt + warp * E;
-        for (int b = wbeg; b < wend; b += 32) {
-            const int i = b + lane;
-            const bool valid = i < wend;
-            const int e = valid ? ids[i] : 0;
-            const bool ok = valid && e >= 0 && e < E;
-            const unsigned peers = peers_of(ok ? e : 0, ok, d.ebits);
-            int r0 = 0;
-            if (ok) {
-                r0 = wc[e];
-                lr[i] = r0 + __popc(peers & lanemask_lt());
-            }
-            __syncwarp();
-            if (ok && lane == __ffs(peers) - 1) wc[e] = r0 + __popc(peers);
-            __syncwarp();
+        for (int i = wbeg + lane; i < wend; i += 32) {
+            const int e = ids[i];
+            if (e >= 0 && e < E) atomicAdd(&wc[e], 1);
         }
     }
     __syncthreads();
@@ -594,14 +599,24 @@ __global__ void __launch_bounds__(ASSIGN_THREADS) assign_kernel(PlanParams a)
     }
     __syncthreads();
 
-    // pass 2: the host interval holding g gives the buffer row
+    // pass 2, in (t, k) order within the warp's sub-range: g = warp base +
+    // earlier pairs of the expert in this sub-range (ballot-matched lanes);
+    // the host interval holding g gives the buffer row
     int remote = 0;
     {
-        const int *wc = cnt + warp * E;
-        for (int i = wbeg + lane; i < wend; i += 32) {
-            const int e = ids[i];
-            if (e < 0 || e >= E) continue;
-            const int g = wc[e] + lr[i];
+        int *wc = cnt + warp * E;
+        for (int b = wbeg; b < wend; b += 32) {
+            const int i = b + lane;
+            const bool valid = i < wend;
+            const int e = valid ? ids[i] : 0;
+            const bool ok = valid && e >= 0 && e < E;
+            const unsigned peers = peers_of(ok ? e : 0, ok, d.ebits);
+            int g = 0;
+            if (ok) g = wc[e] + __popc(peers & lanemask_lt());
+            __syncwarp();
+            if (ok && lane == __ffs(peers) - 1) wc[e] += __popc(peers);
+            __syncwarp();
+            if (!ok) continue;
             int h = hptr[e];
             const int hend = hptr[e + 1];
             while (h + 1 < hend && hstart[h + 1] <= g) ++h;
@@ -614,7 +629,8 @@ __global__ void __launch_bounds__(ASSIGN_THREADS) assign_kernel(PlanParams a)
             }
             a.p.dst_pos[p] = dst;
             a.p.row_src[dst] = p;
-            remote += fdiv((uint32_t)dst, a.fC) != fdiv(fdiv((uint32_t)p, a.fK), a.fS);
+            // source rank of pair p is p / (S*K) = p / C
+            remote += fdiv((uint32_t)dst, a.fC) != fdiv((uint32_t)p, a.fC);
         }
     }
 #pragma unroll
@@ -652,11 +668,9 @@ int launch_plan(const Dims &d, const int32_t *topk, const moonep_plan_t &p, void
     a.sc_exp = reinterpret_cast<int *>(w + wl.sc_exp);
     a.sc_cnt = reinterpret_cast<int *>(w + wl.sc_cnt);
     a.sc_off = reinterpret_cast<int *>(w + wl.sc_off);
-    a.fK = make_fastdiv((uint32_t)d.K);
-    a.fS = make_fastdiv((uint32_t)d.S);
     a.fC = make_fastdiv((uint32_t)d.C);
 
-    const size_t smem1 = sizeof(int) * (size_t)plan_smem_ints(d.E, d.R);
+    const size_t smem1 = sizeof(int) * (size_t)hist_smem_ints(d.E, d.R, d.chunk_tokens * d.K);
     if (!set_smem((const void *)hist_plan_kernel, smem1)) return MOONEP_ERR_CUDA;
     hist_plan_kernel<<<d.nchunk, PLAN_THREADS, smem1, st>>>(a);
     if (cudaGetLastError() != cudaSuccess) return MOONEP_ERR_CUDA;
@@ -679,7 +693,7 @@ int launch_plan(const Dims &d, const int32_t *topk, const moonep_plan_t &p, void
 
 size_t plan_smem_bytes_max(const Dims &d)
 {
-    const size_t a = sizeof(int) * (size_t)plan_smem_ints(d.E, d.R);
+    const size_t a = sizeof(int) * (size_t)hist_smem_ints(d.E, d.R, d.chunk_tokens * d.K);
     const size_t b = sizeof(int) * (size_t)assign_smem_ints(d.E, d.R, d.chunk_tokens * d.K);
     return a > b ? a : b;
 }

@@ -451,43 +451,99 @@ def run_ours(args, world, rank, local):
                           "remote_pair_frac": round(inf["n_remote_pairs"] / wl.pairs, 4)})
             del ps
 
-    # end to end through the public API with pinned host buffers
+    # end to end through the public API with pinned host buffers: every step
+    # copies its routing, weights and hidden states in and its output out.
+    # Double-buffered and pipelined on three streams, so step i+1's inputs
+    # and step i-1's output cross PCIe while step i runs.
     e2e = None
     if not args.no_e2e:
-        h_topk = r.topk_idx.cpu().pin_memory()
-        h_w = r.weights.cpu().pin_memory()
-        h_hidden = hidden.cpu().pin_memory()
-        h_out = torch.empty((wl.tokens, wl.H), dtype=torch.bfloat16).pin_memory()
-        d_topk = torch.empty_like(r.topk_idx)
-        d_w = torch.empty_like(r.weights)
-        d_hidden = torch.empty_like(hidden)
+        nb = 2
+        h_topk = [r.topk_idx.cpu().pin_memory() for _ in range(nb)]
+        h_w = [r.weights.cpu().pin_memory() for _ in range(nb)]
+        h_hidden = [hidden.cpu().pin_memory() for _ in range(nb)]
+        h_out = [torch.empty((wl.tokens, wl.H), dtype=torch.bfloat16).pin_memory() for _ in range(nb)]
+        d_topk = [torch.empty_like(r.topk_idx) for _ in range(nb)]
+        d_w = [torch.empty_like(r.weights) for _ in range(nb)]
+        d_hidden = [hidden] + [torch.empty_like(hidden) for _ in range(nb - 1)]
+        d_out = [out] + [torch.empty_like(out) for _ in range(nb - 1)]
+        s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+        ev_in = [torch.cuda.Event() for _ in range(nb)]
+        ev_used = [torch.cuda.Event() for _ in range(nb)]   # inputs consumed
+        ev_done = [torch.cuda.Event() for _ in range(nb)]   # output written
+        ev_read = [torch.cuda.Event() for _ in range(nb)]   # output copied out
+        for b in range(nb):
+            for ev in (ev_used[b], ev_read[b]):
+                ev.record(s_cmp)
 
-        def e2e_step():
-            d_topk.copy_(h_topk, non_blocking=True)
-            d_w.copy_(h_w, non_blocking=True)
-            d_hidden.copy_(h_hidden, non_blocking=True)
-            mp.plan(cfg, d_topk, out=plan)
-            mp.dispatch(cfg, plan, d_hidden, buf)
-            mp.combine(cfg, plan, buf, d_w, out)
-            h_out.copy_(out, non_blocking=True)
+        def e2e_step(i):
+            b = i % nb
+            with torch.cuda.stream(s_in):
+                s_in.wait_event(ev_used[b])
+                d_topk[b].copy_(h_topk[b], non_blocking=True)
+                d_w[b].copy_(h_w[b], non_blocking=True)
+                d_hidden[b].copy_(h_hidden[b], non_blocking=True)
+                ev_in[b].record(s_in)
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(ev_in[b])
+                s_cmp.wait_event(ev_read[b])
+                mp.plan(cfg, d_topk[b], out=plan, stream=s_cmp)
+                mp.dispatch(cfg, plan, d_hidden[b], buf, stream=s_cmp)
+                mp.combine(cfg, plan, buf, d_w[b], d_out[b], stream=s_cmp)
+                ev_used[b].record(s_cmp)
+                ev_done[b].record(s_cmp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_done[b])
+                h_out[b].copy_(d_out[b], non_blocking=True)
+                ev_read[b].record(s_out)
 
-        for _ in range(2):
-            e2e_step()
+        for i in range(2):
+            e2e_step(i)
         torch.cuda.synchronize()
         barrier(world)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        n_e2e = max(3, min(args.steps, 10))
-        for _ in range(n_e2e):
-            e2e_step()
-        b.record()
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(4, min(args.steps, 10))
+        a.record(s_in)
+        s_cmp.wait_event(a)
+        s_out.wait_event(a)
+        for i in range(n_e2e):
+            e2e_step(i)
+        b_.record(s_out)
         torch.cuda.synchronize()
-        e_ms = max_over_ranks(world, a.elapsed_time(b) / n_e2e)
+        e_ms = max_over_ranks(world, a.elapsed_time(b_) / n_e2e)
         e2e = {"value": round(dc_bytes / (e_ms * 1e-3) / 1e9, 2), "unit": UNIT,
                "ms_per_step": round(e_ms, 3),
-               "h2d_bytes_per_step": int(h_topk.numel() * 4 + h_w.numel() * 4 + h_hidden.numel() * 2),
-               "d2h_bytes_per_step": int(h_out.numel() * 2),
-               "what": "pinned host topk/weights/hidden -> plan -> dispatch -> combine -> host out"}
+               "h2d_bytes_per_step": int(h_topk[0].numel() * 4 + h_w[0].numel() * 4 + h_hidden[0].numel() * 2),
+               "d2h_bytes_per_step": int(h_out[0].numel() * 2),
+               "what": ("pinned host topk/weights/hidden -> plan -> dispatch -> combine -> pinned host "
+                        "out, every step; double-buffered, copies of neighbouring steps overlap")}
+        del d_topk, d_w, d_hidden, d_out
+
+    # replica weight prefetch (a next-row step, timed on its own after the
+    # step: its 68 GB of weights and pool fit once the reduce buffers are freed)
+    if P and not args.no_prefetch:
+        del rb, hg
+        torch.cuda.empty_cache()
+        Pw = wl.grad_elems
+        weights = W.bf16_normal((wl.E, Pw), seed=7 + rank, device=dev)
+        pool = torch.empty((wl.R, wl.B, Pw), dtype=torch.bfloat16, device=dev)
+        wrow = torch.empty((wl.R, wl.E), dtype=torch.int32, device=dev)
+        for _ in range(2):
+            mp.prefetch_replicas(cfg, plan, weights, pool, wrow)
+        torch.cuda.synchronize()
+        pt = Timer()
+        for _ in range(5):
+            ev = pt.mark("prefetch")
+            mp.prefetch_replicas(cfg, plan, weights, pool, wrow)
+            ev.record()
+        torch.cuda.synchronize()
+        pms = pt.total_ms("prefetch") / 5
+        pbytes = n_pref * Pw * 2 * 2 + wl.R * wl.E * 8
+        kernels["prefetch"] = {"ms": round(pms, 4), "bytes": pbytes, "GB/s": round(pbytes / (pms * 1e-3) / 1e9, 1),
+                               "frac": round(pbytes / (pms * 1e-3) / 1e9 / peak, 4), "traffic": traffic.get("prefetch"),
+                               "in_step": False,
+                               "what": f"{n_pref} replicas x {Pw} bf16 (gate+up+down) copied into the pool"}
+        del weights, pool, wrow
+        torch.cuda.empty_cache()
 
     # the CPU oracle on a bounded sample (rank 0, one GPU only)
     cpu = None
@@ -522,9 +578,10 @@ def run_ours(args, world, rank, local):
 
 
 def run_profile_case(args):
-    """--profile: two passes of the whole step on a reduced-size copy of the
-    workload (S tokens per rank, P gradient elements), a few GB on the
-    device, for ncu captures; prints a one-line summary, no timing."""
+    """--profile: two passes of the whole step (plus the replica weight
+    prefetch) on a reduced-size copy of the workload (S tokens per rank, P
+    gradient / weight elements per expert), a few GB on the device, for ncu
+    captures -- 7 launches per pass; prints a one-line summary, no timing."""
     from load_balancing_moonep_b200 import moonep as mp
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
@@ -539,9 +596,12 @@ def run_profile_case(args):
     P = args.profile_P
     rb = W.f32_normal((wl.R, wl.B, P), seed=4, device=dev, std=1e-3)
     hg = W.f32_normal((wl.E, P), seed=5, device=dev, std=1e-3)
+    weights = W.bf16_normal((wl.E, P), seed=7, device=dev)
+    pool = torch.empty((wl.R, wl.B, P), dtype=torch.bfloat16, device=dev)
     plan = mp.Plan(cfg, dev)
     for _ in range(2):
         mp.plan(cfg, r.topk_idx, out=plan)
+        mp.prefetch_replicas(cfg, plan, weights, pool)
         mp.dispatch(cfg, plan, hidden, buf)
         mp.combine(cfg, plan, buf, r.weights, out)
         mp.combine_backward(cfg, plan, dy, r.weights, buf, dy_buf)
@@ -567,6 +627,7 @@ def main():
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefetch", action="store_true")
     ap.add_argument("--profile", action="store_true",
                     help="run two untimed steps of a reduced-size case (for ncu)")
     ap.add_argument("--profile-S", type=int, default=512)

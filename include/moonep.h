@@ -209,6 +209,26 @@ MOONEP_API int moonep_combine_backward(const moonep_config *cfg, const moonep_pl
 MOONEP_API int moonep_reduce_replica_grads(const moonep_config *cfg, const moonep_plan_t *plan,
                                 float *reduce_buf, float *home_grad, int64_t P, void *stream);
 
+/* Replica weight prefetch (MoonEP article, "The core idea": duplicated
+ * experts are prefetched before expert computation; explainer, memory tab:
+ * the prefetch slots are rows [E, E+B) of one contiguous weight pool, E read
+ * here as the rank's L home experts, and a rank needing more than B foreign
+ * experts reads the overflow from the home copy).
+ *   pool[r][b][:] = weights[e][:]  for every replica of expert e on rank r
+ *                                  with ordinal b = slot - L < B
+ *   slot_wrow[r][s] = weight row the expert computation of slot s of rank r
+ *       uses, in the concatenated row space [weights (E rows) | pool (R*B rows)]:
+ *       home slot -> e, prefetched replica -> E + r*B + b, overflow replica
+ *       -> e (read-through), unused slot -> -1.
+ * weights: bf16 [E, P] (one expert's weights per row, e.g. gate+up+down);
+ * pool: bf16 [R, B, P] (may be NULL when B == 0); slot_wrow: int32 [R][E];
+ * P > 0 elements per expert.  Pool rows of unused slots are left as they
+ * are.  A plan with MOONEP_ST_EXPERT_ID_RANGE copies nothing and marks every
+ * slot -1. */
+MOONEP_API int moonep_prefetch_replicas(const moonep_config *cfg, const moonep_plan_t *plan,
+                                        const uint16_t *weights, uint16_t *pool, int32_t *slot_wrow,
+                                        int64_t P, void *stream);
+
 /* Size of the fixed device array behind moonep_plan_noalloc (4 MiB).  The
  * large training shape (R=32, E=384, K=8, S=4096) needs about 0.5 MiB. */
 #define MOONEP_NOALLOC_WORKSPACE_BYTES (4u << 20)

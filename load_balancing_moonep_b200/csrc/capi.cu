@@ -17,6 +17,8 @@ int launch_combine_backward(const Dims &d, const int *dst_pos, int *info, const 
                             const uint16_t *y, uint16_t *dy_buf, float *dw, cudaStream_t st);
 int launch_reduce(const Dims &d, const moonep_plan_t &p, float *reduce_buf, float *home_grad, long long P,
                   cudaStream_t st);
+int launch_prefetch(const Dims &d, const moonep_plan_t &p, const uint16_t *weights, uint16_t *pool,
+                    int32_t *slot_wrow, long long P, cudaStream_t st);
 
 constexpr size_t MAX_DYN_SMEM = 227 * 1024;
 constexpr int MAX_COMBINE_BWD_K = 16;
@@ -210,6 +212,20 @@ int moonep_reduce_replica_grads(const moonep_config *cfg, const moonep_plan_t *p
     if ((reinterpret_cast<uintptr_t>(reduce_buf) & 3u) || (reinterpret_cast<uintptr_t>(home_grad) & 3u))
         return MOONEP_ERR_ALIGN;
     return launch_reduce(d, *plan, reduce_buf, home_grad, (long long)P, static_cast<cudaStream_t>(stream));
+}
+
+int moonep_prefetch_replicas(const moonep_config *cfg, const moonep_plan_t *plan, const uint16_t *weights,
+                             uint16_t *pool, int32_t *slot_wrow, int64_t P, void *stream)
+{
+    Dims d;
+    const int rc = make_dims(cfg, &d);
+    if (rc != MOONEP_OK) return rc;
+    if (!plan_ok(plan) || !weights || !slot_wrow || P <= 0) return MOONEP_ERR_ARG;
+    if (d.B > 0 && !pool) return MOONEP_ERR_ARG;
+    if ((reinterpret_cast<uintptr_t>(weights) & 1u) || (reinterpret_cast<uintptr_t>(pool) & 1u) ||
+        (reinterpret_cast<uintptr_t>(slot_wrow) & 3u))
+        return MOONEP_ERR_ALIGN;
+    return launch_prefetch(d, *plan, weights, pool, slot_wrow, (long long)P, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -439,13 +439,19 @@ __global__ void __launch_bounds__(PLAN_THREADS) hist_plan_kernel(PlanParams a)
             atomicAdd(gsb + e, c);
         }
     }
-    if (bad && tid == 0) atomicOr(a.hdr + WS_STATUS, MOONEP_ST_EXPERT_ID_RANGE);
-    __threadfence();
+    // release: the CTA barrier orders every thread's writes before thread 0's
+    // device-scope fence and ticket increment; the last CTA's thread 0
+    // fences again (acquire) before the barrier that lets the CTA read
     __syncthreads();
-    if (tid == 0) s_last = (atomicAdd(a.hdr + WS_TICKET, 1) == (int)gridDim.x - 1);
+    if (tid == 0) {
+        if (bad) atomicOr(a.hdr + WS_STATUS, MOONEP_ST_EXPERT_ID_RANGE);
+        __threadfence();
+        const bool last = atomicAdd(a.hdr + WS_TICKET, 1) == (int)gridDim.x - 1;
+        if (last) __threadfence();
+        s_last = last;
+    }
     __syncthreads();
     if (!s_last) return;
-    __threadfence();
     plan_block(a, sm, parity);
 }
 

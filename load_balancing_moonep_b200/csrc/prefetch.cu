@@ -1,0 +1,121 @@
+// Replica weight prefetch (sm_100a).
+//
+// MoonEP article ("Moonshot AI Open-Sources MoonEP: A Perfectly Balanced
+// Expert Parallelism Library for MoE Training"), "The core idea": duplicated
+// experts are prefetched before expert computation; explainer, memory tab:
+// the prefetch slots are rows [E, E+B) of one contiguous weight pool per
+// projection, and a rank needing more than B foreign experts reads the
+// overflow from the home copy.  Here each rank's B prefetch rows form
+// pool[r][0..B), the home experts stay in `weights`, and a per-slot table
+// tells the expert computation which row to use.
+//
+// The copy is an HBM stream of 16-byte vectors over work items (prefetched
+// replica, element chunk) taken from the plan on the device, so the launch
+// needs no host synchronisation.
+#include "common.cuh"
+
+namespace moonep {
+
+constexpr int PF_THREADS = 256;
+constexpr int PF_UNROLL = 4;
+
+struct PrefetchParams {
+    const int *slot_expert, *rep_expert, *rep_rank, *rep_slot, *info;
+    const uint8_t *weights;
+    uint8_t *pool;
+    int *slot_wrow;
+    int R, E, L, B;
+    long long row_bytes;  // P * 2
+    long long chunk;      // bytes per work item
+};
+
+template <typename V>
+__global__ void __launch_bounds__(PF_THREADS) prefetch_kernel(PrefetchParams a)
+{
+    const int status = __ldg(a.info + MOONEP_INFO_STATUS);
+    const bool invalid = (status & MOONEP_ST_EXPERT_ID_RANGE) != 0;
+    const long long gtid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long gstride = (long long)gridDim.x * blockDim.x;
+
+    // weight row of every slot: home e, pool E + r*B + b, overflow e (read-through)
+    for (long long x = gtid; x < (long long)a.R * a.E; x += gstride) {
+        const int r = (int)(x / a.E), s = (int)(x - (long long)r * a.E);
+        const int e = invalid ? -1 : __ldg(a.slot_expert + x);
+        int row = -1;
+        if (e >= 0) row = (s < a.L) ? e : (s - a.L < a.B ? a.E + r * a.B + (s - a.L) : e);
+        a.slot_wrow[x] = row;
+    }
+    if (invalid) return;
+
+    const int n_rep = min(max(__ldg(a.info + MOONEP_INFO_N_REP), 0), a.E + a.R);
+    constexpr int W = sizeof(V);
+    const long long vrow = a.row_bytes / W;
+    const long long vchunk = a.chunk / W;
+    const long long nchunks = (vrow + vchunk - 1) / vchunk;
+    const long long n_items = (long long)n_rep * nchunks;
+    for (long long item = blockIdx.x; item < n_items; item += gridDim.x) {
+        const int q = (int)(item / nchunks);
+        const long long ci = item - (long long)q * nchunks;
+        const int b = __ldg(a.rep_slot + q) - a.L;
+        if (b < 0 || b >= a.B) continue;  // overflow: not prefetched
+        const int r = __ldg(a.rep_rank + q), e = __ldg(a.rep_expert + q);
+        if (r < 0 || r >= a.R || e < 0 || e >= a.E) continue;
+        const V *src = reinterpret_cast<const V *>(a.weights + (long long)e * a.row_bytes);
+        V *dst = reinterpret_cast<V *>(a.pool + ((long long)r * a.B + b) * a.row_bytes);
+        const long long v0 = ci * vchunk, v1 = min(vrow, v0 + vchunk);
+        for (long long v = v0 + threadIdx.x; v < v1; v += (long long)PF_THREADS * PF_UNROLL) {
+            V t[PF_UNROLL];
+#pragma unroll
+            for (int u = 0; u < PF_UNROLL; ++u) {
+                const long long x = v + (long long)u * PF_THREADS;
+                if (x < v1) t[u] = src[x];
+            }
+#pragma unroll
+            for (int u = 0; u < PF_UNROLL; ++u) {
+                const long long x = v + (long long)u * PF_THREADS;
+                if (x < v1) dst[x] = t[u];
+            }
+        }
+    }
+}
+
+int launch_prefetch(const Dims &d, const moonep_plan_t &p, const uint16_t *weights, uint16_t *pool,
+                    int32_t *slot_wrow, long long P, cudaStream_t st)
+{
+    static int sms[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    if (!sms[dev]) {
+        int v = 0;
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+        sms[dev] = v > 0 ? v : 148;
+    }
+    PrefetchParams a;
+    a.slot_expert = p.slot_expert;
+    a.rep_expert = p.rep_expert;
+    a.rep_rank = p.rep_rank;
+    a.rep_slot = p.rep_slot;
+    a.info = p.info;
+    a.weights = reinterpret_cast<const uint8_t *>(weights);
+    a.pool = reinterpret_cast<uint8_t *>(pool);
+    a.slot_wrow = slot_wrow;
+    a.R = d.R;
+    a.E = d.E;
+    a.L = d.L;
+    a.B = d.B;
+    a.row_bytes = P * 2;
+    const bool vec = (a.row_bytes % 16 == 0) && (reinterpret_cast<uintptr_t>(weights) % 16 == 0) &&
+                     (reinterpret_cast<uintptr_t>(pool) % 16 == 0);
+    const int grid = sms[dev] * (2048 / PF_THREADS);
+    if (vec) {
+        a.chunk = 256 * 1024;
+        prefetch_kernel<uint4><<<grid, PF_THREADS, 0, st>>>(a);
+    } else {
+        a.chunk = 64 * 1024;
+        prefetch_kernel<uint16_t><<<grid, PF_THREADS, 0, st>>>(a);
+    }
+    return cudaGetLastError() == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
+}
+
+}  // namespace moonep

@@ -50,7 +50,7 @@ PLAN_FIELDS = ("expert_count", "slot_expert", "slot_count", "slot_offset", "rep_
 EXPORTED = ("moonep_check_config", "moonep_plan_sizes", "moonep_plan_layout", "moonep_plan",
             "moonep_dispatch", "moonep_combine", "moonep_combine_backward",
             "moonep_reduce_replica_grads", "moonep_error_string", "moonep_abi_version",
-            "moonep_plan_noalloc")
+            "moonep_plan_noalloc", "moonep_prefetch_replicas")
 
 
 class _CConfig(ctypes.Structure):
@@ -75,6 +75,7 @@ _lib.moonep_combine.argtypes = [_cfgp, _planp, _vp, _vp, _vp, _vp]
 _lib.moonep_combine_backward.argtypes = [_cfgp, _planp, _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.moonep_reduce_replica_grads.argtypes = [_cfgp, _planp, _vp, _vp, ctypes.c_int64, _vp]
 _lib.moonep_plan_noalloc.argtypes = [_cfgp, _vp, _planp, _vp]
+_lib.moonep_prefetch_replicas.argtypes = [_cfgp, _planp, _vp, _vp, _vp, ctypes.c_int64, _vp]
 _lib.moonep_error_string.argtypes = [ctypes.c_int]
 _lib.moonep_error_string.restype = ctypes.c_char_p
 _lib.moonep_abi_version.argtypes = []
@@ -292,6 +293,24 @@ def reduce_replica_grads(cfg: Config, p: Plan, reduce_buf: torch.Tensor, home_gr
                                             reduce_buf.data_ptr() if reduce_buf.numel() else None,
                                             home_grad.data_ptr(), P, _stream(stream)))
     return home_grad
+
+
+def prefetch_replicas(cfg: Config, p: Plan, weights: torch.Tensor, pool: torch.Tensor,
+                      slot_wrow: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Copy each prefetched replica's expert weights (bf16 [E, P]) into its
+    rank's pool slot (bf16 [R, B, P]) and return the per-slot weight-row
+    table (int32 [R, E]: home e, pool E + r*B + b, overflow e, unused -1)."""
+    P = weights.shape[-1]
+    _need(weights, torch.bfloat16, (cfg.E, P), "weights")
+    _need(pool, torch.bfloat16, (cfg.R, cfg.B, P), "pool")
+    if slot_wrow is None:
+        slot_wrow = torch.empty((cfg.R, cfg.E), dtype=torch.int32, device=weights.device)
+    _need(slot_wrow, torch.int32, (cfg.R, cfg.E), "slot_wrow")
+    c = cfg.c()
+    _check(_lib.moonep_prefetch_replicas(ctypes.byref(c), ctypes.byref(p.c_plan), weights.data_ptr(),
+                                         pool.data_ptr() if pool.numel() else None, slot_wrow.data_ptr(),
+                                         P, _stream(stream)))
+    return slot_wrow
 
 
 def views(cfg: Config, p: Plan, buf: torch.Tensor):

@@ -76,6 +76,8 @@ def _load():
         lib.or_combine_backward.restype = ctypes.c_int
         lib.or_reduce_replica_grads.argtypes = [ctypes.c_void_p] * 7 + [ctypes.c_int64] * 3
         lib.or_reduce_replica_grads.restype = ctypes.c_int
+        lib.or_prefetch_replicas.argtypes = [ctypes.c_void_p] * 6 + [ctypes.c_int64] * 3
+        lib.or_prefetch_replicas.restype = ctypes.c_int
         lib.or_f32_to_bf16.argtypes = [ctypes.c_float]
         lib.or_f32_to_bf16.restype = ctypes.c_uint16
         _lib = lib
@@ -231,3 +233,21 @@ def reduce_replica_grads(cfg: Config, p: dict, reduce_buf: np.ndarray, home_grad
                                        _p(p["host_slot"]), _p(p["info"]), _p(reduce_buf),
                                        _p(home_grad), P, i0, i1))
     return reduce_buf, home_grad
+
+
+def prefetch_replicas(cfg: Config, p: dict, weights_bits: np.ndarray, pool_bits: np.ndarray,
+                      P: int, i0: int = 0, i1: int | None = None) -> np.ndarray:
+    """Copy each prefetched replica's expert weights into its rank's pool
+    slot (MoonEP article explainer, memory tab: duplicated experts are
+    prefetched into rows [E, E+B) of the weight pool).  weights_bits: uint16
+    [E, P]; pool_bits: uint16 [R, B, P] (written in place).  Returns the
+    per-slot weight-row table [R, E] (home e, pool E + r*B + b, overflow e,
+    unused -1)."""
+    lib = _load()
+    i1 = P if i1 is None else i1
+    assert weights_bits.dtype == np.uint16 and pool_bits.dtype == np.uint16
+    wrow = np.zeros((cfg.R, cfg.E), np.int32)
+    c = cfg._c()
+    _check(lib.or_prefetch_replicas(ctypes.byref(c), _p(p["slot_expert"]), _p(p["info"]),
+                                    _p(weights_bits), _p(pool_bits), _p(wrow), P, i0, i1))
+    return wrow

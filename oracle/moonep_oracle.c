@@ -470,3 +470,41 @@ int or_reduce_replica_grads(const or_config *c, const int32_t *host_ptr,
         }
     return OR_OK;
 }
+
+/* Replica weight prefetch [P1 explainer, memory tab]: duplicated experts are
+ * copied before expert compute into the rank's prefetch slots, rows [L, L+B)
+ * of its [L+B, ...] weight pool (the page's [E, E+B) with E read as the
+ * rank's L home experts).  pool[r][b][:] = weights[e][:] for every replica
+ * of expert e on rank r with ordinal b = slot - L < B; overflow replicas are
+ * not copied -- they read the home copy (inference read-through).
+ * slot_wrow[r][s] names the weight row each used slot computes with, in the
+ * concatenated row space [weights (E rows) | pool (R*B rows)]:
+ *   home slot -> e;  prefetched replica -> E + r*B + b;  overflow -> e;
+ * unused slots -> -1.  Elements [i0, i1) of each row are copied. */
+int or_prefetch_replicas(const or_config *c, const int32_t *slot_expert, const int32_t *info,
+                         const uint16_t *weights, uint16_t *pool, int32_t *slot_wrow,
+                         int64_t P, int64_t i0, int64_t i1)
+{
+    const int32_t R = c->R, E = c->E, L = c->E / c->R, B = c->B;
+    const int invalid = (info[OR_INFO_STATUS] & OR_ST_EXPERT_ID_RANGE) != 0;
+    for (int32_t r = 0; r < R; ++r)
+        for (int32_t s = 0; s < E; ++s) {
+            int32_t e = invalid ? -1 : slot_expert[(int64_t)r * E + s];
+            int32_t row = -1;
+            if (e >= 0) {
+                if (s < L) {
+                    row = e;
+                } else if (s - L < B) {
+                    int32_t b = s - L;
+                    row = E + r * B + b;
+                    uint16_t *dst = pool + ((int64_t)r * B + b) * P;
+                    const uint16_t *src = weights + (int64_t)e * P;
+                    for (int64_t i = i0; i < i1; ++i) dst[i] = src[i];
+                } else {
+                    row = e; /* overflow: read through to the home copy */
+                }
+            }
+            slot_wrow[(int64_t)r * E + s] = row;
+        }
+    return OR_OK;
+}

@@ -341,3 +341,40 @@ def test_reduce_full_size_sampled(mp):
         assert np.array_equal(rb[:, :, a:b].cpu().numpy(), orb)
     del rb, hg
     torch.cuda.empty_cache()
+
+
+# -------------------------------------------------------------- prefetch
+
+@pytest.mark.parametrize("wname,mv,P", [("tiny", 1.0, 1000), ("tiny", 3.0, 1003), ("mid", 3.0, 4096),
+                                        ("large", 3.0, 2048), ("decode", 13.4, 517)])
+def test_prefetch(mp, wname, mv, P):
+    wl = W.WORKLOADS[wname]
+    r = W.routing(wl, mv, device=DEV)
+    topk = r.topk_idx.cpu().numpy()
+    gcfg, ocfg, gp, op = _plan_both(mp, _wl_cfg(wl), topk)
+    weights = W.bf16_normal((wl.E, P), seed=6, device=DEV)
+    pool = torch.full((wl.R, wl.B, P), float("nan"), dtype=torch.bfloat16, device=DEV)
+    opool = W.bits(pool).copy()
+    wrow = mp.prefetch_replicas(gcfg, gp, weights, pool)
+    owrow = oracle.prefetch_replicas(ocfg, op, W.bits(weights), opool, P)
+    assert np.array_equal(wrow.cpu().numpy(), owrow)
+    assert np.array_equal(W.bits(pool), opool)
+
+
+def test_prefetch_bad_ids_and_no_budget(mp):
+    c = dict(R=4, E=16, K=2, S=64, H=64, B=2)
+    rng = np.random.default_rng(2)
+    topk = rng.integers(0, 16, size=(256, 2)).astype(np.int32)
+    topk[5, 0] = -3
+    gcfg, ocfg, gp, op = _plan_both(mp, c, topk)
+    weights = W.bf16_normal((16, 64), seed=6, device=DEV)
+    pool = torch.full((4, 2, 64), 3.0, dtype=torch.bfloat16, device=DEV)
+    wrow = mp.prefetch_replicas(gcfg, gp, weights, pool)
+    assert (wrow.cpu() == -1).all() and (pool == 3.0).all()
+    # B = 0: every replica is overflow and reads its home row
+    c0 = dict(R=4, E=16, K=2, S=64, H=64, B=0)
+    topk[5, 0] = 1
+    gcfg, ocfg, gp, op = _plan_both(mp, c0, topk)
+    wrow = mp.prefetch_replicas(gcfg, gp, weights, torch.empty((4, 0, 64), dtype=torch.bfloat16, device=DEV))
+    owrow = oracle.prefetch_replicas(ocfg, op, W.bits(weights), np.zeros((4, 0, 64), np.uint16), 64)
+    assert np.array_equal(wrow.cpu().numpy(), owrow)

@@ -428,3 +428,24 @@ def test_combine_uses_fused_multiply_add(oracle_lib):
     out = oracle.combine(cfg, p, y, w)
     ref = torch.tensor([exact], dtype=torch.float64).to(torch.bfloat16).view(torch.int16)
     assert (out == np.uint16(ref.numpy().view(np.uint16)[0])).all()
+
+
+def test_prefetch_hand_worked(oracle_lib):
+    # Example B with B = 2: replicas (e6, r0, slot 2), (e6, r1, slot 2),
+    # (e4, r1, slot 3) are prefetched into pool rows b = slot - L = 0, 0, 1;
+    # (e7, r1, slot 4) has ordinal 2 >= B and reads its home row 7.  Row space
+    # [weights (8 rows) | pool (R*B = 8 rows)]: pool row of (r, b) = 8 + 2r + b.
+    g = json.load(open(os.path.join(GOLDEN, "plan_example_b.json")))
+    cfg = oracle.Config(**{**g["config"], "B": 2})
+    p = oracle.plan(cfg, np.array(g["topk_idx"], np.int32))
+    P = 5
+    w = np.arange(cfg.E * P, dtype=np.uint16).reshape(cfg.E, P)
+    pool = np.full((cfg.R, cfg.B, P), 0xFFFF, np.uint16)
+    wrow = oracle.prefetch_replicas(cfg, p, w, pool, P)
+    assert wrow.tolist() == [[0, 1, 8, -1, -1, -1, -1, -1],
+                             [2, 3, 10, 11, 7, -1, -1, -1],
+                             [4, 5, -1, -1, -1, -1, -1, -1],
+                             [6, 7, -1, -1, -1, -1, -1, -1]]
+    assert np.array_equal(pool[0, 0], w[6]) and np.array_equal(pool[1, 0], w[6])
+    assert np.array_equal(pool[1, 1], w[4])
+    assert (pool[0, 1] == 0xFFFF).all() and (pool[2:] == 0xFFFF).all()

@@ -518,6 +518,99 @@ def run_ours(args, world, rank, local):
                         "out, every step; double-buffered, copies of neighbouring steps overlap")}
         del d_topk, d_w, d_hidden, d_out
 
+    # the pages' own sweep shape: EP=8, maxvio 0.2, 1, 10, 20
+    pages_sweep = []
+    if not args.no_sweep:
+        ewl = W.WORKLOADS["ep8"]
+        ecfg = mp.Config(R=ewl.R, E=ewl.E, K=ewl.K, S=ewl.S, H=ewl.H, B=ewl.B)
+        eh = W.hidden_states(ewl, seed=12 + rank, device=dev)
+        ebuf = torch.empty((ewl.R, ewl.C, ewl.H), dtype=torch.bfloat16, device=dev)
+        eout = torch.empty((ewl.tokens, ewl.H), dtype=torch.bfloat16, device=dev)
+        for mv in ewl.sweep:
+            er = W.routing(ewl, mv, seed=rank, device=dev)
+            ep = mp.Plan(ecfg, dev)
+            for _ in range(3):
+                mp.plan(ecfg, er.topk_idx, out=ep)
+                mp.dispatch(ecfg, ep, eh, ebuf)
+                mp.combine(ecfg, ep, ebuf, er.weights, eout)
+            torch.cuda.synchronize()
+            st = Timer()
+            for _ in range(args.sweep_iters):
+                e = st.mark("plan"); mp.plan(ecfg, er.topk_idx, out=ep); e.record()
+                e = st.mark("dispatch"); mp.dispatch(ecfg, ep, eh, ebuf); e.record()
+                e = st.mark("combine"); mp.combine(ecfg, ep, ebuf, er.weights, eout); e.record()
+            torch.cuda.synchronize()
+            it = args.sweep_iters
+            pd, pc, pp = st.total_ms("dispatch") / it, st.total_ms("combine") / it, st.total_ms("plan") / it
+            inf = ep.info()
+            gd = bytes_dispatch(ewl) / (pd * 1e-3) / 1e9
+            gc = bytes_combine(ewl) / (pc * 1e-3) / 1e9
+            pages_sweep.append({"maxvio": round(er.maxvio, 3), "dispatch_GB/s": round(gd, 1),
+                                "combine_GB/s": round(gc, 1), "dispatch_frac": round(gd / peak, 4),
+                                "combine_frac": round(gc / peak, 4), "planner_us": round(pp * 1e3, 2),
+                                "n_rep": inf["n_rep"], "n_overflow": inf["n_overflow"],
+                                "max_rep_per_rank": inf["max_rep_per_rank"],
+                                "hottest_expert_pairs": W.hottest_expert_count(er.maxvio, ewl.S, ewl.K, ewl.R, ewl.E)})
+            del ep
+        del eh, ebuf, eout
+
+    # decode shape (latency-bound): plan + dispatch + combine of one MoE layer
+    # replayed from a CUDA graph, next to the eager per-kernel times
+    decode = None
+    if not args.no_decode:
+        dwl = W.WORKLOADS["decode"]
+        dcfg = mp.Config(R=dwl.R, E=dwl.E, K=dwl.K, S=dwl.S, H=dwl.H, B=dwl.B)
+        dr = W.routing(dwl, dwl.maxvio, seed=rank, device=dev)
+        dh = W.hidden_states(dwl, seed=11 + rank, device=dev)
+        dbuf = torch.empty((dwl.R, dwl.C, dwl.H), dtype=torch.bfloat16, device=dev)
+        dout = torch.empty((dwl.tokens, dwl.H), dtype=torch.bfloat16, device=dev)
+        dplan = mp.Plan(dcfg, dev)
+        gs_ = torch.cuda.Stream()
+        with torch.cuda.stream(gs_):
+            for _ in range(3):
+                mp.plan(dcfg, dr.topk_idx, out=dplan)
+                mp.dispatch(dcfg, dplan, dh, dbuf)
+                mp.combine(dcfg, dplan, dbuf, dr.weights, dout)
+        torch.cuda.synchronize()
+        et = Timer()
+        for _ in range(20):
+            e = et.mark("plan"); mp.plan(dcfg, dr.topk_idx, out=dplan); e.record()
+            e = et.mark("dispatch"); mp.dispatch(dcfg, dplan, dh, dbuf); e.record()
+            e = et.mark("combine"); mp.combine(dcfg, dplan, dbuf, dr.weights, dout); e.record()
+        torch.cuda.synchronize()
+        layer_us, graph_err = None, None
+        try:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=gs_, capture_error_mode="thread_local"):
+                mp.plan(dcfg, dr.topk_idx, out=dplan)
+                mp.dispatch(dcfg, dplan, dh, dbuf)
+                mp.combine(dcfg, dplan, dbuf, dr.weights, dout)
+            for _ in range(5):
+                graph.replay()
+            torch.cuda.synchronize()
+            g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            g0.record()
+            for _ in range(50):
+                graph.replay()
+            g1.record()
+            torch.cuda.synchronize()
+            layer_us = g0.elapsed_time(g1) / 50 * 1e3
+            del graph
+        except RuntimeError as exc:  # report eager numbers if capture is refused
+            graph_err = str(exc)[:200]
+            torch.cuda.synchronize()
+        if layer_us is None:
+            layer_us = sum(et.total_ms(n) for n in ("plan", "dispatch", "combine")) / 20 * 1e3
+        dinfo = dplan.info()
+        db = bytes_dispatch(dwl) + bytes_combine(dwl)
+        decode = {"workload": f"decode: R={dwl.R} E={dwl.E} K={dwl.K} S={dwl.S} H={dwl.H} B={dwl.B}, one hot expert",
+                  "maxvio": round(dr.maxvio, 3), "graph_layer_us": round(layer_us, 2),
+                  "eager_us": {n: round(et.total_ms(n) / 20 * 1e3, 2) for n in ("plan", "dispatch", "combine")},
+                  "dispatch+combine_GB/s_in_graph": round(db / (layer_us * 1e-6) / 1e9, 1),
+                  "n_rep": dinfo["n_rep"], "n_overflow": dinfo["n_overflow"],
+                  "max_rep_per_rank": dinfo["max_rep_per_rank"], "graph_error": graph_err}
+        del dbuf, dout, dh, dplan
+
     # replica weight prefetch (a next-row step, timed on its own after the
     # step: its 68 GB of weights and pool fit once the reduce buffers are freed)
     if P and not args.no_prefetch:
@@ -571,6 +664,9 @@ def run_ours(args, world, rank, local):
         "planner_us": kernels["plan"]["us"],
         "roofline": roofline, "kernels": kernels, "sweep": sweep,
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
+        "decode": decode,
+        "pages_sweep": {"workload": "ep8: R=8 E=256 K=8 S=4096 H=7168 B=4 (EP=8 as in the pages' sweep)",
+                        "points": pages_sweep},
         "clocks": clocks, "plan_info": info,
     }
     if rank == 0:
@@ -628,6 +724,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefetch", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--profile", action="store_true",
                     help="run two untimed steps of a reduced-size case (for ncu)")
     ap.add_argument("--profile-S", type=int, default=512)

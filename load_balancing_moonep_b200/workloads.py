@@ -89,6 +89,10 @@ WORKLOADS = {
     # Large training shape; the backward config shares its routing.
     "large": Workload("large", R=32, E=384, K=8, S=4096, H=7168, B=12, zipf_s=1.0, maxvio=1.0,
                       sweep=(0.0, 0.5, 1.0, 2.0, 3.0), H_ffn=2048),
+    # The pages' own sweep: EP=8 at maxvio 0.2, 1, 10, 20 (expert count not
+    # stated there; 256 experts, top-8 makes maxvio 20 reachable).
+    "ep8": Workload("ep8", R=8, E=256, K=8, S=4096, H=7168, B=4, zipf_s=1.0, maxvio=1.0,
+                    sweep=(0.2, 1.0, 10.0, 20.0)),
     # Decode: one hot expert, extreme skew, latency bound.
     "decode": Workload("decode", R=64, E=384, K=8, S=128, H=7168, B=4, kind="hot", maxvio=5.0,
                        sweep=(5.0, 10.0, 13.4, 20.0)),

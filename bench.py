@@ -471,6 +471,7 @@ def run_ours(args, world, rank, local):
         ev_used = [torch.cuda.Event() for _ in range(nb)]   # inputs consumed
         ev_done = [torch.cuda.Event() for _ in range(nb)]   # output written
         ev_read = [torch.cuda.Event() for _ in range(nb)]   # output copied out
+        torch.cuda.synchronize()  # inputs, plan and buffers ready before the side streams start
         for b in range(nb):
             for ev in (ev_used[b], ev_read[b]):
                 ev.record(s_cmp)
@@ -565,12 +566,14 @@ def run_ours(args, world, rank, local):
         dbuf = torch.empty((dwl.R, dwl.C, dwl.H), dtype=torch.bfloat16, device=dev)
         dout = torch.empty((dwl.tokens, dwl.H), dtype=torch.bfloat16, device=dev)
         dplan = mp.Plan(dcfg, dev)
+        # the plan block and its zero-filled workspace were made on the
+        # default stream: finish that before another stream uses them
+        torch.cuda.synchronize()
         gs_ = torch.cuda.Stream()
-        with torch.cuda.stream(gs_):
-            for _ in range(3):
-                mp.plan(dcfg, dr.topk_idx, out=dplan)
-                mp.dispatch(dcfg, dplan, dh, dbuf)
-                mp.combine(dcfg, dplan, dbuf, dr.weights, dout)
+        for _ in range(3):
+            mp.plan(dcfg, dr.topk_idx, out=dplan)
+            mp.dispatch(dcfg, dplan, dh, dbuf)
+            mp.combine(dcfg, dplan, dbuf, dr.weights, dout)
         torch.cuda.synchronize()
         et = Timer()
         for _ in range(20):

@@ -82,7 +82,8 @@ extern "C" {
 
 /* ---- device status bits (plan->info[MOONEP_INFO_STATUS]) -------------- */
 /* An id outside [0, E): the plan is empty, dst_pos/row_src are -1, and
- * dispatch / combine / combine_backward / reduce become no-ops. */
+ * dispatch / combine / combine_backward / reduce / prefetch become no-ops.
+ * (MOONEP_ST_WORKSPACE below empties the plan the same way.) */
 #define MOONEP_ST_EXPERT_ID_RANGE 1
 /* Some rank holds more than B replicas; the extra ones (ordinal >= B) are
  * still planned, so every rank still gets exactly S*K slots, but they have
@@ -95,6 +96,11 @@ extern "C" {
 /* A bounded wait inside a kernel (an mbarrier for a bulk copy) ran out of
  * iterations; the kernel stopped early and its output is incomplete. */
 #define MOONEP_ST_WAIT_TIMEOUT 16
+/* The planner workspace did not hold the zeros a call must start from (it
+ * was not zero-filled before first use, or two calls used it at once): the
+ * expert totals do not add up to R*S*K.  The plan is then empty, exactly as
+ * for MOONEP_ST_EXPERT_ID_RANGE; zero-fill the workspace and plan again. */
+#define MOONEP_ST_WORKSPACE 32
 
 /* ---- plan->info[] fields (int32, device) ------------------------------ */
 #define MOONEP_INFO_STATUS 0

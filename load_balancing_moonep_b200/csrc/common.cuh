@@ -42,6 +42,9 @@ struct WsLayout {
 };
 enum { WS_TICKET = 0, WS_STATUS = 1, WS_PARITY = 2 };
 
+// Status bits after which every later call treats the plan as empty.
+constexpr int ST_EMPTY_PLAN = MOONEP_ST_EXPERT_ID_RANGE | MOONEP_ST_WORKSPACE;
+
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 __host__ inline WsLayout ws_layout(const Dims &d)

@@ -68,7 +68,7 @@ __device__ __forceinline__ uint4 pack8(const float f[8])
 
 __device__ __forceinline__ bool plan_invalid(const int *info)
 {
-    return (*(volatile const int *)(info + MOONEP_INFO_STATUS) & MOONEP_ST_EXPERT_ID_RANGE) != 0;
+    return (*(volatile const int *)(info + MOONEP_INFO_STATUS) & ST_EMPTY_PLAN) != 0;
 }
 
 // A row index from the plan outside [0, rows) is never dereferenced: the

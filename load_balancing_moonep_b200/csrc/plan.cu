@@ -125,13 +125,22 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
     int *wsum = flag + E;          // 32
     int *misc = wsum + 32;         // 16: 0 status in, 2 n_over, 3 max replicas per rank
 
+    __shared__ unsigned long long s_total;
+    __shared__ int s_negative;
     for (int i = tid; i < 16; i += nt) misc[i] = 0;
+    if (tid == 0) {
+        s_total = 0;
+        s_negative = 0;
+    }
+    __syncthreads();
     // ---- totals; leave the accumulators zeroed for the next call
     for (int e = tid; e < E; e += nt) {
         const int v = ld_cg(a.t_acc + e);
         T[e] = v;
         a.t_acc[e] = 0;
         a.p.expert_count[e] = v;
+        if (v < 0) s_negative = 1;
+        else atomicAdd(&s_total, (unsigned long long)v);
     }
     // the previous call's group buffer is no longer read: zero it
     {
@@ -146,8 +155,12 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
         a.hdr[WS_PARITY] = parity ^ 1;  // the next call accumulates into the other buffer
     }
     __syncthreads();
-    const int status_in = misc[0];
-    if (status_in & MOONEP_ST_EXPERT_ID_RANGE) {
+    int status_in = misc[0];
+    // with every id valid the totals must be non-negative and add up to the
+    // number of pairs; anything else means the workspace was not zeroed
+    if (!(status_in & MOONEP_ST_EXPERT_ID_RANGE) && (s_negative || s_total != (unsigned long long)d.pairs))
+        status_in |= MOONEP_ST_WORKSPACE;
+    if (status_in & ST_EMPTY_PLAN) {
         if (tid == 0) {
             a.p.info[MOONEP_INFO_STATUS] = status_in;
             for (int i = 1; i < MOONEP_INFO_LEN; ++i) a.p.info[i] = 0;
@@ -484,8 +497,10 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
     pdl_wait();  // the histogram/planner grid has completed; its writes are visible
 
     const int status = ld_cg(a.p.info + MOONEP_INFO_STATUS);
-    const bool empty = (status & MOONEP_ST_EXPERT_ID_RANGE) != 0;
-    const int n_rep = empty ? 0 : ld_cg(a.p.info + MOONEP_INFO_N_REP);
+    const bool empty = (status & ST_EMPTY_PLAN) != 0;
+    // every count and index read back from the plan is clamped, so even a
+    // plan block of garbage cannot steer an access out of its array
+    const int n_rep = empty ? 0 : min(max(ld_cg(a.p.info + MOONEP_INFO_N_REP), 0), E + R - 1);
 
     // ---- padded tables from the compact slot lists, spread over the CTAs
     {
@@ -494,7 +509,8 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
             const int r = (int)(x / E), s = (int)(x - (long long)r * E);
             int ex = -1, ct = 0;
             if (!empty) {
-                const int b0 = ld_cg(a.sc_base + r), b1 = ld_cg(a.sc_base + r + 1);
+                const int b0 = min(max(ld_cg(a.sc_base + r), 0), nh);
+                const int b1 = min(max(ld_cg(a.sc_base + r + 1), b0), nh);
                 if (s < b1 - b0) {
                     ex = ld_cg(a.sc_exp + b0 + s);
                     ct = ld_cg(a.sc_cnt + b0 + s);
@@ -507,7 +523,8 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
             const int r = (int)(x / (E + 1)), s = (int)(x - (long long)r * (E + 1));
             int v = 0;
             if (!empty) {
-                const int b0 = ld_cg(a.sc_base + r), b1 = ld_cg(a.sc_base + r + 1);
+                const int b0 = min(max(ld_cg(a.sc_base + r), 0), nh);
+                const int b1 = min(max(ld_cg(a.sc_base + r + 1), b0), nh);
                 v = s < b1 - b0 ? ld_cg(a.sc_off + b0 + s) : C;
             }
             a.p.slot_offset[x] = v;
@@ -541,7 +558,7 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
         return;
     }
 
-    for (int e = tid; e <= E; e += nt) hptr[e] = ld_cg(a.p.host_ptr + e);
+    for (int e = tid; e <= E; e += nt) hptr[e] = min(max(ld_cg(a.p.host_ptr + e), 0), E + n_rep);
     for (int h = tid; h < E + n_rep; h += nt) {
         hstart[h] = ld_cg(a.p.host_start + h);
         hdst[h] = ld_cg(a.host_dst0 + h);

@@ -33,7 +33,7 @@ template <typename V>
 __global__ void __launch_bounds__(PF_THREADS) prefetch_kernel(PrefetchParams a)
 {
     const int status = __ldg(a.info + MOONEP_INFO_STATUS);
-    const bool invalid = (status & MOONEP_ST_EXPERT_ID_RANGE) != 0;
+    const bool invalid = (status & ST_EMPTY_PLAN) != 0;
     const long long gtid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     const long long gstride = (long long)gridDim.x * blockDim.x;
 

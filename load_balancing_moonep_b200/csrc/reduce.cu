@@ -58,7 +58,7 @@ __global__ void __launch_bounds__(REDUCE_THREADS) reduce_kernel(ReduceParams a)
     __shared__ int s_row[REDUCE_MAX_LIST];
     __shared__ int s_wsum[32];
     const int status = __ldg(a.info + MOONEP_INFO_STATUS);
-    if (status & MOONEP_ST_EXPERT_ID_RANGE) return;
+    if (status & ST_EMPTY_PLAN) return;
     const int n_exp = min(max(__ldg(a.info + MOONEP_INFO_N_REP_EXPERTS), 0), a.E);
     if (n_exp == 0) return;
     const int tid = threadIdx.x;

@@ -38,6 +38,8 @@ ST_EXPERT_ID_RANGE = 1
 ST_OVERFLOW = 2
 ST_STRICT_VIOLATION = 4
 ST_ROW_RANGE = 8
+ST_WAIT_TIMEOUT = 16
+ST_WORKSPACE = 32
 
 INFO_FIELDS = ("status", "n_rep", "n_overflow", "n_pieces", "n_receivers",
                "max_rep_per_rank", "n_rep_experts", "n_remote_pairs")

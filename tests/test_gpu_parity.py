@@ -378,3 +378,32 @@ def test_prefetch_bad_ids_and_no_budget(mp):
     wrow = mp.prefetch_replicas(gcfg, gp, weights, torch.empty((4, 0, 64), dtype=torch.bfloat16, device=DEV))
     owrow = oracle.prefetch_replicas(ocfg, op, W.bits(weights), np.zeros((4, 0, 64), np.uint16), 64)
     assert np.array_equal(wrow.cpu().numpy(), owrow)
+
+
+def test_workspace_not_zeroed_is_detected(mp):
+    # The workspace must start zero-filled; if its expert totals hold
+    # garbage, the planner reports MOONEP_ST_WORKSPACE and an empty plan
+    # (white-box: the totals follow the 256-byte header of the workspace).
+    wl = W.WORKLOADS["tiny"]
+    c = _wl_cfg(wl)
+    cfg = mp.Config(**c)
+    topk = W.routing(wl, 1.0, device=DEV).topk_idx
+    p = mp.Plan(cfg)
+    torch.cuda.synchronize()
+    p.workspace[256:256 + 4 * wl.E] = 0x7F
+    torch.cuda.synchronize()
+    mp.plan(cfg, topk, out=p)
+    info = p.info()
+    assert info["status"] & mp.ST_WORKSPACE
+    f = p.to_numpy()
+    assert (f["dst_pos"] == -1).all() and (f["slot_count"] == 0).all() and info["n_rep"] == 0
+    # dispatch is a no-op on an empty plan
+    hidden = W.hidden_states(wl, seed=1, device=DEV)
+    buf = torch.full((wl.R, wl.C, wl.H), 2.0, dtype=torch.bfloat16, device=DEV)
+    mp.dispatch(cfg, p, hidden, buf)
+    torch.cuda.synchronize()
+    assert (buf == 2.0).all()
+    # zero-filled again, the same workspace plans exactly as the oracle
+    p.workspace.zero_()
+    mp.plan(cfg, topk, out=p)
+    _assert_plan_equal(p, oracle.plan(oracle.Config(**c), topk.cpu().numpy()))

@@ -649,10 +649,16 @@ def run_ours(args, world, rank, local):
         tokens = sample_tokens(wl, args.ref_tokens)
         hid = W.bits(hidden[: len(tokens)])
         y = W.bits(W.bf16_normal((len(tokens) * wl.K, wl.H), seed=2, device="cpu"))
-        ps_, ds_, db_ = oracle_sample(wl, topk_np, w_np, hid, tokens, y)
-        cpu = {"value": round(db_ / ds_ / 1e9, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": (f"dispatch+combine of the first {len(tokens)} of {wl.tokens} tokens "
-                          f"({ds_:.1f} s); plan over all {wl.pairs} pairs took {ps_ * 1e3:.0f} ms; "
+        # repeat the bounded sample until about 10 s of CPU work
+        reps, ds_tot, db_tot, ps_ = 0, 0.0, 0.0, 0.0
+        while ds_tot < 10.0 and reps < 50:
+            ps_, ds_, db_ = oracle_sample(wl, topk_np, w_np, hid, tokens, y)
+            ds_tot += ds_
+            db_tot += db_
+            reps += 1
+        cpu = {"value": round(db_tot / ds_tot / 1e9, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": (f"{reps} x dispatch+combine of the first {len(tokens)} of {wl.tokens} tokens "
+                          f"({ds_tot:.1f} s); plan over all {wl.pairs} pairs took {ps_ * 1e3:.0f} ms; "
                           "single-threaded C")}
 
     launches_per_step = 2 + 1 + 1 + 1 + (1 if P else 0)

@@ -125,29 +125,28 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
     int *wsum = flag + E;          // 32
     int *misc = wsum + 32;         // 16: 0 status in, 2 n_over, 3 max replicas per rank
 
-    __shared__ unsigned long long s_total;
-    __shared__ int s_negative;
+    __shared__ long long s_part[32];
     for (int i = tid; i < 16; i += nt) misc[i] = 0;
-    if (tid == 0) {
-        s_total = 0;
-        s_negative = 0;
-    }
-    __syncthreads();
     // ---- totals; leave the accumulators zeroed for the next call
+    long long part = 0;
+    int negative = 0;
     for (int e = tid; e < E; e += nt) {
         const int v = ld_cg(a.t_acc + e);
         T[e] = v;
         a.t_acc[e] = 0;
         a.p.expert_count[e] = v;
-        if (v < 0) s_negative = 1;
-        else atomicAdd(&s_total, (unsigned long long)v);
+        negative |= v < 0;
+        part += v;
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(FULL_MASK, part, o);
+    if ((tid & 31) == 0) s_part[tid >> 5] = part;
     // the previous call's group buffer is no longer read: zero it
     {
         int *old = a.gs + (size_t)(parity ^ 1) * d.ngroups * E;
         for (int i = tid; i < d.ngroups * E; i += nt) old[i] = 0;
     }
-    __syncthreads();
+    negative = __syncthreads_or(negative);
     if (tid == 0) {
         misc[0] = ld_cg(a.hdr + WS_STATUS);
         a.hdr[WS_STATUS] = 0;
@@ -156,9 +155,11 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
     }
     __syncthreads();
     int status_in = misc[0];
+    long long total = 0;
+    for (int w = 0; w < (nt >> 5); ++w) total += s_part[w];
     // with every id valid the totals must be non-negative and add up to the
     // number of pairs; anything else means the workspace was not zeroed
-    if (!(status_in & MOONEP_ST_EXPERT_ID_RANGE) && (s_negative || s_total != (unsigned long long)d.pairs))
+    if (!(status_in & MOONEP_ST_EXPERT_ID_RANGE) && (negative || total != (long long)d.pairs))
         status_in |= MOONEP_ST_WORKSPACE;
     if (status_in & ST_EMPTY_PLAN) {
         if (tid == 0) {

@@ -407,3 +407,53 @@ def test_workspace_not_zeroed_is_detected(mp):
     p.workspace.zero_()
     mp.plan(cfg, topk, out=p)
     _assert_plan_equal(p, oracle.plan(oracle.Config(**c), topk.cpu().numpy()))
+
+
+@pytest.mark.parametrize("mv", [0.2, 1.0, 10.0, 20.0])
+def test_pages_sweep_shape_plan_and_sampled_data(mp, mv):
+    # the pages' EP=8 sweep shape (256 experts, top-8) up to maxvio 20
+    wl = W.WORKLOADS["ep8"]
+    r = W.routing(wl, mv, device=DEV)
+    topk = r.topk_idx.cpu().numpy()
+    gcfg, ocfg, gp, op = _plan_both(mp, _wl_cfg(wl), topk)
+    _assert_plan_equal(gp, op)
+    check_invariants(ocfg, topk, gp.to_numpy())
+    # every rank still receives exactly S*K rows however hot the hottest expert
+    assert (gp.slot_count.sum(dim=1).cpu() == wl.C).all()
+    hidden = W.hidden_states(wl, seed=1, device=DEV)
+    buf = mp.dispatch(gcfg, gp, hidden)
+    out = mp.combine(gcfg, gp, buf, r.weights)
+    rng = np.random.default_rng(4)
+    tokens = np.unique(np.concatenate([rng.choice(wl.tokens, 64, replace=False), [0, wl.tokens - 1]]))
+    sub, rows = _sub_plan(op, tokens, wl.K)
+    n = len(tokens)
+    scfg = oracle.Config(R=1, E=wl.E, K=wl.K, S=n, H=wl.H, B=0)
+    tt = torch.from_numpy(tokens).to(DEV)
+    ob = np.zeros((n * wl.K, wl.H), np.uint16)
+    oracle.dispatch(scfg, sub, W.bits(hidden[tt]), ob)
+    got = W.bits(buf.view(-1, wl.H)[torch.from_numpy(rows.astype(np.int64)).to(DEV)])
+    assert np.array_equal(got, ob)
+    oo = oracle.combine(scfg, sub, ob, r.weights[tt].cpu().numpy())
+    assert np.array_equal(W.bits(out[tt]), oo)
+
+
+def test_views_slices_match_slot_tables(mp):
+    wl = W.WORKLOADS["tiny"]
+    c = _wl_cfg(wl)
+    r = W.routing(wl, 1.0, device=DEV)
+    gcfg = mp.Config(**c)
+    gp = mp.plan(gcfg, r.topk_idx)
+    buf = mp.dispatch(gcfg, gp, W.hidden_states(wl, seed=1, device=DEV))
+    v = mp.views(gcfg, gp, buf)
+    se = gp.slot_expert.cpu().numpy()
+    sc = gp.slot_count.cpu().numpy()
+    rs = gp.row_src.cpu().numpy()
+    topk = r.topk_idx.cpu().numpy().ravel()
+    for rank, slots in enumerate(v):
+        assert sum(x.shape[0] for _, x in slots) == wl.C
+        row = rank * wl.C
+        for s, (e, x) in enumerate(slots):
+            assert e == se[rank, s] and x.shape[0] == sc[rank, s]
+            # each row of the view holds a token routed to the slot's expert
+            assert (topk[rs[row:row + x.shape[0]]] == e).all()
+            row += x.shape[0]

@@ -423,8 +423,9 @@ def run_ours(args, world, rank, local):
     # maxvio sweep: dispatch / combine GB/s and planner us per point
     sweep = []
     if not args.no_sweep:
-        for mv in wl.sweep:
-            rs = W.routing(wl, mv, seed=rank, device=dev)
+        # the Zipf sweep, then the adversarial placement (all hot experts on rank 0)
+        for mv, adv in [(m, False) for m in wl.sweep] + [(max(wl.sweep), True)]:
+            rs = W.routing(wl, mv, seed=rank, device=dev, adversarial=adv)
             ps = mp.Plan(cfg, dev)
             for _ in range(3):
                 mp.plan(cfg, rs.topk_idx, out=ps)
@@ -442,7 +443,7 @@ def run_ours(args, world, rank, local):
             inf = ps.info()
             gd = bytes_dispatch(wl) / (pd * 1e-3) / 1e9
             gc = bytes_combine(wl) / (pc * 1e-3) / 1e9
-            sweep.append({"maxvio": round(rs.maxvio, 3), "dispatch_GB/s": round(gd, 1),
+            sweep.append({"maxvio": round(rs.maxvio, 3), "adversarial": adv, "dispatch_GB/s": round(gd, 1),
                           "combine_GB/s": round(gc, 1), "dispatch_frac": round(gd / peak, 4),
                           "combine_frac": round(gc / peak, 4), "planner_us": round(pp * 1e3, 2),
                           "dispatch_tok/s": round(wl.tokens / (pd * 1e-3)),

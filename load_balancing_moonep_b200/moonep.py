@@ -185,6 +185,13 @@ class Plan:
         v = self.fields["info"].cpu().tolist()
         return {k: v[i] for i, k in enumerate(INFO_FIELDS)}
 
+    def maxvio(self) -> float:
+        """maxvio = max_e T_e / T_bar - 1 of the planned routing, with
+        T_bar = S*K*R/E (synchronises with the device)."""
+        T = self.fields["expert_count"].cpu()
+        c = self.cfg
+        return float(T.max()) / (c.S * c.K * c.R / c.E) - 1.0
+
     def to_numpy(self) -> dict:
         return {k: v.cpu().numpy() for k, v in self.fields.items()}
 

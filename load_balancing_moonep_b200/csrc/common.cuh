@@ -125,6 +125,7 @@ __device__ __forceinline__ int last_le(const int *a, int n, int x)
 
 // Exclusive prefix sum of a[0..n) in shared memory, in place; returns the
 // total.  Every thread of the block must call it.  wsum: >= 32 ints of smem.
+// Two barriers: after the per-warp scans every thread reads all warp totals.
 __device__ inline int block_exscan(int *a, int n, int *wsum)
 {
     const int tid = threadIdx.x, nt = blockDim.x;
@@ -136,25 +137,20 @@ __device__ inline int block_exscan(int *a, int n, int *wsum)
     int x = local;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        int y = __shfl_up_sync(FULL_MASK, x, o);
+        const int y = __shfl_up_sync(FULL_MASK, x, o);
         if (lane >= o) x += y;
     }
     if (lane == 31) wsum[w] = x;
     __syncthreads();
-    if (w == 0) {
-        int v = lane < nw ? wsum[lane] : 0;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            int y = __shfl_up_sync(FULL_MASK, v, o);
-            if (lane >= o) v += y;
-        }
-        if (lane < nw) wsum[lane] = v;
+    int before = 0, total = 0;
+    for (int j = 0; j < nw; ++j) {
+        const int v = wsum[j];
+        total += v;
+        before += j < w ? v : 0;
     }
-    __syncthreads();
-    int excl = x - local + (w > 0 ? wsum[w - 1] : 0);
-    const int total = wsum[nw - 1];
+    int excl = x - local + before;
     for (int i = beg; i < end; ++i) {
-        int v = a[i];
+        const int v = a[i];
         a[i] = excl;
         excl += v;
     }

@@ -60,7 +60,7 @@ __host__ __device__ inline int plan_smem_ints(int E, int R)
     const int nh = 2 * E + R;
     return 3 * E /*T shed keep*/ + 2 * R /*X D*/ + (E + R + 2) /*scr*/ + 2 * E /*pe pv*/ + 2 * R /*qr qv*/ +
            (E + R + 4) /*A: PS | QS*/ + E /*pilo*/ + (E + R + 4) /*Bs: segments | per rank*/ + R /*jlo*/ +
-           2 * R /*nrr ridx*/ + E /*pof*/ + 4 * nh /*cexp ccnt coff cspare*/ + (E + 1) /*hcnt*/ +
+           2 * R /*nrr ridx*/ + E /*pof*/ + 4 * nh /*cexp ccnt coff cspare*/ + (2 * E + 1) /*HC*/ +
            3 * nh /*hr hs hq*/ + E /*flag*/ + 32 + 16;
 }
 
@@ -73,11 +73,6 @@ __host__ __device__ inline int hist_smem_ints(int E, int R, int max_pairs)
 {
     const int a = plan_smem_ints(E, R), b = E + max_pairs;
     return a > b ? a : b;
-}
-
-__device__ __forceinline__ int seg_quota(const int *PS, const int *QS, int j, int i)
-{
-    return min(PS[j + 1], QS[i + 1]) - max(PS[j], QS[i]);
 }
 
 __device__ __forceinline__ void pdl_launch_dependents()
@@ -117,8 +112,8 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
     int *ccnt = cexp + nh;         // nh  rows
     int *coff = ccnt + nh;         // nh  slot offset
     int *cspare = coff + nh;       // nh  temporary
-    int *hcnt = cspare + nh;       // E + 1
-    int *hr = hcnt + E + 1;        // nh  host rank
+    int *HC = cspare + nh;         // 2E + 1: hosts per expert | 0 | work-list flags
+    int *hr = HC + 2 * E + 1;      // nh  host rank
     int *hs = hr + nh;             // nh  host slot
     int *hq = hs + nh;             // nh  host quota
     int *flag = hq + nh;           // E
@@ -127,6 +122,12 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
 
     __shared__ long long s_part[32];
     for (int i = tid; i < 16; i += nt) misc[i] = 0;
+    if (tid == 0) {  // every other CTA has arrived: take the status, reset the header
+        misc[0] = ld_cg(a.hdr + WS_STATUS);
+        a.hdr[WS_STATUS] = 0;
+        a.hdr[WS_TICKET] = 0;
+        a.hdr[WS_PARITY] = parity ^ 1;  // the next call accumulates into the other buffer
+    }
     // ---- totals; leave the accumulators zeroed for the next call
     long long part = 0;
     int negative = 0;
@@ -147,13 +148,6 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
         for (int i = tid; i < d.ngroups * E; i += nt) old[i] = 0;
     }
     negative = __syncthreads_or(negative);
-    if (tid == 0) {
-        misc[0] = ld_cg(a.hdr + WS_STATUS);
-        a.hdr[WS_STATUS] = 0;
-        a.hdr[WS_TICKET] = 0;
-        a.hdr[WS_PARITY] = parity ^ 1;  // the next call accumulates into the other buffer
-    }
-    __syncthreads();
     int status_in = misc[0];
     long long total = 0;
     for (int w = 0; w < (nt >> 5); ++w) total += s_part[w];
@@ -237,50 +231,50 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
     }
     __syncthreads();
 
-    // ---- prefix sums: A = [pv..., 0, qv..., 0] scanned gives PS and QS
+    // ---- prefix sums: A = [pv..., 0, qv..., 0] scanned gives PS = A[0..nP]
+    // and QS[i] = A[nP+1+i] - qbase, qbase being the pieces' total
+    int *segb = Bs;          // nP + 1: replicas per piece, then their prefix
+    int *rpr = Bs + nP + 1;  // R + 1: replicas per rank, then prefix + n_rep
     for (int x = tid; x < nP + nN + 2; x += nt) {
         int v = 0;
         if (x < nP) v = pv[x];
         else if (x > nP && x < nP + 1 + nN) v = qv[x - nP - 1];
         A[x] = v;
     }
+    for (int r = tid; r <= R; r += nt) rpr[r] = 0;
     __syncthreads();
     block_exscan(A, nP + nN + 2, wsum);
-    const int *PS = A;            // PS[0..nP]
-    int *QS = A + nP + 1;         // QS[0..nN] after removing the pieces' total
-    const int qbase = QS[0];
-    __syncthreads();
-    for (int x = tid; x <= nN; x += nt) QS[x] -= qbase;
-    __syncthreads();
+    const int *PS = A;
+    const int *QSr = A + nP + 1;
+    const int qbase = QSr[0];
+    auto seg_q = [&](int j, int i) {  // rows of the overlap of piece j and receiver i
+        return min(PS[j + 1], QSr[i + 1] - qbase) - max(PS[j], QSr[i] - qbase);
+    };
 
     // ---- water-filling: piece j meets receivers pilo[j].. ; receiver i meets
     // pieces jlo[i].. ; replicas are numbered in (j, i) order
-    int *segb = Bs;           // nP + 1
-    int *rpre = Bs + nP + 1;  // R + 1
     for (int j = tid; j < nP; j += nt) {
-        const int ilo = last_le(QS, nN, PS[j]);
-        const int ihi = last_le(QS, nN, PS[j + 1] - 1);
+        const int ilo = last_le(QSr, nN, PS[j] + qbase);
+        const int ihi = last_le(QSr, nN, PS[j + 1] - 1 + qbase);
         pilo[j] = ilo;
         segb[j] = ihi - ilo + 1;
         pof[pe[j]] = j;
     }
     for (int i = tid; i < nN; i += nt) {
-        const int jl = last_le(PS, nP, QS[i]);
-        const int jh = last_le(PS, nP, QS[i + 1] - 1);
+        const int jl = last_le(PS, nP, QSr[i] - qbase);
+        const int jh = last_le(PS, nP, QSr[i + 1] - 1 - qbase);
+        const int r = qr[i];
         jlo[i] = jl;
-        nrr[qr[i]] = jh - jl + 1;
-        ridx[qr[i]] = i;
+        nrr[r] = jh - jl + 1;
+        rpr[r] = jh - jl + 1;
+        ridx[r] = i;
     }
     if (tid == 0) segb[nP] = 0;
     __syncthreads();
-    for (int r = tid; r <= R; r += nt) rpre[r] = r < R ? nrr[r] : 0;
-    __syncthreads();
-    // one scan over [segments per piece | replicas per rank]
+    // one scan over [replicas per piece | replicas per rank]
     block_exscan(Bs, nP + 1 + R + 1, wsum);
     const int n_rep = Bs[nP];
-    __syncthreads();
-    for (int x = tid; x <= R; x += nt) rpre[x] -= n_rep;
-    __syncthreads();
+    auto rank_base = [&](int r) { return r * L + rpr[r] - n_rep; };  // first compact slot of rank r
 
     // ---- replica list (creation order) and the compact used-slot lists:
     // rank r's used slots sit at r*L + rpre[r] .. (home slots, then replicas)
@@ -289,25 +283,25 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
         const int i = pilo[j] + (q - segb[j]);
         const int ord = j - jlo[i];
         const int r = qr[i];
-        const int quota = seg_quota(PS, QS, j, i);
+        const int quota = seg_q(j, i);
         a.p.rep_expert[q] = pe[j];
         a.p.rep_rank[q] = r;
         a.p.rep_slot[q] = L + ord;
         a.p.rep_quota[q] = quota;
-        const int cs = r * L + rpre[r] + L + ord;
+        const int cs = rank_base(r) + L + ord;
         cexp[cs] = pe[j];
         ccnt[cs] = quota;
         if (ord >= B) atomicAdd(&misc[2], 1);
     }
     for (int e = tid; e < E; e += nt) {
         const int r = e / L;
-        const int cs = r * L + rpre[r] + (e - r * L);
+        const int cs = rank_base(r) + (e - r * L);
         cexp[cs] = e;
         ccnt[cs] = keep[e];
     }
     __syncthreads();
     for (int r = tid; r < R; r += nt) {
-        const int b0 = r * L + rpre[r], used = L + nrr[r];
+        const int b0 = rank_base(r), used = L + nrr[r];
         int off = 0;
         for (int s = 0; s < used; ++s) {
             coff[b0 + s] = off;
@@ -324,19 +318,33 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
         a.sc_off[x] = coff[x];
     }
 
-    // ---- host intervals: home + replicas of e, ascending rank
-    for (int e = tid; e <= E; e += nt) {
-        int c = 0;
-        if (e < E) {
-            c = 1;
-            if (pof[e] >= 0) c += segb[pof[e] + 1] - segb[pof[e]];
+    // ---- host intervals (home + replicas of e, ascending rank) and the
+    // reduce work list (experts with a prefetched replica), one scan for both:
+    // HC = [hosts per expert (E) | 0 | prefetched-replica flag per expert (E)]
+    for (int e = tid; e < E; e += nt) {
+        int c = 1, f = 0;
+        const int j = pof[e];
+        if (j >= 0) {
+            const int ns = segb[j + 1] - segb[j];
+            c += ns;
+            for (int s = 0; s < ns; ++s)
+                if (j - jlo[pilo[j] + s] < B) f = 1;
         }
-        hcnt[e] = c;
+        HC[e] = c;
+        HC[E + 1 + e] = f;
+        flag[e] = f;
     }
+    if (tid == 0) HC[E] = 0;
     __syncthreads();
-    block_exscan(hcnt, E + 1, wsum);
-    for (int e = tid; e <= E; e += nt) a.p.host_ptr[e] = hcnt[e];
-    for (int x = tid; x < E + n_rep; x += nt) {
+    const int hc_total = block_exscan(HC, 2 * E + 1, wsum);
+    const int n_hosts = E + n_rep;                   // == HC[E]
+    const int n_rep_experts = hc_total - n_hosts;
+    for (int e = tid; e <= E; e += nt) a.p.host_ptr[e] = HC[e];
+    for (int e = tid; e < E; e += nt) {
+        if (flag[e]) a.p.rep_home_list[HC[E + 1 + e] - n_hosts] = e;
+        if (e >= n_rep_experts) a.p.rep_home_list[e] = -1;
+    }
+    for (int x = tid; x < n_hosts; x += nt) {
         int e, r0, slot, quota, j, pos;
         if (x < E) {
             e = x;
@@ -352,14 +360,14 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
             e = pe[j];
             r0 = qr[i];
             slot = L + (j - jlo[i]);
-            quota = seg_quota(PS, QS, j, i);
+            quota = seg_q(j, i);
             pos = (e / L) < r0 ? 1 : 0;
         }
         if (j >= 0) {
             const int ns = segb[j + 1] - segb[j];
             for (int s = 0; s < ns; ++s) pos += qr[pilo[j] + s] < r0;
         }
-        const int h = hcnt[e] + pos;
+        const int h = HC[e] + pos;
         hr[h] = r0;
         hs[h] = slot;
         hq[h] = quota;
@@ -367,34 +375,15 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
     __syncthreads();
     for (int e = tid; e < E; e += nt) {
         int st = 0;
-        for (int h = hcnt[e]; h < hcnt[e + 1]; ++h) {
+        for (int h = HC[e]; h < HC[e + 1]; ++h) {
             const int r = hr[h], slot = hs[h];
             a.p.host_rank[h] = r;
             a.p.host_slot[h] = slot;
             a.p.host_quota[h] = hq[h];
             a.p.host_start[h] = st;
-            a.host_dst0[h] = r * C + coff[r * L + rpre[r] + slot] - st;
+            a.host_dst0[h] = r * C + coff[rank_base(r) + slot] - st;
             st += hq[h];
         }
-    }
-
-    // ---- experts with a prefetched replica (reduce work list)
-    for (int e = tid; e < E; e += nt) {
-        int f = 0;
-        const int j = pof[e];
-        if (j >= 0) {
-            const int ns = segb[j + 1] - segb[j];
-            for (int s = 0; s < ns; ++s)
-                if (j - jlo[pilo[j] + s] < B) f = 1;
-        }
-        flag[e] = f;
-        scr[e] = f;
-    }
-    __syncthreads();
-    const int n_rep_experts = block_exscan(scr, E, wsum);
-    for (int e = tid; e < E; e += nt) {
-        if (flag[e]) a.p.rep_home_list[scr[e]] = e;
-        if (e >= n_rep_experts) a.p.rep_home_list[e] = -1;
     }
 
     if (tid == 0) {

@@ -38,9 +38,11 @@ static int make_dims(const moonep_config *c, Dims *d)
     d->C = c->S * c->K;
     d->tokens = c->R * c->S;
     d->pairs = c->R * c->S * c->K;
-    // about two planner CTAs per SM of a B200 (148 SMs); the chunking only
-    // affects speed, never the plan
-    int ct = (d->tokens + 295) / 296;
+    // at most 2 x 148 - 1 chunks: two assignment CTAs fit on each SM of a
+    // B200 but one slot is held by the planner CTA while they start, and all
+    // of them should be resident then.  The chunking affects speed only,
+    // never the plan.
+    int ct = (d->tokens + 294) / 295;
     if (ct < 8) ct = 8;
     int cap = 4096 / d->K;
     if (cap < 1) cap = 1;

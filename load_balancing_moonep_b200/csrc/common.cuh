@@ -29,18 +29,20 @@ constexpr int CHUNK_GROUP = 16;
 
 // Workspace layout (bytes from the workspace base; 256-byte aligned parts).
 struct WsLayout {
-    size_t hdr;        // int32[4]: ticket, status, parity of the group buffers, spare
+    size_t hdr;        // int32[8]: ticket, status, call sequence, counts-ready mark, arrivals
     size_t t_acc;      // int32 [E]: expert totals accumulated by the histogram pass
     size_t gs;         // int32 [2][ngroups][E]: per-group expert counts, double-buffered
     size_t cc;         // int32 [nchunk][E]: per-chunk expert counts
     size_t host_dst0;  // int32 [2E+R]: rank*C + slot_offset - host_start per host
-    size_t sc_base;    // int32 [R+1]: first compact used slot of each rank
-    size_t sc_exp;     // int32 [2E+R]: expert of each used slot (compact)
-    size_t sc_cnt;     // int32 [2E+R]: rows of each used slot
-    size_t sc_off;     // int32 [2E+R]: slot offset of each used slot
+    size_t used;       // int32 [R]: used slots of each rank
     size_t total;
 };
-enum { WS_TICKET = 0, WS_STATUS = 1, WS_PARITY = 2 };
+// The call sequence number SEQ counts completed plan calls on a workspace; its
+// low bit selects the group-count buffer.  The last histogram CTA of a call
+// sets READY = SEQ + 1 once every chunk's counts are in; the assignment CTAs
+// wait for that mark, and the last of them to arrive advances SEQ, so after
+// a call READY == SEQ and a stale mark never passes for a fresh one.
+enum { WS_TICKET = 0, WS_STATUS = 1, WS_SEQ = 2, WS_READY = 3, WS_ARRIVED = 4, WS_HDR_INTS = 8 };
 
 // Status bits after which every later call treats the plan as empty.
 constexpr int ST_EMPTY_PLAN = MOONEP_ST_EXPERT_ID_RANGE | MOONEP_ST_WORKSPACE;
@@ -52,15 +54,12 @@ __host__ inline WsLayout ws_layout(const Dims &d)
     WsLayout w;
     const size_t i4 = sizeof(int32_t), nh = (size_t)(2 * d.E + d.R);
     size_t o = 0;
-    w.hdr = o; o = align256(o + 4 * i4);
+    w.hdr = o; o = align256(o + WS_HDR_INTS * i4);
     w.t_acc = o; o = align256(o + i4 * d.E);
     w.gs = o; o = align256(o + i4 * 2 * (size_t)d.ngroups * d.E);
     w.cc = o; o = align256(o + i4 * (size_t)d.nchunk * d.E);
     w.host_dst0 = o; o = align256(o + i4 * nh);
-    w.sc_base = o; o = align256(o + i4 * (d.R + 1));
-    w.sc_exp = o; o = align256(o + i4 * nh);
-    w.sc_cnt = o; o = align256(o + i4 * nh);
-    w.sc_off = o; o = align256(o + i4 * nh);
+    w.used = o; o = align256(o + i4 * d.R);
     w.total = o;
     return w;
 }
@@ -91,14 +90,20 @@ __device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv &f)
 }
 
 // Lanes holding the same key as this lane, from one ballot per key bit
-// (keys in [0, 2^nbits)); lanes with valid == false match nobody.
+// (keys in [0, 2^nbits), nbits <= MAX_KEY_BITS); lanes with valid == false
+// match nobody.  The loop is unrolled; the bit guard is warp-uniform.
+constexpr int MAX_KEY_BITS = 10;
+static_assert((1 << MAX_KEY_BITS) >= MOONEP_MAX_E, "expert ids need more key bits");
 __device__ __forceinline__ unsigned peers_of(int key, bool valid, int nbits)
 {
     unsigned m = __ballot_sync(0xffffffffu, valid);
-    for (int b = 0; b < nbits; ++b) {
-        const bool bit = (key >> b) & 1;
-        const unsigned bb = __ballot_sync(0xffffffffu, bit);
-        m &= bit ? bb : ~bb;
+#pragma unroll
+    for (int b = 0; b < MAX_KEY_BITS; ++b) {
+        if (b < nbits) {
+            const bool bit = (key >> b) & 1;
+            const unsigned bb = __ballot_sync(0xffffffffu, bit);
+            m &= bit ? bb : ~bb;
+        }
     }
     return valid ? m : 0u;
 }
@@ -112,6 +117,18 @@ __device__ __forceinline__ unsigned lanemask_lt()
 
 __device__ __forceinline__ int ld_cg(const int *p) { return __ldcg(p); }
 
+__device__ __forceinline__ int ld_acquire(const int *p)
+{
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release(int *p, int v)
+{
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 // Largest i in [0, n) with a[i] <= x, for non-decreasing a (a[0] <= x assumed).
 __device__ __forceinline__ int last_le(const int *a, int n, int x)
 {
@@ -123,17 +140,48 @@ __device__ __forceinline__ int last_le(const int *a, int n, int x)
     return lo;
 }
 
+// Largest i in [0, n) with a[i] <= x, for non-decreasing a (a[0] <= x
+// assumed), by one warp: every lane passes the same x and gets the result.
+// Ballots count 32 entries at a time, stopping at the first chunk that is
+// not all <= x.
+__device__ __forceinline__ int warp_last_le(const int *a, int n, int x)
+{
+    const int lane = threadIdx.x & 31;
+    int c = 0;
+    for (int j0 = 0; j0 < n; j0 += 32) {
+        const int j = j0 + lane;
+        const unsigned b = __ballot_sync(FULL_MASK, j < n && a[j] <= x);
+        c += __popc(b);
+        if (b != FULL_MASK) break;
+    }
+    return c - 1;
+}
+
 // Exclusive prefix sum of a[0..n) in shared memory, in place; returns the
 // total.  Every thread of the block must call it.  wsum: >= 32 ints of smem.
-// Two barriers: after the per-warp scans every thread reads all warp totals.
-__device__ inline int block_exscan(int *a, int n, int *wsum)
+// Two barriers.  Each thread takes PER consecutive elements (straight-line
+// code for PER = 1 and 2, a loop beyond), the warps scan with shuffles, and
+// every warp reads the warp totals with one load per lane and scans them
+// with shuffles too: on sm_100 a small runtime-bound loop, or every thread
+// reading every warp total, costs more than the whole scan.
+template <int PER>
+__device__ __forceinline__ int block_exscan_per(int *a, int n, int *wsum, int per)
 {
     const int tid = threadIdx.x, nt = blockDim.x;
     const int lane = tid & 31, w = tid >> 5, nw = nt >> 5;
-    const int per = (n + nt - 1) / nt;
-    const int beg = min(tid * per, n), end = min(beg + per, n);
-    int local = 0;
-    for (int i = beg; i < end; ++i) local += a[i];
+    const int beg = PER > 0 ? tid * PER : min(tid * per, n);
+    int v0 = 0, v1 = 0, local = 0;
+    if (PER == 1) {
+        v0 = beg < n ? a[beg] : 0;
+        local = v0;
+    } else if (PER == 2) {
+        v0 = beg < n ? a[beg] : 0;
+        v1 = beg + 1 < n ? a[beg + 1] : 0;
+        local = v0 + v1;
+    } else {
+        const int end = min(beg + per, n);
+        for (int i = beg; i < end; ++i) local += a[i];
+    }
     int x = local;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -142,20 +190,39 @@ __device__ inline int block_exscan(int *a, int n, int *wsum)
     }
     if (lane == 31) wsum[w] = x;
     __syncthreads();
-    int before = 0, total = 0;
-    for (int j = 0; j < nw; ++j) {
-        const int v = wsum[j];
-        total += v;
-        before += j < w ? v : 0;
+    int s = lane < nw ? wsum[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(FULL_MASK, s, o);
+        if (lane >= o) s += y;
     }
-    int excl = x - local + before;
-    for (int i = beg; i < end; ++i) {
-        const int v = a[i];
-        a[i] = excl;
-        excl += v;
+    const int total = __shfl_sync(FULL_MASK, s, 31);
+    const int upto_w = __shfl_sync(FULL_MASK, s, w);     // warps 0..w
+    const int own_w = __shfl_sync(FULL_MASK, x, 31);     // warp w alone
+    int excl = x - local + upto_w - own_w;
+    if (PER == 1) {
+        if (beg < n) a[beg] = excl;
+    } else if (PER == 2) {
+        if (beg < n) a[beg] = excl;
+        if (beg + 1 < n) a[beg + 1] = excl + v0;
+    } else {
+        const int end = min(beg + per, n);
+        for (int i = beg; i < end; ++i) {
+            const int v = a[i];
+            a[i] = excl;
+            excl += v;
+        }
     }
     __syncthreads();
     return total;
+}
+
+__device__ inline int block_exscan(int *a, int n, int *wsum)
+{
+    const int nt = blockDim.x;
+    if (n <= nt) return block_exscan_per<1>(a, n, wsum, 1);
+    if (n <= 2 * nt) return block_exscan_per<2>(a, n, wsum, 2);
+    return block_exscan_per<0>(a, n, wsum, (n + nt - 1) / nt);
 }
 
 }  // namespace moonep

@@ -6,7 +6,7 @@
 // exactly S*K token slots, by replicating a few experts online from the
 // router output -- and calls the planner near-optimal without giving it.
 // This file implements the water-filling plan described in moonep.h in two
-// launches, with no host synchronisation and no inter-CTA waiting:
+// launches, with no host synchronisation:
 //
 //   hist_plan_kernel  one CTA per token chunk stages the chunk's ids in
 //                     shared memory and counts them with shared-memory
@@ -19,39 +19,45 @@
 //                     index asc) orders by counting rank, prefix sums,
 //                     water-filling as a parallel merge of the two prefix-sum
 //                     partitions, compact per-rank slot lists, rank-ordered
-//                     host intervals.  It writes compact results only.
-//   assign_kernel     one CTA per token chunk: each warp counts its
-//                     contiguous sub-range, a prefix over earlier groups,
-//                     chunks and warps gives every warp its base, then the
-//                     warp walks its sub-range in (t, k) order ranking equal
-//                     experts with ballots, so g is the pair's rank among all
-//                     earlier pairs of its expert; the host interval holding
-//                     g gives the buffer row.  The CTAs also expand the
-//                     compact slot lists into the padded [R][E] tables.
-//                     Launched with programmatic dependent launch: its
-//                     input-only prologue overlaps the planner.
+//                     host intervals.  It writes the used slots of the
+//                     padded [R][E] tables and compact lists.
+//   assign_kernel     one CTA per token chunk, launched with programmatic
+//                     dependent launch, so every histogram CTA is resident
+//                     before it starts.  On its ids alone (pass A) each warp
+//                     walks a contiguous sub-range in (t, k) order ranking
+//                     equal experts with ballots, which gives every pair its
+//                     rank within the sub-range and every warp its counts.
+//                     After a bounded wait for the READY mark that the last
+//                     histogram CTA sets once all counts are in, a prefix
+//                     over earlier groups, chunks and warps gives every warp
+//                     its base -- all of this while the planner CTA runs.
+//                     Only pass B waits for the grid: g = base + rank is the
+//                     pair's rank among all pairs of its expert, and the host
+//                     interval holding g gives the buffer row.  The CTAs also
+//                     fill the unused tails of the padded tables.
 #include "common.cuh"
 
 namespace moonep {
 
 constexpr int PLAN_THREADS = 512;
 constexpr int ASSIGN_THREADS = 512;
+constexpr int READY_SPIN_LIMIT = 1 << 16;  // x 100 ns sleeps: far beyond any histogram pass
 constexpr int ASSIGN_WARPS = ASSIGN_THREADS / 32;
+// pass A packs (rank in the warp's sub-range, expert) into one int
+constexpr int PACK_BITS = 10, PACK_MASK = (1 << PACK_BITS) - 1;
+static_assert((1 << PACK_BITS) >= MOONEP_MAX_E, "expert ids need more pack bits");
 
 struct PlanParams {
     Dims d;
     const int32_t *topk;
     moonep_plan_t p;
-    int *hdr;        // ticket, status, parity
+    int *hdr;        // ticket, status, call sequence, counts-ready mark, arrivals
     int *t_acc;      // [E]
     int *gs;         // [2][ngroups][E]
     int *cc;         // [nchunk][E]
     int *host_dst0;  // [2E+R]
-    int *sc_base;    // [R+1]
-    int *sc_exp;     // [2E+R]
-    int *sc_cnt;     // [2E+R]
-    int *sc_off;     // [2E+R]
-    FastDiv fC;
+    int *used;       // [R] used slots per rank (home, then replicas)
+    FastDiv fC, fE, fE1, fL;  // divisions by C, E, E + 1 and L
 };
 
 // ints of dynamic shared memory used by the planner block
@@ -66,7 +72,7 @@ __host__ __device__ inline int plan_smem_ints(int E, int R)
 
 __host__ __device__ inline int assign_smem_ints(int E, int R, int max_pairs)
 {
-    return E + ASSIGN_WARPS * E + max_pairs + (E + 1) + 2 * (2 * E + R) + 32;
+    return ASSIGN_WARPS * E + max_pairs + (E + 1) + 2 * (2 * E + R) + 32;
 }
 
 __host__ __device__ inline int hist_smem_ints(int E, int R, int max_pairs)
@@ -84,11 +90,12 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 
 // ------------------------------------------------------------- planner CTA
 
-__device__ void plan_block(const PlanParams &a, int *sm, int parity)
+__device__ void plan_block(const PlanParams &a, int *sm)
 {
     const Dims &d = a.d;
     const int E = d.E, R = d.R, L = d.L, C = d.C, B = d.B;
     const int tid = threadIdx.x, nt = blockDim.x;
+    const int lane = tid & 31, warp = tid >> 5, nwarp = nt >> 5;
     const int nh = 2 * E + R;
 
     int *T = sm;
@@ -126,7 +133,6 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
         misc[0] = ld_cg(a.hdr + WS_STATUS);
         a.hdr[WS_STATUS] = 0;
         a.hdr[WS_TICKET] = 0;
-        a.hdr[WS_PARITY] = parity ^ 1;  // the next call accumulates into the other buffer
     }
     // ---- totals; leave the accumulators zeroed for the next call
     long long part = 0;
@@ -142,15 +148,11 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(FULL_MASK, part, o);
     if ((tid & 31) == 0) s_part[tid >> 5] = part;
-    // the previous call's group buffer is no longer read: zero it
-    {
-        int *old = a.gs + (size_t)(parity ^ 1) * d.ngroups * E;
-        for (int i = tid; i < d.ngroups * E; i += nt) old[i] = 0;
-    }
     negative = __syncthreads_or(negative);
     int status_in = misc[0];
-    long long total = 0;
-    for (int w = 0; w < (nt >> 5); ++w) total += s_part[w];
+    long long total = (tid & 31) < (nt >> 5) ? s_part[tid & 31] : 0;  // one load per lane
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) total += __shfl_xor_sync(FULL_MASK, total, o);
     // with every id valid the totals must be non-negative and add up to the
     // number of pairs; anything else means the workspace was not zeroed
     if (!(status_in & MOONEP_ST_EXPERT_ID_RANGE) && (negative || total != (long long)d.pairs))
@@ -166,6 +168,7 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
     // ---- home loads, excess X and deficit D per rank
     for (int r = tid; r < R; r += nt) {
         int h = 0;
+#pragma unroll 4
         for (int j = 0; j < L; ++j) h += T[r * L + j];
         X[r] = h > C ? h - C : 0;
         D[r] = h < C ? C - h : 0;
@@ -175,10 +178,11 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
     // ---- largest-first shedding: expert e sheds what remains of its rank's
     // excess after all larger (T desc, e asc) experts of the rank
     for (int e = tid; e < E; e += nt) {
-        const int r = e / L, v = T[e];
+        const int r = (int)fdiv((uint32_t)e, a.fL), v = T[e];
         int s = 0;
         if (X[r] > 0) {
             int before = 0;
+#pragma unroll 4
             for (int j = r * L; j < r * L + L; ++j) {
                 const int tj = T[j];
                 if (tj > v || (tj == v && j < e)) before += tj;
@@ -213,20 +217,32 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
             cspare[scr[E + r] - nP] = r;
         }
     __syncthreads();
-    // counting-rank sorts: pieces by (shed desc, e asc), receivers by (D desc, r asc)
-    for (int x = tid; x < nP + nN; x += nt) {
-        if (x < nP) {
-            const int v = hr[x], id = hs[x];
-            int pos = 0;
-            for (int j = 0; j < nP; ++j) pos += (hr[j] > v) || (hr[j] == v && hs[j] < id);
-            pe[pos] = id;
-            pv[pos] = v;
-        } else {
-            const int i0 = x - nP, v = hq[i0], id = cspare[i0];
-            int pos = 0;
-            for (int j = 0; j < nN; ++j) pos += (hq[j] > v) || (hq[j] == v && cspare[j] < id);
-            qr[pos] = id;
-            qv[pos] = v;
+    // counting-rank sorts, one warp per element: pieces by (shed desc,
+    // e asc), receivers by (D desc, r asc); an element's position is the
+    // number of entries ordered before it, counted 32 at a time by ballot
+    for (int x = warp; x < nP + nN; x += nwarp) {
+        const bool piece = x < nP;
+        const int m = piece ? nP : nN, xi = piece ? x : x - nP;
+        const int *val = piece ? hr : hq, *key = piece ? hs : cspare;
+        const int v = val[xi], id = key[xi];
+        int pos = 0;
+        for (int j0 = 0; j0 < m; j0 += 32) {
+            const int j = j0 + lane;
+            bool before = false;
+            if (j < m) {
+                const int vj = val[j];
+                before = vj > v || (vj == v && key[j] < id);
+            }
+            pos += __popc(__ballot_sync(FULL_MASK, before));
+        }
+        if (lane == 0) {
+            if (piece) {
+                pe[pos] = id;
+                pv[pos] = v;
+            } else {
+                qr[pos] = id;
+                qv[pos] = v;
+            }
         }
     }
     __syncthreads();
@@ -253,21 +269,29 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
 
     // ---- water-filling: piece j meets receivers pilo[j].. ; receiver i meets
     // pieces jlo[i].. ; replicas are numbered in (j, i) order
-    for (int j = tid; j < nP; j += nt) {
-        const int ilo = last_le(QSr, nN, PS[j] + qbase);
-        const int ihi = last_le(QSr, nN, PS[j + 1] - 1 + qbase);
-        pilo[j] = ilo;
-        segb[j] = ihi - ilo + 1;
-        pof[pe[j]] = j;
-    }
-    for (int i = tid; i < nN; i += nt) {
-        const int jl = last_le(PS, nP, QSr[i] - qbase);
-        const int jh = last_le(PS, nP, QSr[i + 1] - 1 - qbase);
-        const int r = qr[i];
-        jlo[i] = jl;
-        nrr[r] = jh - jl + 1;
-        rpr[r] = jh - jl + 1;
-        ridx[r] = i;
+    // (one warp per piece or receiver, searching by ballot)
+    for (int x = warp; x < nP + nN; x += nwarp) {
+        if (x < nP) {
+            const int j = x;
+            const int ilo = warp_last_le(QSr, nN, PS[j] + qbase);
+            const int ihi = warp_last_le(QSr, nN, PS[j + 1] - 1 + qbase);
+            if (lane == 0) {
+                pilo[j] = ilo;
+                segb[j] = ihi - ilo + 1;
+                pof[pe[j]] = j;
+            }
+        } else {
+            const int i = x - nP;
+            const int jl = warp_last_le(PS, nP, QSr[i] - qbase);
+            const int jh = warp_last_le(PS, nP, QSr[i + 1] - 1 - qbase);
+            if (lane == 0) {
+                const int r = qr[i];
+                jlo[i] = jl;
+                nrr[r] = jh - jl + 1;
+                rpr[r] = jh - jl + 1;
+                ridx[r] = i;
+            }
+        }
     }
     if (tid == 0) segb[nP] = 0;
     __syncthreads();
@@ -277,7 +301,8 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
     auto rank_base = [&](int r) { return r * L + rpr[r] - n_rep; };  // first compact slot of rank r
 
     // ---- replica list (creation order) and the compact used-slot lists:
-    // rank r's used slots sit at r*L + rpre[r] .. (home slots, then replicas)
+    // rank r's used slots sit at rank_base(r) .. (home slots, then replicas);
+    // coff holds the rows of each slot until the scan below
     for (int q = tid; q < n_rep; q += nt) {
         const int j = last_le(segb, nP, q);
         const int i = pilo[j] + (q - segb[j]);
@@ -291,31 +316,32 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
         const int cs = rank_base(r) + L + ord;
         cexp[cs] = pe[j];
         ccnt[cs] = quota;
+        coff[cs] = quota;
+        cspare[cs] = r;
         if (ord >= B) atomicAdd(&misc[2], 1);
     }
     for (int e = tid; e < E; e += nt) {
-        const int r = e / L;
+        const int r = (int)fdiv((uint32_t)e, a.fL);
         const int cs = rank_base(r) + (e - r * L);
         cexp[cs] = e;
         ccnt[cs] = keep[e];
+        coff[cs] = keep[e];
+        cspare[cs] = r;
     }
     __syncthreads();
-    for (int r = tid; r < R; r += nt) {
-        const int b0 = rank_base(r), used = L + nrr[r];
-        int off = 0;
-        for (int s = 0; s < used; ++s) {
-            coff[b0 + s] = off;
-            off += ccnt[b0 + s];
-        }
-        a.sc_base[r] = b0;
-        atomicMax(&misc[3], nrr[r]);
-    }
-    if (tid == 0) a.sc_base[R] = E + n_rep;
-    __syncthreads();
+    // slot offsets: one scan over all used slots; a slot's offset is its
+    // prefix minus that of its rank's first slot.  The used slots go straight
+    // into the padded [R][E] tables; the assignment pass fills the rest.
+    block_exscan(coff, E + n_rep, wsum);
     for (int x = tid; x < E + n_rep; x += nt) {
-        a.sc_exp[x] = cexp[x];
-        a.sc_cnt[x] = ccnt[x];
-        a.sc_off[x] = coff[x];
+        const int r = cspare[x], b0 = rank_base(r), s = x - b0;
+        a.p.slot_expert[(size_t)r * E + s] = cexp[x];
+        a.p.slot_count[(size_t)r * E + s] = ccnt[x];
+        a.p.slot_offset[(size_t)r * (E + 1) + s] = coff[x] - coff[b0];
+    }
+    for (int r = tid; r < R; r += nt) {
+        a.used[r] = L + nrr[r];
+        atomicMax(&misc[3], nrr[r]);
     }
 
     // ---- host intervals (home + replicas of e, ascending rank) and the
@@ -348,7 +374,7 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
         int e, r0, slot, quota, j, pos;
         if (x < E) {
             e = x;
-            r0 = e / L;
+            r0 = (int)fdiv((uint32_t)e, a.fL);
             slot = e - r0 * L;
             quota = keep[e];
             j = pof[e];
@@ -361,7 +387,7 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
             r0 = qr[i];
             slot = L + (j - jlo[i]);
             quota = seg_q(j, i);
-            pos = (e / L) < r0 ? 1 : 0;
+            pos = (int)fdiv((uint32_t)e, a.fL) < r0 ? 1 : 0;
         }
         if (j >= 0) {
             const int ns = segb[j + 1] - segb[j];
@@ -381,7 +407,8 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
             a.p.host_slot[h] = slot;
             a.p.host_quota[h] = hq[h];
             a.p.host_start[h] = st;
-            a.host_dst0[h] = r * C + coff[rank_base(r) + slot] - st;
+            const int b0 = rank_base(r);
+            a.host_dst0[h] = r * C + coff[b0 + slot] - coff[b0] - st;
             st += hq[h];
         }
     }
@@ -407,11 +434,11 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
 __global__ void __launch_bounds__(PLAN_THREADS) hist_plan_kernel(PlanParams a)
 {
     extern __shared__ int sm[];
-    __shared__ int s_last, s_parity;
+    __shared__ int s_last, s_seq;
     const Dims &d = a.d;
     const int E = d.E, K = d.K, tid = threadIdx.x, nt = blockDim.x;
-    // the assignment kernel may be scheduled now; it waits for this whole
-    // grid before it reads anything this grid writes
+    // the assignment kernel may be scheduled now: it reads the counts after
+    // the READY mark and the plan after this whole grid has completed
     pdl_launch_dependents();
 
     const int chunk = blockIdx.x;
@@ -422,9 +449,9 @@ __global__ void __launch_bounds__(PLAN_THREADS) hist_plan_kernel(PlanParams a)
     int *ids = sm + E;    // chunk_tokens * K
     for (int e = tid; e < E; e += nt) hist[e] = 0;
     for (int i = tid; i < n; i += nt) ids[i] = __ldg(a.topk + p0 + i);  // all loads in flight
-    if (tid == 0) s_parity = ld_cg(a.hdr + WS_PARITY) & 1;
+    if (tid == 0) s_seq = ld_cg(a.hdr + WS_SEQ);
     __syncthreads();
-    const int parity = s_parity;
+    const int seq = s_seq, parity = seq & 1;
     // distinct experts within a token: at most 32/K lanes of a warp collide
     int bad = 0;
     for (int i = tid; i < n; i += nt) {
@@ -450,12 +477,17 @@ __global__ void __launch_bounds__(PLAN_THREADS) hist_plan_kernel(PlanParams a)
         if (bad) atomicOr(a.hdr + WS_STATUS, MOONEP_ST_EXPERT_ID_RANGE);
         __threadfence();
         const bool last = atomicAdd(a.hdr + WS_TICKET, 1) == (int)gridDim.x - 1;
-        if (last) __threadfence();
+        if (last) {
+            __threadfence();
+            // every chunk's counts are in: open them to the assignment CTAs
+            a.hdr[WS_ARRIVED] = 0;
+            st_release(a.hdr + WS_READY, seq + 1);
+        }
         s_last = last;
     }
     __syncthreads();
     if (!s_last) return;
-    plan_block(a, sm, parity);
+    plan_block(a, sm);
 }
 
 // ---------------------------------------------------------- assignment
@@ -473,92 +505,85 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
     const int max_pairs = d.chunk_tokens * K;
     const int nh = 2 * E + R;
 
-    int *base = sm;                        // E
-    int *cnt = base + E;                   // ASSIGN_WARPS * E
+    int *cnt = sm;                         // ASSIGN_WARPS * E
     int *ids = cnt + ASSIGN_WARPS * E;     // max_pairs
     int *hptr = ids + max_pairs;           // E + 1
     int *hstart = hptr + E + 1;            // nh
     int *hdst = hstart + nh;               // nh
     int *red = hdst + nh;                  // 32
+    __shared__ int s_seq, s_ready;
 
     // prologue on inputs only, overlapping the histogram/planner grid
     for (int i = tid; i < ASSIGN_WARPS * E; i += nt) cnt[i] = 0;
     for (int i = tid; i < n; i += nt) ids[i] = __ldg(a.topk + p0 + i);
-    pdl_wait();  // the histogram/planner grid has completed; its writes are visible
+    __syncthreads();
 
-    const int status = ld_cg(a.p.info + MOONEP_INFO_STATUS);
-    const bool empty = (status & ST_EMPTY_PLAN) != 0;
-    // every count and index read back from the plan is clamped, so even a
-    // plan block of garbage cannot steer an access out of its array
-    const int n_rep = empty ? 0 : min(max(ld_cg(a.p.info + MOONEP_INFO_N_REP), 0), E + R - 1);
-
-    // ---- padded tables from the compact slot lists, spread over the CTAs
+    // pass A, on the ids alone: each warp walks its contiguous sub-range in
+    // (t, k) order, ranking equal experts with ballots, so loc is the pair's
+    // rank among the sub-range's earlier pairs of its expert and the warp's
+    // counters end as its per-expert counts.  ids[i] becomes loc << 10 | e.
+    // (Out-of-range ids are left as they are; they make the plan empty.)
+    const int per = (n + ASSIGN_WARPS - 1) / ASSIGN_WARPS;
+    const int wbeg = min(warp * per, n), wend = min(wbeg + per, n);
     {
-        const long long g = (long long)gridDim.x * nt, x0 = (long long)blockIdx.x * nt + tid;
-        for (long long x = x0; x < (long long)R * E; x += g) {
-            const int r = (int)(x / E), s = (int)(x - (long long)r * E);
-            int ex = -1, ct = 0;
-            if (!empty) {
-                const int b0 = min(max(ld_cg(a.sc_base + r), 0), nh);
-                const int b1 = min(max(ld_cg(a.sc_base + r + 1), b0), nh);
-                if (s < b1 - b0) {
-                    ex = ld_cg(a.sc_exp + b0 + s);
-                    ct = ld_cg(a.sc_cnt + b0 + s);
-                }
-            }
-            a.p.slot_expert[x] = ex;
-            a.p.slot_count[x] = ct;
-        }
-        for (long long x = x0; x < (long long)R * (E + 1); x += g) {
-            const int r = (int)(x / (E + 1)), s = (int)(x - (long long)r * (E + 1));
-            int v = 0;
-            if (!empty) {
-                const int b0 = min(max(ld_cg(a.sc_base + r), 0), nh);
-                const int b1 = min(max(ld_cg(a.sc_base + r + 1), b0), nh);
-                v = s < b1 - b0 ? ld_cg(a.sc_off + b0 + s) : C;
-            }
-            a.p.slot_offset[x] = v;
-        }
-        for (long long x = x0; x < E + R; x += g)
-            if (x >= n_rep) {
-                a.p.rep_expert[x] = -1;
-                a.p.rep_rank[x] = -1;
-                a.p.rep_slot[x] = -1;
-                a.p.rep_quota[x] = 0;
-            }
-        const int hused = empty ? 0 : E + n_rep;
-        for (long long x = x0; x < nh; x += g)
-            if (x >= hused) {
-                a.p.host_rank[x] = -1;
-                a.p.host_slot[x] = -1;
-                a.p.host_start[x] = 0;
-                a.p.host_quota[x] = 0;
-            }
-        if (empty) {
-            for (long long x = x0; x <= E; x += g) a.p.host_ptr[x] = 0;
-            for (long long x = x0; x < E; x += g) a.p.rep_home_list[x] = -1;
+        int *wc = cnt + warp * E;
+        for (int b = wbeg; b < wend; b += 32) {
+            const int i = b + lane;
+            const bool valid = i < wend;
+            const int e = valid ? ids[i] : 0;
+            const bool ok = valid && e >= 0 && e < E;
+            const unsigned peers = peers_of(ok ? e : 0, ok, d.ebits);
+            int loc = 0;
+            if (ok) loc = wc[e] + __popc(peers & lanemask_lt());
+            __syncwarp();
+            if (ok && lane == __ffs(peers) - 1) wc[e] += __popc(peers);
+            __syncwarp();
+            if (ok) ids[i] = (loc << PACK_BITS) | e;
         }
     }
 
-    if (empty) {
-        for (int i = tid; i < n; i += nt) {
-            a.p.dst_pos[p0 + i] = -1;
-            a.p.row_src[p0 + i] = -1;
+    // ---- the counts are complete once the last histogram CTA has set READY;
+    // the planner CTA is still running then, and the chunk bases and warp
+    // counts below overlap it.  Every histogram CTA is resident before this
+    // grid starts, so the mark comes; the bounded wait falls back to the
+    // grid dependency, which implies it.
+    if (tid == 0) {
+        const int seq = ld_cg(a.hdr + WS_SEQ);
+        int ok = 0;
+        for (int it = 0; it < READY_SPIN_LIMIT; ++it) {
+            if (ld_acquire(a.hdr + WS_READY) == seq + 1) {
+                ok = 1;
+                break;
+            }
+            __nanosleep(100);
         }
-        return;
+        s_seq = seq;
+        s_ready = ok;
+    }
+    __syncthreads();
+    if (!s_ready) pdl_wait();
+    const int seq = s_seq;
+    if (tid == 0) {  // the last CTA past this point advances the sequence
+        if (atomicAdd(a.hdr + WS_ARRIVED, 1) == (int)gridDim.x - 1) {
+            a.hdr[WS_ARRIVED] = 0;
+            a.hdr[WS_SEQ] = seq + 1;
+        }
     }
 
-    for (int e = tid; e <= E; e += nt) hptr[e] = min(max(ld_cg(a.p.host_ptr + e), 0), E + n_rep);
-    for (int h = tid; h < E + n_rep; h += nt) {
-        hstart[h] = ld_cg(a.p.host_start + h);
-        hdst[h] = ld_cg(a.host_dst0 + h);
+    // the previous call's group-count buffer is read by nobody now; zero it
+    // for the next call, which accumulates into it
+    {
+        int *old = a.gs + (size_t)((seq & 1) ^ 1) * d.ngroups * E;
+        const int n_gs = d.ngroups * E;
+        for (int i = blockIdx.x * nt + tid; i < n_gs; i += gridDim.x * nt) old[i] = 0;
     }
+
     // pairs of each expert in earlier chunks: earlier groups + earlier chunks
-    // of this chunk's group, all loads of a batch in flight together
+    // of this chunk's group, all loads of a batch in flight together, then
+    // the warp bases
     {
         const int grp = chunk / CHUNK_GROUP, c0 = grp * CHUNK_GROUP;
-        const int parity = ld_cg(a.hdr + WS_PARITY) ^ 1;  // the buffer this call filled
-        const int *gsb = a.gs + (size_t)parity * d.ngroups * E;
+        const int *gsb = a.gs + (size_t)(seq & 1) * d.ngroups * E;  // the buffer this call filled
         for (int e = tid; e < E; e += nt) {
             int s = 0;
             for (int g0 = 0; g0 < grp; g0 += 16) {
@@ -584,52 +609,90 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
 #pragma unroll
                 for (int j = 0; j < CHUNK_GROUP - 1; ++j) s += w[j];
             }
-            base[e] = s;
+            // warp bases: this prefix plus the earlier warps' counts of
+            // this chunk (pass A's counters are past the barrier above)
+            for (int w = 0; w < ASSIGN_WARPS; ++w) {
+                const int t = cnt[w * E + e];
+                cnt[w * E + e] = s;
+                s += t;
+            }
         }
     }
-    __syncthreads();
 
-    // pass 1: count each expert's pairs in every warp's contiguous sub-range
-    // (distinct experts within a token: at most 32/K lanes collide)
-    const int per = (n + ASSIGN_WARPS - 1) / ASSIGN_WARPS;
-    const int wbeg = min(warp * per, n), wend = min(wbeg + per, n);
+    // ---- the plan: the histogram/planner grid has completed.  Every load
+    // below is issued before any of its results is used (one round trip),
+    // and every count or index read back is clamped, so even a plan block of
+    // garbage cannot steer an access out of its array.
+    pdl_wait();
+    const int status = ld_cg(a.p.info + MOONEP_INFO_STATUS);
+    const int n_rep_raw = ld_cg(a.p.info + MOONEP_INFO_N_REP);
+    // host tables of the whole array; only entries inside the clamped
+    // [host_ptr[e], host_ptr[e+1]) are used
+    for (int e = tid; e <= E; e += nt) hptr[e] = min(max(ld_cg(a.p.host_ptr + e), 0), nh);
+    for (int h = tid; h < nh; h += nt) {
+        hstart[h] = ld_cg(a.p.host_start + h);
+        hdst[h] = ld_cg(a.host_dst0 + h);
+    }
+    const bool empty = (status & ST_EMPTY_PLAN) != 0;
+    const int n_rep = empty ? 0 : min(max(n_rep_raw, 0), E + R - 1);
+
+    // ---- unused tails of the padded tables (the planner wrote the used
+    // slots), the replica and host lists, spread over the CTAs
     {
-        int *wc = cnt + warp * E;
-        for (int i = wbeg + lane; i < wend; i += 32) {
-            const int e = ids[i];
-            if (e >= 0 && e < E) atomicAdd(&wc[e], 1);
+        const int g = gridDim.x * nt, x0 = blockIdx.x * nt + tid;
+        for (int x = x0; x < R * E; x += g) {
+            const int r = (int)fdiv((uint32_t)x, a.fE), s = x - r * E;
+            const int used = empty ? 0 : min(max(ld_cg(a.used + r), 0), E);
+            if (s >= used) {
+                a.p.slot_expert[x] = -1;
+                a.p.slot_count[x] = 0;
+            }
+        }
+        for (int x = x0; x < R * (E + 1); x += g) {
+            const int r = (int)fdiv((uint32_t)x, a.fE1), s = x - r * (E + 1);
+            const int used = empty ? 0 : min(max(ld_cg(a.used + r), 0), E);
+            if (s >= used) a.p.slot_offset[x] = empty ? 0 : C;  // an empty plan is all zeros
+        }
+        for (int x = x0; x < E + R; x += g)
+            if (x >= n_rep) {
+                a.p.rep_expert[x] = -1;
+                a.p.rep_rank[x] = -1;
+                a.p.rep_slot[x] = -1;
+                a.p.rep_quota[x] = 0;
+            }
+        const int hused = empty ? 0 : E + n_rep;
+        for (int x = x0; x < nh; x += g)
+            if (x >= hused) {
+                a.p.host_rank[x] = -1;
+                a.p.host_slot[x] = -1;
+                a.p.host_start[x] = 0;
+                a.p.host_quota[x] = 0;
+            }
+        if (empty) {
+            for (int x = x0; x <= E; x += g) a.p.host_ptr[x] = 0;
+            for (int x = x0; x < E; x += g) a.p.rep_home_list[x] = -1;
         }
     }
-    __syncthreads();
-    // warp bases: chunk prefix plus earlier warps of this chunk
-    for (int e = tid; e < E; e += nt) {
-        int run = base[e];
-        for (int w = 0; w < ASSIGN_WARPS; ++w) {
-            const int t = cnt[w * E + e];
-            cnt[w * E + e] = run;
-            run += t;
+
+    if (empty) {
+        for (int i = tid; i < n; i += nt) {
+            a.p.dst_pos[p0 + i] = -1;
+            a.p.row_src[p0 + i] = -1;
         }
+        return;
     }
     __syncthreads();
 
-    // pass 2, in (t, k) order within the warp's sub-range: g = warp base +
-    // earlier pairs of the expert in this sub-range (ballot-matched lanes);
-    // the host interval holding g gives the buffer row
+    // pass B: g = warp base + loc is the pair's rank among all pairs of its
+    // expert in (t, k) order; the host interval holding g gives the buffer row
     int remote = 0;
     {
-        int *wc = cnt + warp * E;
-        for (int b = wbeg; b < wend; b += 32) {
-            const int i = b + lane;
-            const bool valid = i < wend;
-            const int e = valid ? ids[i] : 0;
-            const bool ok = valid && e >= 0 && e < E;
-            const unsigned peers = peers_of(ok ? e : 0, ok, d.ebits);
-            int g = 0;
-            if (ok) g = wc[e] + __popc(peers & lanemask_lt());
-            __syncwarp();
-            if (ok && lane == __ffs(peers) - 1) wc[e] += __popc(peers);
-            __syncwarp();
-            if (!ok) continue;
+        const int *wb = cnt + warp * E;
+        for (int i = wbeg + lane; i < wend; i += 32) {
+            const int v = ids[i];
+            const int e = v & PACK_MASK, loc = v >> PACK_BITS;
+            if (v < 0 || e >= E) continue;  // cannot happen in a non-empty plan
+            const int g = wb[e] + loc;
             int h = hptr[e];
             const int hend = hptr[e + 1];
             while (h + 1 < hend && hstart[h + 1] <= g) ++h;
@@ -643,7 +706,7 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
             a.p.dst_pos[p] = dst;
             a.p.row_src[dst] = p;
             // source rank of pair p is p / (S*K) = p / C
-            remote += fdiv((uint32_t)dst, a.fC) != fdiv((uint32_t)p, a.fC);
+            remote += (uint32_t)dst - fdiv((uint32_t)p, a.fC) * (uint32_t)C >= (uint32_t)C;
         }
     }
 #pragma unroll
@@ -677,11 +740,11 @@ int launch_plan(const Dims &d, const int32_t *topk, const moonep_plan_t &p, void
     a.gs = reinterpret_cast<int *>(w + wl.gs);
     a.cc = reinterpret_cast<int *>(w + wl.cc);
     a.host_dst0 = reinterpret_cast<int *>(w + wl.host_dst0);
-    a.sc_base = reinterpret_cast<int *>(w + wl.sc_base);
-    a.sc_exp = reinterpret_cast<int *>(w + wl.sc_exp);
-    a.sc_cnt = reinterpret_cast<int *>(w + wl.sc_cnt);
-    a.sc_off = reinterpret_cast<int *>(w + wl.sc_off);
+    a.used = reinterpret_cast<int *>(w + wl.used);
     a.fC = make_fastdiv((uint32_t)d.C);
+    a.fE = make_fastdiv((uint32_t)d.E);
+    a.fE1 = make_fastdiv((uint32_t)(d.E + 1));
+    a.fL = make_fastdiv((uint32_t)d.L);
 
     const size_t smem1 = sizeof(int) * (size_t)hist_smem_ints(d.E, d.R, d.chunk_tokens * d.K);
     if (!set_smem((const void *)hist_plan_kernel, smem1)) return MOONEP_ERR_CUDA;

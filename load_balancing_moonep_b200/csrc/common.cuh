@@ -159,26 +159,29 @@ __device__ __forceinline__ int warp_last_le(const int *a, int n, int x)
 
 // Exclusive prefix sum of a[0..n) in shared memory, in place; returns the
 // total.  Every thread of the block must call it.  wsum: >= 32 ints of smem.
-// Two barriers.  Each thread takes PER consecutive elements (straight-line
-// code for PER = 1 and 2, a loop beyond), the warps scan with shuffles, and
-// every warp reads the warp totals with one load per lane and scans them
-// with shuffles too: on sm_100 a small runtime-bound loop, or every thread
-// reading every warp total, costs more than the whole scan.
+// Two barriers.  Each thread takes PER consecutive elements (PER fixed at
+// compile time, fully unrolled; PER = 0: a runtime loop of per elements),
+// the warps scan with shuffles, and every warp reads the warp totals with one
+// load per lane and scans them with shuffles too: on sm_100 a small
+// runtime-bound loop, or every thread reading every warp total, costs more
+// than the whole scan.
 template <int PER>
 __device__ __forceinline__ int block_exscan_per(int *a, int n, int *wsum, int per)
 {
     const int tid = threadIdx.x, nt = blockDim.x;
     const int lane = tid & 31, w = tid >> 5, nw = nt >> 5;
-    const int beg = PER > 0 ? tid * PER : min(tid * per, n);
-    int v0 = 0, v1 = 0, local = 0;
-    if (PER == 1) {
-        v0 = beg < n ? a[beg] : 0;
-        local = v0;
-    } else if (PER == 2) {
-        v0 = beg < n ? a[beg] : 0;
-        v1 = beg + 1 < n ? a[beg + 1] : 0;
-        local = v0 + v1;
+    constexpr int P = PER > 0 ? PER : 1;
+    int v[P];
+    int local = 0, beg;
+    if (PER > 0) {
+        beg = tid * PER;
+#pragma unroll
+        for (int k = 0; k < P; ++k) {
+            v[k] = beg + k < n ? a[beg + k] : 0;
+            local += v[k];
+        }
     } else {
+        beg = min(tid * per, n);
         const int end = min(beg + per, n);
         for (int i = beg; i < end; ++i) local += a[i];
     }
@@ -197,20 +200,21 @@ __device__ __forceinline__ int block_exscan_per(int *a, int n, int *wsum, int pe
         if (lane >= o) s += y;
     }
     const int total = __shfl_sync(FULL_MASK, s, 31);
-    const int upto_w = __shfl_sync(FULL_MASK, s, w);     // warps 0..w
-    const int own_w = __shfl_sync(FULL_MASK, x, 31);     // warp w alone
+    const int upto_w = __shfl_sync(FULL_MASK, s, w);  // warps 0..w
+    const int own_w = __shfl_sync(FULL_MASK, x, 31);  // warp w alone
     int excl = x - local + upto_w - own_w;
-    if (PER == 1) {
-        if (beg < n) a[beg] = excl;
-    } else if (PER == 2) {
-        if (beg < n) a[beg] = excl;
-        if (beg + 1 < n) a[beg + 1] = excl + v0;
+    if (PER > 0) {
+#pragma unroll
+        for (int k = 0; k < P; ++k) {
+            if (beg + k < n) a[beg + k] = excl;
+            excl += v[k];
+        }
     } else {
         const int end = min(beg + per, n);
         for (int i = beg; i < end; ++i) {
-            const int v = a[i];
+            const int u = a[i];
             a[i] = excl;
-            excl += v;
+            excl += u;
         }
     }
     __syncthreads();
@@ -222,6 +226,8 @@ __device__ inline int block_exscan(int *a, int n, int *wsum)
     const int nt = blockDim.x;
     if (n <= nt) return block_exscan_per<1>(a, n, wsum, 1);
     if (n <= 2 * nt) return block_exscan_per<2>(a, n, wsum, 2);
+    if (n <= 3 * nt) return block_exscan_per<3>(a, n, wsum, 3);
+    if (n <= 4 * nt) return block_exscan_per<4>(a, n, wsum, 4);
     return block_exscan_per<0>(a, n, wsum, (n + nt - 1) / nt);
 }
 

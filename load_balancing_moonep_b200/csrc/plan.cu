@@ -66,8 +66,8 @@ __host__ __device__ inline int plan_smem_ints(int E, int R)
     const int nh = 2 * E + R;
     return 3 * E /*T shed keep*/ + 2 * R /*X D*/ + (E + R + 2) /*scr*/ + 2 * E /*pe pv*/ + 2 * R /*qr qv*/ +
            (E + R + 4) /*A: PS | QS*/ + E /*pilo*/ + (E + R + 4) /*Bs: segments | per rank*/ + R /*jlo*/ +
-           2 * R /*nrr ridx*/ + E /*pof*/ + 4 * nh /*cexp ccnt coff cspare*/ + (2 * E + 1) /*HC*/ +
-           3 * nh /*hr hs hq*/ + E /*flag*/ + 32 + 16;
+           2 * R /*nrr ridx*/ + E /*pof*/ + 3 * nh /*cexp ccnt cspare*/ + 3 * nh /*hr hs hq, then Z*/ +
+           E /*flag*/ + 32 + 16;
 }
 
 __host__ __device__ inline int assign_smem_ints(int E, int R, int max_pairs)
@@ -117,12 +117,10 @@ __device__ void plan_block(const PlanParams &a, int *sm)
     int *pof = ridx + R;           // E   piece index of expert e, -1 if none
     int *cexp = pof + E;           // nh  compact used slots: expert
     int *ccnt = cexp + nh;         // nh  rows
-    int *coff = ccnt + nh;         // nh  slot offset
-    int *cspare = coff + nh;       // nh  temporary
-    int *HC = cspare + nh;         // 2E + 1: hosts per expert | 0 | work-list flags
-    int *hr = HC + 2 * E + 1;      // nh  host rank
-    int *hs = hr + nh;             // nh  host slot
-    int *hq = hs + nh;             // nh  host quota
+    int *cspare = ccnt + nh;       // nh  receiver ids while sorting, then the rank of each used slot
+    int *hr = cspare + nh;         // nh  piece rows, while sorting
+    int *hs = hr + nh;             // nh  piece experts, while sorting
+    int *hq = hs + nh;             // nh  receiver deficits, while sorting
     int *flag = hq + nh;           // E
     int *wsum = flag + E;          // 32
     int *misc = wsum + 32;         // 16: 0 status in, 2 n_over, 3 max replicas per rank
@@ -235,30 +233,29 @@ __device__ void plan_block(const PlanParams &a, int *sm)
             }
             pos += __popc(__ballot_sync(FULL_MASK, before));
         }
-        if (lane == 0) {
+        if (lane == 0) {  // A = [pv..., 0, qv..., 0] for the prefix sums below
             if (piece) {
                 pe[pos] = id;
                 pv[pos] = v;
+                A[pos] = v;
             } else {
                 qr[pos] = id;
                 qv[pos] = v;
+                A[nP + 1 + pos] = v;
             }
         }
     }
-    __syncthreads();
-
-    // ---- prefix sums: A = [pv..., 0, qv..., 0] scanned gives PS = A[0..nP]
-    // and QS[i] = A[nP+1+i] - qbase, qbase being the pieces' total
+    if (tid == 0) {
+        A[nP] = 0;
+        A[nP + nN + 1] = 0;
+    }
     int *segb = Bs;          // nP + 1: replicas per piece, then their prefix
     int *rpr = Bs + nP + 1;  // R + 1: replicas per rank, then prefix + n_rep
-    for (int x = tid; x < nP + nN + 2; x += nt) {
-        int v = 0;
-        if (x < nP) v = pv[x];
-        else if (x > nP && x < nP + 1 + nN) v = qv[x - nP - 1];
-        A[x] = v;
-    }
     for (int r = tid; r <= R; r += nt) rpr[r] = 0;
     __syncthreads();
+
+    // ---- prefix sums: A scanned gives PS = A[0..nP] and QS[i] =
+    // A[nP+1+i] - qbase, qbase being the pieces' total
     block_exscan(A, nP + nN + 2, wsum);
     const int *PS = A;
     const int *QSr = A + nP + 1;
@@ -300,9 +297,13 @@ __device__ void plan_block(const PlanParams &a, int *sm)
     const int n_rep = Bs[nP];
     auto rank_base = [&](int r) { return r * L + rpr[r] - n_rep; };  // first compact slot of rank r
 
-    // ---- replica list (creation order) and the compact used-slot lists:
-    // rank r's used slots sit at rank_base(r) .. (home slots, then replicas);
-    // coff holds the rows of each slot until the scan below
+    // ---- replica list (creation order), the compact used-slot lists and
+    // the per-expert host counts, all into one array Z for one scan:
+    //   Z = [rows of each used slot (E + n_rep) | hosts per expert (E) | 0 |
+    //        prefetched-replica flag per expert (E) | 0]
+    // Rank r's used slots sit at rank_base(r) .. (home slots, then replicas).
+    int *Z = hr;  // 4E + R + 2 <= 3 nh ints, free after the sort
+    const int zh = E + n_rep, zf = zh + E + 1, nz = zf + E + 1;
     for (int q = tid; q < n_rep; q += nt) {
         const int j = last_le(segb, nP, q);
         const int i = pilo[j] + (q - segb[j]);
@@ -316,7 +317,7 @@ __device__ void plan_block(const PlanParams &a, int *sm)
         const int cs = rank_base(r) + L + ord;
         cexp[cs] = pe[j];
         ccnt[cs] = quota;
-        coff[cs] = quota;
+        Z[cs] = quota;
         cspare[cs] = r;
         if (ord >= B) atomicAdd(&misc[2], 1);
     }
@@ -325,29 +326,9 @@ __device__ void plan_block(const PlanParams &a, int *sm)
         const int cs = rank_base(r) + (e - r * L);
         cexp[cs] = e;
         ccnt[cs] = keep[e];
-        coff[cs] = keep[e];
+        Z[cs] = keep[e];
         cspare[cs] = r;
-    }
-    __syncthreads();
-    // slot offsets: one scan over all used slots; a slot's offset is its
-    // prefix minus that of its rank's first slot.  The used slots go straight
-    // into the padded [R][E] tables; the assignment pass fills the rest.
-    block_exscan(coff, E + n_rep, wsum);
-    for (int x = tid; x < E + n_rep; x += nt) {
-        const int r = cspare[x], b0 = rank_base(r), s = x - b0;
-        a.p.slot_expert[(size_t)r * E + s] = cexp[x];
-        a.p.slot_count[(size_t)r * E + s] = ccnt[x];
-        a.p.slot_offset[(size_t)r * (E + 1) + s] = coff[x] - coff[b0];
-    }
-    for (int r = tid; r < R; r += nt) {
-        a.used[r] = L + nrr[r];
-        atomicMax(&misc[3], nrr[r]);
-    }
-
-    // ---- host intervals (home + replicas of e, ascending rank) and the
-    // reduce work list (experts with a prefetched replica), one scan for both:
-    // HC = [hosts per expert (E) | 0 | prefetched-replica flag per expert (E)]
-    for (int e = tid; e < E; e += nt) {
+        // hosts: home + one per replica; flag: a replica within the budget
         int c = 1, f = 0;
         const int j = pof[e];
         if (j >= 0) {
@@ -356,29 +337,47 @@ __device__ void plan_block(const PlanParams &a, int *sm)
             for (int s = 0; s < ns; ++s)
                 if (j - jlo[pilo[j] + s] < B) f = 1;
         }
-        HC[e] = c;
-        HC[E + 1 + e] = f;
+        Z[zh + e] = c;
+        Z[zf + e] = f;
         flag[e] = f;
     }
-    if (tid == 0) HC[E] = 0;
+    if (tid == 0) {
+        Z[zh + E] = 0;
+        Z[zf + E] = 0;
+    }
     __syncthreads();
-    const int hc_total = block_exscan(HC, 2 * E + 1, wsum);
-    const int n_hosts = E + n_rep;                   // == HC[E]
-    const int n_rep_experts = hc_total - n_hosts;
-    for (int e = tid; e <= E; e += nt) a.p.host_ptr[e] = HC[e];
+    block_exscan(Z, nz, wsum);
+    // slot offset = prefix minus that of the rank's first slot; host_ptr[e]
+    // and the work-list position likewise relative to their part's start
+    const int zh0 = Z[zh], zf0 = Z[zf];
+    const int n_hosts = E + n_rep;                  // == Z[zh + E] - zh0
+    const int n_rep_experts = Z[zf + E] - zf0;
+    auto hptr = [&](int e) { return Z[zh + e] - zh0; };
+    for (int x = tid; x < E + n_rep; x += nt) {  // used slots into the padded [R][E] tables
+        const int r = cspare[x], b0 = rank_base(r), sl = x - b0;
+        a.p.slot_expert[(size_t)r * E + sl] = cexp[x];
+        a.p.slot_count[(size_t)r * E + sl] = ccnt[x];
+        a.p.slot_offset[(size_t)r * (E + 1) + sl] = Z[x] - Z[b0];
+    }
+    for (int r = tid; r < R; r += nt) {
+        a.used[r] = L + nrr[r];
+        atomicMax(&misc[3], nrr[r]);
+    }
+    for (int e = tid; e <= E; e += nt) a.p.host_ptr[e] = hptr(e);
     for (int e = tid; e < E; e += nt) {
-        if (flag[e]) a.p.rep_home_list[HC[E + 1 + e] - n_hosts] = e;
+        if (flag[e]) a.p.rep_home_list[Z[zf + e] - zf0] = e;
         if (e >= n_rep_experts) a.p.rep_home_list[e] = -1;
     }
+    // ---- host intervals: the hosts of e in ascending rank; a host's start
+    // is the rows of the hosts of e on lower ranks
     for (int x = tid; x < n_hosts; x += nt) {
-        int e, r0, slot, quota, j, pos;
+        int e, r0, slot, quota, j, pos = 0, st = 0;
         if (x < E) {
             e = x;
             r0 = (int)fdiv((uint32_t)e, a.fL);
             slot = e - r0 * L;
             quota = keep[e];
             j = pof[e];
-            pos = 0;
         } else {
             const int q = x - E;
             j = last_le(segb, nP, q);
@@ -387,30 +386,28 @@ __device__ void plan_block(const PlanParams &a, int *sm)
             r0 = qr[i];
             slot = L + (j - jlo[i]);
             quota = seg_q(j, i);
-            pos = (int)fdiv((uint32_t)e, a.fL) < r0 ? 1 : 0;
+            if ((int)fdiv((uint32_t)e, a.fL) < r0) {  // the home rank is lower
+                pos = 1;
+                st = keep[e];
+            }
         }
         if (j >= 0) {
             const int ns = segb[j + 1] - segb[j];
-            for (int s = 0; s < ns; ++s) pos += qr[pilo[j] + s] < r0;
+            for (int s = 0; s < ns; ++s) {
+                const int i = pilo[j] + s;
+                if (qr[i] < r0) {
+                    ++pos;
+                    st += seg_q(j, i);
+                }
+            }
         }
-        const int h = HC[e] + pos;
-        hr[h] = r0;
-        hs[h] = slot;
-        hq[h] = quota;
-    }
-    __syncthreads();
-    for (int e = tid; e < E; e += nt) {
-        int st = 0;
-        for (int h = HC[e]; h < HC[e + 1]; ++h) {
-            const int r = hr[h], slot = hs[h];
-            a.p.host_rank[h] = r;
-            a.p.host_slot[h] = slot;
-            a.p.host_quota[h] = hq[h];
-            a.p.host_start[h] = st;
-            const int b0 = rank_base(r);
-            a.host_dst0[h] = r * C + coff[b0 + slot] - coff[b0] - st;
-            st += hq[h];
-        }
+        const int h = hptr(e) + pos;
+        const int b0 = rank_base(r0);
+        a.p.host_rank[h] = r0;
+        a.p.host_slot[h] = slot;
+        a.p.host_quota[h] = quota;
+        a.p.host_start[h] = st;
+        a.host_dst0[h] = r0 * C + Z[b0 + slot] - Z[b0] - st;
     }
 
     if (tid == 0) {

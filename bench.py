@@ -23,7 +23,6 @@ from __future__ import annotations
 
 import argparse
 import hashlib
-import glob
 import json
 import os
 import statistics
@@ -87,23 +86,35 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
-def kernel_sources_hash() -> str:
+# the source files each measured kernel is compiled from: a kernel's ncu
+# counters stay valid while these are unchanged
+KERNEL_SOURCES = {
+    "dispatch": ("data.cu", "common.cuh"),
+    "combine": ("data.cu", "common.cuh"),
+    "combine_bwd": ("data.cu", "common.cuh"),
+    "reduce": ("reduce.cu", "common.cuh"),
+    "prefetch": ("prefetch.cu", "common.cuh"),
+}
+
+
+def kernel_sources_hash(kernel: str) -> str:
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "load_balancing_moonep_b200", "csrc", "*"))):
-        h.update(open(f, "rb").read())
+    for f in KERNEL_SOURCES[kernel]:
+        h.update(open(os.path.join(ROOT, "load_balancing_moonep_b200", "csrc", f), "rb").read())
+    h.update(open(os.path.join(ROOT, "include", "moonep.h"), "rb").read())
     return h.hexdigest()[:16]
 
 
 def ncu_traffic():
-    """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel sources."""
+    """DRAM bytes per launch from the committed ncu summary, for each kernel
+    whose sources are unchanged since the capture."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return {}
     d = json.load(open(p))
-    if d.get("csrc_sha") != kernel_sources_hash():
-        return {}
-    return d.get("per_launch_bytes", {})
+    sha = d.get("sources_sha", {})
+    return {k: v for k, v in d.get("per_launch_bytes", {}).items()
+            if k in KERNEL_SOURCES and sha.get(k) == kernel_sources_hash(k)}
 
 
 # ----------------------------------------------------------------- clocks

@@ -30,7 +30,6 @@ constexpr int CHUNK_GROUP = 16;
 // Workspace layout (bytes from the workspace base; 256-byte aligned parts).
 struct WsLayout {
     size_t hdr;        // int32[8]: ticket, status, call sequence, counts-ready mark, arrivals
-    size_t t_acc;      // int32 [E]: expert totals accumulated by the histogram pass
     size_t gs;         // int32 [2][ngroups][E]: per-group expert counts, double-buffered
     size_t cc;         // int32 [nchunk][E]: per-chunk expert counts
     size_t host_dst0;  // int32 [2E+R]: rank*C + slot_offset - host_start per host
@@ -55,7 +54,6 @@ __host__ inline WsLayout ws_layout(const Dims &d)
     const size_t i4 = sizeof(int32_t), nh = (size_t)(2 * d.E + d.R);
     size_t o = 0;
     w.hdr = o; o = align256(o + WS_HDR_INTS * i4);
-    w.t_acc = o; o = align256(o + i4 * d.E);
     w.gs = o; o = align256(o + i4 * 2 * (size_t)d.ngroups * d.E);
     w.cc = o; o = align256(o + i4 * (size_t)d.nchunk * d.E);
     w.host_dst0 = o; o = align256(o + i4 * nh);

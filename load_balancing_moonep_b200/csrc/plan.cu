@@ -12,8 +12,9 @@
 //                     shared memory and counts them with shared-memory
 //                     atomics (a token's K experts are distinct, so few lanes
 //                     of a warp collide), stores the counts for the second
-//                     pass and adds them to per-group and total counts with
-//                     global atomics (sums: order-free, so deterministic).
+//                     pass and adds them to the counts of its group of
+//                     CHUNK_GROUP chunks with global atomics (sums:
+//                     order-free, so deterministic).
 //                     The CTA that finishes last (atomic ticket) runs the
 //                     planner: loads, largest-first shedding, (value desc,
 //                     index asc) orders by counting rank, prefix sums,
@@ -52,7 +53,6 @@ struct PlanParams {
     const int32_t *topk;
     moonep_plan_t p;
     int *hdr;        // ticket, status, call sequence, counts-ready mark, arrivals
-    int *t_acc;      // [E]
     int *gs;         // [2][ngroups][E]
     int *cc;         // [nchunk][E]
     int *host_dst0;  // [2E+R]
@@ -81,6 +81,22 @@ __host__ __device__ inline int hist_smem_ints(int E, int R, int max_pairs)
     return a > b ? a : b;
 }
 
+// p[0] + p[stride] + ... + p[(n-1) stride], read through L2 with BATCH
+// loads in flight at a time (one round trip for n <= BATCH)
+template <int BATCH>
+__device__ __forceinline__ int sum_strided(const int *p, int stride, int n)
+{
+    int s = 0;
+    for (int g0 = 0; g0 < n; g0 += BATCH) {
+        int v[BATCH];
+#pragma unroll
+        for (int j = 0; j < BATCH; ++j) v[j] = g0 + j < n ? ld_cg(p + (size_t)(g0 + j) * stride) : 0;
+#pragma unroll
+        for (int j = 0; j < BATCH; ++j) s += v[j];
+    }
+    return s;
+}
+
 __device__ __forceinline__ void pdl_launch_dependents()
 {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -90,7 +106,7 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 
 // ------------------------------------------------------------- planner CTA
 
-__device__ void plan_block(const PlanParams &a, int *sm)
+__device__ void plan_block(const PlanParams &a, int *sm, int parity)
 {
     const Dims &d = a.d;
     const int E = d.E, R = d.R, L = d.L, C = d.C, B = d.B;
@@ -132,16 +148,21 @@ __device__ void plan_block(const PlanParams &a, int *sm)
         a.hdr[WS_STATUS] = 0;
         a.hdr[WS_TICKET] = 0;
     }
-    // ---- totals; leave the accumulators zeroed for the next call
+    // ---- totals: the sum of this call's group counts (one atomic sum per
+    // chunk and expert lands in a group of CHUNK_GROUP chunks, so no address
+    // takes more than CHUNK_GROUP atomics; per-expert totals accumulated
+    // by every CTA serialised some 300 atomics per address)
     long long part = 0;
     int negative = 0;
-    for (int e = tid; e < E; e += nt) {
-        const int v = ld_cg(a.t_acc + e);
-        T[e] = v;
-        a.t_acc[e] = 0;
-        a.p.expert_count[e] = v;
-        negative |= v < 0;
-        part += v;
+    {
+        const int *gsb = a.gs + (size_t)parity * d.ngroups * E;
+        for (int e = tid; e < E; e += nt) {
+            const int v = sum_strided<32>(gsb + e, E, d.ngroups);
+            T[e] = v;
+            a.p.expert_count[e] = v;
+            negative |= v < 0;
+            part += v;
+        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(FULL_MASK, part, o);
@@ -461,10 +482,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) hist_plan_kernel(PlanParams a)
     for (int e = tid; e < E; e += nt) {
         const int c = hist[e];
         a.cc[(size_t)chunk * E + e] = c;
-        if (c) {
-            atomicAdd(a.t_acc + e, c);  // sums: order-free
-            atomicAdd(gsb + e, c);
-        }
+        if (c) atomicAdd(gsb + e, c);  // sums: order-free
     }
     // release: the CTA barrier orders every thread's writes before thread 0's
     // device-scope fence and ticket increment; the last CTA's thread 0
@@ -484,7 +502,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) hist_plan_kernel(PlanParams a)
     }
     __syncthreads();
     if (!s_last) return;
-    plan_block(a, sm);
+    plan_block(a, sm, parity);
 }
 
 // ---------------------------------------------------------- assignment
@@ -583,10 +601,10 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
         const int *gsb = a.gs + (size_t)(seq & 1) * d.ngroups * E;  // the buffer this call filled
         for (int e = tid; e < E; e += nt) {
             int s = 0;
-            for (int g0 = 0; g0 < grp; g0 += 16) {
-                int v[16];
+            for (int g0 = 0; g0 < grp; g0 += 32) {
+                int v[32];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) v[j] = (g0 + j < grp) ? ld_cg(gsb + (size_t)(g0 + j) * E + e) : 0;
+                for (int j = 0; j < 32; ++j) v[j] = (g0 + j < grp) ? ld_cg(gsb + (size_t)(g0 + j) * E + e) : 0;
                 int w[CHUNK_GROUP - 1];
                 if (g0 == 0) {
 #pragma unroll
@@ -596,7 +614,7 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
                     for (int j = 0; j < CHUNK_GROUP - 1; ++j) s += w[j];
                 }
 #pragma unroll
-                for (int j = 0; j < 16; ++j) s += v[j];
+                for (int j = 0; j < 32; ++j) s += v[j];
             }
             if (grp == 0) {
                 int w[CHUNK_GROUP - 1];
@@ -719,9 +737,14 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
 
 // ---------------------------------------------------------------- launch
 
+// Both planner kernels ask for the largest shared-memory carveout: an SM
+// that runs histogram CTAs must also fit two assignment CTAs as the
+// histogram CTAs retire (the carveout changes only when an SM is idle).
 static bool set_smem(const void *fn, size_t bytes)
 {
-    return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess;
+    return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess &&
+           cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                (int)cudaSharedmemCarveoutMaxShared) == cudaSuccess;
 }
 
 int launch_plan(const Dims &d, const int32_t *topk, const moonep_plan_t &p, void *ws, cudaStream_t st)
@@ -733,7 +756,6 @@ int launch_plan(const Dims &d, const int32_t *topk, const moonep_plan_t &p, void
     a.topk = topk;
     a.p = p;
     a.hdr = reinterpret_cast<int *>(w + wl.hdr);
-    a.t_acc = reinterpret_cast<int *>(w + wl.t_acc);
     a.gs = reinterpret_cast<int *>(w + wl.gs);
     a.cc = reinterpret_cast<int *>(w + wl.cc);
     a.host_dst0 = reinterpret_cast<int *>(w + wl.host_dst0);

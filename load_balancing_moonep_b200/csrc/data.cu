@@ -288,21 +288,18 @@ __global__ void __launch_bounds__(DATA_THREADS) combine_bwd_kernel(
 
 // ----------------------------------------------------------------- launch
 
+// One token per warp: a block of DATA_THREADS / 32 warps per group of
+// tokens, as many blocks as that takes.  A grid of one resident wave
+// (SMs x 2048 / DATA_THREADS blocks) walking the tokens left about 14 tokens
+// per warp, and the warps that drew one more token set the kernel's tail:
+// one token per warp, with the block scheduler refilling SMs, measured 5 %
+// faster on dispatch and combine backward at the large shape.  The kernels
+// keep their grid-stride loops, so any grid is correct.
 static int data_grid(int tokens)
 {
-    static int sms[64] = {0};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64) dev = 0;
-    if (!sms[dev]) {
-        int v = 0;
-        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-        sms[dev] = v > 0 ? v : 148;
-    }
     const int wpb = DATA_THREADS / 32;
-    const int want = (tokens + wpb - 1) / wpb;
-    const int full = sms[dev] * (2048 / DATA_THREADS);
-    return want < full ? (want > 0 ? want : 1) : full;
+    const long long want = ((long long)tokens + wpb - 1) / wpb;
+    return want < 1 ? 1 : (want > (1LL << 30) ? (1 << 30) : (int)want);
 }
 
 int launch_dispatch(const Dims &d, const int *dst_pos, int *info, const uint16_t *hidden, uint16_t *buf,

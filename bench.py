@@ -460,6 +460,11 @@ def run_ours(args, world, rank, local):
                           "dispatch_tok/s": round(wl.tokens / (pd * 1e-3)),
                           "n_rep": inf["n_rep"], "n_overflow": inf["n_overflow"],
                           "max_rep_per_rank": inf["max_rep_per_rank"],
+                          # plan quality: any exact plan needs at least
+                          # max(pieces, receivers) replicas; the greedy makes
+                          # at most pieces + receivers - 1
+                          "n_rep_bounds": [max(inf["n_pieces"], inf["n_receivers"]),
+                                           max(inf["n_pieces"] + inf["n_receivers"] - 1, 0)],
                           "remote_pair_frac": round(inf["n_remote_pairs"] / wl.pairs, 4)})
             del ps
 

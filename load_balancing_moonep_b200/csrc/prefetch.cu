@@ -107,9 +107,9 @@ int launch_prefetch(const Dims &d, const moonep_plan_t &p, const uint16_t *weigh
     a.row_bytes = P * 2;
     const bool vec = (a.row_bytes % 16 == 0) && (reinterpret_cast<uintptr_t>(weights) % 16 == 0) &&
                      (reinterpret_cast<uintptr_t>(pool) % 16 == 0);
-    // four waves of blocks: the block scheduler refills SMs as blocks finish,
-    // which evens out the tail of the item loop (9 % over one wave)
-    const int grid = sms[dev] * (2048 / PF_THREADS) * 4;
+    // eight waves of blocks: the block scheduler refills SMs as blocks
+    // finish, which evens out the tail of the item loop (9 % over one wave)
+    const int grid = sms[dev] * (2048 / PF_THREADS) * 8;
     if (vec) {
         a.chunk = 256 * 1024;
         prefetch_kernel<uint4><<<grid, PF_THREADS, 0, st>>>(a);

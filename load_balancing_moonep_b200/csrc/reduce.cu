@@ -199,9 +199,9 @@ int launch_reduce(const Dims &d, const moonep_plan_t &p, float *reduce_buf, floa
     a.P = P;
     const bool vec = (P % 4 == 0) && (reinterpret_cast<uintptr_t>(reduce_buf) % 16 == 0) &&
                      (reinterpret_cast<uintptr_t>(home_grad) % 16 == 0);
-    // four waves of blocks: the block scheduler refills SMs as blocks finish,
-    // which evens out the tail of the item loop (2 % over one wave)
-    const int grid = sms[dev] * (2048 / REDUCE_THREADS) * 4;
+    // eight waves of blocks: the block scheduler refills SMs as blocks
+    // finish, which evens out the tail of the item loop (4 % over one wave)
+    const int grid = sms[dev] * (2048 / REDUCE_THREADS) * 8;
     if (vec) {
         a.chunk = (long long)REDUCE_THREADS * REDUCE_UNROLL * 8;
         reduce_kernel<float4><<<grid, REDUCE_THREADS, 0, st>>>(a);

@@ -184,6 +184,50 @@ def test_plan_repeat_deterministic(mp):
             assert np.array_equal(p1[k], p2[k])
 
 
+def test_plan_alternating_routings_reuse_workspace(mp):
+    """Many calls on one plan block and workspace, alternating two routings.
+    Every call flips the group-count buffer (low bit of the call sequence),
+    the assignment CTAs zero the other one, and the counts-ready mark of one
+    call must never pass for the next: every plan must equal the oracle's."""
+    wl = W.WORKLOADS["mid"]
+    gcfg, ocfg = _cfgs(_wl_cfg(wl), mp)
+    rs = [W.routing(wl, mv, device="cpu") for mv in (0.5, 3.0)]
+    ops = [oracle.plan(ocfg, r.topk_idx.numpy()) for r in rs]
+    tks = [r.topk_idx.to(DEV) for r in rs]
+    p = mp.Plan(gcfg)
+    for it in range(24):
+        mp.plan(gcfg, tks[it % 2], out=p)
+        _assert_plan_equal(p, ops[it % 2])
+
+
+def test_plan_in_cuda_graph_replays(mp):
+    """The plan captured in a CUDA graph (its programmatic launch edge and
+    counts-ready handshake replayed) with fresh routings written into the
+    captured input between replays: every replay equals the oracle."""
+    wl = W.WORKLOADS["decode"]
+    gcfg, ocfg = _cfgs(_wl_cfg(wl), mp)
+    rs = [W.routing(wl, mv, seed=sd, device="cpu") for sd, mv in ((0, 5.0), (1, 5.0), (2, 1.0))]
+    ops = [oracle.plan(ocfg, r.topk_idx.numpy()) for r in rs]
+    topk = rs[0].topk_idx.to(DEV).clone()
+    p = mp.Plan(gcfg)
+    torch.cuda.synchronize()  # the plan block was zero-filled on the default stream
+    cs = torch.cuda.Stream()
+    with torch.cuda.stream(cs):
+        for _ in range(2):
+            mp.plan(gcfg, topk, out=p)
+    cs.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=cs, capture_error_mode="thread_local"):
+        mp.plan(gcfg, topk, out=p)
+    for it in range(6):
+        topk.copy_(rs[it % 3].topk_idx.to(DEV))
+        torch.cuda.synchronize()
+        graph.replay()
+        torch.cuda.synchronize()
+        _assert_plan_equal(p, ops[it % 3])
+    del graph
+
+
 def test_host_errors(mp):
     with pytest.raises(mp.MoonepError):
         mp.plan(mp.Config(R=3, E=16, K=2, S=8, H=8, B=2), torch.zeros(24, 2, dtype=torch.int32, device=DEV))

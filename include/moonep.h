@@ -74,7 +74,7 @@ extern "C" {
 #define MOONEP_ERR_BUDGET_RULE 3    /* TRAIN_B_RULE set and B != E/R */
 #define MOONEP_ERR_B_RANGE 4        /* B < 0 or B > E - L */
 #define MOONEP_ERR_CUDA 5           /* a kernel launch failed */
-#define MOONEP_ERR_LIMIT 7          /* E > MOONEP_MAX_E */
+#define MOONEP_ERR_LIMIT 7          /* E > MOONEP_MAX_E; K > 16 in moonep_combine_backward */
 #define MOONEP_ERR_ALIGN 8          /* H % 8 != 0 or a data pointer not 16-byte aligned */
 #define MOONEP_ERR_NOALLOC_SIZE 9   /* moonep_plan_noalloc: workspace above MOONEP_NOALLOC_WORKSPACE_BYTES */
 
@@ -198,7 +198,8 @@ MOONEP_API int moonep_combine(const moonep_config *cfg, const moonep_plan_t *pla
  *                                dy itself with MOONEP_FLAG_BWD_UNSCALED)
  *   dw[t, k] = sum_h dy[t,h] * y[dst_pos[t*K+k], h]          (fp32 accumulation)
  * dy: bf16 [R*S, H]; w: fp32 [R*S, K]; y: bf16 [R, S*K, H];
- * dy_buf: bf16 [R, S*K, H]; dw: fp32 [R*S, K]. */
+ * dy_buf: bf16 [R, S*K, H]; dw: fp32 [R*S, K].  K <= 16 (each of a token's
+ * K dot products is kept in registers); MOONEP_ERR_LIMIT above that. */
 MOONEP_API int moonep_combine_backward(const moonep_config *cfg, const moonep_plan_t *plan, const uint16_t *dy,
                             const float *w, const uint16_t *y, uint16_t *dy_buf, float *dw,
                             void *stream);

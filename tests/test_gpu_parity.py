@@ -292,6 +292,51 @@ def test_data_steps_full(mp, wname, mv):
     assert gp.info()["status"] == op["info"][0]  # no row-range fault raised by the data kernels
 
 
+@pytest.mark.parametrize("K", [1, 3, 4, 5, 7, 12, 40])
+def test_data_steps_every_k_path(mp, K):
+    """The compile-time-K specialisations (1, 2, 4, 6, 8), the any-K kernels
+    (3, 5, 7, 12) and K > 32 (destination rows beyond one warp's lanes), on a
+    skewed routing with a ragged row (H = 136: 17 vectors, not a multiple of
+    32 lanes), every element against the oracle."""
+    c = dict(R=4, E=48, K=K, S=48, H=136, B=3, flags=0)
+    rng = np.random.default_rng(100 + K)
+    T = c["R"] * c["S"]
+    bias = -1.5 * np.log(rng.permutation(np.arange(1, c["E"] + 1)))
+    scores = rng.standard_normal((T, c["E"])) + bias
+    topk = np.argsort(-scores, axis=1, kind="stable")[:, :K].astype(np.int32)
+    gcfg, ocfg, gp, op = _plan_both(mp, c, topk)
+    _assert_plan_equal(gp, op)
+    check_invariants(ocfg, topk, gp.to_numpy())
+    C = c["S"] * K
+    wl = W.Workload("k", c["R"], c["E"], K, c["S"], c["H"], c["B"])
+    hidden = W.hidden_states(wl, seed=1, device=DEV)
+    buf = torch.full((c["R"], C, c["H"]), float("nan"), dtype=torch.bfloat16, device=DEV)
+    mp.dispatch(gcfg, gp, hidden, buf)
+    ob = np.zeros((c["R"], C, c["H"]), np.uint16)
+    oracle.dispatch(ocfg, op, W.bits(hidden), ob)
+    assert np.array_equal(W.bits(buf), ob)
+    y = W.bf16_normal((c["R"], C, c["H"]), seed=2, device=DEV)
+    w = torch.from_numpy(rng.random((T, K)).astype(np.float32)).to(DEV)
+    out = mp.combine(gcfg, gp, y, w)
+    assert np.array_equal(W.bits(out), oracle.combine(ocfg, op, W.bits(y), w.cpu().numpy()))
+    dy = W.bf16_normal((T, c["H"]), seed=3, device=DEV)
+    if K > 16:  # combine backward keeps a token's K dot products in registers
+        with pytest.raises(mp.MoonepError) as ei:
+            mp.combine_backward(gcfg, gp, dy, w, y)
+        assert ei.value.code == 7
+        return
+    dyb, dw = mp.combine_backward(gcfg, gp, dy, w, y)
+    odyb = np.zeros_like(ob)
+    odw = np.zeros((T, K), np.float32)
+    oracle.combine_backward(ocfg, op, W.bits(dy), w.cpu().numpy(), W.bits(y), odyb, odw)
+    assert np.array_equal(W.bits(dyb), odyb)
+    dyf = dy.float().cpu().numpy().astype(np.float64)
+    yf = y.float().cpu().numpy().reshape(-1, c["H"]).astype(np.float64)
+    mag = np.einsum("th,tkh->tk", np.abs(dyf), np.abs(yf[op["dst_pos"]]))
+    assert (np.abs(dw.cpu().numpy().astype(np.float64) - odw) <= 1e-5 * mag + 1e-30).all()
+    assert gp.info()["status"] == op["info"][0]
+
+
 @pytest.mark.parametrize("wname,mv", [("large", 1.0), ("large", 3.0), ("decode", 5.0)])
 def test_data_steps_full_size_sampled(mp, wname, mv):
     wl = W.WORKLOADS[wname]

@@ -16,12 +16,16 @@
 //                     CHUNK_GROUP chunks with global atomics (sums:
 //                     order-free, so deterministic).
 //                     The CTA that finishes last (atomic ticket) runs the
-//                     planner: loads, largest-first shedding, (value desc,
-//                     index asc) orders by counting rank, prefix sums,
-//                     water-filling as a parallel merge of the two prefix-sum
-//                     partitions, compact per-rank slot lists, rank-ordered
-//                     host intervals.  It writes the used slots of the
-//                     padded [R][E] tables and compact lists.
+//                     planner: expert totals from the group counts, loads,
+//                     largest-first shedding, (value desc, index asc) orders
+//                     by counting rank, prefix sums, water-filling as a
+//                     parallel merge of the two prefix-sum partitions,
+//                     per-rank slot lists, rank-ordered host intervals.  Its
+//                     primitives are shuffle scans and warp ballots: on
+//                     sm_100 a runtime-bound shared-memory loop costs a full
+//                     load latency per step.  It writes the used slots of the
+//                     padded [R][E] tables, the replica list, the host CSR
+//                     and the reduce work list.
 //   assign_kernel     one CTA per token chunk, launched with programmatic
 //                     dependent launch, so every histogram CTA is resident
 //                     before it starts.  On its ids alone (pass A) each warp
@@ -64,9 +68,9 @@ struct PlanParams {
 __host__ __device__ inline int plan_smem_ints(int E, int R)
 {
     const int nh = 2 * E + R;
-    return 3 * E /*T shed keep*/ + 2 * R /*X D*/ + (E + R + 2) /*scr*/ + 2 * E /*pe pv*/ + 2 * R /*qr qv*/ +
+    return 3 * E /*T shed keep*/ + 2 * R /*X D*/ + (E + R + 2) /*scr*/ + E /*pe*/ + R /*qr*/ +
            (E + R + 4) /*A: PS | QS*/ + E /*pilo*/ + (E + R + 4) /*Bs: segments | per rank*/ + R /*jlo*/ +
-           2 * R /*nrr ridx*/ + E /*pof*/ + 3 * nh /*cexp ccnt cspare*/ + 3 * nh /*hr hs hq, then Z*/ +
+           R /*nrr*/ + E /*pof*/ + 3 * nh /*cexp ccnt cspare*/ + 3 * nh /*hr hs hq, then Z*/ +
            E /*flag*/ + 32 + 16;
 }
 
@@ -121,16 +125,13 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
     int *D = X + R;
     int *scr = D + R;              // E + R + 2
     int *pe = scr + E + R + 2;     // E   pieces: expert, sorted
-    int *pv = pe + E;              // E   pieces: shed, sorted
-    int *qr = pv + E;              // R   receivers: rank, sorted
-    int *qv = qr + R;              // R   receivers: deficit, sorted
-    int *A = qv + R;               // E + R + 4: PS (nP+1) then QS (nN+1)
+    int *qr = pe + E;              // R   receivers: rank, sorted
+    int *A = qr + R;               // E + R + 4: sorted sizes, then PS (nP+1) and QS (nN+1)
     int *pilo = A + E + R + 4;     // E   first receiver of piece j
     int *Bs = pilo + E;            // E + R + 4: segments per piece (nP+1) | replicas per rank (R+1)
     int *jlo = Bs + E + R + 4;     // R   first piece of receiver i
     int *nrr = jlo + R;            // R   replicas on rank r
-    int *ridx = nrr + R;           // R   receiver index of rank r, -1 if none
-    int *pof = ridx + R;           // E   piece index of expert e, -1 if none
+    int *pof = nrr + R;            // E   piece index of expert e, -1 if none
     int *cexp = pof + E;           // nh  compact used slots: expert
     int *ccnt = cexp + nh;         // nh  rows
     int *cspare = ccnt + nh;       // nh  receiver ids while sorting, then the rank of each used slot
@@ -217,7 +218,6 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
     for (int r = tid; r < R; r += nt) {
         scr[E + r] = D[r] > 0;
         nrr[r] = 0;
-        ridx[r] = -1;
     }
     __syncthreads();
 
@@ -257,11 +257,9 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
         if (lane == 0) {  // A = [pv..., 0, qv..., 0] for the prefix sums below
             if (piece) {
                 pe[pos] = id;
-                pv[pos] = v;
                 A[pos] = v;
             } else {
                 qr[pos] = id;
-                qv[pos] = v;
                 A[nP + 1 + pos] = v;
             }
         }
@@ -307,7 +305,6 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
                 jlo[i] = jl;
                 nrr[r] = jh - jl + 1;
                 rpr[r] = jh - jl + 1;
-                ridx[r] = i;
             }
         }
     }

@@ -93,8 +93,11 @@ extern "C" {
 /* A buffer row taken from the plan was outside [0, R*S*K) (a corrupted or
  * mismatched plan); that row access was skipped. */
 #define MOONEP_ST_ROW_RANGE 8
-/* A bounded wait inside a kernel (an mbarrier for a bulk copy) ran out of
- * iterations; the kernel stopped early and its output is incomplete. */
+/* A bounded wait inside a kernel ran out of iterations: the assignment
+ * pass's wait for the counts-ready mark of the histogram pass (about 6 ms at
+ * the bound).  The pass then waits for the whole histogram grid instead, so
+ * the plan is still complete; the bit reports that the mark never came,
+ * which points at a workspace used by two overlapping calls. */
 #define MOONEP_ST_WAIT_TIMEOUT 16
 /* The planner workspace did not hold the zeros a call must start from (it
  * was not zero-filled before first use, or two calls used it at once): the
@@ -266,6 +269,13 @@ MOONEP_API int moonep_plan_noalloc(const moonep_config *cfg, const int32_t *topk
 
 /* Human-readable text for a MOONEP_* return code. */
 MOONEP_API const char *moonep_error_string(int code);
+
+/* Human-readable text for a device status word (plan->info[MOONEP_INFO_STATUS],
+ * a set of MOONEP_ST_* bits): "ok" for 0, else the set bits' names joined by
+ * '|' (unknown bits as "bit<n>").  The text is written into buf (at most len
+ * bytes, always NUL-terminated when len > 0); the return value is buf, or an
+ * empty static string when buf is NULL or len == 0.  Host-only. */
+MOONEP_API const char *moonep_status_string(int status, char *buf, size_t len);
 
 /* MOONEP_ABI_VERSION of the loaded library. */
 MOONEP_API int moonep_abi_version(void);

@@ -112,6 +112,34 @@ const char *moonep_error_string(int code)
     }
 }
 
+const char *moonep_status_string(int status, char *buf, size_t len)
+{
+    static const char empty[1] = {0};
+    if (!buf || len == 0) return empty;
+    static const char *const names[6] = {"EXPERT_ID_RANGE", "OVERFLOW", "STRICT_VIOLATION",
+                                         "ROW_RANGE",       "WAIT_TIMEOUT", "WORKSPACE"};
+    size_t n = 0;
+    auto put = [&](const char *t) {
+        for (; *t && n + 1 < len; ++t) buf[n++] = *t;
+    };
+    if (status == 0) put("ok");
+    for (int b = 0; b < 32; ++b) {
+        if (!((unsigned)status & (1u << b))) continue;
+        if (n > 0) put("|");
+        if (b < 6) {
+            put(names[b]);
+        } else {
+            char t[8] = {'b', 'i', 't', 0, 0, 0, 0, 0};
+            t[3] = (char)('0' + b / 10);
+            t[4] = (char)('0' + b % 10);
+            if (b < 10) { t[3] = (char)('0' + b); t[4] = 0; }
+            put(t);
+        }
+    }
+    buf[n] = 0;
+    return buf;
+}
+
 int moonep_check_config(const moonep_config *c)
 {
     if (!c) return MOONEP_ERR_ARG;

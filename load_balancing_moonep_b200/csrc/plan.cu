@@ -573,7 +573,10 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
         s_ready = ok;
     }
     __syncthreads();
-    if (!s_ready) pdl_wait();
+    if (!s_ready) {  // complete either way; report that the mark came late
+        pdl_wait();
+        if (tid == 0) atomicOr(a.p.info + MOONEP_INFO_STATUS, MOONEP_ST_WAIT_TIMEOUT);
+    }
     const int seq = s_seq;
     if (tid == 0) {  // the last CTA past this point advances the sequence
         if (atomicAdd(a.hdr + WS_ARRIVED, 1) == (int)gridDim.x - 1) {

@@ -52,7 +52,7 @@ PLAN_FIELDS = ("expert_count", "slot_expert", "slot_count", "slot_offset", "rep_
 EXPORTED = ("moonep_check_config", "moonep_plan_sizes", "moonep_plan_layout", "moonep_plan",
             "moonep_dispatch", "moonep_combine", "moonep_combine_backward",
             "moonep_reduce_replica_grads", "moonep_error_string", "moonep_abi_version",
-            "moonep_plan_noalloc", "moonep_prefetch_replicas")
+            "moonep_plan_noalloc", "moonep_prefetch_replicas", "moonep_status_string")
 
 
 class _CConfig(ctypes.Structure):
@@ -80,9 +80,11 @@ _lib.moonep_plan_noalloc.argtypes = [_cfgp, _vp, _planp, _vp]
 _lib.moonep_prefetch_replicas.argtypes = [_cfgp, _planp, _vp, _vp, _vp, ctypes.c_int64, _vp]
 _lib.moonep_error_string.argtypes = [ctypes.c_int]
 _lib.moonep_error_string.restype = ctypes.c_char_p
+_lib.moonep_status_string.argtypes = [ctypes.c_int, ctypes.c_char_p, ctypes.c_size_t]
+_lib.moonep_status_string.restype = ctypes.c_char_p
 _lib.moonep_abi_version.argtypes = []
 for _f in EXPORTED:
-    if _f not in ("moonep_error_string",):
+    if _f not in ("moonep_error_string", "moonep_status_string"):
         getattr(_lib, _f).restype = ctypes.c_int
 
 LIB_PATH = _LIB_PATH
@@ -342,3 +344,9 @@ def views(cfg: Config, p: Plan, buf: torch.Tensor):
 
 def abi_version() -> int:
     return _lib.moonep_abi_version()
+
+
+def status_string(status: int) -> str:
+    """Names of the MOONEP_ST_* bits set in a plan's status word ("ok" for 0)."""
+    buf = ctypes.create_string_buffer(256)
+    return _lib.moonep_status_string(int(status), buf, len(buf)).decode()

@@ -78,3 +78,19 @@ def test_plan_sizes_and_layout(cuda_lib_path):
     assert offs[-1] < pb
     # misaligned base is rejected
     assert moonep._lib.moonep_plan_layout(ctypes.byref(c), base + 16, ctypes.byref(cp)) == 8
+
+
+def test_status_string(cuda_lib_path):
+    from load_balancing_moonep_b200 import moonep
+    assert moonep.status_string(0) == "ok"
+    assert moonep.status_string(moonep.ST_EXPERT_ID_RANGE) == "EXPERT_ID_RANGE"
+    assert moonep.status_string(moonep.ST_OVERFLOW | moonep.ST_STRICT_VIOLATION) == "OVERFLOW|STRICT_VIOLATION"
+    assert moonep.status_string(moonep.ST_WAIT_TIMEOUT | moonep.ST_WORKSPACE) == "WAIT_TIMEOUT|WORKSPACE"
+    assert moonep.status_string(moonep.ST_ROW_RANGE | (1 << 7) | (1 << 12)) == "ROW_RANGE|bit7|bit12"
+    import ctypes
+    lib = ctypes.CDLL(cuda_lib_path)
+    lib.moonep_status_string.restype = ctypes.c_char_p
+    lib.moonep_status_string.argtypes = [ctypes.c_int, ctypes.c_char_p, ctypes.c_size_t]
+    small = ctypes.create_string_buffer(6)
+    assert lib.moonep_status_string(3, small, 6) == b"EXPER"  # truncated, NUL-terminated
+    assert lib.moonep_status_string(3, None, 0) == b""

@@ -33,7 +33,6 @@ struct WsLayout {
     size_t gs;         // int32 [2][ngroups][E]: per-group expert counts, double-buffered
     size_t cc;         // int32 [nchunk][E]: per-chunk expert counts
     size_t host_dst0;  // int32 [2E+R]: rank*C + slot_offset - host_start per host
-    size_t used;       // int32 [R]: used slots of each rank
     size_t total;
 };
 // The call sequence number SEQ counts completed plan calls on a workspace; its
@@ -57,7 +56,6 @@ __host__ inline WsLayout ws_layout(const Dims &d)
     w.gs = o; o = align256(o + i4 * 2 * (size_t)d.ngroups * d.E);
     w.cc = o; o = align256(o + i4 * (size_t)d.nchunk * d.E);
     w.host_dst0 = o; o = align256(o + i4 * nh);
-    w.used = o; o = align256(o + i4 * d.R);
     w.total = o;
     return w;
 }

@@ -38,8 +38,10 @@
 //                     its base -- all of this while the planner CTA runs.
 //                     Only pass B waits for the grid: g = base + rank is the
 //                     pair's rank among all pairs of its expert, and the host
-//                     interval holding g gives the buffer row.  The CTAs also
-//                     fill the unused tails of the padded tables.
+//                     interval holding g gives the buffer row.  (The
+//                     histogram CTAs write the tables' empty defaults
+//                     before the planner writes over them, so no pass fills
+//                     the unused rest afterwards.)
 #include "common.cuh"
 
 namespace moonep {
@@ -60,8 +62,7 @@ struct PlanParams {
     int *gs;         // [2][ngroups][E]
     int *cc;         // [nchunk][E]
     int *host_dst0;  // [2E+R]
-    int *used;       // [R] used slots per rank (home, then replicas)
-    FastDiv fC, fE, fE1, fL;  // divisions by C, E, E + 1 and L
+    FastDiv fC, fL;  // divisions by C and L
 };
 
 // ints of dynamic shared memory used by the planner block
@@ -377,10 +378,7 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
         a.p.slot_count[(size_t)r * E + sl] = ccnt[x];
         a.p.slot_offset[(size_t)r * (E + 1) + sl] = Z[x] - Z[b0];
     }
-    for (int r = tid; r < R; r += nt) {
-        a.used[r] = L + nrr[r];
-        atomicMax(&misc[3], nrr[r]);
-    }
+    for (int r = tid; r < R; r += nt) atomicMax(&misc[3], nrr[r]);
     for (int e = tid; e <= E; e += nt) a.p.host_ptr[e] = hptr(e);
     for (int e = tid; e < E; e += nt) {
         if (flag[e]) a.p.rep_home_list[Z[zf + e] - zf0] = e;
@@ -462,6 +460,30 @@ __global__ void __launch_bounds__(PLAN_THREADS) hist_plan_kernel(PlanParams a)
     const int p0 = t0 * K, n = (t1 - t0) * K;
     int *hist = sm;       // E
     int *ids = sm + E;    // chunk_tokens * K
+    // this CTA's share of the tables' empty defaults (unused slots, replica
+    // and host entries); the planner CTA writes the used entries over them
+    // after every CTA's ticket, so no later pass fills the unused rest
+    {
+        const int R = d.R, nh = 2 * E + R;
+        const int g = gridDim.x * nt, x0 = blockIdx.x * nt + tid;
+        for (int x = x0; x < R * E; x += g) {
+            a.p.slot_expert[x] = -1;
+            a.p.slot_count[x] = 0;
+        }
+        for (int x = x0; x < R * (E + 1); x += g) a.p.slot_offset[x] = d.C;
+        for (int x = x0; x < E + R; x += g) {
+            a.p.rep_expert[x] = -1;
+            a.p.rep_rank[x] = -1;
+            a.p.rep_slot[x] = -1;
+            a.p.rep_quota[x] = 0;
+        }
+        for (int x = x0; x < nh; x += g) {
+            a.p.host_rank[x] = -1;
+            a.p.host_slot[x] = -1;
+            a.p.host_start[x] = 0;
+            a.p.host_quota[x] = 0;
+        }
+    }
     for (int e = tid; e < E; e += nt) hist[e] = 0;
     for (int i = tid; i < n; i += nt) ids[i] = __ldg(a.topk + p0 + i);  // all loads in flight
     if (tid == 0) s_seq = ld_cg(a.hdr + WS_SEQ);
@@ -640,7 +662,6 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
     // garbage cannot steer an access out of its array.
     pdl_wait();
     const int status = ld_cg(a.p.info + MOONEP_INFO_STATUS);
-    const int n_rep_raw = ld_cg(a.p.info + MOONEP_INFO_N_REP);
     // host tables of the whole array; only entries inside the clamped
     // [host_ptr[e], host_ptr[e+1]) are used
     for (int e = tid; e <= E; e += nt) hptr[e] = min(max(ld_cg(a.p.host_ptr + e), 0), nh);
@@ -649,47 +670,31 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
         hdst[h] = ld_cg(a.host_dst0 + h);
     }
     const bool empty = (status & ST_EMPTY_PLAN) != 0;
-    const int n_rep = empty ? 0 : min(max(n_rep_raw, 0), E + R - 1);
 
-    // ---- unused tails of the padded tables (the planner wrote the used
-    // slots), the replica and host lists, spread over the CTAs
-    {
+    // ---- an empty plan: every table empty, spread over the CTAs.  (For a
+    // plan, the histogram CTAs wrote the empty defaults before the planner
+    // wrote its entries over them.)
+    if (empty) {
         const int g = gridDim.x * nt, x0 = blockIdx.x * nt + tid;
         for (int x = x0; x < R * E; x += g) {
-            const int r = (int)fdiv((uint32_t)x, a.fE), s = x - r * E;
-            const int used = empty ? 0 : min(max(ld_cg(a.used + r), 0), E);
-            if (s >= used) {
-                a.p.slot_expert[x] = -1;
-                a.p.slot_count[x] = 0;
-            }
+            a.p.slot_expert[x] = -1;
+            a.p.slot_count[x] = 0;
         }
-        for (int x = x0; x < R * (E + 1); x += g) {
-            const int r = (int)fdiv((uint32_t)x, a.fE1), s = x - r * (E + 1);
-            const int used = empty ? 0 : min(max(ld_cg(a.used + r), 0), E);
-            if (s >= used) a.p.slot_offset[x] = empty ? 0 : C;  // an empty plan is all zeros
+        for (int x = x0; x < R * (E + 1); x += g) a.p.slot_offset[x] = 0;
+        for (int x = x0; x < E + R; x += g) {
+            a.p.rep_expert[x] = -1;
+            a.p.rep_rank[x] = -1;
+            a.p.rep_slot[x] = -1;
+            a.p.rep_quota[x] = 0;
         }
-        for (int x = x0; x < E + R; x += g)
-            if (x >= n_rep) {
-                a.p.rep_expert[x] = -1;
-                a.p.rep_rank[x] = -1;
-                a.p.rep_slot[x] = -1;
-                a.p.rep_quota[x] = 0;
-            }
-        const int hused = empty ? 0 : E + n_rep;
-        for (int x = x0; x < nh; x += g)
-            if (x >= hused) {
-                a.p.host_rank[x] = -1;
-                a.p.host_slot[x] = -1;
-                a.p.host_start[x] = 0;
-                a.p.host_quota[x] = 0;
-            }
-        if (empty) {
-            for (int x = x0; x <= E; x += g) a.p.host_ptr[x] = 0;
-            for (int x = x0; x < E; x += g) a.p.rep_home_list[x] = -1;
+        for (int x = x0; x < nh; x += g) {
+            a.p.host_rank[x] = -1;
+            a.p.host_slot[x] = -1;
+            a.p.host_start[x] = 0;
+            a.p.host_quota[x] = 0;
         }
-    }
-
-    if (empty) {
+        for (int x = x0; x <= E; x += g) a.p.host_ptr[x] = 0;
+        for (int x = x0; x < E; x += g) a.p.rep_home_list[x] = -1;
         for (int i = tid; i < n; i += nt) {
             a.p.dst_pos[p0 + i] = -1;
             a.p.row_src[p0 + i] = -1;
@@ -759,10 +764,7 @@ int launch_plan(const Dims &d, const int32_t *topk, const moonep_plan_t &p, void
     a.gs = reinterpret_cast<int *>(w + wl.gs);
     a.cc = reinterpret_cast<int *>(w + wl.cc);
     a.host_dst0 = reinterpret_cast<int *>(w + wl.host_dst0);
-    a.used = reinterpret_cast<int *>(w + wl.used);
     a.fC = make_fastdiv((uint32_t)d.C);
-    a.fE = make_fastdiv((uint32_t)d.E);
-    a.fE1 = make_fastdiv((uint32_t)(d.E + 1));
     a.fL = make_fastdiv((uint32_t)d.L);
 
     const size_t smem1 = sizeof(int) * (size_t)hist_smem_ints(d.E, d.R, d.chunk_tokens * d.K);

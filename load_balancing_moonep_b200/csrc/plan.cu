@@ -255,7 +255,7 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
             }
             pos += __popc(__ballot_sync(FULL_MASK, before));
         }
-        if (lane == 0) {  // A = [pv..., 0, qv..., 0] for the prefix sums below
+        if (lane == 0) {  // A = [sorted piece sizes, 0, sorted deficits, 0]
             if (piece) {
                 pe[pos] = id;
                 A[pos] = v;

@@ -200,6 +200,23 @@ def test_plan_alternating_routings_reuse_workspace(mp):
         _assert_plan_equal(p, ops[it % 2])
 
 
+def test_plan_many_chunks_multi_wave(mp):
+    """More token chunks (512, in 32 groups) than two CTAs per SM can hold at
+    once: both planner grids run in several waves, and assignment CTAs wait
+    for the counts-ready mark while later histogram CTAs still run.  The plan
+    must equal the oracle's."""
+    c = dict(R=64, E=256, K=8, S=4096, H=16, B=4, flags=0)
+    T = c["R"] * c["S"]
+    g = torch.Generator(device=DEV).manual_seed(7)
+    bias = -1.2 * torch.log(torch.randperm(c["E"], generator=g, device=DEV).float() + 1.0)
+    scores = torch.randn((T, c["E"]), generator=g, device=DEV) + bias
+    topk = torch.topk(scores, c["K"], dim=1).indices.to(torch.int32).cpu().numpy()
+    del scores
+    gcfg, ocfg, gp, op = _plan_both(mp, c, topk)
+    _assert_plan_equal(gp, op)
+    assert op["info"][1] > 0  # the skew made replicas
+
+
 def test_plan_in_cuda_graph_replays(mp):
     """The plan captured in a CUDA graph (its programmatic launch edge and
     counts-ready handshake replayed) with fresh routings written into the

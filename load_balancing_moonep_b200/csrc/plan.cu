@@ -115,8 +115,12 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
 {
     const Dims &d = a.d;
     const int E = d.E, R = d.R, L = d.L, C = d.C, B = d.B;
-    const int tid = threadIdx.x, nt = blockDim.x;
-    const int lane = tid & 31, warp = tid >> 5, nwarp = nt >> 5;
+    // the planner runs in the last histogram CTA: PLAN_THREADS threads, a
+    // compile-time stride for every loop below
+    const int tid = threadIdx.x;
+    constexpr int nt = PLAN_THREADS;
+    const int lane = tid & 31, warp = tid >> 5;
+    constexpr int nwarp = PLAN_THREADS / 32;
     const int nh = 2 * E + R;
 
     int *T = sm;
@@ -143,18 +147,18 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
     int *wsum = flag + E;          // 32
     int *misc = wsum + 32;         // 16: 0 status in, 2 n_over, 3 max replicas per rank
 
-    __shared__ long long s_part[32];
+    __shared__ unsigned s_part[2][32];
     for (int i = tid; i < 16; i += nt) misc[i] = 0;
-    if (tid == 0) {  // every other CTA has arrived: take the status, reset the header
-        misc[0] = ld_cg(a.hdr + WS_STATUS);
-        a.hdr[WS_STATUS] = 0;
-        a.hdr[WS_TICKET] = 0;
-    }
+    // every other CTA has arrived: take the status (the load is issued here
+    // and waited for after the totals' loads) and reset the header
+    int st_hdr = 0;
+    if (tid == 0) st_hdr = ld_cg(a.hdr + WS_STATUS);
     // ---- totals: the sum of this call's group counts (one atomic sum per
     // chunk and expert lands in a group of CHUNK_GROUP chunks, so no address
     // takes more than CHUNK_GROUP atomics; per-expert totals accumulated
     // by every CTA serialised some 300 atomics per address)
-    long long part = 0;
+    static_assert(MOONEP_MAX_E <= 2 * PLAN_THREADS, "at most two experts per planner thread");
+    unsigned part = 0;  // <= 2 values < 2^31 each (negative ones are flagged)
     int negative = 0;
     {
         const int *gsb = a.gs + (size_t)parity * d.ngroups * E;
@@ -163,17 +167,31 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
             T[e] = v;
             a.p.expert_count[e] = v;
             negative |= v < 0;
-            part += v;
+            part += (unsigned)v;
         }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(FULL_MASK, part, o);
-    if ((tid & 31) == 0) s_part[tid >> 5] = part;
+    if (tid == 0) {
+        misc[0] = st_hdr;
+        a.hdr[WS_STATUS] = 0;
+        a.hdr[WS_TICKET] = 0;
+    }
+    // exact 64-bit total from 16-bit halves, each warp sum by one reduction
+    {
+        const unsigned lo = __reduce_add_sync(FULL_MASK, part & 0xffffu);
+        const unsigned hi = __reduce_add_sync(FULL_MASK, part >> 16);
+        if (lane == 0) {
+            s_part[0][warp] = lo;
+            s_part[1][warp] = hi;
+        }
+    }
     negative = __syncthreads_or(negative);
     int status_in = misc[0];
-    long long total = (tid & 31) < (nt >> 5) ? s_part[tid & 31] : 0;  // one load per lane
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) total += __shfl_xor_sync(FULL_MASK, total, o);
+    long long total;
+    {
+        const unsigned lo = __reduce_add_sync(FULL_MASK, lane < nwarp ? s_part[0][lane] : 0u);
+        const unsigned hi = __reduce_add_sync(FULL_MASK, lane < nwarp ? s_part[1][lane] : 0u);
+        total = ((long long)hi << 16) + (long long)lo;
+    }
     // with every id valid the totals must be non-negative and add up to the
     // number of pairs; anything else means the workspace was not zeroed
     if (!(status_in & MOONEP_ST_EXPERT_ID_RANGE) && (negative || total != (long long)d.pairs))

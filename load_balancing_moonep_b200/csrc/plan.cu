@@ -71,7 +71,7 @@ __host__ __device__ inline int plan_smem_ints(int E, int R)
     const int nh = 2 * E + R;
     return 3 * E /*T shed keep*/ + 2 * R /*X D*/ + (E + R + 2) /*scr*/ + E /*pe*/ + R /*qr*/ +
            (E + R + 4) /*A: PS | QS*/ + E /*pilo*/ + (E + R + 4) /*Bs: segments | per rank*/ + R /*jlo*/ +
-           R /*nrr*/ + E /*pof*/ + 3 * nh /*cexp ccnt cspare*/ + 3 * nh /*hr hs hq, then Z*/ +
+           E /*pof*/ + 3 * nh /*cexp ccnt cspare*/ + 3 * nh /*hr hs hq, then Z*/ +
            E /*flag*/ + 32 + 16;
 }
 
@@ -135,8 +135,7 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
     int *pilo = A + E + R + 4;     // E   first receiver of piece j
     int *Bs = pilo + E;            // E + R + 4: segments per piece (nP+1) | replicas per rank (R+1)
     int *jlo = Bs + E + R + 4;     // R   first piece of receiver i
-    int *nrr = jlo + R;            // R   replicas on rank r
-    int *pof = nrr + R;            // E   piece index of expert e, -1 if none
+    int *pof = jlo + R;            // E   piece index of expert e, -1 if none
     int *cexp = pof + E;           // nh  compact used slots: expert
     int *ccnt = cexp + nh;         // nh  rows
     int *cspare = ccnt + nh;       // nh  receiver ids while sorting, then the rank of each used slot
@@ -234,10 +233,7 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
         scr[e] = s > 0;
         pof[e] = -1;
     }
-    for (int r = tid; r < R; r += nt) {
-        scr[E + r] = D[r] > 0;
-        nrr[r] = 0;
-    }
+    for (int r = tid; r < R; r += nt) scr[E + r] = D[r] > 0;
     __syncthreads();
 
     // ---- compact pieces and receivers with one scan over [E experts | R ranks]
@@ -322,8 +318,8 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
             if (lane == 0) {
                 const int r = qr[i];
                 jlo[i] = jl;
-                nrr[r] = jh - jl + 1;
                 rpr[r] = jh - jl + 1;
+                atomicMax(&misc[3], jh - jl + 1);  // read after later barriers
             }
         }
     }
@@ -339,10 +335,12 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
     //   Z = [rows of each used slot (E + n_rep) | hosts per expert (E) | 0 |
     //        prefetched-replica flag per expert (E) | 0]
     // Rank r's used slots sit at rank_base(r) .. (home slots, then replicas).
-    int *Z = hr;  // 4E + R + 2 <= 3 nh ints, free after the sort
+    int *Z = hr;     // 4E + R + 2 <= 3 nh ints, free after the sort
+    int *rq_j = scr;  // n_rep <= E + R - 1: piece of each replica (scr is free)
     const int zh = E + n_rep, zf = zh + E + 1, nz = zf + E + 1;
     for (int q = tid; q < n_rep; q += nt) {
         const int j = last_le(segb, nP, q);
+        rq_j[q] = j;
         const int i = pilo[j] + (q - segb[j]);
         const int ord = j - jlo[i];
         const int r = qr[i];
@@ -390,17 +388,21 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
     const int n_hosts = E + n_rep;                  // == Z[zh + E] - zh0
     const int n_rep_experts = Z[zf + E] - zf0;
     auto hptr = [&](int e) { return Z[zh + e] - zh0; };
-    for (int x = tid; x < E + n_rep; x += nt) {  // used slots into the padded [R][E] tables
-        const int r = cspare[x], b0 = rank_base(r), sl = x - b0;
-        a.p.slot_expert[(size_t)r * E + sl] = cexp[x];
-        a.p.slot_count[(size_t)r * E + sl] = ccnt[x];
-        a.p.slot_offset[(size_t)r * (E + 1) + sl] = Z[x] - Z[b0];
-    }
-    for (int r = tid; r < R; r += nt) atomicMax(&misc[3], nrr[r]);
-    for (int e = tid; e <= E; e += nt) a.p.host_ptr[e] = hptr(e);
-    for (int e = tid; e < E; e += nt) {
-        if (flag[e]) a.p.rep_home_list[Z[zf + e] - zf0] = e;
-        if (e >= n_rep_experts) a.p.rep_home_list[e] = -1;
+    // one pass writes the used slots into the padded [R][E] tables, the host
+    // pointers, the reduce work list and (below) the host intervals: x runs
+    // over max(E + n_rep, E + 1) = n_hosts + (n_rep == 0) entries
+    for (int x = tid; x <= n_hosts; x += nt) {
+        if (x < E + n_rep) {
+            const int r = cspare[x], b0 = rank_base(r), sl = x - b0;
+            a.p.slot_expert[(size_t)r * E + sl] = cexp[x];
+            a.p.slot_count[(size_t)r * E + sl] = ccnt[x];
+            a.p.slot_offset[(size_t)r * (E + 1) + sl] = Z[x] - Z[b0];
+        }
+        if (x <= E) a.p.host_ptr[x] = hptr(x);
+        if (x < E) {
+            if (flag[x]) a.p.rep_home_list[Z[zf + x] - zf0] = x;
+            if (x >= n_rep_experts) a.p.rep_home_list[x] = -1;
+        }
     }
     // ---- host intervals: the hosts of e in ascending rank; a host's start
     // is the rows of the hosts of e on lower ranks
@@ -414,7 +416,7 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
             j = pof[e];
         } else {
             const int q = x - E;
-            j = last_le(segb, nP, q);
+            j = rq_j[q];
             const int i = pilo[j] + (q - segb[j]);
             e = pe[j];
             r0 = qr[i];

@@ -93,11 +93,12 @@ extern "C" {
 /* A buffer row taken from the plan was outside [0, R*S*K) (a corrupted or
  * mismatched plan); that row access was skipped. */
 #define MOONEP_ST_ROW_RANGE 8
-/* A bounded wait inside a kernel ran out of iterations: the assignment
- * pass's wait for the counts-ready mark of the histogram pass (about 6 ms at
- * the bound).  The pass then waits for the whole histogram grid instead, so
- * the plan is still complete; the bit reports that the mark never came,
- * which points at a workspace used by two overlapping calls. */
+/* A bounded wait inside a kernel ran out of iterations: one of the
+ * assignment pass's waits for a mark of the histogram/planner pass (counts
+ * ready, plan ready; about 6 ms at the bound).  The pass then waits for the
+ * whole histogram grid instead, so the plan is still complete; the bit
+ * reports that a mark never came, which points at a workspace used by two
+ * overlapping calls. */
 #define MOONEP_ST_WAIT_TIMEOUT 16
 /* The planner workspace did not hold the zeros a call must start from (it
  * was not zero-filled before first use, or two calls used it at once): the

@@ -111,8 +111,9 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 
 // ------------------------------------------------------------- planner CTA
 
-__device__ void plan_block(const PlanParams &a, int *sm, int parity)
+__device__ void plan_block(const PlanParams &a, int *sm, int seq)
 {
+    const int parity = seq & 1;
     const Dims &d = a.d;
     const int E = d.E, R = d.R, L = d.L, C = d.C, B = d.B;
     // the planner runs in the last histogram CTA: PLAN_THREADS threads, a
@@ -199,6 +200,8 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
         if (tid == 0) {
             a.p.info[MOONEP_INFO_STATUS] = status_in;
             for (int i = 1; i < MOONEP_INFO_LEN; ++i) a.p.info[i] = 0;
+            __threadfence();
+            st_release(a.hdr + WS_PLANNED, seq + 1);
         }
         return;  // the assignment pass writes the empty tables
     }
@@ -462,6 +465,12 @@ __device__ void plan_block(const PlanParams &a, int *sm, int parity)
         a.p.info[MOONEP_INFO_N_REP_EXPERTS] = n_rep_experts;
         for (int i = MOONEP_INFO_N_REMOTE_PAIRS; i < MOONEP_INFO_LEN; ++i) a.p.info[i] = 0;
     }
+    // every thread's plan writes precede the plan-ready mark
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        st_release(a.hdr + WS_PLANNED, seq + 1);
+    }
 }
 
 __global__ void __launch_bounds__(PLAN_THREADS) hist_plan_kernel(PlanParams a)
@@ -541,7 +550,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) hist_plan_kernel(PlanParams a)
     }
     __syncthreads();
     if (!s_last) return;
-    plan_block(a, sm, parity);
+    plan_block(a, sm, seq);
 }
 
 // ---------------------------------------------------------- assignment
@@ -565,7 +574,7 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
     int *hstart = hptr + E + 1;            // nh
     int *hdst = hstart + nh;               // nh
     int *red = hdst + nh;                  // 32
-    __shared__ int s_seq, s_ready;
+    __shared__ int s_seq, s_ready, s_planned;
 
     // prologue on inputs only, overlapping the histogram/planner grid
     for (int i = tid; i < ASSIGN_WARPS * E; i += nt) cnt[i] = 0;
@@ -676,11 +685,28 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
         }
     }
 
-    // ---- the plan: the histogram/planner grid has completed.  Every load
-    // below is issued before any of its results is used (one round trip),
-    // and every count or index read back is clamped, so even a plan block of
-    // garbage cannot steer an access out of its array.
-    pdl_wait();
+    // ---- the plan is complete once the planner CTA has set PLANNED (a
+    // bounded wait, as for READY: the planner CTA is resident, and the grid
+    // dependency implies the mark).  Every load below is issued before any
+    // of its results is used (one round trip), and every count or index read
+    // back is clamped, so even a plan block of garbage cannot steer an
+    // access out of its array.
+    if (tid == 0) {
+        int ok = 0;
+        for (int it = 0; it < READY_SPIN_LIMIT; ++it) {
+            if (ld_acquire(a.hdr + WS_PLANNED) == seq + 1) {
+                ok = 1;
+                break;
+            }
+            __nanosleep(64);
+        }
+        s_planned = ok;
+    }
+    __syncthreads();
+    if (!s_planned) {
+        pdl_wait();
+        if (tid == 0) atomicOr(a.p.info + MOONEP_INFO_STATUS, MOONEP_ST_WAIT_TIMEOUT);
+    }
     const int status = ld_cg(a.p.info + MOONEP_INFO_STATUS);
     // host tables of the whole array; only entries inside the clamped
     // [host_ptr[e], host_ptr[e+1]) are used

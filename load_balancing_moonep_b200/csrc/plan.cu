@@ -479,8 +479,13 @@ __global__ void __launch_bounds__(PLAN_THREADS) hist_plan_kernel(PlanParams a)
     __shared__ int s_last, s_seq;
     const Dims &d = a.d;
     const int E = d.E, K = d.K, tid = threadIdx.x, nt = blockDim.x;
+    // launched with programmatic dependent launch after whatever the stream
+    // ran before (the router, or the last reader of this plan): its CTAs may
+    // be placed while that kernel drains, and wait here for its completion
+    // before touching any memory
+    pdl_wait();
     // the assignment kernel may be scheduled now: it reads the counts after
-    // the READY mark and the plan after this whole grid has completed
+    // the READY mark and the plan after the PLANNED mark
     pdl_launch_dependents();
 
     const int chunk = blockIdx.x;
@@ -813,24 +818,30 @@ int launch_plan(const Dims &d, const int32_t *topk, const moonep_plan_t &p, void
     a.fC = make_fastdiv((uint32_t)d.C);
     a.fL = make_fastdiv((uint32_t)d.L);
 
-    const size_t smem1 = sizeof(int) * (size_t)hist_smem_ints(d.E, d.R, d.chunk_tokens * d.K);
-    if (!set_smem((const void *)hist_plan_kernel, smem1)) return MOONEP_ERR_CUDA;
-    hist_plan_kernel<<<d.nchunk, PLAN_THREADS, smem1, st>>>(a);
-    if (cudaGetLastError() != cudaSuccess) return MOONEP_ERR_CUDA;
-
-    const size_t smem2 = sizeof(int) * (size_t)assign_smem_ints(d.E, d.R, d.chunk_tokens * d.K);
-    if (!set_smem((const void *)assign_kernel, smem2)) return MOONEP_ERR_CUDA;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(d.nchunk);
-    cfg.blockDim = dim3(ASSIGN_THREADS);
-    cfg.dynamicSmemBytes = smem2;
-    cfg.stream = st;
+    // both kernels with programmatic dependent launch: each may be placed
+    // while its predecessor drains and waits (griddepcontrol.wait, or the
+    // marks) before it reads anything the predecessor writes
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, assign_kernel, a) != cudaSuccess) return MOONEP_ERR_CUDA;
+
+    const size_t smem1 = sizeof(int) * (size_t)hist_smem_ints(d.E, d.R, d.chunk_tokens * d.K);
+    if (!set_smem((const void *)hist_plan_kernel, smem1)) return MOONEP_ERR_CUDA;
+    cudaLaunchConfig_t c1 = {};
+    c1.gridDim = dim3(d.nchunk);
+    c1.blockDim = dim3(PLAN_THREADS);
+    c1.dynamicSmemBytes = smem1;
+    c1.stream = st;
+    c1.attrs = attr;
+    c1.numAttrs = 1;
+    if (cudaLaunchKernelEx(&c1, hist_plan_kernel, a) != cudaSuccess) return MOONEP_ERR_CUDA;
+
+    const size_t smem2 = sizeof(int) * (size_t)assign_smem_ints(d.E, d.R, d.chunk_tokens * d.K);
+    if (!set_smem((const void *)assign_kernel, smem2)) return MOONEP_ERR_CUDA;
+    cudaLaunchConfig_t c2 = c1;
+    c2.blockDim = dim3(ASSIGN_THREADS);
+    c2.dynamicSmemBytes = smem2;
+    if (cudaLaunchKernelEx(&c2, assign_kernel, a) != cudaSuccess) return MOONEP_ERR_CUDA;
     return MOONEP_OK;
 }
 

@@ -66,10 +66,15 @@ extern "C" {
 #define MOONEP_FLAG_TRAIN_B_RULE 2u
 /* combine_backward dispatches dy unscaled instead of w * dy. */
 #define MOONEP_FLAG_BWD_UNSCALED 4u
+/* Reserved for the relay cascade, which keeps ranks that water-filling
+ * leaves over the budget B within it (defined by the test oracle); this
+ * library version does not implement it and returns MOONEP_ERR_ARG, as for
+ * any other unknown flag bit. */
+#define MOONEP_FLAG_CASCADE 8u
 
 /* ---- host return codes ------------------------------------------------- */
 #define MOONEP_OK 0
-#define MOONEP_ERR_ARG 1            /* null pointer, non-positive size, K > E, R*S*K >= 2^31 */
+#define MOONEP_ERR_ARG 1            /* null pointer, non-positive size, K > E, R*S*K >= 2^31, unsupported flag */
 #define MOONEP_ERR_E_NOT_DIVISIBLE 2 /* E % R != 0 (the explainer flags it) */
 #define MOONEP_ERR_BUDGET_RULE 3    /* TRAIN_B_RULE set and B != E/R */
 #define MOONEP_ERR_B_RANGE 4        /* B < 0 or B > E - L */

@@ -27,6 +27,7 @@ _LIB = os.path.join(_HERE, "libmoonep_oracle.so")
 FLAG_STRICT_BUDGET = 1
 FLAG_TRAIN_B_RULE = 2
 FLAG_BWD_UNSCALED = 4
+FLAG_CASCADE = 8
 
 ST_EXPERT_ID_RANGE = 1
 ST_OVERFLOW = 2

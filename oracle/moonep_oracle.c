@@ -43,6 +43,8 @@
  *      receiver i's interval is one replica of expert e(p_j) on rank r(q_i),
  *      created in (j, i) order; a rank's replicas take slots L, L+1, ... in
  *      creation order; ordinal >= B means overflow (read-through);
+ *   O5b (only with the cascade flag, and only when O5 left a rank with more
+ *      than B replicas) relay cascade, described at or_cascade below;
  *   O6 per-rank slot tables (home slots 0..L-1, then replicas);
  *   O7 per-expert host intervals, hosts in ascending rank order;
  *   O8 pairs in global (t, k) order fill their expert's host intervals.
@@ -60,6 +62,7 @@
 #define OR_FLAG_STRICT_BUDGET 1u
 #define OR_FLAG_TRAIN_B_RULE 2u
 #define OR_FLAG_BWD_UNSCALED 4u
+#define OR_FLAG_CASCADE 8u
 
 #define OR_ST_EXPERT_ID_RANGE 1
 #define OR_ST_OVERFLOW 2
@@ -123,6 +126,8 @@ int or_check_config(const or_config *c)
         return OR_ERR_ARG;
     if (c->K > c->E) return OR_ERR_ARG;
     if ((int64_t)c->R * c->S * c->K > INT32_MAX) return OR_ERR_ARG;
+    if (c->flags & ~(OR_FLAG_STRICT_BUDGET | OR_FLAG_TRAIN_B_RULE | OR_FLAG_BWD_UNSCALED | OR_FLAG_CASCADE))
+        return OR_ERR_ARG;
     /* the explainer flags E % R != 0 as a configuration error [P1 explainer] */
     if (c->E % c->R != 0) return OR_ERR_E_NOT_DIVISIBLE;
     int32_t L = c->E / c->R;
@@ -155,6 +160,173 @@ static int cmp_host_rank(const void *a, const void *b)
 
 static int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
 static int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
+
+/* O5b, relay cascade.  The pages require at most B = E/R prefetched replica
+ * slots per rank in training [P1 explainer, memory tab] and give no
+ * algorithm; water-filling can exceed B when a rank with a large deficit is
+ * filled from many small pieces.  This step repairs such ranks one at a
+ * time, always the rank with the most replicas (ties: lowest rank) among
+ * those over B and not yet closed:
+ *   - its replicas are ordered by (quota desc, list position asc); for the
+ *     smallest m in 0..B it keeps the first B-m and moves the rest (total
+ *     Q) away, provided the providers can carry Q.  The providers are, in
+ *     order, the kept replicas (each can grow by its expert's remaining home
+ *     quota keep[e], unless its home rank is closed) and then m relay
+ *     experts: those with keep > 0 whose home rank is not this rank, not
+ *     closed and not already a relay home, and that have no replica on this
+ *     rank, taken in (keep desc, expert asc) order;
+ *   - Q is poured into the providers in that order, each taking min(its
+ *     capacity, what is left): a kept replica's quota grows, a relay becomes
+ *     a new replica on this rank (appended to the list), and the provider's
+ *     home keeps that much less;
+ *   - the moved quotas are water-filled, in the moved order, into the
+ *     providers' home ranks in provider order (capacity = what each took):
+ *     an amount of expert e landing on e's own home returns to keep[e]; on a
+ *     rank that already holds a replica of e it is added to that replica;
+ *     otherwise it is a new replica appended to the list;
+ *   - the rank is closed.  A rank no m works for is closed unchanged.
+ * Every step keeps every rank's total at C and every expert's hosts summing
+ * to T[e]; it closes one rank, so there are at most R steps.  A step adds at
+ * most m + B - 1 live replicas (the relays, and the water-fill's splits
+ * beyond the moved replicas it replaces); a step for which the live count
+ * plus m + B - 1 would exceed cap is not taken (the rank is closed over B),
+ * so the list never outgrows the plan's replica arrays.  Replicas keep list
+ * order (dead entries are dropped after each step); ordinals are re-derived
+ * by the caller.  re/rr/rq/alive: list arrays of capacity
+ * lcap >= 2 * cap + 2 * B + 2; *nl: entries used. */
+static int or_cascade(int32_t R, int32_t E, int32_t L, int32_t B, int32_t cap, int32_t *keep,
+                      int32_t *re, int32_t *rr, int32_t *rq, int32_t *alive, int32_t *nl, int32_t lcap)
+{
+    int32_t *cnt = calloc((size_t)R, sizeof(int32_t));
+    int32_t *closed = calloc((size_t)R, sizeof(int32_t));
+    int32_t *on_r = calloc((size_t)E, sizeof(int32_t));
+    int32_t *home_used = calloc((size_t)R, sizeof(int32_t));
+    vi_t *S = calloc((size_t)lcap, sizeof(vi_t));
+    vi_t *cand = calloc((size_t)E, sizeof(vi_t));
+    int32_t *pe = calloc((size_t)lcap + B + 1, sizeof(int32_t));   /* provider expert */
+    int32_t *pq = calloc((size_t)lcap + B + 1, sizeof(int32_t));   /* kept replica index, -1 for a relay */
+    int32_t *pa = calloc((size_t)lcap + B + 1, sizeof(int32_t));   /* amount taken */
+    int32_t *sv_e = calloc((size_t)lcap, sizeof(int32_t)), *sv_q = calloc((size_t)lcap, sizeof(int32_t));
+    int rc = OR_OK;
+    if (!cnt || !closed || !on_r || !home_used || !S || !cand || !pe || !pq || !pa || !sv_e || !sv_q) {
+        rc = OR_ERR_NOMEM;
+        goto done;
+    }
+    for (;;) {
+        for (int32_t r = 0; r < R; ++r) cnt[r] = 0;
+        for (int32_t q = 0; q < *nl; ++q)
+            if (alive[q]) cnt[rr[q]] += 1;
+        int32_t rs = -1;
+        for (int32_t r = 0; r < R; ++r)
+            if (!closed[r] && cnt[r] > B && (rs < 0 || cnt[r] > cnt[rs])) rs = r;
+        if (rs < 0) break;
+        /* the rank's replicas by (quota desc, list position asc) */
+        int32_t n = 0;
+        for (int32_t e = 0; e < E; ++e) on_r[e] = 0;
+        for (int32_t q = 0; q < *nl; ++q)
+            if (alive[q] && rr[q] == rs) { S[n].val = rq[q]; S[n].idx = q; ++n; on_r[re[q]] = 1; }
+        qsort(S, (size_t)n, sizeof(vi_t), cmp_val_desc_idx_asc);
+        /* relay candidates by (keep desc, expert asc) */
+        int32_t nc = 0;
+        for (int32_t e = 0; e < E; ++e) {
+            const int32_t h = e / L;
+            if (keep[e] > 0 && h != rs && !closed[h] && !on_r[e]) { cand[nc].val = keep[e]; cand[nc].idx = e; ++nc; }
+        }
+        qsort(cand, (size_t)nc, sizeof(vi_t), cmp_val_desc_idx_asc);
+        /* the smallest m whose providers carry the moved quota */
+        int32_t m_found = -1, np = 0;
+        int64_t Q = 0;
+        for (int32_t m = 0; m <= B && m_found < 0; ++m) {
+            Q = 0;
+            for (int32_t k = B - m; k < n; ++k) Q += S[k].val;
+            int64_t room = 0;
+            np = 0;
+            for (int32_t k = 0; k < B - m; ++k) {
+                const int32_t e = re[S[k].idx];
+                pe[np] = e;
+                pq[np] = S[k].idx;
+                room += closed[e / L] ? 0 : keep[e];
+                ++np;
+            }
+            for (int32_t r = 0; r < R; ++r) home_used[r] = 0;
+            int32_t got = 0;
+            for (int32_t c = 0; c < nc && got < m; ++c) {
+                const int32_t h = cand[c].idx / L;
+                if (home_used[h]) continue;
+                home_used[h] = 1;
+                pe[np] = cand[c].idx;
+                pq[np] = -1;
+                room += cand[c].val;
+                ++np;
+                ++got;
+            }
+            if (got < m) break; /* fewer distinct relay homes than m: no larger m works either */
+            if (room >= Q) m_found = m;
+        }
+        closed[rs] = 1;
+        if (m_found < 0) continue;
+        if (*nl + m_found + B - 1 > cap) continue; /* the list could outgrow the plan's arrays */
+        /* the moved replicas' experts and quotas, before anything changes */
+        for (int32_t k = 0; k < n; ++k) { sv_e[k] = re[S[k].idx]; sv_q[k] = rq[S[k].idx]; }
+        int overfull = 0;
+        /* pour Q into the providers */
+        int64_t rem = Q;
+        for (int32_t k = 0; k < np; ++k) {
+            const int32_t e = pe[k];
+            const int64_t capk = (pq[k] >= 0 && closed[e / L] && e / L != rs) ? 0 : keep[e];
+            const int64_t amt = min64(capk, rem);
+            pa[k] = (int32_t)amt;
+            rem -= amt;
+            if (amt <= 0) continue;
+            keep[e] -= (int32_t)amt;
+            if (pq[k] >= 0) {
+                rq[pq[k]] += (int32_t)amt;
+            } else if (*nl < lcap) {
+                re[*nl] = e; rr[*nl] = rs; rq[*nl] = (int32_t)amt; alive[*nl] = 1; *nl += 1;
+            } else {
+                overfull = 1;
+            }
+        }
+        /* the moved replicas leave this rank ... */
+        const int32_t k0 = B - m_found;
+        for (int32_t k = k0; k < n; ++k) alive[S[k].idx] = 0;
+        /* ... and are water-filled into the providers' homes */
+        int32_t mk = k0, pi = 0;
+        int64_t a_left = mk < n ? sv_q[mk] : 0, c_left = np > 0 ? pa[0] : 0;
+        while (!overfull && mk < n && pi < np) {
+            if (c_left <= 0) { ++pi; c_left = pi < np ? pa[pi] : 0; continue; }
+            if (a_left <= 0) { ++mk; a_left = mk < n ? sv_q[mk] : 0; continue; }
+            const int64_t amt = min64(a_left, c_left);
+            const int32_t ek = sv_e[mk], h = pe[pi] / L;
+            if (ek / L == h) {
+                keep[ek] += (int32_t)amt;
+            } else {
+                int32_t found = -1;
+                for (int32_t q = 0; q < *nl; ++q)
+                    if (alive[q] && re[q] == ek && rr[q] == h) { found = q; break; }
+                if (found >= 0) {
+                    rq[found] += (int32_t)amt;
+                } else if (*nl < lcap) {
+                    re[*nl] = ek; rr[*nl] = h; rq[*nl] = (int32_t)amt; alive[*nl] = 1; *nl += 1;
+                } else {
+                    overfull = 1;
+                }
+            }
+            a_left -= amt;
+            c_left -= amt;
+        }
+        if (overfull) { rc = OR_ERR_ARG; goto done; } /* cannot happen: lcap covers a step */
+        /* drop the dead entries, keeping list order */
+        int32_t w = 0;
+        for (int32_t q = 0; q < *nl; ++q)
+            if (alive[q]) { re[w] = re[q]; rr[w] = rr[q]; rq[w] = rq[q]; alive[w] = 1; ++w; }
+        *nl = w;
+    }
+done:
+    free(cnt); free(closed); free(on_r); free(home_used); free(S); free(cand); free(pe); free(pq); free(pa);
+    free(sv_e); free(sv_q);
+    return rc;
+}
 
 /*
  * Array sizes (all int32, caller-allocated):
@@ -270,6 +442,42 @@ int or_plan(const or_config *c, const int32_t *topk,
             rep_quota[nrep] = (int32_t)len;
             nrep_on[r] += 1;
             ++nrep;
+        }
+    }
+
+    /* O5b: relay cascade, only with the flag and only over the budget */
+    if ((c->flags & OR_FLAG_CASCADE) && B > 0) {
+        int32_t mx = 0;
+        for (int32_t r = 0; r < R; ++r)
+            if (nrep_on[r] > mx) mx = nrep_on[r];
+        if (mx > B) {
+            const int32_t lcap = 2 * NREP_MAX + 2 * B + 2;
+            int32_t *le = calloc((size_t)lcap, sizeof(int32_t)), *lr = calloc((size_t)lcap, sizeof(int32_t));
+            int32_t *lq = calloc((size_t)lcap, sizeof(int32_t)), *la = calloc((size_t)lcap, sizeof(int32_t));
+            if (!le || !lr || !lq || !la) {
+                free(le); free(lr); free(lq); free(la);
+                rc = OR_ERR_NOMEM;
+                goto out;
+            }
+            for (int32_t q = 0; q < nrep; ++q) { le[q] = rep_expert[q]; lr[q] = rep_rank[q]; lq[q] = rep_quota[q]; la[q] = 1; }
+            int32_t nl = nrep;
+            rc = or_cascade(R, E, L, B, NREP_MAX - 1, keep, le, lr, lq, la, &nl, lcap);
+            if (rc == OR_OK) {
+                /* the final list, ordinals re-derived in list order */
+                for (int32_t r = 0; r < R; ++r) nrep_on[r] = 0;
+                for (int32_t q = 0; q < NREP_MAX; ++q) { rep_expert[q] = -1; rep_rank[q] = -1; rep_slot[q] = -1; rep_quota[q] = 0; }
+                for (int32_t q = 0; q < nl; ++q) {
+                    rep_expert[q] = le[q];
+                    rep_rank[q] = lr[q];
+                    rep_quota[q] = lq[q];
+                    rep_ord[q] = nrep_on[lr[q]];
+                    rep_slot[q] = L + nrep_on[lr[q]];
+                    nrep_on[lr[q]] += 1;
+                }
+                nrep = nl;
+            }
+            free(le); free(lr); free(lq); free(la);
+            if (rc != OR_OK) goto out;
         }
     }
 

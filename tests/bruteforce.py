@@ -72,6 +72,21 @@ def min_replicas(T, R, L, C, max_size=None) -> int:
     return -1
 
 
+def feasible_within_budget(T, R, L, C, B) -> bool:
+    """Whether some replica set with at most B replicas on every rank gives
+    every rank exactly C slots (sets enumerated by increasing size)."""
+    E = len(T)
+    cand = [(e, r) for e in range(E) for r in range(R) if r != e // L and T[e] > 0]
+    for k in range(len(cand) + 1):
+        for combo in itertools.combinations(cand, k):
+            per = [0] * R
+            for _, r in combo:
+                per[r] += 1
+            if max(per) <= B and feasible(T, R, L, C, combo):
+                return True
+    return False
+
+
 def min_cover_count(values, target) -> int:
     """Fewest of ``values`` whose sum reaches ``target`` (brute force)."""
     if target <= 0:

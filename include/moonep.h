@@ -66,15 +66,19 @@ extern "C" {
 #define MOONEP_FLAG_TRAIN_B_RULE 2u
 /* combine_backward dispatches dy unscaled instead of w * dy. */
 #define MOONEP_FLAG_BWD_UNSCALED 4u
-/* Reserved for the relay cascade, which keeps ranks that water-filling
- * leaves over the budget B within it (defined by the test oracle); this
- * library version does not implement it and returns MOONEP_ERR_ARG, as for
- * any other unknown flag bit. */
+/* Relay cascade: when water-filling leaves a rank with more than B
+ * replicas, repair such ranks one at a time (most replicas first): the rank
+ * keeps its B - m largest replicas, grows them and adds m relay replicas of
+ * other ranks' experts to carry the rest, and the moved replicas go to the
+ * providers' home ranks, which may in turn be repaired.  Within the budget
+ * the plan is exactly water-filling's.  Costs a larger planner shared-memory
+ * allocation (MOONEP_ERR_LIMIT if it does not fit) and a serial slow path
+ * when it runs.  Unknown flag bits are MOONEP_ERR_ARG. */
 #define MOONEP_FLAG_CASCADE 8u
 
 /* ---- host return codes ------------------------------------------------- */
 #define MOONEP_OK 0
-#define MOONEP_ERR_ARG 1            /* null pointer, non-positive size, K > E, R*S*K >= 2^31, unsupported flag */
+#define MOONEP_ERR_ARG 1            /* null pointer, non-positive size, K > E, R*S*K >= 2^31, unknown flag bit */
 #define MOONEP_ERR_E_NOT_DIVISIBLE 2 /* E % R != 0 (the explainer flags it) */
 #define MOONEP_ERR_BUDGET_RULE 3    /* TRAIN_B_RULE set and B != E/R */
 #define MOONEP_ERR_B_RANGE 4        /* B < 0 or B > E - L */

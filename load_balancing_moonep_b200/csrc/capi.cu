@@ -100,8 +100,7 @@ const char *moonep_error_string(int code)
     switch (code) {
     case MOONEP_OK: return "ok";
     case MOONEP_ERR_ARG:
-        return "invalid argument (null pointer, non-positive size, K > E, R*S*K >= 2^31, or a flag this "
-               "library does not implement)";
+        return "invalid argument (null pointer, non-positive size, K > E, R*S*K >= 2^31, or an unknown flag bit)";
     case MOONEP_ERR_E_NOT_DIVISIBLE: return "E is not divisible by R";
     case MOONEP_ERR_BUDGET_RULE: return "training budget rule violated: B must equal E/R";
     case MOONEP_ERR_B_RANGE: return "replica budget B out of range [0, E - E/R]";
@@ -148,8 +147,8 @@ int moonep_check_config(const moonep_config *c)
     if (c->R <= 0 || c->E <= 0 || c->K <= 0 || c->S <= 0 || c->H <= 0) return MOONEP_ERR_ARG;
     if (c->K > c->E) return MOONEP_ERR_ARG;
     if ((int64_t)c->R * c->S * c->K > INT32_MAX) return MOONEP_ERR_ARG;
-    // the flags this library implements (MOONEP_FLAG_CASCADE is not one yet)
-    if (c->flags & ~(MOONEP_FLAG_STRICT_BUDGET | MOONEP_FLAG_TRAIN_B_RULE | MOONEP_FLAG_BWD_UNSCALED))
+    if (c->flags & ~(MOONEP_FLAG_STRICT_BUDGET | MOONEP_FLAG_TRAIN_B_RULE | MOONEP_FLAG_BWD_UNSCALED |
+                     MOONEP_FLAG_CASCADE))
         return MOONEP_ERR_ARG;
     if (c->E % c->R != 0) return MOONEP_ERR_E_NOT_DIVISIBLE;
     const int L = c->E / c->R;

@@ -80,9 +80,21 @@ __host__ __device__ inline int assign_smem_ints(int E, int R, int max_pairs)
     return ASSIGN_WARPS * E + max_pairs + (E + 1) + 2 * (2 * E + R) + 32;
 }
 
-__host__ __device__ inline int hist_smem_ints(int E, int R, int max_pairs)
+// ints of the relay cascade's own region, after the planner's (allocated
+// only with MOONEP_FLAG_CASCADE).  lc: the list's length during a step.
+__host__ __device__ inline int cascade_list_cap(int E, int R, int B) { return 2 * (E + R - 1) + 2 * B + 2; }
+__host__ __device__ inline int cascade_smem_ints(int E, int R, int B)
 {
-    const int a = plan_smem_ints(E, R), b = E + max_pairs;
+    const int lc = cascade_list_cap(E, R, B), nh = 2 * E + R;
+    return 4 * lc /*le lr lq la*/ + 3 * lc /*order, moved experts and quotas*/ + 4 * (B + 1) /*providers, relays*/ +
+           E /*on_r*/ + 3 * R /*cnt closed hused*/ + 2 * lc /*ordinal, slot offset per entry*/ +
+           E /*home slot offset*/ + 2 * (E + 1) /*host counts, flag prefix*/ + E /*flag*/ + 4 * nh /*hosts*/ + 16;
+}
+
+__host__ __device__ inline int hist_smem_ints(int E, int R, int max_pairs, unsigned flags, int B)
+{
+    const int a = plan_smem_ints(E, R) + ((flags & MOONEP_FLAG_CASCADE) ? cascade_smem_ints(E, R, B) : 0);
+    const int b = E + max_pairs;
     return a > b ? a : b;
 }
 
@@ -108,6 +120,338 @@ __device__ __forceinline__ void pdl_launch_dependents()
 }
 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// ------------------------------------------------ relay cascade (slow path)
+
+// The planner's tail when MOONEP_FLAG_CASCADE is set and water-filling left
+// some rank with more than B replicas.  It keeps such ranks within B by the
+// relay cascade: repeatedly, the rank with the most replicas (ties: lowest
+// rank) among those over B and not yet closed keeps its B - m largest
+// replicas (quota desc, list position asc) for the smallest m in 0..B whose
+// providers can carry the rest; the providers are those kept replicas (each
+// can grow by its expert's remaining home quota, unless that home is closed)
+// and then m relay experts (home quota left, home not this rank, not closed
+// and not yet a relay home, no replica on this rank), chosen by largest home
+// quota, lowest expert first.  The moved quota is poured into the providers
+// in that order, and the moved replicas are water-filled into the providers'
+// home ranks: an amount on its own expert's home returns there, one on a
+// rank already holding the expert joins that replica, any other is a new
+// replica at the end of the list.  The rank is then closed; a step that
+// could make the list longer than E + R - 1 live entries is not taken.
+// The steps are inherently one after another and run on one thread over
+// shared-memory lists; the tables are then rebuilt from the list by the
+// whole CTA.  Every index the step loops use is bounded by the list
+// capacity.
+__device__ void cascade_tail(const PlanParams &a, int *cz, int *keep, const int *pe, const int *qr,
+                             const int *segb, const int *pilo, const int *PS, const int *QSr, int qbase,
+                             int n_rep, int nP, int nN, int *misc, int *wsum, int seq)
+{
+    const Dims &d = a.d;
+    const int E = d.E, R = d.R, L = d.L, C = d.C, B = d.B;
+    const int tid = threadIdx.x;
+    constexpr int nt = PLAN_THREADS;
+    const int cap = E + R - 1, lc = cascade_list_cap(E, R, B), nh = 2 * E + R;
+    int *le = cz, *lr = le + lc, *lq = lr + lc, *la = lq + lc;  // list: expert, rank, quota, alive
+    int *ordx = la + lc;                                          // a rank's replicas in step order
+    int *me = ordx + lc, *mq = me + lc;                           // their experts and quotas
+    int *pve = mq + lc, *pvq = pve + B + 1, *pva = pvq + B + 1;   // providers: expert, kept entry or -1, amount
+    int *rel = pva + B + 1;                                       // relays in pick order
+    int *on_r = rel + B + 1;                                      // E
+    int *cnt = on_r + E, *closed = cnt + R, *hused = closed + R;  // R each
+    int *lo = hused + R, *loff = lo + lc;                         // per entry: ordinal, slot offset
+    int *hoff = loff + lc;                                        // E: home slot offset
+    int *hc = hoff + E, *fpre = hc + E + 1, *fl = fpre + E + 1;   // host counts, flag prefix, flags
+    int *xr = fl + E, *xs = xr + nh, *xq = xs + nh, *xo = xq + nh;  // hosts: rank, slot, quota, slot offset
+    __shared__ int s_nl;
+
+    // the water-filling list in creation order
+    for (int q = tid; q < n_rep; q += nt) {
+        const int j = last_le(segb, nP, q);
+        const int i = pilo[j] + (q - segb[j]);
+        le[q] = pe[j];
+        lr[q] = qr[i];
+        lq[q] = min(PS[j + 1], QSr[i + 1] - qbase) - max(PS[j], QSr[i] - qbase);
+        la[q] = 1;
+    }
+    for (int r = tid; r < R; r += nt) closed[r] = 0;
+    __syncthreads();
+
+    if (tid == 0) {
+        // every thread has passed the branch that read misc[3]: recount it
+        misc[2] = 0;
+        misc[3] = 0;
+        int nl = n_rep;
+        for (int step = 0; step <= R; ++step) {
+            for (int r = 0; r < R; ++r) cnt[r] = 0;
+            for (int q = 0; q < nl; ++q)
+                if (la[q]) ++cnt[lr[q]];
+            int rs = -1;
+            for (int r = 0; r < R; ++r)
+                if (!closed[r] && cnt[r] > B && (rs < 0 || cnt[r] > cnt[rs])) rs = r;
+            if (rs < 0) break;
+            // its replicas by (quota desc, list position asc): insertion sort
+            int n = 0;
+            for (int e = 0; e < E; ++e) on_r[e] = 0;
+            for (int q = 0; q < nl && n < lc; ++q) {
+                if (!la[q] || lr[q] != rs) continue;
+                int k = n++;
+                while (k > 0 && lq[ordx[k - 1]] < lq[q]) {
+                    ordx[k] = ordx[k - 1];
+                    --k;
+                }
+                ordx[k] = q;
+                on_r[le[q]] = 1;
+            }
+            // the smallest m whose providers carry the moved quota
+            for (int r = 0; r < R; ++r) hused[r] = 0;
+            int npick = 0, m_found = -1;
+            long long Q = 0;
+            for (int m = 0; m <= B; ++m) {
+                while (npick < m) {  // next relay: largest home quota, lowest expert
+                    int best = -1;
+                    for (int e = 0; e < E; ++e) {
+                        const int h = e / L;
+                        if (keep[e] > 0 && h != rs && !closed[h] && !on_r[e] && !hused[h] &&
+                            (best < 0 || keep[e] > keep[best]))
+                            best = e;
+                    }
+                    if (best < 0) break;
+                    rel[npick++] = best;
+                    hused[best / L] = 1;
+                }
+                if (npick < m) break;  // fewer distinct relay homes than m
+                Q = 0;
+                for (int k = B - m; k < n; ++k) Q += lq[ordx[k]];
+                long long room = 0;
+                for (int k = 0; k < B - m; ++k) {
+                    const int e = le[ordx[k]];
+                    room += closed[e / L] ? 0 : keep[e];
+                }
+                for (int k = 0; k < m; ++k) room += keep[rel[k]];
+                if (room >= Q) {
+                    m_found = m;
+                    break;
+                }
+            }
+            closed[rs] = 1;
+            if (m_found < 0) continue;
+            if (nl + m_found + B - 1 > cap) continue;  // the list could outgrow the plan's arrays
+            for (int k = 0; k < n; ++k) {
+                me[k] = le[ordx[k]];
+                mq[k] = lq[ordx[k]];
+            }
+            // providers: the kept replicas, then the relays; pour Q into them
+            int np = 0;
+            for (int k = 0; k < B - m_found; ++k) {
+                pve[np] = le[ordx[k]];
+                pvq[np] = ordx[k];
+                ++np;
+            }
+            for (int k = 0; k < m_found; ++k) {
+                pve[np] = rel[k];
+                pvq[np] = -1;
+                ++np;
+            }
+            long long rem = Q;
+            for (int k = 0; k < np; ++k) {
+                const int e = pve[k];
+                const long long capk = (pvq[k] >= 0 && closed[e / L]) ? 0 : keep[e];
+                const int amt = (int)(capk < rem ? capk : rem);
+                pva[k] = amt;
+                rem -= amt;
+                if (amt <= 0) continue;
+                keep[e] -= amt;
+                if (pvq[k] >= 0) {
+                    lq[pvq[k]] += amt;
+                } else if (nl < lc) {
+                    le[nl] = e;
+                    lr[nl] = rs;
+                    lq[nl] = amt;
+                    la[nl] = 1;
+                    ++nl;
+                }
+            }
+            // the moved replicas leave this rank for the providers' homes
+            const int k0 = B - m_found;
+            for (int k = k0; k < n; ++k) la[ordx[k]] = 0;
+            int mk = k0, pi = 0;
+            int al = mk < n ? mq[mk] : 0, cl = np > 0 ? pva[0] : 0;
+            while (mk < n && pi < np) {
+                if (cl <= 0) {
+                    ++pi;
+                    cl = pi < np ? pva[pi] : 0;
+                    continue;
+                }
+                if (al <= 0) {
+                    ++mk;
+                    al = mk < n ? mq[mk] : 0;
+                    continue;
+                }
+                const int amt = al < cl ? al : cl;
+                const int ek = me[mk], h = pve[pi] / L;
+                if (ek / L == h) {
+                    keep[ek] += amt;
+                } else {
+                    int found = -1;
+                    for (int q = 0; q < nl; ++q)
+                        if (la[q] && le[q] == ek && lr[q] == h) {
+                            found = q;
+                            break;
+                        }
+                    if (found >= 0) {
+                        lq[found] += amt;
+                    } else if (nl < lc) {
+                        le[nl] = ek;
+                        lr[nl] = h;
+                        lq[nl] = amt;
+                        la[nl] = 1;
+                        ++nl;
+                    }
+                }
+                al -= amt;
+                cl -= amt;
+            }
+            int w = 0;  // drop the dead entries, keeping list order
+            for (int q = 0; q < nl; ++q)
+                if (la[q]) {
+                    le[w] = le[q];
+                    lr[w] = lr[q];
+                    lq[w] = lq[q];
+                    la[w] = 1;
+                    ++w;
+                }
+            nl = w;
+        }
+        s_nl = nl;
+    }
+    __syncthreads();
+    const int nl = s_nl;
+
+    // ordinals in list order, slot offsets and the used slots of every rank
+    for (int r = tid; r < R; r += nt) {
+        int off = 0;
+        for (int sl = 0; sl < L; ++sl) {
+            const int e = r * L + sl;
+            hoff[e] = off;
+            a.p.slot_expert[(size_t)r * E + sl] = e;
+            a.p.slot_count[(size_t)r * E + sl] = keep[e];
+            a.p.slot_offset[(size_t)r * (E + 1) + sl] = off;
+            off += keep[e];
+        }
+        int ord = 0;
+        for (int q = 0; q < nl; ++q) {
+            if (lr[q] != r) continue;
+            lo[q] = ord;
+            loff[q] = off;
+            const int sl = min(L + ord, E - 1);
+            a.p.slot_expert[(size_t)r * E + sl] = le[q];
+            a.p.slot_count[(size_t)r * E + sl] = lq[q];
+            a.p.slot_offset[(size_t)r * (E + 1) + sl] = off;
+            off += lq[q];
+            ++ord;
+        }
+        atomicMax(&misc[3], ord);
+    }
+    __syncthreads();
+    for (int q = tid; q < nl; q += nt) {
+        a.p.rep_expert[q] = le[q];
+        a.p.rep_rank[q] = lr[q];
+        a.p.rep_slot[q] = L + lo[q];
+        a.p.rep_quota[q] = lq[q];
+        if (lo[q] >= B) atomicAdd(&misc[2], 1);
+    }
+    // hosts per expert (home + its replicas) and the work-list flags
+    for (int e = tid; e < E; e += nt) {
+        int c = 1, f = 0;
+        for (int q = 0; q < nl; ++q)
+            if (le[q] == e) {
+                ++c;
+                f |= lo[q] < B;
+            }
+        hc[e] = c;
+        fl[e] = f;
+        fpre[e] = f;
+    }
+    if (tid == 0) {
+        hc[E] = 0;
+        fpre[E] = 0;
+    }
+    __syncthreads();
+    block_exscan(hc, E + 1, wsum);
+    const int n_rep_experts = block_exscan(fpre, E + 1, wsum);
+    for (int e = tid; e <= E; e += nt) a.p.host_ptr[e] = hc[e];
+    for (int e = tid; e < E; e += nt) {
+        if (fl[e]) a.p.rep_home_list[fpre[e]] = e;
+        if (e >= n_rep_experts) a.p.rep_home_list[e] = -1;
+    }
+    // host intervals: the hosts of e in ascending rank, starts in that order
+    for (int e = tid; e < E; e += nt) {
+        const int b0 = hc[e], b1 = min(hc[e + 1], nh);
+        int k = b0;
+        if (k < b1) {
+            xr[k] = e / L;
+            xs[k] = e - (e / L) * L;
+            xq[k] = keep[e];
+            xo[k] = hoff[e];
+            ++k;
+        }
+        for (int q = 0; q < nl && k < b1; ++q)
+            if (le[q] == e) {
+                xr[k] = lr[q];
+                xs[k] = L + lo[q];
+                xq[k] = lq[q];
+                xo[k] = loff[q];
+                ++k;
+            }
+        for (int x = b0 + 1; x < k; ++x) {  // insertion sort by rank (ranks are distinct)
+            const int vr = xr[x], vs = xs[x], vq = xq[x], vo = xo[x];
+            int y = x;
+            while (y > b0 && xr[y - 1] > vr) {
+                xr[y] = xr[y - 1];
+                xs[y] = xs[y - 1];
+                xq[y] = xq[y - 1];
+                xo[y] = xo[y - 1];
+                --y;
+            }
+            xr[y] = vr;
+            xs[y] = vs;
+            xq[y] = vq;
+            xo[y] = vo;
+        }
+        int st = 0;
+        for (int h = b0; h < k; ++h) {
+            a.p.host_rank[h] = xr[h];
+            a.p.host_slot[h] = xs[h];
+            a.p.host_quota[h] = xq[h];
+            a.p.host_start[h] = st;
+            a.host_dst0[h] = xr[h] * C + xo[h] - st;
+            st += xq[h];
+        }
+    }
+    __syncthreads();
+    if (tid == 0) {
+        const int n_over = misc[2];
+        int st = 0;
+        if (n_over > 0) {
+            st |= MOONEP_ST_OVERFLOW;
+            if (d.flags & MOONEP_FLAG_STRICT_BUDGET) st |= MOONEP_ST_STRICT_VIOLATION;
+        }
+        a.p.info[MOONEP_INFO_STATUS] = st;
+        a.p.info[MOONEP_INFO_N_REP] = nl;
+        a.p.info[MOONEP_INFO_N_OVERFLOW] = n_over;
+        a.p.info[MOONEP_INFO_N_PIECES] = nP;
+        a.p.info[MOONEP_INFO_N_RECEIVERS] = nN;
+        a.p.info[MOONEP_INFO_MAX_REP_PER_RANK] = misc[3];
+        a.p.info[MOONEP_INFO_N_REP_EXPERTS] = n_rep_experts;
+        for (int i = MOONEP_INFO_N_REMOTE_PAIRS; i < MOONEP_INFO_LEN; ++i) a.p.info[i] = 0;
+    }
+    // every thread's plan writes precede the plan-ready mark
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        st_release(a.hdr + WS_PLANNED, seq + 1);
+    }
+}
 
 // ------------------------------------------------------------- planner CTA
 
@@ -331,6 +675,12 @@ __device__ void plan_block(const PlanParams &a, int *sm, int seq)
     // one scan over [replicas per piece | replicas per rank]
     block_exscan(Bs, nP + 1 + R + 1, wsum);
     const int n_rep = Bs[nP];
+    // over the budget with the cascade asked for: the slow path plans the rest
+    if ((d.flags & MOONEP_FLAG_CASCADE) && B > 0 && misc[3] > B) {
+        cascade_tail(a, sm + plan_smem_ints(E, R), keep, pe, qr, segb, pilo, PS, QSr, qbase, n_rep, nP, nN, misc,
+                     wsum, seq);
+        return;
+    }
     auto rank_base = [&](int r) { return r * L + rpr[r] - n_rep; };  // first compact slot of rank r
 
     // ---- replica list (creation order), the compact used-slot lists and
@@ -825,7 +1175,7 @@ int launch_plan(const Dims &d, const int32_t *topk, const moonep_plan_t &p, void
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
 
-    const size_t smem1 = sizeof(int) * (size_t)hist_smem_ints(d.E, d.R, d.chunk_tokens * d.K);
+    const size_t smem1 = sizeof(int) * (size_t)hist_smem_ints(d.E, d.R, d.chunk_tokens * d.K, d.flags, d.B);
     if (!set_smem((const void *)hist_plan_kernel, smem1)) return MOONEP_ERR_CUDA;
     cudaLaunchConfig_t c1 = {};
     c1.gridDim = dim3(d.nchunk);
@@ -847,7 +1197,7 @@ int launch_plan(const Dims &d, const int32_t *topk, const moonep_plan_t &p, void
 
 size_t plan_smem_bytes_max(const Dims &d)
 {
-    const size_t a = sizeof(int) * (size_t)hist_smem_ints(d.E, d.R, d.chunk_tokens * d.K);
+    const size_t a = sizeof(int) * (size_t)hist_smem_ints(d.E, d.R, d.chunk_tokens * d.K, d.flags, d.B);
     const size_t b = sizeof(int) * (size_t)assign_smem_ints(d.E, d.R, d.chunk_tokens * d.K);
     return a > b ? a : b;
 }

@@ -33,7 +33,7 @@ _lib = ctypes.CDLL(_LIB_PATH)
 FLAG_STRICT_BUDGET = 1
 FLAG_TRAIN_B_RULE = 2
 FLAG_BWD_UNSCALED = 4
-FLAG_CASCADE = 8  # reserved: refused (MoonepError 1) until the library implements it
+FLAG_CASCADE = 8
 
 ST_EXPERT_ID_RANGE = 1
 ST_OVERFLOW = 2

@@ -54,11 +54,16 @@ def test_config_checks_match_oracle(cuda_lib_path):
     for c in cases:
         assert moonep.check_config(moonep.Config(**c)) == oracle.check_config(oracle.Config(**c)), c
     # flags: unknown bits are an argument error on both sides; the cascade
-    # flag is defined by the oracle and not implemented by the library yet
+    # flag is known to both
     assert moonep.check_config(moonep.Config(R=4, E=16, K=2, S=8, H=8, B=2, flags=64)) == 1
     assert oracle.check_config(oracle.Config(R=4, E=16, K=2, S=8, H=8, B=2, flags=64)) == 1
     assert oracle.check_config(oracle.Config(R=4, E=16, K=2, S=8, H=8, B=2, flags=8)) == 0
-    assert moonep.check_config(moonep.Config(R=4, E=16, K=2, S=8, H=8, B=2, flags=8)) == 1
+    assert moonep.check_config(moonep.Config(R=4, E=16, K=2, S=8, H=8, B=2, flags=8)) == 0
+    # the cascade's shared memory: the large shape fits, E = R = 1024 does not
+    moonep.plan_sizes(moonep.Config(R=32, E=384, K=8, S=4096, H=7168, B=12, flags=8))
+    assert moonep.check_config(moonep.Config(R=1024, E=1024, K=4, S=4, H=8, B=1, flags=8)) == 0
+    with pytest.raises(moonep.MoonepError):
+        moonep.plan_sizes(moonep.Config(R=1024, E=1024, K=4, S=4, H=8, B=1, flags=8))
     # CUDA-only limits
     assert moonep.check_config(moonep.Config(R=4, E=16, K=2, S=8, H=12, B=2)) == 8
     assert moonep.check_config(moonep.Config(R=2, E=2048, K=2, S=8, H=8, B=2)) == 7

@@ -200,6 +200,89 @@ def test_plan_alternating_routings_reuse_workspace(mp):
         _assert_plan_equal(p, ops[it % 2])
 
 
+# ------------------------------------------------------- relay cascade
+
+def _cascade_routing(rng, R, L, S, K=1):
+    """Skewed routing with an empty expert or two, so water-filling overflows
+    small budgets often; token order shuffled."""
+    E = R * L
+    w = rng.random(E) ** 3
+    w[rng.integers(0, E, size=2)] = 0
+    T = rng.multinomial(R * S * K, w / w.sum())
+    ids = np.repeat(np.arange(E), T)
+    rng.shuffle(ids)
+    return ids.reshape(R * S, K).astype(np.int32)
+
+
+def test_plan_cascade_golden(mp):
+    g = json.load(open(os.path.join(GOLDEN, "plan_example_cascade.json")))
+    topk = np.array(g["topk_idx"], np.int32)
+    gcfg, ocfg, gp, op = _plan_both(mp, g["config"], topk)
+    _assert_plan_equal(gp, op)
+    for k, v in g["expect"].items():
+        if k != "info":
+            assert gp.fields[k].cpu().numpy().tolist() == v, k
+
+
+def test_plan_cascade_counterexample_and_data(mp):
+    """The 31-replica counterexample: the cascade's plan, then dispatch and
+    combine over it, element for element against the oracle."""
+    R, E, S, B, H = 32, 384, 3100, 12, 16
+    L = E // R
+    T = np.zeros(E, np.int64)
+    for r in range(1, R):
+        T[r * L:(r + 1) * L] = [300] * 10 + [100] * 2
+    ids = np.repeat(np.arange(E), T)
+    np.random.default_rng(0).shuffle(ids)
+    topk = ids.reshape(R * S, 1).astype(np.int32)
+    c = dict(R=R, E=E, K=1, S=S, H=H, B=B, flags=mp.FLAG_CASCADE)
+    gcfg, ocfg, gp, op = _plan_both(mp, c, topk)
+    _assert_plan_equal(gp, op)
+    assert gp.info()["status"] == 0 and gp.info()["max_rep_per_rank"] == B
+    wl = W.Workload("cx", R, E, 1, S, H, B)
+    hidden = W.hidden_states(wl, seed=1, device=DEV)
+    buf = torch.full((R, S, H), float("nan"), dtype=torch.bfloat16, device=DEV)
+    mp.dispatch(gcfg, gp, hidden, buf)
+    ob = np.zeros((R, S, H), np.uint16)
+    oracle.dispatch(ocfg, op, W.bits(hidden), ob)
+    assert np.array_equal(W.bits(buf), ob)
+    w = W.f32_normal((R * S, 1), seed=4, device=DEV)
+    out = mp.combine(gcfg, gp, buf, w)
+    assert np.array_equal(W.bits(out), oracle.combine(ocfg, op, ob, w.cpu().numpy()))
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_plan_cascade_random(mp, seed):
+    """Random skewed routings over small budgets, with and without strict
+    mode: the cascade plan (or the overflow it could not avoid) equals the
+    oracle's."""
+    rng = np.random.default_rng(300 + seed)
+    for trial in range(6):
+        R = int(rng.choice([4, 8, 16]))
+        L = int(rng.choice([2, 3, 4]))
+        K = int(rng.choice([1, 2]))
+        S = int(rng.integers(8, 64))
+        B = int(rng.choice([1, 2]))
+        flags = mp.FLAG_CASCADE | (mp.FLAG_STRICT_BUDGET if trial % 3 == 0 else 0)
+        topk = _cascade_routing(rng, R, L, S, K)
+        c = dict(R=R, E=R * L, K=K, S=S, H=8, B=B, flags=flags)
+        _, ocfg, gp, op = _plan_both(mp, c, topk)
+        _assert_plan_equal(gp, op)
+        check_invariants(ocfg, topk, gp.to_numpy())
+
+
+def test_plan_cascade_within_budget_is_water_filling(mp):
+    wl = W.WORKLOADS["mid"]
+    r = W.routing(wl, 2.0, device=DEV)
+    topk = r.topk_idx.cpu().numpy()
+    _, _, g0, _ = _plan_both(mp, _wl_cfg(wl), topk)
+    _, _, g1, o1 = _plan_both(mp, _wl_cfg(wl, flags=mp.FLAG_CASCADE), topk)
+    _assert_plan_equal(g1, o1)
+    a0, a1 = g0.to_numpy(), g1.to_numpy()
+    for k in a0:
+        assert np.array_equal(a0[k], a1[k]), k
+
+
 def test_plan_many_chunks_multi_wave(mp):
     """More token chunks (512, in 32 groups) than two CTAs per SM can hold at
     once: both planner grids run in several waves, and assignment CTAs wait

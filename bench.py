@@ -572,6 +572,41 @@ def run_ours(args, world, rank, local):
             del ep
         del eh, ebuf, eout
 
+    # over-budget routing (one empty rank, the rest evenly overloaded): the
+    # planner without and with the relay cascade, and the data kernels over
+    # the cascade's plan
+    cascade = None
+    if not args.no_sweep:
+        cr = W.over_budget_routing(wl, seed=rank, device=dev)
+        cascade = {"workload": f"{wl.name} shape, rank 0's experts empty, the other "
+                               f"{wl.R - 1} ranks evenly overloaded", "points": []}
+        for flags in (0, mp.FLAG_CASCADE):
+            ccfg = mp.Config(R=wl.R, E=wl.E, K=wl.K, S=wl.S, H=wl.H, B=wl.B, flags=flags)
+            cp = mp.Plan(ccfg, dev)
+            for _ in range(3):
+                mp.plan(ccfg, cr.topk_idx, out=cp)
+                mp.dispatch(ccfg, cp, hidden, buf)
+                mp.combine(ccfg, cp, buf, cr.weights, out)
+            torch.cuda.synchronize()
+            st = Timer()
+            for _ in range(args.sweep_iters):
+                e = st.mark("plan"); mp.plan(ccfg, cr.topk_idx, out=cp); e.record()
+                e = st.mark("dispatch"); mp.dispatch(ccfg, cp, hidden, buf); e.record()
+                e = st.mark("combine"); mp.combine(ccfg, cp, buf, cr.weights, out); e.record()
+            torch.cuda.synchronize()
+            it = args.sweep_iters
+            pd, pc, pp = st.total_ms("dispatch") / it, st.total_ms("combine") / it, st.total_ms("plan") / it
+            inf = cp.info()
+            cascade["points"].append({
+                "cascade": bool(flags), "planner_us": round(pp * 1e3, 2),
+                "dispatch_GB/s": round(bytes_dispatch(wl) / (pd * 1e-3) / 1e9, 1),
+                "combine_GB/s": round(bytes_combine(wl) / (pc * 1e-3) / 1e9, 1),
+                "status": inf["status"], "n_rep": inf["n_rep"], "n_overflow": inf["n_overflow"],
+                "max_rep_per_rank": inf["max_rep_per_rank"],
+                "remote_pair_frac": round(inf["n_remote_pairs"] / wl.pairs, 4)})
+            del cp
+        del cr
+
     # decode shape (latency-bound): plan + dispatch + combine of one MoE layer
     # replayed from a CUDA graph, next to the eager per-kernel times
     decode = None
@@ -693,7 +728,7 @@ def run_ours(args, world, rank, local):
         "decode": decode,
         "pages_sweep": {"workload": "ep8: R=8 E=256 K=8 S=4096 H=7168 B=4 (EP=8 as in the pages' sweep)",
                         "points": pages_sweep},
-        "clocks": clocks, "plan_info": info,
+        "cascade": cascade, "clocks": clocks, "plan_info": info,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -210,6 +210,36 @@ def f32_normal(shape, seed: int, device="cpu", std: float = 1.0,
     return out
 
 
+def over_budget_routing(wl: Workload, seed: int = 0, device="cpu") -> Routing:
+    """One empty rank among R - 1 evenly overloaded ones: rank 0's experts get
+    no tokens and every other rank's load is C * R / (R - 1) (rounded), so
+    each of the R - 1 ranks sheds its excess to rank 0, which water-filling
+    turns into R - 1 replicas on rank 0 (more than a budget B < R - 1).
+    A rank's first expert carries the rank's rounding remainder; the others
+    share the rest evenly.  Each token's K experts are distinct (pair slots
+    are dealt expert-sorted with stride R*S, longer than any expert's run),
+    and tokens are shuffled."""
+    R, S, K, E, L = wl.R, wl.S, wl.K, wl.E, wl.L
+    C = S * K
+    T = np.zeros(E, np.int64)
+    load = np.full(R - 1, (R * C) // (R - 1), np.int64)
+    load[: (R * C) % (R - 1)] += 1
+    for r in range(1, R):
+        q = load[r - 1] // L
+        T[r * L:(r + 1) * L] = q
+        T[r * L] += load[r - 1] - q * L
+    assert T.sum() == R * C and T.max() <= R * S
+    ids = np.repeat(np.arange(E, dtype=np.int32), T)
+    topk = ids.reshape(K, R * S).T.copy()
+    rng = np.random.default_rng(seed)
+    topk = topk[rng.permutation(R * S)]
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    z, _ = torch.sort(torch.randn(R * S, K, generator=g), dim=1, descending=True)
+    w = torch.softmax(z.double(), dim=1).float().contiguous()
+    mv = maxvio_of_counts(T, R, S, K, E)
+    return Routing(torch.from_numpy(np.ascontiguousarray(topk)).to(device), w.to(device), mv, mv, 0.0)
+
+
 def hidden_states(wl: Workload, seed: int = 1, device="cpu") -> torch.Tensor:
     return bf16_normal((wl.tokens, wl.H), seed, device)
 
@@ -225,6 +255,7 @@ def from_bits(a: np.ndarray, device="cpu") -> torch.Tensor:
 
 
 __all__ = [
-    "Workload", "WORKLOADS", "Routing", "routing", "balanced_routing", "maxvio_of_counts",
+    "Workload", "WORKLOADS", "Routing", "routing", "balanced_routing", "over_budget_routing",
+    "maxvio_of_counts",
     "hottest_expert_count", "bf16_normal", "f32_normal", "hidden_states", "bits", "from_bits",
 ]

@@ -283,6 +283,20 @@ def test_plan_cascade_within_budget_is_water_filling(mp):
         assert np.array_equal(a0[k], a1[k]), k
 
 
+@pytest.mark.parametrize("flags", [0, 8])
+def test_plan_over_budget_full_size(mp, flags):
+    """The large training shape with one empty rank: water-filling puts 31
+    replicas on it; the cascade keeps every rank within B = 12.  Every plan
+    field against the oracle."""
+    wl = W.WORKLOADS["large"]
+    topk = W.over_budget_routing(wl).topk_idx.numpy()
+    _, ocfg, gp, op = _plan_both(mp, _wl_cfg(wl, flags=flags), topk)
+    _assert_plan_equal(gp, op)
+    inf = gp.info()
+    assert inf["max_rep_per_rank"] == (wl.B if flags else wl.R - 1)
+    check_invariants(ocfg, topk, gp.to_numpy())
+
+
 def test_plan_many_chunks_multi_wave(mp):
     """More token chunks (512, in 32 groups) than two CTAs per SM can hold at
     once: both planner grids run in several waves, and assignment CTAs wait

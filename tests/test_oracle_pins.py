@@ -115,6 +115,28 @@ def test_cascade_empty_rank_counterexample(oracle_lib):
     check_invariants(cfg, topk, p)
 
 
+def test_cascade_over_budget_routing_large(oracle_lib):
+    """The benchmark's over-budget routing at the large training shape:
+    distinct experts per token, rank 0's experts empty, the greedy over B on
+    rank 0 alone (R - 1 replicas there), and the cascade within B with a
+    valid plan."""
+    wl = W.WORKLOADS["large"]
+    topk = W.over_budget_routing(wl).topk_idx.numpy()
+    assert topk.shape == (wl.tokens, wl.K)
+    s = np.sort(topk, axis=1)
+    assert (s[:, 1:] != s[:, :-1]).all()
+    T = np.bincount(topk.ravel(), minlength=wl.E)
+    assert T[:wl.L].sum() == 0 and T.sum() == wl.pairs
+    c0 = oracle.Config(R=wl.R, E=wl.E, K=wl.K, S=wl.S, H=wl.H, B=wl.B)
+    i0 = oracle.info_dict(oracle.plan(c0, topk))
+    assert i0["status"] == oracle.ST_OVERFLOW and i0["max_rep_per_rank"] == wl.R - 1
+    cfg = oracle.Config(R=wl.R, E=wl.E, K=wl.K, S=wl.S, H=wl.H, B=wl.B, flags=oracle.FLAG_CASCADE)
+    p = oracle.plan(cfg, topk)
+    info = oracle.info_dict(p)
+    assert info["status"] == 0 and info["max_rep_per_rank"] == wl.B
+    check_invariants(cfg, topk, p)
+
+
 def test_cascade_against_bruteforce_budget(oracle_lib):
     """Micro routings the water-filling takes over B = 1: the cascade keeps
     the invariants, reports overflow exactly when a rank is over B, and finds

@@ -71,9 +71,10 @@ extern "C" {
  * keeps its B - m largest replicas, grows them and adds m relay replicas of
  * other ranks' experts to carry the rest, and the moved replicas go to the
  * providers' home ranks, which may in turn be repaired.  Within the budget
- * the plan is exactly water-filling's.  Costs a larger planner shared-memory
- * allocation (MOONEP_ERR_LIMIT if it does not fit) and a serial slow path
- * when it runs.  Unknown flag bits are MOONEP_ERR_ARG. */
+ * the plan is exactly water-filling's.  Costs 7 (E + R) + 4 (B + 1) + 16
+ * more ints of planner shared memory (MOONEP_ERR_LIMIT if the total does not
+ * fit; at E = R = MOONEP_MAX_E it does) and a slow path, one warp stepping
+ * through the repairs, when it runs.  Unknown flag bits are MOONEP_ERR_ARG. */
 #define MOONEP_FLAG_CASCADE 8u
 
 /* ---- host return codes ------------------------------------------------- */

@@ -29,7 +29,8 @@ constexpr int CHUNK_GROUP = 16;
 
 // Workspace layout (bytes from the workspace base; 256-byte aligned parts).
 struct WsLayout {
-    size_t hdr;        // int32[8]: ticket, status, call sequence, counts-ready mark, arrivals, plan-ready mark
+    size_t hdr;        // int32[8]: ticket, status, call sequence, counts-ready mark, arrivals, plan-ready mark,
+                       // slow-path mark
     size_t gs;         // int32 [2][ngroups][E]: per-group expert counts, double-buffered
     size_t cc;         // int32 [nchunk][E]: per-chunk expert counts
     size_t host_dst0;  // int32 [2E+R]: rank*C + slot_offset - host_start per host
@@ -40,8 +41,14 @@ struct WsLayout {
 // sets READY = SEQ + 1 once every chunk's counts are in, and PLANNED = SEQ + 1
 // once the plan is written; the assignment CTAs wait for those marks, and the
 // last of them to arrive advances SEQ, so after a call READY == PLANNED == SEQ
-// and a stale mark never passes for a fresh one.
-enum { WS_TICKET = 0, WS_STATUS = 1, WS_SEQ = 2, WS_READY = 3, WS_ARRIVED = 4, WS_PLANNED = 5, WS_HDR_INTS = 8 };
+// and a stale mark never passes for a fresh one.  SLOW = SEQ + 1 announces
+// that the planner took a slow path (the relay cascade) whose length has no
+// useful bound for a spin: the assignment CTAs then wait for the whole
+// histogram grid instead.
+enum {
+    WS_TICKET = 0, WS_STATUS = 1, WS_SEQ = 2, WS_READY = 3, WS_ARRIVED = 4, WS_PLANNED = 5, WS_SLOW = 6,
+    WS_HDR_INTS = 8
+};
 
 // Status bits after which every later call treats the plan as empty.
 constexpr int ST_EMPTY_PLAN = MOONEP_ST_EXPERT_ID_RANGE | MOONEP_ST_WORKSPACE;

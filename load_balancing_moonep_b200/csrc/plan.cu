@@ -80,15 +80,27 @@ __host__ __device__ inline int assign_smem_ints(int E, int R, int max_pairs)
     return ASSIGN_WARPS * E + max_pairs + (E + 1) + 2 * (2 * E + R) + 32;
 }
 
-// ints of the relay cascade's own region, after the planner's (allocated
-// only with MOONEP_FLAG_CASCADE).  lc: the list's length during a step.
-__host__ __device__ inline int cascade_list_cap(int E, int R, int B) { return 2 * (E + R - 1) + 2 * B + 2; }
+// The relay cascade's shared memory.  Its step lists take a region of their
+// own after the planner's (allocated only with MOONEP_FLAG_CASCADE); its host
+// and per-expert tables reuse the planner's arrays from jlo to flag, which are
+// dead once water-filling has been counted, when they fit there.
+// lc: the list's capacity; a step never makes it longer than E + R - 1.
+__host__ __device__ inline int cascade_list_cap(int E, int R) { return E + R; }
+__host__ __device__ inline int plan_dead_ints(int E, int R) { return R + E + 6 * (2 * E + R) + E; }
+__host__ __device__ inline int cascade_table_ints(int E, int R)
+{
+    return 4 * (2 * E + R) /*hosts*/ + E /*on_r*/ + 3 * R /*cnt closed hused*/ + E /*home slot offset*/ +
+           2 * (E + 1) /*host counts, flag prefix*/ + E /*flag*/;
+}
+__host__ __device__ inline bool cascade_tables_in_dead(int E, int R)
+{
+    return cascade_table_ints(E, R) <= plan_dead_ints(E, R);
+}
 __host__ __device__ inline int cascade_smem_ints(int E, int R, int B)
 {
-    const int lc = cascade_list_cap(E, R, B), nh = 2 * E + R;
-    return 4 * lc /*le lr lq la*/ + 3 * lc /*order, moved experts and quotas*/ + 4 * (B + 1) /*providers, relays*/ +
-           E /*on_r*/ + 3 * R /*cnt closed hused*/ + 2 * lc /*ordinal, slot offset per entry*/ +
-           E /*home slot offset*/ + 2 * (E + 1) /*host counts, flag prefix*/ + E /*flag*/ + 4 * nh /*hosts*/ + 16;
+    const int lc = cascade_list_cap(E, R);
+    return 7 * lc /*le lr lq la, order, moved experts and quotas*/ + 4 * (B + 1) /*providers, relays*/ +
+           (cascade_tables_in_dead(E, R) ? 0 : cascade_table_ints(E, R)) + 16;
 }
 
 __host__ __device__ inline int hist_smem_ints(int E, int R, int max_pairs, unsigned flags, int B)
@@ -138,11 +150,11 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 // rank already holding the expert joins that replica, any other is a new
 // replica at the end of the list.  The rank is then closed; a step that
 // could make the list longer than E + R - 1 live entries is not taken.
-// The steps are inherently one after another and run on one thread over
-// shared-memory lists; the tables are then rebuilt from the list by the
-// whole CTA.  Every index the step loops use is bounded by the list
+// The steps are inherently one after another and run on one warp over
+// shared-memory lists (searches, sums and compaction by ballot and shuffle);
+// the tables are then rebuilt from the list by the whole CTA.  Every index the step loops use is bounded by the list
 // capacity.
-__device__ void cascade_tail(const PlanParams &a, int *cz, int *keep, const int *pe, const int *qr,
+__device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep, const int *pe, const int *qr,
                              const int *segb, const int *pilo, const int *PS, const int *QSr, int qbase,
                              int n_rep, int nP, int nN, int *misc, int *wsum, int seq)
 {
@@ -150,22 +162,26 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *keep, const int 
     const int E = d.E, R = d.R, L = d.L, C = d.C, B = d.B;
     const int tid = threadIdx.x;
     constexpr int nt = PLAN_THREADS;
-    const int cap = E + R - 1, lc = cascade_list_cap(E, R, B), nh = 2 * E + R;
+    const int cap = E + R - 1, lc = cascade_list_cap(E, R), nh = 2 * E + R;
     int *le = cz, *lr = le + lc, *lq = lr + lc, *la = lq + lc;  // list: expert, rank, quota, alive
     int *ordx = la + lc;                                          // a rank's replicas in step order
     int *me = ordx + lc, *mq = me + lc;                           // their experts and quotas
     int *pve = mq + lc, *pvq = pve + B + 1, *pva = pvq + B + 1;   // providers: expert, kept entry or -1, amount
     int *rel = pva + B + 1;                                       // relays in pick order
-    int *on_r = rel + B + 1;                                      // E
+    int *tb = cascade_tables_in_dead(E, R) ? dead : rel + B + 1;
+    int *xr = tb, *xs = xr + nh, *xq = xs + nh, *xo = xq + nh;    // hosts: rank, slot, quota, slot offset
+    int *on_r = xo + nh;                                          // E
     int *cnt = on_r + E, *closed = cnt + R, *hused = closed + R;  // R each
-    int *lo = hused + R, *loff = lo + lc;                         // per entry: ordinal, slot offset
-    int *hoff = loff + lc;                                        // E: home slot offset
+    int *hoff = hused + R;                                        // E: home slot offset
     int *hc = hoff + E, *fpre = hc + E + 1, *fl = fpre + E + 1;   // host counts, flag prefix, flags
-    int *xr = fl + E, *xs = xr + nh, *xq = xs + nh, *xo = xq + nh;  // hosts: rank, slot, quota, slot offset
+    int *lo = ordx, *loff = me;                                   // after the steps: ordinal, slot offset per entry
     __shared__ int s_nl;
 
+    // announce the slow path: the assignment CTAs stop spinning on the
+    // plan-ready mark and wait for this grid to finish
+    if (tid == 0) st_release(a.hdr + WS_SLOW, seq + 1);
     // the water-filling list in creation order
-    for (int q = tid; q < n_rep; q += nt) {
+    for (int q = tid; q < min(n_rep, lc); q += nt) {
         const int j = last_le(segb, nP, q);
         const int i = pilo[j] + (q - segb[j]);
         le[q] = pe[j];
@@ -176,104 +192,193 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *keep, const int 
     for (int r = tid; r < R; r += nt) closed[r] = 0;
     __syncthreads();
 
-    if (tid == 0) {
-        // every thread has passed the branch that read misc[3]: recount it
-        misc[2] = 0;
-        misc[3] = 0;
-        int nl = n_rep;
+    if (tid < 32) {
+        // warp 0 runs the steps: every lane holds the same step state, lane 0
+        // makes the scalar writes, searches and sums use the whole warp
+        const int lane = tid;
+        const unsigned lt = lanemask_lt();
+        if (lane == 0) {  // every thread has passed the branch that read misc[3]: recount it
+            misc[2] = 0;
+            misc[3] = 0;
+        }
+        int nl = min(n_rep, lc);
         for (int step = 0; step <= R; ++step) {
-            for (int r = 0; r < R; ++r) cnt[r] = 0;
-            for (int q = 0; q < nl; ++q)
-                if (la[q]) ++cnt[lr[q]];
-            int rs = -1;
-            for (int r = 0; r < R; ++r)
-                if (!closed[r] && cnt[r] > B && (rs < 0 || cnt[r] > cnt[rs])) rs = r;
-            if (rs < 0) break;
-            // its replicas by (quota desc, list position asc): insertion sort
-            int n = 0;
-            for (int e = 0; e < E; ++e) on_r[e] = 0;
-            for (int q = 0; q < nl && n < lc; ++q) {
-                if (!la[q] || lr[q] != rs) continue;
-                int k = n++;
-                while (k > 0 && lq[ordx[k - 1]] < lq[q]) {
-                    ordx[k] = ordx[k - 1];
-                    --k;
+            for (int r = lane; r < R; r += 32) cnt[r] = 0;
+            __syncwarp();
+            for (int q = lane; q < nl; q += 32)
+                if (la[q]) atomicAdd(&cnt[lr[q]], 1);
+            __syncwarp();
+            // the open rank over B with the most replicas, lowest rank on ties
+            int bc = -1, br = R;
+            for (int r = lane; r < R; r += 32) {
+                const int c = cnt[r];
+                if (!closed[r] && c > B && c > bc) {
+                    bc = c;
+                    br = r;
                 }
-                ordx[k] = q;
-                on_r[le[q]] = 1;
             }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const int oc = __shfl_xor_sync(FULL_MASK, bc, o), orr = __shfl_xor_sync(FULL_MASK, br, o);
+                if (oc > bc || (oc == bc && orr < br)) {
+                    bc = oc;
+                    br = orr;
+                }
+            }
+            if (bc < 0) break;
+            const int rs = br;
+            // its replicas: positions in list order (in mq), then ranked by
+            // (quota desc, position asc) into ordx
+            for (int e = lane; e < E; e += 32) on_r[e] = 0;
+            for (int r = lane; r < R; r += 32) hused[r] = 0;
+            int n = 0;
+            for (int q0 = 0; q0 < nl; q0 += 32) {
+                const int q = q0 + lane;
+                const bool mine = q < nl && la[q] && lr[q] == rs;
+                const unsigned b = __ballot_sync(FULL_MASK, mine);
+                const int k = n + __popc(b & lt);
+                if (mine && k < lc) mq[k] = q;
+                n += __popc(b);
+            }
+            n = min(n, lc);
+            __syncwarp();
+            for (int k = lane; k < n; k += 32) {
+                const int qk = mq[k], vk = lq[qk];
+                int rk = 0;
+                for (int j = 0; j < n; ++j) {
+                    const int v = lq[mq[j]];
+                    rk += (v > vk) || (v == vk && j < k);
+                }
+                ordx[rk] = qk;
+                on_r[le[qk]] = 1;
+            }
+            __syncwarp();
             // the smallest m whose providers carry the moved quota
-            for (int r = 0; r < R; ++r) hused[r] = 0;
             int npick = 0, m_found = -1;
-            long long Q = 0;
             for (int m = 0; m <= B; ++m) {
                 while (npick < m) {  // next relay: largest home quota, lowest expert
-                    int best = -1;
-                    for (int e = 0; e < E; ++e) {
-                        const int h = e / L;
-                        if (keep[e] > 0 && h != rs && !closed[h] && !on_r[e] && !hused[h] &&
-                            (best < 0 || keep[e] > keep[best]))
-                            best = e;
+                    int bk = 0, be = E;
+                    for (int e = lane; e < E; e += 32) {
+                        const int h = (int)fdiv((uint32_t)e, a.fL), kv = keep[e];
+                        if (kv > bk && h != rs && !closed[h] && !on_r[e] && !hused[h]) {
+                            bk = kv;
+                            be = e;
+                        }
                     }
-                    if (best < 0) break;
-                    rel[npick++] = best;
-                    hused[best / L] = 1;
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) {
+                        const int ok = __shfl_xor_sync(FULL_MASK, bk, o), oe = __shfl_xor_sync(FULL_MASK, be, o);
+                        if (ok > bk || (ok == bk && oe < be)) {
+                            bk = ok;
+                            be = oe;
+                        }
+                    }
+                    if (be >= E) break;
+                    if (lane == 0) {
+                        rel[npick] = be;
+                        hused[fdiv((uint32_t)be, a.fL)] = 1;
+                    }
+                    ++npick;
+                    __syncwarp();
                 }
                 if (npick < m) break;  // fewer distinct relay homes than m
-                Q = 0;
-                for (int k = B - m; k < n; ++k) Q += lq[ordx[k]];
-                long long room = 0;
-                for (int k = 0; k < B - m; ++k) {
+                long long Q = 0, room = 0;
+                for (int k = B - m + lane; k < n; k += 32) Q += lq[ordx[k]];
+                for (int k = lane; k < B - m; k += 32) {
                     const int e = le[ordx[k]];
-                    room += closed[e / L] ? 0 : keep[e];
+                    room += closed[fdiv((uint32_t)e, a.fL)] ? 0 : keep[e];
                 }
-                for (int k = 0; k < m; ++k) room += keep[rel[k]];
+                for (int k = lane; k < m; k += 32) room += keep[rel[k]];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    Q += __shfl_xor_sync(FULL_MASK, Q, o);
+                    room += __shfl_xor_sync(FULL_MASK, room, o);
+                }
                 if (room >= Q) {
                     m_found = m;
                     break;
                 }
             }
-            closed[rs] = 1;
+            if (lane == 0) closed[rs] = 1;
+            __syncwarp();
             if (m_found < 0) continue;
             if (nl + m_found + B - 1 > cap) continue;  // the list could outgrow the plan's arrays
-            for (int k = 0; k < n; ++k) {
-                me[k] = le[ordx[k]];
-                mq[k] = lq[ordx[k]];
-            }
-            // providers: the kept replicas, then the relays; pour Q into them
-            int np = 0;
-            for (int k = 0; k < B - m_found; ++k) {
-                pve[np] = le[ordx[k]];
-                pvq[np] = ordx[k];
-                ++np;
-            }
-            for (int k = 0; k < m_found; ++k) {
-                pve[np] = rel[k];
-                pvq[np] = -1;
-                ++np;
-            }
-            long long rem = Q;
-            for (int k = 0; k < np; ++k) {
-                const int e = pve[k];
-                const long long capk = (pvq[k] >= 0 && closed[e / L]) ? 0 : keep[e];
-                const int amt = (int)(capk < rem ? capk : rem);
-                pva[k] = amt;
-                rem -= amt;
-                if (amt <= 0) continue;
-                keep[e] -= amt;
-                if (pvq[k] >= 0) {
-                    lq[pvq[k]] += amt;
-                } else if (nl < lc) {
-                    le[nl] = e;
-                    lr[nl] = rs;
-                    lq[nl] = amt;
-                    la[nl] = 1;
-                    ++nl;
+            const int k0 = B - m_found;
+            // the rank's replicas by step order: experts and quotas; a kept
+            // replica's position once the moved ones are dropped
+            for (int k = lane; k < n; k += 32) {
+                const int q = ordx[k];
+                me[k] = le[q];
+                mq[k] = lq[q];
+                if (k < k0) {
+                    int before = 0;
+                    for (int j = k0; j < n; ++j) before += ordx[j] < q;
+                    pvq[k] = q - before;
                 }
             }
-            // the moved replicas leave this rank for the providers' homes
-            const int k0 = B - m_found;
-            for (int k = k0; k < n; ++k) la[ordx[k]] = 0;
+            __syncwarp();
+            for (int k = k0 + lane; k < n; k += 32) la[ordx[k]] = 0;  // the moved replicas leave this rank
+            __syncwarp();
+            // drop them, keeping list order (a destination never lies past its
+            // source, so a chunk only writes where its reads are done)
+            int w = 0;
+            for (int q0 = 0; q0 < nl; q0 += 32) {
+                const int q = q0 + lane;
+                const bool alive = q < nl && la[q];
+                int ve = 0, vr = 0, vq = 0;
+                if (alive) {
+                    ve = le[q];
+                    vr = lr[q];
+                    vq = lq[q];
+                }
+                const unsigned b = __ballot_sync(FULL_MASK, alive);
+                __syncwarp();
+                if (alive) {
+                    const int dd = w + __popc(b & lt);
+                    le[dd] = ve;
+                    lr[dd] = vr;
+                    lq[dd] = vq;
+                    la[dd] = 1;
+                }
+                w += __popc(b);
+                __syncwarp();
+            }
+            nl = w;
+            // providers: the kept replicas, then the relays; pour the moved
+            // quota into them (lane 0)
+            int np = 0;
+            if (lane == 0) {
+                long long rem = 0;
+                for (int k = k0; k < n; ++k) rem += mq[k];
+                for (int k = 0; k < k0; ++k) pve[np++] = me[k];
+                for (int k = 0; k < m_found; ++k) {
+                    pve[np] = rel[k];
+                    pvq[np] = -1;
+                    ++np;
+                }
+                for (int k = 0; k < np; ++k) {
+                    const int e = pve[k];
+                    const long long capk = (pvq[k] >= 0 && closed[fdiv((uint32_t)e, a.fL)]) ? 0 : keep[e];
+                    const int amt = (int)(capk < rem ? capk : rem);
+                    pva[k] = amt;
+                    rem -= amt;
+                    if (amt <= 0) continue;
+                    keep[e] -= amt;
+                    if (pvq[k] >= 0) {
+                        lq[pvq[k]] += amt;
+                    } else if (nl < lc) {
+                        le[nl] = e;
+                        lr[nl] = rs;
+                        lq[nl] = amt;
+                        la[nl] = 1;
+                        ++nl;
+                    }
+                }
+            }
+            np = __shfl_sync(FULL_MASK, np, 0);
+            nl = __shfl_sync(FULL_MASK, nl, 0);
+            __syncwarp();
+            // water-fill the moved replicas into the providers' home ranks
             int mk = k0, pi = 0;
             int al = mk < n ? mq[mk] : 0, cl = np > 0 ? pva[0] : 0;
             while (mk < n && pi < np) {
@@ -288,41 +393,34 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *keep, const int 
                     continue;
                 }
                 const int amt = al < cl ? al : cl;
-                const int ek = me[mk], h = pve[pi] / L;
-                if (ek / L == h) {
-                    keep[ek] += amt;
+                const int ek = me[mk], h = (int)fdiv((uint32_t)pve[pi], a.fL);
+                if ((int)fdiv((uint32_t)ek, a.fL) == h) {
+                    if (lane == 0) keep[ek] += amt;
                 } else {
                     int found = -1;
-                    for (int q = 0; q < nl; ++q)
-                        if (la[q] && le[q] == ek && lr[q] == h) {
-                            found = q;
-                            break;
-                        }
+                    for (int q0 = 0; q0 < nl && found < 0; q0 += 32) {
+                        const int q = q0 + lane;
+                        const unsigned b = __ballot_sync(FULL_MASK, q < nl && le[q] == ek && lr[q] == h);
+                        if (b) found = q0 + __ffs(b) - 1;
+                    }
                     if (found >= 0) {
-                        lq[found] += amt;
+                        if (lane == 0) lq[found] += amt;
                     } else if (nl < lc) {
-                        le[nl] = ek;
-                        lr[nl] = h;
-                        lq[nl] = amt;
-                        la[nl] = 1;
+                        if (lane == 0) {
+                            le[nl] = ek;
+                            lr[nl] = h;
+                            lq[nl] = amt;
+                            la[nl] = 1;
+                        }
                         ++nl;
                     }
                 }
+                __syncwarp();
                 al -= amt;
                 cl -= amt;
             }
-            int w = 0;  // drop the dead entries, keeping list order
-            for (int q = 0; q < nl; ++q)
-                if (la[q]) {
-                    le[w] = le[q];
-                    lr[w] = lr[q];
-                    lq[w] = lq[q];
-                    la[w] = 1;
-                    ++w;
-                }
-            nl = w;
         }
-        s_nl = nl;
+        if (lane == 0) s_nl = nl;
     }
     __syncthreads();
     const int nl = s_nl;
@@ -677,8 +775,8 @@ __device__ void plan_block(const PlanParams &a, int *sm, int seq)
     const int n_rep = Bs[nP];
     // over the budget with the cascade asked for: the slow path plans the rest
     if ((d.flags & MOONEP_FLAG_CASCADE) && B > 0 && misc[3] > B) {
-        cascade_tail(a, sm + plan_smem_ints(E, R), keep, pe, qr, segb, pilo, PS, QSr, qbase, n_rep, nP, nN, misc,
-                     wsum, seq);
+        cascade_tail(a, sm + plan_smem_ints(E, R), jlo, keep, pe, qr, segb, pilo, PS, QSr, qbase, n_rep, nP, nN,
+                     misc, wsum, seq);
         return;
     }
     auto rank_base = [&](int r) { return r * L + rpr[r] - n_rep; };  // first compact slot of rank r
@@ -1046,6 +1144,8 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
     // of its results is used (one round trip), and every count or index read
     // back is clamped, so even a plan block of garbage cannot steer an
     // access out of its array.
+    // A slow path announced by the planner is waited for through the grid
+    // dependency, without a timeout report.
     if (tid == 0) {
         int ok = 0;
         for (int it = 0; it < READY_SPIN_LIMIT; ++it) {
@@ -1053,14 +1153,18 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
                 ok = 1;
                 break;
             }
+            if (ld_acquire(a.hdr + WS_SLOW) == seq + 1) {
+                ok = 2;
+                break;
+            }
             __nanosleep(64);
         }
         s_planned = ok;
     }
     __syncthreads();
-    if (!s_planned) {
+    if (s_planned != 1) {
         pdl_wait();
-        if (tid == 0) atomicOr(a.p.info + MOONEP_INFO_STATUS, MOONEP_ST_WAIT_TIMEOUT);
+        if (tid == 0 && s_planned == 0) atomicOr(a.p.info + MOONEP_INFO_STATUS, MOONEP_ST_WAIT_TIMEOUT);
     }
     const int status = ld_cg(a.p.info + MOONEP_INFO_STATUS);
     // host tables of the whole array; only entries inside the clamped

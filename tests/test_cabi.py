@@ -59,11 +59,10 @@ def test_config_checks_match_oracle(cuda_lib_path):
     assert oracle.check_config(oracle.Config(R=4, E=16, K=2, S=8, H=8, B=2, flags=64)) == 1
     assert oracle.check_config(oracle.Config(R=4, E=16, K=2, S=8, H=8, B=2, flags=8)) == 0
     assert moonep.check_config(moonep.Config(R=4, E=16, K=2, S=8, H=8, B=2, flags=8)) == 0
-    # the cascade's shared memory: the large shape fits, E = R = 1024 does not
-    moonep.plan_sizes(moonep.Config(R=32, E=384, K=8, S=4096, H=7168, B=12, flags=8))
-    assert moonep.check_config(moonep.Config(R=1024, E=1024, K=4, S=4, H=8, B=1, flags=8)) == 0
-    with pytest.raises(moonep.MoonepError):
-        moonep.plan_sizes(moonep.Config(R=1024, E=1024, K=4, S=4, H=8, B=1, flags=8))
+    # the cascade's shared memory fits the large shape and E = R = 1024 with
+    # the largest budget, and costs the plan nothing in device memory
+    for c in (dict(R=32, E=384, K=8, S=4096, H=7168, B=12), dict(R=1024, E=1024, K=4, S=4, H=8, B=1023)):
+        assert moonep.plan_sizes(moonep.Config(**c, flags=8)) == moonep.plan_sizes(moonep.Config(**c))
     # CUDA-only limits
     assert moonep.check_config(moonep.Config(R=4, E=16, K=2, S=8, H=12, B=2)) == 8
     assert moonep.check_config(moonep.Config(R=2, E=2048, K=2, S=8, H=8, B=2)) == 7

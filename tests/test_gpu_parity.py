@@ -297,6 +297,19 @@ def test_plan_over_budget_full_size(mp, flags):
     check_invariants(ocfg, topk, gp.to_numpy())
 
 
+@pytest.mark.parametrize("R,E,K,S,B", [(1024, 1024, 4, 64, 1), (256, 1024, 8, 256, 4), (64, 384, 8, 128, 4)])
+def test_plan_cascade_wide_shapes(mp, R, E, K, S, B):
+    """One empty rank among many: at E = R = 1024 the cascade makes 255
+    repairs on the largest lists; at R = 64, B = 4 no plan within budget
+    exists (rank 0 needs C rows from at most 4 replicas, each below C / 4)
+    and the overflow stays.  Against the oracle, with the host invariants."""
+    wl = W.Workload("wide", R, E, K, S, 8, B)
+    topk = W.over_budget_routing(wl).topk_idx.numpy()
+    _, ocfg, gp, op = _plan_both(mp, dict(R=R, E=E, K=K, S=S, H=8, B=B, flags=mp.FLAG_CASCADE), topk)
+    _assert_plan_equal(gp, op)
+    check_invariants(ocfg, topk, gp.to_numpy())
+
+
 def test_plan_many_chunks_multi_wave(mp):
     """More token chunks (512, in 32 groups) than two CTAs per SM can hold at
     once: both planner grids run in several waves, and assignment CTAs wait

@@ -378,46 +378,82 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
             np = __shfl_sync(FULL_MASK, np, 0);
             nl = __shfl_sync(FULL_MASK, nl, 0);
             __syncwarp();
-            // water-fill the moved replicas into the providers' home ranks
-            int mk = k0, pi = 0;
-            int al = mk < n ? mq[mk] : 0, cl = np > 0 ? pva[0] : 0;
-            while (mk < n && pi < np) {
-                if (cl <= 0) {
-                    ++pi;
-                    cl = pi < np ? pva[pi] : 0;
-                    continue;
-                }
-                if (al <= 0) {
-                    ++mk;
-                    al = mk < n ? mq[mk] : 0;
-                    continue;
-                }
-                const int amt = al < cl ? al : cl;
-                const int ek = me[mk], h = (int)fdiv((uint32_t)pve[pi], a.fL);
-                if ((int)fdiv((uint32_t)ek, a.fL) == h) {
-                    if (lane == 0) keep[ek] += amt;
-                } else {
-                    int found = -1;
-                    for (int q0 = 0; q0 < nl && found < 0; q0 += 32) {
-                        const int q = q0 + lane;
-                        const unsigned b = __ballot_sync(FULL_MASK, q < nl && le[q] == ek && lr[q] == h);
-                        if (b) found = q0 + __ffs(b) - 1;
+            // water-fill the moved replicas into the providers' home ranks:
+            // the moved quota [MS[i], MS[i+1]) of replica k0 + i meets
+            // provider p's [PV[p], PV[p+1]); each overlap, in (p, i) order,
+            // returns home, joins the replica of that expert already on the
+            // home rank (found through a per-expert tag of the rank's
+            // entries), or is appended
+            const int nm = n - k0;
+            int *MS = ordx, *PV = pvq, *tag = on_r;  // free by now: order, kept positions, relay marks
+            {
+                int run = 0;
+                for (int b0 = 0; b0 < nm; b0 += 32) {
+                    const int i = b0 + lane, v = i < nm ? mq[k0 + i] : 0;
+                    int x = v;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const int y = __shfl_up_sync(FULL_MASK, x, o);
+                        if (lane >= o) x += y;
                     }
-                    if (found >= 0) {
-                        if (lane == 0) lq[found] += amt;
-                    } else if (nl < lc) {
-                        if (lane == 0) {
-                            le[nl] = ek;
-                            lr[nl] = h;
-                            lq[nl] = amt;
-                            la[nl] = 1;
+                    if (i < nm) MS[i] = run + x - v;
+                    run += __shfl_sync(FULL_MASK, x, 31);
+                }
+                if (lane == 0) MS[nm] = run;
+                run = 0;
+                for (int b0 = 0; b0 < np; b0 += 32) {
+                    const int i = b0 + lane, v = i < np ? pva[i] : 0;
+                    int x = v;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const int y = __shfl_up_sync(FULL_MASK, x, o);
+                        if (lane >= o) x += y;
+                    }
+                    if (i < np) PV[i] = run + x - v;
+                    run += __shfl_sync(FULL_MASK, x, 31);
+                }
+                if (lane == 0) PV[np] = run;
+            }
+            for (int e = lane; e < E; e += 32) tag[e] = -1;
+            __syncwarp();
+            for (int pi = 0; pi < np; ++pi) {
+                const int lo = PV[pi], hi = PV[pi + 1];
+                if (hi <= lo || nm <= 0) continue;
+                const int h = (int)fdiv((uint32_t)pve[pi], a.fL);
+                const int i_lo = warp_last_le(MS, nm, lo), i_hi = warp_last_le(MS, nm, hi - 1);
+                const int nl0 = nl;
+                for (int q = lane; q < nl0; q += 32)
+                    if (lr[q] == h) tag[le[q]] = q;
+                __syncwarp();
+                for (int i0 = i_lo; i0 <= i_hi; i0 += 32) {
+                    const int i = i0 + lane;
+                    bool fresh = false;
+                    int ek = 0, amt = 0;
+                    if (i <= i_hi) {
+                        ek = me[k0 + i];
+                        amt = min(MS[i + 1], hi) - max(MS[i], lo);
+                        if ((int)fdiv((uint32_t)ek, a.fL) == h) {
+                            keep[ek] += amt;
+                        } else {
+                            const int t = tag[ek];
+                            if (t >= 0) lq[t] += amt;
+                            else fresh = true;
                         }
-                        ++nl;
                     }
+                    const unsigned b = __ballot_sync(FULL_MASK, fresh);
+                    const int pos = nl + __popc(b & lt);
+                    if (fresh && pos < lc) {
+                        le[pos] = ek;
+                        lr[pos] = h;
+                        lq[pos] = amt;
+                        la[pos] = 1;
+                    }
+                    nl = min(nl + __popc(b), lc);
                 }
                 __syncwarp();
-                al -= amt;
-                cl -= amt;
+                for (int q = lane; q < nl0; q += 32)
+                    if (lr[q] == h) tag[le[q]] = -1;
+                __syncwarp();
             }
         }
         if (lane == 0) s_nl = nl;

@@ -310,6 +310,33 @@ def test_plan_cascade_wide_shapes(mp, R, E, K, S, B):
     check_invariants(ocfg, topk, gp.to_numpy())
 
 
+@pytest.mark.parametrize("R,E,K,S,B", [(32, 384, 1, 3100, 12), (16, 64, 2, 40, 4), (16, 128, 2, 64, 8)])
+def test_cascade_plan_reduce_and_prefetch(mp, R, E, K, S, B):
+    """The replica-gradient reduce and the weight prefetch over a cascade
+    plan (relay replicas, merged replicas, returned quota), every element
+    against the oracle."""
+    wl = W.Workload("cx", R, E, K, S, 8, B)
+    topk = W.over_budget_routing(wl).topk_idx.numpy()
+    gcfg, ocfg, gp, op = _plan_both(mp, dict(R=R, E=E, K=K, S=S, H=8, B=B, flags=mp.FLAG_CASCADE), topk)
+    _assert_plan_equal(gp, op)
+    assert op["info"][0] == 0 and op["info"][2] == 0  # within budget, nothing overflows
+    P = 72
+    rb = W.f32_normal((R, B, P), seed=4, device=DEV, std=1e-3)
+    hg = W.f32_normal((E, P), seed=5, device=DEV, std=1e-3)
+    orb, ohg = rb.cpu().numpy(), hg.cpu().numpy()
+    mp.reduce_replica_grads(gcfg, gp, rb, hg)
+    oracle.reduce_replica_grads(ocfg, op, orb, ohg, P)
+    assert np.array_equal(hg.cpu().numpy(), ohg)
+    assert np.array_equal(rb.cpu().numpy(), orb)
+    weights = W.bf16_normal((E, P), seed=6, device=DEV)
+    pool = torch.full((R, B, P), float("nan"), dtype=torch.bfloat16, device=DEV)
+    opool = W.bits(pool).copy()
+    wrow = mp.prefetch_replicas(gcfg, gp, weights, pool)
+    owrow = oracle.prefetch_replicas(ocfg, op, W.bits(weights), opool, P)
+    assert np.array_equal(wrow.cpu().numpy(), owrow)
+    assert np.array_equal(W.bits(pool), opool)
+
+
 def test_plan_many_chunks_multi_wave(mp):
     """More token chunks (512, in 32 groups) than two CTAs per SM can hold at
     once: both planner grids run in several waves, and assignment CTAs wait

@@ -214,13 +214,17 @@ def _cascade_routing(rng, R, L, S, K=1):
     return ids.reshape(R * S, K).astype(np.int32)
 
 
-def test_plan_cascade_golden(mp):
-    g = json.load(open(os.path.join(GOLDEN, "plan_example_cascade.json")))
+@pytest.mark.parametrize("name", ["plan_example_cascade", "plan_example_cascade_relay"])
+def test_plan_cascade_golden(mp, name):
+    g = json.load(open(os.path.join(GOLDEN, name + ".json")))
     topk = np.array(g["topk_idx"], np.int32)
     gcfg, ocfg, gp, op = _plan_both(mp, g["config"], topk)
     _assert_plan_equal(gp, op)
     for k, v in g["expect"].items():
-        if k != "info":
+        if k == "info":
+            inf = gp.info()
+            assert {f: inf[f] for f in v} == v
+        else:
             assert gp.fields[k].cpu().numpy().tolist() == v, k
 
 

@@ -63,11 +63,16 @@ def test_golden_b_strict_flag(oracle_lib):
 
 # ------------------------------------------------------- relay cascade
 
-def test_golden_cascade_plan(oracle_lib):
-    """Hand-worked cascade: an empty rank filled from three small pieces with
-    B = 2 keeps two replicas, grows one of them, and relays the third piece to
-    the grown replica's home rank."""
-    g = json.load(open(os.path.join(GOLDEN, "plan_example_cascade.json")))
+@pytest.mark.parametrize("name,over_greedy", [("plan_example_cascade", 3), ("plan_example_cascade_relay", 2)])
+def test_golden_cascade_plan(oracle_lib, name, over_greedy):
+    """Hand-worked cascades.  plan_example_cascade: an empty rank filled from
+    three small pieces with B = 2 keeps two replicas, grows one of them, and
+    sends the third piece to the grown replica's home rank.
+    plan_example_cascade_relay: with B = 1 no kept replica can carry the
+    rest, so a relay expert of a third rank takes the empty rank's rows; the
+    moved replicas land on the relay's home rank, whose own repair finds no
+    provider with room, so it stays over B (one overflow replica)."""
+    g = json.load(open(os.path.join(GOLDEN, name + ".json")))
     cfg = oracle.Config(**g["config"])
     topk = np.array(g["topk_idx"], np.int32)
     p = oracle.plan(cfg, topk)
@@ -79,7 +84,7 @@ def test_golden_cascade_plan(oracle_lib):
     check_invariants(cfg, topk, p)
     # without the flag the same routing overflows the budget
     p0 = oracle.plan(oracle.Config(**{**g["config"], "flags": 0}), topk)
-    assert p0["info"][0] == oracle.ST_OVERFLOW and p0["info"][5] == 3
+    assert p0["info"][0] == oracle.ST_OVERFLOW and p0["info"][5] == over_greedy
 
 
 @pytest.mark.parametrize("wname,mv", [("tiny", 1.0), ("tiny", 0.0), ("mid", 1.0), ("mid", 3.0)])

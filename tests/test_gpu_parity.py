@@ -214,7 +214,8 @@ def _cascade_routing(rng, R, L, S, K=1):
     return ids.reshape(R * S, K).astype(np.int32)
 
 
-@pytest.mark.parametrize("name", ["plan_example_cascade", "plan_example_cascade_relay"])
+@pytest.mark.parametrize("name", ["plan_example_cascade", "plan_example_cascade_relay", "plan_example_cascade_merge",
+                                  "plan_example_cascade_chain", "plan_example_cascade_two_relays"])
 def test_plan_cascade_golden(mp, name):
     g = json.load(open(os.path.join(GOLDEN, name + ".json")))
     topk = np.array(g["topk_idx"], np.int32)

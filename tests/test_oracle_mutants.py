@@ -1,13 +1,25 @@
-"""Planted mistakes in the relay cascade of the oracle, each of which the
-hand-worked cascade plans (tests/golden/plan_example_cascade*.json) must
-reject.  Each mutant is a copy of oracle/moonep_oracle.c with one rule of
-the cascade changed, compiled with the oracle's own flags into a temporary
-directory; the test then plans every cascade golden with it and requires at
-least one expected field to differ.  Nothing here touches the CUDA library.
+"""Planted mistakes in the oracle, each of which its pins must reject.
 
-Not pinned: the capacity guard's threshold (a step is skipped when the live
-list plus m + B - 1 would exceed E + R - 1).  It binds only when the list is
-within one step of full, which no small routing reaches."""
+Each mutant is a copy of oracle/moonep_oracle.c with one plausible mistake
+(a reversed order or tie-break, a dropped rule or term, an off-by-one, a
+missing rounding or a wrong accumulation type), compiled with the oracle's
+own flags into a temporary directory.
+* Relay cascade mutants: every hand-worked cascade plan
+  (tests/golden/plan_example_cascade*.json) is planned with the mutant and
+  at least one expected field must differ.
+* Core plan, data-step, rounding and configuration mutants: the pin of
+  tests/test_oracle_pins.py that covers the step is run against the mutant
+  (the module's oracle swapped for it) and must fail.
+Nothing here touches the CUDA library.
+
+Not pinned, with the reason:
+* the cascade's capacity guard threshold (a step is skipped when the live
+  list plus m + B - 1 would exceed E + R - 1): it binds only when the list
+  is within one step of full, which no small routing reaches;
+* water-filling loops nested receiver-major instead of piece-major: an
+  equivalent program, since the north-west-corner overlaps form a staircase
+  rising in both the piece and the receiver index, so both nestings list
+  the replicas in the same order."""
 import importlib.util
 import json
 import os
@@ -35,8 +47,13 @@ static int cmp_val_asc_idx_asc(const void *a, const void *b)
     if (x->val != y->val) return x->val < y->val ? -1 : 1;
     return (x->idx > y->idx) - (x->idx < y->idx);
 }
+static int cmp_host_rank_desc(const void *a, const void *b)
+{
+    const host_t *x = (const host_t *)a, *y = (const host_t *)b;
+    return (x->rank < y->rank) - (x->rank > y->rank);
+}
 """
-CMP_ANCHOR = "typedef struct { int32_t rank, slot, quota, is_home; } host_t;"
+CMP_ANCHOR = "static int64_t min64(int64_t a, int64_t b)"
 
 # name -> [(text in the oracle, replacement)]
 MUTANTS = {
@@ -75,6 +92,105 @@ MUTANTS = {
          "if (alive[q]) { re[w] = re[q]; rr[w] = rr[q]; rq[w] = rq[q]; alive[w] = 1; ++w; }\n        *nl = w;\n"
          "        for (int32_t i = 0, j = w - 1; i < j; ++i, --j) { int32_t t; t = re[i]; re[i] = re[j]; re[j] = t;"
          " t = rr[i]; rr[i] = rr[j]; rr[j] = t; t = rq[i]; rq[i] = rq[j]; rq[j] = t; }")],
+}
+
+# name -> (edits, [(pin in test_oracle_pins, its arguments besides oracle_lib)])
+GOLDEN_A = [("test_golden_plan", {"name": "plan_example_a"})]
+GOLDEN_B = [("test_golden_plan", {"name": "plan_example_b"})]
+CASCADE_PINS = [("test_golden_cascade_plan", {"name": "plan_example_cascade", "over_greedy": 3}),
+                ("test_golden_cascade_plan", {"name": "plan_example_cascade_merge", "over_greedy": 2}),
+                ("test_golden_cascade_plan", {"name": "plan_example_cascade_chain", "over_greedy": 3})]
+CORE_MUTANTS = {
+    "O3 sheds the smallest experts first": (
+        [("qsort(order, (size_t)L, sizeof(vi_t), cmp_val_desc_idx_asc);",
+          "qsort(order, (size_t)L, sizeof(vi_t), cmp_val_asc_idx_asc);")], GOLDEN_A + CASCADE_PINS),
+    "O3 shedding ties by the higher expert": (
+        [("qsort(order, (size_t)L, sizeof(vi_t), cmp_val_desc_idx_asc);",
+          "qsort(order, (size_t)L, sizeof(vi_t), cmp_val_desc_idx_desc);")], GOLDEN_A),
+    "O4 pieces left in expert order": (
+        [("qsort(pieces, (size_t)nP, sizeof(vi_t), cmp_val_desc_idx_asc);", "")], GOLDEN_B),
+    "O4 piece ties by the higher expert": (
+        [("qsort(pieces, (size_t)nP, sizeof(vi_t), cmp_val_desc_idx_asc);",
+          "qsort(pieces, (size_t)nP, sizeof(vi_t), cmp_val_desc_idx_desc);")], CASCADE_PINS),
+    "O4 receivers left in rank order": (
+        [("qsort(recv, (size_t)nN, sizeof(vi_t), cmp_val_desc_idx_asc);", "")], CASCADE_PINS),
+    "O4 receiver ties by the higher rank": (
+        [("qsort(recv, (size_t)nN, sizeof(vi_t), cmp_val_desc_idx_asc);",
+          "qsort(recv, (size_t)nN, sizeof(vi_t), cmp_val_desc_idx_desc);")], CASCADE_PINS),
+    "O2 deficit off by one": (
+        [("        D[r] = h < C ? C - h : 0;", "        D[r] = h <= C ? C - h + 1 : 0;")], GOLDEN_B),
+    "O5 replica slots without the home offset": (
+        [("            rep_slot[nrep] = L + nrep_on[r];", "            rep_slot[nrep] = nrep_on[r];")], GOLDEN_A),
+    "O6 home slots count T instead of what stays home": (
+        [("            slot_count[(int64_t)r * E + j] = keep[r * L + j];",
+          "            slot_count[(int64_t)r * E + j] = T[r * L + j];")], GOLDEN_A),
+    "O7 home host first instead of rank order": (
+        [("        qsort(hosts, (size_t)nh, sizeof(host_t), cmp_host_rank);\n", "")], GOLDEN_B),
+    "O7 hosts in descending rank": (
+        [("        qsort(hosts, (size_t)nh, sizeof(host_t), cmp_host_rank);\n",
+          "        qsort(hosts, (size_t)nh, sizeof(host_t), cmp_host_rank_desc);\n")], GOLDEN_A),
+    "O8 pairs in (k, t) order": (
+        [("    for (int64_t p = 0; p < NP; ++p) {\n        int32_t e = topk[p];\n        int32_t g = gcount[e]++;",
+          "    for (int64_t pp = 0; pp < NP; ++pp) {\n        int64_t p = (pp % ((int64_t)R * S)) * K + pp / ((int64_t)R * S);\n"
+          "        int32_t e = topk[p];\n        int32_t g = gcount[e]++;")], GOLDEN_B),
+    "remote pairs: source rank without dividing by K": (
+        [("        int64_t src_rank = (p / K) / S;", "        int64_t src_rank = p / S;")], GOLDEN_B),
+    "overflow only above B": (
+        [("        if (rep_ord[q] >= B) ++n_over;", "        if (rep_ord[q] > B) ++n_over;")], GOLDEN_B),
+    "work list includes overflow replicas": (
+        [("            if (rep_expert[q] == e && rep_ord[q] < B) has = 1;",
+          "            if (rep_expert[q] == e) has = 1;")], GOLDEN_B),
+    "strict flag ignored": (
+        [("        if (c->flags & OR_FLAG_STRICT_BUDGET) status |= OR_ST_STRICT_VIOLATION;", "")],
+        [("test_golden_b_strict_flag", {})]),
+    "combine sums k in reverse": (
+        [("            for (int64_t k = 0; k < K; ++k) {\n                int64_t d = dst_pos[t * K + k];\n                acc = fmaf(",
+          "            for (int64_t k = K - 1; k >= 0; --k) {\n                int64_t d = dst_pos[t * K + k];\n                acc = fmaf(")],
+        [("test_combine_uses_fused_multiply_add", {})]),
+    "combine without fused multiply-add": (
+        [("acc = fmaf(w[t * K + k], bf16_to_f32(y[d * H + h]), acc);",
+          "acc = acc + w[t * K + k] * bf16_to_f32(y[d * H + h]);")], [("test_combine_uses_fused_multiply_add", {})]),
+    "combine rounds to bf16 after every k": (
+        [("acc = fmaf(w[t * K + k], bf16_to_f32(y[d * H + h]), acc);",
+          "acc = bf16_to_f32(or_f32_to_bf16(fmaf(w[t * K + k], bf16_to_f32(y[d * H + h]), acc)));")],
+        [("test_combine_error_bound", {})]),
+    "combine backward sums dw in fp32": (
+        [("            double s = 0.0;", "            float s = 0.0f;"),
+         ("                s += (double)g * (double)bf16_to_f32(y[d * H + h]);",
+          "                s += g * bf16_to_f32(y[d * H + h]);")], [("test_combine_backward_library", {})]),
+    "combine backward never scales dy": (
+        [("dy_buf[d * H + h] = unscaled ? dy[t * H + h] : or_f32_to_bf16(w[p] * g);",
+          "dy_buf[d * H + h] = dy[t * H + h];")], [("test_combine_backward_library", {})]),
+    "combine backward unscaled flag inverted": (
+        [("dy_buf[d * H + h] = unscaled ? dy[t * H + h] : or_f32_to_bf16(w[p] * g);",
+          "dy_buf[d * H + h] = !unscaled ? dy[t * H + h] : or_f32_to_bf16(w[p] * g);")],
+        [("test_combine_backward_library", {})]),
+    "reduce in descending rank order": (
+        [("        for (int32_t h = host_ptr[e]; h < host_ptr[e + 1]; ++h) {\n            int32_t r = host_rank[h], b = host_slot[h] - L;\n"
+          "            if (r == e / L) continue; /* the home copy */",
+          "        for (int32_t h = host_ptr[e + 1] - 1; h >= host_ptr[e]; --h) {\n            int32_t r = host_rank[h], b = host_slot[h] - L;\n"
+          "            if (r == e / L) continue; /* the home copy */")], [("test_reduce_order_is_rank_ascending", {})]),
+    "reduce leaves the replica rows": (
+        [("            for (int64_t i = i0; i < i1; ++i) src[i] = 0.0f;", "")], [("test_reduce_exact_integers", {})]),
+    "reduce includes overflow replicas": (
+        [("            if (b < 0 || b >= B) continue; /* overflow replica: no reduce rows */", "            if (b < 0) continue;")],
+        [("test_reduce_exact_integers", {})]),
+    "prefetch without read-through for overflow": (
+        [("                    row = e; /* overflow: read through to the home copy */", "                    row = -1;")],
+        [("test_prefetch_hand_worked", {})]),
+    "bf16 by truncation": ([("    u += 0x7fffu + lsb;", "    (void)lsb;")], [("test_bf16_rounding_matches_torch", {})]),
+    "bf16 ties away from zero": (
+        [("    u += 0x7fffu + lsb;", "    (void)lsb; u += 0x8000u;")], [("test_bf16_rounding_matches_torch", {})]),
+    "dispatch writes only the first k": (
+        [("        for (int64_t k = 0; k < K; ++k) {\n            int64_t d = dst_pos[t * K + k];\n            for (int64_t h = 0; h < H; ++h) buf",
+          "        for (int64_t k = 0; k < 1; ++k) {\n            int64_t d = dst_pos[t * K + k];\n            for (int64_t h = 0; h < H; ++h) buf")],
+        [("test_dispatch_rows", {})]),
+    "B range check against E": (
+        [("    if (c->B > c->E - L) return OR_ERR_B_RANGE;", "    if (c->B > c->E) return OR_ERR_B_RANGE;")],
+        [("test_config_errors", {})]),
+    "training budget rule ignored": (
+        [("    if ((c->flags & OR_FLAG_TRAIN_B_RULE) && c->B != L) return OR_ERR_BUDGET_RULE;", "")],
+        [("test_config_errors", {})]),
 }
 
 
@@ -128,3 +244,32 @@ def test_planted_mistake_is_caught(tmp_path, goldens, what):
     mod = _load_mutant(str(tmp_path), tag, MUTANTS[what])
     held = [n for n, g in zip(CASCADE_GOLDENS, goldens) if _golden_holds(mod, g)]
     assert len(held) < len(goldens), f"'{what}' passes every hand-worked cascade plan"
+
+
+@pytest.mark.parametrize("what", sorted(CORE_MUTANTS))
+def test_planted_core_mistake_is_caught(tmp_path, monkeypatch, what):
+    import test_oracle_pins as pins
+    edits, killers = CORE_MUTANTS[what]
+    tag = "".join(c if c.isalnum() else "_" for c in what)
+    mod = _load_mutant(str(tmp_path), tag, edits)
+    monkeypatch.setattr(pins, "oracle", mod)
+    caught = []
+    for fn, kw in killers:
+        try:
+            getattr(pins, fn)(mod, **kw)
+        except AssertionError:
+            caught.append(fn)
+    assert caught, f"'{what}' passes {[fn for fn, _ in killers]}"
+
+
+def test_unmutated_copy_passes_every_core_pin(tmp_path, monkeypatch):
+    import test_oracle_pins as pins
+    mod = _load_mutant(str(tmp_path), "none_core", [])
+    monkeypatch.setattr(pins, "oracle", mod)
+    seen = set()
+    for _, killers in CORE_MUTANTS.values():
+        for fn, kw in killers:
+            key = (fn, tuple(sorted(kw.items())))
+            if key not in seen:
+                seen.add(key)
+                getattr(pins, fn)(mod, **kw)

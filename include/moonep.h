@@ -108,7 +108,9 @@ extern "C" {
  * ready, plan ready; about 6 ms at the bound).  The pass then waits for the
  * whole histogram grid instead, so the plan is still complete; the bit
  * reports that a mark never came, which points at a workspace used by two
- * overlapping calls. */
+ * overlapping calls.  A relay cascade (MOONEP_FLAG_CASCADE), which can run
+ * for milliseconds, announces itself and is waited for the same way without
+ * setting this bit. */
 #define MOONEP_ST_WAIT_TIMEOUT 16
 /* The planner workspace did not hold the zeros a call must start from (it
  * was not zero-filled before first use, or two calls used it at once): the

@@ -14,6 +14,7 @@ implements.
 from __future__ import annotations
 
 import ctypes
+import struct
 import os
 import subprocess
 from dataclasses import dataclass
@@ -130,6 +131,13 @@ def check_config(cfg: Config) -> int:
 def f32_to_bf16(x: float) -> int:
     """Round-to-nearest-even fp32 -> bf16 bit pattern (oracle's own routine)."""
     return int(_load().or_f32_to_bf16(ctypes.c_float(x)))
+
+
+def f32_bits_to_bf16(bits: int) -> int:
+    """The same routine on an fp32 given by its bit pattern, passed unchanged
+    (a signalling NaN is not quieted on the way in)."""
+    f = ctypes.c_float.from_buffer_copy(struct.pack("<I", bits & 0xFFFFFFFF))
+    return int(_load().or_f32_to_bf16(f))
 
 
 def plan(cfg: Config, topk_idx: np.ndarray) -> dict:

@@ -376,6 +376,20 @@ def test_bf16_rounding_matches_torch(oracle_lib):
     assert (nan & 0x7f80) == 0x7f80 and (nan & 0x7f) != 0
 
 
+def test_bf16_nan_patterns(oracle_lib):
+    """A NaN stays a NaN with its sign: exponent all ones and a nonzero
+    mantissa in bf16, whatever the fp32 payload, including payloads wholly
+    below bit 16 that a plain truncation would turn into an infinity."""
+    for bits in (0x7F800001, 0xFF800001, 0x7F80FFFF, 0x7F810000, 0x7FA00000, 0x7FC00000, 0xFFFFFFFF):
+        r = oracle.f32_bits_to_bf16(bits)
+        assert (r & 0x7F80) == 0x7F80 and (r & 0x7F) != 0, hex(bits)
+        assert (r >> 15) == (bits >> 31), hex(bits)
+    # the default quiet NaN keeps its pattern
+    assert oracle.f32_bits_to_bf16(0x7FC00000) == 0x7FC0
+    # infinities stay infinities
+    assert oracle.f32_bits_to_bf16(0x7F800000) == 0x7F80 and oracle.f32_bits_to_bf16(0xFF800000) == 0xFF80
+
+
 def _tiny_plan(seed=0, mv=1.0):
     wl = W.WORKLOADS["tiny"]
     cfg = _cfg(wl)
@@ -578,3 +592,24 @@ def test_prefetch_hand_worked(oracle_lib):
     assert np.array_equal(pool[0, 0], w[6]) and np.array_equal(pool[1, 0], w[6])
     assert np.array_equal(pool[1, 1], w[4])
     assert (pool[0, 1] == 0xFFFF).all() and (pool[2:] == 0xFFFF).all()
+
+
+def test_prefetch_budget_above_L(oracle_lib):
+    # Example B with B = 3 != L = 2: all four replicas are prefetched,
+    # (e6, r0, slot 2) -> b 0, (e6, r1, slot 2) -> b 0, (e4, r1, slot 3) -> b 1,
+    # (e7, r1, slot 4) -> b 2.  Row space [weights (8 rows) | pool (R*B = 12
+    # rows)]: pool row of (r, b) = 8 + 3r + b.
+    g = json.load(open(os.path.join(GOLDEN, "plan_example_b.json")))
+    cfg = oracle.Config(**{**g["config"], "B": 3})
+    p = oracle.plan(cfg, np.array(g["topk_idx"], np.int32))
+    P = 3
+    w = np.arange(cfg.E * P, dtype=np.uint16).reshape(cfg.E, P)
+    pool = np.full((cfg.R, cfg.B, P), 0xFFFF, np.uint16)
+    wrow = oracle.prefetch_replicas(cfg, p, w, pool, P)
+    assert wrow.tolist() == [[0, 1, 8, -1, -1, -1, -1, -1],
+                             [2, 3, 11, 12, 13, -1, -1, -1],
+                             [4, 5, -1, -1, -1, -1, -1, -1],
+                             [6, 7, -1, -1, -1, -1, -1, -1]]
+    assert np.array_equal(pool[0, 0], w[6]) and np.array_equal(pool[1, 0], w[6])
+    assert np.array_equal(pool[1, 1], w[4]) and np.array_equal(pool[1, 2], w[7])
+    assert (pool[0, 1:] == 0xFFFF).all() and (pool[2:] == 0xFFFF).all()

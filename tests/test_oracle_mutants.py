@@ -21,7 +21,10 @@ Not pinned, with the reason:
   rising in both the piece and the receiver index, so both nestings list
   the replicas in the same order;
 * dropping the reduce's skip of the home host: equivalent, since the home
-  host's slot is below L and the prefetched-ordinal check skips it too."""
+  host's slot is below L and the prefetched-ordinal check skips it too;
+* starting the cascade, or picking a rank to repair, at exactly B replicas
+  instead of above B: equivalent, since a rank at B is picked only once no
+  open rank is over B, and its repair moves nothing."""
 import importlib.util
 import json
 import os
@@ -89,6 +92,18 @@ MUTANTS = {
         ("for (int32_t m = 0; m <= B && m_found < 0; ++m) {", "for (int32_t m = 0; m <= B; ++m) {")],
     "moved quota never joins an existing replica": [
         ("if (found >= 0) {\n                    rq[found]", "if (0) {\n                    rq[found]")],
+    "moved replicas water-filled in reverse order": [
+        ("        int32_t mk = k0, pi = 0;\n        int64_t a_left = mk < n ? sv_q[mk] : 0, c_left = np > 0 ? pa[0] : 0;",
+         "        for (int32_t i = k0, j = n - 1; i < j; ++i, --j) { int32_t t = sv_e[i]; sv_e[i] = sv_e[j]; sv_e[j] = t;"
+         " t = sv_q[i]; sv_q[i] = sv_q[j]; sv_q[j] = t; }\n"
+         "        int32_t mk = k0, pi = 0;\n        int64_t a_left = mk < n ? sv_q[mk] : 0, c_left = np > 0 ? pa[0] : 0;")],
+    "providers in reverse order": [
+        ("        /* pour Q into the providers */",
+         "        for (int32_t i = 0, j = np - 1; i < j; ++i, --j) { int32_t t = pe[i]; pe[i] = pe[j]; pe[j] = t;"
+         " t = pq[i]; pq[i] = pq[j]; pq[j] = t; }\n        /* pour Q into the providers */")],
+    "moved quota summed over the kept end of the order": [
+        ("            for (int32_t k = B - m; k < n; ++k) Q += S[k].val;",
+         "            for (int32_t k = 0; k < n - (B - m); ++k) Q += S[k].val;")],
     "list order reversed after a step": [
         ("if (alive[q]) { re[w] = re[q]; rr[w] = rr[q]; rq[w] = rq[q]; alive[w] = 1; ++w; }\n        *nl = w;",
          "if (alive[q]) { re[w] = re[q]; rr[w] = rr[q]; rq[w] = rq[q]; alive[w] = 1; ++w; }\n        *nl = w;\n"

@@ -104,6 +104,13 @@ def _check(rc: int):
 
 @dataclass(frozen=True)
 class Config:
+    """One MoE layer's shape (moonep_config in moonep.h): R simulated ranks,
+    E experts (E % R == 0, L = E/R home experts per rank), top-K, S tokens
+    per rank, hidden size H (a multiple of 8), replica budget B per rank, and
+    flags: FLAG_STRICT_BUDGET (overflow beyond B is a violation status),
+    FLAG_TRAIN_B_RULE (require B == E/R), FLAG_BWD_UNSCALED (combine
+    backward dispatches dy unscaled) and FLAG_CASCADE (the planner repairs
+    ranks that water-filling leaves over B by a relay cascade)."""
     R: int
     E: int
     K: int

@@ -112,6 +112,26 @@ def test_cascade_is_the_greedy_within_budget(oracle_lib, wname, mv):
         assert np.array_equal(p0[k], p1[k]), k
 
 
+def test_cascade_degenerate_configs_are_water_filling(oracle_lib):
+    """With no replica slots (B = 0) there is nothing to repair into, and a
+    single rank (R = 1) has no replicas: the cascade flag leaves the plan
+    exactly as water-filling makes it, overflow included."""
+    rng = np.random.default_rng(11)
+    for R, E, K, S, B in [(4, 16, 2, 64, 0), (8, 32, 1, 50, 0), (1, 8, 2, 40, 0)]:  # R = 1 allows only B = 0
+        w = rng.random(E) ** 4
+        T = rng.multinomial(R * S * K, w / w.sum())
+        ids = np.repeat(np.arange(E), T).astype(np.int32)
+        rng.shuffle(ids)
+        topk = ids.reshape(R * S, K)
+        c = dict(R=R, E=E, K=K, S=S, H=8, B=B)
+        p0 = oracle.plan(oracle.Config(**c), topk)
+        p1 = oracle.plan(oracle.Config(**c, flags=oracle.FLAG_CASCADE), topk)
+        for k in p0:
+            assert np.array_equal(p0[k], p1[k]), (c, k)
+        if B == 0 and R > 1:
+            assert p1["info"][0] & oracle.ST_OVERFLOW  # every replica overflows
+
+
 def test_cascade_empty_rank_counterexample(oracle_lib):
     """One empty rank and 31 ranks each C + C/31: water-filling puts 31
     replicas on the empty rank (B = 12); the cascade keeps every rank within

@@ -151,9 +151,11 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 // replica at the end of the list.  The rank is then closed; a step that
 // could make the list longer than E + R - 1 live entries is not taken.
 // The steps are inherently one after another and run on one warp over
-// shared-memory lists (searches, sums and compaction by ballot and shuffle);
-// the tables are then rebuilt from the list by the whole CTA.  Every index the step loops use is bounded by the list
-// capacity.
+// shared-memory lists (searches, sums and compaction by ballot and shuffle;
+// the water-fill one provider at a time, through a per-expert tag of the
+// entries on the provider's home rank); the tables are then rebuilt from the
+// list by the whole CTA.  Every index the step loops use is bounded by the
+// list capacity.
 __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep, const int *pe, const int *qr,
                              const int *segb, const int *pilo, const int *PS, const int *QSr, int qbase,
                              int n_rep, int nP, int nN, int *misc, int *wsum, int seq)

@@ -87,7 +87,8 @@ def measured_peaks():
 
 
 # the source files each measured kernel is compiled from: a kernel's ncu
-# counters stay valid while these are unchanged
+# counters stay valid while these are unchanged (the ABI header holds only
+# declarations and constants and is left out)
 KERNEL_SOURCES = {
     "dispatch": ("data.cu", "common.cuh"),
     "combine": ("data.cu", "common.cuh"),
@@ -101,20 +102,25 @@ def kernel_sources_hash(kernel: str) -> str:
     h = hashlib.sha256()
     for f in KERNEL_SOURCES[kernel]:
         h.update(open(os.path.join(ROOT, "load_balancing_moonep_b200", "csrc", f), "rb").read())
-    h.update(open(os.path.join(ROOT, "include", "moonep.h"), "rb").read())
     return h.hexdigest()[:16]
 
 
-def ncu_traffic():
-    """DRAM bytes per launch from the committed ncu summary, for each kernel
-    whose sources are unchanged since the capture."""
+def ncu_traffic_ratio():
+    """DRAM traffic / algorithmic bytes per launch, from the committed ncu
+    summary of the reduced-size profile cases (``bench.py --profile KERNEL``),
+    for each kernel whose sources are unchanged since the capture.  The
+    per-launch traffic of a timed launch is this ratio times its algorithmic
+    bytes: the per-token (per-row) bytes of these kernels do not depend on
+    the number of tokens (rows), so traffic scales with the units processed."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return {}
     d = json.load(open(p))
-    sha = d.get("sources_sha", {})
-    return {k: v for k, v in d.get("per_launch_bytes", {}).items()
-            if k in KERNEL_SOURCES and sha.get(k) == kernel_sources_hash(k)}
+    out = {}
+    for k, v in d.get("kernels", {}).items():
+        if k in KERNEL_SOURCES and v.get("sources_sha") == kernel_sources_hash(k):
+            out[k] = v["dram_bytes_per_launch"] / v["alg_bytes_per_launch"]
+    return out
 
 
 # ----------------------------------------------------------------- clocks
@@ -419,7 +425,8 @@ def run_ours(args, world, rank, local):
           "combine_bwd": bytes_combine_bwd(wl)}
     if P:
         kb["reduce"] = bytes_reduce(n_pref, info["n_rep_experts"], P)
-    traffic = ncu_traffic()
+    ratio = ncu_traffic_ratio()
+    traffic = {n: int(round(ratio[n] * b)) for n, b in kb.items() if n in ratio}
     kernels = {}
     for n, ms in t.items():
         gbs = kb[n] / (ms * 1e-3) / 1e9
@@ -429,7 +436,10 @@ def run_ours(args, world, rank, local):
     dom = max((n for n in t if n != "plan"), key=lambda n: t[n])
     roofline = {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["GB/s"], "peak": peak,
                 "peak_kind": peak_kind + " (MEASURED_PEAKS.json hbm_gbs, copy read+write)",
-                "unit": "GB/s", "frac": kernels[dom]["frac"], "traffic": traffic.get(dom)}
+                "unit": "GB/s", "frac": kernels[dom]["frac"], "traffic": traffic.get(dom),
+                "traffic_how": ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch of the "
+                                "reduced-size profile case (profiles/ncu_traffic.json), scaled to this "
+                                "launch by algorithmic bytes")}
 
     # maxvio sweep: dispatch / combine GB/s and planner us per point
     sweep = []
@@ -686,8 +696,9 @@ def run_ours(args, world, rank, local):
         torch.cuda.synchronize()
         pms = pt.total_ms("prefetch") / 5
         pbytes = n_pref * Pw * 2 * 2 + wl.R * wl.E * 8
+        ptraffic = int(round(ratio["prefetch"] * pbytes)) if "prefetch" in ratio else None
         kernels["prefetch"] = {"ms": round(pms, 4), "bytes": pbytes, "GB/s": round(pbytes / (pms * 1e-3) / 1e9, 1),
-                               "frac": round(pbytes / (pms * 1e-3) / 1e9 / peak, 4), "traffic": traffic.get("prefetch"),
+                               "frac": round(pbytes / (pms * 1e-3) / 1e9 / peak, 4), "traffic": ptraffic,
                                "in_step": False,
                                "what": f"{n_pref} replicas x {Pw} bf16 (gate+up+down) copied into the pool"}
         del weights, pool, wrow
@@ -715,7 +726,6 @@ def run_ours(args, world, rank, local):
 
     launches_per_step = 2 + 1 + 1 + 1 + (1 if P else 0)
     cfgd = workload_config(wl, r, args)
-    cfgd["reduce"] = f"P={P} fp32 ({reduce_note}), {n_pref} prefetched replicas over {info['n_rep_experts']} experts"
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
@@ -729,43 +739,81 @@ def run_ours(args, world, rank, local):
         "pages_sweep": {"workload": "ep8: R=8 E=256 K=8 S=4096 H=7168 B=4 (EP=8 as in the pages' sweep)",
                         "points": pages_sweep},
         "cascade": cascade, "clocks": clocks, "plan_info": info,
+        "reduce": (f"P={P} fp32 ({reduce_note}), {n_pref} prefetched replicas over "
+                   f"{info['n_rep_experts']} experts"),
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
 
 
+PROFILE_KERNELS = ("dispatch", "combine", "combine_bwd", "reduce", "prefetch", "plan")
+# elements per expert gradient / weight row in the profile case: enough that
+# the rows the plan touches exceed the 126 MB L2, while every buffer of the
+# case stays within a few GB
+PROFILE_P = {"reduce": 1 << 20, "prefetch": 1 << 21}
+
+
 def run_profile_case(args):
-    """--profile: two passes of the whole step (plus the replica weight
-    prefetch) on a reduced-size copy of the workload (S tokens per rank, P
-    gradient / weight elements per expert), a few GB on the device, for ncu
-    captures -- 7 launches per pass; prints a one-line summary, no timing."""
+    """--profile KERNEL: a reduced-size copy of the workload (S tokens per
+    rank, default 256; P gradient / weight elements per expert) for ncu
+    captures of ONE kernel: the plan, then two launches of that kernel (the
+    capture skips the first: ``-k regex:<kernel> -s 1 -c 1``).  Only the
+    buffers that kernel needs are allocated: at most about 3 GB on the
+    device.  Prints the case and the kernel's algorithmic bytes per launch
+    (the same byte model as the timed run), no timing."""
     from load_balancing_moonep_b200 import moonep as mp
+    kern = args.profile
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     wl = W.WORKLOADS[args.workload].with_(S=args.profile_S)
     cfg = mp.Config(R=wl.R, E=wl.E, K=wl.K, S=wl.S, H=wl.H, B=wl.B)
     r = W.routing(wl, args.maxvio, seed=0, device=dev)
-    hidden = W.hidden_states(wl, seed=1, device=dev)
-    dy = W.bf16_normal((wl.tokens, wl.H), seed=3, device=dev)
-    buf = torch.empty((wl.R, wl.C, wl.H), dtype=torch.bfloat16, device=dev)
-    dy_buf = torch.empty_like(buf)
-    out = torch.empty((wl.tokens, wl.H), dtype=torch.bfloat16, device=dev)
-    P = args.profile_P
-    rb = W.f32_normal((wl.R, wl.B, P), seed=4, device=dev, std=1e-3)
-    hg = W.f32_normal((wl.E, P), seed=5, device=dev, std=1e-3)
-    weights = W.bf16_normal((wl.E, P), seed=7, device=dev)
-    pool = torch.empty((wl.R, wl.B, P), dtype=torch.bfloat16, device=dev)
     plan = mp.Plan(cfg, dev)
-    for _ in range(2):
-        mp.plan(cfg, r.topk_idx, out=plan)
-        mp.prefetch_replicas(cfg, plan, weights, pool)
-        mp.dispatch(cfg, plan, hidden, buf)
-        mp.combine(cfg, plan, buf, r.weights, out)
-        mp.combine_backward(cfg, plan, dy, r.weights, buf, dy_buf)
-        mp.reduce_replica_grads(cfg, plan, rb, hg)
+    mp.plan(cfg, r.topk_idx, out=plan)
     torch.cuda.synchronize()
     info = plan.info()
-    print(json.dumps({"profile_case": f"{wl.name} S={wl.S} P={P}", "tokens": wl.tokens, "P": P,
+    n_pref = info["n_rep"] - info["n_overflow"]
+    P = args.profile_P or PROFILE_P.get(kern, 0)
+    if kern == "plan":
+        for _ in range(2):
+            mp.plan(cfg, r.topk_idx, out=plan)
+        alg = bytes_plan(wl)
+    elif kern == "dispatch":
+        hidden = W.hidden_states(wl, seed=1, device=dev)
+        buf = torch.empty((wl.R, wl.C, wl.H), dtype=torch.bfloat16, device=dev)
+        for _ in range(2):
+            mp.dispatch(cfg, plan, hidden, buf)
+        alg = bytes_dispatch(wl)
+    elif kern == "combine":
+        y = W.bf16_normal((wl.R, wl.C, wl.H), seed=2, device=dev)
+        out = torch.empty((wl.tokens, wl.H), dtype=torch.bfloat16, device=dev)
+        for _ in range(2):
+            mp.combine(cfg, plan, y, r.weights, out)
+        alg = bytes_combine(wl)
+    elif kern == "combine_bwd":
+        y = W.bf16_normal((wl.R, wl.C, wl.H), seed=2, device=dev)
+        dy = W.bf16_normal((wl.tokens, wl.H), seed=3, device=dev)
+        dy_buf = torch.empty_like(y)
+        for _ in range(2):
+            mp.combine_backward(cfg, plan, dy, r.weights, y, dy_buf)
+        alg = bytes_combine_bwd(wl)
+    elif kern == "reduce":
+        rb = W.f32_normal((wl.R, wl.B, P), seed=4, device=dev, std=1e-3)
+        hg = W.f32_normal((wl.E, P), seed=5, device=dev, std=1e-3)
+        for _ in range(2):
+            mp.reduce_replica_grads(cfg, plan, rb, hg)
+        alg = bytes_reduce(n_pref, info["n_rep_experts"], P)
+    elif kern == "prefetch":
+        weights = W.bf16_normal((wl.E, P), seed=7, device=dev)
+        pool = torch.empty((wl.R, wl.B, P), dtype=torch.bfloat16, device=dev)
+        for _ in range(2):
+            mp.prefetch_replicas(cfg, plan, weights, pool)
+        alg = n_pref * P * 2 * 2 + wl.R * wl.E * 8
+    else:
+        raise SystemExit(f"--profile: unknown kernel {kern}")
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": f"{wl.name} S={wl.S}" + (f" P={P}" if P else ""), "kernel": kern,
+                      "tokens": wl.tokens, "P": P, "alg_bytes_per_launch": alg,
                       "n_rep": info["n_rep"], "n_overflow": info["n_overflow"],
                       "n_rep_experts": info["n_rep_experts"],
                       "device_GB": round(torch.cuda.max_memory_allocated() / 1e9, 2)}), flush=True)
@@ -786,10 +834,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefetch", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--profile", action="store_true",
-                    help="run two untimed steps of a reduced-size case (for ncu)")
-    ap.add_argument("--profile-S", type=int, default=512)
-    ap.add_argument("--profile-P", type=int, default=1 << 20)
+    ap.add_argument("--profile", default=None, choices=PROFILE_KERNELS,
+                    help="run one kernel twice on a reduced-size case of a few GB (for ncu)")
+    ap.add_argument("--profile-S", type=int, default=256)
+    ap.add_argument("--profile-P", type=int, default=0,
+                    help="elements per expert row for reduce / prefetch (0: the kernel's default)")
     args = ap.parse_args()
     if args.profile:
         run_profile_case(args)

@@ -169,7 +169,11 @@ MOONEP_API int moonep_check_config(const moonep_config *cfg);
 
 /* Bytes of the plan block and of the planner workspace for `cfg`.
  * The workspace must be zero-filled once after allocation (for example
- * cudaMemset); every moonep_plan() call leaves it zero-filled again. */
+ * cudaMemset).  Every moonep_plan() call leaves it ready for the next call
+ * with the SAME configuration (its counters and sequence marks advanced, the
+ * count buffer of the next call zeroed); before it is used with a different
+ * configuration it must be zero-filled again, or the planner reports
+ * MOONEP_ST_WORKSPACE and returns an empty plan. */
 MOONEP_API int moonep_plan_sizes(const moonep_config *cfg, size_t *plan_bytes, size_t *workspace_bytes);
 
 /* Fills `out` with pointers into the device block `plan_base` of
@@ -271,9 +275,11 @@ MOONEP_API int moonep_prefetch_replicas(const moonep_config *cfg, const moonep_p
  *    launch.
  *  - The first call on a device looks up the array's device address with
  *    cudaGetSymbolAddress (once per device, the device current); make that
- *    first call before any stream capture.
- *  - Each call first clears the part of the array it uses (an async memset
- *    on `stream`), because the array keeps the previous call's contents.
+ *    first call before any stream capture.  Host threads may make their
+ *    first calls at the same time: the lookup is serialised and runs once.
+ *  - Each call first clears the front of the array that must start at zero
+ *    (the planner's counters and count buffers: an async memset on
+ *    `stream`), because the array keeps the previous call's contents.
  *  - All calls on a device share the one array: calls that can overlap on
  *    the GPU (different streams without ordering) race and give wrong plans.
  */
@@ -289,6 +295,18 @@ MOONEP_API const char *moonep_error_string(int code);
  * bytes, always NUL-terminated when len > 0); the return value is buf, or an
  * empty static string when buf is NULL or len == 0.  Host-only. */
 MOONEP_API const char *moonep_status_string(int status, char *buf, size_t len);
+
+/* Iteration bound of the assignment pass's two bounded waits (for the
+ * counts-ready and plan-ready marks of the histogram/planner pass; about
+ * 100 ns per iteration) for every moonep_plan / moonep_plan_noalloc call
+ * this process makes afterwards.  Default 65536; a negative value restores
+ * it.  With 0 both waits give up at once: the pass then waits for the whole
+ * histogram grid to finish (which that grid never depends on), so the plan
+ * is still complete and exact, and MOONEP_ST_WAIT_TIMEOUT is set.  This is
+ * how the fallback is tested without making a mark late.  Host-only; returns
+ * the previous bound.  Calls already enqueued keep the bound they were
+ * launched with. */
+MOONEP_API int moonep_set_wait_limit(int iterations);
 
 /* MOONEP_ABI_VERSION of the loaded library. */
 MOONEP_API int moonep_abi_version(void);

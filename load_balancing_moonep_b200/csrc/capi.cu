@@ -1,6 +1,7 @@
 // C ABI entry points (declared in include/moonep.h): host-side argument
 // checks, plan layout and kernel launches.  No call allocates memory or
 // synchronises the host.
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 
@@ -8,6 +9,7 @@
 
 namespace moonep {
 int launch_plan(const Dims &d, const int32_t *topk, const moonep_plan_t &p, void *ws, cudaStream_t st);
+int set_wait_limit(int iterations);
 size_t plan_smem_bytes_max(const Dims &d);
 int launch_dispatch(const Dims &d, const int *dst_pos, int *info, const uint16_t *hidden, uint16_t *buf,
                     cudaStream_t st);
@@ -23,7 +25,37 @@ int launch_prefetch(const Dims &d, const moonep_plan_t &p, const uint16_t *weigh
 constexpr size_t MAX_DYN_SMEM = 227 * 1024;
 constexpr int MAX_COMBINE_BWD_K = 16;
 
-static int make_dims(const moonep_config *c, Dims *d)
+// SMs of a B200.  The planner's token chunking is sized for it: the
+// workspace is laid out for that many chunks, so its size never depends on
+// which device is current when it is sized.
+constexpr int B200_SMS = 148;
+constexpr int MAX_DEVICES = 64;
+
+// SM count of the current device, cached per device (B200_SMS when no device
+// can be queried, e.g. for host-only sizing on a machine without a GPU).
+static int current_device_sms()
+{
+    static std::atomic<int> cache[MAX_DEVICES];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) {
+        (void)cudaGetLastError();
+        return B200_SMS;
+    }
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (n > 0) return n;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        (void)cudaGetLastError();
+        n = B200_SMS;
+    }
+    cache[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+
+// nsm: the SM count the chunking targets, at most B200_SMS (sizing uses
+// B200_SMS; a launch uses min(device SMs, B200_SMS), which never gives more
+// chunks than the sizing did, so the launch's workspace layout fits in the
+// sized workspace).
+static int make_dims(const moonep_config *c, Dims *d, int nsm = B200_SMS)
 {
     const int rc = moonep_check_config(c);
     if (rc != MOONEP_OK) return rc;
@@ -38,11 +70,14 @@ static int make_dims(const moonep_config *c, Dims *d)
     d->C = c->S * c->K;
     d->tokens = c->R * c->S;
     d->pairs = c->R * c->S * c->K;
-    // at most 2 x 148 - 1 chunks: two assignment CTAs fit on each SM of a
-    // B200 but one slot is held by the planner CTA while they start, and all
-    // of them should be resident then.  The chunking affects speed only,
-    // never the plan.
-    int ct = (d->tokens + 294) / 295;
+    // at most 2 x SMs - 1 chunks: two assignment CTAs fit on each SM but one
+    // slot is held by the planner CTA while they start, and all of them
+    // should be resident then.  The chunking affects speed only, never the
+    // plan.
+    if (nsm < 1) nsm = 1;
+    if (nsm > B200_SMS) nsm = B200_SMS;
+    const int target = 2 * nsm - 1;
+    int ct = (d->tokens + target - 1) / target;
     if (ct < 8) ct = 8;
     int cap = 4096 / d->K;
     if (cap < 1) cap = 1;
@@ -87,6 +122,19 @@ static PlanLayout plan_layout(const Dims &d)
     return l;
 }
 
+// Bytes at the start of the workspace that a call must find zeroed when the
+// workspace holds another configuration's leftovers: the header and both
+// group-count buffers (the per-chunk counts and host rows after them are
+// written in full before they are read).  Laid out for the current device.
+int workspace_clear_bytes(const moonep_config *cfg, size_t *bytes)
+{
+    Dims d;
+    const int rc = make_dims(cfg, &d, current_device_sms());
+    if (rc != MOONEP_OK) return rc;
+    *bytes = ws_layout(d).cc;
+    return MOONEP_OK;
+}
+
 }  // namespace moonep
 
 using namespace moonep;
@@ -94,6 +142,8 @@ using namespace moonep;
 extern "C" {
 
 int moonep_abi_version(void) { return MOONEP_ABI_VERSION; }
+
+int moonep_set_wait_limit(int iterations) { return set_wait_limit(iterations); }
 
 const char *moonep_error_string(int code)
 {
@@ -191,7 +241,7 @@ int moonep_plan(const moonep_config *cfg, const int32_t *topk_idx, const moonep_
                 void *stream)
 {
     Dims d;
-    const int rc = make_dims(cfg, &d);
+    const int rc = make_dims(cfg, &d, current_device_sms());
     if (rc != MOONEP_OK) return rc;
     if (!topk_idx || !plan_ok(plan) || !workspace) return MOONEP_ERR_ARG;
     return launch_plan(d, topk_idx, *plan, workspace, static_cast<cudaStream_t>(stream));

@@ -42,6 +42,8 @@
 //                     histogram CTAs write the tables' empty defaults
 //                     before the planner writes over them, so no pass fills
 //                     the unused rest afterwards.)
+#include <atomic>
+
 #include "common.cuh"
 
 namespace moonep {
@@ -63,7 +65,17 @@ struct PlanParams {
     int *cc;         // [nchunk][E]
     int *host_dst0;  // [2E+R]
     FastDiv fC, fL;  // divisions by C and L
+    int spin_limit;  // iterations of each bounded wait of the assignment pass
 };
+
+// The bound of the assignment pass's two waits, for every later launch in
+// the process (moonep_set_wait_limit).
+static std::atomic<int> g_wait_limit{READY_SPIN_LIMIT};
+
+int set_wait_limit(int iterations)
+{
+    return g_wait_limit.exchange(iterations < 0 ? READY_SPIN_LIMIT : iterations);
+}
 
 // ints of dynamic shared memory used by the planner block
 __host__ __device__ inline int plan_smem_ints(int E, int R)
@@ -1104,7 +1116,7 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
     if (tid == 0) {
         const int seq = ld_cg(a.hdr + WS_SEQ);
         int ok = 0;
-        for (int it = 0; it < READY_SPIN_LIMIT; ++it) {
+        for (int it = 0; it < a.spin_limit; ++it) {
             if (ld_acquire(a.hdr + WS_READY) == seq + 1) {
                 ok = 1;
                 break;
@@ -1186,7 +1198,7 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
     // dependency, without a timeout report.
     if (tid == 0) {
         int ok = 0;
-        for (int it = 0; it < READY_SPIN_LIMIT; ++it) {
+        for (int it = 0; it < a.spin_limit; ++it) {
             if (ld_acquire(a.hdr + WS_PLANNED) == seq + 1) {
                 ok = 1;
                 break;
@@ -1309,6 +1321,7 @@ int launch_plan(const Dims &d, const int32_t *topk, const moonep_plan_t &p, void
     a.host_dst0 = reinterpret_cast<int *>(w + wl.host_dst0);
     a.fC = make_fastdiv((uint32_t)d.C);
     a.fL = make_fastdiv((uint32_t)d.L);
+    a.spin_limit = g_wait_limit.load(std::memory_order_relaxed);
 
     // both kernels with programmatic dependent launch: each may be placed
     // while its predecessor drains and waits (griddepcontrol.wait, or the

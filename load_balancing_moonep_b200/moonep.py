@@ -53,7 +53,8 @@ PLAN_FIELDS = ("expert_count", "slot_expert", "slot_count", "slot_offset", "rep_
 EXPORTED = ("moonep_check_config", "moonep_plan_sizes", "moonep_plan_layout", "moonep_plan",
             "moonep_dispatch", "moonep_combine", "moonep_combine_backward",
             "moonep_reduce_replica_grads", "moonep_error_string", "moonep_abi_version",
-            "moonep_plan_noalloc", "moonep_prefetch_replicas", "moonep_status_string")
+            "moonep_plan_noalloc", "moonep_prefetch_replicas", "moonep_status_string",
+            "moonep_set_wait_limit")
 
 
 class _CConfig(ctypes.Structure):
@@ -84,6 +85,7 @@ _lib.moonep_error_string.restype = ctypes.c_char_p
 _lib.moonep_status_string.argtypes = [ctypes.c_int, ctypes.c_char_p, ctypes.c_size_t]
 _lib.moonep_status_string.restype = ctypes.c_char_p
 _lib.moonep_abi_version.argtypes = []
+_lib.moonep_set_wait_limit.argtypes = [ctypes.c_int]
 for _f in EXPORTED:
     if _f not in ("moonep_error_string", "moonep_status_string"):
         getattr(_lib, _f).restype = ctypes.c_int
@@ -160,7 +162,8 @@ class Plan:
         self.cfg = cfg
         pb, wb = plan_sizes(cfg)
         self.block = torch.zeros(pb, dtype=torch.uint8, device=device)
-        # zero-filled once; every plan call leaves it zero-filled again
+        # zero-filled once; every plan call leaves it ready for the next call
+        # with this configuration
         self.workspace = torch.zeros(max(wb, 256), dtype=torch.uint8, device=device)
         self.c_plan = _CPlan()
         c = cfg.c()
@@ -194,13 +197,6 @@ class Plan:
         """Status and statistics (synchronises with the device)."""
         v = self.fields["info"].cpu().tolist()
         return {k: v[i] for i, k in enumerate(INFO_FIELDS)}
-
-    def maxvio(self) -> float:
-        """maxvio = max_e T_e / T_bar - 1 of the planned routing, with
-        T_bar = S*K*R/E (synchronises with the device)."""
-        T = self.fields["expert_count"].cpu()
-        c = self.cfg
-        return float(T.max()) / (c.S * c.K * c.R / c.E) - 1.0
 
     def to_numpy(self) -> dict:
         return {k: v.cpu().numpy() for k, v in self.fields.items()}
@@ -348,6 +344,14 @@ def views(cfg: Config, p: Plan, buf: torch.Tensor):
             row.append((e, buf[r, int(so[r, s]):int(so[r, s + 1])]))
         out.append(row)
     return out
+
+
+def set_wait_limit(iterations: int) -> int:
+    """Iteration bound of the planner's two bounded waits for later plan
+    calls in this process (negative: the default); returns the previous one.
+    0 makes both waits take their fallback (MOONEP_ST_WAIT_TIMEOUT set, plan
+    still exact)."""
+    return _lib.moonep_set_wait_limit(int(iterations))
 
 
 def abi_version() -> int:

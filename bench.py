@@ -746,26 +746,32 @@ def run_ours(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
-PROFILE_KERNELS = ("dispatch", "combine", "combine_bwd", "reduce", "prefetch", "plan")
-# elements per expert gradient / weight row in the profile case: enough that
-# the rows the plan touches exceed the 126 MB L2, while every buffer of the
-# case stays within a few GB
-PROFILE_P = {"reduce": 1 << 20, "prefetch": 1 << 21}
+# The ncu profile case of each kernel: (workload, tokens per rank S, elements
+# per expert row P).  The data kernels run the large training shape with
+# fewer tokens per rank; the reduce and the prefetch run the tiny shape with
+# long rows, so that the few rows its plan touches still move several times
+# the 126 MB L2 while every buffer of the case stays within a few GB.
+PROFILE_CASES = {
+    "dispatch": ("large", 512, 0), "combine": ("large", 512, 0), "combine_bwd": ("large", 512, 0),
+    "reduce": ("tiny", 256, 1 << 24), "prefetch": ("tiny", 256, 1 << 25), "plan": ("large", 4096, 0),
+}
+PROFILE_KERNELS = tuple(PROFILE_CASES)
 
 
 def run_profile_case(args):
-    """--profile KERNEL: a reduced-size copy of the workload (S tokens per
-    rank, default 256; P gradient / weight elements per expert) for ncu
+    """--profile KERNEL: the kernel's reduced-size profile case
+    (PROFILE_CASES; --profile-S / --profile-P override S and P) for ncu
     captures of ONE kernel: the plan, then two launches of that kernel (the
-    capture skips the first: ``-k regex:<kernel> -s 1 -c 1``).  Only the
-    buffers that kernel needs are allocated: at most about 3 GB on the
+    capture skips the first: ``-k regex:moonep::<kernel> -s 1 -c 1``).  Only
+    the buffers that kernel needs are allocated: at most about 4 GB on the
     device.  Prints the case and the kernel's algorithmic bytes per launch
     (the same byte model as the timed run), no timing."""
     from load_balancing_moonep_b200 import moonep as mp
     kern = args.profile
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    wl = W.WORKLOADS[args.workload].with_(S=args.profile_S)
+    wname, S_case, P_case = PROFILE_CASES[kern]
+    wl = W.WORKLOADS[wname].with_(S=args.profile_S or S_case)
     cfg = mp.Config(R=wl.R, E=wl.E, K=wl.K, S=wl.S, H=wl.H, B=wl.B)
     r = W.routing(wl, args.maxvio, seed=0, device=dev)
     plan = mp.Plan(cfg, dev)
@@ -773,7 +779,7 @@ def run_profile_case(args):
     torch.cuda.synchronize()
     info = plan.info()
     n_pref = info["n_rep"] - info["n_overflow"]
-    P = args.profile_P or PROFILE_P.get(kern, 0)
+    P = args.profile_P or P_case
     if kern == "plan":
         for _ in range(2):
             mp.plan(cfg, r.topk_idx, out=plan)
@@ -836,9 +842,9 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--profile", default=None, choices=PROFILE_KERNELS,
                     help="run one kernel twice on a reduced-size case of a few GB (for ncu)")
-    ap.add_argument("--profile-S", type=int, default=256)
+    ap.add_argument("--profile-S", type=int, default=0, help="tokens per rank (0: the kernel's case)")
     ap.add_argument("--profile-P", type=int, default=0,
-                    help="elements per expert row for reduce / prefetch (0: the kernel's default)")
+                    help="elements per expert row for reduce / prefetch (0: the kernel's case)")
     args = ap.parse_args()
     if args.profile:
         run_profile_case(args)

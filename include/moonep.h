@@ -127,6 +127,12 @@ extern "C" {
 #define MOONEP_INFO_MAX_REP_PER_RANK 5
 #define MOONEP_INFO_N_REP_EXPERTS 6    /* experts with >= 1 prefetched replica */
 #define MOONEP_INFO_N_REMOTE_PAIRS 7   /* pairs whose buffer rank != source rank */
+/* Relay cascade (MOONEP_FLAG_CASCADE) only, 0 otherwise: the repair steps
+ * that found providers and so reached the capacity guard, and the least
+ * slack the guard saw, (E + R - 1) - (live replicas + m + B - 1); a step
+ * with negative slack is not taken. */
+#define MOONEP_INFO_CASCADE_GUARD_STEPS 8
+#define MOONEP_INFO_CASCADE_GUARD_SLACK 9
 #define MOONEP_INFO_LEN 16
 
 typedef struct moonep_config {

@@ -216,6 +216,7 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
             misc[3] = 0;
         }
         int nl = min(n_rep, lc);
+        int n_guard = 0, min_slack = 0;  // steps that reached the capacity guard, its least slack
         for (int step = 0; step <= R; ++step) {
             for (int r = lane; r < R; r += 32) cnt[r] = 0;
             __syncwarp();
@@ -316,7 +317,12 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
             if (lane == 0) closed[rs] = 1;
             __syncwarp();
             if (m_found < 0) continue;
-            if (nl + m_found + B - 1 > cap) continue;  // the list could outgrow the plan's arrays
+            // the step may add m + B - 1 live replicas: the list could
+            // outgrow the plan's arrays when the slack is negative
+            const int slack = cap - (nl + m_found + B - 1);
+            if (n_guard == 0 || slack < min_slack) min_slack = slack;
+            ++n_guard;
+            if (slack < 0) continue;
             const int k0 = B - m_found;
             // the rank's replicas by step order: experts and quotas; a kept
             // replica's position once the moved ones are dropped
@@ -470,7 +476,11 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
                 __syncwarp();
             }
         }
-        if (lane == 0) s_nl = nl;
+        if (lane == 0) {
+            s_nl = nl;
+            misc[4] = n_guard;
+            misc[5] = min_slack;
+        }
     }
     __syncthreads();
     const int nl = s_nl;
@@ -592,6 +602,8 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
         a.p.info[MOONEP_INFO_MAX_REP_PER_RANK] = misc[3];
         a.p.info[MOONEP_INFO_N_REP_EXPERTS] = n_rep_experts;
         for (int i = MOONEP_INFO_N_REMOTE_PAIRS; i < MOONEP_INFO_LEN; ++i) a.p.info[i] = 0;
+        a.p.info[MOONEP_INFO_CASCADE_GUARD_STEPS] = misc[4];
+        a.p.info[MOONEP_INFO_CASCADE_GUARD_SLACK] = misc[5];
     }
     // every thread's plan writes precede the plan-ready mark
     __syncthreads();
@@ -637,7 +649,7 @@ __device__ void plan_block(const PlanParams &a, int *sm, int seq)
     int *hq = hs + nh;             // nh  receiver deficits, while sorting
     int *flag = hq + nh;           // E
     int *wsum = flag + E;          // 32
-    int *misc = wsum + 32;         // 16: 0 status in, 2 n_over, 3 max replicas per rank
+    int *misc = wsum + 32;         // 16: 0 status in, 2 n_over, 3 max replicas per rank, 4-5 cascade guard
 
     __shared__ unsigned s_part[2][32];
     for (int i = tid; i < 16; i += nt) misc[i] = 0;

@@ -43,7 +43,8 @@ ST_WAIT_TIMEOUT = 16
 ST_WORKSPACE = 32
 
 INFO_FIELDS = ("status", "n_rep", "n_overflow", "n_pieces", "n_receivers",
-               "max_rep_per_rank", "n_rep_experts", "n_remote_pairs")
+               "max_rep_per_rank", "n_rep_experts", "n_remote_pairs", "cascade_guard_steps",
+               "cascade_guard_slack")
 INFO_LEN = 16
 
 PLAN_FIELDS = ("expert_count", "slot_expert", "slot_count", "slot_offset", "rep_expert", "rep_rank",

@@ -36,7 +36,8 @@ ST_STRICT_VIOLATION = 4
 
 INFO_FIELDS = (
     "status", "n_rep", "n_overflow", "n_pieces", "n_receivers",
-    "max_rep_per_rank", "n_rep_experts", "n_remote_pairs",
+    "max_rep_per_rank", "n_rep_experts", "n_remote_pairs", "cascade_guard_steps",
+    "cascade_guard_slack",
 )
 INFO_LEN = 16
 

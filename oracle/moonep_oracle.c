@@ -84,6 +84,8 @@
 #define OR_INFO_MAX_REP_PER_RANK 5
 #define OR_INFO_N_REP_EXPERTS 6
 #define OR_INFO_N_REMOTE_PAIRS 7
+#define OR_INFO_CASCADE_GUARD_STEPS 8
+#define OR_INFO_CASCADE_GUARD_SLACK 9
 #define OR_INFO_LEN 16
 
 typedef struct {
@@ -195,7 +197,8 @@ static int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
  * by the caller.  re/rr/rq/alive: list arrays of capacity
  * lcap >= 2 * cap + 2 * B + 2; *nl: entries used. */
 static int or_cascade(int32_t R, int32_t E, int32_t L, int32_t B, int32_t cap, int32_t *keep,
-                      int32_t *re, int32_t *rr, int32_t *rq, int32_t *alive, int32_t *nl, int32_t lcap)
+                      int32_t *re, int32_t *rr, int32_t *rq, int32_t *alive, int32_t *nl, int32_t lcap,
+                      int32_t *n_guard, int32_t *min_slack)
 {
     int32_t *cnt = calloc((size_t)R, sizeof(int32_t));
     int32_t *closed = calloc((size_t)R, sizeof(int32_t));
@@ -265,7 +268,12 @@ static int or_cascade(int32_t R, int32_t E, int32_t L, int32_t B, int32_t cap, i
         }
         closed[rs] = 1;
         if (m_found < 0) continue;
-        if (*nl + m_found + B - 1 > cap) continue; /* the list could outgrow the plan's arrays */
+        /* the guard: the step may add m + B - 1 live replicas; its slack is
+         * recorded (the smallest over the steps that reach it) */
+        const int32_t slack = cap - (*nl + m_found + B - 1);
+        if (*n_guard == 0 || slack < *min_slack) *min_slack = slack;
+        *n_guard += 1;
+        if (slack < 0) continue; /* the list could outgrow the plan's arrays */
         /* the moved replicas' experts and quotas, before anything changes */
         for (int32_t k = 0; k < n; ++k) { sv_e[k] = re[S[k].idx]; sv_q[k] = rq[S[k].idx]; }
         int overfull = 0;
@@ -349,6 +357,7 @@ int or_plan(const or_config *c, const int32_t *topk,
     const int64_t C = (int64_t)S * K;      /* slots per rank [P1 core idea] */
     const int64_t NP = (int64_t)R * S * K; /* number of (token, k) pairs */
     const int32_t NREP_MAX = E + R, NHOST_MAX = 2 * E + R;
+    int32_t n_guard = 0, min_slack = 0; /* cascade steps that reached the capacity guard, its least slack */
 
     /* default (empty) outputs */
     for (int64_t i = 0; i < (int64_t)R * E; ++i) { slot_expert[i] = -1; slot_count[i] = 0; }
@@ -461,7 +470,7 @@ int or_plan(const or_config *c, const int32_t *topk,
             }
             for (int32_t q = 0; q < nrep; ++q) { le[q] = rep_expert[q]; lr[q] = rep_rank[q]; lq[q] = rep_quota[q]; la[q] = 1; }
             int32_t nl = nrep;
-            rc = or_cascade(R, E, L, B, NREP_MAX - 1, keep, le, lr, lq, la, &nl, lcap);
+            rc = or_cascade(R, E, L, B, NREP_MAX - 1, keep, le, lr, lq, la, &nl, lcap, &n_guard, &min_slack);
             if (rc == OR_OK) {
                 /* the final list, ordinals re-derived in list order */
                 for (int32_t r = 0; r < R; ++r) nrep_on[r] = 0;
@@ -575,6 +584,8 @@ int or_plan(const or_config *c, const int32_t *topk,
     info[OR_INFO_MAX_REP_PER_RANK] = max_rep;
     info[OR_INFO_N_REP_EXPERTS] = n_rep_experts;
     info[OR_INFO_N_REMOTE_PAIRS] = (int32_t)n_remote;
+    info[OR_INFO_CASCADE_GUARD_STEPS] = n_guard;
+    info[OR_INFO_CASCADE_GUARD_SLACK] = min_slack;
 
 out:
     free(Hl); free(X); free(D); free(shed); free(keep); free(order); free(pieces);

@@ -12,10 +12,17 @@ own flags into a temporary directory.
   (the module's oracle swapped for it) and must fail.
 Nothing here touches the CUDA library.
 
+The cascade's capacity guard (a step is skipped when the live list plus
+m + B - 1 would exceed E + R - 1) is pinned in two parts.  Its arithmetic:
+the slack it computes is reported in the plan's info, hand-worked in every
+cascade golden, so the mutants below that change the sum or the capacity are
+caught there.  Its comparison: on every routing of the small shapes that
+tests/test_oracle_pins.py enumerates exhaustively, the least slack any step
+reaches is 3, so moving the threshold by one or two either way (taking the
+step at a slack of -1 or -2, refusing it at 0 or 1) gives the same plan on
+all of them; those variants are not planted.
+
 Not pinned, with the reason:
-* the cascade's capacity guard threshold (a step is skipped when the live
-  list plus m + B - 1 would exceed E + R - 1): it binds only when the list
-  is within one step of full, which no small routing reaches;
 * water-filling loops nested receiver-major instead of piece-major: an
   equivalent program, since the north-west-corner overlaps form a staircase
   rising in both the piece and the receiver index, so both nestings list
@@ -104,6 +111,16 @@ MUTANTS = {
     "moved quota summed over the kept end of the order": [
         ("            for (int32_t k = B - m; k < n; ++k) Q += S[k].val;",
          "            for (int32_t k = 0; k < n - (B - m); ++k) Q += S[k].val;")],
+    "guard counts the step's growth as m + B": [
+        ("const int32_t slack = cap - (*nl + m_found + B - 1);", "const int32_t slack = cap - (*nl + m_found + B);")],
+    "guard leaves the relays out": [
+        ("const int32_t slack = cap - (*nl + m_found + B - 1);", "const int32_t slack = cap - (*nl + B - 1);")],
+    "guard counts the rank's replicas instead of the list": [
+        ("const int32_t slack = cap - (*nl + m_found + B - 1);", "const int32_t slack = cap - (n + m_found + B - 1);")],
+    "guard capacity E + R": [
+        ("const int32_t slack = cap - (*nl + m_found + B - 1);", "const int32_t slack = cap + 1 - (*nl + m_found + B - 1);")],
+    "guard slack kept from the last step, not the least": [
+        ("if (*n_guard == 0 || slack < *min_slack) *min_slack = slack;", "*min_slack = slack;")],
     "list order reversed after a step": [
         ("if (alive[q]) { re[w] = re[q]; rr[w] = rr[q]; rq[w] = rq[q]; alive[w] = 1; ++w; }\n        *nl = w;",
          "if (alive[q]) { re[w] = re[q]; rr[w] = rr[q]; rq[w] = rq[q]; alive[w] = 1; ++w; }\n        *nl = w;\n"

@@ -10,6 +10,7 @@
 * library routines for the floating-point steps (torch's bf16 rounding,
   numpy's fp64 dot, numpy fp32 products) and exact integer-valued cases.
 """
+import itertools
 import json
 import os
 
@@ -99,6 +100,45 @@ def test_golden_cascade_plan(oracle_lib, name, over_greedy):
     # without the flag the same routing overflows the budget
     p0 = oracle.plan(oracle.Config(**{**g["config"], "flags": 0}), topk)
     assert p0["info"][0] == oracle.ST_OVERFLOW and p0["info"][5] == over_greedy
+
+
+def _compositions(n, k):
+    """Every way to write n as an ordered sum of k non-negative parts."""
+    for cut in itertools.combinations(range(n + k - 1), k - 1):
+        prev, parts = -1, []
+        for c in cut:
+            parts.append(c - prev - 1)
+            prev = c
+        parts.append(n + k - 2 - prev)
+        yield parts
+
+
+@pytest.mark.parametrize("R,L,S_max", [(3, 1, 8), (4, 1, 5), (5, 1, 2), (2, 2, 6), (2, 3, 3), (3, 2, 3),
+                                       (4, 2, 2)])
+def test_cascade_guard_slack_over_every_small_routing(oracle_lib, R, L, S_max):
+    """The relay cascade's capacity guard, exhaustively on small shapes: for
+    every expert-count vector of every S <= S_max (K = 1, so the counts are
+    the routing) and every budget B, each step that reaches the guard must
+    leave a slack of at least 3 (E + R - 1 minus the live replicas, m and
+    B - 1).  So no threshold within two of the guard's can change a plan on
+    these inputs; the least slack reached is exactly 3 on the single-expert
+    ranks (R = 3, 4), showing the check is not vacuous.  (Hand-worked slacks
+    pin the guard's arithmetic in the cascade goldens.)"""
+    E = R * L
+    least = None
+    for S in range(1, S_max + 1):
+        for T in _compositions(R * S, E):
+            topk = np.repeat(np.arange(E, dtype=np.int32), T).reshape(R * S, 1)
+            for B in range(1, E - L + 1):
+                p = oracle.plan(oracle.Config(R=R, E=E, K=1, S=S, H=8, B=B, flags=oracle.FLAG_CASCADE), topk)
+                inf = oracle.info_dict(p)
+                if inf["cascade_guard_steps"] > 0:
+                    assert inf["cascade_guard_slack"] >= 3, (S, T, B, inf)
+                    least = inf["cascade_guard_slack"] if least is None else min(least, inf["cascade_guard_slack"])
+                else:
+                    assert inf["cascade_guard_slack"] == 0
+    if L == 1 and R in (3, 4):
+        assert least == 3
 
 
 @pytest.mark.parametrize("wname,mv", [("tiny", 1.0), ("tiny", 0.0), ("mid", 1.0), ("mid", 3.0)])

@@ -240,26 +240,52 @@ def sum_over_ranks(world, x: float) -> float:
 
 # ------------------------------------------------------------ CPU oracle
 
-def oracle_sample(wl, topk_np, w_np, hidden_sample_bits, tokens, y_rows_bits):
+def oracle_sample(wl, topk_np, w_np, hidden_sample_bits, tokens, y_rows_bits, lib=None, plan=True):
     """Time the CPU oracle on a bounded sample: the plan over the whole
-    routing, dispatch and combine over the sampled tokens.  Returns
-    (plan_s, data_s, data_bytes)."""
+    routing (unless plan=False), dispatch and combine over the sampled
+    tokens (lib: the oracle build to run them with; default the
+    single-threaded oracle).  Returns (plan_s, data_s, data_bytes)."""
     import oracle
     ocfg = oracle.Config(R=wl.R, E=wl.E, K=wl.K, S=wl.S, H=wl.H, B=wl.B)
     t0 = time.perf_counter()
-    op = oracle.plan(ocfg, topk_np)
+    info = oracle.plan(ocfg, topk_np)["info"] if plan else np.zeros(16, np.int32)
     t1 = time.perf_counter()
     n = len(tokens)
-    sub = {"dst_pos": np.arange(n * wl.K, dtype=np.int32).reshape(n, wl.K), "info": op["info"]}
+    sub = {"dst_pos": np.arange(n * wl.K, dtype=np.int32).reshape(n, wl.K), "info": info}
     scfg = oracle.Config(R=1, E=wl.E, K=wl.K, S=n, H=wl.H, B=0)
     buf = np.zeros((n * wl.K, wl.H), np.uint16)
+    wsub = np.ascontiguousarray(w_np[tokens])
     t2 = time.perf_counter()
-    oracle.dispatch(scfg, sub, hidden_sample_bits, buf)
-    oracle.combine(scfg, sub, y_rows_bits, np.ascontiguousarray(w_np[tokens]))
+    oracle.dispatch(scfg, sub, hidden_sample_bits, buf, lib=lib)
+    oracle.combine(scfg, sub, y_rows_bits, wsub, lib=lib)
     t3 = time.perf_counter()
     frac = n / wl.tokens
     data_bytes = (bytes_dispatch(wl) + bytes_combine(wl)) * frac
     return t1 - t0, t3 - t2, data_bytes
+
+
+def oracle_reduce_sample(wl, topk_np, P, lib=None):
+    """Time the oracle's replica-gradient reduce over the real plan on rows
+    of P elements (a bounded sample of the gate+up+down rows).  Returns
+    (seconds, algorithmic bytes)."""
+    import oracle
+    ocfg = oracle.Config(R=wl.R, E=wl.E, K=wl.K, S=wl.S, H=wl.H, B=wl.B)
+    op = oracle.plan(ocfg, topk_np)
+    inf = oracle.info_dict(op)
+    rng = np.random.default_rng(4)
+    rb = rng.standard_normal((wl.R, wl.B, P), dtype=np.float32)
+    hg = rng.standard_normal((wl.E, P), dtype=np.float32)
+    t0 = time.perf_counter()
+    oracle.reduce_replica_grads(ocfg, op, rb, hg, P, lib=lib)
+    dt = time.perf_counter() - t0
+    return dt, bytes_reduce(inf["n_rep"] - inf["n_overflow"], inf["n_rep_experts"], P)
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
 
 
 def sample_tokens(wl, n):
@@ -300,7 +326,7 @@ def run_reference(args, world, rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic", "config": workload_config(wl, r, args),
         "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, "host_cores": host_cores()},
         "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "planner_us": round(statistics.median(plan_s) * 1e6, 1),
     }
@@ -336,6 +362,77 @@ class Timer:
 
     def count(self, name):
         return len(self.pairs.get(name, []))
+
+
+def workload_name(wl) -> str:
+    return f"{wl.name}: R={wl.R} E={wl.E} K={wl.K} S={wl.S} H={wl.H} B={wl.B}"
+
+
+def time_layer(mp, wl, rt, hidden, buf, out, dev, iters, peak, graph=False):
+    """One MoE layer's plan -> dispatch -> combine on routing ``rt``: CUDA-event
+    times of each call (mean over ``iters`` eager layers, after 3 warm-up
+    layers) and, with ``graph``, the whole layer replayed from a CUDA graph
+    (mean over 50 replays).  Returns the point's line."""
+    cfg = mp.Config(R=wl.R, E=wl.E, K=wl.K, S=wl.S, H=wl.H, B=wl.B)
+    p = mp.Plan(cfg, dev)
+    # the plan block and its zero-filled workspace were made on the default
+    # stream: finish that before a capture stream uses them
+    torch.cuda.synchronize()
+    for _ in range(3):
+        mp.plan(cfg, rt.topk_idx, out=p)
+        mp.dispatch(cfg, p, hidden, buf)
+        mp.combine(cfg, p, buf, rt.weights, out)
+    torch.cuda.synchronize()
+    st = Timer()
+    for _ in range(iters):
+        e = st.mark("plan"); mp.plan(cfg, rt.topk_idx, out=p); e.record()
+        e = st.mark("dispatch"); mp.dispatch(cfg, p, hidden, buf); e.record()
+        e = st.mark("combine"); mp.combine(cfg, p, buf, rt.weights, out); e.record()
+    torch.cuda.synchronize()
+    pd, pc, pp = (st.total_ms(n) / iters for n in ("dispatch", "combine", "plan"))
+    inf = p.info()
+    gd = bytes_dispatch(wl) / (pd * 1e-3) / 1e9
+    gc = bytes_combine(wl) / (pc * 1e-3) / 1e9
+    pt = {"maxvio": round(rt.maxvio, 3), "planner_us": round(pp * 1e3, 2),
+          "dispatch_us": round(pd * 1e3, 2), "combine_us": round(pc * 1e3, 2),
+          "dispatch_GB/s": round(gd, 1), "combine_GB/s": round(gc, 1),
+          "dispatch_frac": round(gd / peak, 4), "combine_frac": round(gc / peak, 4),
+          "dispatch+combine_tok/s": round(wl.tokens / ((pd + pc) * 1e-3)),
+          "n_rep": inf["n_rep"], "n_overflow": inf["n_overflow"],
+          "max_rep_per_rank": inf["max_rep_per_rank"],
+          # plan quality: any exact plan needs at least max(pieces, receivers)
+          # replicas; the greedy makes at most pieces + receivers - 1
+          "n_rep_bounds": [max(inf["n_pieces"], inf["n_receivers"]),
+                           max(inf["n_pieces"] + inf["n_receivers"] - 1, 0)],
+          "remote_pair_frac": round(inf["n_remote_pairs"] / wl.pairs, 4),
+          "hottest_expert_pairs": W.hottest_expert_count(rt.maxvio, wl.S, wl.K, wl.R, wl.E)}
+    if graph:
+        gs_ = torch.cuda.Stream()
+        try:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=gs_, capture_error_mode="thread_local"):
+                mp.plan(cfg, rt.topk_idx, out=p)
+                mp.dispatch(cfg, p, hidden, buf)
+                mp.combine(cfg, p, buf, rt.weights, out)
+            for _ in range(5):
+                g.replay()
+            torch.cuda.synchronize()
+            g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            g0.record()
+            for _ in range(50):
+                g.replay()
+            g1.record()
+            torch.cuda.synchronize()
+            us = g0.elapsed_time(g1) / 50 * 1e3
+            pt["graph_layer_us"] = round(us, 2)
+            pt["dispatch+combine_GB/s_in_graph"] = round(
+                (bytes_dispatch(wl) + bytes_combine(wl)) / (us * 1e-6) / 1e9, 1)
+            del g
+        except RuntimeError as exc:  # report the eager numbers if capture is refused
+            pt["graph_error"] = str(exc)[:200]
+            torch.cuda.synchronize()
+    del p
+    return pt
 
 
 def run_ours(args, world, rank, local):
@@ -441,42 +538,15 @@ def run_ours(args, world, rank, local):
                                 "reduced-size profile case (profiles/ncu_traffic.json), scaled to this "
                                 "launch by algorithmic bytes")}
 
-    # maxvio sweep: dispatch / combine GB/s and planner us per point
+    # maxvio sweep of the large shape (the Zipf sweep, then the adversarial
+    # placement with all hot experts on rank 0)
     sweep = []
     if not args.no_sweep:
-        # the Zipf sweep, then the adversarial placement (all hot experts on rank 0)
         for mv, adv in [(m, False) for m in wl.sweep] + [(max(wl.sweep), True)]:
             rs = W.routing(wl, mv, seed=rank, device=dev, adversarial=adv)
-            ps = mp.Plan(cfg, dev)
-            for _ in range(3):
-                mp.plan(cfg, rs.topk_idx, out=ps)
-                mp.dispatch(cfg, ps, hidden, buf)
-                mp.combine(cfg, ps, buf, rs.weights, out)
-            torch.cuda.synchronize()
-            st = Timer()
-            for _ in range(args.sweep_iters):
-                e = st.mark("plan"); mp.plan(cfg, rs.topk_idx, out=ps); e.record()
-                e = st.mark("dispatch"); mp.dispatch(cfg, ps, hidden, buf); e.record()
-                e = st.mark("combine"); mp.combine(cfg, ps, buf, rs.weights, out); e.record()
-            torch.cuda.synchronize()
-            it = args.sweep_iters
-            pd, pc, pp = st.total_ms("dispatch") / it, st.total_ms("combine") / it, st.total_ms("plan") / it
-            inf = ps.info()
-            gd = bytes_dispatch(wl) / (pd * 1e-3) / 1e9
-            gc = bytes_combine(wl) / (pc * 1e-3) / 1e9
-            sweep.append({"maxvio": round(rs.maxvio, 3), "adversarial": adv, "dispatch_GB/s": round(gd, 1),
-                          "combine_GB/s": round(gc, 1), "dispatch_frac": round(gd / peak, 4),
-                          "combine_frac": round(gc / peak, 4), "planner_us": round(pp * 1e3, 2),
-                          "dispatch_tok/s": round(wl.tokens / (pd * 1e-3)),
-                          "n_rep": inf["n_rep"], "n_overflow": inf["n_overflow"],
-                          "max_rep_per_rank": inf["max_rep_per_rank"],
-                          # plan quality: any exact plan needs at least
-                          # max(pieces, receivers) replicas; the greedy makes
-                          # at most pieces + receivers - 1
-                          "n_rep_bounds": [max(inf["n_pieces"], inf["n_receivers"]),
-                                           max(inf["n_pieces"] + inf["n_receivers"] - 1, 0)],
-                          "remote_pair_frac": round(inf["n_remote_pairs"] / wl.pairs, 4)})
-            del ps
+            pt = time_layer(mp, wl, rs, hidden, buf, out, dev, args.sweep_iters, peak)
+            pt["adversarial"] = adv
+            sweep.append(pt)
 
     # end to end through the public API with pinned host buffers: every step
     # copies its routing, weights and hidden states in and its output out.
@@ -546,41 +616,25 @@ def run_ours(args, world, rank, local):
                         "out, every step; double-buffered, copies of neighbouring steps overlap")}
         del d_topk, d_w, d_hidden, d_out
 
-    # the pages' own sweep shape: EP=8, maxvio 0.2, 1, 10, 20
-    pages_sweep = []
+    # the other workloads, each across its maxvio sweep: the mid shape, the
+    # pages' own sweep shape (EP=8, maxvio 0.2, 1, 10, 20), the tiny shape
+    # (latency, L2-resident) and the decode shape (latency, each layer also
+    # replayed from a CUDA graph)
+    workloads = {}
     if not args.no_sweep:
-        ewl = W.WORKLOADS["ep8"]
-        ecfg = mp.Config(R=ewl.R, E=ewl.E, K=ewl.K, S=ewl.S, H=ewl.H, B=ewl.B)
-        eh = W.hidden_states(ewl, seed=12 + rank, device=dev)
-        ebuf = torch.empty((ewl.R, ewl.C, ewl.H), dtype=torch.bfloat16, device=dev)
-        eout = torch.empty((ewl.tokens, ewl.H), dtype=torch.bfloat16, device=dev)
-        for mv in ewl.sweep:
-            er = W.routing(ewl, mv, seed=rank, device=dev)
-            ep = mp.Plan(ecfg, dev)
-            for _ in range(3):
-                mp.plan(ecfg, er.topk_idx, out=ep)
-                mp.dispatch(ecfg, ep, eh, ebuf)
-                mp.combine(ecfg, ep, ebuf, er.weights, eout)
-            torch.cuda.synchronize()
-            st = Timer()
-            for _ in range(args.sweep_iters):
-                e = st.mark("plan"); mp.plan(ecfg, er.topk_idx, out=ep); e.record()
-                e = st.mark("dispatch"); mp.dispatch(ecfg, ep, eh, ebuf); e.record()
-                e = st.mark("combine"); mp.combine(ecfg, ep, ebuf, er.weights, eout); e.record()
-            torch.cuda.synchronize()
-            it = args.sweep_iters
-            pd, pc, pp = st.total_ms("dispatch") / it, st.total_ms("combine") / it, st.total_ms("plan") / it
-            inf = ep.info()
-            gd = bytes_dispatch(ewl) / (pd * 1e-3) / 1e9
-            gc = bytes_combine(ewl) / (pc * 1e-3) / 1e9
-            pages_sweep.append({"maxvio": round(er.maxvio, 3), "dispatch_GB/s": round(gd, 1),
-                                "combine_GB/s": round(gc, 1), "dispatch_frac": round(gd / peak, 4),
-                                "combine_frac": round(gc / peak, 4), "planner_us": round(pp * 1e3, 2),
-                                "n_rep": inf["n_rep"], "n_overflow": inf["n_overflow"],
-                                "max_rep_per_rank": inf["max_rep_per_rank"],
-                                "hottest_expert_pairs": W.hottest_expert_count(er.maxvio, ewl.S, ewl.K, ewl.R, ewl.E)})
-            del ep
-        del eh, ebuf, eout
+        for wname, graph in (("mid", False), ("ep8", False), ("tiny", True)):
+            owl = W.WORKLOADS[wname]
+            oh = W.hidden_states(owl, seed=12 + rank, device=dev)
+            obuf = torch.empty((owl.R, owl.C, owl.H), dtype=torch.bfloat16, device=dev)
+            oout = torch.empty((owl.tokens, owl.H), dtype=torch.bfloat16, device=dev)
+            pts = []
+            for mv in owl.sweep:
+                orr = W.routing(owl, mv, seed=rank, device=dev)
+                pts.append(time_layer(mp, owl, orr, oh, obuf, oout, dev, args.sweep_iters, peak, graph=graph))
+            workloads[wname] = {"workload": workload_name(owl), "points": pts,
+                                "l2": ("inputs within L2: latency" if owl.tokens * owl.H * 2 * (owl.K + 1) < L2_BYTES
+                                       else "buffers larger than L2")}
+            del oh, obuf, oout
 
     # over-budget routing (one empty rank, the rest evenly overloaded): the
     # planner without and with the relay cascade, and the data kernels over
@@ -618,63 +672,21 @@ def run_ours(args, world, rank, local):
         del cr
 
     # decode shape (latency-bound): plan + dispatch + combine of one MoE layer
-    # replayed from a CUDA graph, next to the eager per-kernel times
+    # replayed from a CUDA graph, next to the eager per-kernel times, at each
+    # point of its sweep
     decode = None
     if not args.no_decode:
         dwl = W.WORKLOADS["decode"]
-        dcfg = mp.Config(R=dwl.R, E=dwl.E, K=dwl.K, S=dwl.S, H=dwl.H, B=dwl.B)
-        dr = W.routing(dwl, dwl.maxvio, seed=rank, device=dev)
         dh = W.hidden_states(dwl, seed=11 + rank, device=dev)
         dbuf = torch.empty((dwl.R, dwl.C, dwl.H), dtype=torch.bfloat16, device=dev)
         dout = torch.empty((dwl.tokens, dwl.H), dtype=torch.bfloat16, device=dev)
-        dplan = mp.Plan(dcfg, dev)
-        # the plan block and its zero-filled workspace were made on the
-        # default stream: finish that before another stream uses them
-        torch.cuda.synchronize()
-        gs_ = torch.cuda.Stream()
-        for _ in range(3):
-            mp.plan(dcfg, dr.topk_idx, out=dplan)
-            mp.dispatch(dcfg, dplan, dh, dbuf)
-            mp.combine(dcfg, dplan, dbuf, dr.weights, dout)
-        torch.cuda.synchronize()
-        et = Timer()
-        for _ in range(20):
-            e = et.mark("plan"); mp.plan(dcfg, dr.topk_idx, out=dplan); e.record()
-            e = et.mark("dispatch"); mp.dispatch(dcfg, dplan, dh, dbuf); e.record()
-            e = et.mark("combine"); mp.combine(dcfg, dplan, dbuf, dr.weights, dout); e.record()
-        torch.cuda.synchronize()
-        layer_us, graph_err = None, None
-        try:
-            graph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(graph, stream=gs_, capture_error_mode="thread_local"):
-                mp.plan(dcfg, dr.topk_idx, out=dplan)
-                mp.dispatch(dcfg, dplan, dh, dbuf)
-                mp.combine(dcfg, dplan, dbuf, dr.weights, dout)
-            for _ in range(5):
-                graph.replay()
-            torch.cuda.synchronize()
-            g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            g0.record()
-            for _ in range(50):
-                graph.replay()
-            g1.record()
-            torch.cuda.synchronize()
-            layer_us = g0.elapsed_time(g1) / 50 * 1e3
-            del graph
-        except RuntimeError as exc:  # report eager numbers if capture is refused
-            graph_err = str(exc)[:200]
-            torch.cuda.synchronize()
-        if layer_us is None:
-            layer_us = sum(et.total_ms(n) for n in ("plan", "dispatch", "combine")) / 20 * 1e3
-        dinfo = dplan.info()
-        db = bytes_dispatch(dwl) + bytes_combine(dwl)
-        decode = {"workload": f"decode: R={dwl.R} E={dwl.E} K={dwl.K} S={dwl.S} H={dwl.H} B={dwl.B}, one hot expert",
-                  "maxvio": round(dr.maxvio, 3), "graph_layer_us": round(layer_us, 2),
-                  "eager_us": {n: round(et.total_ms(n) / 20 * 1e3, 2) for n in ("plan", "dispatch", "combine")},
-                  "dispatch+combine_GB/s_in_graph": round(db / (layer_us * 1e-6) / 1e9, 1),
-                  "n_rep": dinfo["n_rep"], "n_overflow": dinfo["n_overflow"],
-                  "max_rep_per_rank": dinfo["max_rep_per_rank"], "graph_error": graph_err}
-        del dbuf, dout, dh, dplan
+        pts = []
+        for mv in dwl.sweep:
+            dr = W.routing(dwl, mv, seed=rank, device=dev)
+            pts.append(time_layer(mp, dwl, dr, dh, dbuf, dout, dev, 20, peak, graph=True))
+        decode = {"workload": workload_name(dwl) + ", one hot expert", "points": pts,
+                  "l2": "buffers larger than L2 (940 MB)"}
+        del dbuf, dout, dh
 
     # replica weight prefetch (a next-row step, timed on its own after the
     # step: its 68 GB of weights and pool fit once the reduce buffers are freed)
@@ -704,14 +716,18 @@ def run_ours(args, world, rank, local):
         del weights, pool, wrow
         torch.cuda.empty_cache()
 
-    # the CPU oracle on a bounded sample (rank 0, one GPU only)
+    # the CPU oracle on a bounded sample (rank 0, one GPU only): the
+    # single-threaded oracle, then the same loops built with OpenMP on all of
+    # the host's cores
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
         topk_np = r.topk_idx.cpu().numpy()
         w_np = r.weights.cpu().numpy()
         tokens = sample_tokens(wl, args.ref_tokens)
         hid = W.bits(hidden[: len(tokens)])
         y = W.bits(W.bf16_normal((len(tokens) * wl.K, wl.H), seed=2, device="cpu"))
+        ncores = host_cores()
         # repeat the bounded sample until about 10 s of CPU work
         reps, ds_tot, db_tot, ps_ = 0, 0.0, 0.0, 0.0
         while ds_tot < 10.0 and reps < 50:
@@ -719,10 +735,32 @@ def run_ours(args, world, rank, local):
             ds_tot += ds_
             db_tot += db_
             reps += 1
+        rs_, rb_ = oracle_reduce_sample(wl, topk_np, 1 << 18)
+        olib, nthr = oracle.openmp_lib(ncores)
+        oreps, ods, odb = 0, 0.0, 0.0
+        while ods < 5.0 and oreps < 200:
+            _, d_, b_ = oracle_sample(wl, topk_np, w_np, hid, tokens, y, lib=olib, plan=False)
+            ods += d_
+            odb += b_
+            oreps += 1
+        ors_, orb_ = oracle_reduce_sample(wl, topk_np, 1 << 18, lib=olib)
+        tok = len(tokens)
+        gpu_tok = wl.tokens / ((t["dispatch"] + t["combine"]) * 1e-3)
         cpu = {"value": round(db_tot / ds_tot / 1e9, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": (f"{reps} x dispatch+combine of the first {len(tokens)} of {wl.tokens} tokens "
+               "sample": (f"{reps} x dispatch+combine of the first {tok} of {wl.tokens} tokens "
                           f"({ds_tot:.1f} s); plan over all {wl.pairs} pairs took {ps_ * 1e3:.0f} ms; "
-                          "single-threaded C")}
+                          "single-threaded C"),
+               "host_cores": ncores,
+               "dispatch+combine_tok/s": round(reps * tok / ds_tot),
+               "planner_us": round(ps_ * 1e6, 1),
+               "reduce_GB/s": round(rb_ / rs_ / 1e9, 4),
+               "openmp": {"value": round(odb / ods / 1e9, 4), "unit": UNIT, "threads": nthr,
+                          "dispatch+combine_tok/s": round(oreps * tok / ods),
+                          "reduce_GB/s": round(orb_ / ors_ / 1e9, 4),
+                          "sample": (f"{oreps} x the same token sample ({ods:.1f} s), the oracle's loops "
+                                     f"built with OpenMP over tokens on {nthr} threads; reduce over "
+                                     f"elements, rows of 2^18 of the {wl.grad_elems} gradient elements")},
+               "gpu_dispatch+combine_tok/s": round(gpu_tok)}
 
     launches_per_step = 2 + 1 + 1 + 1 + (1 if P else 0)
     cfgd = workload_config(wl, r, args)
@@ -735,9 +773,7 @@ def run_ours(args, world, rank, local):
         "planner_us": kernels["plan"]["us"],
         "roofline": roofline, "kernels": kernels, "sweep": sweep,
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
-        "decode": decode,
-        "pages_sweep": {"workload": "ep8: R=8 E=256 K=8 S=4096 H=7168 B=4 (EP=8 as in the pages' sweep)",
-                        "points": pages_sweep},
+        "decode": decode, "workloads": workloads,
         "cascade": cascade, "clocks": clocks, "plan_info": info,
         "reduce": (f"P={P} fp32 ({reduce_note}), {n_pref} prefetched replicas over "
                    f"{info['n_rep_experts']} experts"),

@@ -2,7 +2,10 @@
 
 A plain, slow, single-threaded C implementation (``moonep_oracle.c``) of the
 plan, dispatch, combine, combine-backward and replica-gradient reduction,
-wrapped here with ctypes and numpy.  Only the test suite, the smoke check
+wrapped here with ctypes and numpy.  (The same source is also built with
+OpenMP, whose pragmas spread the data steps' token loops over the host's
+cores; that build only times a multi-core CPU baseline and never checks
+anything.)  Only the test suite, the smoke check
 and the benchmark's CPU-baseline / reference legs may import this package;
 the product (``load_balancing_moonep_b200``) never does, and this package
 never imports the product.
@@ -24,6 +27,9 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "moonep_oracle.c")
 _LIB = os.path.join(_HERE, "libmoonep_oracle.so")
+# the same source built with OpenMP: its data-step loops run on all host
+# cores; used only to time a multi-core CPU baseline, never as the checker
+_LIB_OMP = os.path.join(_HERE, "libmoonep_oracle_omp.so")
 
 FLAG_STRICT_BUDGET = 1
 FLAG_TRAIN_B_RULE = 2
@@ -51,22 +57,42 @@ class OracleError(RuntimeError):
 
 
 def build(force: bool = False) -> str:
-    """Compile the oracle with gcc (plain C11, -O2, no fast-math)."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        cmd = ["gcc", "-std=c11", "-O2", "-fno-fast-math", "-ffp-contract=off",
-               "-fPIC", "-shared", "-o", _LIB, _SRC, "-lm"]
-        subprocess.check_call(cmd)
+    """Compile the oracle with gcc (plain C11, -O2, no fast-math), and the
+    same source with OpenMP for the timed multi-core CPU baseline."""
+    for lib, extra in ((_LIB, []), (_LIB_OMP, ["-fopenmp"])):
+        if force or not os.path.exists(lib) or os.path.getmtime(lib) < os.path.getmtime(_SRC):
+            cmd = ["gcc", "-std=c11", "-O2", "-fno-fast-math", "-ffp-contract=off", *extra,
+                   "-fPIC", "-shared", "-o", lib, _SRC, "-lm"]
+            subprocess.check_call(cmd)
     return _LIB
 
 
 _lib = None
+_lib_omp = None
 
 
 def _load():
     global _lib
     if _lib is None:
         build()
-        lib = ctypes.CDLL(_LIB)
+        _lib = _bind(ctypes.CDLL(_LIB))
+    return _lib
+
+
+def openmp_lib(threads: int = 0):
+    """The OpenMP build (data-step loops over all host cores), for timing a
+    multi-core CPU baseline only; pass it as ``lib=`` to dispatch, combine
+    and reduce_replica_grads.  threads > 0 sets the thread count.  Returns
+    (lib, threads in use)."""
+    global _lib_omp
+    if _lib_omp is None:
+        build()
+        _lib_omp = _bind(ctypes.CDLL(_LIB_OMP))
+    return _lib_omp, int(_lib_omp.or_omp_threads(int(threads)))
+
+
+def _bind(lib):
+    if True:
         lib.or_plan.argtypes = [ctypes.c_void_p] + [ctypes.c_void_p] * 18
         lib.or_plan.restype = ctypes.c_int
         lib.or_check_config.argtypes = [ctypes.c_void_p]
@@ -83,8 +109,9 @@ def _load():
         lib.or_prefetch_replicas.restype = ctypes.c_int
         lib.or_f32_to_bf16.argtypes = [ctypes.c_float]
         lib.or_f32_to_bf16.restype = ctypes.c_uint16
-        _lib = lib
-    return _lib
+        lib.or_omp_threads.argtypes = [ctypes.c_int]
+        lib.or_omp_threads.restype = ctypes.c_int
+    return lib
 
 
 class _Cfg(ctypes.Structure):
@@ -185,11 +212,11 @@ def info_dict(p: dict) -> dict:
 
 
 def dispatch(cfg: Config, p: dict, hidden_bits: np.ndarray, buf_bits: np.ndarray,
-             t0: int = 0, t1: int | None = None) -> np.ndarray:
+             t0: int = 0, t1: int | None = None, lib=None) -> np.ndarray:
     """Zero-copy permute: hidden row t lands in buffer row dst_pos[t, k] for
     every k (MoonEP article, 'The core idea', zero copy and static shapes).
     hidden_bits: uint16 [R*S, H]; buf_bits: uint16 [R, S*K, H] (written in place)."""
-    lib = _load()
+    lib = lib or _load()
     t1 = cfg.R * cfg.S if t1 is None else t1
     assert hidden_bits.dtype == np.uint16 and hidden_bits.flags.c_contiguous
     assert buf_bits.dtype == np.uint16 and buf_bits.flags.c_contiguous
@@ -200,10 +227,11 @@ def dispatch(cfg: Config, p: dict, hidden_bits: np.ndarray, buf_bits: np.ndarray
 
 
 def combine(cfg: Config, p: dict, y_bits: np.ndarray, w: np.ndarray,
-            out_bits: np.ndarray | None = None, t0: int = 0, t1: int | None = None) -> np.ndarray:
+            out_bits: np.ndarray | None = None, t0: int = 0, t1: int | None = None,
+            lib=None) -> np.ndarray:
     """Weighted unpermute with fp32 fused multiply-add accumulation in k order
     and one bf16 rounding.  y_bits: uint16 [R, S*K, H]; w: float32 [R*S, K]."""
-    lib = _load()
+    lib = lib or _load()
     t1 = cfg.R * cfg.S if t1 is None else t1
     if out_bits is None:
         out_bits = np.zeros((cfg.R * cfg.S, cfg.H), np.uint16)
@@ -230,11 +258,11 @@ def combine_backward(cfg: Config, p: dict, dy_bits: np.ndarray, w: np.ndarray,
 
 
 def reduce_replica_grads(cfg: Config, p: dict, reduce_buf: np.ndarray, home_grad: np.ndarray,
-                         P: int, i0: int = 0, i1: int | None = None):
+                         P: int, i0: int = 0, i1: int | None = None, lib=None):
     """Sum prefetched replicas' fp32 grads into their home expert, ascending
     host rank order, then zero the replica rows (MoonEP article explainer,
     memory tab, training branch).  reduce_buf: f32 [R, B, P]; home_grad: f32 [E, P]."""
-    lib = _load()
+    lib = lib or _load()
     i1 = P if i1 is None else i1
     assert reduce_buf.dtype == np.float32 and reduce_buf.flags.c_contiguous
     assert home_grad.dtype == np.float32 and home_grad.flags.c_contiguous

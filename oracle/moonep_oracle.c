@@ -595,6 +595,28 @@ out:
 
 /* --------------------------------------------------------- data steps --- */
 
+/* The data steps' token (or element) loops carry OpenMP pragmas.  The
+ * oracle proper is compiled without OpenMP, so they are single-threaded
+ * loops; a second build with OpenMP, used only to time a multi-core CPU
+ * baseline, runs the same loops over the host's cores.  Each iteration
+ * writes its own outputs, so both builds compute identical results.
+ * or_omp_threads(n) sets the thread count (n > 0) and returns the count in
+ * use: always 1 without OpenMP. */
+#ifdef _OPENMP
+#include <omp.h>
+int or_omp_threads(int n)
+{
+    if (n > 0) omp_set_num_threads(n);
+    return omp_get_max_threads();
+}
+#else
+int or_omp_threads(int n)
+{
+    (void)n;
+    return 1;
+}
+#endif
+
 /* Dispatch (zero-copy permute) [P1 core idea; P2 README]: the row of token t
  * is written, unchanged, into the buffer row dst_pos[t*K+k] for every k.
  * Tokens [t0, t1) only; buf is the [R, S*K, H] buffer as R*S*K rows. */
@@ -603,6 +625,7 @@ int or_dispatch(const or_config *c, const int32_t *dst_pos, const int32_t *info,
 {
     if (info[OR_INFO_STATUS] & OR_ST_EXPERT_ID_RANGE) return OR_OK;
     const int64_t K = c->K, H = c->H;
+#pragma omp parallel for schedule(static)
     for (int64_t t = t0; t < t1; ++t)
         for (int64_t k = 0; k < K; ++k) {
             int64_t d = dst_pos[t * K + k];
@@ -619,6 +642,7 @@ int or_combine(const or_config *c, const int32_t *dst_pos, const int32_t *info,
 {
     if (info[OR_INFO_STATUS] & OR_ST_EXPERT_ID_RANGE) return OR_OK;
     const int64_t K = c->K, H = c->H;
+#pragma omp parallel for schedule(static)
     for (int64_t t = t0; t < t1; ++t)
         for (int64_t h = 0; h < H; ++h) {
             float acc = 0.0f;
@@ -677,6 +701,7 @@ int or_reduce_replica_grads(const or_config *c, const int32_t *host_ptr,
             if (b < 0 || b >= B) continue; /* overflow replica: no reduce rows */
             float *src = reduce_buf + ((int64_t)r * B + b) * P;
             float *dst = home_grad + (int64_t)e * P;
+#pragma omp parallel for schedule(static)
             for (int64_t i = i0; i < i1; ++i) dst[i] = dst[i] + src[i];
         }
     }
@@ -685,6 +710,7 @@ int or_reduce_replica_grads(const or_config *c, const int32_t *host_ptr,
             int32_t r = host_rank[h], b = host_slot[h] - L;
             if (r == e / L || b < 0 || b >= B) continue;
             float *src = reduce_buf + ((int64_t)r * B + b) * P;
+#pragma omp parallel for schedule(static)
             for (int64_t i = i0; i < i1; ++i) src[i] = 0.0f;
         }
     return OR_OK;

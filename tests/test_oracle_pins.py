@@ -673,3 +673,32 @@ def test_prefetch_budget_above_L(oracle_lib):
     assert np.array_equal(pool[0, 0], w[6]) and np.array_equal(pool[1, 0], w[6])
     assert np.array_equal(pool[1, 1], w[4]) and np.array_equal(pool[1, 2], w[7])
     assert (pool[0, 1:] == 0xFFFF).all() and (pool[2:] == 0xFFFF).all()
+
+
+def test_openmp_build_computes_what_the_oracle_computes(oracle_lib):
+    """The OpenMP build of the oracle (used only to time a multi-core CPU
+    baseline) runs the same data-step loops on several threads: its dispatch,
+    combine and reduce must equal the single-threaded oracle's bit for bit."""
+    wl = W.WORKLOADS["mid"]
+    r = W.routing(wl, 2.0)
+    cfg = oracle.Config(R=wl.R, E=wl.E, K=wl.K, S=wl.S, H=wl.H, B=wl.B)
+    topk = r.topk_idx.numpy()
+    p = oracle.plan(cfg, topk)
+    olib, nthr = oracle.openmp_lib(4)
+    assert nthr == 4
+    hid = W.bits(W.bf16_normal((wl.tokens, wl.H), seed=1))
+    b1 = np.zeros((wl.R, wl.C, wl.H), np.uint16)
+    b2 = np.zeros_like(b1)
+    oracle.dispatch(cfg, p, hid, b1)
+    oracle.dispatch(cfg, p, hid, b2, lib=olib)
+    assert np.array_equal(b1, b2)
+    w = r.weights.numpy()
+    assert np.array_equal(oracle.combine(cfg, p, b1, w), oracle.combine(cfg, p, b1, w, lib=olib))
+    P = 4096
+    rng = np.random.default_rng(0)
+    rb1 = rng.standard_normal((wl.R, wl.B, P), dtype=np.float32)
+    hg1 = rng.standard_normal((wl.E, P), dtype=np.float32)
+    rb2, hg2 = rb1.copy(), hg1.copy()
+    oracle.reduce_replica_grads(cfg, p, rb1, hg1, P)
+    oracle.reduce_replica_grads(cfg, p, rb2, hg2, P, lib=olib)
+    assert np.array_equal(hg1, hg2) and np.array_equal(rb1, rb2)

@@ -71,6 +71,13 @@ def bytes_reduce(n_rep_prefetched: int, n_rep_experts: int, P: int) -> int:
     return (n_rep_prefetched + n_rep_experts) * P * 4 * 2
 
 
+def bytes_prefetch(n_rep_prefetched: int, n_rep_experts: int, P: int, wl) -> int:
+    """each expert with prefetched replicas read once, each replica's pool
+    row written once (bf16), the slot table read and the weight-row table
+    written"""
+    return (n_rep_experts + n_rep_prefetched) * P * 2 + wl.R * wl.E * 8
+
+
 def bytes_plan(wl) -> int:
     """two passes over the ids, dst_pos and row_src written"""
     return wl.pairs * 4 * 2 + wl.pairs * 4 * 2
@@ -707,14 +714,75 @@ def run_ours(args, world, rank, local):
             ev.record()
         torch.cuda.synchronize()
         pms = pt.total_ms("prefetch") / 5
-        pbytes = n_pref * Pw * 2 * 2 + wl.R * wl.E * 8
+        pbytes = bytes_prefetch(n_pref, info["n_rep_experts"], Pw, wl)
         ptraffic = int(round(ratio["prefetch"] * pbytes)) if "prefetch" in ratio else None
         kernels["prefetch"] = {"ms": round(pms, 4), "bytes": pbytes, "GB/s": round(pbytes / (pms * 1e-3) / 1e9, 1),
                                "frac": round(pbytes / (pms * 1e-3) / 1e9 / peak, 4), "traffic": ptraffic,
                                "in_step": False,
-                               "what": f"{n_pref} replicas x {Pw} bf16 (gate+up+down) copied into the pool"}
+                               "what": (f"{n_pref} replicas of {info['n_rep_experts']} experts x {Pw} bf16 "
+                                        "(gate+up+down) copied into the pool, each source row read once")}
         del weights, pool, wrow
         torch.cuda.empty_cache()
+
+    # expert parallelism's calls on one GPU: every rank's count and plan from
+    # the stacked counts rows (what the all-gather leaves), then its dispatch
+    # and combine through an array of R per-rank row-buffer pointers (here
+    # the R slices of the one buffer), one launch per rank as one process
+    # per GPU would issue them
+    ep = None
+    if not args.no_ep:
+        eplans = [mp.Plan(cfg, dev, ep=True) for _ in range(wl.R)]
+        counts_all = torch.empty((wl.R, wl.E + 1), dtype=torch.int32, device=dev)
+        tl = [r.topk_idx[k * wl.S:(k + 1) * wl.S].contiguous() for k in range(wl.R)]
+        hl = [hidden[k * wl.S:(k + 1) * wl.S] for k in range(wl.R)]
+        wloc = [r.weights[k * wl.S:(k + 1) * wl.S].contiguous() for k in range(wl.R)]
+        ol = [out[k * wl.S:(k + 1) * wl.S] for k in range(wl.R)]
+        bptr = mp.pointer_array([buf[k] for k in range(wl.R)])
+        torch.cuda.synchronize()
+
+        def ep_layer(tm):
+            for k in range(wl.R):
+                e = tm.mark("count") if tm and k == 0 else None
+                mp.ep_count(cfg, tl[k], eplans[k], counts_row=counts_all[k])
+                if e:
+                    e.record()
+            for k in range(wl.R):
+                e = tm.mark("plan") if tm and k == 0 else None
+                mp.ep_plan(cfg, k, tl[k], counts_all, eplans[k])
+                if e:
+                    e.record()
+            e = tm.mark("dispatch") if tm else None
+            for k in range(wl.R):
+                mp.ep_dispatch(cfg, eplans[k], hl[k], bptr)
+            if e:
+                e.record()
+                e = tm.mark("combine")
+            for k in range(wl.R):
+                mp.ep_combine(cfg, eplans[k], bptr, wloc[k], ol[k])
+            if e:
+                e.record()
+
+        for _ in range(3):
+            ep_layer(None)
+        torch.cuda.synchronize()
+        et = Timer()
+        for _ in range(args.sweep_iters):
+            ep_layer(et)
+        torch.cuda.synchronize()
+        it = args.sweep_iters
+        pd, pc = et.total_ms("dispatch") / it, et.total_ms("combine") / it
+        einf = eplans[0].info()
+        gd = bytes_dispatch(wl) / (pd * 1e-3) / 1e9
+        gc = bytes_combine(wl) / (pc * 1e-3) / 1e9
+        ep = {"what": (f"{wl.R} ranks on one GPU: each rank's ep_count and ep_plan (rank 0 timed), then "
+                       f"{wl.R} ep_dispatch and {wl.R} ep_combine launches through per-rank row pointers"),
+              "count_us": round(et.total_ms("count") / it * 1e3, 2),
+              "plan_us": round(et.total_ms("plan") / it * 1e3, 2),
+              "dispatch_GB/s": round(gd, 1), "combine_GB/s": round(gc, 1),
+              "dispatch_frac": round(gd / peak, 4), "combine_frac": round(gc / peak, 4),
+              "rank0_remote_pair_frac": round(einf["n_remote_pairs"] / (wl.S * wl.K), 4),
+              "status": einf["status"]}
+        del eplans, bptr
 
     # the CPU oracle on a bounded sample (rank 0, one GPU only): the
     # single-threaded oracle, then the same loops built with OpenMP on all of
@@ -773,7 +841,7 @@ def run_ours(args, world, rank, local):
         "planner_us": kernels["plan"]["us"],
         "roofline": roofline, "kernels": kernels, "sweep": sweep,
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
-        "decode": decode, "workloads": workloads,
+        "decode": decode, "workloads": workloads, "ep_one_gpu": ep,
         "cascade": cascade, "clocks": clocks, "plan_info": info,
         "reduce": (f"P={P} fp32 ({reduce_note}), {n_pref} prefetched replicas over "
                    f"{info['n_rep_experts']} experts"),
@@ -789,7 +857,7 @@ def run_ours(args, world, rank, local):
 # the 126 MB L2 while every buffer of the case stays within a few GB.
 PROFILE_CASES = {
     "dispatch": ("large", 512, 0), "combine": ("large", 512, 0), "combine_bwd": ("large", 512, 0),
-    "reduce": ("tiny", 256, 1 << 24), "prefetch": ("tiny", 256, 1 << 25), "plan": ("large", 4096, 0),
+    "reduce": ("tiny", 256, 1 << 25), "prefetch": ("tiny", 256, 1 << 26), "plan": ("large", 4096, 0),
 }
 PROFILE_KERNELS = tuple(PROFILE_CASES)
 
@@ -850,7 +918,7 @@ def run_profile_case(args):
         pool = torch.empty((wl.R, wl.B, P), dtype=torch.bfloat16, device=dev)
         for _ in range(2):
             mp.prefetch_replicas(cfg, plan, weights, pool)
-        alg = n_pref * P * 2 * 2 + wl.R * wl.E * 8
+        alg = bytes_prefetch(n_pref, info["n_rep_experts"], P, wl)
     else:
         raise SystemExit(f"--profile: unknown kernel {kern}")
     torch.cuda.synchronize()
@@ -876,6 +944,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefetch", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-ep", action="store_true")
     ap.add_argument("--profile", default=None, choices=PROFILE_KERNELS,
                     help="run one kernel twice on a reduced-size case of a few GB (for ncu)")
     ap.add_argument("--profile-S", type=int, default=0, help="tokens per rank (0: the kernel's case)")

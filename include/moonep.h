@@ -262,6 +262,82 @@ MOONEP_API int moonep_prefetch_replicas(const moonep_config *cfg, const moonep_p
                                         const uint16_t *weights, uint16_t *pool, int32_t *slot_wrow,
                                         int64_t P, void *stream);
 
+/* ---- expert parallelism over several GPUs ---------------------------- */
+/* The pages' deployment (MoonEP article, "The core idea: dynamic redundant
+ * experts": tokens are written directly into their expert-grouped positions
+ * on remote ranks; explainer, pillars tab: NVLink and symmetric memory;
+ * memory tab: the home rank pulls its replicas' gradient rows back over
+ * NVLink).  One process per GPU; rank `rank` of R owns its S tokens
+ * (topk_local [S, K], hidden_local / out_local / dy_local [S, H], w_local and
+ * dw_local [S, K]), its receive buffer [S*K, H] (row j is global row
+ * rank*S*K + j of the single-GPU buffer), its reduce buffer [B, P] and the
+ * gradients of its L home experts [L, P].  Other ranks' buffers are reached
+ * through device arrays of R device pointers (index = rank; peer memory
+ * mapped into this process, e.g. symmetric memory or CUDA IPC, or R
+ * allocations of one GPU); each pointer must be 16-byte aligned, and a null
+ * or misaligned one is skipped and reported as MOONEP_ST_ROW_RANGE.  Loads
+ * and stores to peers are plain 16-byte vector accesses.
+ * Per MoE layer:
+ *   1. moonep_ep_count: this rank's counts row [E + 1] (pairs per expert,
+ *      then the number of ids outside [0, E));
+ *   2. the caller all-gathers the R rows into counts_all [R, E + 1] (row r
+ *      from rank r; 4 (E + 1) bytes per rank, e.g. an NCCL all-gather);
+ *   3. moonep_ep_plan: every rank plans from counts_all -- plan tables equal
+ *      to moonep_plan's for the concatenation of all ranks' routings, on
+ *      every rank -- and places its own pairs: plan->dst_pos[0 .. S*K) holds
+ *      the global buffer rows of its pairs (t*K + k, t local); plan->row_src
+ *      is not written, and info[MOONEP_INFO_N_REMOTE_PAIRS] counts this
+ *      rank's pairs placed on other ranks;
+ *   4. moonep_ep_dispatch / combine / combine_backward /
+ *      reduce_replica_grads move the data over the peer pointers.
+ * No call synchronises the host, and none issues a collective.
+ * Sizes: moonep_ep_sizes (the plan block is laid out by moonep_plan_layout;
+ * the workspace, one per rank, is zero-filled once and left ready for the
+ * next call with the same configuration). */
+MOONEP_API int moonep_ep_sizes(const moonep_config *cfg, size_t *plan_bytes, size_t *workspace_bytes);
+
+/* counts_row[e] = pairs of this rank's topk_local [S, K] routed to expert e;
+ * counts_row[E] = its ids outside [0, E).  One launch. */
+MOONEP_API int moonep_ep_count(const moonep_config *cfg, const int32_t *topk_local, int32_t *counts_row,
+                               void *workspace, void *stream);
+
+/* The plan from the gathered counts [R, E + 1] (an id outside [0, E) on any
+ * rank empties the plan, as in moonep_plan; counts that do not add up to
+ * R*S*K give MOONEP_ST_WORKSPACE), and the global rows of this rank's pairs:
+ * a pair's rank within its expert is the lower ranks' counts of that expert
+ * plus its rank among this rank's own pairs in (t, k) order, the global
+ * order of moonep_plan.  Uses the per-chunk counts moonep_ep_count left in
+ * `workspace`: call it with the same workspace and topk_local.  Two
+ * launches. */
+MOONEP_API int moonep_ep_plan(const moonep_config *cfg, int32_t rank, const int32_t *topk_local,
+                              const int32_t *counts_all, const moonep_plan_t *plan, void *workspace,
+                              void *stream);
+
+/* bufs[r] + (g - r*S*K)*H receives hidden_local[t] for every pair (t, k) of
+ * this rank with global row g = plan->dst_pos[t*K + k], r = g / (S*K). */
+MOONEP_API int moonep_ep_dispatch(const moonep_config *cfg, const moonep_plan_t *plan,
+                                  const uint16_t *hidden_local, uint16_t *const *bufs, void *stream);
+
+/* out_local[t] = bf16_rne(sum_k w_local[t,k] * y[g]) with the rows y[g] read
+ * from ys[r] as in moonep_ep_dispatch, fp32 fmaf in k order from 0. */
+MOONEP_API int moonep_ep_combine(const moonep_config *cfg, const moonep_plan_t *plan, const uint16_t *const *ys,
+                                 const float *w_local, uint16_t *out_local, void *stream);
+
+/* The backward of moonep_ep_combine: dy_bufs rows get bf16_rne(w * dy)
+ * (dy with MOONEP_FLAG_BWD_UNSCALED), dw_local[t,k] = sum_h dy * y; K <= 16. */
+MOONEP_API int moonep_ep_combine_backward(const moonep_config *cfg, const moonep_plan_t *plan,
+                                          const uint16_t *dy_local, const float *w_local,
+                                          const uint16_t *const *ys, uint16_t *const *dy_bufs, float *dw_local,
+                                          void *stream);
+
+/* On home rank `rank`: for each of its experts e with prefetched replicas,
+ * in ascending host rank order, home_grad_local[e - rank*L] += the replica's
+ * row reduce_bufs[r] + (slot - L)*P (separate fp32 adds), then that remote
+ * row is zeroed.  reduce_bufs: device array of R pointers to [B, P] fp32. */
+MOONEP_API int moonep_ep_reduce_replica_grads(const moonep_config *cfg, int32_t rank, const moonep_plan_t *plan,
+                                              float *const *reduce_bufs, float *home_grad_local, int64_t P,
+                                              void *stream);
+
 /* Size of the fixed device array behind moonep_plan_noalloc (4 MiB).  The
  * large training shape (R=32, E=384, K=8, S=4096) needs about 0.5 MiB. */
 #define MOONEP_NOALLOC_WORKSPACE_BYTES (4u << 20)

@@ -21,6 +21,18 @@ int launch_reduce(const Dims &d, const moonep_plan_t &p, float *reduce_buf, floa
                   cudaStream_t st);
 int launch_prefetch(const Dims &d, const moonep_plan_t &p, const uint16_t *weights, uint16_t *pool,
                     int32_t *slot_wrow, long long P, cudaStream_t st);
+int launch_ep_count(const Dims &d, const int32_t *topk, int32_t *counts_row, void *ws, cudaStream_t st);
+int launch_ep_plan(const Dims &d, int rank, const int32_t *topk, const int32_t *counts_all,
+                   const moonep_plan_t &p, void *ws, cudaStream_t st);
+size_t ep_smem_bytes_max(const Dims &d);
+int launch_dispatch_ep(const Dims &d, const int *dst_pos, int *info, const uint16_t *hidden,
+                       uint16_t *const *bufs, cudaStream_t st);
+int launch_combine_ep(const Dims &d, const int *dst_pos, int *info, const uint16_t *const *ys, const float *w,
+                      uint16_t *out, cudaStream_t st);
+int launch_combine_backward_ep(const Dims &d, const int *dst_pos, int *info, const uint16_t *dy, const float *w,
+                               const uint16_t *const *ys, uint16_t *const *dy_bufs, float *dw, cudaStream_t st);
+int launch_reduce_ep(const Dims &d, int rank, const moonep_plan_t &p, float *const *reduce_bufs,
+                     float *home_grad, long long P, cudaStream_t st);
 
 constexpr size_t MAX_DYN_SMEM = 227 * 1024;
 constexpr int MAX_COMBINE_BWD_K = 16;
@@ -89,6 +101,26 @@ static int make_dims(const moonep_config *c, Dims *d, int nsm = B200_SMS)
     d->ebits = 0;
     while ((1 << d->ebits) < d->E) ++d->ebits;
     if (plan_smem_bytes_max(*d) > MAX_DYN_SMEM) return MOONEP_ERR_LIMIT;
+    return MOONEP_OK;
+}
+
+// Expert parallelism: the chunking covers one rank's S tokens (about 128
+// chunks, at least 8 tokens and at most 4096 pairs each) and the planner sums
+// the R rows of the gathered counts.
+static int make_dims_ep(const moonep_config *c, Dims *d)
+{
+    const int rc = make_dims(c, d);
+    if (rc != MOONEP_OK) return rc;
+    int ct = (d->S + 127) / 128;
+    if (ct < 8) ct = 8;
+    int cap = 4096 / d->K;
+    if (cap < 1) cap = 1;
+    if (ct > cap) ct = cap;
+    if (ct > d->S) ct = d->S;
+    d->chunk_tokens = ct;
+    d->nchunk = (d->S + ct - 1) / ct;
+    d->ngroups = d->R;
+    if (ep_smem_bytes_max(*d) > MAX_DYN_SMEM) return MOONEP_ERR_LIMIT;
     return MOONEP_OK;
 }
 
@@ -310,6 +342,92 @@ int moonep_prefetch_replicas(const moonep_config *cfg, const moonep_plan_t *plan
         (reinterpret_cast<uintptr_t>(slot_wrow) & 3u))
         return MOONEP_ERR_ALIGN;
     return launch_prefetch(d, *plan, weights, pool, slot_wrow, (long long)P, static_cast<cudaStream_t>(stream));
+}
+
+// ---- expert parallelism over several GPUs
+
+int moonep_ep_sizes(const moonep_config *cfg, size_t *plan_bytes, size_t *workspace_bytes)
+{
+    Dims d;
+    const int rc = make_dims_ep(cfg, &d);
+    if (rc != MOONEP_OK) return rc;
+    if (plan_bytes) *plan_bytes = plan_layout(d).total;
+    if (workspace_bytes) *workspace_bytes = ws_layout_ep(d).total;
+    return MOONEP_OK;
+}
+
+int moonep_ep_count(const moonep_config *cfg, const int32_t *topk_local, int32_t *counts_row, void *workspace,
+                    void *stream)
+{
+    Dims d;
+    const int rc = make_dims_ep(cfg, &d);
+    if (rc != MOONEP_OK) return rc;
+    if (!topk_local || !counts_row || !workspace) return MOONEP_ERR_ARG;
+    return launch_ep_count(d, topk_local, counts_row, workspace, static_cast<cudaStream_t>(stream));
+}
+
+int moonep_ep_plan(const moonep_config *cfg, int32_t rank, const int32_t *topk_local, const int32_t *counts_all,
+                   const moonep_plan_t *plan, void *workspace, void *stream)
+{
+    Dims d;
+    const int rc = make_dims_ep(cfg, &d);
+    if (rc != MOONEP_OK) return rc;
+    if (rank < 0 || rank >= d.R || !topk_local || !counts_all || !plan_ok(plan) || !workspace)
+        return MOONEP_ERR_ARG;
+    return launch_ep_plan(d, rank, topk_local, counts_all, *plan, workspace, static_cast<cudaStream_t>(stream));
+}
+
+int moonep_ep_dispatch(const moonep_config *cfg, const moonep_plan_t *plan, const uint16_t *hidden_local,
+                       uint16_t *const *bufs, void *stream)
+{
+    Dims d;
+    const int rc = make_dims(cfg, &d);
+    if (rc != MOONEP_OK) return rc;
+    if (!plan_ok(plan) || !hidden_local || !bufs) return MOONEP_ERR_ARG;
+    if (!aligned16(hidden_local)) return MOONEP_ERR_ALIGN;
+    return launch_dispatch_ep(d, plan->dst_pos, plan->info, hidden_local, bufs, static_cast<cudaStream_t>(stream));
+}
+
+int moonep_ep_combine(const moonep_config *cfg, const moonep_plan_t *plan, const uint16_t *const *ys,
+                      const float *w_local, uint16_t *out_local, void *stream)
+{
+    Dims d;
+    const int rc = make_dims(cfg, &d);
+    if (rc != MOONEP_OK) return rc;
+    if (!plan_ok(plan) || !ys || !w_local || !out_local) return MOONEP_ERR_ARG;
+    if (!aligned16(out_local) || (reinterpret_cast<uintptr_t>(w_local) & 3u)) return MOONEP_ERR_ALIGN;
+    return launch_combine_ep(d, plan->dst_pos, plan->info, ys, w_local, out_local,
+                             static_cast<cudaStream_t>(stream));
+}
+
+int moonep_ep_combine_backward(const moonep_config *cfg, const moonep_plan_t *plan, const uint16_t *dy_local,
+                               const float *w_local, const uint16_t *const *ys, uint16_t *const *dy_bufs,
+                               float *dw_local, void *stream)
+{
+    Dims d;
+    const int rc = make_dims(cfg, &d);
+    if (rc != MOONEP_OK) return rc;
+    if (!plan_ok(plan) || !dy_local || !w_local || !ys || !dy_bufs || !dw_local) return MOONEP_ERR_ARG;
+    if (d.K > MAX_COMBINE_BWD_K) return MOONEP_ERR_LIMIT;
+    if (!aligned16(dy_local) || (reinterpret_cast<uintptr_t>(w_local) & 3u) ||
+        (reinterpret_cast<uintptr_t>(dw_local) & 3u))
+        return MOONEP_ERR_ALIGN;
+    return launch_combine_backward_ep(d, plan->dst_pos, plan->info, dy_local, w_local, ys, dy_bufs, dw_local,
+                                      static_cast<cudaStream_t>(stream));
+}
+
+int moonep_ep_reduce_replica_grads(const moonep_config *cfg, int32_t rank, const moonep_plan_t *plan,
+                                   float *const *reduce_bufs, float *home_grad_local, int64_t P, void *stream)
+{
+    Dims d;
+    const int rc = make_dims(cfg, &d);
+    if (rc != MOONEP_OK) return rc;
+    if (rank < 0 || rank >= d.R || !plan_ok(plan) || !home_grad_local || P <= 0) return MOONEP_ERR_ARG;
+    if (d.B > 0 && !reduce_bufs) return MOONEP_ERR_ARG;
+    if (d.B == 0) return MOONEP_OK;  // no prefetched replica can exist
+    if (reinterpret_cast<uintptr_t>(home_grad_local) & 3u) return MOONEP_ERR_ALIGN;
+    return launch_reduce_ep(d, rank, *plan, reduce_bufs, home_grad_local, (long long)P,
+                            static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -68,6 +68,28 @@ __host__ inline WsLayout ws_layout(const Dims &d)
     return w;
 }
 
+// Workspace of one rank in expert parallelism (moonep_ep_*): the header
+// (the count kernel's ticket and invalid-id count, the planner's status
+// word), this rank's per-chunk expert counts, and the host rows.
+struct EpWsLayout {
+    size_t hdr;        // int32[8]
+    size_t cc;         // int32 [nchunk][E] over the rank's S tokens
+    size_t host_dst0;  // int32 [2E+R]
+    size_t total;
+};
+
+__host__ inline EpWsLayout ws_layout_ep(const Dims &d)
+{
+    EpWsLayout w;
+    const size_t i4 = sizeof(int32_t);
+    size_t o = 0;
+    w.hdr = o; o = align256(o + WS_HDR_INTS * i4);
+    w.cc = o; o = align256(o + i4 * (size_t)d.nchunk * d.E);
+    w.host_dst0 = o; o = align256(o + i4 * (size_t)(2 * d.E + d.R));
+    w.total = o;
+    return w;
+}
+
 // Division by a run-time invariant 31-bit divisor with a multiply-high and a
 // shift (Granlund & Montgomery, "Division by invariant integers using
 // multiplication", 1994): for 0 <= n < 2^31 and d >= 1,
@@ -233,6 +255,58 @@ __device__ inline int block_exscan(int *a, int n, int *wsum)
     if (n <= 3 * nt) return block_exscan_per<3>(a, n, wsum, 3);
     if (n <= 4 * nt) return block_exscan_per<4>(a, n, wsum, 4);
     return block_exscan_per<0>(a, n, wsum, (n + nt - 1) / nt);
+}
+
+// Rows of the plan's prefetched replicas, grouped by expert, built by one
+// block in shared memory (used by the replica-gradient reduce and the weight
+// prefetch): for i < n (the return value), expert s_e[i] -- the plan's
+// rep_home_list order, or -1 where take(e) rejects it -- has the replica
+// rows s_row[s_off[i] .. s_off[i+1]) = r*B + b (b = slot - L < B) in
+// ascending host rank order.  Every count and index read from the plan is
+// clamped: s_row holds at most max_list rows.  An empty plan gives 0.
+// Every thread of the block must call it (two barriers of its own, one of
+// the scan's).  s_e: MOONEP_MAX_E ints, s_off: MOONEP_MAX_E + 1, wsum: 32.
+template <typename Take>
+__device__ int replica_lists(const moonep_plan_t &p, int E, int L, int B, int R, Take take, int *s_e, int *s_off,
+                             int *s_row, int max_list, int *wsum)
+{
+    const int status = __ldg(p.info + MOONEP_INFO_STATUS);
+    if (status & ST_EMPTY_PLAN) return 0;
+    const int n_exp = min(max(__ldg(p.info + MOONEP_INFO_N_REP_EXPERTS), 0), E);
+    if (n_exp == 0) return 0;
+    const int tid = threadIdx.x, nh = 2 * E + R;
+    for (int i = tid; i <= n_exp; i += blockDim.x) {
+        int c = 0, e = -1;
+        if (i < n_exp) {
+            e = __ldg(p.rep_home_list + i);
+            if (e >= 0 && e < E && !take(e)) e = -1;
+            if (e >= 0 && e < E) {
+                const int home = e / L;
+                const int h0 = max(0, __ldg(p.host_ptr + e)), h1 = min(nh, __ldg(p.host_ptr + e + 1));
+                for (int h = h0; h < h1; ++h) {
+                    const int r = __ldg(p.host_rank + h), b = __ldg(p.host_slot + h) - L;
+                    c += (r != home && r >= 0 && r < R && b >= 0 && b < B);
+                }
+            }
+        }
+        if (i < n_exp) s_e[i] = e;
+        s_off[i] = c;
+    }
+    __syncthreads();
+    block_exscan(s_off, n_exp + 1, wsum);
+    for (int i = tid; i < n_exp; i += blockDim.x) {
+        const int e = s_e[i];
+        if (e < 0 || e >= E) continue;
+        const int home = e / L;
+        int o = s_off[i];
+        const int h0 = max(0, __ldg(p.host_ptr + e)), h1 = min(nh, __ldg(p.host_ptr + e + 1));
+        for (int h = h0; h < h1; ++h) {
+            const int r = __ldg(p.host_rank + h), b = __ldg(p.host_slot + h) - L;
+            if (r != home && r >= 0 && r < R && b >= 0 && b < B && o < max_list) s_row[o++] = r * B + b;
+        }
+    }
+    __syncthreads();
+    return n_exp;
 }
 
 }  // namespace moonep

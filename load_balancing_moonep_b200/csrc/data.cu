@@ -80,15 +80,56 @@ __device__ __forceinline__ bool row_ok(int row, int rows, int *info)
     return false;
 }
 
+// ------------------------------------------------------ buffer addressing
+
+// Where buffer row g (a global row in [0, R*S*K), rank g / (S*K)) lives.
+// row() returns nullptr, and raises MOONEP_ST_ROW_RANGE, for a row outside
+// [0, rows) or a buffer that cannot be addressed; the caller skips it.
+
+// One allocation holds every rank's rows: the single-GPU layout [R, S*K, H]
+// (its base is checked on the host).
+template <typename T>
+struct FlatRows {
+    T *base;
+    int vpr;  // 16-byte vectors per row
+    __device__ __forceinline__ T *row(int g, int rows, int *info) const
+    {
+        return row_ok(g, rows, info) ? base + (size_t)g * vpr : nullptr;
+    }
+};
+
+// Each rank's [S*K, H] buffer is its own allocation, reached through a
+// device array of R pointers (peer memory of the other GPUs in expert
+// parallelism): row g is local row g - r*C of rank r = g / C.  A null or
+// misaligned pointer in the array is reported, never dereferenced.
+template <typename T>
+struct RankRows {
+    T *const *bases;  // [R] device pointers
+    FastDiv fC;       // division by C = S*K
+    int C;
+    int vpr;
+    __device__ __forceinline__ T *row(int g, int rows, int *info) const
+    {
+        if (!row_ok(g, rows, info)) return nullptr;
+        const int r = (int)fdiv((uint32_t)g, fC);
+        T *b = bases[r];
+        if (b == nullptr || (reinterpret_cast<uintptr_t>(b) & 15u)) {
+            atomicOr(info + MOONEP_INFO_STATUS, MOONEP_ST_ROW_RANGE);
+            return nullptr;
+        }
+        return b + (size_t)(g - r * C) * vpr;
+    }
+};
+
 // --------------------------------------------------------------- dispatch
 
 // One warp per token: the row is read once, in U 16-byte vectors per lane,
 // and stored to each of the K destination rows (broadcast by shuffles).
 // A compile-time K with the K row pointers held in registers measured
 // slower on B200 (2.99 vs 2.80 ms at the large shape), so K stays run-time.
-template <int U>
+template <int U, typename Rows>
 __global__ void __launch_bounds__(DATA_THREADS) dispatch_kernel(const uint4 *__restrict__ hidden,
-                                                               uint4 *__restrict__ buf,
+                                                               const Rows buf,
                                                                const int *__restrict__ dst_pos,
                                                                int *info, int tokens, int K, int vpr,
                                                                int rows)
@@ -110,8 +151,8 @@ __global__ void __launch_bounds__(DATA_THREADS) dispatch_kernel(const uint4 *__r
             }
             for (int k = 0; k < K; ++k) {
                 const int dk = k < 32 ? __shfl_sync(FULL_MASK, dl, k) : __ldg(dp + k);
-                if (!row_ok(dk, rows, info)) continue;
-                uint4 *dst = buf + (size_t)dk * vpr;
+                uint4 *dst = buf.row(dk, rows, info);
+                if (dst == nullptr) continue;
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
                     const int c = c0 + u * 32 + lane;
@@ -126,8 +167,8 @@ __global__ void __launch_bounds__(DATA_THREADS) dispatch_kernel(const uint4 *__r
 
 // KT > 0: compile-time K (all K loads of a vector issued together);
 // KT == 0: any K, one expert row at a time.
-template <int KT, int U>
-__global__ void __launch_bounds__(DATA_THREADS) combine_kernel(const uint4 *__restrict__ y,
+template <int KT, int U, typename Rows>
+__global__ void __launch_bounds__(DATA_THREADS) combine_kernel(const Rows y,
                                                               const float *__restrict__ w,
                                                               uint4 *__restrict__ out,
                                                               const int *__restrict__ dst_pos, int *info,
@@ -153,9 +194,9 @@ __global__ void __launch_bounds__(DATA_THREADS) combine_kernel(const uint4 *__re
                 uint4 v[KT][U];
 #pragma unroll
                 for (int k = 0; k < KT; ++k) {
-                    int dk = __shfl_sync(FULL_MASK, dl, k);
-                    const bool ok = row_ok(dk, rows, info);
-                    const uint4 *row = y + (size_t)(ok ? dk : 0) * vpr;
+                    const int dk = __shfl_sync(FULL_MASK, dl, k);
+                    const uint4 *row = y.row(dk, rows, info);
+                    const bool ok = row != nullptr;
 #pragma unroll
                     for (int u = 0; u < U; ++u) {
                         const int c = c0 + u * 32 + lane;
@@ -178,8 +219,8 @@ __global__ void __launch_bounds__(DATA_THREADS) combine_kernel(const uint4 *__re
                 for (int k = 0; k < K; ++k) {
                     const int dk = k < 32 ? __shfl_sync(FULL_MASK, dl, k) : __ldg(dp + k);
                     const float wk = k < 32 ? __shfl_sync(FULL_MASK, wl, k) : __ldg(wp + k);
-                    if (!row_ok(dk, rows, info)) continue;
-                    const uint4 *row = y + (size_t)dk * vpr;
+                    const uint4 *row = y.row(dk, rows, info);
+                    if (row == nullptr) continue;
 #pragma unroll
                     for (int u = 0; u < U; ++u) {
                         const int c = c0 + u * 32 + lane;
@@ -212,10 +253,10 @@ __device__ __forceinline__ float dot8(const float a[8], const float b[8])
     return ((p0 + p1) + (p2 + p3)) + ((p4 + p5) + (p6 + p7));
 }
 
-template <int KT, int U>
+template <int KT, int U, typename YRows, typename BRows>
 __global__ void __launch_bounds__(DATA_THREADS) combine_bwd_kernel(
-    const uint4 *__restrict__ dy, const float *__restrict__ w, const uint4 *__restrict__ y,
-    uint4 *__restrict__ dy_buf, float *__restrict__ dw, const int *__restrict__ dst_pos, int *info,
+    const uint4 *__restrict__ dy, const float *__restrict__ w, const YRows y,
+    const BRows dy_buf, float *__restrict__ dw, const int *__restrict__ dst_pos, int *info,
     int tokens, int vpr, int unscaled, int rows)
 {
     if (plan_invalid(info)) return;
@@ -245,9 +286,10 @@ __global__ void __launch_bounds__(DATA_THREADS) combine_bwd_kernel(
 #pragma unroll
             for (int k = 0; k < K; ++k) {
                 const int dk = __shfl_sync(FULL_MASK, dl, k);
-                const bool ok = row_ok(dk, rows, info);
+                // a pair is taken only when both of its rows can be addressed
+                const uint4 *yr = y.row(dk, rows, info);
+                const bool ok = yr != nullptr && dy_buf.row(dk, rows, info) != nullptr;
                 okm |= ok ? (1u << k) : 0u;
-                const uint4 *yr = y + (size_t)(ok ? dk : 0) * vpr;
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
                     const int c = c0 + u * 32 + lane;
@@ -260,7 +302,8 @@ __global__ void __launch_bounds__(DATA_THREADS) combine_bwd_kernel(
                 const int dk = __shfl_sync(FULL_MASK, dl, k);
                 const float wk = __shfl_sync(FULL_MASK, wl, k);
                 if (!(okm & (1u << k))) continue;
-                uint4 *br = dy_buf + (size_t)dk * vpr;
+                uint4 *br = dy_buf.row(dk, rows, info);
+                if (br == nullptr) continue;
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
                     const int c = c0 + u * 32 + lane;
@@ -302,56 +345,64 @@ static int data_grid(int tokens)
     return want < 1 ? 1 : (want > (1LL << 30) ? (1 << 30) : (int)want);
 }
 
-int launch_dispatch(const Dims &d, const int *dst_pos, int *info, const uint16_t *hidden, uint16_t *buf,
-                    cudaStream_t st)
+template <typename T>
+static FlatRows<T> flat_rows(const Dims &d, T *base)
 {
-    const int vpr = d.H / 8;
-    const int grid = data_grid(d.tokens);
-    dispatch_kernel<4><<<grid, DATA_THREADS, 0, st>>>(reinterpret_cast<const uint4 *>(hidden),
-                                                     reinterpret_cast<uint4 *>(buf), dst_pos, info, d.tokens,
-                                                     d.K, vpr, d.pairs);
+    return FlatRows<T>{base, d.H / 8};
+}
+
+template <typename T>
+static RankRows<T> rank_rows(const Dims &d, T *const *bases)
+{
+    return RankRows<T>{bases, make_fastdiv((uint32_t)d.C), d.C, d.H / 8};
+}
+
+// tokens: the tokens this launch reads (R*S for one GPU, S for one rank);
+// buffer rows are global rows in [0, R*S*K) either way
+template <typename Rows>
+static int dispatch_rows(const Dims &d, int tokens, const int *dst_pos, int *info, const uint16_t *hidden,
+                         const Rows &buf, cudaStream_t st)
+{
+    dispatch_kernel<4, Rows><<<data_grid(tokens), DATA_THREADS, 0, st>>>(
+        reinterpret_cast<const uint4 *>(hidden), buf, dst_pos, info, tokens, d.K, d.H / 8, d.pairs);
     return cudaGetLastError() == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
 }
 
-int launch_combine(const Dims &d, const int *dst_pos, int *info, const uint16_t *y, const float *w,
-                   uint16_t *out, cudaStream_t st)
+template <typename Rows>
+static int combine_rows(const Dims &d, int T, const int *dst_pos, int *info, const Rows &yv, const float *w,
+                        uint16_t *out, cudaStream_t st)
 {
-    const int vpr = d.H / 8;
-    const int grid = data_grid(d.tokens);
-    const uint4 *yv = reinterpret_cast<const uint4 *>(y);
+    const int vpr = d.H / 8, grid = data_grid(T), K = d.K, rows = d.pairs;
     uint4 *ov = reinterpret_cast<uint4 *>(out);
-    const int T = d.tokens, K = d.K, rows = d.pairs;
     switch (K) {
-    case 1: combine_kernel<1, 4><<<grid, DATA_THREADS, 0, st>>>(yv, w, ov, dst_pos, info, T, K, vpr, rows); break;
-    case 2: combine_kernel<2, 4><<<grid, DATA_THREADS, 0, st>>>(yv, w, ov, dst_pos, info, T, K, vpr, rows); break;
-    case 4: combine_kernel<4, 2><<<grid, DATA_THREADS, 0, st>>>(yv, w, ov, dst_pos, info, T, K, vpr, rows); break;
-    case 6: combine_kernel<6, 2><<<grid, DATA_THREADS, 0, st>>>(yv, w, ov, dst_pos, info, T, K, vpr, rows); break;
-    case 8: combine_kernel<8, 2><<<grid, DATA_THREADS, 0, st>>>(yv, w, ov, dst_pos, info, T, K, vpr, rows); break;
-    default: combine_kernel<0, 2><<<grid, DATA_THREADS, 0, st>>>(yv, w, ov, dst_pos, info, T, K, vpr, rows); break;
+    case 1: combine_kernel<1, 4, Rows><<<grid, DATA_THREADS, 0, st>>>(yv, w, ov, dst_pos, info, T, K, vpr, rows); break;
+    case 2: combine_kernel<2, 4, Rows><<<grid, DATA_THREADS, 0, st>>>(yv, w, ov, dst_pos, info, T, K, vpr, rows); break;
+    case 4: combine_kernel<4, 2, Rows><<<grid, DATA_THREADS, 0, st>>>(yv, w, ov, dst_pos, info, T, K, vpr, rows); break;
+    case 6: combine_kernel<6, 2, Rows><<<grid, DATA_THREADS, 0, st>>>(yv, w, ov, dst_pos, info, T, K, vpr, rows); break;
+    case 8: combine_kernel<8, 2, Rows><<<grid, DATA_THREADS, 0, st>>>(yv, w, ov, dst_pos, info, T, K, vpr, rows); break;
+    default: combine_kernel<0, 2, Rows><<<grid, DATA_THREADS, 0, st>>>(yv, w, ov, dst_pos, info, T, K, vpr, rows); break;
     }
     return cudaGetLastError() == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
 }
 
-template <int KT>
-static void launch_bwd_k(const Dims &d, int grid, const uint4 *dy, const float *w, const uint4 *y, uint4 *dyb,
+template <int KT, typename YRows, typename BRows>
+static void launch_bwd_k(const Dims &d, int T, const uint4 *dy, const float *w, const YRows &y, const BRows &dyb,
                          float *dw, const int *dst_pos, int *info, int unscaled, cudaStream_t st)
 {
     constexpr int U = KT <= 8 ? 2 : 1;  // U = 1 measured slower at K = 8
-    combine_bwd_kernel<KT, U><<<grid, DATA_THREADS, 0, st>>>(dy, w, y, dyb, dw, dst_pos, info, d.tokens,
-                                                            d.H / 8, unscaled, d.pairs);
+    combine_bwd_kernel<KT, U, YRows, BRows><<<data_grid(T), DATA_THREADS, 0, st>>>(
+        dy, w, y, dyb, dw, dst_pos, info, T, d.H / 8, unscaled, d.pairs);
 }
 
-int launch_combine_backward(const Dims &d, const int *dst_pos, int *info, const uint16_t *dy, const float *w,
-                            const uint16_t *y, uint16_t *dy_buf, float *dw, cudaStream_t st)
+template <typename YRows, typename BRows>
+static int bwd_rows(const Dims &d, int T, const int *dst_pos, int *info, const uint16_t *dy, const float *w,
+                    const YRows &yv, const BRows &bv, float *dw, cudaStream_t st)
 {
-    const int grid = data_grid(d.tokens);
     const uint4 *dyv = reinterpret_cast<const uint4 *>(dy);
-    const uint4 *yv = reinterpret_cast<const uint4 *>(y);
-    uint4 *bv = reinterpret_cast<uint4 *>(dy_buf);
     const int uns = (d.flags & MOONEP_FLAG_BWD_UNSCALED) ? 1 : 0;
     switch (d.K) {
 #define MOONEP_BWD_CASE(k) \
-    case k: launch_bwd_k<k>(d, grid, dyv, w, yv, bv, dw, dst_pos, info, uns, st); break;
+    case k: launch_bwd_k<k>(d, T, dyv, w, yv, bv, dw, dst_pos, info, uns, st); break;
     MOONEP_BWD_CASE(1) MOONEP_BWD_CASE(2) MOONEP_BWD_CASE(3) MOONEP_BWD_CASE(4)
     MOONEP_BWD_CASE(5) MOONEP_BWD_CASE(6) MOONEP_BWD_CASE(7) MOONEP_BWD_CASE(8)
     MOONEP_BWD_CASE(9) MOONEP_BWD_CASE(10) MOONEP_BWD_CASE(11) MOONEP_BWD_CASE(12)
@@ -360,6 +411,50 @@ int launch_combine_backward(const Dims &d, const int *dst_pos, int *info, const 
     default: return MOONEP_ERR_LIMIT;
     }
     return cudaGetLastError() == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
+}
+
+// ---- one GPU: every rank's rows in one allocation
+
+int launch_dispatch(const Dims &d, const int *dst_pos, int *info, const uint16_t *hidden, uint16_t *buf,
+                    cudaStream_t st)
+{
+    return dispatch_rows(d, d.tokens, dst_pos, info, hidden, flat_rows(d, reinterpret_cast<uint4 *>(buf)), st);
+}
+
+int launch_combine(const Dims &d, const int *dst_pos, int *info, const uint16_t *y, const float *w,
+                   uint16_t *out, cudaStream_t st)
+{
+    return combine_rows(d, d.tokens, dst_pos, info, flat_rows(d, reinterpret_cast<const uint4 *>(y)), w, out, st);
+}
+
+int launch_combine_backward(const Dims &d, const int *dst_pos, int *info, const uint16_t *dy, const float *w,
+                            const uint16_t *y, uint16_t *dy_buf, float *dw, cudaStream_t st)
+{
+    return bwd_rows(d, d.tokens, dst_pos, info, dy, w, flat_rows(d, reinterpret_cast<const uint4 *>(y)),
+                    flat_rows(d, reinterpret_cast<uint4 *>(dy_buf)), dw, st);
+}
+
+// ---- expert parallelism: one rank's S tokens, every rank's rows in its own
+// allocation (peer memory), bases = device array of R row-buffer pointers
+
+int launch_dispatch_ep(const Dims &d, const int *dst_pos, int *info, const uint16_t *hidden,
+                       uint16_t *const *bufs, cudaStream_t st)
+{
+    return dispatch_rows(d, d.S, dst_pos, info, hidden, rank_rows(d, reinterpret_cast<uint4 *const *>(bufs)), st);
+}
+
+int launch_combine_ep(const Dims &d, const int *dst_pos, int *info, const uint16_t *const *ys, const float *w,
+                      uint16_t *out, cudaStream_t st)
+{
+    return combine_rows(d, d.S, dst_pos, info, rank_rows(d, reinterpret_cast<const uint4 *const *>(ys)), w, out,
+                        st);
+}
+
+int launch_combine_backward_ep(const Dims &d, const int *dst_pos, int *info, const uint16_t *dy, const float *w,
+                               const uint16_t *const *ys, uint16_t *const *dy_bufs, float *dw, cudaStream_t st)
+{
+    return bwd_rows(d, d.S, dst_pos, info, dy, w, rank_rows(d, reinterpret_cast<const uint4 *const *>(ys)),
+                    rank_rows(d, reinterpret_cast<uint4 *const *>(dy_bufs)), dw, st);
 }
 
 }  // namespace moonep

@@ -61,7 +61,8 @@ struct PlanParams {
     const int32_t *topk;
     moonep_plan_t p;
     int *hdr;        // ticket, status, call sequence, counts-ready mark, arrivals
-    int *gs;         // [2][ngroups][E]
+    int *gs;         // [2][ngroups][E] (expert parallelism: the gathered counts [R][E+1])
+    int gs_stride;   // ints between the count rows of gs: E (E + 1 for the gathered counts)
     int *cc;         // [nchunk][E]
     int *host_dst0;  // [2E+R]
     FastDiv fC, fL;  // divisions by C and L
@@ -665,9 +666,9 @@ __device__ void plan_block(const PlanParams &a, int *sm, int seq)
     unsigned part = 0;  // <= 2 values < 2^31 each (negative ones are flagged)
     int negative = 0;
     {
-        const int *gsb = a.gs + (size_t)parity * d.ngroups * E;
+        const int *gsb = a.gs + (size_t)parity * d.ngroups * a.gs_stride;
         for (int e = tid; e < E; e += nt) {
-            const int v = sum_strided<32>(gsb + e, E, d.ngroups);
+            const int v = sum_strided<32>(gsb + e, a.gs_stride, d.ngroups);
             T[e] = v;
             a.p.expert_count[e] = v;
             negative |= v < 0;
@@ -1070,6 +1071,68 @@ __global__ void __launch_bounds__(PLAN_THREADS) hist_plan_kernel(PlanParams a)
 
 // ---------------------------------------------------------- assignment
 
+// Pass A, on the ids alone: the calling warp walks its contiguous sub-range
+// [wbeg, wend) of the staged ids in (t, k) order, ranking equal experts with
+// ballots, so loc is the pair's rank among the sub-range's earlier pairs of
+// its expert and the warp's counters wc[E] end as its per-expert counts.
+// ids[i] becomes loc << PACK_BITS | e.  (Out-of-range ids are left as they
+// are; they make the plan empty.)
+__device__ __forceinline__ void assign_pass_a(int *ids, int *wc, int wbeg, int wend, int E, int ebits)
+{
+    const int lane = threadIdx.x & 31;
+    for (int b = wbeg; b < wend; b += 32) {
+        const int i = b + lane;
+        const bool valid = i < wend;
+        const int e = valid ? ids[i] : 0;
+        const bool ok = valid && e >= 0 && e < E;
+        const unsigned peers = peers_of(ok ? e : 0, ok, ebits);
+        int loc = 0;
+        if (ok) loc = wc[e] + __popc(peers & lanemask_lt());
+        __syncwarp();
+        if (ok && lane == __ffs(peers) - 1) wc[e] += __popc(peers);
+        __syncwarp();
+        if (ok) ids[i] = (loc << PACK_BITS) | e;
+    }
+}
+
+// Pass B for the calling warp's sub-range: g = warp base wb[e] + loc is the
+// pair's rank among all pairs of its expert in (t, k) order; the host
+// interval holding g gives the buffer row hdst[h] + g, a global row in
+// [0, rows).  Pair i of the sub-range is pair p0 + i of dst_pos; row_src
+// (may be null) gets the inverse.  Returns the number of the warp's pairs
+// that land on another rank than their source rank: src_rank >= 0 is the
+// source rank of every pair (one rank's pairs), -1 derives it as p / C.
+__device__ __forceinline__ int assign_pass_b(const int *ids, const int *wb, const int *hptr, const int *hstart,
+                                             const int *hdst, int wbeg, int wend, int p0, int E, int rows, int C,
+                                             const FastDiv &fC, int src_rank, int *dst_pos, int *row_src,
+                                             int *info)
+{
+    const int lane = threadIdx.x & 31;
+    int remote = 0;
+    for (int i = wbeg + lane; i < wend; i += 32) {
+        const int v = ids[i];
+        const int e = v & PACK_MASK, loc = v >> PACK_BITS;
+        if (v < 0 || e >= E) continue;  // cannot happen in a non-empty plan
+        const int g = wb[e] + loc;
+        int h = hptr[e];
+        const int hend = hptr[e + 1];
+        while (h + 1 < hend && hstart[h + 1] <= g) ++h;
+        const int dst = hdst[h] + g;
+        const int p = p0 + i;
+        if (dst < 0 || dst >= rows) {  // cannot happen for a consistent plan
+            atomicOr(info + MOONEP_INFO_STATUS, MOONEP_ST_ROW_RANGE);
+            dst_pos[p] = -1;
+            continue;
+        }
+        dst_pos[p] = dst;
+        if (row_src) row_src[dst] = p;
+        // the source rank's first row: the rank of pair p is p / (S*K) = p / C
+        const uint32_t src0 = (src_rank >= 0 ? (uint32_t)src_rank : fdiv((uint32_t)p, fC)) * (uint32_t)C;
+        remote += (uint32_t)dst - src0 >= (uint32_t)C;
+    }
+    return remote;
+}
+
 __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
 {
     extern __shared__ int sm[];
@@ -1103,22 +1166,7 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
     // (Out-of-range ids are left as they are; they make the plan empty.)
     const int per = (n + ASSIGN_WARPS - 1) / ASSIGN_WARPS;
     const int wbeg = min(warp * per, n), wend = min(wbeg + per, n);
-    {
-        int *wc = cnt + warp * E;
-        for (int b = wbeg; b < wend; b += 32) {
-            const int i = b + lane;
-            const bool valid = i < wend;
-            const int e = valid ? ids[i] : 0;
-            const bool ok = valid && e >= 0 && e < E;
-            const unsigned peers = peers_of(ok ? e : 0, ok, d.ebits);
-            int loc = 0;
-            if (ok) loc = wc[e] + __popc(peers & lanemask_lt());
-            __syncwarp();
-            if (ok && lane == __ffs(peers) - 1) wc[e] += __popc(peers);
-            __syncwarp();
-            if (ok) ids[i] = (loc << PACK_BITS) | e;
-        }
-    }
+    assign_pass_a(ids, cnt + warp * E, wbeg, wend, E, d.ebits);
 
     // ---- the counts are complete once the last histogram CTA has set READY;
     // the planner CTA is still running then, and the chunk bases and warp
@@ -1272,30 +1320,8 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
 
     // pass B: g = warp base + loc is the pair's rank among all pairs of its
     // expert in (t, k) order; the host interval holding g gives the buffer row
-    int remote = 0;
-    {
-        const int *wb = cnt + warp * E;
-        for (int i = wbeg + lane; i < wend; i += 32) {
-            const int v = ids[i];
-            const int e = v & PACK_MASK, loc = v >> PACK_BITS;
-            if (v < 0 || e >= E) continue;  // cannot happen in a non-empty plan
-            const int g = wb[e] + loc;
-            int h = hptr[e];
-            const int hend = hptr[e + 1];
-            while (h + 1 < hend && hstart[h + 1] <= g) ++h;
-            const int dst = hdst[h] + g;
-            const int p = p0 + i;
-            if (dst < 0 || dst >= R * C) {  // cannot happen for a consistent plan
-                atomicOr(a.p.info + MOONEP_INFO_STATUS, MOONEP_ST_ROW_RANGE);
-                a.p.dst_pos[p] = -1;
-                continue;
-            }
-            a.p.dst_pos[p] = dst;
-            a.p.row_src[dst] = p;
-            // source rank of pair p is p / (S*K) = p / C
-            remote += (uint32_t)dst - fdiv((uint32_t)p, a.fC) * (uint32_t)C >= (uint32_t)C;
-        }
-    }
+    int remote = assign_pass_b(ids, cnt + warp * E, hptr, hstart, hdst, wbeg, wend, p0, E, R * C, C, a.fC, -1,
+                               a.p.dst_pos, a.p.row_src, a.p.info);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) remote += __shfl_xor_sync(FULL_MASK, remote, o);
     if (lane == 0) red[warp] = remote;
@@ -1331,6 +1357,7 @@ int launch_plan(const Dims &d, const int32_t *topk, const moonep_plan_t &p, void
     a.gs = reinterpret_cast<int *>(w + wl.gs);
     a.cc = reinterpret_cast<int *>(w + wl.cc);
     a.host_dst0 = reinterpret_cast<int *>(w + wl.host_dst0);
+    a.gs_stride = d.E;
     a.fC = make_fastdiv((uint32_t)d.C);
     a.fL = make_fastdiv((uint32_t)d.L);
     a.spin_limit = g_wait_limit.load(std::memory_order_relaxed);
@@ -1360,6 +1387,262 @@ int launch_plan(const Dims &d, const int32_t *topk, const moonep_plan_t &p, void
     c2.dynamicSmemBytes = smem2;
     if (cudaLaunchKernelEx(&c2, assign_kernel, a) != cudaSuccess) return MOONEP_ERR_CUDA;
     return MOONEP_OK;
+}
+
+// ------------------------------------------------------- expert parallelism
+//
+// One process per GPU; rank `rank` of R owns S tokens (its topk rows [S, K]).
+// The MoonEP article ("The core idea: dynamic redundant experts") writes
+// every pair straight into its expert-grouped row on a remote rank; the plan
+// needs every rank's per-expert counts, which are small ([E] per rank) and
+// all-gathered by the caller between the count and the plan.  Every rank then
+// runs the same planner on the same counts, so all ranks hold identical plan
+// tables, and places its own pairs: the pair's rank g within its expert is
+// the counts of the lower ranks plus its rank among this rank's own pairs,
+// exactly the global (t, k) order of the single-GPU plan.  The per-rank
+// chunking is over the S local tokens (d.nchunk, d.chunk_tokens); d.ngroups
+// is R, the rows of the gathered counts.
+
+// EP workspace header slots: the count kernel's ticket and invalid-id count,
+// the planner's status word
+enum { EP_TICKET = WS_TICKET, EP_STATUS = WS_STATUS, EP_BAD = WS_ARRIVED };
+
+struct EpCountParams {
+    Dims d;
+    const int32_t *topk;  // [S, K]
+    int *hdr, *cc;
+    int32_t *counts_row;  // [E + 1]
+};
+
+// Per-chunk histograms of the rank's own ids (into the workspace, for the
+// assignment), then, in the CTA that finishes last, their sums: the rank's
+// counts row [E] and, in slot E, its number of ids outside [0, E).
+__global__ void __launch_bounds__(PLAN_THREADS) ep_count_kernel(EpCountParams a)
+{
+    extern __shared__ int sm[];
+    __shared__ int s_last;
+    const Dims &d = a.d;
+    const int E = d.E, K = d.K, tid = threadIdx.x, nt = blockDim.x;
+    pdl_wait();  // the producer of the ids
+    const int chunk = blockIdx.x;
+    const int t0 = chunk * d.chunk_tokens, t1 = min(t0 + d.chunk_tokens, d.S);
+    const int p0 = t0 * K, n = (t1 - t0) * K;
+    int *hist = sm, *ids = sm + E;
+    for (int e = tid; e < E; e += nt) hist[e] = 0;
+    for (int i = tid; i < n; i += nt) ids[i] = __ldg(a.topk + p0 + i);
+    __syncthreads();
+    int bad = 0;
+    for (int i = tid; i < n; i += nt) {
+        const int e = ids[i];
+        if (e < 0 || e >= E) ++bad;
+        else atomicAdd(&hist[e], 1);
+    }
+    bad = __syncthreads_count(bad > 0) > 0 ? __reduce_add_sync(FULL_MASK, bad) : 0;
+    if ((tid & 31) == 0 && bad) atomicAdd(a.hdr + EP_BAD, bad);
+    for (int e = tid; e < E; e += nt) a.cc[(size_t)chunk * E + e] = hist[e];
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        const bool last = atomicAdd(a.hdr + EP_TICKET, 1) == (int)gridDim.x - 1;
+        if (last) __threadfence();
+        s_last = last;
+    }
+    __syncthreads();
+    if (!s_last) return;
+    for (int e = tid; e < E; e += nt) a.counts_row[e] = sum_strided<32>(a.cc + e, E, d.nchunk);
+    if (tid == 0) {
+        a.counts_row[E] = ld_cg(a.hdr + EP_BAD);
+        a.hdr[EP_BAD] = 0;
+        a.hdr[EP_TICKET] = 0;
+    }
+}
+
+// The planner on the gathered counts [R][E+1], in one CTA: the tables'
+// empty defaults, the status (an invalid id on any rank empties the plan),
+// then the single-GPU planner with the counts as its R count rows.
+__global__ void __launch_bounds__(PLAN_THREADS) ep_plan_kernel(PlanParams a)
+{
+    extern __shared__ int sm[];
+    const Dims &d = a.d;
+    const int E = d.E, R = d.R, tid = threadIdx.x;
+    constexpr int nt = PLAN_THREADS;
+    const int nh = 2 * E + R;
+    // the assignment grid may start its prologue on the ids
+    pdl_launch_dependents();
+    for (int x = tid; x < R * E; x += nt) {
+        a.p.slot_expert[x] = -1;
+        a.p.slot_count[x] = 0;
+    }
+    for (int x = tid; x < R * (E + 1); x += nt) a.p.slot_offset[x] = d.C;
+    for (int x = tid; x < E + R; x += nt) {
+        a.p.rep_expert[x] = -1;
+        a.p.rep_rank[x] = -1;
+        a.p.rep_slot[x] = -1;
+        a.p.rep_quota[x] = 0;
+    }
+    for (int x = tid; x < nh; x += nt) {
+        a.p.host_rank[x] = -1;
+        a.p.host_slot[x] = -1;
+        a.p.host_start[x] = 0;
+        a.p.host_quota[x] = 0;
+    }
+    if (tid < 32) {
+        int bad = 0;
+        for (int r = tid; r < R; r += 32) bad |= ld_cg(a.gs + (size_t)r * a.gs_stride + E) != 0;
+        bad = __any_sync(FULL_MASK, bad);
+        if (tid == 0) a.hdr[WS_STATUS] = bad ? MOONEP_ST_EXPERT_ID_RANGE : 0;
+    }
+    __syncthreads();
+    plan_block(a, sm, 0);
+    __syncthreads();
+    // an empty plan: the tables as moonep_plan leaves them
+    if (ld_cg(a.p.info + MOONEP_INFO_STATUS) & ST_EMPTY_PLAN) {
+        for (int x = tid; x < R * (E + 1); x += nt) a.p.slot_offset[x] = 0;
+        for (int x = tid; x <= E; x += nt) a.p.host_ptr[x] = 0;
+        for (int x = tid; x < E; x += nt) a.p.rep_home_list[x] = -1;
+    }
+}
+
+// The rank's own pairs: pass A on the ids while the planner runs, chunk
+// bases from the lower ranks' counts and this rank's earlier chunks, then
+// (after the planner grid) pass B.  dst_pos[0 .. S*K) gets global rows;
+// row_src is not written (the rows of this rank's buffer are filled by every
+// rank).  info[MOONEP_INFO_N_REMOTE_PAIRS] counts this rank's pairs placed
+// on another rank.
+__global__ void __launch_bounds__(ASSIGN_THREADS, 2) ep_assign_kernel(PlanParams a, int rank)
+{
+    extern __shared__ int sm[];
+    const Dims &d = a.d;
+    const int E = d.E, K = d.K, R = d.R, C = d.C;
+    const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5;
+    const int chunk = blockIdx.x;
+    const int t0 = chunk * d.chunk_tokens, t1 = min(t0 + d.chunk_tokens, d.S);
+    const int p0 = t0 * K, n = (t1 - t0) * K;
+    const int max_pairs = d.chunk_tokens * K;
+    const int nh = 2 * E + R;
+    int *cnt = sm;                      // ASSIGN_WARPS * E
+    int *ids = cnt + ASSIGN_WARPS * E;  // max_pairs
+    int *hptr = ids + max_pairs;        // E + 1
+    int *hstart = hptr + E + 1;         // nh
+    int *hdst = hstart + nh;            // nh
+    int *red = hdst + nh;               // 32
+
+    // on the ids and the counts only, overlapping the planner
+    for (int i = tid; i < ASSIGN_WARPS * E; i += nt) cnt[i] = 0;
+    for (int i = tid; i < n; i += nt) ids[i] = __ldg(a.topk + p0 + i);
+    __syncthreads();
+    const int per = (n + ASSIGN_WARPS - 1) / ASSIGN_WARPS;
+    const int wbeg = min(warp * per, n), wend = min(wbeg + per, n);
+    assign_pass_a(ids, cnt + warp * E, wbeg, wend, E, d.ebits);
+    __syncthreads();
+    // chunk base: pairs of e on lower ranks plus on this rank's earlier
+    // chunks; then the warp bases
+    for (int e = tid; e < E; e += nt) {
+        int s = sum_strided<32>(a.gs + e, a.gs_stride, rank) + sum_strided<32>(a.cc + e, E, chunk);
+        for (int w = 0; w < ASSIGN_WARPS; ++w) {
+            const int t = cnt[w * E + e];
+            cnt[w * E + e] = s;
+            s += t;
+        }
+    }
+    // the plan is complete once the planner grid has finished
+    pdl_wait();
+    const int status = ld_cg(a.p.info + MOONEP_INFO_STATUS);
+    for (int e = tid; e <= E; e += nt) hptr[e] = min(max(ld_cg(a.p.host_ptr + e), 0), nh);
+    for (int h = tid; h < nh; h += nt) {
+        hstart[h] = ld_cg(a.p.host_start + h);
+        hdst[h] = ld_cg(a.host_dst0 + h);
+    }
+    if (status & ST_EMPTY_PLAN) {
+        for (int i = tid; i < n; i += nt) a.p.dst_pos[p0 + i] = -1;
+        return;
+    }
+    __syncthreads();
+    int remote = assign_pass_b(ids, cnt + warp * E, hptr, hstart, hdst, wbeg, wend, p0, E, R * C, C, a.fC, rank,
+                               a.p.dst_pos, nullptr, a.p.info);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) remote += __shfl_xor_sync(FULL_MASK, remote, o);
+    if (lane == 0) red[warp] = remote;
+    __syncthreads();
+    if (tid == 0) {
+        int s = 0;
+        for (int w = 0; w < (nt >> 5); ++w) s += red[w];
+        if (s) atomicAdd(a.p.info + MOONEP_INFO_N_REMOTE_PAIRS, s);
+    }
+}
+
+int launch_ep_count(const Dims &d, const int32_t *topk, int32_t *counts_row, void *ws, cudaStream_t st)
+{
+    const EpWsLayout wl = ws_layout_ep(d);
+    char *w = static_cast<char *>(ws);
+    EpCountParams a;
+    a.d = d;
+    a.topk = topk;
+    a.hdr = reinterpret_cast<int *>(w + wl.hdr);
+    a.cc = reinterpret_cast<int *>(w + wl.cc);
+    a.counts_row = counts_row;
+    const size_t smem = sizeof(int) * (size_t)(d.E + d.chunk_tokens * d.K);
+    if (!set_smem((const void *)ep_count_kernel, smem)) return MOONEP_ERR_CUDA;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t c = {};
+    c.gridDim = dim3(d.nchunk);
+    c.blockDim = dim3(PLAN_THREADS);
+    c.dynamicSmemBytes = smem;
+    c.stream = st;
+    c.attrs = attr;
+    c.numAttrs = 1;
+    return cudaLaunchKernelEx(&c, ep_count_kernel, a) == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
+}
+
+int launch_ep_plan(const Dims &d, int rank, const int32_t *topk, const int32_t *counts_all,
+                   const moonep_plan_t &p, void *ws, cudaStream_t st)
+{
+    const EpWsLayout wl = ws_layout_ep(d);
+    char *w = static_cast<char *>(ws);
+    PlanParams a;
+    a.d = d;
+    a.d.ngroups = d.R;  // the planner sums R count rows
+    a.topk = topk;
+    a.p = p;
+    a.hdr = reinterpret_cast<int *>(w + wl.hdr);
+    a.gs = const_cast<int *>(counts_all);
+    a.gs_stride = d.E + 1;
+    a.cc = reinterpret_cast<int *>(w + wl.cc);
+    a.host_dst0 = reinterpret_cast<int *>(w + wl.host_dst0);
+    a.fC = make_fastdiv((uint32_t)d.C);
+    a.fL = make_fastdiv((uint32_t)d.L);
+    a.spin_limit = 0;
+
+    const size_t smem1 = sizeof(int) * (size_t)(plan_smem_ints(d.E, d.R) +
+                                                ((d.flags & MOONEP_FLAG_CASCADE) ? cascade_smem_ints(d.E, d.R, d.B) : 0));
+    if (!set_smem((const void *)ep_plan_kernel, smem1)) return MOONEP_ERR_CUDA;
+    ep_plan_kernel<<<1, PLAN_THREADS, smem1, st>>>(a);
+    if (cudaGetLastError() != cudaSuccess) return MOONEP_ERR_CUDA;
+
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    const size_t smem2 = sizeof(int) * (size_t)assign_smem_ints(d.E, d.R, d.chunk_tokens * d.K);
+    if (!set_smem((const void *)ep_assign_kernel, smem2)) return MOONEP_ERR_CUDA;
+    cudaLaunchConfig_t c = {};
+    c.gridDim = dim3(d.nchunk);
+    c.blockDim = dim3(ASSIGN_THREADS);
+    c.dynamicSmemBytes = smem2;
+    c.stream = st;
+    c.attrs = attr;
+    c.numAttrs = 1;
+    return cudaLaunchKernelEx(&c, ep_assign_kernel, a, rank) == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
+}
+
+size_t ep_smem_bytes_max(const Dims &d)
+{
+    const size_t a = sizeof(int) * (size_t)(plan_smem_ints(d.E, d.R) +
+                                            ((d.flags & MOONEP_FLAG_CASCADE) ? cascade_smem_ints(d.E, d.R, d.B) : 0));
+    const size_t b = sizeof(int) * (size_t)assign_smem_ints(d.E, d.R, d.chunk_tokens * d.K);
+    const size_t c = sizeof(int) * (size_t)(d.E + d.chunk_tokens * d.K);
+    return a > b ? (a > c ? a : c) : (b > c ? b : c);
 }
 
 size_t plan_smem_bytes_max(const Dims &d)

@@ -9,18 +9,21 @@
 // pool[r][0..B), the home experts stay in `weights`, and a per-slot table
 // tells the expert computation which row to use.
 //
-// The copy is an HBM stream of 16-byte vectors over work items (prefetched
-// replica, element chunk) taken from the plan on the device, so the launch
-// needs no host synchronisation.
+// The copy is an HBM stream of 16-byte vectors over work items (expert with
+// prefetched replicas, element chunk) taken from the plan on the device, so
+// the launch needs no host synchronisation: each chunk of an expert's row is
+// read once and written to every one of its prefetched replicas, so the
+// bytes moved are the minimum, (experts with replicas + replicas) x row.
 #include "common.cuh"
 
 namespace moonep {
 
 constexpr int PF_THREADS = 256;
 constexpr int PF_UNROLL = 4;
+constexpr int PF_MAX_LIST = 2048;  // >= E + R - 1 >= prefetched replicas
 
 struct PrefetchParams {
-    const int *slot_expert, *rep_expert, *rep_rank, *rep_slot, *info;
+    moonep_plan_t p;
     const uint8_t *weights;
     uint8_t *pool;
     int *slot_wrow;
@@ -32,7 +35,11 @@ struct PrefetchParams {
 template <typename V>
 __global__ void __launch_bounds__(PF_THREADS) prefetch_kernel(PrefetchParams a)
 {
-    const int status = __ldg(a.info + MOONEP_INFO_STATUS);
+    __shared__ int s_e[MOONEP_MAX_E];
+    __shared__ int s_off[MOONEP_MAX_E + 1];
+    __shared__ int s_row[PF_MAX_LIST];
+    __shared__ int s_wsum[32];
+    const int status = __ldg(a.p.info + MOONEP_INFO_STATUS);
     const bool invalid = (status & ST_EMPTY_PLAN) != 0;
     const long long gtid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     const long long gstride = (long long)gridDim.x * blockDim.x;
@@ -40,28 +47,28 @@ __global__ void __launch_bounds__(PF_THREADS) prefetch_kernel(PrefetchParams a)
     // weight row of every slot: home e, pool E + r*B + b, overflow e (read-through)
     for (long long x = gtid; x < (long long)a.R * a.E; x += gstride) {
         const int r = (int)(x / a.E), s = (int)(x - (long long)r * a.E);
-        const int e = invalid ? -1 : __ldg(a.slot_expert + x);
+        const int e = invalid ? -1 : __ldg(a.p.slot_expert + x);
         int row = -1;
         if (e >= 0) row = (s < a.L) ? e : (s - a.L < a.B ? a.E + r * a.B + (s - a.L) : e);
         a.slot_wrow[x] = row;
     }
-    if (invalid) return;
+    // per block: every expert with prefetched replicas and their pool rows r*B + b
+    const int n_exp = replica_lists(a.p, a.E, a.L, a.B, a.R, [](int) { return true; }, s_e, s_off, s_row,
+                                    PF_MAX_LIST, s_wsum);
+    if (n_exp == 0) return;
 
-    const int n_rep = min(max(__ldg(a.info + MOONEP_INFO_N_REP), 0), a.E + a.R);
     constexpr int W = sizeof(V);
     const long long vrow = a.row_bytes / W;
     const long long vchunk = a.chunk / W;
     const long long nchunks = (vrow + vchunk - 1) / vchunk;
-    const long long n_items = (long long)n_rep * nchunks;
+    const long long n_items = (long long)n_exp * nchunks;
     for (long long item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const int q = (int)(item / nchunks);
-        const long long ci = item - (long long)q * nchunks;
-        const int b = __ldg(a.rep_slot + q) - a.L;
-        if (b < 0 || b >= a.B) continue;  // overflow: not prefetched
-        const int r = __ldg(a.rep_rank + q), e = __ldg(a.rep_expert + q);
-        if (r < 0 || r >= a.R || e < 0 || e >= a.E) continue;
+        const int ei = (int)(item / nchunks);
+        const long long ci = item - (long long)ei * nchunks;
+        const int e = s_e[ei];
+        if (e < 0 || e >= a.E) continue;
+        const int r0 = s_off[ei], n = min(s_off[ei + 1], PF_MAX_LIST) - r0;
         const V *src = reinterpret_cast<const V *>(a.weights + (long long)e * a.row_bytes);
-        V *dst = reinterpret_cast<V *>(a.pool + ((long long)r * a.B + b) * a.row_bytes);
         const long long v0 = ci * vchunk, v1 = min(vrow, v0 + vchunk);
         for (long long v = v0 + threadIdx.x; v < v1; v += (long long)PF_THREADS * PF_UNROLL) {
             V t[PF_UNROLL];
@@ -70,10 +77,13 @@ __global__ void __launch_bounds__(PF_THREADS) prefetch_kernel(PrefetchParams a)
                 const long long x = v + (long long)u * PF_THREADS;
                 if (x < v1) t[u] = src[x];
             }
+            for (int m = 0; m < n; ++m) {
+                V *dst = reinterpret_cast<V *>(a.pool + (long long)s_row[r0 + m] * a.row_bytes);
 #pragma unroll
-            for (int u = 0; u < PF_UNROLL; ++u) {
-                const long long x = v + (long long)u * PF_THREADS;
-                if (x < v1) dst[x] = t[u];
+                for (int u = 0; u < PF_UNROLL; ++u) {
+                    const long long x = v + (long long)u * PF_THREADS;
+                    if (x < v1) dst[x] = t[u];
+                }
             }
         }
     }
@@ -92,11 +102,7 @@ int launch_prefetch(const Dims &d, const moonep_plan_t &p, const uint16_t *weigh
         sms[dev] = v > 0 ? v : 148;
     }
     PrefetchParams a;
-    a.slot_expert = p.slot_expert;
-    a.rep_expert = p.rep_expert;
-    a.rep_rank = p.rep_rank;
-    a.rep_slot = p.rep_slot;
-    a.info = p.info;
+    a.p = p;
     a.weights = reinterpret_cast<const uint8_t *>(weights);
     a.pool = reinterpret_cast<uint8_t *>(pool);
     a.slot_wrow = slot_wrow;

@@ -21,12 +21,56 @@ constexpr int REDUCE_GROUP = 4;
 constexpr int REDUCE_MAX_LIST = 2048;  // >= E + R - 1 >= prefetched replicas
 
 struct ReduceParams {
-    float *reduce_buf;
-    float *home_grad;
-    const int *host_ptr, *host_rank, *host_slot, *rep_home_list, *info;
+    moonep_plan_t p;
+    int *status;        // the plan's status word (for MOONEP_ST_ROW_RANGE)
     int L, B, E, R, n_hosts;
     long long P;        // elements per gradient row
     long long chunk;    // vectors per work item
+};
+
+// Where the gradient rows live.  The replica row of slot b of rank r is
+// reduce-buffer row r * B + b.
+// One GPU: reduce_buf [R, B, P] and home_grad [E, P], every expert reduced.
+struct FlatGrads {
+    static constexpr bool may_skip = false;  // rep() never returns null
+    float *reduce_buf, *home_grad;
+    __device__ __forceinline__ bool takes(int e) const { return true; }
+    template <typename V>
+    __device__ __forceinline__ V *home(int e, long long PV) const
+    {
+        return reinterpret_cast<V *>(home_grad) + (long long)e * PV;
+    }
+    template <typename V>
+    __device__ __forceinline__ V *rep(int row, long long PV) const
+    {
+        return reinterpret_cast<V *>(reduce_buf) + (long long)row * PV;
+    }
+};
+
+// Expert parallelism, on home rank `rank`: its own experts only, home_grad
+// [L, P] local, each rank's reduce buffer [B, P] reached through a device
+// array of R pointers (peer memory).  A null or misaligned pointer is
+// reported (MOONEP_ST_ROW_RANGE) and its rows are skipped.
+struct RankGrads {
+    static constexpr bool may_skip = true;
+    float *const *reduce_bufs;
+    float *home_grad;
+    int rank, L, B;
+    FastDiv fB;
+    __device__ __forceinline__ bool takes(int e) const { return e / L == rank; }
+    template <typename V>
+    __device__ __forceinline__ V *home(int e, long long PV) const
+    {
+        return reinterpret_cast<V *>(home_grad) + (long long)(e - rank * L) * PV;
+    }
+    template <typename V>
+    __device__ __forceinline__ V *rep(int row, long long PV) const
+    {
+        const int r = (int)fdiv((uint32_t)row, fB);
+        float *b = reduce_bufs[r];
+        if (b == nullptr || (reinterpret_cast<uintptr_t>(b) & (sizeof(V) - 1))) return nullptr;
+        return reinterpret_cast<V *>(b) + (long long)(row - r * B) * PV;
+    }
 };
 
 template <typename V>
@@ -48,8 +92,8 @@ __device__ __forceinline__ float4 vzero<float4>() { return make_float4(0.f, 0.f,
 template <>
 __device__ __forceinline__ float vzero<float>() { return 0.f; }
 
-template <typename V>
-__global__ void __launch_bounds__(REDUCE_THREADS) reduce_kernel(ReduceParams a)
+template <typename V, typename G>
+__global__ void __launch_bounds__(REDUCE_THREADS) reduce_kernel(ReduceParams a, G gr)
 {
     // Per block, once: for every expert with prefetched replicas, the list
     // of its reduce_buf rows (r*B + b) in ascending host rank order.
@@ -57,49 +101,15 @@ __global__ void __launch_bounds__(REDUCE_THREADS) reduce_kernel(ReduceParams a)
     __shared__ int s_off[MOONEP_MAX_E + 1];
     __shared__ int s_row[REDUCE_MAX_LIST];
     __shared__ int s_wsum[32];
-    const int status = __ldg(a.info + MOONEP_INFO_STATUS);
-    if (status & ST_EMPTY_PLAN) return;
-    const int n_exp = min(max(__ldg(a.info + MOONEP_INFO_N_REP_EXPERTS), 0), a.E);
-    if (n_exp == 0) return;
     const int tid = threadIdx.x;
-    for (int i = tid; i <= n_exp; i += blockDim.x) {
-        int c = 0, e = -1;
-        if (i < n_exp) {
-            e = __ldg(a.rep_home_list + i);
-            if (e >= 0 && e < a.E) {
-                const int home = e / a.L;
-                const int h0 = max(0, __ldg(a.host_ptr + e)), h1 = min(a.n_hosts, __ldg(a.host_ptr + e + 1));
-                for (int h = h0; h < h1; ++h) {
-                    const int r = __ldg(a.host_rank + h), b = __ldg(a.host_slot + h) - a.L;
-                    c += (r != home && r >= 0 && r < a.R && b >= 0 && b < a.B);
-                }
-            }
-        }
-        if (i < n_exp) s_e[i] = e;
-        s_off[i] = c;
-    }
-    __syncthreads();
-    block_exscan(s_off, n_exp + 1, s_wsum);
-    for (int i = tid; i < n_exp; i += blockDim.x) {
-        const int e = s_e[i];
-        if (e < 0 || e >= a.E) continue;
-        const int home = e / a.L;
-        int o = s_off[i];
-        const int h0 = max(0, __ldg(a.host_ptr + e)), h1 = min(a.n_hosts, __ldg(a.host_ptr + e + 1));
-        for (int h = h0; h < h1; ++h) {
-            const int r = __ldg(a.host_rank + h), b = __ldg(a.host_slot + h) - a.L;
-            if (r != home && r >= 0 && r < a.R && b >= 0 && b < a.B && o < REDUCE_MAX_LIST)
-                s_row[o++] = r * a.B + b;
-        }
-    }
-    __syncthreads();
+    const int n_exp = replica_lists(a.p, a.E, a.L, a.B, a.R, [&](int e) { return gr.takes(e); }, s_e, s_off, s_row,
+                                    REDUCE_MAX_LIST, s_wsum);
+    if (n_exp == 0) return;
 
     constexpr int W = sizeof(V) / sizeof(float);
     const long long PV = a.P / W;  // vectors per row
     const long long nchunks = (PV + a.chunk - 1) / a.chunk;
     const long long n_items = (long long)n_exp * nchunks;
-    V *rb = reinterpret_cast<V *>(a.reduce_buf);
-    V *hg = reinterpret_cast<V *>(a.home_grad);
 
     // Phase 1: sums into home_grad.  Phase 2: zero the replica rows of the
     // same items.  Interleaving the zero stores with the summing loads per
@@ -112,7 +122,7 @@ __global__ void __launch_bounds__(REDUCE_THREADS) reduce_kernel(ReduceParams a)
         const int e = s_e[ei];
         if (e < 0 || e >= a.E) continue;
         const int r0 = s_off[ei], n = min(s_off[ei + 1], REDUCE_MAX_LIST) - r0;
-        V *home_row = hg + (long long)e * PV;
+        V *home_row = gr.template home<V>(e, PV);
         const long long v0 = ci * a.chunk;
         const long long v1 = min(PV, v0 + a.chunk);
         for (long long v = v0 + tid; v < v1; v += (long long)REDUCE_THREADS * REDUCE_UNROLL) {
@@ -126,13 +136,15 @@ __global__ void __launch_bounds__(REDUCE_THREADS) reduce_kernel(ReduceParams a)
             // flight before the adds, which keep ascending host rank order
             for (int m0 = 0; m0 < n; m0 += REDUCE_GROUP) {
                 V r[REDUCE_GROUP][REDUCE_UNROLL];
+                bool live[REDUCE_GROUP];
 #pragma unroll
                 for (int m = 0; m < REDUCE_GROUP; ++m) {
-                    const V *rrow = rb + (long long)s_row[r0 + min(m0 + m, n - 1)] * PV;
+                    const V *rrow = gr.template rep<V>(s_row[r0 + min(m0 + m, n - 1)], PV);
+                    live[m] = m0 + m < n && (!G::may_skip || rrow != nullptr);
 #pragma unroll
                     for (int u = 0; u < REDUCE_UNROLL; ++u) {
                         const long long x = v + (long long)u * REDUCE_THREADS;
-                        if (m0 + m < n && x < v1) r[m][u] = rrow[x];
+                        if (live[m] && x < v1) r[m][u] = rrow[x];
                     }
                 }
 #pragma unroll
@@ -140,7 +152,7 @@ __global__ void __launch_bounds__(REDUCE_THREADS) reduce_kernel(ReduceParams a)
 #pragma unroll
                     for (int u = 0; u < REDUCE_UNROLL; ++u) {
                         const long long x = v + (long long)u * REDUCE_THREADS;
-                        if (m0 + m < n && x < v1) acc[u] = vadd(acc[u], r[m][u]);
+                        if (live[m] && x < v1) acc[u] = vadd(acc[u], r[m][u]);
                     }
             }
 #pragma unroll
@@ -159,7 +171,11 @@ __global__ void __launch_bounds__(REDUCE_THREADS) reduce_kernel(ReduceParams a)
         const long long v0 = ci * a.chunk;
         const long long v1 = min(PV, v0 + a.chunk);
         for (int m = 0; m < n; ++m) {
-            V *rrow = rb + (long long)s_row[r0 + m] * PV;
+            V *rrow = gr.template rep<V>(s_row[r0 + m], PV);
+            if (G::may_skip && rrow == nullptr) {
+                if (tid == 0 && ci == 0) atomicOr(a.status, MOONEP_ST_ROW_RANGE);
+                continue;
+            }
             for (long long v = v0 + tid; v < v1; v += (long long)REDUCE_THREADS * REDUCE_UNROLL) {
 #pragma unroll
                 for (int u = 0; u < REDUCE_UNROLL; ++u) {
@@ -171,8 +187,7 @@ __global__ void __launch_bounds__(REDUCE_THREADS) reduce_kernel(ReduceParams a)
     }
 }
 
-int launch_reduce(const Dims &d, const moonep_plan_t &p, float *reduce_buf, float *home_grad, long long P,
-                  cudaStream_t st)
+static int device_sms()
 {
     static int sms[64] = {0};
     int dev = 0;
@@ -183,33 +198,51 @@ int launch_reduce(const Dims &d, const moonep_plan_t &p, float *reduce_buf, floa
         cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
         sms[dev] = v > 0 ? v : 148;
     }
+    return sms[dev];
+}
+
+template <typename G>
+static int reduce_with(const Dims &d, const moonep_plan_t &p, const G &gr, bool vec, long long P, cudaStream_t st)
+{
     ReduceParams a;
-    a.reduce_buf = reduce_buf;
-    a.home_grad = home_grad;
-    a.host_ptr = p.host_ptr;
-    a.host_rank = p.host_rank;
-    a.host_slot = p.host_slot;
-    a.rep_home_list = p.rep_home_list;
-    a.info = p.info;
+    a.p = p;
+    a.status = p.info + MOONEP_INFO_STATUS;
     a.L = d.L;
     a.B = d.B;
     a.E = d.E;
     a.R = d.R;
     a.n_hosts = 2 * d.E + d.R;
     a.P = P;
-    const bool vec = (P % 4 == 0) && (reinterpret_cast<uintptr_t>(reduce_buf) % 16 == 0) &&
-                     (reinterpret_cast<uintptr_t>(home_grad) % 16 == 0);
     // eight waves of blocks: the block scheduler refills SMs as blocks
     // finish, which evens out the tail of the item loop (4 % over one wave)
-    const int grid = sms[dev] * (2048 / REDUCE_THREADS) * 8;
+    const int grid = device_sms() * (2048 / REDUCE_THREADS) * 8;
     if (vec) {
         a.chunk = (long long)REDUCE_THREADS * REDUCE_UNROLL * 8;
-        reduce_kernel<float4><<<grid, REDUCE_THREADS, 0, st>>>(a);
+        reduce_kernel<float4, G><<<grid, REDUCE_THREADS, 0, st>>>(a, gr);
     } else {
         a.chunk = (long long)REDUCE_THREADS * REDUCE_UNROLL * 32;
-        reduce_kernel<float><<<grid, REDUCE_THREADS, 0, st>>>(a);
+        reduce_kernel<float, G><<<grid, REDUCE_THREADS, 0, st>>>(a, gr);
     }
     return cudaGetLastError() == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
+}
+
+int launch_reduce(const Dims &d, const moonep_plan_t &p, float *reduce_buf, float *home_grad, long long P,
+                  cudaStream_t st)
+{
+    const bool vec = (P % 4 == 0) && (reinterpret_cast<uintptr_t>(reduce_buf) % 16 == 0) &&
+                     (reinterpret_cast<uintptr_t>(home_grad) % 16 == 0);
+    return reduce_with(d, p, FlatGrads{reduce_buf, home_grad}, vec, P, st);
+}
+
+// Expert parallelism: home rank `rank` pulls its experts' replica rows from
+// every rank's reduce buffer (reduce_bufs: device array of R pointers, each
+// 16-byte aligned for the vector path) into its local home_grad [L, P].
+int launch_reduce_ep(const Dims &d, int rank, const moonep_plan_t &p, float *const *reduce_bufs,
+                     float *home_grad, long long P, cudaStream_t st)
+{
+    const bool vec = (P % 4 == 0) && (reinterpret_cast<uintptr_t>(home_grad) % 16 == 0);
+    RankGrads gr{reduce_bufs, home_grad, rank, d.L, d.B, make_fastdiv((uint32_t)d.B)};
+    return reduce_with(d, p, gr, vec, P, st);
 }
 
 }  // namespace moonep

@@ -55,7 +55,9 @@ EXPORTED = ("moonep_check_config", "moonep_plan_sizes", "moonep_plan_layout", "m
             "moonep_dispatch", "moonep_combine", "moonep_combine_backward",
             "moonep_reduce_replica_grads", "moonep_error_string", "moonep_abi_version",
             "moonep_plan_noalloc", "moonep_prefetch_replicas", "moonep_status_string",
-            "moonep_set_wait_limit")
+            "moonep_set_wait_limit", "moonep_ep_sizes", "moonep_ep_count", "moonep_ep_plan",
+            "moonep_ep_dispatch", "moonep_ep_combine", "moonep_ep_combine_backward",
+            "moonep_ep_reduce_replica_grads")
 
 
 class _CConfig(ctypes.Structure):
@@ -87,6 +89,13 @@ _lib.moonep_status_string.argtypes = [ctypes.c_int, ctypes.c_char_p, ctypes.c_si
 _lib.moonep_status_string.restype = ctypes.c_char_p
 _lib.moonep_abi_version.argtypes = []
 _lib.moonep_set_wait_limit.argtypes = [ctypes.c_int]
+_lib.moonep_ep_sizes.argtypes = [_cfgp, ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)]
+_lib.moonep_ep_count.argtypes = [_cfgp, _vp, _vp, _vp, _vp]
+_lib.moonep_ep_plan.argtypes = [_cfgp, ctypes.c_int32, _vp, _vp, _planp, _vp, _vp]
+_lib.moonep_ep_dispatch.argtypes = [_cfgp, _planp, _vp, _vp, _vp]
+_lib.moonep_ep_combine.argtypes = [_cfgp, _planp, _vp, _vp, _vp, _vp]
+_lib.moonep_ep_combine_backward.argtypes = [_cfgp, _planp, _vp, _vp, _vp, _vp, _vp, _vp]
+_lib.moonep_ep_reduce_replica_grads.argtypes = [_cfgp, ctypes.c_int32, _planp, _vp, _vp, ctypes.c_int64, _vp]
 for _f in EXPORTED:
     if _f not in ("moonep_error_string", "moonep_status_string"):
         getattr(_lib, _f).restype = ctypes.c_int
@@ -154,14 +163,24 @@ def plan_sizes(cfg: Config):
     return pb.value, wb.value
 
 
+def ep_sizes(cfg: Config):
+    """(plan bytes, workspace bytes) of one rank in expert parallelism."""
+    c = cfg.c()
+    pb, wb = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    _check(_lib.moonep_ep_sizes(ctypes.byref(c), ctypes.byref(pb), ctypes.byref(wb)))
+    return pb.value, wb.value
+
+
 class Plan:
     """Device plan block plus the planner workspace, with int32 views of
-    every field (shapes as in moonep.h)."""
+    every field (shapes as in moonep.h).  ep=True sizes the workspace for
+    one rank of expert parallelism (moonep_ep_count / moonep_ep_plan)."""
 
-    def __init__(self, cfg: Config, device=None):
+    def __init__(self, cfg: Config, device=None, ep: bool = False):
         device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
         self.cfg = cfg
-        pb, wb = plan_sizes(cfg)
+        self.ep = ep
+        pb, wb = ep_sizes(cfg) if ep else plan_sizes(cfg)
         self.block = torch.zeros(pb, dtype=torch.uint8, device=device)
         # zero-filled once; every plan call leaves it ready for the next call
         # with this configuration
@@ -198,6 +217,13 @@ class Plan:
         """Status and statistics (synchronises with the device)."""
         v = self.fields["info"].cpu().tolist()
         return {k: v[i] for i, k in enumerate(INFO_FIELDS)}
+
+    @property
+    def dst_pos_local(self) -> torch.Tensor:
+        """Expert parallelism: the global buffer rows of this rank's own
+        pairs [S, K] (the first S*K entries of dst_pos)."""
+        c = self.cfg
+        return self.fields["dst_pos"].view(-1)[: c.S * c.K].view(c.S, c.K)
 
     def to_numpy(self) -> dict:
         return {k: v.cpu().numpy() for k, v in self.fields.items()}
@@ -327,6 +353,116 @@ def prefetch_replicas(cfg: Config, p: Plan, weights: torch.Tensor, pool: torch.T
                                          pool.data_ptr() if pool.numel() else None, slot_wrow.data_ptr(),
                                          P, _stream(stream)))
     return slot_wrow
+
+
+# ------------------------------------------------- expert parallelism
+
+def pointer_array(tensors, device=None) -> torch.Tensor:
+    """A device int64 array of the tensors' data pointers (index = rank): the
+    form in which the expert-parallel calls take the R ranks' buffers.  The
+    tensors may live in other GPUs' memory mapped into this process (peer
+    memory) or, on one GPU, be R separate allocations."""
+    dev = device if device is not None else tensors[0].device
+    return torch.tensor([t.data_ptr() if t is not None else 0 for t in tensors], dtype=torch.int64, device=dev)
+
+
+def ep_count(cfg: Config, topk_local: torch.Tensor, p: Plan, counts_row: torch.Tensor | None = None,
+             stream=None) -> torch.Tensor:
+    """This rank's counts row [E + 1] int32 (pairs per expert, then invalid ids)."""
+    _need(topk_local, torch.int32, (cfg.S, cfg.K), "topk_local")
+    if counts_row is None:
+        counts_row = torch.empty(cfg.E + 1, dtype=torch.int32, device=topk_local.device)
+    _need(counts_row, torch.int32, (cfg.E + 1,), "counts_row")
+    c = cfg.c()
+    _check(_lib.moonep_ep_count(ctypes.byref(c), topk_local.data_ptr(), counts_row.data_ptr(),
+                                p.workspace.data_ptr(), _stream(stream)))
+    return counts_row
+
+
+def ep_gather_counts(counts_row: torch.Tensor, group=None) -> torch.Tensor:
+    """All-gather every rank's counts row into [R, E + 1] (row r from rank r)
+    with torch.distributed: 4 (E + 1) bytes per rank, the one collective of
+    an expert-parallel layer's plan."""
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    n = counts_row.numel()
+    out = torch.empty(world * n, dtype=counts_row.dtype, device=counts_row.device)
+    dist.all_gather_into_tensor(out, counts_row.contiguous().view(-1), group=group)
+    return out.view(world, n)
+
+
+def ep_plan(cfg: Config, rank: int, topk_local: torch.Tensor, counts_all: torch.Tensor, p: Plan,
+            stream=None) -> Plan:
+    """Every rank's identical plan tables from the gathered counts, and the
+    global rows of this rank's own pairs (p.dst_pos_local)."""
+    _need(topk_local, torch.int32, (cfg.S, cfg.K), "topk_local")
+    _need(counts_all, torch.int32, (cfg.R, cfg.E + 1), "counts_all")
+    c = cfg.c()
+    _check(_lib.moonep_ep_plan(ctypes.byref(c), int(rank), topk_local.data_ptr(), counts_all.data_ptr(),
+                               ctypes.byref(p.c_plan), p.workspace.data_ptr(), _stream(stream)))
+    return p
+
+
+def _need_ptrs(t: torch.Tensor, cfg: Config, name: str):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.int64 or t.numel() != cfg.R:
+        raise ValueError(f"{name} must be a CUDA int64 tensor of {cfg.R} pointers (see pointer_array)")
+
+
+def ep_dispatch(cfg: Config, p: Plan, hidden_local: torch.Tensor, buf_ptrs: torch.Tensor, stream=None):
+    """Write this rank's token rows into every rank's [S*K, H] buffer."""
+    _need(hidden_local, torch.bfloat16, (cfg.S, cfg.H), "hidden_local")
+    _need_ptrs(buf_ptrs, cfg, "buf_ptrs")
+    c = cfg.c()
+    _check(_lib.moonep_ep_dispatch(ctypes.byref(c), ctypes.byref(p.c_plan), hidden_local.data_ptr(),
+                                   buf_ptrs.data_ptr(), _stream(stream)))
+
+
+def ep_combine(cfg: Config, p: Plan, y_ptrs: torch.Tensor, w_local: torch.Tensor,
+               out_local: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """This rank's tokens' weighted sum of their K expert-output rows, read
+    from every rank's buffer."""
+    _need_ptrs(y_ptrs, cfg, "y_ptrs")
+    _need(w_local, torch.float32, (cfg.S, cfg.K), "w_local")
+    if out_local is None:
+        out_local = torch.empty((cfg.S, cfg.H), dtype=torch.bfloat16, device=w_local.device)
+    _need(out_local, torch.bfloat16, (cfg.S, cfg.H), "out_local")
+    c = cfg.c()
+    _check(_lib.moonep_ep_combine(ctypes.byref(c), ctypes.byref(p.c_plan), y_ptrs.data_ptr(), w_local.data_ptr(),
+                                  out_local.data_ptr(), _stream(stream)))
+    return out_local
+
+
+def ep_combine_backward(cfg: Config, p: Plan, dy_local: torch.Tensor, w_local: torch.Tensor,
+                        y_ptrs: torch.Tensor, dy_buf_ptrs: torch.Tensor, dw_local: torch.Tensor | None = None,
+                        stream=None) -> torch.Tensor:
+    """Backward of ep_combine: scaled dy rows into every rank's dy buffer,
+    and this rank's dw [S, K]."""
+    _need(dy_local, torch.bfloat16, (cfg.S, cfg.H), "dy_local")
+    _need(w_local, torch.float32, (cfg.S, cfg.K), "w_local")
+    _need_ptrs(y_ptrs, cfg, "y_ptrs")
+    _need_ptrs(dy_buf_ptrs, cfg, "dy_buf_ptrs")
+    if dw_local is None:
+        dw_local = torch.empty((cfg.S, cfg.K), dtype=torch.float32, device=dy_local.device)
+    _need(dw_local, torch.float32, (cfg.S, cfg.K), "dw_local")
+    c = cfg.c()
+    _check(_lib.moonep_ep_combine_backward(ctypes.byref(c), ctypes.byref(p.c_plan), dy_local.data_ptr(),
+                                           w_local.data_ptr(), y_ptrs.data_ptr(), dy_buf_ptrs.data_ptr(),
+                                           dw_local.data_ptr(), _stream(stream)))
+    return dw_local
+
+
+def ep_reduce_replica_grads(cfg: Config, rank: int, p: Plan, reduce_buf_ptrs: torch.Tensor,
+                            home_grad_local: torch.Tensor, stream=None) -> torch.Tensor:
+    """On home rank `rank`: pull its experts' replica gradient rows from every
+    rank's [B, P] reduce buffer into home_grad_local [L, P], zeroing them."""
+    P = home_grad_local.shape[-1]
+    _need(home_grad_local, torch.float32, (cfg.L, P), "home_grad_local")
+    _need_ptrs(reduce_buf_ptrs, cfg, "reduce_buf_ptrs")
+    c = cfg.c()
+    _check(_lib.moonep_ep_reduce_replica_grads(ctypes.byref(c), int(rank), ctypes.byref(p.c_plan),
+                                               reduce_buf_ptrs.data_ptr(), home_grad_local.data_ptr(), P,
+                                               _stream(stream)))
+    return home_grad_local
 
 
 def views(cfg: Config, p: Plan, buf: torch.Tensor):

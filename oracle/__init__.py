@@ -56,10 +56,11 @@ class OracleError(RuntimeError):
     pass
 
 
-def build(force: bool = False) -> str:
-    """Compile the oracle with gcc (plain C11, -O2, no fast-math), and the
-    same source with OpenMP for the timed multi-core CPU baseline."""
-    for lib, extra in ((_LIB, []), (_LIB_OMP, ["-fopenmp"])):
+def build(force: bool = False, openmp: bool = True) -> str:
+    """Compile the oracle with gcc (plain C11, -O2, no fast-math), and (with
+    openmp) the same source with OpenMP for the timed multi-core CPU
+    baseline."""
+    for lib, extra in ((_LIB, []), (_LIB_OMP, ["-fopenmp"]))[: 2 if openmp else 1]:
         if force or not os.path.exists(lib) or os.path.getmtime(lib) < os.path.getmtime(_SRC):
             cmd = ["gcc", "-std=c11", "-O2", "-fno-fast-math", "-ffp-contract=off", *extra,
                    "-fPIC", "-shared", "-o", lib, _SRC, "-lm"]

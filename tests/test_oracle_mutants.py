@@ -205,7 +205,8 @@ CORE_MUTANTS = {
           "        for (int32_t h = host_ptr[e + 1] - 1; h >= host_ptr[e]; --h) {\n            int32_t r = host_rank[h], b = host_slot[h] - L;\n"
           "            if (r == e / L) continue; /* the home copy */")], [("test_reduce_order_is_rank_ascending", {})]),
     "reduce leaves the replica rows": (
-        [("            for (int64_t i = i0; i < i1; ++i) src[i] = 0.0f;", "")], [("test_reduce_exact_integers", {})]),
+        [("#pragma omp parallel for schedule(static)\n            for (int64_t i = i0; i < i1; ++i) src[i] = 0.0f;", "")],
+        [("test_reduce_exact_integers", {})]),
     "reduce includes overflow replicas": (
         [("            if (b < 0 || b >= B) continue; /* overflow replica: no reduce rows */", "            if (b < 0) continue;")],
         [("test_reduce_exact_integers", {})]),
@@ -294,7 +295,7 @@ def _load_mutant(tmp, tag, edits):
     mod = importlib.util.module_from_spec(spec)
     sys.modules[name] = mod
     spec.loader.exec_module(mod)
-    mod.build(force=True)
+    mod.build(force=True, openmp=False)
     return mod
 
 

@@ -902,24 +902,9 @@ __device__ void plan_block(const PlanParams &a, int *sm, int seq)
     const int n_hosts = E + n_rep;                  // == Z[zh + E] - zh0
     const int n_rep_experts = Z[zf + E] - zf0;
     auto hptr = [&](int e) { return Z[zh + e] - zh0; };
-    // one pass writes the used slots into the padded [R][E] tables, the host
-    // pointers, the reduce work list and (below) the host intervals: x runs
-    // over max(E + n_rep, E + 1) = n_hosts + (n_rep == 0) entries
-    for (int x = tid; x <= n_hosts; x += nt) {
-        if (x < E + n_rep) {
-            const int r = cspare[x], b0 = rank_base(r), sl = x - b0;
-            a.p.slot_expert[(size_t)r * E + sl] = cexp[x];
-            a.p.slot_count[(size_t)r * E + sl] = ccnt[x];
-            a.p.slot_offset[(size_t)r * (E + 1) + sl] = Z[x] - Z[b0];
-        }
-        if (x <= E) a.p.host_ptr[x] = hptr(x);
-        if (x < E) {
-            if (flag[x]) a.p.rep_home_list[Z[zf + x] - zf0] = x;
-            if (x >= n_rep_experts) a.p.rep_home_list[x] = -1;
-        }
-    }
-    // ---- host intervals: the hosts of e in ascending rank; a host's start
-    // is the rows of the hosts of e on lower ranks
+    // ---- host intervals first: they are all the assignment CTAs wait for.
+    // The hosts of e in ascending rank; a host's start is the rows of the
+    // hosts of e on lower ranks.
     for (int x = tid; x < n_hosts; x += nt) {
         int e, r0, slot, quota, j, pos = 0, st = 0;
         if (x < E) {
@@ -959,6 +944,7 @@ __device__ void plan_block(const PlanParams &a, int *sm, int seq)
         a.p.host_start[h] = st;
         a.host_dst0[h] = r0 * C + Z[b0 + slot] - Z[b0] - st;
     }
+    for (int x = tid; x <= E; x += nt) a.p.host_ptr[x] = hptr(x);
 
     if (tid == 0) {
         const int n_over = misc[2];
@@ -976,11 +962,24 @@ __device__ void plan_block(const PlanParams &a, int *sm, int seq)
         a.p.info[MOONEP_INFO_N_REP_EXPERTS] = n_rep_experts;
         for (int i = MOONEP_INFO_N_REMOTE_PAIRS; i < MOONEP_INFO_LEN; ++i) a.p.info[i] = 0;
     }
-    // every thread's plan writes precede the plan-ready mark
+    // the host tables and the status precede the plan-ready mark
     __syncthreads();
     if (tid == 0) {
         __threadfence();
         st_release(a.hdr + WS_PLANNED, seq + 1);
+    }
+    // ---- then, while the assignment CTAs place the pairs, the used slots of
+    // the padded [R][E] tables and the reduce work list (read only by later
+    // kernels, which start after this grid has finished)
+    for (int x = tid; x < E + n_rep; x += nt) {
+        const int r = cspare[x], b0 = rank_base(r), sl = x - b0;
+        a.p.slot_expert[(size_t)r * E + sl] = cexp[x];
+        a.p.slot_count[(size_t)r * E + sl] = ccnt[x];
+        a.p.slot_offset[(size_t)r * (E + 1) + sl] = Z[x] - Z[b0];
+    }
+    for (int x = tid; x < E; x += nt) {
+        if (flag[x]) a.p.rep_home_list[Z[zf + x] - zf0] = x;
+        if (x >= n_rep_experts) a.p.rep_home_list[x] = -1;
     }
 }
 
@@ -1314,6 +1313,7 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
             a.p.dst_pos[p0 + i] = -1;
             a.p.row_src[p0 + i] = -1;
         }
+        pdl_wait();  // as below: finish after the histogram grid
         return;
     }
     __syncthreads();
@@ -1331,6 +1331,10 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
         for (int w = 0; w < (nt >> 5); ++w) s += red[w];
         if (s) atomicAdd(a.p.info + MOONEP_INFO_N_REMOTE_PAIRS, s);
     }
+    // this grid finishes only after the histogram grid: the planner CTA
+    // writes its last tables after the plan-ready mark, and a kernel that
+    // follows the plan in the stream must see them
+    pdl_wait();
 }
 
 // ---------------------------------------------------------------- launch
@@ -1338,11 +1342,29 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
 // Both planner kernels ask for the largest shared-memory carveout: an SM
 // that runs histogram CTAs must also fit two assignment CTAs as the
 // histogram CTAs retire (the carveout changes only when an SM is idle).
-static bool set_smem(const void *fn, size_t bytes)
+// The attributes are set once per device and kernel, and again only when a
+// launch needs more dynamic shared memory than was allowed so far: the
+// driver calls cost host time on every plan of a latency-bound layer.
+constexpr int SMEM_CACHE_DEVICES = 64;
+enum { K_HIST, K_ASSIGN, K_EP_COUNT, K_EP_PLAN, K_EP_ASSIGN, K_N };
+static std::atomic<size_t> g_smem_set[SMEM_CACHE_DEVICES][K_N];  // bytes allowed so far, 0 = never set
+
+static bool set_smem(int which, const void *fn, size_t bytes)
 {
-    return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess &&
-           cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                (int)cudaSharedmemCarveoutMaxShared) == cudaSuccess;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    std::atomic<size_t> *slot = (dev >= 0 && dev < SMEM_CACHE_DEVICES) ? &g_smem_set[dev][which] : nullptr;
+    if (slot && slot->load(std::memory_order_relaxed) >= bytes && bytes > 0) return true;
+    const bool ok =
+        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess &&
+        cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared) == cudaSuccess;
+    if (ok && slot) {
+        size_t cur = slot->load(std::memory_order_relaxed);
+        while (cur < bytes && !slot->compare_exchange_weak(cur, bytes, std::memory_order_relaxed)) {
+        }
+    }
+    return ok;
 }
 
 int launch_plan(const Dims &d, const int32_t *topk, const moonep_plan_t &p, void *ws, cudaStream_t st)
@@ -1370,7 +1392,7 @@ int launch_plan(const Dims &d, const int32_t *topk, const moonep_plan_t &p, void
     attr[0].val.programmaticStreamSerializationAllowed = 1;
 
     const size_t smem1 = sizeof(int) * (size_t)hist_smem_ints(d.E, d.R, d.chunk_tokens * d.K, d.flags, d.B);
-    if (!set_smem((const void *)hist_plan_kernel, smem1)) return MOONEP_ERR_CUDA;
+    if (!set_smem(K_HIST, (const void *)hist_plan_kernel, smem1)) return MOONEP_ERR_CUDA;
     cudaLaunchConfig_t c1 = {};
     c1.gridDim = dim3(d.nchunk);
     c1.blockDim = dim3(PLAN_THREADS);
@@ -1381,7 +1403,7 @@ int launch_plan(const Dims &d, const int32_t *topk, const moonep_plan_t &p, void
     if (cudaLaunchKernelEx(&c1, hist_plan_kernel, a) != cudaSuccess) return MOONEP_ERR_CUDA;
 
     const size_t smem2 = sizeof(int) * (size_t)assign_smem_ints(d.E, d.R, d.chunk_tokens * d.K);
-    if (!set_smem((const void *)assign_kernel, smem2)) return MOONEP_ERR_CUDA;
+    if (!set_smem(K_ASSIGN, (const void *)assign_kernel, smem2)) return MOONEP_ERR_CUDA;
     cudaLaunchConfig_t c2 = c1;
     c2.blockDim = dim3(ASSIGN_THREADS);
     c2.dynamicSmemBytes = smem2;
@@ -1582,7 +1604,7 @@ int launch_ep_count(const Dims &d, const int32_t *topk, int32_t *counts_row, voi
     a.cc = reinterpret_cast<int *>(w + wl.cc);
     a.counts_row = counts_row;
     const size_t smem = sizeof(int) * (size_t)(d.E + d.chunk_tokens * d.K);
-    if (!set_smem((const void *)ep_count_kernel, smem)) return MOONEP_ERR_CUDA;
+    if (!set_smem(K_EP_COUNT, (const void *)ep_count_kernel, smem)) return MOONEP_ERR_CUDA;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -1617,7 +1639,7 @@ int launch_ep_plan(const Dims &d, int rank, const int32_t *topk, const int32_t *
 
     const size_t smem1 = sizeof(int) * (size_t)(plan_smem_ints(d.E, d.R) +
                                                 ((d.flags & MOONEP_FLAG_CASCADE) ? cascade_smem_ints(d.E, d.R, d.B) : 0));
-    if (!set_smem((const void *)ep_plan_kernel, smem1)) return MOONEP_ERR_CUDA;
+    if (!set_smem(K_EP_PLAN, (const void *)ep_plan_kernel, smem1)) return MOONEP_ERR_CUDA;
     ep_plan_kernel<<<1, PLAN_THREADS, smem1, st>>>(a);
     if (cudaGetLastError() != cudaSuccess) return MOONEP_ERR_CUDA;
 
@@ -1625,7 +1647,7 @@ int launch_ep_plan(const Dims &d, int rank, const int32_t *topk, const int32_t *
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     const size_t smem2 = sizeof(int) * (size_t)assign_smem_ints(d.E, d.R, d.chunk_tokens * d.K);
-    if (!set_smem((const void *)ep_assign_kernel, smem2)) return MOONEP_ERR_CUDA;
+    if (!set_smem(K_EP_ASSIGN, (const void *)ep_assign_kernel, smem2)) return MOONEP_ERR_CUDA;
     cudaLaunchConfig_t c = {};
     c.gridDim = dim3(d.nchunk);
     c.blockDim = dim3(ASSIGN_THREADS);

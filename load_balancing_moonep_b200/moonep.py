@@ -148,7 +148,13 @@ class Config:
         return self.R * self.S * self.K
 
     def c(self) -> _CConfig:
-        return _CConfig(self.R, self.E, self.K, self.S, self.H, self.B, self.flags)
+        """The C struct (built once per Config: the calls pass it by reference
+        on every plan of a latency-bound layer)."""
+        cc = self.__dict__.get("_cc")
+        if cc is None:
+            cc = _CConfig(self.R, self.E, self.K, self.S, self.H, self.B, self.flags)
+            object.__setattr__(self, "_cc", cc)
+        return cc
 
 
 def check_config(cfg: Config) -> int:

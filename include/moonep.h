@@ -289,7 +289,8 @@ MOONEP_API int moonep_prefetch_replicas(const moonep_config *cfg, const moonep_p
  *      is not written, and info[MOONEP_INFO_N_REMOTE_PAIRS] counts this
  *      rank's pairs placed on other ranks;
  *   4. moonep_ep_dispatch / combine / combine_backward /
- *      reduce_replica_grads move the data over the peer pointers.
+ *      reduce_replica_grads / prefetch_replicas move the data over the peer
+ *      pointers.
  * No call synchronises the host, and none issues a collective.
  * Sizes: moonep_ep_sizes (the plan block is laid out by moonep_plan_layout;
  * the workspace, one per rank, is zero-filled once and left ready for the
@@ -337,6 +338,18 @@ MOONEP_API int moonep_ep_combine_backward(const moonep_config *cfg, const moonep
 MOONEP_API int moonep_ep_reduce_replica_grads(const moonep_config *cfg, int32_t rank, const moonep_plan_t *plan,
                                               float *const *reduce_bufs, float *home_grad_local, int64_t P,
                                               void *stream);
+
+/* Replica weight prefetch on rank `rank` (the expert-parallel form of
+ * moonep_prefetch_replicas): each prefetched replica of this rank (ordinal
+ * b = slot - L < B) pulls its expert e's weight row from the home rank
+ * h = e / L, weights[h] + (e - h*L)*P (each rank's [L, P] bf16 home weights,
+ * through the pointer array), into pool_local[b] ([B, P] bf16).
+ * slot_wrow_local [E] int32: home slot s -> s and prefetched replica -> L + b
+ * (rows of this rank's [own weights | pool]); overflow replica of expert e
+ * -> L + B + e (read through from its home rank); unused slot -> -1. */
+MOONEP_API int moonep_ep_prefetch_replicas(const moonep_config *cfg, int32_t rank, const moonep_plan_t *plan,
+                                           const uint16_t *const *weights, uint16_t *pool_local,
+                                           int32_t *slot_wrow_local, int64_t P, void *stream);
 
 /* Size of the fixed device array behind moonep_plan_noalloc (4 MiB).  The
  * large training shape (R=32, E=384, K=8, S=4096) needs about 0.5 MiB. */

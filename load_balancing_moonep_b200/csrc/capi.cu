@@ -33,6 +33,8 @@ int launch_combine_backward_ep(const Dims &d, const int *dst_pos, int *info, con
                                const uint16_t *const *ys, uint16_t *const *dy_bufs, float *dw, cudaStream_t st);
 int launch_reduce_ep(const Dims &d, int rank, const moonep_plan_t &p, float *const *reduce_bufs,
                      float *home_grad, long long P, cudaStream_t st);
+int launch_prefetch_ep(const Dims &d, int rank, const moonep_plan_t &p, const uint16_t *const *weights,
+                       uint16_t *pool, int32_t *slot_wrow, long long P, cudaStream_t st);
 
 constexpr size_t MAX_DYN_SMEM = 227 * 1024;
 constexpr int MAX_COMBINE_BWD_K = 16;
@@ -428,6 +430,21 @@ int moonep_ep_reduce_replica_grads(const moonep_config *cfg, int32_t rank, const
     if (reinterpret_cast<uintptr_t>(home_grad_local) & 3u) return MOONEP_ERR_ALIGN;
     return launch_reduce_ep(d, rank, *plan, reduce_bufs, home_grad_local, (long long)P,
                             static_cast<cudaStream_t>(stream));
+}
+
+int moonep_ep_prefetch_replicas(const moonep_config *cfg, int32_t rank, const moonep_plan_t *plan,
+                                const uint16_t *const *weights, uint16_t *pool_local, int32_t *slot_wrow_local,
+                                int64_t P, void *stream)
+{
+    Dims d;
+    const int rc = make_dims(cfg, &d);
+    if (rc != MOONEP_OK) return rc;
+    if (rank < 0 || rank >= d.R || !plan_ok(plan) || !weights || !slot_wrow_local || P <= 0) return MOONEP_ERR_ARG;
+    if (d.B > 0 && !pool_local) return MOONEP_ERR_ARG;
+    if ((reinterpret_cast<uintptr_t>(pool_local) & 1u) || (reinterpret_cast<uintptr_t>(slot_wrow_local) & 3u))
+        return MOONEP_ERR_ALIGN;
+    return launch_prefetch_ep(d, rank, *plan, weights, pool_local, slot_wrow_local, (long long)P,
+                              static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -89,6 +89,71 @@ __global__ void __launch_bounds__(PF_THREADS) prefetch_kernel(PrefetchParams a)
     }
 }
 
+// Expert parallelism, on rank `rank`: each of its prefetched replicas (list
+// entries on this rank with ordinal b < B) pulls its expert's weight row from
+// the home rank's [L, P] weights (peer memory, through the pointer array)
+// into the local pool row b.  The local slot table: home slot s -> s (own
+// weights), prefetched replica -> L + b (own pool), overflow replica ->
+// L + B + e (expert e read through from its home rank), unused -> -1.
+struct EpPrefetchParams {
+    moonep_plan_t p;
+    const uint8_t *const *weights;  // [R] pointers to each rank's [L, P] bf16 weights
+    uint8_t *pool;                  // this rank's [B, P]
+    int *slot_wrow;                 // this rank's [E]
+    int R, E, L, B, rank;
+    long long row_bytes, chunk;
+};
+
+template <typename V>
+__global__ void __launch_bounds__(PF_THREADS) ep_prefetch_kernel(EpPrefetchParams a)
+{
+    const int status = __ldg(a.p.info + MOONEP_INFO_STATUS);
+    const bool invalid = (status & ST_EMPTY_PLAN) != 0;
+    const long long gtid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long gstride = (long long)gridDim.x * blockDim.x;
+    for (long long s = gtid; s < a.E; s += gstride) {
+        const int e = invalid ? -1 : __ldg(a.p.slot_expert + (long long)a.rank * a.E + s);
+        int row = -1;
+        if (e >= 0 && e < a.E) row = (s < a.L) ? (int)s : (s - a.L < a.B ? (int)s : a.L + a.B + e);
+        a.slot_wrow[s] = row;
+    }
+    if (invalid) return;
+    const int n_rep = min(max(__ldg(a.p.info + MOONEP_INFO_N_REP), 0), a.E + a.R);
+    constexpr int W = sizeof(V);
+    const long long vrow = a.row_bytes / W, vchunk = a.chunk / W;
+    const long long nchunks = (vrow + vchunk - 1) / vchunk;
+    const long long n_items = (long long)n_rep * nchunks;
+    for (long long item = blockIdx.x; item < n_items; item += gridDim.x) {
+        const int q = (int)(item / nchunks);
+        if (__ldg(a.p.rep_rank + q) != a.rank) continue;
+        const int b = __ldg(a.p.rep_slot + q) - a.L, e = __ldg(a.p.rep_expert + q);
+        if (b < 0 || b >= a.B || e < 0 || e >= a.E) continue;  // overflow: read through
+        const int h = e / a.L;
+        const uint8_t *wb = a.weights[h];
+        if (wb == nullptr || (reinterpret_cast<uintptr_t>(wb) & (W - 1))) {
+            if (threadIdx.x == 0) atomicOr(a.p.info + MOONEP_INFO_STATUS, MOONEP_ST_ROW_RANGE);
+            continue;
+        }
+        const long long ci = item - (long long)q * nchunks;
+        const V *src = reinterpret_cast<const V *>(wb + (long long)(e - h * a.L) * a.row_bytes);
+        V *dst = reinterpret_cast<V *>(a.pool + (long long)b * a.row_bytes);
+        const long long v0 = ci * vchunk, v1 = min(vrow, v0 + vchunk);
+        for (long long v = v0 + threadIdx.x; v < v1; v += (long long)PF_THREADS * PF_UNROLL) {
+            V t[PF_UNROLL];
+#pragma unroll
+            for (int u = 0; u < PF_UNROLL; ++u) {
+                const long long x = v + (long long)u * PF_THREADS;
+                if (x < v1) t[u] = src[x];
+            }
+#pragma unroll
+            for (int u = 0; u < PF_UNROLL; ++u) {
+                const long long x = v + (long long)u * PF_THREADS;
+                if (x < v1) dst[x] = t[u];
+            }
+        }
+    }
+}
+
 int launch_prefetch(const Dims &d, const moonep_plan_t &p, const uint16_t *weights, uint16_t *pool,
                     int32_t *slot_wrow, long long P, cudaStream_t st)
 {
@@ -122,6 +187,36 @@ int launch_prefetch(const Dims &d, const moonep_plan_t &p, const uint16_t *weigh
     } else {
         a.chunk = 64 * 1024;
         prefetch_kernel<uint16_t><<<grid, PF_THREADS, 0, st>>>(a);
+    }
+    return cudaGetLastError() == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
+}
+
+int launch_prefetch_ep(const Dims &d, int rank, const moonep_plan_t &p, const uint16_t *const *weights,
+                       uint16_t *pool, int32_t *slot_wrow, long long P, cudaStream_t st)
+{
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+    EpPrefetchParams a;
+    a.p = p;
+    a.weights = reinterpret_cast<const uint8_t *const *>(weights);
+    a.pool = reinterpret_cast<uint8_t *>(pool);
+    a.slot_wrow = slot_wrow;
+    a.R = d.R;
+    a.E = d.E;
+    a.L = d.L;
+    a.B = d.B;
+    a.rank = rank;
+    a.row_bytes = P * 2;
+    const bool vec = (a.row_bytes % 16 == 0) && (reinterpret_cast<uintptr_t>(pool) % 16 == 0);
+    const int grid = sms * (2048 / PF_THREADS) * 8;
+    if (vec) {
+        a.chunk = 256 * 1024;
+        ep_prefetch_kernel<uint4><<<grid, PF_THREADS, 0, st>>>(a);
+    } else {
+        a.chunk = 64 * 1024;
+        ep_prefetch_kernel<uint16_t><<<grid, PF_THREADS, 0, st>>>(a);
     }
     return cudaGetLastError() == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
 }

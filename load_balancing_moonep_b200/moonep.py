@@ -57,7 +57,7 @@ EXPORTED = ("moonep_check_config", "moonep_plan_sizes", "moonep_plan_layout", "m
             "moonep_plan_noalloc", "moonep_prefetch_replicas", "moonep_status_string",
             "moonep_set_wait_limit", "moonep_ep_sizes", "moonep_ep_count", "moonep_ep_plan",
             "moonep_ep_dispatch", "moonep_ep_combine", "moonep_ep_combine_backward",
-            "moonep_ep_reduce_replica_grads")
+            "moonep_ep_reduce_replica_grads", "moonep_ep_prefetch_replicas")
 
 
 class _CConfig(ctypes.Structure):
@@ -96,6 +96,7 @@ _lib.moonep_ep_dispatch.argtypes = [_cfgp, _planp, _vp, _vp, _vp]
 _lib.moonep_ep_combine.argtypes = [_cfgp, _planp, _vp, _vp, _vp, _vp]
 _lib.moonep_ep_combine_backward.argtypes = [_cfgp, _planp, _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.moonep_ep_reduce_replica_grads.argtypes = [_cfgp, ctypes.c_int32, _planp, _vp, _vp, ctypes.c_int64, _vp]
+_lib.moonep_ep_prefetch_replicas.argtypes = [_cfgp, ctypes.c_int32, _planp, _vp, _vp, _vp, ctypes.c_int64, _vp]
 for _f in EXPORTED:
     if _f not in ("moonep_error_string", "moonep_status_string"):
         getattr(_lib, _f).restype = ctypes.c_int
@@ -469,6 +470,26 @@ def ep_reduce_replica_grads(cfg: Config, rank: int, p: Plan, reduce_buf_ptrs: to
                                                reduce_buf_ptrs.data_ptr(), home_grad_local.data_ptr(), P,
                                                _stream(stream)))
     return home_grad_local
+
+
+def ep_prefetch_replicas(cfg: Config, rank: int, p: Plan, weight_ptrs: torch.Tensor, pool_local: torch.Tensor,
+                         slot_wrow_local: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """On rank `rank`: pull each prefetched replica's weight row ([L, P] bf16
+    home weights of every rank, through weight_ptrs) into pool_local [B, P];
+    returns the local slot table [E] (home s, pool L + b, overflow L + B + e
+    read through from the home rank, unused -1)."""
+    P = pool_local.shape[-1]
+    _need(pool_local, torch.bfloat16, (cfg.B, P), "pool_local")
+    _need_ptrs(weight_ptrs, cfg, "weight_ptrs")
+    if slot_wrow_local is None:
+        slot_wrow_local = torch.empty(cfg.E, dtype=torch.int32, device=pool_local.device)
+    _need(slot_wrow_local, torch.int32, (cfg.E,), "slot_wrow_local")
+    c = cfg.c()
+    _check(_lib.moonep_ep_prefetch_replicas(ctypes.byref(c), int(rank), ctypes.byref(p.c_plan),
+                                            weight_ptrs.data_ptr(),
+                                            pool_local.data_ptr() if pool_local.numel() else None,
+                                            slot_wrow_local.data_ptr(), P, _stream(stream)))
+    return slot_wrow_local
 
 
 def views(cfg: Config, p: Plan, buf: torch.Tensor):

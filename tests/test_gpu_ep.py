@@ -238,3 +238,44 @@ def test_ep_null_peer_pointer_is_skipped_and_reported(mp):
     for k in range(wl.R):
         sends_to_1 = ((dp[k] // wl.C) == 1).any()
         assert bool(plans[k].info()["status"] & mp.ST_ROW_RANGE) == bool(sends_to_1)
+
+
+@pytest.mark.parametrize("wname,mv,B", [("tiny", 1.0, None), ("mid", 3.0, None), ("mid", 3.0, 1)])
+def test_ep_prefetch_matches_the_oracle(mp, wname, mv, B):
+    """Each rank pulls its prefetched replicas' weight rows from the home
+    ranks' [L, P] weights (R separate allocations): its pool rows equal the
+    oracle's pool[r], and its slot table is the oracle's in the rank's own
+    row numbering (home s, pool L + b, overflow read-through L + B + e).
+    B = 1 on the mid shape leaves overflow replicas."""
+    wl = W.WORKLOADS[wname]
+    Bv = wl.B if B is None else B
+    c = dict(R=wl.R, E=wl.E, K=wl.K, S=wl.S, H=wl.H, B=Bv, flags=0)
+    cfg, ocfg = mp.Config(**c), oracle.Config(**c)
+    r = W.routing(wl, mv, device=DEV)
+    op = oracle.plan(ocfg, r.topk_idx.cpu().numpy())
+    plans, _ = _ep_plans(mp, cfg, r.topk_idx)
+    R, E, L, P = wl.R, wl.E, wl.L, 1000
+    weights = W.bf16_normal((E, P), seed=7, device=DEV)
+    owners = [weights[h * L:(h + 1) * L].clone() for h in range(R)]  # each rank's home weights
+    wp = mp.pointer_array(owners)
+    pools = [torch.zeros((Bv, P), dtype=torch.bfloat16, device=DEV) for _ in range(R)]
+    tables = [mp.ep_prefetch_replicas(cfg, k, plans[k], wp, pools[k]) for k in range(R)]
+    torch.cuda.synchronize()
+    opool = np.zeros((R, Bv, P), np.uint16)
+    owrow = oracle.prefetch_replicas(ocfg, op, W.bits(weights), opool, P)
+    if wname == "mid" and B == 1:
+        assert op["info"][2] > 0  # overflow replicas present
+    for k in range(R):
+        assert np.array_equal(W.bits(pools[k]), opool[k]), f"rank {k}: pool differs"
+        exp = np.full(E, -1, np.int32)
+        for s in range(E):
+            e, row = op["slot_expert"][k, s], owrow[k, s]
+            if e < 0:
+                continue
+            if s < L:
+                exp[s] = s
+            elif row >= E:  # a prefetched replica: pool row E + k*B + b
+                exp[s] = L + (row - E - k * Bv)
+            else:  # overflow: read through from the home rank
+                exp[s] = L + Bv + e
+        assert np.array_equal(tables[k].cpu().numpy(), exp), f"rank {k}: slot table differs"

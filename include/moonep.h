@@ -50,7 +50,7 @@
 extern "C" {
 #endif
 
-#define MOONEP_ABI_VERSION 1
+#define MOONEP_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define MOONEP_API __attribute__((visibility("default")))
@@ -76,6 +76,17 @@ extern "C" {
  * fit; at E = R = MOONEP_MAX_E it does) and a slow path, one warp stepping
  * through the repairs, when it runs.  Unknown flag bits are MOONEP_ERR_ARG. */
 #define MOONEP_FLAG_CASCADE 8u
+/* Locality-aware host intervals (expert parallelism: moonep_ep_plan only;
+ * moonep_plan, where a pair on another rank costs no transfer, refuses it
+ * with MOONEP_ERR_ARG).  Each host of an expert first takes up to its quota
+ * of the pairs from its own rank (the first ones, in (t, k) order:
+ * host_local[h] = min(quota, those pairs)); the pairs left over, in (t, k)
+ * order, fill the rest of the quotas in ascending rank order, host_start[h]
+ * being where host h's share of them starts.  The replicas, quotas and slots
+ * are water-filling's; the pairs kept on their source rank are the most any
+ * choice of intervals keeps for them.  A host's rows hold its local pairs
+ * first, then its leftover ones, each part in (t, k) order. */
+#define MOONEP_FLAG_LOCALITY 16u
 
 /* ---- host return codes ------------------------------------------------- */
 #define MOONEP_OK 0
@@ -162,12 +173,14 @@ typedef struct moonep_plan_s {
     int32_t *host_ptr;      /* [E+1] CSR: hosts of expert e are [host_ptr[e], host_ptr[e+1]) */
     int32_t *host_rank;     /* [2E+R] hosts in ascending rank order (home copy included) */
     int32_t *host_slot;     /* [2E+R] */
-    int32_t *host_start;    /* [2E+R] first within-expert rank g served by the host */
+    int32_t *host_start;    /* [2E+R] first within-expert rank g served by the host (with
+                               MOONEP_FLAG_LOCALITY: the start of its share of the leftover pairs) */
     int32_t *host_quota;    /* [2E+R] number of g served by the host */
     int32_t *rep_home_list; /* [E] experts with >= 1 prefetched replica, ascending, then -1 */
     int32_t *dst_pos;       /* [R*S*K] buffer row of pair (t, k), index t*K + k */
     int32_t *row_src;       /* [R*S*K] inverse: pair t*K + k held by a buffer row */
     int32_t *info;          /* [MOONEP_INFO_LEN] status and statistics */
+    int32_t *host_local;    /* [2E+R] pairs of the host's own rank it serves first (MOONEP_FLAG_LOCALITY), else 0 */
 } moonep_plan_t;
 
 /* Host-side validation of a configuration.  Returns MOONEP_OK or an error. */

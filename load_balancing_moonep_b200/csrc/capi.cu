@@ -132,23 +132,25 @@ static bool plan_ok(const moonep_plan_t *p)
 {
     return p && p->expert_count && p->slot_expert && p->slot_count && p->slot_offset && p->rep_expert &&
            p->rep_rank && p->rep_slot && p->rep_quota && p->host_ptr && p->host_rank && p->host_slot &&
-           p->host_start && p->host_quota && p->rep_home_list && p->dst_pos && p->row_src && p->info;
+           p->host_start && p->host_quota && p->rep_home_list && p->dst_pos && p->row_src && p->info &&
+           p->host_local;
 }
 
+constexpr int PLAN_ARRAYS = 18;
 struct PlanLayout {
-    size_t off[17];
+    size_t off[PLAN_ARRAYS];
     size_t total;
 };
 
 static PlanLayout plan_layout(const Dims &d)
 {
     const size_t E = d.E, R = d.R, NP = (size_t)d.pairs;
-    const size_t n[17] = {E,         R * E,     R * E,     R * (E + 1), E + R,      E + R,
-                          E + R,     E + R,     E + 1,     2 * E + R,   2 * E + R,  2 * E + R,
-                          2 * E + R, E,         NP,        NP,          MOONEP_INFO_LEN};
+    const size_t n[PLAN_ARRAYS] = {E,         R * E,     R * E,     R * (E + 1), E + R,      E + R,
+                                   E + R,     E + R,     E + 1,     2 * E + R,   2 * E + R,  2 * E + R,
+                                   2 * E + R, E,         NP,        NP,          MOONEP_INFO_LEN, 2 * E + R};
     PlanLayout l;
     size_t o = 0;
-    for (int i = 0; i < 17; ++i) {
+    for (int i = 0; i < PLAN_ARRAYS; ++i) {
         l.off[i] = o;
         o = align256(o + n[i] * sizeof(int32_t));
     }
@@ -232,7 +234,7 @@ int moonep_check_config(const moonep_config *c)
     if (c->K > c->E) return MOONEP_ERR_ARG;
     if ((int64_t)c->R * c->S * c->K > INT32_MAX) return MOONEP_ERR_ARG;
     if (c->flags & ~(MOONEP_FLAG_STRICT_BUDGET | MOONEP_FLAG_TRAIN_B_RULE | MOONEP_FLAG_BWD_UNSCALED |
-                     MOONEP_FLAG_CASCADE))
+                     MOONEP_FLAG_CASCADE | MOONEP_FLAG_LOCALITY))
         return MOONEP_ERR_ARG;
     if (c->E % c->R != 0) return MOONEP_ERR_E_NOT_DIVISIBLE;
     const int L = c->E / c->R;
@@ -262,12 +264,12 @@ int moonep_plan_layout(const moonep_config *cfg, void *plan_base, moonep_plan_t 
     if (reinterpret_cast<uintptr_t>(plan_base) & 255u) return MOONEP_ERR_ALIGN;
     const PlanLayout l = plan_layout(d);
     char *b = static_cast<char *>(plan_base);
-    int32_t **f[17] = {&out->expert_count, &out->slot_expert, &out->slot_count, &out->slot_offset,
-                       &out->rep_expert,   &out->rep_rank,    &out->rep_slot,   &out->rep_quota,
-                       &out->host_ptr,     &out->host_rank,   &out->host_slot,  &out->host_start,
-                       &out->host_quota,   &out->rep_home_list, &out->dst_pos,  &out->row_src,
-                       &out->info};
-    for (int i = 0; i < 17; ++i) *f[i] = reinterpret_cast<int32_t *>(b + l.off[i]);
+    int32_t **f[PLAN_ARRAYS] = {&out->expert_count, &out->slot_expert,   &out->slot_count, &out->slot_offset,
+                                &out->rep_expert,   &out->rep_rank,      &out->rep_slot,   &out->rep_quota,
+                                &out->host_ptr,     &out->host_rank,     &out->host_slot,  &out->host_start,
+                                &out->host_quota,   &out->rep_home_list, &out->dst_pos,    &out->row_src,
+                                &out->info,         &out->host_local};
+    for (int i = 0; i < PLAN_ARRAYS; ++i) *f[i] = reinterpret_cast<int32_t *>(b + l.off[i]);
     return MOONEP_OK;
 }
 
@@ -278,6 +280,9 @@ int moonep_plan(const moonep_config *cfg, const int32_t *topk_idx, const moonep_
     const int rc = make_dims(cfg, &d, current_device_sms());
     if (rc != MOONEP_OK) return rc;
     if (!topk_idx || !plan_ok(plan) || !workspace) return MOONEP_ERR_ARG;
+    // one GPU holds every rank: no pair crosses a link, and the locality
+    // flag's per-rank counts exist only in expert parallelism
+    if (d.flags & MOONEP_FLAG_LOCALITY) return MOONEP_ERR_ARG;
     return launch_plan(d, topk_idx, *plan, workspace, static_cast<cudaStream_t>(stream));
 }
 

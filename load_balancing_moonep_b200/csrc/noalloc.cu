@@ -62,6 +62,7 @@ int moonep_plan_noalloc(const moonep_config *cfg, const int32_t *topk_idx, const
     if (rc != MOONEP_OK) return rc;
     if (ws_bytes > MOONEP_NOALLOC_WORKSPACE_BYTES) return MOONEP_ERR_NOALLOC_SIZE;
     if (!topk_idx || !plan) return MOONEP_ERR_ARG;
+    if (cfg->flags & MOONEP_FLAG_LOCALITY) return MOONEP_ERR_ARG;  // as moonep_plan: expert parallelism only
     const int crc = moonep::workspace_clear_bytes(cfg, &clear_bytes);
     if (crc != MOONEP_OK) return crc;
     void *ws = nullptr;

@@ -579,12 +579,17 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
         }
         int st = 0;
         for (int h = b0; h < k; ++h) {
+            // the locality flag as in the water-filling tail
+            const int loc = (d.flags & MOONEP_FLAG_LOCALITY)
+                                ? min(xq[h], ld_cg(a.gs + (size_t)xr[h] * a.gs_stride + e))
+                                : 0;
             a.p.host_rank[h] = xr[h];
             a.p.host_slot[h] = xs[h];
             a.p.host_quota[h] = xq[h];
             a.p.host_start[h] = st;
+            a.p.host_local[h] = loc;
             a.host_dst0[h] = xr[h] * C + xo[h] - st;
-            st += xq[h];
+            st += xq[h] - loc;
         }
     }
     __syncthreads();
@@ -905,8 +910,13 @@ __device__ void plan_block(const PlanParams &a, int *sm, int seq)
     // ---- host intervals first: they are all the assignment CTAs wait for.
     // The hosts of e in ascending rank; a host's start is the rows of the
     // hosts of e on lower ranks.
+    // With MOONEP_FLAG_LOCALITY (expert parallelism, where the count rows are
+    // the ranks' own counts) a host first takes min(quota, its rank's pairs
+    // of e), and its start is in the order of the pairs left over.
+    const bool locality = (d.flags & MOONEP_FLAG_LOCALITY) != 0;
+    auto own_pairs = [&](int r, int e) { return ld_cg(a.gs + (size_t)r * a.gs_stride + e); };
     for (int x = tid; x < n_hosts; x += nt) {
-        int e, r0, slot, quota, j, pos = 0, st = 0;
+        int e, r0, slot, quota, j, pos = 0, st = 0, locsum = 0;
         if (x < E) {
             e = x;
             r0 = (int)fdiv((uint32_t)e, a.fL);
@@ -921,9 +931,11 @@ __device__ void plan_block(const PlanParams &a, int *sm, int seq)
             r0 = qr[i];
             slot = L + (j - jlo[i]);
             quota = seg_q(j, i);
-            if ((int)fdiv((uint32_t)e, a.fL) < r0) {  // the home rank is lower
+            const int home = (int)fdiv((uint32_t)e, a.fL);
+            if (home < r0) {  // the home rank is lower
                 pos = 1;
                 st = keep[e];
+                if (locality) locsum = min(keep[e], own_pairs(home, e));
             }
         }
         if (j >= 0) {
@@ -932,16 +944,21 @@ __device__ void plan_block(const PlanParams &a, int *sm, int seq)
                 const int i = pilo[j] + s;
                 if (qr[i] < r0) {
                     ++pos;
-                    st += seg_q(j, i);
+                    const int qi = seg_q(j, i);
+                    st += qi;
+                    if (locality) locsum += min(qi, own_pairs(qr[i], e));
                 }
             }
         }
+        const int loc = locality ? min(quota, own_pairs(r0, e)) : 0;
+        st -= locsum;
         const int h = hptr(e) + pos;
         const int b0 = rank_base(r0);
         a.p.host_rank[h] = r0;
         a.p.host_slot[h] = slot;
         a.p.host_quota[h] = quota;
         a.p.host_start[h] = st;
+        a.p.host_local[h] = loc;
         a.host_dst0[h] = r0 * C + Z[b0 + slot] - Z[b0] - st;
     }
     for (int x = tid; x <= E; x += nt) a.p.host_ptr[x] = hptr(x);
@@ -1026,6 +1043,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) hist_plan_kernel(PlanParams a)
             a.p.host_slot[x] = -1;
             a.p.host_start[x] = 0;
             a.p.host_quota[x] = 0;
+            a.p.host_local[x] = 0;
         }
     }
     for (int e = tid; e < E; e += nt) hist[e] = 0;
@@ -1306,6 +1324,7 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
             a.p.host_slot[x] = -1;
             a.p.host_start[x] = 0;
             a.p.host_quota[x] = 0;
+            a.p.host_local[x] = 0;
         }
         for (int x = x0; x <= E; x += g) a.p.host_ptr[x] = 0;
         for (int x = x0; x < E; x += g) a.p.rep_home_list[x] = -1;
@@ -1507,6 +1526,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) ep_plan_kernel(PlanParams a)
         a.p.host_slot[x] = -1;
         a.p.host_start[x] = 0;
         a.p.host_quota[x] = 0;
+        a.p.host_local[x] = 0;
     }
     if (tid < 32) {
         int bad = 0;
@@ -1531,6 +1551,61 @@ __global__ void __launch_bounds__(PLAN_THREADS) ep_plan_kernel(PlanParams a)
 // row_src is not written (the rows of this rank's buffer are filled by every
 // rank).  info[MOONEP_INFO_N_REMOTE_PAIRS] counts this rank's pairs placed
 // on another rank.
+__host__ __device__ inline int ep_assign_smem_ints(int E, int R, int max_pairs)
+{
+    const int nh = 2 * E + R;
+    return assign_smem_ints(E, R, max_pairs) + 3 * nh /*local quota rank*/ + 3 * E /*own before G*/;
+}
+
+// Pass B with MOONEP_FLAG_LOCALITY for the calling warp's sub-range, all of
+// whose pairs come from rank `rank`: the pair's rank g within its expert and
+// gs within this rank's pairs of it (g - G[e]); the host on this rank takes
+// it as local pair gs when gs < its local count, otherwise it is leftover
+// number u = g - before[e] (the local pairs of the hosts on ranks <= rank),
+// served by the host whose leftover share [start, start + quota - local)
+// holds u, at row dst0 + local + u.
+__device__ __forceinline__ int assign_pass_b_local(const int *ids, const int *wb, const int *hptr,
+                                                   const int *hstart, const int *hdst, const int *hloc,
+                                                   const int *hq, const int *own, const int *before,
+                                                   const int *G, int wbeg, int wend, int p0, int E, int rows,
+                                                   int C, int rank, int *dst_pos, int *info)
+{
+    const int lane = threadIdx.x & 31;
+    int remote = 0;
+    for (int i = wbeg + lane; i < wend; i += 32) {
+        const int v = ids[i];
+        const int e = v & PACK_MASK, loc = v >> PACK_BITS;
+        if (v < 0 || e >= E) continue;  // cannot happen in a non-empty plan
+        const int g = wb[e] + loc, gs = g - G[e], ho = own[e];
+        int dst = -1;
+        if (ho >= 0 && gs < hloc[ho]) {
+            dst = hdst[ho] + hstart[ho] + gs;
+        } else {
+            const int u = g - before[e];
+            for (int h = hptr[e]; h < hptr[e + 1]; ++h)
+                if (hstart[h] <= u && u < hstart[h] + hq[h] - hloc[h]) {
+                    dst = hdst[h] + hloc[h] + u;
+                    break;
+                }
+        }
+        const int p = p0 + i;
+        if (dst < 0 || dst >= rows) {  // cannot happen for a consistent plan
+            atomicOr(info + MOONEP_INFO_STATUS, MOONEP_ST_ROW_RANGE);
+            dst_pos[p] = -1;
+            continue;
+        }
+        dst_pos[p] = dst;
+        remote += (uint32_t)dst - (uint32_t)rank * (uint32_t)C >= (uint32_t)C;
+    }
+    return remote;
+}
+
+// The rank's own pairs: pass A on the ids while the planner runs, chunk
+// bases from the lower ranks' counts and this rank's earlier chunks, then
+// (after the planner grid) pass B.  dst_pos[0 .. S*K) gets global rows;
+// row_src is not written (the rows of this rank's buffer are filled by every
+// rank).  info[MOONEP_INFO_N_REMOTE_PAIRS] counts this rank's pairs placed
+// on another rank.
 __global__ void __launch_bounds__(ASSIGN_THREADS, 2) ep_assign_kernel(PlanParams a, int rank)
 {
     extern __shared__ int sm[];
@@ -1542,12 +1617,19 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) ep_assign_kernel(PlanParams
     const int p0 = t0 * K, n = (t1 - t0) * K;
     const int max_pairs = d.chunk_tokens * K;
     const int nh = 2 * E + R;
+    const bool locality = (d.flags & MOONEP_FLAG_LOCALITY) != 0;
     int *cnt = sm;                      // ASSIGN_WARPS * E
     int *ids = cnt + ASSIGN_WARPS * E;  // max_pairs
     int *hptr = ids + max_pairs;        // E + 1
     int *hstart = hptr + E + 1;         // nh
     int *hdst = hstart + nh;            // nh
     int *red = hdst + nh;               // 32
+    int *hloc = red + 32;               // nh  (locality only, from here on)
+    int *hq = hloc + nh;                // nh
+    int *hr = hq + nh;                  // nh
+    int *own = hr + nh;                 // E: the expert's host on this rank, or -1
+    int *before = own + E;              // E: local pairs of the hosts on ranks <= rank
+    int *G = before + E;                // E: the expert's pairs on lower ranks
 
     // on the ids and the counts only, overlapping the planner
     for (int i = tid; i < ASSIGN_WARPS * E; i += nt) cnt[i] = 0;
@@ -1560,7 +1642,9 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) ep_assign_kernel(PlanParams
     // chunk base: pairs of e on lower ranks plus on this rank's earlier
     // chunks; then the warp bases
     for (int e = tid; e < E; e += nt) {
-        int s = sum_strided<32>(a.gs + e, a.gs_stride, rank) + sum_strided<32>(a.cc + e, E, chunk);
+        const int lower = sum_strided<32>(a.gs + e, a.gs_stride, rank);
+        G[e] = lower;
+        int s = lower + sum_strided<32>(a.cc + e, E, chunk);
         for (int w = 0; w < ASSIGN_WARPS; ++w) {
             const int t = cnt[w * E + e];
             cnt[w * E + e] = s;
@@ -1574,14 +1658,35 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) ep_assign_kernel(PlanParams
     for (int h = tid; h < nh; h += nt) {
         hstart[h] = ld_cg(a.p.host_start + h);
         hdst[h] = ld_cg(a.host_dst0 + h);
+        if (locality) {
+            hloc[h] = ld_cg(a.p.host_local + h);
+            hq[h] = ld_cg(a.p.host_quota + h);
+            hr[h] = ld_cg(a.p.host_rank + h);
+        }
     }
     if (status & ST_EMPTY_PLAN) {
         for (int i = tid; i < n; i += nt) a.p.dst_pos[p0 + i] = -1;
         return;
     }
     __syncthreads();
-    int remote = assign_pass_b(ids, cnt + warp * E, hptr, hstart, hdst, wbeg, wend, p0, E, R * C, C, a.fC, rank,
+    int remote;
+    if (locality) {
+        for (int e = tid; e < E; e += nt) {
+            int o = -1, b = 0;
+            for (int h = hptr[e]; h < hptr[e + 1]; ++h) {
+                if (hr[h] <= rank) b += hloc[h];
+                if (hr[h] == rank) o = h;
+            }
+            own[e] = o;
+            before[e] = b;
+        }
+        __syncthreads();
+        remote = assign_pass_b_local(ids, cnt + warp * E, hptr, hstart, hdst, hloc, hq, own, before, G, wbeg, wend,
+                                     p0, E, R * C, C, rank, a.p.dst_pos, a.p.info);
+    } else {
+        remote = assign_pass_b(ids, cnt + warp * E, hptr, hstart, hdst, wbeg, wend, p0, E, R * C, C, a.fC, rank,
                                a.p.dst_pos, nullptr, a.p.info);
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) remote += __shfl_xor_sync(FULL_MASK, remote, o);
     if (lane == 0) red[warp] = remote;
@@ -1646,7 +1751,7 @@ int launch_ep_plan(const Dims &d, int rank, const int32_t *topk, const int32_t *
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
-    const size_t smem2 = sizeof(int) * (size_t)assign_smem_ints(d.E, d.R, d.chunk_tokens * d.K);
+    const size_t smem2 = sizeof(int) * (size_t)ep_assign_smem_ints(d.E, d.R, d.chunk_tokens * d.K);
     if (!set_smem(K_EP_ASSIGN, (const void *)ep_assign_kernel, smem2)) return MOONEP_ERR_CUDA;
     cudaLaunchConfig_t c = {};
     c.gridDim = dim3(d.nchunk);
@@ -1662,7 +1767,7 @@ size_t ep_smem_bytes_max(const Dims &d)
 {
     const size_t a = sizeof(int) * (size_t)(plan_smem_ints(d.E, d.R) +
                                             ((d.flags & MOONEP_FLAG_CASCADE) ? cascade_smem_ints(d.E, d.R, d.B) : 0));
-    const size_t b = sizeof(int) * (size_t)assign_smem_ints(d.E, d.R, d.chunk_tokens * d.K);
+    const size_t b = sizeof(int) * (size_t)ep_assign_smem_ints(d.E, d.R, d.chunk_tokens * d.K);
     const size_t c = sizeof(int) * (size_t)(d.E + d.chunk_tokens * d.K);
     return a > b ? (a > c ? a : c) : (b > c ? b : c);
 }

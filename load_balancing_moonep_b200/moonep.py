@@ -34,6 +34,7 @@ FLAG_STRICT_BUDGET = 1
 FLAG_TRAIN_B_RULE = 2
 FLAG_BWD_UNSCALED = 4
 FLAG_CASCADE = 8
+FLAG_LOCALITY = 16
 
 ST_EXPERT_ID_RANGE = 1
 ST_OVERFLOW = 2
@@ -49,7 +50,7 @@ INFO_LEN = 16
 
 PLAN_FIELDS = ("expert_count", "slot_expert", "slot_count", "slot_offset", "rep_expert", "rep_rank",
                "rep_slot", "rep_quota", "host_ptr", "host_rank", "host_slot", "host_start",
-               "host_quota", "rep_home_list", "dst_pos", "row_src", "info")
+               "host_quota", "rep_home_list", "dst_pos", "row_src", "info", "host_local")
 
 EXPORTED = ("moonep_check_config", "moonep_plan_sizes", "moonep_plan_layout", "moonep_plan",
             "moonep_dispatch", "moonep_combine", "moonep_combine_backward",
@@ -202,7 +203,7 @@ class Plan:
             "rep_slot": (E + R,), "rep_quota": (E + R,), "host_ptr": (E + 1,),
             "host_rank": (2 * E + R,), "host_slot": (2 * E + R,), "host_start": (2 * E + R,),
             "host_quota": (2 * E + R,), "rep_home_list": (E,), "dst_pos": (R * S, K),
-            "row_src": (R * S * K,), "info": (INFO_LEN,),
+            "row_src": (R * S * K,), "info": (INFO_LEN,), "host_local": (2 * E + R,),
         }
         base = self.block.data_ptr()
         i32 = self.block.view(torch.int32) if pb % 4 == 0 else None

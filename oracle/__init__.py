@@ -35,6 +35,7 @@ FLAG_STRICT_BUDGET = 1
 FLAG_TRAIN_B_RULE = 2
 FLAG_BWD_UNSCALED = 4
 FLAG_CASCADE = 8
+FLAG_LOCALITY = 16
 
 ST_EXPERT_ID_RANGE = 1
 ST_OVERFLOW = 2
@@ -94,7 +95,7 @@ def openmp_lib(threads: int = 0):
 
 def _bind(lib):
     if True:
-        lib.or_plan.argtypes = [ctypes.c_void_p] + [ctypes.c_void_p] * 18
+        lib.or_plan.argtypes = [ctypes.c_void_p] + [ctypes.c_void_p] * 19
         lib.or_plan.restype = ctypes.c_int
         lib.or_check_config.argtypes = [ctypes.c_void_p]
         lib.or_check_config.restype = ctypes.c_int
@@ -191,6 +192,7 @@ def plan(cfg: Config, topk_idx: np.ndarray) -> dict:
         "host_slot": np.zeros(2 * E + R, np.int32),
         "host_start": np.zeros(2 * E + R, np.int32),
         "host_quota": np.zeros(2 * E + R, np.int32),
+        "host_local": np.zeros(2 * E + R, np.int32),
         "rep_home_list": np.zeros(E, np.int32),
         "dst_pos": np.zeros((R * S, K), np.int32),
         "row_src": np.zeros(R * S * K, np.int32),
@@ -202,7 +204,7 @@ def plan(cfg: Config, topk_idx: np.ndarray) -> dict:
                      _p(out["slot_offset"]), _p(out["rep_expert"]), _p(out["rep_rank"]),
                      _p(out["rep_slot"]), _p(out["rep_quota"]), _p(out["host_ptr"]),
                      _p(out["host_rank"]), _p(out["host_slot"]), _p(out["host_start"]),
-                     _p(out["host_quota"]), _p(out["rep_home_list"]), _p(out["dst_pos"]),
+                     _p(out["host_quota"]), _p(out["host_local"]), _p(out["rep_home_list"]), _p(out["dst_pos"]),
                      _p(out["row_src"]), _p(out["info"]))
     _check(rc)
     return out

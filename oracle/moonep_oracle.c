@@ -46,7 +46,8 @@
  *   O5b (only with the cascade flag, and only when O5 left a rank with more
  *      than B replicas) relay cascade, described at or_cascade below;
  *   O6 per-rank slot tables (home slots 0..L-1, then replicas);
- *   O7 per-expert host intervals, hosts in ascending rank order;
+ *   O7 per-expert host intervals, hosts in ascending rank order (with
+ *      OR_FLAG_LOCALITY each host first serves the pairs of its own rank);
  *   O8 pairs in global (t, k) order fill their expert's host intervals.
  *
  * Floating point: the precision is the one the method fixes -- bf16 data,
@@ -63,6 +64,7 @@
 #define OR_FLAG_TRAIN_B_RULE 2u
 #define OR_FLAG_BWD_UNSCALED 4u
 #define OR_FLAG_CASCADE 8u
+#define OR_FLAG_LOCALITY 16u
 
 #define OR_ST_EXPERT_ID_RANGE 1
 #define OR_ST_OVERFLOW 2
@@ -128,7 +130,8 @@ int or_check_config(const or_config *c)
         return OR_ERR_ARG;
     if (c->K > c->E) return OR_ERR_ARG;
     if ((int64_t)c->R * c->S * c->K > INT32_MAX) return OR_ERR_ARG;
-    if (c->flags & ~(OR_FLAG_STRICT_BUDGET | OR_FLAG_TRAIN_B_RULE | OR_FLAG_BWD_UNSCALED | OR_FLAG_CASCADE))
+    if (c->flags & ~(OR_FLAG_STRICT_BUDGET | OR_FLAG_TRAIN_B_RULE | OR_FLAG_BWD_UNSCALED | OR_FLAG_CASCADE |
+                     OR_FLAG_LOCALITY))
         return OR_ERR_ARG;
     /* the explainer flags E % R != 0 as a configuration error [P1 explainer] */
     if (c->E % c->R != 0) return OR_ERR_E_NOT_DIVISIBLE;
@@ -347,8 +350,8 @@ int or_plan(const or_config *c, const int32_t *topk,
             int32_t *T, int32_t *slot_expert, int32_t *slot_count, int32_t *slot_offset,
             int32_t *rep_expert, int32_t *rep_rank, int32_t *rep_slot, int32_t *rep_quota,
             int32_t *host_ptr, int32_t *host_rank, int32_t *host_slot, int32_t *host_start,
-            int32_t *host_quota, int32_t *rep_home_list, int32_t *dst_pos, int32_t *row_src,
-            int32_t *info)
+            int32_t *host_quota, int32_t *host_local, int32_t *rep_home_list, int32_t *dst_pos,
+            int32_t *row_src, int32_t *info)
 {
     int rc = or_check_config(c);
     if (rc != OR_OK) return rc;
@@ -364,7 +367,9 @@ int or_plan(const or_config *c, const int32_t *topk,
     for (int64_t i = 0; i < (int64_t)R * (E + 1); ++i) slot_offset[i] = 0;
     for (int32_t i = 0; i < NREP_MAX; ++i) { rep_expert[i] = -1; rep_rank[i] = -1; rep_slot[i] = -1; rep_quota[i] = 0; }
     for (int32_t i = 0; i <= E; ++i) host_ptr[i] = 0;
-    for (int32_t i = 0; i < NHOST_MAX; ++i) { host_rank[i] = -1; host_slot[i] = -1; host_start[i] = 0; host_quota[i] = 0; }
+    for (int32_t i = 0; i < NHOST_MAX; ++i) {
+        host_rank[i] = -1; host_slot[i] = -1; host_start[i] = 0; host_quota[i] = 0; host_local[i] = 0;
+    }
     for (int32_t i = 0; i < E; ++i) rep_home_list[i] = -1;
     for (int64_t p = 0; p < NP; ++p) { dst_pos[p] = -1; row_src[p] = -1; }
     for (int i = 0; i < OR_INFO_LEN; ++i) info[i] = 0;
@@ -393,6 +398,7 @@ int or_plan(const or_config *c, const int32_t *topk,
     int32_t *rep_ord = calloc((size_t)NREP_MAX, sizeof(int32_t));
     host_t *hosts = calloc((size_t)R + 1, sizeof(host_t));
     int32_t *gcount = calloc((size_t)E, sizeof(int32_t));
+    int32_t *src_count = NULL, *src_seen = NULL;  /* [R][E]: pairs per (source rank, expert) */
     if (!Hl || !X || !D || !shed || !keep || !order || !pieces || !recv || !PS || !QS ||
         !nrep_on || !rep_ord || !hosts || !gcount) {
         rc = OR_ERR_NOMEM;
@@ -509,7 +515,20 @@ int or_plan(const or_config *c, const int32_t *topk,
         slot_offset[(int64_t)r * (E + 1) + E] = (int32_t)acc;
     }
 
-    /* O7: host intervals per expert, hosts in ascending rank order */
+    /* O7: host intervals per expert, hosts in ascending rank order.  Without
+     * OR_FLAG_LOCALITY host h serves the pairs g in [start_h, start_h + q_h)
+     * of its expert, the quotas laid out in rank order.  With it, host h
+     * first serves loc_h = min(q_h, pairs of the expert from h's own rank)
+     * of its own rank's pairs (the first ones, in (t, k) order), and the
+     * pairs left over, in (t, k) order, fill the rest of the quotas
+     * q_h - loc_h in rank order: host_start then holds where host h's share
+     * of the leftover pairs starts and host_local holds loc_h. */
+    const int locality = (c->flags & OR_FLAG_LOCALITY) != 0;
+    if (locality) {
+        src_count = calloc((size_t)R * E, sizeof(int32_t));
+        if (!src_count) { rc = OR_ERR_NOMEM; goto out; }
+        for (int64_t p = 0; p < NP; ++p) src_count[((p / K) / S) * E + topk[p]] += 1;
+    }
     int32_t hcur = 0;
     for (int32_t e = 0; e < E; ++e) {
         int32_t nh = 0;
@@ -530,33 +549,61 @@ int or_plan(const or_config *c, const int32_t *topk,
         host_ptr[e] = hcur;
         int32_t start = 0;
         for (int32_t h = 0; h < nh; ++h) {
+            const int32_t q = hosts[h].quota;
+            const int32_t loc = locality ? (int32_t)min64(q, src_count[(int64_t)hosts[h].rank * E + e]) : 0;
             host_rank[hcur] = hosts[h].rank;
             host_slot[hcur] = hosts[h].slot;
             host_start[hcur] = start;
-            host_quota[hcur] = hosts[h].quota;
-            start += hosts[h].quota;
+            host_quota[hcur] = q;
+            host_local[hcur] = loc;
+            start += q - loc;
             ++hcur;
         }
     }
     host_ptr[E] = hcur;
 
-    /* O8: pairs in global (t, k) order fill their expert's host intervals */
+    /* O8: pairs in global (t, k) order.  The g-th pair of expert e, the
+     * gs-th of e among the pairs of its own source rank s: if the host on
+     * rank s serves gs among its local pairs (gs < loc), it takes the pair
+     * at offset gs; otherwise the pair is leftover number
+     * u = g - (local pairs of the hosts on ranks <= s), and the host whose
+     * leftover share [start, start + q - loc) holds u takes it at offset
+     * loc + (u - start).  Without the flag loc = 0: u = g, the plain
+     * interval layout. */
     int64_t n_remote = 0;
+    src_seen = calloc((size_t)R * E, sizeof(int32_t));
+    if (!src_seen) { rc = OR_ERR_NOMEM; goto out; }
     for (int32_t e = 0; e < E; ++e) gcount[e] = 0;
     for (int64_t p = 0; p < NP; ++p) {
-        int32_t e = topk[p];
-        int32_t g = gcount[e]++;
-        int32_t found = -1;
-        for (int32_t h = host_ptr[e]; h < host_ptr[e + 1]; ++h)
-            if (host_start[h] <= g && g < host_start[h] + host_quota[h]) { found = h; break; }
+        const int32_t e = topk[p];
+        const int32_t g = gcount[e]++;
+        const int32_t s_rank = (int32_t)((p / K) / S);
+        const int32_t gs = src_seen[(int64_t)s_rank * E + e]++;
+        int32_t found = -1, own = -1;
+        int64_t off = 0, before = 0;
+        for (int32_t h = host_ptr[e]; h < host_ptr[e + 1]; ++h) {
+            if (host_rank[h] <= s_rank) before += host_local[h];
+            if (host_rank[h] == s_rank) own = h;
+        }
+        if (own >= 0 && gs < host_local[own]) {
+            found = own;
+            off = gs;
+        } else {
+            const int64_t u = g - before;
+            for (int32_t h = host_ptr[e]; h < host_ptr[e + 1]; ++h)
+                if (host_start[h] <= u && u < host_start[h] + host_quota[h] - host_local[h]) {
+                    found = h;
+                    off = host_local[h] + (u - host_start[h]);
+                    break;
+                }
+        }
         if (found < 0) { rc = OR_ERR_ARG; goto out; } /* cannot happen: quotas sum to T[e] */
         int32_t r = host_rank[found];
-        int64_t d = (int64_t)r * C + slot_offset[(int64_t)r * (E + 1) + host_slot[found]] +
-                    (g - host_start[found]);
+        int64_t d = (int64_t)r * C + slot_offset[(int64_t)r * (E + 1) + host_slot[found]] + off;
+        if (d < 0 || d >= (int64_t)R * C) { rc = OR_ERR_ARG; goto out; } /* cannot happen */
         dst_pos[p] = (int32_t)d;
         row_src[d] = (int32_t)p;
-        int64_t src_rank = (p / K) / S;
-        if (src_rank != r) ++n_remote;
+        if (s_rank != r) ++n_remote;
     }
 
     /* statistics and the reduce work list */
@@ -590,6 +637,7 @@ int or_plan(const or_config *c, const int32_t *topk,
 out:
     free(Hl); free(X); free(D); free(shed); free(keep); free(order); free(pieces);
     free(recv); free(PS); free(QS); free(nrep_on); free(rep_ord); free(hosts); free(gcount);
+    free(src_count); free(src_seen);
     return rc;
 }
 

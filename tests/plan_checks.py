@@ -17,7 +17,9 @@ ST_EXPERT_ID_RANGE, ST_OVERFLOW, ST_STRICT = 1, 2, 4
 
 def check_invariants(cfg, topk, p) -> dict:
     """Assert the constraints the pages fix plus the structural properties of
-    the water-filling plan.  Returns a few derived quantities."""
+    the water-filling plan (with the locality flag, of its host intervals).
+    Returns a few derived quantities."""
+    locality = bool(getattr(cfg, "flags", 0) & 16)
     R, E, K, S, B = cfg.R, cfg.E, cfg.K, cfg.S, cfg.B
     L, C = E // R, S * K
     topk = np.asarray(topk).reshape(R * S, K)
@@ -69,14 +71,21 @@ def check_invariants(cfg, topk, p) -> dict:
         ranks = [int(p["host_rank"][h]) for h in hs]
         assert ranks == sorted(ranks) and len(set(ranks)) == len(ranks)
         assert e // L in ranks
-        start = 0
+        start, n_loc = 0, 0
         for h in hs:
             assert p["host_start"][h] == start
             r, s = int(p["host_rank"][h]), int(p["host_slot"][h])
             assert p["slot_expert"][r, s] == e
-            assert p["host_quota"][h] == p["slot_count"][r, s]
-            start += int(p["host_quota"][h])
-        assert start == T[e]
+            q = int(p["host_quota"][h])
+            assert q == p["slot_count"][r, s]
+            loc = int(p["host_local"][h])
+            if locality:  # its own rank's pairs first, as many as its quota takes
+                assert loc == min(q, int((topk[r * S:(r + 1) * S] == e).sum()))
+            else:
+                assert loc == 0
+            start += q - loc
+            n_loc += loc
+        assert start + n_loc == T[e]
 
     # pair placement: every pair on a rank hosting its expert; row_src is the
     # inverse permutation; each slot holds its expert's pairs in (t, k) order
@@ -98,15 +107,33 @@ def check_invariants(cfg, topk, p) -> dict:
         m = r_rank == r
         r_slot[m] = np.searchsorted(so[r], row[m] % C, side="right") - 1
     same = (r_rank[1:] == r_rank[:-1]) & (r_slot[1:] == r_slot[:-1])
-    assert (rs[1:][same] > rs[:-1][same]).all(), "slot rows not in (t, k) order"
-    # for each expert, destination ranks are non-decreasing over (t, k)
-    flat = topk.ravel()
-    by_e = np.argsort(flat, kind="stable")
-    same_e = flat[by_e][1:] == flat[by_e][:-1]
-    assert (np.diff(d_rank[by_e])[same_e] >= 0).all()
+    src_rank = (np.arange(R * S * K) // K) // S
+    if not locality:
+        assert (rs[1:][same] > rs[:-1][same]).all(), "slot rows not in (t, k) order"
+        # for each expert, destination ranks are non-decreasing over (t, k)
+        flat = topk.ravel()
+        by_e = np.argsort(flat, kind="stable")
+        same_e = flat[by_e][1:] == flat[by_e][:-1]
+        assert (np.diff(d_rank[by_e])[same_e] >= 0).all()
+    else:
+        # a slot holds its own rank's pairs first, then leftover pairs, each
+        # part in (t, k) order; the local pairs are exactly those
+        local_row = src_rank[rs] == r_rank
+        part_same = same & (local_row[1:] == local_row[:-1])
+        assert (rs[1:][part_same] > rs[:-1][part_same]).all(), "slot parts not in (t, k) order"
+        starts = np.r_[True, ~same]
+        # no local row after a leftover row within a slot
+        seen_left = False
+        for i in range(R * C):
+            if starts[i]:
+                seen_left = False
+            if not local_row[i]:
+                seen_left = True
+            else:
+                assert not seen_left, "a local pair after a leftover pair in a slot"
+        assert int(local_row.sum()) == int(p["host_local"].sum())
 
     # remote-pair statistic
-    src_rank = (np.arange(R * S * K) // K) // S
     assert info[7] == int((src_rank != d_rank).sum())
 
     # reduce work list: experts with a prefetched replica, ascending

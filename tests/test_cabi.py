@@ -32,7 +32,7 @@ def test_library_exports_every_declared_symbol(cuda_lib_path):
 
 def test_binding_loads(cuda_lib_path):
     from load_balancing_moonep_b200 import moonep
-    assert moonep.abi_version() == 1
+    assert moonep.abi_version() == 2
     for n in _declared():
         assert n in moonep.EXPORTED
 
@@ -104,3 +104,18 @@ def test_status_string(cuda_lib_path):
     small = ctypes.create_string_buffer(6)
     assert lib.moonep_status_string(3, small, 6) == b"EXPER"  # truncated, NUL-terminated
     assert lib.moonep_status_string(3, None, 0) == b""
+
+
+def test_single_gpu_planner_refuses_the_locality_flag(cuda_lib_path):
+    """MOONEP_FLAG_LOCALITY is for expert parallelism (moonep_ep_plan): the
+    one-GPU planner refuses it before touching memory."""
+    import ctypes
+    from load_balancing_moonep_b200 import moonep
+    cfg = moonep.Config(R=4, E=16, K=2, S=8, H=8, B=2, flags=moonep.FLAG_LOCALITY)
+    assert moonep.check_config(cfg) == 0
+    cp = moonep._CPlan()
+    for f in moonep.PLAN_FIELDS:  # non-null stand-ins: the call must not touch them
+        setattr(cp, f, 1 << 20)
+    c = cfg.c()
+    assert moonep._lib.moonep_plan(ctypes.byref(c), 1 << 20, ctypes.byref(cp), 1 << 20, None) == 1
+    assert moonep._lib.moonep_plan_noalloc(ctypes.byref(c), 1 << 20, ctypes.byref(cp), None) == 1

@@ -26,7 +26,8 @@ from load_balancing_moonep_b200 import workloads as W
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
 TABLES = ("expert_count", "slot_expert", "slot_count", "slot_offset", "rep_expert", "rep_rank", "rep_slot",
-          "rep_quota", "host_ptr", "host_rank", "host_slot", "host_start", "host_quota", "rep_home_list")
+          "rep_quota", "host_ptr", "host_rank", "host_slot", "host_start", "host_quota", "rep_home_list",
+          "host_local")
 
 
 @pytest.fixture(scope="module")
@@ -148,6 +149,32 @@ def test_ep_plan_and_data_match_the_oracle(mp, wname, mv, flags):
     plans, counts_all = _ep_plans(mp, cfg, r.topk_idx)
     _check_plans(cfg, plans, counts_all, topk_np, op)
     _ranks_data_check(mp, cfg, ocfg, plans, op, r.weights, P=1000 if wname != "decode" else 64)
+
+
+@pytest.mark.parametrize("wname,mv,flags", [("tiny", 1.0, 16), ("mid", 2.0, 16), ("mid", 3.0, 16 | 8),
+                                            ("decode", 13.4, 16), ("ep8", 20.0, 16)])
+def test_ep_locality_plan_and_data_match_the_oracle(mp, wname, mv, flags):
+    """MOONEP_FLAG_LOCALITY (with the relay cascade too on one case): every
+    rank's tables, including host_local and the leftover starts, the rows of
+    its pairs, and the data steps through the per-rank buffers, against the
+    oracle; and the ranks keep on their source rank exactly the pairs the
+    oracle does, never fewer than without the flag."""
+    wl = W.WORKLOADS[wname]
+    c = dict(R=wl.R, E=wl.E, K=wl.K, S=wl.S, H=wl.H, B=wl.B, flags=flags)
+    if wname == "ep8":
+        c["S"], c["H"] = 512, 256
+        wl = wl.with_(S=512, H=256)
+    if flags & 8:
+        c["B"] = 1
+    cfg, ocfg = mp.Config(**c), oracle.Config(**c)
+    r = W.routing(wl, mv, device=DEV)
+    topk_np = r.topk_idx.cpu().numpy()
+    op = oracle.plan(ocfg, topk_np)
+    op0 = oracle.plan(oracle.Config(**{**c, "flags": flags & ~16}), topk_np)
+    assert op["info"][7] <= op0["info"][7]
+    plans, counts_all = _ep_plans(mp, cfg, r.topk_idx)
+    _check_plans(cfg, plans, counts_all, topk_np, op)
+    _ranks_data_check(mp, cfg, ocfg, plans, op, r.weights, P=256 if wname != "decode" else 64)
 
 
 def test_ep_plan_large_training_shape(mp):

@@ -134,6 +134,8 @@ GOLDEN_B = [("test_golden_plan", {"name": "plan_example_b"})]
 CASCADE_PINS = [("test_golden_cascade_plan", {"name": "plan_example_cascade", "over_greedy": 3}),
                 ("test_golden_cascade_plan", {"name": "plan_example_cascade_merge", "over_greedy": 2}),
                 ("test_golden_cascade_plan", {"name": "plan_example_cascade_chain", "over_greedy": 3})]
+LOCALITY_PINS = [("test_golden_locality_plan", {}),
+                 ("test_locality_reaches_the_bound_for_its_placement", {"wname": "mid", "mv": 2.0})]
 CORE_MUTANTS = {
     "O3 sheds the smallest experts first": (
         [("qsort(order, (size_t)L, sizeof(vi_t), cmp_val_desc_idx_asc);",
@@ -164,11 +166,11 @@ CORE_MUTANTS = {
         [("        qsort(hosts, (size_t)nh, sizeof(host_t), cmp_host_rank);\n",
           "        qsort(hosts, (size_t)nh, sizeof(host_t), cmp_host_rank_desc);\n")], GOLDEN_A),
     "O8 pairs in (k, t) order": (
-        [("    for (int64_t p = 0; p < NP; ++p) {\n        int32_t e = topk[p];\n        int32_t g = gcount[e]++;",
+        [("    for (int64_t p = 0; p < NP; ++p) {\n        const int32_t e = topk[p];\n        const int32_t g = gcount[e]++;",
           "    for (int64_t pp = 0; pp < NP; ++pp) {\n        int64_t p = (pp % ((int64_t)R * S)) * K + pp / ((int64_t)R * S);\n"
-          "        int32_t e = topk[p];\n        int32_t g = gcount[e]++;")], GOLDEN_B),
+          "        const int32_t e = topk[p];\n        const int32_t g = gcount[e]++;")], GOLDEN_B),
     "remote pairs: source rank without dividing by K": (
-        [("        int64_t src_rank = (p / K) / S;", "        int64_t src_rank = p / S;")], GOLDEN_B),
+        [("        if (s_rank != r) ++n_remote;", "        if ((int32_t)(p / S) != r) ++n_remote;")], GOLDEN_B),
     "overflow only above B": (
         [("        if (rep_ord[q] >= B) ++n_over;", "        if (rep_ord[q] > B) ++n_over;")], GOLDEN_B),
     "work list includes overflow replicas": (
@@ -244,20 +246,20 @@ CORE_MUTANTS = {
           "            acc += slot_count[(int64_t)r * E + s];\n            slot_offset[(int64_t)r * (E + 1) + s] = (int32_t)acc;")],
         GOLDEN_A),
     "O7 host starts not accumulated": (
-        [("            start += hosts[h].quota;", "")], GOLDEN_A),
+        [("            start += q - loc;", "")], GOLDEN_A),
     "O8 host interval closed at its end": (
-        [("if (host_start[h] <= g && g < host_start[h] + host_quota[h]) { found = h; break; }",
-          "if (host_start[h] <= g && g <= host_start[h] + host_quota[h]) { found = h; break; }")], GOLDEN_A),
+        [("if (host_start[h] <= u && u < host_start[h] + host_quota[h] - host_local[h]) {",
+          "if (host_start[h] <= u && u <= host_start[h] + host_quota[h] - host_local[h]) {")], GOLDEN_A),
     "O8 row without the slot offset": (
-        [("        int64_t d = (int64_t)r * C + slot_offset[(int64_t)r * (E + 1) + host_slot[found]] +\n                    (g - host_start[found]);",
-          "        int64_t d = (int64_t)r * C + (g - host_start[found]);")], GOLDEN_A),
+        [("        int64_t d = (int64_t)r * C + slot_offset[(int64_t)r * (E + 1) + host_slot[found]] + off;",
+          "        int64_t d = (int64_t)r * C + off;")], GOLDEN_A),
     "O8 row without subtracting the host start": (
-        [("        int64_t d = (int64_t)r * C + slot_offset[(int64_t)r * (E + 1) + host_slot[found]] +\n                    (g - host_start[found]);",
-          "        int64_t d = (int64_t)r * C + slot_offset[(int64_t)r * (E + 1) + host_slot[found]] + g;")], GOLDEN_A),
+        [("                    off = host_local[h] + (u - host_start[h]);", "                    off = host_local[h] + u;")],
+        GOLDEN_A),
     "row_src names the token instead of the pair": (
         [("        row_src[d] = (int32_t)p;", "        row_src[d] = (int32_t)(p / K);")], GOLDEN_B),
     "remote pairs never counted": (
-        [("        if (src_rank != r) ++n_remote;", "")], GOLDEN_A),
+        [("        if (s_rank != r) ++n_remote;", "")], GOLDEN_A),
     "largest replica count only over B": (
         [("        if (nrep_on[r] > max_rep) max_rep = nrep_on[r];",
           "        if (nrep_on[r] > max_rep && nrep_on[r] > B) max_rep = nrep_on[r];")], GOLDEN_A),
@@ -275,6 +277,25 @@ CORE_MUTANTS = {
     "prefetch pool row strided by L instead of B": (
         [("                    row = E + r * B + b;", "                    row = E + r * L + b;")],
         [("test_prefetch_budget_above_L", {})]),
+    "locality takes the whole quota locally": (
+        [("const int32_t loc = locality ? (int32_t)min64(q, src_count[(int64_t)hosts[h].rank * E + e]) : 0;",
+          "const int32_t loc = locality ? q : 0;")], LOCALITY_PINS),
+    "locality counts the next rank's pairs": (
+        [("const int32_t loc = locality ? (int32_t)min64(q, src_count[(int64_t)hosts[h].rank * E + e]) : 0;",
+          "const int32_t loc = locality ? (int32_t)min64(q, src_count[(int64_t)((hosts[h].rank + 1) % R) * E + e]) : 0;")],
+        LOCALITY_PINS),
+    "leftover starts count the whole quota": (
+        [("            start += q - loc;", "            start += q;")], LOCALITY_PINS),
+    "local pairs before a pair leave out its own rank": (
+        [("if (host_rank[h] <= s_rank) before += host_local[h];", "if (host_rank[h] < s_rank) before += host_local[h];")],
+        LOCALITY_PINS),
+    "leftover offset without the local rows": (
+        [("                    off = host_local[h] + (u - host_start[h]);", "                    off = (u - host_start[h]);")],
+        LOCALITY_PINS),
+    "local test on the expert-wide index": (
+        [("        if (own >= 0 && gs < host_local[own]) {\n            found = own;\n            off = gs;",
+          "        if (own >= 0 && g < host_local[own]) {\n            found = own;\n            off = g;")],
+        LOCALITY_PINS),
     "bf16 NaN truncated without forcing the quiet bit": (
         [("        return (uint16_t)((u >> 16) | 0x0040u);", "        return (uint16_t)(u >> 16);")],
         [("test_bf16_nan_patterns", {})]),

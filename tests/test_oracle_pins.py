@@ -702,3 +702,55 @@ def test_openmp_build_computes_what_the_oracle_computes(oracle_lib):
     oracle.reduce_replica_grads(cfg, p, rb1, hg1, P)
     oracle.reduce_replica_grads(cfg, p, rb2, hg2, P, lib=olib)
     assert np.array_equal(hg1, hg2) and np.array_equal(rb1, rb2)
+
+
+# ------------------------------------------------- locality-aware intervals
+
+def test_golden_locality_plan(oracle_lib):
+    """The hand-worked locality plan (tests/golden/plan_example_locality.json):
+    hosts take their own rank's pairs first; the leftover pairs fill the
+    rest of the quotas in rank order.  Without the flag the same routing
+    keeps one pair fewer on its source rank."""
+    g = json.load(open(os.path.join(GOLDEN, "plan_example_locality.json")))
+    cfg = oracle.Config(**g["config"])
+    topk = np.array(g["topk_idx"], np.int32)
+    p = oracle.plan(cfg, topk)
+    for k, v in g["expect"].items():
+        if k == "info":
+            assert oracle.info_dict(p) == v
+        else:
+            assert p[k].tolist() == v, k
+    check_invariants(cfg, topk, p)
+    p0 = oracle.plan(oracle.Config(**{**g["config"], "flags": 0}), topk)
+    assert p0["dst_pos"].tolist() == g["without_flag"]["dst_pos"]
+    assert p0["info"][7] == g["without_flag"]["n_remote_pairs"]
+    for f in ("slot_expert", "slot_count", "slot_offset", "rep_expert", "rep_quota", "host_quota"):
+        assert np.array_equal(p[f], p0[f])
+
+
+@pytest.mark.parametrize("wname,mv", [("tiny", 1.0), ("mid", 2.0), ("ep8", 20.0), ("decode", 5.0)])
+def test_locality_reaches_the_bound_for_its_placement(oracle_lib, wname, mv):
+    """With the locality flag the pairs kept on their source rank are exactly
+    the most any interval choice can keep for the same replica placement,
+    sum over experts and hosts of min(host quota, the expert's pairs from the
+    host's rank); the placement and quotas are those of the plain plan, and
+    the plain plan never keeps more."""
+    wl = W.WORKLOADS[wname]
+    if wname == "ep8":
+        wl = wl.with_(S=1024)
+    c = dict(R=wl.R, E=wl.E, K=wl.K, S=wl.S, H=wl.H, B=wl.B)
+    topk = W.routing(wl, mv).topk_idx.numpy()
+    p = oracle.plan(oracle.Config(**c, flags=oracle.FLAG_LOCALITY), topk)
+    p0 = oracle.plan(oracle.Config(**c), topk)
+    check_invariants(oracle.Config(**c, flags=oracle.FLAG_LOCALITY), topk, p)
+    for f in ("slot_expert", "slot_count", "slot_offset", "rep_expert", "rep_rank", "rep_quota", "host_ptr",
+              "host_rank", "host_quota"):
+        assert np.array_equal(p[f], p0[f]), f
+    R, S, E = wl.R, wl.S, wl.E
+    src = np.stack([np.bincount(topk[r * S:(r + 1) * S].ravel(), minlength=E) for r in range(R)])
+    bound = 0
+    for e in range(E):
+        for h in range(p["host_ptr"][e], p["host_ptr"][e + 1]):
+            bound += min(int(p["host_quota"][h]), int(src[p["host_rank"][h], e]))
+    local, local0 = wl.pairs - int(p["info"][7]), wl.pairs - int(p0["info"][7])
+    assert local == bound >= local0

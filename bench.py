@@ -774,6 +774,33 @@ def run_ours(args, world, rank, local):
         einf = eplans[0].info()
         gd = bytes_dispatch(wl) / (pd * 1e-3) / 1e9
         gc = bytes_combine(wl) / (pc * 1e-3) / 1e9
+        # locality-aware intervals: the pairs kept on their source rank, with
+        # and without the flag, on the pages' EP = 8 shape at maxvio 20 and on
+        # this shape at maxvio 3 (plans only)
+        locality = []
+        for lname, lmv in (("ep8", 20.0), (wl.name, 3.0)):
+            lwl = W.WORKLOADS[lname]
+            lr = W.routing(lwl, lmv, seed=rank, device=dev)
+            row = {"workload": workload_name(lwl), "maxvio": round(lr.maxvio, 3)}
+            for lflags, key in ((0, "remote_pair_frac"), (mp.FLAG_LOCALITY, "remote_pair_frac_locality")):
+                lcfg = mp.Config(R=lwl.R, E=lwl.E, K=lwl.K, S=lwl.S, H=lwl.H, B=lwl.B, flags=lflags)
+                lps = [mp.Plan(lcfg, dev, ep=True) for _ in range(lwl.R)]
+                lca = torch.empty((lwl.R, lwl.E + 1), dtype=torch.int32, device=dev)
+                ltl = [lr.topk_idx[k * lwl.S:(k + 1) * lwl.S].contiguous() for k in range(lwl.R)]
+                torch.cuda.synchronize()
+                for k in range(lwl.R):
+                    mp.ep_count(lcfg, ltl[k], lps[k], counts_row=lca[k])
+                lt = Timer()
+                for k in range(lwl.R):
+                    e = lt.mark("plan") if k == 0 else None
+                    mp.ep_plan(lcfg, k, ltl[k], lca, lps[k])
+                    if e:
+                        e.record()
+                torch.cuda.synchronize()
+                row[key] = round(sum(q.info()["n_remote_pairs"] for q in lps) / lwl.pairs, 4)
+                row["plan_us" + ("_locality" if lflags else "")] = round(lt.total_ms("plan") * 1e3, 2)
+                del lps
+            locality.append(row)
         ep = {"what": (f"{wl.R} ranks on one GPU: each rank's ep_count and ep_plan (rank 0 timed), then "
                        f"{wl.R} ep_dispatch and {wl.R} ep_combine launches through per-rank row pointers"),
               "count_us": round(et.total_ms("count") / it * 1e3, 2),
@@ -781,7 +808,7 @@ def run_ours(args, world, rank, local):
               "dispatch_GB/s": round(gd, 1), "combine_GB/s": round(gc, 1),
               "dispatch_frac": round(gd / peak, 4), "combine_frac": round(gc / peak, 4),
               "rank0_remote_pair_frac": round(einf["n_remote_pairs"] / (wl.S * wl.K), 4),
-              "status": einf["status"]}
+              "status": einf["status"], "locality": locality}
         del eplans, bptr
 
     # the CPU oracle on a bounded sample (rank 0, one GPU only): the

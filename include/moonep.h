@@ -416,6 +416,16 @@ MOONEP_API const char *moonep_status_string(int status, char *buf, size_t len);
  * launched with. */
 MOONEP_API int moonep_set_wait_limit(int iterations);
 
+/* The replica capacity the relay cascade's guard (MOONEP_FLAG_CASCADE)
+ * compares with, for every moonep_plan / moonep_ep_plan call this process
+ * makes afterwards: a repair step that could leave more live replicas than
+ * this is not taken.  Default (capacity <= 0): the plan's E + R - 1, which
+ * no tested routing comes within 3 of.  A smaller value only makes the
+ * guard stricter (the plan's arrays keep their size), so tests use it to put
+ * a step exactly on the limit and one over it.  Host-only; returns the
+ * previous setting (0 for the default). */
+MOONEP_API int moonep_set_cascade_capacity(int capacity);
+
 /* MOONEP_ABI_VERSION of the loaded library. */
 MOONEP_API int moonep_abi_version(void);
 

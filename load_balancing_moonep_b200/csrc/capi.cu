@@ -10,6 +10,7 @@
 namespace moonep {
 int launch_plan(const Dims &d, const int32_t *topk, const moonep_plan_t &p, void *ws, cudaStream_t st);
 int set_wait_limit(int iterations);
+int set_cascade_capacity(int c);
 size_t plan_smem_bytes_max(const Dims &d);
 int launch_dispatch(const Dims &d, const int *dst_pos, int *info, const uint16_t *hidden, uint16_t *buf,
                     cudaStream_t st);
@@ -180,6 +181,8 @@ extern "C" {
 int moonep_abi_version(void) { return MOONEP_ABI_VERSION; }
 
 int moonep_set_wait_limit(int iterations) { return set_wait_limit(iterations); }
+
+int moonep_set_cascade_capacity(int capacity) { return set_cascade_capacity(capacity); }
 
 const char *moonep_error_string(int code)
 {

@@ -67,6 +67,7 @@ struct PlanParams {
     int *host_dst0;  // [2E+R]
     FastDiv fC, fL;  // divisions by C and L
     int spin_limit;  // iterations of each bounded wait of the assignment pass
+    int cascade_cap; // the relay cascade guard's replica capacity: E + R - 1, or less in a test
 };
 
 // The bound of the assignment pass's two waits, for every later launch in
@@ -76,6 +77,21 @@ static std::atomic<int> g_wait_limit{READY_SPIN_LIMIT};
 int set_wait_limit(int iterations)
 {
     return g_wait_limit.exchange(iterations < 0 ? READY_SPIN_LIMIT : iterations);
+}
+
+// The replica capacity the cascade's guard compares with, for every later
+// launch (moonep_set_cascade_capacity): the plan's E + R - 1 by default.
+static std::atomic<int> g_cascade_cap{0};
+
+int set_cascade_capacity(int c)
+{
+    return g_cascade_cap.exchange(c > 0 ? c : 0);
+}
+
+static int cascade_cap_for(const Dims &d)
+{
+    const int full = d.E + d.R - 1, c = g_cascade_cap.load(std::memory_order_relaxed);
+    return c > 0 && c < full ? c : full;
 }
 
 // ints of dynamic shared memory used by the planner block
@@ -177,7 +193,7 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
     const int E = d.E, R = d.R, L = d.L, C = d.C, B = d.B;
     const int tid = threadIdx.x;
     constexpr int nt = PLAN_THREADS;
-    const int cap = E + R - 1, lc = cascade_list_cap(E, R), nh = 2 * E + R;
+    const int cap = a.cascade_cap, lc = cascade_list_cap(E, R), nh = 2 * E + R;
     int *le = cz, *lr = le + lc, *lq = lr + lc, *la = lq + lc;  // list: expert, rank, quota, alive
     int *ordx = la + lc;                                          // a rank's replicas in step order
     int *me = ordx + lc, *mq = me + lc;                           // their experts and quotas
@@ -1402,6 +1418,7 @@ int launch_plan(const Dims &d, const int32_t *topk, const moonep_plan_t &p, void
     a.fC = make_fastdiv((uint32_t)d.C);
     a.fL = make_fastdiv((uint32_t)d.L);
     a.spin_limit = g_wait_limit.load(std::memory_order_relaxed);
+    a.cascade_cap = cascade_cap_for(d);
 
     // both kernels with programmatic dependent launch: each may be placed
     // while its predecessor drains and waits (griddepcontrol.wait, or the
@@ -1741,6 +1758,7 @@ int launch_ep_plan(const Dims &d, int rank, const int32_t *topk, const int32_t *
     a.fC = make_fastdiv((uint32_t)d.C);
     a.fL = make_fastdiv((uint32_t)d.L);
     a.spin_limit = 0;
+    a.cascade_cap = cascade_cap_for(d);
 
     const size_t smem1 = sizeof(int) * (size_t)(plan_smem_ints(d.E, d.R) +
                                                 ((d.flags & MOONEP_FLAG_CASCADE) ? cascade_smem_ints(d.E, d.R, d.B) : 0));

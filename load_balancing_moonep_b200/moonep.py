@@ -58,7 +58,7 @@ EXPORTED = ("moonep_check_config", "moonep_plan_sizes", "moonep_plan_layout", "m
             "moonep_plan_noalloc", "moonep_prefetch_replicas", "moonep_status_string",
             "moonep_set_wait_limit", "moonep_ep_sizes", "moonep_ep_count", "moonep_ep_plan",
             "moonep_ep_dispatch", "moonep_ep_combine", "moonep_ep_combine_backward",
-            "moonep_ep_reduce_replica_grads", "moonep_ep_prefetch_replicas")
+            "moonep_ep_reduce_replica_grads", "moonep_ep_prefetch_replicas", "moonep_set_cascade_capacity")
 
 
 class _CConfig(ctypes.Structure):
@@ -90,6 +90,7 @@ _lib.moonep_status_string.argtypes = [ctypes.c_int, ctypes.c_char_p, ctypes.c_si
 _lib.moonep_status_string.restype = ctypes.c_char_p
 _lib.moonep_abi_version.argtypes = []
 _lib.moonep_set_wait_limit.argtypes = [ctypes.c_int]
+_lib.moonep_set_cascade_capacity.argtypes = [ctypes.c_int]
 _lib.moonep_ep_sizes.argtypes = [_cfgp, ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)]
 _lib.moonep_ep_count.argtypes = [_cfgp, _vp, _vp, _vp, _vp]
 _lib.moonep_ep_plan.argtypes = [_cfgp, ctypes.c_int32, _vp, _vp, _planp, _vp, _vp]
@@ -517,6 +518,14 @@ def set_wait_limit(iterations: int) -> int:
     0 makes both waits take their fallback (MOONEP_ST_WAIT_TIMEOUT set, plan
     still exact)."""
     return _lib.moonep_set_wait_limit(int(iterations))
+
+
+def set_cascade_capacity(capacity: int) -> int:
+    """The replica capacity the relay cascade's guard compares with for later
+    plan calls (<= 0: the plan's E + R - 1); returns the previous setting
+    (0 for the default).  Lowering it makes the guard stricter; tests use it
+    to put a repair step exactly on the limit."""
+    return _lib.moonep_set_cascade_capacity(int(capacity))
 
 
 def abi_version() -> int:

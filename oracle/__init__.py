@@ -113,6 +113,8 @@ def _bind(lib):
         lib.or_f32_to_bf16.restype = ctypes.c_uint16
         lib.or_omp_threads.argtypes = [ctypes.c_int]
         lib.or_omp_threads.restype = ctypes.c_int
+        lib.or_set_cascade_capacity.argtypes = [ctypes.c_int32]
+        lib.or_set_cascade_capacity.restype = ctypes.c_int32
     return lib
 
 
@@ -208,6 +210,13 @@ def plan(cfg: Config, topk_idx: np.ndarray) -> dict:
                      _p(out["row_src"]), _p(out["info"]))
     _check(rc)
     return out
+
+
+def set_cascade_capacity(c: int) -> int:
+    """Lower the replica capacity the relay cascade's guard compares with
+    (c <= 0: the plan's E + R - 1); returns the previous setting (0 for the
+    default).  For tests that put a cascade step exactly on the limit."""
+    return int(_load().or_set_cascade_capacity(int(c)))
 
 
 def info_dict(p: dict) -> dict:

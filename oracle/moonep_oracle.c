@@ -199,6 +199,18 @@ static int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
  * order (dead entries are dropped after each step); ordinals are re-derived
  * by the caller.  re/rr/rq/alive: list arrays of capacity
  * lcap >= 2 * cap + 2 * B + 2; *nl: entries used. */
+/* The capacity the cascade's guard compares with: the plan's E + R - 1
+ * replica entries, or less when a test lowers it (or_set_cascade_capacity)
+ * to put a step exactly on the limit. */
+static int32_t or_cascade_cap_limit = INT32_MAX;
+
+int32_t or_set_cascade_capacity(int32_t c)
+{
+    const int32_t prev = or_cascade_cap_limit;
+    or_cascade_cap_limit = c > 0 ? c : INT32_MAX;
+    return prev == INT32_MAX ? 0 : prev;
+}
+
 static int or_cascade(int32_t R, int32_t E, int32_t L, int32_t B, int32_t cap, int32_t *keep,
                       int32_t *re, int32_t *rr, int32_t *rq, int32_t *alive, int32_t *nl, int32_t lcap,
                       int32_t *n_guard, int32_t *min_slack)
@@ -476,7 +488,8 @@ int or_plan(const or_config *c, const int32_t *topk,
             }
             for (int32_t q = 0; q < nrep; ++q) { le[q] = rep_expert[q]; lr[q] = rep_rank[q]; lq[q] = rep_quota[q]; la[q] = 1; }
             int32_t nl = nrep;
-            rc = or_cascade(R, E, L, B, NREP_MAX - 1, keep, le, lr, lq, la, &nl, lcap, &n_guard, &min_slack);
+            const int32_t cap = NREP_MAX - 1 < or_cascade_cap_limit ? NREP_MAX - 1 : or_cascade_cap_limit;
+            rc = or_cascade(R, E, L, B, cap, keep, le, lr, lq, la, &nl, lcap, &n_guard, &min_slack);
             if (rc == OR_OK) {
                 /* the final list, ordinals re-derived in list order */
                 for (int32_t r = 0; r < R; ++r) nrep_on[r] = 0;

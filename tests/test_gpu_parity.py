@@ -229,6 +229,28 @@ def test_plan_cascade_golden(mp, name):
             assert gp.fields[k].cpu().numpy().tolist() == v, k
 
 
+@pytest.mark.parametrize("name,caps", [("plan_example_cascade", (4, 3)),
+                                       ("plan_example_cascade_chain", (5, 6, 7)),
+                                       ("plan_example_cascade_merge", (4, 5))])
+def test_plan_cascade_guard_at_lowered_capacities(mp, name, caps):
+    """The cascade guard's comparison on the GPU: with the capacity lowered in
+    both the CUDA planner and the oracle, steps exactly on the limit are
+    taken and steps one over are skipped, identically, whole plan."""
+    g = json.load(open(os.path.join(GOLDEN, name + ".json")))
+    topk = np.array(g["topk_idx"], np.int32)
+    try:
+        for cap in caps:
+            mp.set_cascade_capacity(cap)
+            oracle.set_cascade_capacity(cap)
+            gcfg, ocfg, gp, op = _plan_both(mp, g["config"], topk)
+            _assert_plan_equal(gp, op)
+            if name == "plan_example_cascade":
+                assert op["info"][9] == (0 if cap == 4 else -1)
+    finally:
+        mp.set_cascade_capacity(0)
+        oracle.set_cascade_capacity(0)
+
+
 def test_plan_cascade_counterexample_and_data(mp):
     """The 31-replica counterexample: the cascade's plan, then dispatch and
     combine over it, element for element against the oracle."""

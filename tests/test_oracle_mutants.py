@@ -16,11 +16,11 @@ The cascade's capacity guard (a step is skipped when the live list plus
 m + B - 1 would exceed E + R - 1) is pinned in two parts.  Its arithmetic:
 the slack it computes is reported in the plan's info, hand-worked in every
 cascade golden, so the mutants below that change the sum or the capacity are
-caught there.  Its comparison: on every routing of the small shapes that
-tests/test_oracle_pins.py enumerates exhaustively, the least slack any step
-reaches is 3, so moving the threshold by one or two either way (taking the
-step at a slack of -1 or -2, refusing it at 0 or 1) gives the same plan on
-all of them; those variants are not planted.
+caught there.  Its comparison: with the capacity lowered (a test setting of
+both the oracle and the CUDA planner), the hand-worked plan_example_cascade
+puts its one step exactly on the limit and one over it, so a threshold moved
+either way is caught (on every routing the tests enumerate the default
+capacity leaves a slack of at least 3).
 
 Not pinned, with the reason:
 * water-filling loops nested receiver-major instead of piece-major: an
@@ -134,6 +134,7 @@ GOLDEN_B = [("test_golden_plan", {"name": "plan_example_b"})]
 CASCADE_PINS = [("test_golden_cascade_plan", {"name": "plan_example_cascade", "over_greedy": 3}),
                 ("test_golden_cascade_plan", {"name": "plan_example_cascade_merge", "over_greedy": 2}),
                 ("test_golden_cascade_plan", {"name": "plan_example_cascade_chain", "over_greedy": 3})]
+GUARD_PINS = [("test_cascade_guard_threshold_at_and_over_a_lowered_capacity", {})]
 LOCALITY_PINS = [("test_golden_locality_plan", {}),
                  ("test_locality_reaches_the_bound_for_its_placement", {"wname": "mid", "mv": 2.0})]
 CORE_MUTANTS = {
@@ -277,6 +278,15 @@ CORE_MUTANTS = {
     "prefetch pool row strided by L instead of B": (
         [("                    row = E + r * B + b;", "                    row = E + r * L + b;")],
         [("test_prefetch_budget_above_L", {})]),
+    "cascade guard refuses a step at zero slack": (
+        [("        if (slack < 0) continue; /* the list could outgrow the plan's arrays */",
+          "        if (slack <= 0) continue; /* the list could outgrow the plan's arrays */")], GUARD_PINS),
+    "cascade guard takes a step one over the capacity": (
+        [("        if (slack < 0) continue; /* the list could outgrow the plan's arrays */",
+          "        if (slack < -1) continue; /* the list could outgrow the plan's arrays */")], GUARD_PINS),
+    "cascade guard ignores a lowered capacity": (
+        [("            const int32_t cap = NREP_MAX - 1 < or_cascade_cap_limit ? NREP_MAX - 1 : or_cascade_cap_limit;",
+          "            const int32_t cap = NREP_MAX - 1;")], GUARD_PINS),
     "locality takes the whole quota locally": (
         [("const int32_t loc = locality ? (int32_t)min64(q, src_count[(int64_t)hosts[h].rank * E + e]) : 0;",
           "const int32_t loc = locality ? q : 0;")], LOCALITY_PINS),

@@ -754,3 +754,46 @@ def test_locality_reaches_the_bound_for_its_placement(oracle_lib, wname, mv):
             bound += min(int(p["host_quota"][h]), int(src[p["host_rank"][h], e]))
     local, local0 = wl.pairs - int(p["info"][7]), wl.pairs - int(p0["info"][7])
     assert local == bound >= local0
+
+
+def test_cascade_guard_threshold_at_and_over_a_lowered_capacity(oracle_lib):
+    """The guard's comparison, pinned by lowering the capacity it compares
+    with (the default E + R - 1 is never reached by a tested routing): in the
+    hand-worked plan_example_cascade the one repair step may leave 4 live
+    replicas.  At capacity 4 (slack 0) the step is taken and the plan is the
+    golden one; at capacity 3 (slack -1) it is not, and the plan is
+    water-filling's (the derivation is in the golden file)."""
+    g = json.load(open(os.path.join(GOLDEN, "plan_example_cascade.json")))
+    cfg = oracle.Config(**g["config"])
+    topk = np.array(g["topk_idx"], np.int32)
+    plain = oracle.plan(oracle.Config(**{**g["config"], "flags": 0}), topk)
+    at, over = g["capacity_checks"]["at_limit"], g["capacity_checks"]["one_over"]
+    try:
+        oracle.set_cascade_capacity(at["capacity"])
+        p = oracle.plan(cfg, topk)
+        for k, v in g["expect"].items():
+            if k == "info":
+                inf = oracle.info_dict(p)
+                assert {f: inf[f] for f in v if f != "cascade_guard_slack"} == \
+                    {f: v[f] for f in v if f != "cascade_guard_slack"}
+                assert inf["cascade_guard_steps"] == at["cascade_guard_steps"]
+                assert inf["cascade_guard_slack"] == at["cascade_guard_slack"]
+            else:
+                assert p[k].tolist() == v, k
+        oracle.set_cascade_capacity(over["capacity"])
+        q = oracle.plan(cfg, topk)
+        n = len(over["rep_expert"])
+        for f in ("rep_expert", "rep_rank", "rep_slot", "rep_quota"):
+            assert q[f][:n].tolist() == over[f], f
+        inf = oracle.info_dict(q)
+        assert (inf["status"], inf["n_overflow"], inf["max_rep_per_rank"]) == \
+            (over["status"], over["n_overflow"], over["max_rep_per_rank"])
+        assert (inf["cascade_guard_steps"], inf["cascade_guard_slack"]) == \
+            (over["cascade_guard_steps"], over["cascade_guard_slack"])
+        for k in plain:  # a skipped step leaves water-filling's plan
+            if k != "info":
+                assert np.array_equal(q[k], plain[k]), k
+        assert np.array_equal(q["info"][:8], plain["info"][:8])
+    finally:
+        oracle.set_cascade_capacity(0)
+    assert oracle.info_dict(oracle.plan(cfg, topk))["cascade_guard_slack"] == 7

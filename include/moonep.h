@@ -114,14 +114,17 @@ extern "C" {
 /* A buffer row taken from the plan was outside [0, R*S*K) (a corrupted or
  * mismatched plan); that row access was skipped. */
 #define MOONEP_ST_ROW_RANGE 8
-/* A bounded wait inside a kernel ran out of iterations: one of the
- * assignment pass's waits for a mark of the histogram/planner pass (counts
- * ready, plan ready; about 6 ms at the bound).  The pass then waits for the
- * whole histogram grid instead, so the plan is still complete; the bit
- * reports that a mark never came, which points at a workspace used by two
- * overlapping calls.  A relay cascade (MOONEP_FLAG_CASCADE), which can run
- * for milliseconds, announces itself and is waited for the same way without
- * setting this bit. */
+/* A bounded wait inside a kernel ran out of iterations (about 6 ms at the
+ * bound).  In the two-kernel planner: one of the assignment pass's waits for
+ * a mark of the histogram/planner pass (counts ready, plan ready); the pass
+ * then waits for the whole histogram grid instead.  In the one-kernel
+ * planner: a CTA's wait for every chunk's counts (its peers were not all
+ * resident, e.g. because another stream's kernels held SMs); that CTA then
+ * counts every pair of the call itself.  Either way the plan is still
+ * complete and exact; the bit reports the slow path, or a workspace used by
+ * two overlapping calls.  A relay cascade (MOONEP_FLAG_CASCADE), which can
+ * run for milliseconds, announces itself in the two-kernel planner and is
+ * waited for the same way without setting this bit. */
 #define MOONEP_ST_WAIT_TIMEOUT 16
 /* The planner workspace did not hold the zeros a call must start from (it
  * was not zero-filled before first use, or two calls used it at once): the
@@ -214,7 +217,13 @@ MOONEP_API int moonep_plan_layout(const moonep_config *cfg, void *plan_base, moo
  *     dst_pos = rank*S*K + slot_offset[rank][slot] + (g - host_start)
  *   where g is the pair's rank among earlier pairs of the same expert.
  * plan: laid out by moonep_plan_layout; workspace: workspace_bytes bytes,
- * zero-filled before the first call.  Two kernel launches. */
+ * zero-filled before the first call.
+ * One kernel launch when all of its CTAs (one per token chunk, at most two
+ * per SM) fit on the device at once: every CTA counts its chunk, waits
+ * (bounded) for the others' counts, computes the whole plan in its own
+ * shared memory and places its own pairs.  Otherwise (shapes whose planner
+ * needs more shared memory) two launches: a histogram pass whose last CTA
+ * plans, and an assignment pass.  Both give the same plan, bit for bit. */
 MOONEP_API int moonep_plan(const moonep_config *cfg, const int32_t *topk_idx, const moonep_plan_t *plan,
                 void *workspace, void *stream);
 
@@ -404,17 +413,26 @@ MOONEP_API const char *moonep_error_string(int code);
  * empty static string when buf is NULL or len == 0.  Host-only. */
 MOONEP_API const char *moonep_status_string(int status, char *buf, size_t len);
 
-/* Iteration bound of the assignment pass's two bounded waits (for the
- * counts-ready and plan-ready marks of the histogram/planner pass; about
- * 100 ns per iteration) for every moonep_plan / moonep_plan_noalloc call
- * this process makes afterwards.  Default 65536; a negative value restores
- * it.  With 0 both waits give up at once: the pass then waits for the whole
- * histogram grid to finish (which that grid never depends on), so the plan
- * is still complete and exact, and MOONEP_ST_WAIT_TIMEOUT is set.  This is
- * how the fallback is tested without making a mark late.  Host-only; returns
- * the previous bound.  Calls already enqueued keep the bound they were
- * launched with. */
+/* Iteration bound of the planner's bounded waits (about 100 ns per
+ * iteration) for every moonep_plan / moonep_plan_noalloc call this process
+ * makes afterwards: the two-kernel path's waits for the counts-ready and
+ * plan-ready marks, the one-kernel path's wait for every chunk's counts.
+ * Default 65536; a negative value restores it.  With 0 every wait gives up at
+ * once and takes its fallback (the two-kernel path waits for the whole
+ * histogram grid, which never depends on it; a one-kernel CTA counts every
+ * pair itself), so the plan is still complete and exact, and
+ * MOONEP_ST_WAIT_TIMEOUT is set.  This is how the fallbacks are tested
+ * without making a mark late.  Host-only; returns the previous bound.  Calls
+ * already enqueued keep the bound they were launched with. */
 MOONEP_API int moonep_set_wait_limit(int iterations);
+
+/* Which planner moonep_plan / moonep_plan_noalloc launch afterwards in this
+ * process: 1 the two-kernel planner always; any other value (0, the
+ * default) the one-kernel planner wherever all of its CTAs fit on the device
+ * at once, else the two-kernel one.  Both give the same plan; tests use 1 to
+ * compare them.  A workspace may pass between the two.  Host-only; returns
+ * the previous setting (0 or 1). */
+MOONEP_API int moonep_set_plan_path(int mode);
 
 /* The replica capacity the relay cascade's guard (MOONEP_FLAG_CASCADE)
  * compares with, for every moonep_plan / moonep_ep_plan call this process

@@ -11,6 +11,7 @@ namespace moonep {
 int launch_plan(const Dims &d, const int32_t *topk, const moonep_plan_t &p, void *ws, cudaStream_t st);
 int set_wait_limit(int iterations);
 int set_cascade_capacity(int c);
+int set_plan_path(int mode);
 size_t plan_smem_bytes_max(const Dims &d);
 int launch_dispatch(const Dims &d, const int *dst_pos, int *info, const uint16_t *hidden, uint16_t *buf,
                     cudaStream_t st);
@@ -103,6 +104,7 @@ static int make_dims(const moonep_config *c, Dims *d, int nsm = B200_SMS)
     d->ngroups = (d->nchunk + CHUNK_GROUP - 1) / CHUNK_GROUP;
     d->ebits = 0;
     while ((1 << d->ebits) < d->E) ++d->ebits;
+    d->nsm = nsm;
     if (plan_smem_bytes_max(*d) > MAX_DYN_SMEM) return MOONEP_ERR_LIMIT;
     return MOONEP_OK;
 }
@@ -183,6 +185,8 @@ int moonep_abi_version(void) { return MOONEP_ABI_VERSION; }
 int moonep_set_wait_limit(int iterations) { return set_wait_limit(iterations); }
 
 int moonep_set_cascade_capacity(int capacity) { return set_cascade_capacity(capacity); }
+
+int moonep_set_plan_path(int mode) { return set_plan_path(mode); }
 
 const char *moonep_error_string(int code)
 {

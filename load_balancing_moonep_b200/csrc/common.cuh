@@ -21,6 +21,7 @@ struct Dims {
     int chunk_tokens;
     int ngroups;  // groups of CHUNK_GROUP consecutive chunks
     int ebits;    // bits of an expert id: 2^ebits >= E
+    int nsm;      // SMs the chunking targets (the launch device's, at most 148)
 };
 
 // Chunks per group: the assignment pass sums at most CHUNK_GROUP - 1
@@ -29,8 +30,8 @@ constexpr int CHUNK_GROUP = 16;
 
 // Workspace layout (bytes from the workspace base; 256-byte aligned parts).
 struct WsLayout {
-    size_t hdr;        // int32[8]: ticket, status, call sequence, counts-ready mark, arrivals, plan-ready mark,
-                       // slow-path mark
+    size_t hdr;        // int32[16]: ticket, status, call sequence, counts-ready mark, arrivals, plan-ready mark,
+                       // slow-path mark, late status bits, remote pairs
     size_t gs;         // int32 [2][ngroups][E]: per-group expert counts, double-buffered
     size_t cc;         // int32 [nchunk][E]: per-chunk expert counts
     size_t host_dst0;  // int32 [2E+R]: rank*C + slot_offset - host_start per host
@@ -45,9 +46,14 @@ struct WsLayout {
 // that the planner took a slow path (the relay cascade) whose length has no
 // useful bound for a spin: the assignment CTAs then wait for the whole
 // histogram grid instead.
+// The one-kernel planner uses TICKET, STATUS, SEQ and ARRIVED the same way
+// (TICKET: chunks whose counts are in; ARRIVED: CTAs done), and two words of
+// its own that the CTA finishing last folds into the info block: FLAGS (status
+// bits raised after the plan) and REMOTE (pairs placed off their source
+// rank).  It leaves READY == PLANNED == SEQ too, so either path may follow it.
 enum {
     WS_TICKET = 0, WS_STATUS = 1, WS_SEQ = 2, WS_READY = 3, WS_ARRIVED = 4, WS_PLANNED = 5, WS_SLOW = 6,
-    WS_HDR_INTS = 8
+    WS_FLAGS = 7, WS_REMOTE = 8, WS_HDR_INTS = 16
 };
 
 // Status bits after which every later call treats the plan as empty.
@@ -72,7 +78,7 @@ __host__ inline WsLayout ws_layout(const Dims &d)
 // (the count kernel's ticket and invalid-id count, the planner's status
 // word), this rank's per-chunk expert counts, and the host rows.
 struct EpWsLayout {
-    size_t hdr;        // int32[8]
+    size_t hdr;        // int32[16]
     size_t cc;         // int32 [nchunk][E] over the rank's S tokens
     size_t host_dst0;  // int32 [2E+R]
     size_t total;
@@ -247,7 +253,10 @@ __device__ __forceinline__ int block_exscan_per(int *a, int n, int *wsum, int pe
     return total;
 }
 
-__device__ inline int block_exscan(int *a, int n, int *wsum)
+// Out of line: the planner calls it at a dozen places, and five inlined
+// variants at each made its code several times larger than the instruction
+// caches, so that its one-after-another steps waited on instruction fetch.
+static __device__ __noinline__ int block_exscan(int *a, int n, int *wsum)
 {
     const int nt = blockDim.x;
     if (n <= nt) return block_exscan_per<1>(a, n, wsum, 1);

@@ -43,6 +43,8 @@
 //                     before the planner writes over them, so no pass fills
 //                     the unused rest afterwards.)
 #include <atomic>
+#include <climits>
+#include <mutex>
 
 #include "common.cuh"
 
@@ -63,12 +65,33 @@ struct PlanParams {
     int *hdr;        // ticket, status, call sequence, counts-ready mark, arrivals
     int *gs;         // [2][ngroups][E] (expert parallelism: the gathered counts [R][E+1])
     int gs_stride;   // ints between the count rows of gs: E (E + 1 for the gathered counts)
+    int gs_buf;      // ints of one of the two group-count buffers as the workspace lays them out
     int *cc;         // [nchunk][E]
     int *host_dst0;  // [2E+R]
     FastDiv fC, fL;  // divisions by C and L
     int spin_limit;  // iterations of each bounded wait of the assignment pass
     int cascade_cap; // the relay cascade guard's replica capacity: E + R - 1, or less in a test
 };
+
+// Where the planner's results go.  In the two-kernel path one planner CTA
+// computes the plan, writes every table and the info block, keeps the host
+// rows in the workspace for the assignment CTAs and sets the marks they wait
+// for (legacy).  In the one-kernel path every CTA computes the same plan in
+// its own shared memory and keeps the host tables there for its own pass B;
+// one CTA (writer) stores the plan tables, and the info values are left in
+// the planner's misc words for the CTA that finishes last.
+struct PlanSink {
+    bool legacy;
+    bool writer;
+    int *hptr, *hstart, *hdst;  // one-kernel path: [E+1], [2E+R], [2E+R] in shared memory
+};
+
+// The planner's misc words (16 ints of shared memory): 0 status in, 2
+// replicas over the budget, 3 most replicas on a rank, 4-5 the cascade
+// guard's steps and least slack, 6 replicas, 7 pieces, 8 receivers, 9
+// experts with a prefetched replica, 10 the plan's status bits.
+enum { MISC_STATUS_IN = 0, MISC_N_OVER = 2, MISC_MAX_REP = 3, MISC_GUARD_STEPS = 4, MISC_GUARD_SLACK = 5,
+       MISC_N_REP = 6, MISC_N_PIECES = 7, MISC_N_RECEIVERS = 8, MISC_N_REP_EXPERTS = 9, MISC_PLAN_STATUS = 10 };
 
 // The bound of the assignment pass's two waits, for every later launch in
 // the process (moonep_set_wait_limit).
@@ -187,7 +210,7 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 // list capacity.
 __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep, const int *pe, const int *qr,
                              const int *segb, const int *pilo, const int *PS, const int *QSr, int qbase,
-                             int n_rep, int nP, int nN, int *misc, int *wsum, int seq)
+                             int n_rep, int nP, int nN, int *misc, int *wsum, int seq, const PlanSink &sink)
 {
     const Dims &d = a.d;
     const int E = d.E, R = d.R, L = d.L, C = d.C, B = d.B;
@@ -210,8 +233,10 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
 
     // announce the slow path: the assignment CTAs stop spinning on the
     // plan-ready mark and wait for this grid to finish
-    if (tid == 0) st_release(a.hdr + WS_SLOW, seq + 1);
+    if (sink.legacy && tid == 0) st_release(a.hdr + WS_SLOW, seq + 1);
+    const bool wr = sink.writer;
     // the water-filling list in creation order
+    #pragma unroll 1
     for (int q = tid; q < min(n_rep, lc); q += nt) {
         const int j = last_le(segb, nP, q);
         const int i = pilo[j] + (q - segb[j]);
@@ -220,6 +245,7 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
         lq[q] = min(PS[j + 1], QSr[i + 1] - qbase) - max(PS[j], QSr[i] - qbase);
         la[q] = 1;
     }
+    #pragma unroll 1
     for (int r = tid; r < R; r += nt) closed[r] = 0;
     __syncthreads();
 
@@ -234,14 +260,18 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
         }
         int nl = min(n_rep, lc);
         int n_guard = 0, min_slack = 0;  // steps that reached the capacity guard, its least slack
+        #pragma unroll 1
         for (int step = 0; step <= R; ++step) {
+            #pragma unroll 1
             for (int r = lane; r < R; r += 32) cnt[r] = 0;
             __syncwarp();
+            #pragma unroll 1
             for (int q = lane; q < nl; q += 32)
                 if (la[q]) atomicAdd(&cnt[lr[q]], 1);
             __syncwarp();
             // the open rank over B with the most replicas, lowest rank on ties
             int bc = -1, br = R;
+            #pragma unroll 1
             for (int r = lane; r < R; r += 32) {
                 const int c = cnt[r];
                 if (!closed[r] && c > B && c > bc) {
@@ -261,9 +291,12 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
             const int rs = br;
             // its replicas: positions in list order (in mq), then ranked by
             // (quota desc, position asc) into ordx
+            #pragma unroll 1
             for (int e = lane; e < E; e += 32) on_r[e] = 0;
+            #pragma unroll 1
             for (int r = lane; r < R; r += 32) hused[r] = 0;
             int n = 0;
+            #pragma unroll 1
             for (int q0 = 0; q0 < nl; q0 += 32) {
                 const int q = q0 + lane;
                 const bool mine = q < nl && la[q] && lr[q] == rs;
@@ -274,9 +307,11 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
             }
             n = min(n, lc);
             __syncwarp();
+            #pragma unroll 1
             for (int k = lane; k < n; k += 32) {
                 const int qk = mq[k], vk = lq[qk];
                 int rk = 0;
+                #pragma unroll 1
                 for (int j = 0; j < n; ++j) {
                     const int v = lq[mq[j]];
                     rk += (v > vk) || (v == vk && j < k);
@@ -287,9 +322,11 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
             __syncwarp();
             // the smallest m whose providers carry the moved quota
             int npick = 0, m_found = -1;
+            #pragma unroll 1
             for (int m = 0; m <= B; ++m) {
                 while (npick < m) {  // next relay: largest home quota, lowest expert
                     int bk = 0, be = E;
+                    #pragma unroll 1
                     for (int e = lane; e < E; e += 32) {
                         const int h = (int)fdiv((uint32_t)e, a.fL), kv = keep[e];
                         if (kv > bk && h != rs && !closed[h] && !on_r[e] && !hused[h]) {
@@ -315,11 +352,14 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
                 }
                 if (npick < m) break;  // fewer distinct relay homes than m
                 long long Q = 0, room = 0;
+                #pragma unroll 1
                 for (int k = B - m + lane; k < n; k += 32) Q += lq[ordx[k]];
+                #pragma unroll 1
                 for (int k = lane; k < B - m; k += 32) {
                     const int e = le[ordx[k]];
                     room += closed[fdiv((uint32_t)e, a.fL)] ? 0 : keep[e];
                 }
+                #pragma unroll 1
                 for (int k = lane; k < m; k += 32) room += keep[rel[k]];
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) {
@@ -343,22 +383,26 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
             const int k0 = B - m_found;
             // the rank's replicas by step order: experts and quotas; a kept
             // replica's position once the moved ones are dropped
+            #pragma unroll 1
             for (int k = lane; k < n; k += 32) {
                 const int q = ordx[k];
                 me[k] = le[q];
                 mq[k] = lq[q];
                 if (k < k0) {
                     int before = 0;
+                    #pragma unroll 1
                     for (int j = k0; j < n; ++j) before += ordx[j] < q;
                     pvq[k] = q - before;
                 }
             }
             __syncwarp();
+            #pragma unroll 1
             for (int k = k0 + lane; k < n; k += 32) la[ordx[k]] = 0;  // the moved replicas leave this rank
             __syncwarp();
             // drop them, keeping list order (a destination never lies past its
             // source, so a chunk only writes where its reads are done)
             int w = 0;
+            #pragma unroll 1
             for (int q0 = 0; q0 < nl; q0 += 32) {
                 const int q = q0 + lane;
                 const bool alive = q < nl && la[q];
@@ -386,13 +430,17 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
             int np = 0;
             if (lane == 0) {
                 long long rem = 0;
+                #pragma unroll 1
                 for (int k = k0; k < n; ++k) rem += mq[k];
+                #pragma unroll 1
                 for (int k = 0; k < k0; ++k) pve[np++] = me[k];
+                #pragma unroll 1
                 for (int k = 0; k < m_found; ++k) {
                     pve[np] = rel[k];
                     pvq[np] = -1;
                     ++np;
                 }
+                #pragma unroll 1
                 for (int k = 0; k < np; ++k) {
                     const int e = pve[k];
                     const long long capk = (pvq[k] >= 0 && closed[fdiv((uint32_t)e, a.fL)]) ? 0 : keep[e];
@@ -425,6 +473,7 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
             int *MS = ordx, *PV = pvq, *tag = on_r;  // free by now: order, kept positions, relay marks
             {
                 int run = 0;
+                #pragma unroll 1
                 for (int b0 = 0; b0 < nm; b0 += 32) {
                     const int i = b0 + lane, v = i < nm ? mq[k0 + i] : 0;
                     int x = v;
@@ -438,6 +487,7 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
                 }
                 if (lane == 0) MS[nm] = run;
                 run = 0;
+                #pragma unroll 1
                 for (int b0 = 0; b0 < np; b0 += 32) {
                     const int i = b0 + lane, v = i < np ? pva[i] : 0;
                     int x = v;
@@ -451,17 +501,21 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
                 }
                 if (lane == 0) PV[np] = run;
             }
+            #pragma unroll 1
             for (int e = lane; e < E; e += 32) tag[e] = -1;
             __syncwarp();
+            #pragma unroll 1
             for (int pi = 0; pi < np; ++pi) {
                 const int lo = PV[pi], hi = PV[pi + 1];
                 if (hi <= lo || nm <= 0) continue;
                 const int h = (int)fdiv((uint32_t)pve[pi], a.fL);
                 const int i_lo = warp_last_le(MS, nm, lo), i_hi = warp_last_le(MS, nm, hi - 1);
                 const int nl0 = nl;
+                #pragma unroll 1
                 for (int q = lane; q < nl0; q += 32)
                     if (lr[q] == h) tag[le[q]] = q;
                 __syncwarp();
+                #pragma unroll 1
                 for (int i0 = i_lo; i0 <= i_hi; i0 += 32) {
                     const int i = i0 + lane;
                     bool fresh = false;
@@ -488,6 +542,7 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
                     nl = min(nl + __popc(b), lc);
                 }
                 __syncwarp();
+                #pragma unroll 1
                 for (int q = lane; q < nl0; q += 32)
                     if (lr[q] == h) tag[le[q]] = -1;
                 __syncwarp();
@@ -503,41 +558,76 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
     const int nl = s_nl;
 
     // ordinals in list order, slot offsets and the used slots of every rank
+    // (in the one-kernel path each rank's row is written by the CTA that owns
+    // the rank, r mod gridDim.x, empty slots included)
+    #pragma unroll 1
     for (int r = tid; r < R; r += nt) {
+        const bool own = sink.legacy ? wr : (int)(r % gridDim.x) == (int)blockIdx.x;
         int off = 0;
+        #pragma unroll 1
         for (int sl = 0; sl < L; ++sl) {
             const int e = r * L + sl;
             hoff[e] = off;
-            a.p.slot_expert[(size_t)r * E + sl] = e;
-            a.p.slot_count[(size_t)r * E + sl] = keep[e];
-            a.p.slot_offset[(size_t)r * (E + 1) + sl] = off;
+            if (own) {
+                a.p.slot_expert[(size_t)r * E + sl] = e;
+                a.p.slot_count[(size_t)r * E + sl] = keep[e];
+                a.p.slot_offset[(size_t)r * (E + 1) + sl] = off;
+            }
             off += keep[e];
         }
         int ord = 0;
+        #pragma unroll 1
         for (int q = 0; q < nl; ++q) {
             if (lr[q] != r) continue;
             lo[q] = ord;
             loff[q] = off;
             const int sl = min(L + ord, E - 1);
-            a.p.slot_expert[(size_t)r * E + sl] = le[q];
-            a.p.slot_count[(size_t)r * E + sl] = lq[q];
-            a.p.slot_offset[(size_t)r * (E + 1) + sl] = off;
+            if (own) {
+                a.p.slot_expert[(size_t)r * E + sl] = le[q];
+                a.p.slot_count[(size_t)r * E + sl] = lq[q];
+                a.p.slot_offset[(size_t)r * (E + 1) + sl] = off;
+            }
             off += lq[q];
             ++ord;
         }
         atomicMax(&misc[3], ord);
+        cnt[r] = min(L + ord, E);  // used slots of rank r (cnt is free after the steps)
     }
     __syncthreads();
+    if (!sink.legacy)
+        #pragma unroll 1
+        for (int r = blockIdx.x; r < R; r += gridDim.x)
+            #pragma unroll 1
+            for (int sl = cnt[r] + tid; sl <= E; sl += nt) {
+                if (sl < E) {
+                    a.p.slot_expert[(size_t)r * E + sl] = -1;
+                    a.p.slot_count[(size_t)r * E + sl] = 0;
+                }
+                a.p.slot_offset[(size_t)r * (E + 1) + sl] = C;
+            }
+    #pragma unroll 1
     for (int q = tid; q < nl; q += nt) {
-        a.p.rep_expert[q] = le[q];
-        a.p.rep_rank[q] = lr[q];
-        a.p.rep_slot[q] = L + lo[q];
-        a.p.rep_quota[q] = lq[q];
+        if (wr) {
+            a.p.rep_expert[q] = le[q];
+            a.p.rep_rank[q] = lr[q];
+            a.p.rep_slot[q] = L + lo[q];
+            a.p.rep_quota[q] = lq[q];
+        }
         if (lo[q] >= B) atomicAdd(&misc[2], 1);
     }
+    if (wr && !sink.legacy)  // the one-kernel path writes no defaults beforehand
+        #pragma unroll 1
+        for (int q = nl + tid; q < E + R; q += nt) {
+            a.p.rep_expert[q] = -1;
+            a.p.rep_rank[q] = -1;
+            a.p.rep_slot[q] = -1;
+            a.p.rep_quota[q] = 0;
+        }
     // hosts per expert (home + its replicas) and the work-list flags
+    #pragma unroll 1
     for (int e = tid; e < E; e += nt) {
         int c = 1, f = 0;
+        #pragma unroll 1
         for (int q = 0; q < nl; ++q)
             if (le[q] == e) {
                 ++c;
@@ -554,12 +644,28 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
     __syncthreads();
     block_exscan(hc, E + 1, wsum);
     const int n_rep_experts = block_exscan(fpre, E + 1, wsum);
-    for (int e = tid; e <= E; e += nt) a.p.host_ptr[e] = hc[e];
-    for (int e = tid; e < E; e += nt) {
-        if (fl[e]) a.p.rep_home_list[fpre[e]] = e;
-        if (e >= n_rep_experts) a.p.rep_home_list[e] = -1;
+    #pragma unroll 1
+    for (int e = tid; e <= E; e += nt) {
+        if (wr) a.p.host_ptr[e] = hc[e];
+        if (!sink.legacy) sink.hptr[e] = hc[e];
     }
+    if (wr && !sink.legacy)
+        #pragma unroll 1
+        for (int h = hc[E] + tid; h < nh; h += nt) {
+            a.p.host_rank[h] = -1;
+            a.p.host_slot[h] = -1;
+            a.p.host_start[h] = 0;
+            a.p.host_quota[h] = 0;
+            a.p.host_local[h] = 0;
+        }
+    if (wr)
+        #pragma unroll 1
+        for (int e = tid; e < E; e += nt) {
+            if (fl[e]) a.p.rep_home_list[fpre[e]] = e;
+            if (e >= n_rep_experts) a.p.rep_home_list[e] = -1;
+        }
     // host intervals: the hosts of e in ascending rank, starts in that order
+    #pragma unroll 1
     for (int e = tid; e < E; e += nt) {
         const int b0 = hc[e], b1 = min(hc[e + 1], nh);
         int k = b0;
@@ -570,6 +676,7 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
             xo[k] = hoff[e];
             ++k;
         }
+        #pragma unroll 1
         for (int q = 0; q < nl && k < b1; ++q)
             if (le[q] == e) {
                 xr[k] = lr[q];
@@ -578,6 +685,7 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
                 xo[k] = loff[q];
                 ++k;
             }
+        #pragma unroll 1
         for (int x = b0 + 1; x < k; ++x) {  // insertion sort by rank (ranks are distinct)
             const int vr = xr[x], vs = xs[x], vq = xq[x], vo = xo[x];
             int y = x;
@@ -594,17 +702,26 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
             xo[y] = vo;
         }
         int st = 0;
+        #pragma unroll 1
         for (int h = b0; h < k; ++h) {
             // the locality flag as in the water-filling tail
             const int loc = (d.flags & MOONEP_FLAG_LOCALITY)
                                 ? min(xq[h], ld_cg(a.gs + (size_t)xr[h] * a.gs_stride + e))
                                 : 0;
-            a.p.host_rank[h] = xr[h];
-            a.p.host_slot[h] = xs[h];
-            a.p.host_quota[h] = xq[h];
-            a.p.host_start[h] = st;
-            a.p.host_local[h] = loc;
-            a.host_dst0[h] = xr[h] * C + xo[h] - st;
+            if (wr) {
+                a.p.host_rank[h] = xr[h];
+                a.p.host_slot[h] = xs[h];
+                a.p.host_quota[h] = xq[h];
+                a.p.host_start[h] = st;
+                a.p.host_local[h] = loc;
+            }
+            const int dst0 = xr[h] * C + xo[h] - st;
+            if (sink.legacy) {
+                a.host_dst0[h] = dst0;
+            } else {
+                sink.hstart[h] = st;
+                sink.hdst[h] = dst0;
+            }
             st += xq[h] - loc;
         }
     }
@@ -616,20 +733,28 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
             st |= MOONEP_ST_OVERFLOW;
             if (d.flags & MOONEP_FLAG_STRICT_BUDGET) st |= MOONEP_ST_STRICT_VIOLATION;
         }
-        a.p.info[MOONEP_INFO_STATUS] = st;
-        a.p.info[MOONEP_INFO_N_REP] = nl;
-        a.p.info[MOONEP_INFO_N_OVERFLOW] = n_over;
-        a.p.info[MOONEP_INFO_N_PIECES] = nP;
-        a.p.info[MOONEP_INFO_N_RECEIVERS] = nN;
-        a.p.info[MOONEP_INFO_MAX_REP_PER_RANK] = misc[3];
-        a.p.info[MOONEP_INFO_N_REP_EXPERTS] = n_rep_experts;
-        for (int i = MOONEP_INFO_N_REMOTE_PAIRS; i < MOONEP_INFO_LEN; ++i) a.p.info[i] = 0;
-        a.p.info[MOONEP_INFO_CASCADE_GUARD_STEPS] = misc[4];
-        a.p.info[MOONEP_INFO_CASCADE_GUARD_SLACK] = misc[5];
+        misc[MISC_N_REP] = nl;
+        misc[MISC_N_PIECES] = nP;
+        misc[MISC_N_RECEIVERS] = nN;
+        misc[MISC_N_REP_EXPERTS] = n_rep_experts;
+        misc[MISC_PLAN_STATUS] = st;
+        if (sink.legacy) {
+            a.p.info[MOONEP_INFO_STATUS] = st;
+            a.p.info[MOONEP_INFO_N_REP] = nl;
+            a.p.info[MOONEP_INFO_N_OVERFLOW] = n_over;
+            a.p.info[MOONEP_INFO_N_PIECES] = nP;
+            a.p.info[MOONEP_INFO_N_RECEIVERS] = nN;
+            a.p.info[MOONEP_INFO_MAX_REP_PER_RANK] = misc[3];
+            a.p.info[MOONEP_INFO_N_REP_EXPERTS] = n_rep_experts;
+            #pragma unroll 1
+            for (int i = MOONEP_INFO_N_REMOTE_PAIRS; i < MOONEP_INFO_LEN; ++i) a.p.info[i] = 0;
+            a.p.info[MOONEP_INFO_CASCADE_GUARD_STEPS] = misc[4];
+            a.p.info[MOONEP_INFO_CASCADE_GUARD_SLACK] = misc[5];
+        }
     }
     // every thread's plan writes precede the plan-ready mark
     __syncthreads();
-    if (tid == 0) {
+    if (sink.legacy && tid == 0) {
         __threadfence();
         st_release(a.hdr + WS_PLANNED, seq + 1);
     }
@@ -637,44 +762,27 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
 
 // ------------------------------------------------------------- planner CTA
 
+// The planner's shared-memory layout, from the base sm (plan_smem_ints(E, R)
+// ints): the expert totals T come first, the misc words last.
+__device__ __forceinline__ int *plan_misc(int *sm, int E, int R) { return sm + plan_smem_ints(E, R) - 16; }
+
+__device__ void plan_core(const PlanParams &a, int *sm, int seq, const PlanSink &sink);
+
+// The two-kernel path's planner CTA: the expert totals from this call's
+// group counts, the checks that empty the plan, then the plan itself.
 __device__ void plan_block(const PlanParams &a, int *sm, int seq)
 {
     const int parity = seq & 1;
     const Dims &d = a.d;
-    const int E = d.E, R = d.R, L = d.L, C = d.C, B = d.B;
-    // the planner runs in the last histogram CTA: PLAN_THREADS threads, a
-    // compile-time stride for every loop below
+    const int E = d.E, R = d.R;
     const int tid = threadIdx.x;
     constexpr int nt = PLAN_THREADS;
     const int lane = tid & 31, warp = tid >> 5;
     constexpr int nwarp = PLAN_THREADS / 32;
-    const int nh = 2 * E + R;
-
     int *T = sm;
-    int *shed = T + E;
-    int *keep = shed + E;
-    int *X = keep + E;
-    int *D = X + R;
-    int *scr = D + R;              // E + R + 2
-    int *pe = scr + E + R + 2;     // E   pieces: expert, sorted
-    int *qr = pe + E;              // R   receivers: rank, sorted
-    int *A = qr + R;               // E + R + 4: sorted sizes, then PS (nP+1) and QS (nN+1)
-    int *pilo = A + E + R + 4;     // E   first receiver of piece j
-    int *Bs = pilo + E;            // E + R + 4: segments per piece (nP+1) | replicas per rank (R+1)
-    int *jlo = Bs + E + R + 4;     // R   first piece of receiver i
-    int *pof = jlo + R;            // E   piece index of expert e, -1 if none
-    int *cexp = pof + E;           // nh  compact used slots: expert
-    int *ccnt = cexp + nh;         // nh  rows
-    int *cspare = ccnt + nh;       // nh  receiver ids while sorting, then the rank of each used slot
-    int *hr = cspare + nh;         // nh  piece rows, while sorting
-    int *hs = hr + nh;             // nh  piece experts, while sorting
-    int *hq = hs + nh;             // nh  receiver deficits, while sorting
-    int *flag = hq + nh;           // E
-    int *wsum = flag + E;          // 32
-    int *misc = wsum + 32;         // 16: 0 status in, 2 n_over, 3 max replicas per rank, 4-5 cascade guard
+    int *misc = plan_misc(sm, E, R);
 
     __shared__ unsigned s_part[2][32];
-    for (int i = tid; i < 16; i += nt) misc[i] = 0;
     // every other CTA has arrived: take the status (the load is issued here
     // and waited for after the totals' loads) and reset the header
     int st_hdr = 0;
@@ -697,7 +805,7 @@ __device__ void plan_block(const PlanParams &a, int *sm, int seq)
         }
     }
     if (tid == 0) {
-        misc[0] = st_hdr;
+        misc[MISC_STATUS_IN] = st_hdr;
         a.hdr[WS_STATUS] = 0;
         a.hdr[WS_TICKET] = 0;
     }
@@ -711,7 +819,7 @@ __device__ void plan_block(const PlanParams &a, int *sm, int seq)
         }
     }
     negative = __syncthreads_or(negative);
-    int status_in = misc[0];
+    int status_in = misc[MISC_STATUS_IN];
     long long total;
     {
         const unsigned lo = __reduce_add_sync(FULL_MASK, lane < nwarp ? s_part[0][lane] : 0u);
@@ -731,8 +839,56 @@ __device__ void plan_block(const PlanParams &a, int *sm, int seq)
         }
         return;  // the assignment pass writes the empty tables
     }
+    __syncthreads();  // misc[0] read by every thread before plan_core clears it
+    plan_core(a, sm, seq, PlanSink{true, true, nullptr, nullptr, nullptr});
+}
+
+// The plan from the expert totals T = sm[0..E) (every id valid, the totals
+// adding up to the pairs), by the whole CTA: loads, shedding, orders,
+// water-filling, slot lists and host intervals, or the relay cascade.
+// Its loops (and the cascade's) are kept rolled: the steps run one after
+// another, each on data already in shared memory, and the unrolled code did
+// not fit the instruction caches -- after a kernel that streams through L2,
+// every step then waited on instruction fetch from memory.
+__device__ void plan_core(const PlanParams &a, int *sm, int seq, const PlanSink &sink)
+{
+    const Dims &d = a.d;
+    const int E = d.E, R = d.R, L = d.L, C = d.C, B = d.B;
+    // PLAN_THREADS threads, a compile-time stride for every loop below
+    const int tid = threadIdx.x;
+    constexpr int nt = PLAN_THREADS;
+    const int lane = tid & 31, warp = tid >> 5;
+    constexpr int nwarp = PLAN_THREADS / 32;
+    const int nh = 2 * E + R;
+    const bool wr = sink.writer;
+
+    int *T = sm;
+    int *shed = T + E;
+    int *keep = shed + E;
+    int *X = keep + E;
+    int *D = X + R;
+    int *scr = D + R;              // E + R + 2
+    int *pe = scr + E + R + 2;     // E   pieces: expert, sorted
+    int *qr = pe + E;              // R   receivers: rank, sorted
+    int *A = qr + R;               // E + R + 4: sorted sizes, then PS (nP+1) and QS (nN+1)
+    int *pilo = A + E + R + 4;     // E   first receiver of piece j
+    int *Bs = pilo + E;            // E + R + 4: segments per piece (nP+1) | replicas per rank (R+1)
+    int *jlo = Bs + E + R + 4;     // R   first piece of receiver i
+    int *pof = jlo + R;            // E   piece index of expert e, -1 if none
+    int *cexp = pof + E;           // nh  compact used slots: expert
+    int *ccnt = cexp + nh;         // nh  rows
+    int *cspare = ccnt + nh;       // nh  receiver ids while sorting, then the rank of each used slot
+    int *hr = cspare + nh;         // nh  piece rows, while sorting
+    int *hs = hr + nh;             // nh  piece experts, while sorting
+    int *hq = hs + nh;             // nh  receiver deficits, while sorting
+    int *flag = hq + nh;           // E
+    int *wsum = flag + E;          // 32
+    int *misc = wsum + 32;         // 16 (MISC_*)
+    #pragma unroll 1
+    for (int i = tid; i < 16; i += nt) misc[i] = 0;
 
     // ---- home loads, excess X and deficit D per rank
+    #pragma unroll 1
     for (int r = tid; r < R; r += nt) {
         int h = 0;
 #pragma unroll 4
@@ -744,6 +900,7 @@ __device__ void plan_block(const PlanParams &a, int *sm, int seq)
 
     // ---- largest-first shedding: expert e sheds what remains of its rank's
     // excess after all larger (T desc, e asc) experts of the rank
+    #pragma unroll 1
     for (int e = tid; e < E; e += nt) {
         const int r = (int)fdiv((uint32_t)e, a.fL), v = T[e];
         int s = 0;
@@ -762,6 +919,7 @@ __device__ void plan_block(const PlanParams &a, int *sm, int seq)
         scr[e] = s > 0;
         pof[e] = -1;
     }
+    #pragma unroll 1
     for (int r = tid; r < R; r += nt) scr[E + r] = D[r] > 0;
     __syncthreads();
 
@@ -769,11 +927,13 @@ __device__ void plan_block(const PlanParams &a, int *sm, int seq)
     const int nPN = block_exscan(scr, E + R, wsum);
     const int nP = scr[E];
     const int nN = nPN - nP;
+    #pragma unroll 1
     for (int e = tid; e < E; e += nt)
         if (shed[e] > 0) {
             hr[scr[e]] = shed[e];
             hs[scr[e]] = e;
         }
+    #pragma unroll 1
     for (int r = tid; r < R; r += nt)
         if (D[r] > 0) {
             hq[scr[E + r] - nP] = D[r];
@@ -783,12 +943,14 @@ __device__ void plan_block(const PlanParams &a, int *sm, int seq)
     // counting-rank sorts, one warp per element: pieces by (shed desc,
     // e asc), receivers by (D desc, r asc); an element's position is the
     // number of entries ordered before it, counted 32 at a time by ballot
+    #pragma unroll 1
     for (int x = warp; x < nP + nN; x += nwarp) {
         const bool piece = x < nP;
         const int m = piece ? nP : nN, xi = piece ? x : x - nP;
         const int *val = piece ? hr : hq, *key = piece ? hs : cspare;
         const int v = val[xi], id = key[xi];
         int pos = 0;
+        #pragma unroll 1
         for (int j0 = 0; j0 < m; j0 += 32) {
             const int j = j0 + lane;
             bool before = false;
@@ -814,6 +976,7 @@ __device__ void plan_block(const PlanParams &a, int *sm, int seq)
     }
     int *segb = Bs;          // nP + 1: replicas per piece, then their prefix
     int *rpr = Bs + nP + 1;  // R + 1: replicas per rank, then prefix + n_rep
+    #pragma unroll 1
     for (int r = tid; r <= R; r += nt) rpr[r] = 0;
     __syncthreads();
 
@@ -830,6 +993,7 @@ __device__ void plan_block(const PlanParams &a, int *sm, int seq)
     // ---- water-filling: piece j meets receivers pilo[j].. ; receiver i meets
     // pieces jlo[i].. ; replicas are numbered in (j, i) order
     // (one warp per piece or receiver, searching by ballot)
+    #pragma unroll 1
     for (int x = warp; x < nP + nN; x += nwarp) {
         if (x < nP) {
             const int j = x;
@@ -860,7 +1024,7 @@ __device__ void plan_block(const PlanParams &a, int *sm, int seq)
     // over the budget with the cascade asked for: the slow path plans the rest
     if ((d.flags & MOONEP_FLAG_CASCADE) && B > 0 && misc[3] > B) {
         cascade_tail(a, sm + plan_smem_ints(E, R), jlo, keep, pe, qr, segb, pilo, PS, QSr, qbase, n_rep, nP, nN,
-                     misc, wsum, seq);
+                     misc, wsum, seq, sink);
         return;
     }
     auto rank_base = [&](int r) { return r * L + rpr[r] - n_rep; };  // first compact slot of rank r
@@ -873,6 +1037,7 @@ __device__ void plan_block(const PlanParams &a, int *sm, int seq)
     int *Z = hr;     // 4E + R + 2 <= 3 nh ints, free after the sort
     int *rq_j = scr;  // n_rep <= E + R - 1: piece of each replica (scr is free)
     const int zh = E + n_rep, zf = zh + E + 1, nz = zf + E + 1;
+    #pragma unroll 1
     for (int q = tid; q < n_rep; q += nt) {
         const int j = last_le(segb, nP, q);
         rq_j[q] = j;
@@ -880,10 +1045,12 @@ __device__ void plan_block(const PlanParams &a, int *sm, int seq)
         const int ord = j - jlo[i];
         const int r = qr[i];
         const int quota = seg_q(j, i);
-        a.p.rep_expert[q] = pe[j];
-        a.p.rep_rank[q] = r;
-        a.p.rep_slot[q] = L + ord;
-        a.p.rep_quota[q] = quota;
+        if (wr) {
+            a.p.rep_expert[q] = pe[j];
+            a.p.rep_rank[q] = r;
+            a.p.rep_slot[q] = L + ord;
+            a.p.rep_quota[q] = quota;
+        }
         const int cs = rank_base(r) + L + ord;
         cexp[cs] = pe[j];
         ccnt[cs] = quota;
@@ -891,6 +1058,7 @@ __device__ void plan_block(const PlanParams &a, int *sm, int seq)
         cspare[cs] = r;
         if (ord >= B) atomicAdd(&misc[2], 1);
     }
+    #pragma unroll 1
     for (int e = tid; e < E; e += nt) {
         const int r = (int)fdiv((uint32_t)e, a.fL);
         const int cs = rank_base(r) + (e - r * L);
@@ -904,6 +1072,7 @@ __device__ void plan_block(const PlanParams &a, int *sm, int seq)
         if (j >= 0) {
             const int ns = segb[j + 1] - segb[j];
             c += ns;
+            #pragma unroll 1
             for (int s = 0; s < ns; ++s)
                 if (j - jlo[pilo[j] + s] < B) f = 1;
         }
@@ -931,6 +1100,7 @@ __device__ void plan_block(const PlanParams &a, int *sm, int seq)
     // of e), and its start is in the order of the pairs left over.
     const bool locality = (d.flags & MOONEP_FLAG_LOCALITY) != 0;
     auto own_pairs = [&](int r, int e) { return ld_cg(a.gs + (size_t)r * a.gs_stride + e); };
+    #pragma unroll 1
     for (int x = tid; x < n_hosts; x += nt) {
         int e, r0, slot, quota, j, pos = 0, st = 0, locsum = 0;
         if (x < E) {
@@ -956,6 +1126,7 @@ __device__ void plan_block(const PlanParams &a, int *sm, int seq)
         }
         if (j >= 0) {
             const int ns = segb[j + 1] - segb[j];
+            #pragma unroll 1
             for (int s = 0; s < ns; ++s) {
                 const int i = pilo[j] + s;
                 if (qr[i] < r0) {
@@ -970,14 +1141,26 @@ __device__ void plan_block(const PlanParams &a, int *sm, int seq)
         st -= locsum;
         const int h = hptr(e) + pos;
         const int b0 = rank_base(r0);
-        a.p.host_rank[h] = r0;
-        a.p.host_slot[h] = slot;
-        a.p.host_quota[h] = quota;
-        a.p.host_start[h] = st;
-        a.p.host_local[h] = loc;
-        a.host_dst0[h] = r0 * C + Z[b0 + slot] - Z[b0] - st;
+        if (wr) {
+            a.p.host_rank[h] = r0;
+            a.p.host_slot[h] = slot;
+            a.p.host_quota[h] = quota;
+            a.p.host_start[h] = st;
+            a.p.host_local[h] = loc;
+        }
+        const int dst0 = r0 * C + Z[b0 + slot] - Z[b0] - st;
+        if (sink.legacy) {
+            a.host_dst0[h] = dst0;
+        } else {
+            sink.hstart[h] = st;
+            sink.hdst[h] = dst0;
+        }
     }
-    for (int x = tid; x <= E; x += nt) a.p.host_ptr[x] = hptr(x);
+    #pragma unroll 1
+    for (int x = tid; x <= E; x += nt) {
+        if (wr) a.p.host_ptr[x] = hptr(x);
+        if (!sink.legacy) sink.hptr[x] = hptr(x);
+    }
 
     if (tid == 0) {
         const int n_over = misc[2];
@@ -986,33 +1169,143 @@ __device__ void plan_block(const PlanParams &a, int *sm, int seq)
             st |= MOONEP_ST_OVERFLOW;
             if (d.flags & MOONEP_FLAG_STRICT_BUDGET) st |= MOONEP_ST_STRICT_VIOLATION;
         }
-        a.p.info[MOONEP_INFO_STATUS] = st;
-        a.p.info[MOONEP_INFO_N_REP] = n_rep;
-        a.p.info[MOONEP_INFO_N_OVERFLOW] = n_over;
-        a.p.info[MOONEP_INFO_N_PIECES] = nP;
-        a.p.info[MOONEP_INFO_N_RECEIVERS] = nN;
-        a.p.info[MOONEP_INFO_MAX_REP_PER_RANK] = misc[3];
-        a.p.info[MOONEP_INFO_N_REP_EXPERTS] = n_rep_experts;
-        for (int i = MOONEP_INFO_N_REMOTE_PAIRS; i < MOONEP_INFO_LEN; ++i) a.p.info[i] = 0;
+        misc[MISC_N_REP] = n_rep;
+        misc[MISC_N_PIECES] = nP;
+        misc[MISC_N_RECEIVERS] = nN;
+        misc[MISC_N_REP_EXPERTS] = n_rep_experts;
+        misc[MISC_PLAN_STATUS] = st;
+        if (sink.legacy) {
+            a.p.info[MOONEP_INFO_STATUS] = st;
+            a.p.info[MOONEP_INFO_N_REP] = n_rep;
+            a.p.info[MOONEP_INFO_N_OVERFLOW] = n_over;
+            a.p.info[MOONEP_INFO_N_PIECES] = nP;
+            a.p.info[MOONEP_INFO_N_RECEIVERS] = nN;
+            a.p.info[MOONEP_INFO_MAX_REP_PER_RANK] = misc[3];
+            a.p.info[MOONEP_INFO_N_REP_EXPERTS] = n_rep_experts;
+            #pragma unroll 1
+            for (int i = MOONEP_INFO_N_REMOTE_PAIRS; i < MOONEP_INFO_LEN; ++i) a.p.info[i] = 0;
+        }
     }
     // the host tables and the status precede the plan-ready mark
     __syncthreads();
-    if (tid == 0) {
+    if (sink.legacy && tid == 0) {
         __threadfence();
         st_release(a.hdr + WS_PLANNED, seq + 1);
     }
-    // ---- then, while the assignment CTAs place the pairs, the used slots of
-    // the padded [R][E] tables and the reduce work list (read only by later
-    // kernels, which start after this grid has finished)
-    for (int x = tid; x < E + n_rep; x += nt) {
-        const int r = cspare[x], b0 = rank_base(r), sl = x - b0;
-        a.p.slot_expert[(size_t)r * E + sl] = cexp[x];
-        a.p.slot_count[(size_t)r * E + sl] = ccnt[x];
-        a.p.slot_offset[(size_t)r * (E + 1) + sl] = Z[x] - Z[b0];
+    if (!sink.legacy)
+        // the one-kernel path: the rows of the padded slot tables of this
+        // CTA's ranks (r mod gridDim.x), used and empty slots alike, so every
+        // entry is written once and no defaults precede them
+        #pragma unroll 1
+        for (int r = blockIdx.x; r < R; r += gridDim.x) {
+            const int b0 = rank_base(r), ns = rank_base(r + 1) - b0;
+            #pragma unroll 1
+            for (int sl = tid; sl <= E; sl += nt) {
+                const bool used = sl < ns;
+                if (sl < E) {
+                    a.p.slot_expert[(size_t)r * E + sl] = used ? cexp[b0 + sl] : -1;
+                    a.p.slot_count[(size_t)r * E + sl] = used ? ccnt[b0 + sl] : 0;
+                }
+                a.p.slot_offset[(size_t)r * (E + 1) + sl] = used ? Z[b0 + sl] - Z[b0] : C;
+            }
+        }
+    if (!wr) return;
+    if (sink.legacy) {
+        // ---- then, while the assignment CTAs place the pairs, the used
+        // slots of the padded [R][E] tables (read only by later kernels,
+        // which start after this grid has finished)
+        #pragma unroll 1
+        for (int x = tid; x < E + n_rep; x += nt) {
+            const int r = cspare[x], b0 = rank_base(r), sl = x - b0;
+            a.p.slot_expert[(size_t)r * E + sl] = cexp[x];
+            a.p.slot_count[(size_t)r * E + sl] = ccnt[x];
+            a.p.slot_offset[(size_t)r * (E + 1) + sl] = Z[x] - Z[b0];
+        }
+    } else {
+        // the writer: the empty rest of the replica and host tables
+        #pragma unroll 1
+        for (int q = n_rep + tid; q < E + R; q += nt) {
+            a.p.rep_expert[q] = -1;
+            a.p.rep_rank[q] = -1;
+            a.p.rep_slot[q] = -1;
+            a.p.rep_quota[q] = 0;
+        }
+        #pragma unroll 1
+        for (int h = n_hosts + tid; h < nh; h += nt) {
+            a.p.host_rank[h] = -1;
+            a.p.host_slot[h] = -1;
+            a.p.host_start[h] = 0;
+            a.p.host_quota[h] = 0;
+            a.p.host_local[h] = 0;
+        }
     }
+    // the reduce work list
+    #pragma unroll 1
     for (int x = tid; x < E; x += nt) {
         if (flag[x]) a.p.rep_home_list[Z[zf + x] - zf0] = x;
         if (x >= n_rep_experts) a.p.rep_home_list[x] = -1;
+    }
+}
+
+// The plan tables' empty defaults (unused slots, replica and host entries),
+// entries x0, x0 + g, ...: the grid's share of the calling thread, or the
+// CTA's.  The planner writes the used entries over them afterwards, so no
+// later pass fills the unused rest.
+__device__ __forceinline__ void write_table_defaults(const PlanParams &a, int x0, int g)
+{
+    const Dims &d = a.d;
+    const int E = d.E, R = d.R, nh = 2 * E + R;
+    for (int x = x0; x < R * E; x += g) {
+        a.p.slot_expert[x] = -1;
+        a.p.slot_count[x] = 0;
+    }
+    for (int x = x0; x < R * (E + 1); x += g) a.p.slot_offset[x] = d.C;
+    for (int x = x0; x < E + R; x += g) {
+        a.p.rep_expert[x] = -1;
+        a.p.rep_rank[x] = -1;
+        a.p.rep_slot[x] = -1;
+        a.p.rep_quota[x] = 0;
+    }
+    for (int x = x0; x < nh; x += g) {
+        a.p.host_rank[x] = -1;
+        a.p.host_slot[x] = -1;
+        a.p.host_start[x] = 0;
+        a.p.host_quota[x] = 0;
+        a.p.host_local[x] = 0;
+    }
+}
+
+// An empty plan: every table empty, spread over the grid, and dst_pos and
+// row_src -1 for this CTA's pairs [p0, p0 + n) (the rows are as many as the
+// pairs, so the CTAs cover row_src too).
+__device__ __forceinline__ void write_empty_plan(const PlanParams &a, int p0, int n)
+{
+    const Dims &d = a.d;
+    const int E = d.E, R = d.R, nh = 2 * E + R;
+    const int g = gridDim.x * blockDim.x, x0 = blockIdx.x * blockDim.x + threadIdx.x;
+    for (int x = x0; x < R * E; x += g) {
+        a.p.slot_expert[x] = -1;
+        a.p.slot_count[x] = 0;
+    }
+    for (int x = x0; x < R * (E + 1); x += g) a.p.slot_offset[x] = 0;
+    for (int x = x0; x < E + R; x += g) {
+        a.p.rep_expert[x] = -1;
+        a.p.rep_rank[x] = -1;
+        a.p.rep_slot[x] = -1;
+        a.p.rep_quota[x] = 0;
+    }
+    for (int x = x0; x < nh; x += g) {
+        a.p.host_rank[x] = -1;
+        a.p.host_slot[x] = -1;
+        a.p.host_start[x] = 0;
+        a.p.host_quota[x] = 0;
+        a.p.host_local[x] = 0;
+    }
+    for (int x = x0; x <= E; x += g) a.p.host_ptr[x] = 0;
+    for (int x = x0; x < E; x += g) a.p.rep_home_list[x] = -1;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        a.p.dst_pos[p0 + i] = -1;
+        a.p.row_src[p0 + i] = -1;
     }
 }
 
@@ -1037,31 +1330,9 @@ __global__ void __launch_bounds__(PLAN_THREADS) hist_plan_kernel(PlanParams a)
     const int p0 = t0 * K, n = (t1 - t0) * K;
     int *hist = sm;       // E
     int *ids = sm + E;    // chunk_tokens * K
-    // this CTA's share of the tables' empty defaults (unused slots, replica
-    // and host entries); the planner CTA writes the used entries over them
-    // after every CTA's ticket, so no later pass fills the unused rest
-    {
-        const int R = d.R, nh = 2 * E + R;
-        const int g = gridDim.x * nt, x0 = blockIdx.x * nt + tid;
-        for (int x = x0; x < R * E; x += g) {
-            a.p.slot_expert[x] = -1;
-            a.p.slot_count[x] = 0;
-        }
-        for (int x = x0; x < R * (E + 1); x += g) a.p.slot_offset[x] = d.C;
-        for (int x = x0; x < E + R; x += g) {
-            a.p.rep_expert[x] = -1;
-            a.p.rep_rank[x] = -1;
-            a.p.rep_slot[x] = -1;
-            a.p.rep_quota[x] = 0;
-        }
-        for (int x = x0; x < nh; x += g) {
-            a.p.host_rank[x] = -1;
-            a.p.host_slot[x] = -1;
-            a.p.host_start[x] = 0;
-            a.p.host_quota[x] = 0;
-            a.p.host_local[x] = 0;
-        }
-    }
+    // this CTA's share of the defaults; the planner CTA writes the used
+    // entries after every CTA's ticket
+    write_table_defaults(a, blockIdx.x * nt + tid, gridDim.x * nt);
     for (int e = tid; e < E; e += nt) hist[e] = 0;
     for (int i = tid; i < n; i += nt) ids[i] = __ldg(a.topk + p0 + i);  // all loads in flight
     if (tid == 0) s_seq = ld_cg(a.hdr + WS_SEQ);
@@ -1128,17 +1399,50 @@ __device__ __forceinline__ void assign_pass_a(int *ids, int *wc, int wbeg, int w
     }
 }
 
+// Pass A as above, with the lanes of a batch that hold the same expert found
+// by one shared-memory atomicOr per pair into a lane mask per expert (mk: the
+// warp's E words, zero on entry and again on exit) instead of one ballot per
+// id bit: the vote unit's throughput, not latency, bounds the ballot form
+// when all warps of an SM run it.  Same ranks, bit for bit.
+__device__ __forceinline__ void assign_pass_a_mask(int *ids, int *wc, unsigned *mk, int wbeg, int wend, int E)
+{
+    const int lane = threadIdx.x & 31;
+    for (int b = wbeg; b < wend; b += 32) {
+        const int i = b + lane;
+        const int e = i < wend ? ids[i] : -1;
+        const bool ok = e >= 0 && e < E;
+        if (ok) atomicOr(&mk[e], 1u << lane);
+        __syncwarp();
+        unsigned peers = 0;
+        int base = 0;
+        if (ok) {
+            peers = mk[e];
+            base = wc[e];
+        }
+        __syncwarp();  // every lane has read its expert's words before the first lane updates them
+        if (ok) {
+            if (lane == __ffs(peers) - 1) {
+                wc[e] = base + __popc(peers);
+                mk[e] = 0;
+            }
+            ids[i] = ((base + __popc(peers & lanemask_lt())) << PACK_BITS) | e;
+        }
+        __syncwarp();
+    }
+}
+
 // Pass B for the calling warp's sub-range: g = warp base wb[e] + loc is the
 // pair's rank among all pairs of its expert in (t, k) order; the host
 // interval holding g gives the buffer row hdst[h] + g, a global row in
 // [0, rows).  Pair i of the sub-range is pair p0 + i of dst_pos; row_src
-// (may be null) gets the inverse.  Returns the number of the warp's pairs
-// that land on another rank than their source rank: src_rank >= 0 is the
-// source rank of every pair (one rank's pairs), -1 derives it as p / C.
+// (may be null) gets the inverse; a row out of range sets MOONEP_ST_ROW_RANGE
+// in *status.  Returns the number of the warp's pairs that land on another
+// rank than their source rank: src_rank >= 0 is the source rank of every pair
+// (one rank's pairs), -1 derives it as p / C.
 __device__ __forceinline__ int assign_pass_b(const int *ids, const int *wb, const int *hptr, const int *hstart,
                                              const int *hdst, int wbeg, int wend, int p0, int E, int rows, int C,
                                              const FastDiv &fC, int src_rank, int *dst_pos, int *row_src,
-                                             int *info)
+                                             int *status)
 {
     const int lane = threadIdx.x & 31;
     int remote = 0;
@@ -1153,7 +1457,7 @@ __device__ __forceinline__ int assign_pass_b(const int *ids, const int *wb, cons
         const int dst = hdst[h] + g;
         const int p = p0 + i;
         if (dst < 0 || dst >= rows) {  // cannot happen for a consistent plan
-            atomicOr(info + MOONEP_INFO_STATUS, MOONEP_ST_ROW_RANGE);
+            atomicOr(status, MOONEP_ST_ROW_RANGE);
             dst_pos[p] = -1;
             continue;
         }
@@ -1162,6 +1466,55 @@ __device__ __forceinline__ int assign_pass_b(const int *ids, const int *wb, cons
         // the source rank's first row: the rank of pair p is p / (S*K) = p / C
         const uint32_t src0 = (src_rank >= 0 ? (uint32_t)src_rank : fdiv((uint32_t)p, fC)) * (uint32_t)C;
         remote += (uint32_t)dst - src0 >= (uint32_t)C;
+    }
+    return remote;
+}
+
+// Pass B of the one-kernel planner.  The tables are per warp and expert:
+// dw = the row of rank wb (the warp base) in the expert's first host, pw =
+// the place of that rank among the chunk's pairs sorted by (expert, rank);
+// dlim (per expert) = the first row past the first host (INT_MAX when the
+// expert has one host).  A pair of rank loc in the warp's sub-range thus has
+// row dw + loc, unless that is past the first host, where the host intervals
+// give it; its sorted place is pw + loc.  Its row and pair go to srow[pos] and
+// spair[pos], from which the caller writes row_src in that order (consecutive
+// ranks of an expert have consecutive rows, so those stores coalesce, where
+// one scattered store per pair would be bound by the store unit).  Three
+// shared-memory loads per pair on the common path: the random expert index
+// makes each of them conflict, and they bound this pass.  n: the chunk's pairs.
+__device__ __forceinline__ int assign_pass_b_fused(const int *ids, const int *dw, const int *pw, const int *dlim,
+                                                   const int *hptr, const int *hstart, const int *hdst, int wbeg,
+                                                   int wend, int n, int p0, int E, int rows, int C,
+                                                   const FastDiv &fC, int *dst_pos, int *srow, int *spair,
+                                                   int *status)
+{
+    const int lane = threadIdx.x & 31;
+    int remote = 0;
+    for (int i = wbeg + lane; i < wend; i += 32) {
+        const int v = ids[i];
+        const int e = v & PACK_MASK, loc = v >> PACK_BITS;
+        if (v < 0 || e >= E) continue;  // cannot happen in a non-empty plan
+        int dst = dw[e] + loc;
+        const int pos = pw[e] + loc;
+        if (dst >= dlim[e]) {  // past the expert's first host
+            int h = hptr[e];
+            const int hend = hptr[e + 1];
+            const int g = dst - hdst[h];
+            while (h + 1 < hend && hstart[h + 1] <= g) ++h;
+            dst = hdst[h] + g;
+        }
+        const int p = p0 + i;
+        const bool pos_ok = pos >= 0 && pos < n;
+        if (dst < 0 || dst >= rows || !pos_ok) {  // cannot happen for a consistent plan
+            atomicOr(status, MOONEP_ST_ROW_RANGE);
+            dst_pos[p] = -1;
+            if (pos_ok) srow[pos] = -1;
+            continue;
+        }
+        dst_pos[p] = dst;
+        srow[pos] = dst;
+        spair[pos] = p;
+        remote += (uint32_t)dst - fdiv((uint32_t)p, fC) * (uint32_t)C >= (uint32_t)C;
     }
     return remote;
 }
@@ -1323,31 +1676,7 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
     // plan, the histogram CTAs wrote the empty defaults before the planner
     // wrote its entries over them.)
     if (empty) {
-        const int g = gridDim.x * nt, x0 = blockIdx.x * nt + tid;
-        for (int x = x0; x < R * E; x += g) {
-            a.p.slot_expert[x] = -1;
-            a.p.slot_count[x] = 0;
-        }
-        for (int x = x0; x < R * (E + 1); x += g) a.p.slot_offset[x] = 0;
-        for (int x = x0; x < E + R; x += g) {
-            a.p.rep_expert[x] = -1;
-            a.p.rep_rank[x] = -1;
-            a.p.rep_slot[x] = -1;
-            a.p.rep_quota[x] = 0;
-        }
-        for (int x = x0; x < nh; x += g) {
-            a.p.host_rank[x] = -1;
-            a.p.host_slot[x] = -1;
-            a.p.host_start[x] = 0;
-            a.p.host_quota[x] = 0;
-            a.p.host_local[x] = 0;
-        }
-        for (int x = x0; x <= E; x += g) a.p.host_ptr[x] = 0;
-        for (int x = x0; x < E; x += g) a.p.rep_home_list[x] = -1;
-        for (int i = tid; i < n; i += nt) {
-            a.p.dst_pos[p0 + i] = -1;
-            a.p.row_src[p0 + i] = -1;
-        }
+        write_empty_plan(a, p0, n);
         pdl_wait();  // as below: finish after the histogram grid
         return;
     }
@@ -1356,7 +1685,7 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
     // pass B: g = warp base + loc is the pair's rank among all pairs of its
     // expert in (t, k) order; the host interval holding g gives the buffer row
     int remote = assign_pass_b(ids, cnt + warp * E, hptr, hstart, hdst, wbeg, wend, p0, E, R * C, C, a.fC, -1,
-                               a.p.dst_pos, a.p.row_src, a.p.info);
+                               a.p.dst_pos, a.p.row_src, a.p.info + MOONEP_INFO_STATUS);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) remote += __shfl_xor_sync(FULL_MASK, remote, o);
     if (lane == 0) red[warp] = remote;
@@ -1372,6 +1701,324 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
     pdl_wait();
 }
 
+// ------------------------------------------------------- one-kernel planner
+//
+// When one CTA per SM can hold a chunk of about tokens / SMs tokens beside
+// the planner's shared memory, one launch does the whole plan.  Every CTA stages its chunk's ids, ranks them (pass A),
+// adds the chunk's counts to its group's and takes a ticket.  Once every
+// chunk's counts are in, it sums the expert totals and its chunk's base, runs
+// the planner on them in its own shared memory -- every CTA computes the same
+// plan, so no CTA waits for another's tables -- and places its pairs from its
+// own copy of the host tables (pass B).  One CTA (the last chunk's, which has
+// the fewest pairs) stores the plan tables; the CTA that finishes last writes
+// the info block and resets the header for the next call.  One CTA per SM,
+// not two with half the tokens each: the planner is a chain of short
+// dependent steps, and two of them on one SM take nearly twice as long.
+// The chunking is this kernel's own (at most one chunk per SM); the group
+// counts use the workspace's buffers at its layout (gs_buf), so a workspace
+// may pass between this path and the two-kernel one.
+// The wait for the ticket is bounded: a CTA that gives up (its peers not all
+// resident) counts every pair of the call itself, which is slower but gives
+// the same totals and base, and reports MOONEP_ST_WAIT_TIMEOUT.  A ticket past
+// the chunk count can only come from a workspace that was not zero-filled.
+__host__ __device__ inline int fused_smem_ints(int E, int R, int max_pairs, unsigned flags, int B)
+{
+    // (pass A's lane masks and pass B's places, ASSIGN_WARPS * E words each,
+    // fit in the planner's 22 E + 13 R + 58 ints before its misc words, idle
+    // until the totals and again after the plan)
+    static_assert(ASSIGN_WARPS <= 22, "pass A's lane masks and pass B's places alias the planner's shared memory");
+    return ASSIGN_WARPS * E + (max_pairs + 4) + (E + 1) + 2 * (2 * E + R) + 32 + (E + 1) + 2 * max_pairs +
+           plan_smem_ints(E, R) + ((flags & MOONEP_FLAG_CASCADE) ? cascade_smem_ints(E, R, B) : 0);
+}
+
+__global__ void __launch_bounds__(PLAN_THREADS, 1) plan_fused_kernel(PlanParams a)
+{
+    extern __shared__ __align__(16) int sm[];
+    const Dims &d = a.d;
+    const int E = d.E, K = d.K, R = d.R, C = d.C;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int nt = PLAN_THREADS;
+    static_assert(PLAN_THREADS == ASSIGN_THREADS, "one block size for the planner and the passes");
+    const int chunk = blockIdx.x, nchunk = gridDim.x;
+    const int t0 = chunk * d.chunk_tokens;
+    const int t1 = min(t0 + d.chunk_tokens, d.tokens);
+    const int p0 = t0 * K, n = (t1 - t0) * K;
+    const int max_pairs = d.chunk_tokens * K;
+    const int nh = 2 * E + R;
+
+    int *cnt = sm;                           // ASSIGN_WARPS * E: warp counts, then warp bases
+    int *ids_raw = cnt + ASSIGN_WARPS * E;   // max_pairs + 4, 16-byte aligned: from pair p0 & ~3 on
+    int *ids = ids_raw + (p0 & 3);           // the chunk's pairs
+    int *hptr = ids_raw + max_pairs + 4;     // E + 1
+    int *hstart = hptr + E + 1;              // nh
+    int *hdst = hstart + nh;                 // nh; first each expert's pairs in earlier chunks
+    int *red = hdst + nh;                    // 32
+    int *cho = red + 32;                     // E (+1 pad): the chunk's counts, then their exclusive prefix
+    int *srow = cho + E + 1;                 // max_pairs: the chunk's rows in (expert, rank) order
+    int *spair = srow + max_pairs;           // max_pairs: and their pairs
+    int *psm = spair + max_pairs;            // the planner's; first pass A's lane masks (ASSIGN_WARPS * E)
+    unsigned *mk = reinterpret_cast<unsigned *>(psm);
+    int *T = psm;
+    const int *misc = plan_misc(psm, E, R);
+    __shared__ int s_seq, s_wait, s_status;
+
+    // placed while the stream's previous kernel drains: wait for it before
+    // touching memory
+    pdl_wait();
+    for (int i = tid; i < ASSIGN_WARPS * E; i += nt) {
+        cnt[i] = 0;
+        mk[i] = 0;
+    }
+    // the chunk's ids: 16-byte loads, all of a thread's in flight together
+    // (from pair p0 & ~3 on, so the loads are aligned; the few before p0 are
+    // the previous chunk's and are not used), then the last < 4 one by one
+    int bad = 0;
+    {
+        const int q0 = p0 >> 2, q1 = (p0 + n) >> 2;  // 16-byte words wholly or partly before p0 + n
+        const bool vec = (reinterpret_cast<uintptr_t>(a.topk) & 15) == 0;
+        const int nv = vec ? q1 - q0 : 0;
+        const int4 *src = reinterpret_cast<const int4 *>(a.topk) + q0;
+        constexpr int VB = 4;
+        for (int k0 = tid; k0 < nv; k0 += VB * nt) {
+            int4 v[VB];
+#pragma unroll
+            for (int j = 0; j < VB; ++j)
+                if (k0 + j * nt < nv) v[j] = __ldg(src + k0 + j * nt);
+#pragma unroll
+            for (int j = 0; j < VB; ++j) {
+                const int k = k0 + j * nt;
+                if (k < nv) {
+                    reinterpret_cast<int4 *>(ids_raw)[k] = v[j];
+                    const int q = 4 * (q0 + k);  // pair of v[j].x
+                    const int x[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        if (q + c >= p0) bad |= x[c] < 0 || x[c] >= E;
+                }
+            }
+        }
+        for (int i = (vec ? max(4 * q1 - p0, 0) : 0) + tid; i < n; i += nt) {
+            const int e = __ldg(a.topk + p0 + i);
+            ids[i] = e;
+            bad |= e < 0 || e >= E;
+        }
+    }
+    if (tid == 0) s_seq = ld_cg(a.hdr + WS_SEQ);
+    for (int x = tid; x < n; x += nt) srow[x] = -1;  // a place pass B leaves unset writes no row_src
+    bad = __syncthreads_or(bad);
+    const int seq = s_seq, parity = seq & 1;
+    {  // the previous call's group counts are read by nobody now: zero them for the next call
+        int *old = a.gs + (size_t)(parity ^ 1) * a.gs_buf;
+        for (int i = chunk * nt + tid; i < a.gs_buf; i += nchunk * nt) old[i] = 0;
+    }
+
+    // pass A, then the chunk's counts (column sums of the warp counters)
+    const int per = (n + ASSIGN_WARPS - 1) / ASSIGN_WARPS;
+    const int wbeg = min(warp * per, n), wend = min(wbeg + per, n);
+    assign_pass_a_mask(ids, cnt + warp * E, mk + warp * E, wbeg, wend, E);
+    __syncthreads();
+    {
+        int *gsb = a.gs + (size_t)parity * a.gs_buf + (size_t)(chunk / CHUNK_GROUP) * E;
+        for (int e = tid; e < E; e += nt) {
+            int c = 0;
+#pragma unroll 4
+            for (int w = 0; w < ASSIGN_WARPS; ++w) c += cnt[w * E + e];
+            a.cc[(size_t)chunk * E + e] = c;
+            cho[e] = c;
+            if (c) atomicAdd(gsb + e, c);  // sums: order-free
+        }
+    }
+    // release the counts with the ticket, then wait (bounded) for every chunk's
+    __syncthreads();
+    int mine = 0;
+    if (tid == 0) {
+        if (bad) atomicOr(a.hdr + WS_STATUS, MOONEP_ST_EXPERT_ID_RANGE);
+        __threadfence();
+        mine = atomicAdd(a.hdr + WS_TICKET, 1) + 1;
+    }
+    // while the other chunks arrive: where each expert's pairs start among
+    // this chunk's pairs sorted by expert
+    block_exscan(cho, E, red);
+    if (tid == 0) {
+        int w = 0, st = 0;  // w: 0 gave up, 1 every chunk in, 2 ticket past the chunk count
+        if (mine == nchunk) w = 1;
+        else if (mine > nchunk || mine <= 0) w = 2;
+        for (int it = 0; w == 0 && it < a.spin_limit; ++it) {
+            const int tk = ld_acquire(a.hdr + WS_TICKET);
+            if (tk == nchunk) w = 1;
+            else if (tk > nchunk || tk <= 0) w = 2;
+            else __nanosleep(32);
+        }
+        if (w == 1) {
+            __threadfence();
+            st = ld_cg(a.hdr + WS_STATUS);
+        }
+        s_wait = w;
+        s_status = st;
+    }
+    __syncthreads();
+    const int wstate = s_wait;
+    int status_in = s_status;
+
+    // ---- the expert totals T and this chunk's base (pairs of each expert in
+    // earlier chunks, into hdst for now)
+    const int grp = chunk / CHUNK_GROUP, c0 = grp * CHUNK_GROUP;
+    unsigned part = 0;  // <= 2 values < 2^31 each (negative ones are flagged)
+    int negative = 0;
+    if (wstate == 1) {
+        const int *gsb = a.gs + (size_t)parity * a.gs_buf;
+        for (int e = tid; e < E; e += nt) {
+            int w[CHUNK_GROUP - 1];
+#pragma unroll
+            for (int j = 0; j < CHUNK_GROUP - 1; ++j)
+                w[j] = (c0 + j < chunk) ? ld_cg(a.cc + (size_t)(c0 + j) * E + e) : 0;
+            int tot = 0, before = 0;
+            for (int g0 = 0; g0 < d.ngroups; g0 += 32) {
+                int v[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] = (g0 + j < d.ngroups) ? ld_cg(gsb + (size_t)(g0 + j) * E + e) : 0;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    tot += v[j];
+                    before += (g0 + j < grp) ? v[j] : 0;
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < CHUNK_GROUP - 1; ++j) before += w[j];
+            T[e] = tot;
+            hdst[e] = before;
+            negative |= tot < 0;
+            part += (unsigned)tot;
+        }
+    } else {
+        for (int e = tid; e < E; e += nt) {
+            T[e] = 0;
+            hdst[e] = 0;
+        }
+        if (wstate == 0) {  // gave up waiting: count every pair of the call here
+            __syncthreads();
+            int bad_any = 0;
+            for (int p = tid; p < d.pairs; p += nt) {
+                const int e = __ldg(a.topk + p);
+                if (e < 0 || e >= E) {
+                    bad_any = 1;
+                    continue;
+                }
+                atomicAdd(&T[e], 1);
+                if (p < p0) atomicAdd(&hdst[e], 1);
+            }
+            bad_any = __syncthreads_or(bad_any);
+            status_in = bad_any ? MOONEP_ST_EXPERT_ID_RANGE : 0;
+            if (tid == 0) atomicOr(a.hdr + WS_FLAGS, MOONEP_ST_WAIT_TIMEOUT);
+        } else {
+            status_in = MOONEP_ST_WORKSPACE;
+        }
+    }
+    // with every id valid the summed totals must be non-negative and add up
+    // to the pairs; anything else means the workspace was not zeroed (exact
+    // 64-bit total from 16-bit halves, each warp sum by one reduction)
+    {
+        const unsigned lo = __reduce_add_sync(FULL_MASK, part & 0xffffu);
+        const unsigned hi = __reduce_add_sync(FULL_MASK, part >> 16);
+        if (lane == 0) {
+            red[warp] = (int)lo;
+            red[16 + warp] = (int)hi;
+        }
+    }
+    negative = __syncthreads_or(negative);
+    if (wstate == 1) {
+        const unsigned lo = __reduce_add_sync(FULL_MASK, lane < ASSIGN_WARPS ? (unsigned)red[lane] : 0u);
+        const unsigned hi = __reduce_add_sync(FULL_MASK, lane < ASSIGN_WARPS ? (unsigned)red[16 + lane] : 0u);
+        const long long total = ((long long)hi << 16) + (long long)lo;
+        if (!(status_in & MOONEP_ST_EXPERT_ID_RANGE) && (negative || total != (long long)d.pairs))
+            status_in |= MOONEP_ST_WORKSPACE;
+    }
+    // warp bases: the chunk's base plus the earlier warps' counts
+    for (int e = tid; e < E; e += nt) {
+        int sb = hdst[e];
+        for (int w = 0; w < ASSIGN_WARPS; ++w) {
+            const int t = cnt[w * E + e];
+            cnt[w * E + e] = sb;
+            sb += t;
+        }
+    }
+    const bool writer = chunk == nchunk - 1;
+    if (writer)
+        for (int e = tid; e < E; e += nt) a.p.expert_count[e] = T[e];
+    __syncthreads();
+
+    const bool empty = (status_in & ST_EMPTY_PLAN) != 0;
+    int remote = 0;
+    if (empty) {
+        write_empty_plan(a, p0, n);
+    } else {
+        plan_core(a, psm, seq, PlanSink{false, writer, hptr, hstart, hdst});
+        __syncthreads();
+        // pass B's tables, from this CTA's own host tables: dw over the warp
+        // bases, pw in the planner's shared memory (its first ASSIGN_WARPS * E
+        // ints, clear of the misc words at its end), dlim over cho
+        int *dw = cnt, *pw = psm, *dlim = cho;
+        for (int e = tid; e < E; e += nt) {
+            const int h0 = hptr[e], d0 = hdst[h0];
+            const int po = cho[e] - cnt[e];  // cnt[e]: warp 0's base, the chunk's first rank of e
+            for (int w = 0; w < ASSIGN_WARPS; ++w) {
+                const int wb = cnt[w * E + e];
+                dw[w * E + e] = d0 + wb;
+                pw[w * E + e] = po + wb;
+            }
+            dlim[e] = hptr[e + 1] - h0 > 1 ? d0 + hstart[h0 + 1] : INT_MAX;
+        }
+        __syncthreads();
+        // pass B, then row_src in (expert, rank) order
+        remote = assign_pass_b_fused(ids, dw + warp * E, pw + warp * E, dlim, hptr, hstart, hdst, wbeg, wend, n, p0,
+                                     E, R * C, C, a.fC, a.p.dst_pos, srow, spair, a.hdr + WS_FLAGS);
+        __syncthreads();
+        for (int x = tid; x < n; x += nt) {
+            const int r = srow[x];
+            if (r >= 0) a.p.row_src[r] = spair[x];
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) remote += __shfl_xor_sync(FULL_MASK, remote, o);
+    if (lane == 0) red[warp] = remote;
+    __syncthreads();
+    if (tid == 0) {
+        int sr = 0;
+        for (int w = 0; w < ASSIGN_WARPS; ++w) sr += red[w];
+        if (sr) atomicAdd(a.hdr + WS_REMOTE, sr);
+        // the CTA that finishes last: the info block, and the header reset
+        // for the next call (which starts after this grid has finished)
+        __threadfence();
+        if (atomicAdd(a.hdr + WS_ARRIVED, 1) == nchunk - 1) {
+            __threadfence();
+            const int late = atomicExch(a.hdr + WS_FLAGS, 0);
+            const int remote_all = atomicExch(a.hdr + WS_REMOTE, 0);
+            int *info = a.p.info;
+            for (int i = 1; i < MOONEP_INFO_LEN; ++i) info[i] = 0;
+            if (empty) {
+                info[MOONEP_INFO_STATUS] = status_in | late;
+            } else {
+                info[MOONEP_INFO_STATUS] = misc[MISC_PLAN_STATUS] | late;
+                info[MOONEP_INFO_N_REP] = misc[MISC_N_REP];
+                info[MOONEP_INFO_N_OVERFLOW] = misc[MISC_N_OVER];
+                info[MOONEP_INFO_N_PIECES] = misc[MISC_N_PIECES];
+                info[MOONEP_INFO_N_RECEIVERS] = misc[MISC_N_RECEIVERS];
+                info[MOONEP_INFO_MAX_REP_PER_RANK] = misc[MISC_MAX_REP];
+                info[MOONEP_INFO_N_REP_EXPERTS] = misc[MISC_N_REP_EXPERTS];
+                info[MOONEP_INFO_N_REMOTE_PAIRS] = remote_all;
+                info[MOONEP_INFO_CASCADE_GUARD_STEPS] = misc[MISC_GUARD_STEPS];
+                info[MOONEP_INFO_CASCADE_GUARD_SLACK] = misc[MISC_GUARD_SLACK];
+            }
+            a.hdr[WS_TICKET] = 0;
+            a.hdr[WS_STATUS] = 0;
+            a.hdr[WS_ARRIVED] = 0;
+            a.hdr[WS_READY] = seq + 1;
+            a.hdr[WS_PLANNED] = seq + 1;
+            a.hdr[WS_SEQ] = seq + 1;
+        }
+    }
+}
+
 // ---------------------------------------------------------------- launch
 
 // Both planner kernels ask for the largest shared-memory carveout: an SM
@@ -1381,7 +2028,7 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
 // launch needs more dynamic shared memory than was allowed so far: the
 // driver calls cost host time on every plan of a latency-bound layer.
 constexpr int SMEM_CACHE_DEVICES = 64;
-enum { K_HIST, K_ASSIGN, K_EP_COUNT, K_EP_PLAN, K_EP_ASSIGN, K_N };
+enum { K_HIST, K_ASSIGN, K_EP_COUNT, K_EP_PLAN, K_EP_ASSIGN, K_FUSED, K_N };
 static std::atomic<size_t> g_smem_set[SMEM_CACHE_DEVICES][K_N];  // bytes allowed so far, 0 = never set
 
 static bool set_smem(int which, const void *fn, size_t bytes)
@@ -1402,6 +2049,45 @@ static bool set_smem(int which, const void *fn, size_t bytes)
     return ok;
 }
 
+// moonep_set_plan_path: 0 lets launch_plan choose, 1 keeps it on the
+// two-kernel path (for tests that compare the two)
+static std::atomic<int> g_plan_path{0};
+
+int set_plan_path(int mode) { return g_plan_path.exchange(mode == 1 ? 1 : 0); }
+
+// Resident CTAs per SM of the one-kernel planner with `smem` bytes of dynamic
+// shared memory, on the current device (cached per device for the last few
+// sizes: a plan call makes no occupancy query once its size has been seen).
+constexpr int OCC_SLOTS = 4;
+struct OccCache {
+    std::mutex m;
+    size_t smem[OCC_SLOTS] = {};
+    int blocks[OCC_SLOTS] = {};
+    int next = 0;
+};
+static OccCache g_occ[SMEM_CACHE_DEVICES];
+
+static int fused_blocks_per_sm(size_t smem)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= SMEM_CACHE_DEVICES) return 0;
+    OccCache &c = g_occ[dev];
+    std::lock_guard<std::mutex> lock(c.m);
+    for (int i = 0; i < OCC_SLOTS; ++i)
+        if (c.smem[i] == smem && c.blocks[i] > 0) return c.blocks[i];
+    int nb = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, plan_fused_kernel, PLAN_THREADS, smem) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return 0;
+    }
+    c.smem[c.next] = smem;
+    c.blocks[c.next] = nb;
+    c.next = (c.next + 1) % OCC_SLOTS;
+    return nb;
+}
+
+constexpr size_t MAX_BLOCK_SMEM = 227 * 1024;
+
 int launch_plan(const Dims &d, const int32_t *topk, const moonep_plan_t &p, void *ws, cudaStream_t st)
 {
     const WsLayout wl = ws_layout(d);
@@ -1415,6 +2101,7 @@ int launch_plan(const Dims &d, const int32_t *topk, const moonep_plan_t &p, void
     a.cc = reinterpret_cast<int *>(w + wl.cc);
     a.host_dst0 = reinterpret_cast<int *>(w + wl.host_dst0);
     a.gs_stride = d.E;
+    a.gs_buf = d.ngroups * d.E;
     a.fC = make_fastdiv((uint32_t)d.C);
     a.fL = make_fastdiv((uint32_t)d.L);
     a.spin_limit = g_wait_limit.load(std::memory_order_relaxed);
@@ -1426,6 +2113,33 @@ int launch_plan(const Dims &d, const int32_t *topk, const moonep_plan_t &p, void
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+
+    // one kernel when one CTA per SM holds a chunk of tokens / SMs tokens (at
+    // least 8) beside the planner: its chunking is coarser than the
+    // two-kernel path's, so it fits in the workspace laid out for that
+    if (g_plan_path.load(std::memory_order_relaxed) == 0) {
+        PlanParams af = a;
+        Dims &df = af.d;
+        int ct = (d.tokens + d.nsm - 1) / d.nsm;
+        if (ct < 8) ct = 8;
+        if (ct > d.tokens) ct = d.tokens;
+        df.chunk_tokens = ct;
+        df.nchunk = (d.tokens + ct - 1) / ct;
+        df.ngroups = (df.nchunk + CHUNK_GROUP - 1) / CHUNK_GROUP;
+        const size_t smemf = sizeof(int) * (size_t)fused_smem_ints(d.E, d.R, ct * d.K, d.flags, d.B);
+        if (df.nchunk <= d.nchunk && df.nchunk <= d.nsm && smemf <= MAX_BLOCK_SMEM &&
+            set_smem(K_FUSED, (const void *)plan_fused_kernel, smemf) && fused_blocks_per_sm(smemf) >= 1) {
+            cudaLaunchConfig_t cf = {};
+            cf.gridDim = dim3(df.nchunk);
+            cf.blockDim = dim3(PLAN_THREADS);
+            cf.dynamicSmemBytes = smemf;
+            cf.stream = st;
+            cf.attrs = attr;
+            cf.numAttrs = 1;
+            return cudaLaunchKernelEx(&cf, plan_fused_kernel, af) == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
+        }
+        (void)cudaGetLastError();  // a refused attribute leaves the two-kernel path
+    }
 
     const size_t smem1 = sizeof(int) * (size_t)hist_smem_ints(d.E, d.R, d.chunk_tokens * d.K, d.flags, d.B);
     if (!set_smem(K_HIST, (const void *)hist_plan_kernel, smem1)) return MOONEP_ERR_CUDA;
@@ -1702,7 +2416,7 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) ep_assign_kernel(PlanParams
                                      p0, E, R * C, C, rank, a.p.dst_pos, a.p.info);
     } else {
         remote = assign_pass_b(ids, cnt + warp * E, hptr, hstart, hdst, wbeg, wend, p0, E, R * C, C, a.fC, rank,
-                               a.p.dst_pos, nullptr, a.p.info);
+                               a.p.dst_pos, nullptr, a.p.info + MOONEP_INFO_STATUS);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) remote += __shfl_xor_sync(FULL_MASK, remote, o);
@@ -1753,6 +2467,7 @@ int launch_ep_plan(const Dims &d, int rank, const int32_t *topk, const int32_t *
     a.hdr = reinterpret_cast<int *>(w + wl.hdr);
     a.gs = const_cast<int *>(counts_all);
     a.gs_stride = d.E + 1;
+    a.gs_buf = 0;  // the gathered counts are one buffer, rewritten by the caller every call
     a.cc = reinterpret_cast<int *>(w + wl.cc);
     a.host_dst0 = reinterpret_cast<int *>(w + wl.host_dst0);
     a.fC = make_fastdiv((uint32_t)d.C);

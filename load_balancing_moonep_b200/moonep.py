@@ -58,7 +58,8 @@ EXPORTED = ("moonep_check_config", "moonep_plan_sizes", "moonep_plan_layout", "m
             "moonep_plan_noalloc", "moonep_prefetch_replicas", "moonep_status_string",
             "moonep_set_wait_limit", "moonep_ep_sizes", "moonep_ep_count", "moonep_ep_plan",
             "moonep_ep_dispatch", "moonep_ep_combine", "moonep_ep_combine_backward",
-            "moonep_ep_reduce_replica_grads", "moonep_ep_prefetch_replicas", "moonep_set_cascade_capacity")
+            "moonep_ep_reduce_replica_grads", "moonep_ep_prefetch_replicas", "moonep_set_cascade_capacity",
+            "moonep_set_plan_path")
 
 
 class _CConfig(ctypes.Structure):
@@ -91,6 +92,7 @@ _lib.moonep_status_string.restype = ctypes.c_char_p
 _lib.moonep_abi_version.argtypes = []
 _lib.moonep_set_wait_limit.argtypes = [ctypes.c_int]
 _lib.moonep_set_cascade_capacity.argtypes = [ctypes.c_int]
+_lib.moonep_set_plan_path.argtypes = [ctypes.c_int]
 _lib.moonep_ep_sizes.argtypes = [_cfgp, ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)]
 _lib.moonep_ep_count.argtypes = [_cfgp, _vp, _vp, _vp, _vp]
 _lib.moonep_ep_plan.argtypes = [_cfgp, ctypes.c_int32, _vp, _vp, _planp, _vp, _vp]
@@ -526,6 +528,16 @@ def set_cascade_capacity(capacity: int) -> int:
     (0 for the default).  Lowering it makes the guard stricter; tests use it
     to put a repair step exactly on the limit."""
     return _lib.moonep_set_cascade_capacity(int(capacity))
+
+
+def set_plan_path(mode: int) -> int:
+    """Which planner later plan calls launch: 1 the two-kernel planner
+    always, 0 (the default) the one-kernel planner where its CTAs all fit on
+    the device at once; returns the previous setting.  Both give the same
+    plan."""
+    if mode not in (0, 1):
+        raise ValueError(f"plan path must be 0 or 1, got {mode}")
+    return _lib.moonep_set_plan_path(int(mode))
 
 
 def abi_version() -> int:

@@ -32,6 +32,15 @@ def mp(oracle_lib, cuda_lib_path):
     return moonep
 
 
+@pytest.fixture(autouse=True, params=["one-kernel", "two-kernel"])
+def plan_path(request, mp):
+    """Every test runs under both planners (moonep_set_plan_path): the one
+    kernel wherever its CTAs all fit on the GPU, and the two-kernel path."""
+    prev = mp.set_plan_path(1 if request.param == "two-kernel" else 0)
+    yield request.param
+    mp.set_plan_path(prev)
+
+
 def _cfg(mp, wl, flags=0):
     c = dict(R=wl.R, E=wl.E, K=wl.K, S=wl.S, H=wl.H, B=wl.B, flags=flags)
     return mp.Config(**c), oracle.Config(**c)

@@ -38,6 +38,15 @@ def mp(oracle_lib, cuda_lib_path):
     return moonep
 
 
+@pytest.fixture(autouse=True, params=["one-kernel", "two-kernel"])
+def plan_path(request, mp):
+    """Every test runs under both planners (moonep_set_plan_path): the one
+    kernel wherever its CTAs all fit on the GPU, and the two-kernel path."""
+    prev = mp.set_plan_path(1 if request.param == "two-kernel" else 0)
+    yield request.param
+    mp.set_plan_path(prev)
+
+
 def _cfgs(c: dict, mp):
     return mp.Config(**c), oracle.Config(**c)
 

@@ -1,0 +1,120 @@
+"""The two planners of moonep_plan.
+
+moonep_plan launches one kernel when every CTA of its grid fits on the GPU
+at once (every CTA then computes the whole plan in its own shared memory),
+and two kernels otherwise (a histogram pass whose last CTA plans, then an
+assignment pass); moonep_set_plan_path(1) keeps it on the two.  The parity
+and failure-path modules run every test under both; this one checks which
+kernels a call launches, that one workspace may pass between the two from
+call to call, and that a shape too large for the one kernel takes the two
+without being asked.
+"""
+import numpy as np
+import pytest
+import torch
+from torch.profiler import ProfilerActivity, profile
+
+import oracle
+from load_balancing_moonep_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module")
+def mp(oracle_lib, cuda_lib_path):
+    if not torch.cuda.is_available():
+        pytest.fail("CUDA device required for -m gpu tests")
+    from load_balancing_moonep_b200 import moonep
+    return moonep
+
+
+def _kernels(fn):
+    """Names of the CUDA kernels fn launches (profiler trace)."""
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        fn()
+        torch.cuda.synchronize()
+    return [e.name for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA]
+
+
+def _cfg(mp, wl, flags=0):
+    c = dict(R=wl.R, E=wl.E, K=wl.K, S=wl.S, H=wl.H, B=wl.B, flags=flags)
+    return mp.Config(**c), oracle.Config(**c)
+
+
+def _assert_equal(gp, op, label):
+    g = gp.to_numpy()
+    for k, v in op.items():
+        assert np.array_equal(g[k], v), f"{label}: plan field {k} differs"
+
+
+@pytest.mark.parametrize("wname", ["tiny", "decode", "large"])
+def test_a_call_launches_the_chosen_planner(mp, wname):
+    wl = W.WORKLOADS[wname]
+    gcfg, _ = _cfg(mp, wl)
+    topk = W.routing(wl, 1.0, device=DEV).topk_idx
+    p = mp.Plan(gcfg)
+    prev = mp.set_plan_path(0)
+    try:
+        one = _kernels(lambda: mp.plan(gcfg, topk, out=p))
+        mp.set_plan_path(1)
+        two = _kernels(lambda: mp.plan(gcfg, topk, out=p))
+    finally:
+        mp.set_plan_path(prev)
+    assert any("plan_fused_kernel" in k for k in one), one
+    assert not any("hist_plan_kernel" in k or "assign_kernel" in k for k in one), one
+    assert any("hist_plan_kernel" in k for k in two) and any("assign_kernel" in k for k in two), two
+    assert not any("plan_fused_kernel" in k for k in two), two
+
+
+def test_one_workspace_alternates_between_the_planners(mp):
+    # the two leave the workspace header in the same state after a call, so
+    # a workspace may switch path from one call to the next
+    wl = W.WORKLOADS["mid"]
+    gcfg, ocfg = _cfg(mp, wl)
+    routings = [W.routing(wl, mv, seed=s, device=DEV).topk_idx for s, mv in ((0, 0.5), (1, 3.0))]
+    expect = [oracle.plan(ocfg, t.cpu().numpy()) for t in routings]
+    p = mp.Plan(gcfg)
+    prev = mp.set_plan_path(0)
+    try:
+        for call in range(8):
+            mp.set_plan_path((call // 2) % 2)
+            i = call % 2
+            mp.plan(gcfg, routings[i], out=p)
+            torch.cuda.synchronize()
+            _assert_equal(p, expect[i], f"call {call} (path {(call // 2) % 2})")
+    finally:
+        mp.set_plan_path(prev)
+
+
+def test_a_shape_too_large_for_one_kernel_takes_two(mp):
+    # E = R = 1024 with the relay cascade: the planner's shared memory does
+    # not fit two CTAs per SM beside the pass's, so the two kernels run
+    c = dict(R=1024, E=1024, K=1, S=4, H=8, B=1, flags=8)
+    gcfg, ocfg = mp.Config(**c), oracle.Config(**c)
+    rng = np.random.default_rng(3)
+    topk = rng.integers(0, 1024, size=(1024 * 4, 1)).astype(np.int32)
+    t = torch.from_numpy(topk).to(DEV)
+    holder = {}
+    names = _kernels(lambda: holder.setdefault("p", mp.plan(gcfg, t)))
+    assert any("hist_plan_kernel" in k for k in names), names
+    assert not any("plan_fused_kernel" in k for k in names), names
+    _assert_equal(holder["p"], oracle.plan(ocfg, topk), "E = R = 1024")
+
+
+@pytest.mark.parametrize("wname,shift", [("mid", 1), ("mid", 3), ("large", 2)])
+def test_ids_not_16_byte_aligned(mp, wname, shift):
+    # the one-kernel planner reads the ids in 16-byte words when topk_idx is
+    # 16-byte aligned, one by one otherwise: a view starting `shift` ints
+    # into a buffer takes the second way, and the plan is the same
+    wl = W.WORKLOADS[wname]
+    gcfg, ocfg = _cfg(mp, wl)
+    topk = W.routing(wl, 2.0, device=DEV).topk_idx
+    buf = torch.empty(topk.numel() + 4, dtype=torch.int32, device=DEV)
+    view = buf[shift:shift + topk.numel()].view(topk.shape)
+    view.copy_(topk)
+    assert view.data_ptr() % 16 != 0
+    gp = mp.plan(gcfg, view)
+    torch.cuda.synchronize()
+    _assert_equal(gp, oracle.plan(ocfg, topk.cpu().numpy()), f"{wname} shift {shift}")

@@ -1470,23 +1470,20 @@ __device__ __forceinline__ int assign_pass_b(const int *ids, const int *wb, cons
     return remote;
 }
 
-// Pass B of the one-kernel planner.  The tables are per warp and expert:
-// dw = the row of rank wb (the warp base) in the expert's first host, pw =
-// the place of that rank among the chunk's pairs sorted by (expert, rank);
-// dlim (per expert) = the first row past the first host (INT_MAX when the
-// expert has one host).  A pair of rank loc in the warp's sub-range thus has
-// row dw + loc, unless that is past the first host, where the host intervals
-// give it; its sorted place is pw + loc.  Its row and pair go to srow[pos] and
-// spair[pos], from which the caller writes row_src in that order (consecutive
-// ranks of an expert have consecutive rows, so those stores coalesce, where
-// one scattered store per pair would be bound by the store unit).  Three
-// shared-memory loads per pair on the common path: the random expert index
-// makes each of them conflict, and they bound this pass.  n: the chunk's pairs.
-__device__ __forceinline__ int assign_pass_b_fused(const int *ids, const int *dw, const int *pw, const int *dlim,
-                                                   const int *hptr, const int *hstart, const int *hdst, int wbeg,
-                                                   int wend, int n, int p0, int E, int rows, int C,
-                                                   const FastDiv &fC, int *dst_pos, int *srow, int *spair,
-                                                   int *status)
+// Pass B of the one-kernel planner.  dw (per warp and expert) = the row of
+// rank wb (the warp base) in the expert's first host; dlim (per expert) = the
+// first row past the first host (INT_MAX when the expert has one host).  A
+// pair of rank loc in the warp's sub-range thus has row dw + loc, unless that
+// is past the first host, where the host intervals give it: two
+// shared-memory loads per pair on the common path, where the generic pass
+// makes about six.  Their random expert index makes each of them conflict,
+// and they bound this pass.  (Staging row_src in shared memory in (expert,
+// rank) order, so that its stores coalesce, measured 1.9 µs slower at the
+// large shape than these scattered stores.)
+__device__ __forceinline__ int assign_pass_b_fused(const int *ids, const int *dw, const int *dlim, const int *hptr,
+                                                   const int *hstart, const int *hdst, int wbeg, int wend, int p0,
+                                                   int E, int rows, int C, const FastDiv &fC, int *dst_pos,
+                                                   int *row_src, int *status)
 {
     const int lane = threadIdx.x & 31;
     int remote = 0;
@@ -1495,7 +1492,6 @@ __device__ __forceinline__ int assign_pass_b_fused(const int *ids, const int *dw
         const int e = v & PACK_MASK, loc = v >> PACK_BITS;
         if (v < 0 || e >= E) continue;  // cannot happen in a non-empty plan
         int dst = dw[e] + loc;
-        const int pos = pw[e] + loc;
         if (dst >= dlim[e]) {  // past the expert's first host
             int h = hptr[e];
             const int hend = hptr[e + 1];
@@ -1504,16 +1500,13 @@ __device__ __forceinline__ int assign_pass_b_fused(const int *ids, const int *dw
             dst = hdst[h] + g;
         }
         const int p = p0 + i;
-        const bool pos_ok = pos >= 0 && pos < n;
-        if (dst < 0 || dst >= rows || !pos_ok) {  // cannot happen for a consistent plan
+        if (dst < 0 || dst >= rows) {  // cannot happen for a consistent plan
             atomicOr(status, MOONEP_ST_ROW_RANGE);
             dst_pos[p] = -1;
-            if (pos_ok) srow[pos] = -1;
             continue;
         }
         dst_pos[p] = dst;
-        srow[pos] = dst;
-        spair[pos] = p;
+        row_src[dst] = p;
         remote += (uint32_t)dst - fdiv((uint32_t)p, fC) * (uint32_t)C >= (uint32_t)C;
     }
     return remote;
@@ -1723,12 +1716,11 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
 // the chunk count can only come from a workspace that was not zero-filled.
 __host__ __device__ inline int fused_smem_ints(int E, int R, int max_pairs, unsigned flags, int B)
 {
-    // (pass A's lane masks and pass B's places, ASSIGN_WARPS * E words each,
-    // fit in the planner's 22 E + 13 R + 58 ints before its misc words, idle
-    // until the totals and again after the plan)
-    static_assert(ASSIGN_WARPS <= 22, "pass A's lane masks and pass B's places alias the planner's shared memory");
-    return ASSIGN_WARPS * E + (max_pairs + 4) + (E + 1) + 2 * (2 * E + R) + 32 + (E + 1) + 2 * max_pairs +
-           plan_smem_ints(E, R) + ((flags & MOONEP_FLAG_CASCADE) ? cascade_smem_ints(E, R, B) : 0);
+    // (pass A's lane masks, ASSIGN_WARPS * E words, fit in the planner's
+    // 22 E + 13 R + 58 ints, which are idle until the totals)
+    static_assert(ASSIGN_WARPS <= 22, "pass A's lane masks alias the planner's shared memory");
+    return ASSIGN_WARPS * E + (max_pairs + 4) + (E + 1) + 2 * (2 * E + R) + 32 + (E + 1) + plan_smem_ints(E, R) +
+           ((flags & MOONEP_FLAG_CASCADE) ? cascade_smem_ints(E, R, B) : 0);
 }
 
 __global__ void __launch_bounds__(PLAN_THREADS, 1) plan_fused_kernel(PlanParams a)
@@ -1753,10 +1745,8 @@ __global__ void __launch_bounds__(PLAN_THREADS, 1) plan_fused_kernel(PlanParams 
     int *hstart = hptr + E + 1;              // nh
     int *hdst = hstart + nh;                 // nh; first each expert's pairs in earlier chunks
     int *red = hdst + nh;                    // 32
-    int *cho = red + 32;                     // E (+1 pad): the chunk's counts, then their exclusive prefix
-    int *srow = cho + E + 1;                 // max_pairs: the chunk's rows in (expert, rank) order
-    int *spair = srow + max_pairs;           // max_pairs: and their pairs
-    int *psm = spair + max_pairs;            // the planner's; first pass A's lane masks (ASSIGN_WARPS * E)
+    int *dlim = red + 32;                    // E (+1 pad): pass B's first row past each expert's first host
+    int *psm = dlim + E + 1;                 // the planner's; first pass A's lane masks (ASSIGN_WARPS * E)
     unsigned *mk = reinterpret_cast<unsigned *>(psm);
     int *T = psm;
     const int *misc = plan_misc(psm, E, R);
@@ -1804,7 +1794,6 @@ __global__ void __launch_bounds__(PLAN_THREADS, 1) plan_fused_kernel(PlanParams 
         }
     }
     if (tid == 0) s_seq = ld_cg(a.hdr + WS_SEQ);
-    for (int x = tid; x < n; x += nt) srow[x] = -1;  // a place pass B leaves unset writes no row_src
     bad = __syncthreads_or(bad);
     const int seq = s_seq, parity = seq & 1;
     {  // the previous call's group counts are read by nobody now: zero them for the next call
@@ -1824,7 +1813,6 @@ __global__ void __launch_bounds__(PLAN_THREADS, 1) plan_fused_kernel(PlanParams 
 #pragma unroll 4
             for (int w = 0; w < ASSIGN_WARPS; ++w) c += cnt[w * E + e];
             a.cc[(size_t)chunk * E + e] = c;
-            cho[e] = c;
             if (c) atomicAdd(gsb + e, c);  // sums: order-free
         }
     }
@@ -1836,9 +1824,6 @@ __global__ void __launch_bounds__(PLAN_THREADS, 1) plan_fused_kernel(PlanParams 
         __threadfence();
         mine = atomicAdd(a.hdr + WS_TICKET, 1) + 1;
     }
-    // while the other chunks arrive: where each expert's pairs start among
-    // this chunk's pairs sorted by expert
-    block_exscan(cho, E, red);
     if (tid == 0) {
         int w = 0, st = 0;  // w: 0 gave up, 1 every chunk in, 2 ticket past the chunk count
         if (mine == nchunk) w = 1;
@@ -1954,29 +1939,18 @@ __global__ void __launch_bounds__(PLAN_THREADS, 1) plan_fused_kernel(PlanParams 
     } else {
         plan_core(a, psm, seq, PlanSink{false, writer, hptr, hstart, hdst});
         __syncthreads();
-        // pass B's tables, from this CTA's own host tables: dw over the warp
-        // bases, pw in the planner's shared memory (its first ASSIGN_WARPS * E
-        // ints, clear of the misc words at its end), dlim over cho
-        int *dw = cnt, *pw = psm, *dlim = cho;
+        // pass B's tables from this CTA's own host tables: dw over the warp
+        // bases, and dlim
+        int *dw = cnt;
         for (int e = tid; e < E; e += nt) {
             const int h0 = hptr[e], d0 = hdst[h0];
-            const int po = cho[e] - cnt[e];  // cnt[e]: warp 0's base, the chunk's first rank of e
-            for (int w = 0; w < ASSIGN_WARPS; ++w) {
-                const int wb = cnt[w * E + e];
-                dw[w * E + e] = d0 + wb;
-                pw[w * E + e] = po + wb;
-            }
+#pragma unroll 4
+            for (int w = 0; w < ASSIGN_WARPS; ++w) dw[w * E + e] = d0 + cnt[w * E + e];
             dlim[e] = hptr[e + 1] - h0 > 1 ? d0 + hstart[h0 + 1] : INT_MAX;
         }
         __syncthreads();
-        // pass B, then row_src in (expert, rank) order
-        remote = assign_pass_b_fused(ids, dw + warp * E, pw + warp * E, dlim, hptr, hstart, hdst, wbeg, wend, n, p0,
-                                     E, R * C, C, a.fC, a.p.dst_pos, srow, spair, a.hdr + WS_FLAGS);
-        __syncthreads();
-        for (int x = tid; x < n; x += nt) {
-            const int r = srow[x];
-            if (r >= 0) a.p.row_src[r] = spair[x];
-        }
+        remote = assign_pass_b_fused(ids, dw + warp * E, dlim, hptr, hstart, hdst, wbeg, wend, p0, E, R * C, C, a.fC,
+                                     a.p.dst_pos, a.p.row_src, a.hdr + WS_FLAGS);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) remote += __shfl_xor_sync(FULL_MASK, remote, o);

@@ -236,7 +236,7 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
     if (sink.legacy && tid == 0) st_release(a.hdr + WS_SLOW, seq + 1);
     const bool wr = sink.writer;
     // the water-filling list in creation order
-    #pragma unroll 1
+#pragma unroll 1
     for (int q = tid; q < min(n_rep, lc); q += nt) {
         const int j = last_le(segb, nP, q);
         const int i = pilo[j] + (q - segb[j]);
@@ -245,7 +245,7 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
         lq[q] = min(PS[j + 1], QSr[i + 1] - qbase) - max(PS[j], QSr[i] - qbase);
         la[q] = 1;
     }
-    #pragma unroll 1
+#pragma unroll 1
     for (int r = tid; r < R; r += nt) closed[r] = 0;
     __syncthreads();
 
@@ -260,18 +260,18 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
         }
         int nl = min(n_rep, lc);
         int n_guard = 0, min_slack = 0;  // steps that reached the capacity guard, its least slack
-        #pragma unroll 1
+#pragma unroll 1
         for (int step = 0; step <= R; ++step) {
-            #pragma unroll 1
+#pragma unroll 1
             for (int r = lane; r < R; r += 32) cnt[r] = 0;
             __syncwarp();
-            #pragma unroll 1
+#pragma unroll 1
             for (int q = lane; q < nl; q += 32)
                 if (la[q]) atomicAdd(&cnt[lr[q]], 1);
             __syncwarp();
             // the open rank over B with the most replicas, lowest rank on ties
             int bc = -1, br = R;
-            #pragma unroll 1
+#pragma unroll 1
             for (int r = lane; r < R; r += 32) {
                 const int c = cnt[r];
                 if (!closed[r] && c > B && c > bc) {
@@ -291,12 +291,12 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
             const int rs = br;
             // its replicas: positions in list order (in mq), then ranked by
             // (quota desc, position asc) into ordx
-            #pragma unroll 1
+#pragma unroll 1
             for (int e = lane; e < E; e += 32) on_r[e] = 0;
-            #pragma unroll 1
+#pragma unroll 1
             for (int r = lane; r < R; r += 32) hused[r] = 0;
             int n = 0;
-            #pragma unroll 1
+#pragma unroll 1
             for (int q0 = 0; q0 < nl; q0 += 32) {
                 const int q = q0 + lane;
                 const bool mine = q < nl && la[q] && lr[q] == rs;
@@ -307,11 +307,11 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
             }
             n = min(n, lc);
             __syncwarp();
-            #pragma unroll 1
+#pragma unroll 1
             for (int k = lane; k < n; k += 32) {
                 const int qk = mq[k], vk = lq[qk];
                 int rk = 0;
-                #pragma unroll 1
+#pragma unroll 1
                 for (int j = 0; j < n; ++j) {
                     const int v = lq[mq[j]];
                     rk += (v > vk) || (v == vk && j < k);
@@ -322,11 +322,11 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
             __syncwarp();
             // the smallest m whose providers carry the moved quota
             int npick = 0, m_found = -1;
-            #pragma unroll 1
+#pragma unroll 1
             for (int m = 0; m <= B; ++m) {
                 while (npick < m) {  // next relay: largest home quota, lowest expert
                     int bk = 0, be = E;
-                    #pragma unroll 1
+#pragma unroll 1
                     for (int e = lane; e < E; e += 32) {
                         const int h = (int)fdiv((uint32_t)e, a.fL), kv = keep[e];
                         if (kv > bk && h != rs && !closed[h] && !on_r[e] && !hused[h]) {
@@ -352,14 +352,14 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
                 }
                 if (npick < m) break;  // fewer distinct relay homes than m
                 long long Q = 0, room = 0;
-                #pragma unroll 1
+#pragma unroll 1
                 for (int k = B - m + lane; k < n; k += 32) Q += lq[ordx[k]];
-                #pragma unroll 1
+#pragma unroll 1
                 for (int k = lane; k < B - m; k += 32) {
                     const int e = le[ordx[k]];
                     room += closed[fdiv((uint32_t)e, a.fL)] ? 0 : keep[e];
                 }
-                #pragma unroll 1
+#pragma unroll 1
                 for (int k = lane; k < m; k += 32) room += keep[rel[k]];
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) {
@@ -383,26 +383,26 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
             const int k0 = B - m_found;
             // the rank's replicas by step order: experts and quotas; a kept
             // replica's position once the moved ones are dropped
-            #pragma unroll 1
+#pragma unroll 1
             for (int k = lane; k < n; k += 32) {
                 const int q = ordx[k];
                 me[k] = le[q];
                 mq[k] = lq[q];
                 if (k < k0) {
                     int before = 0;
-                    #pragma unroll 1
+#pragma unroll 1
                     for (int j = k0; j < n; ++j) before += ordx[j] < q;
                     pvq[k] = q - before;
                 }
             }
             __syncwarp();
-            #pragma unroll 1
+#pragma unroll 1
             for (int k = k0 + lane; k < n; k += 32) la[ordx[k]] = 0;  // the moved replicas leave this rank
             __syncwarp();
             // drop them, keeping list order (a destination never lies past its
             // source, so a chunk only writes where its reads are done)
             int w = 0;
-            #pragma unroll 1
+#pragma unroll 1
             for (int q0 = 0; q0 < nl; q0 += 32) {
                 const int q = q0 + lane;
                 const bool alive = q < nl && la[q];
@@ -430,17 +430,17 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
             int np = 0;
             if (lane == 0) {
                 long long rem = 0;
-                #pragma unroll 1
+#pragma unroll 1
                 for (int k = k0; k < n; ++k) rem += mq[k];
-                #pragma unroll 1
+#pragma unroll 1
                 for (int k = 0; k < k0; ++k) pve[np++] = me[k];
-                #pragma unroll 1
+#pragma unroll 1
                 for (int k = 0; k < m_found; ++k) {
                     pve[np] = rel[k];
                     pvq[np] = -1;
                     ++np;
                 }
-                #pragma unroll 1
+#pragma unroll 1
                 for (int k = 0; k < np; ++k) {
                     const int e = pve[k];
                     const long long capk = (pvq[k] >= 0 && closed[fdiv((uint32_t)e, a.fL)]) ? 0 : keep[e];
@@ -473,7 +473,7 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
             int *MS = ordx, *PV = pvq, *tag = on_r;  // free by now: order, kept positions, relay marks
             {
                 int run = 0;
-                #pragma unroll 1
+#pragma unroll 1
                 for (int b0 = 0; b0 < nm; b0 += 32) {
                     const int i = b0 + lane, v = i < nm ? mq[k0 + i] : 0;
                     int x = v;
@@ -487,7 +487,7 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
                 }
                 if (lane == 0) MS[nm] = run;
                 run = 0;
-                #pragma unroll 1
+#pragma unroll 1
                 for (int b0 = 0; b0 < np; b0 += 32) {
                     const int i = b0 + lane, v = i < np ? pva[i] : 0;
                     int x = v;
@@ -501,21 +501,21 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
                 }
                 if (lane == 0) PV[np] = run;
             }
-            #pragma unroll 1
+#pragma unroll 1
             for (int e = lane; e < E; e += 32) tag[e] = -1;
             __syncwarp();
-            #pragma unroll 1
+#pragma unroll 1
             for (int pi = 0; pi < np; ++pi) {
                 const int lo = PV[pi], hi = PV[pi + 1];
                 if (hi <= lo || nm <= 0) continue;
                 const int h = (int)fdiv((uint32_t)pve[pi], a.fL);
                 const int i_lo = warp_last_le(MS, nm, lo), i_hi = warp_last_le(MS, nm, hi - 1);
                 const int nl0 = nl;
-                #pragma unroll 1
+#pragma unroll 1
                 for (int q = lane; q < nl0; q += 32)
                     if (lr[q] == h) tag[le[q]] = q;
                 __syncwarp();
-                #pragma unroll 1
+#pragma unroll 1
                 for (int i0 = i_lo; i0 <= i_hi; i0 += 32) {
                     const int i = i0 + lane;
                     bool fresh = false;
@@ -542,7 +542,7 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
                     nl = min(nl + __popc(b), lc);
                 }
                 __syncwarp();
-                #pragma unroll 1
+#pragma unroll 1
                 for (int q = lane; q < nl0; q += 32)
                     if (lr[q] == h) tag[le[q]] = -1;
                 __syncwarp();
@@ -560,11 +560,11 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
     // ordinals in list order, slot offsets and the used slots of every rank
     // (in the one-kernel path each rank's row is written by the CTA that owns
     // the rank, r mod gridDim.x, empty slots included)
-    #pragma unroll 1
+#pragma unroll 1
     for (int r = tid; r < R; r += nt) {
         const bool own = sink.legacy ? wr : (int)(r % gridDim.x) == (int)blockIdx.x;
         int off = 0;
-        #pragma unroll 1
+#pragma unroll 1
         for (int sl = 0; sl < L; ++sl) {
             const int e = r * L + sl;
             hoff[e] = off;
@@ -576,7 +576,7 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
             off += keep[e];
         }
         int ord = 0;
-        #pragma unroll 1
+#pragma unroll 1
         for (int q = 0; q < nl; ++q) {
             if (lr[q] != r) continue;
             lo[q] = ord;
@@ -595,9 +595,9 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
     }
     __syncthreads();
     if (!sink.legacy)
-        #pragma unroll 1
+#pragma unroll 1
         for (int r = blockIdx.x; r < R; r += gridDim.x)
-            #pragma unroll 1
+#pragma unroll 1
             for (int sl = cnt[r] + tid; sl <= E; sl += nt) {
                 if (sl < E) {
                     a.p.slot_expert[(size_t)r * E + sl] = -1;
@@ -605,7 +605,7 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
                 }
                 a.p.slot_offset[(size_t)r * (E + 1) + sl] = C;
             }
-    #pragma unroll 1
+#pragma unroll 1
     for (int q = tid; q < nl; q += nt) {
         if (wr) {
             a.p.rep_expert[q] = le[q];
@@ -616,7 +616,7 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
         if (lo[q] >= B) atomicAdd(&misc[2], 1);
     }
     if (wr && !sink.legacy)  // the one-kernel path writes no defaults beforehand
-        #pragma unroll 1
+#pragma unroll 1
         for (int q = nl + tid; q < E + R; q += nt) {
             a.p.rep_expert[q] = -1;
             a.p.rep_rank[q] = -1;
@@ -624,10 +624,10 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
             a.p.rep_quota[q] = 0;
         }
     // hosts per expert (home + its replicas) and the work-list flags
-    #pragma unroll 1
+#pragma unroll 1
     for (int e = tid; e < E; e += nt) {
         int c = 1, f = 0;
-        #pragma unroll 1
+#pragma unroll 1
         for (int q = 0; q < nl; ++q)
             if (le[q] == e) {
                 ++c;
@@ -644,13 +644,13 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
     __syncthreads();
     block_exscan(hc, E + 1, wsum);
     const int n_rep_experts = block_exscan(fpre, E + 1, wsum);
-    #pragma unroll 1
+#pragma unroll 1
     for (int e = tid; e <= E; e += nt) {
         if (wr) a.p.host_ptr[e] = hc[e];
         if (!sink.legacy) sink.hptr[e] = hc[e];
     }
     if (wr && !sink.legacy)
-        #pragma unroll 1
+#pragma unroll 1
         for (int h = hc[E] + tid; h < nh; h += nt) {
             a.p.host_rank[h] = -1;
             a.p.host_slot[h] = -1;
@@ -659,13 +659,13 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
             a.p.host_local[h] = 0;
         }
     if (wr)
-        #pragma unroll 1
+#pragma unroll 1
         for (int e = tid; e < E; e += nt) {
             if (fl[e]) a.p.rep_home_list[fpre[e]] = e;
             if (e >= n_rep_experts) a.p.rep_home_list[e] = -1;
         }
     // host intervals: the hosts of e in ascending rank, starts in that order
-    #pragma unroll 1
+#pragma unroll 1
     for (int e = tid; e < E; e += nt) {
         const int b0 = hc[e], b1 = min(hc[e + 1], nh);
         int k = b0;
@@ -676,7 +676,7 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
             xo[k] = hoff[e];
             ++k;
         }
-        #pragma unroll 1
+#pragma unroll 1
         for (int q = 0; q < nl && k < b1; ++q)
             if (le[q] == e) {
                 xr[k] = lr[q];
@@ -685,7 +685,7 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
                 xo[k] = loff[q];
                 ++k;
             }
-        #pragma unroll 1
+#pragma unroll 1
         for (int x = b0 + 1; x < k; ++x) {  // insertion sort by rank (ranks are distinct)
             const int vr = xr[x], vs = xs[x], vq = xq[x], vo = xo[x];
             int y = x;
@@ -702,7 +702,7 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
             xo[y] = vo;
         }
         int st = 0;
-        #pragma unroll 1
+#pragma unroll 1
         for (int h = b0; h < k; ++h) {
             // the locality flag as in the water-filling tail
             const int loc = (d.flags & MOONEP_FLAG_LOCALITY)
@@ -746,7 +746,7 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
             a.p.info[MOONEP_INFO_N_RECEIVERS] = nN;
             a.p.info[MOONEP_INFO_MAX_REP_PER_RANK] = misc[3];
             a.p.info[MOONEP_INFO_N_REP_EXPERTS] = n_rep_experts;
-            #pragma unroll 1
+#pragma unroll 1
             for (int i = MOONEP_INFO_N_REMOTE_PAIRS; i < MOONEP_INFO_LEN; ++i) a.p.info[i] = 0;
             a.p.info[MOONEP_INFO_CASCADE_GUARD_STEPS] = misc[4];
             a.p.info[MOONEP_INFO_CASCADE_GUARD_SLACK] = misc[5];
@@ -884,11 +884,11 @@ __device__ void plan_core(const PlanParams &a, int *sm, int seq, const PlanSink 
     int *flag = hq + nh;           // E
     int *wsum = flag + E;          // 32
     int *misc = wsum + 32;         // 16 (MISC_*)
-    #pragma unroll 1
+#pragma unroll 1
     for (int i = tid; i < 16; i += nt) misc[i] = 0;
 
     // ---- home loads, excess X and deficit D per rank
-    #pragma unroll 1
+#pragma unroll 1
     for (int r = tid; r < R; r += nt) {
         int h = 0;
 #pragma unroll 4
@@ -900,7 +900,7 @@ __device__ void plan_core(const PlanParams &a, int *sm, int seq, const PlanSink 
 
     // ---- largest-first shedding: expert e sheds what remains of its rank's
     // excess after all larger (T desc, e asc) experts of the rank
-    #pragma unroll 1
+#pragma unroll 1
     for (int e = tid; e < E; e += nt) {
         const int r = (int)fdiv((uint32_t)e, a.fL), v = T[e];
         int s = 0;
@@ -919,7 +919,7 @@ __device__ void plan_core(const PlanParams &a, int *sm, int seq, const PlanSink 
         scr[e] = s > 0;
         pof[e] = -1;
     }
-    #pragma unroll 1
+#pragma unroll 1
     for (int r = tid; r < R; r += nt) scr[E + r] = D[r] > 0;
     __syncthreads();
 
@@ -927,13 +927,13 @@ __device__ void plan_core(const PlanParams &a, int *sm, int seq, const PlanSink 
     const int nPN = block_exscan(scr, E + R, wsum);
     const int nP = scr[E];
     const int nN = nPN - nP;
-    #pragma unroll 1
+#pragma unroll 1
     for (int e = tid; e < E; e += nt)
         if (shed[e] > 0) {
             hr[scr[e]] = shed[e];
             hs[scr[e]] = e;
         }
-    #pragma unroll 1
+#pragma unroll 1
     for (int r = tid; r < R; r += nt)
         if (D[r] > 0) {
             hq[scr[E + r] - nP] = D[r];
@@ -943,14 +943,14 @@ __device__ void plan_core(const PlanParams &a, int *sm, int seq, const PlanSink 
     // counting-rank sorts, one warp per element: pieces by (shed desc,
     // e asc), receivers by (D desc, r asc); an element's position is the
     // number of entries ordered before it, counted 32 at a time by ballot
-    #pragma unroll 1
+#pragma unroll 1
     for (int x = warp; x < nP + nN; x += nwarp) {
         const bool piece = x < nP;
         const int m = piece ? nP : nN, xi = piece ? x : x - nP;
         const int *val = piece ? hr : hq, *key = piece ? hs : cspare;
         const int v = val[xi], id = key[xi];
         int pos = 0;
-        #pragma unroll 1
+#pragma unroll 4
         for (int j0 = 0; j0 < m; j0 += 32) {
             const int j = j0 + lane;
             bool before = false;
@@ -976,7 +976,7 @@ __device__ void plan_core(const PlanParams &a, int *sm, int seq, const PlanSink 
     }
     int *segb = Bs;          // nP + 1: replicas per piece, then their prefix
     int *rpr = Bs + nP + 1;  // R + 1: replicas per rank, then prefix + n_rep
-    #pragma unroll 1
+#pragma unroll 1
     for (int r = tid; r <= R; r += nt) rpr[r] = 0;
     __syncthreads();
 
@@ -993,7 +993,7 @@ __device__ void plan_core(const PlanParams &a, int *sm, int seq, const PlanSink 
     // ---- water-filling: piece j meets receivers pilo[j].. ; receiver i meets
     // pieces jlo[i].. ; replicas are numbered in (j, i) order
     // (one warp per piece or receiver, searching by ballot)
-    #pragma unroll 1
+#pragma unroll 1
     for (int x = warp; x < nP + nN; x += nwarp) {
         if (x < nP) {
             const int j = x;
@@ -1037,7 +1037,7 @@ __device__ void plan_core(const PlanParams &a, int *sm, int seq, const PlanSink 
     int *Z = hr;     // 4E + R + 2 <= 3 nh ints, free after the sort
     int *rq_j = scr;  // n_rep <= E + R - 1: piece of each replica (scr is free)
     const int zh = E + n_rep, zf = zh + E + 1, nz = zf + E + 1;
-    #pragma unroll 1
+#pragma unroll 1
     for (int q = tid; q < n_rep; q += nt) {
         const int j = last_le(segb, nP, q);
         rq_j[q] = j;
@@ -1058,7 +1058,7 @@ __device__ void plan_core(const PlanParams &a, int *sm, int seq, const PlanSink 
         cspare[cs] = r;
         if (ord >= B) atomicAdd(&misc[2], 1);
     }
-    #pragma unroll 1
+#pragma unroll 1
     for (int e = tid; e < E; e += nt) {
         const int r = (int)fdiv((uint32_t)e, a.fL);
         const int cs = rank_base(r) + (e - r * L);
@@ -1070,11 +1070,14 @@ __device__ void plan_core(const PlanParams &a, int *sm, int seq, const PlanSink 
         int c = 1, f = 0;
         const int j = pof[e];
         if (j >= 0) {
-            const int ns = segb[j + 1] - segb[j];
+            const int ns = segb[j + 1] - segb[j], i0 = pilo[j];
             c += ns;
-            #pragma unroll 1
+#pragma unroll 1
             for (int s = 0; s < ns; ++s)
-                if (j - jlo[pilo[j] + s] < B) f = 1;
+                if (j - jlo[i0 + s] < B) {
+                    f = 1;
+                    break;
+                }
         }
         Z[zh + e] = c;
         Z[zf + e] = f;
@@ -1100,7 +1103,7 @@ __device__ void plan_core(const PlanParams &a, int *sm, int seq, const PlanSink 
     // of e), and its start is in the order of the pairs left over.
     const bool locality = (d.flags & MOONEP_FLAG_LOCALITY) != 0;
     auto own_pairs = [&](int r, int e) { return ld_cg(a.gs + (size_t)r * a.gs_stride + e); };
-    #pragma unroll 1
+#pragma unroll 1
     for (int x = tid; x < n_hosts; x += nt) {
         int e, r0, slot, quota, j, pos = 0, st = 0, locsum = 0;
         if (x < E) {
@@ -1125,15 +1128,18 @@ __device__ void plan_core(const PlanParams &a, int *sm, int seq, const PlanSink 
             }
         }
         if (j >= 0) {
-            const int ns = segb[j + 1] - segb[j];
-            #pragma unroll 1
+            // the other hosts of e on lower ranks (a hot expert has tens of
+            // them, and every host walks them all: the loads of four steps
+            // are in flight together)
+            const int ns = segb[j + 1] - segb[j], i0 = pilo[j], ps0 = PS[j], ps1 = PS[j + 1];
+#pragma unroll 4
             for (int s = 0; s < ns; ++s) {
-                const int i = pilo[j] + s;
-                if (qr[i] < r0) {
+                const int i = i0 + s, ri = qr[i];
+                if (ri < r0) {
                     ++pos;
-                    const int qi = seg_q(j, i);
+                    const int qi = min(ps1, QSr[i + 1] - qbase) - max(ps0, QSr[i] - qbase);
                     st += qi;
-                    if (locality) locsum += min(qi, own_pairs(qr[i], e));
+                    if (locality) locsum += min(qi, own_pairs(ri, e));
                 }
             }
         }
@@ -1156,7 +1162,7 @@ __device__ void plan_core(const PlanParams &a, int *sm, int seq, const PlanSink 
             sink.hdst[h] = dst0;
         }
     }
-    #pragma unroll 1
+#pragma unroll 1
     for (int x = tid; x <= E; x += nt) {
         if (wr) a.p.host_ptr[x] = hptr(x);
         if (!sink.legacy) sink.hptr[x] = hptr(x);
@@ -1182,7 +1188,7 @@ __device__ void plan_core(const PlanParams &a, int *sm, int seq, const PlanSink 
             a.p.info[MOONEP_INFO_N_RECEIVERS] = nN;
             a.p.info[MOONEP_INFO_MAX_REP_PER_RANK] = misc[3];
             a.p.info[MOONEP_INFO_N_REP_EXPERTS] = n_rep_experts;
-            #pragma unroll 1
+#pragma unroll 1
             for (int i = MOONEP_INFO_N_REMOTE_PAIRS; i < MOONEP_INFO_LEN; ++i) a.p.info[i] = 0;
         }
     }
@@ -1196,10 +1202,10 @@ __device__ void plan_core(const PlanParams &a, int *sm, int seq, const PlanSink 
         // the one-kernel path: the rows of the padded slot tables of this
         // CTA's ranks (r mod gridDim.x), used and empty slots alike, so every
         // entry is written once and no defaults precede them
-        #pragma unroll 1
+#pragma unroll 1
         for (int r = blockIdx.x; r < R; r += gridDim.x) {
             const int b0 = rank_base(r), ns = rank_base(r + 1) - b0;
-            #pragma unroll 1
+#pragma unroll 1
             for (int sl = tid; sl <= E; sl += nt) {
                 const bool used = sl < ns;
                 if (sl < E) {
@@ -1214,7 +1220,7 @@ __device__ void plan_core(const PlanParams &a, int *sm, int seq, const PlanSink 
         // ---- then, while the assignment CTAs place the pairs, the used
         // slots of the padded [R][E] tables (read only by later kernels,
         // which start after this grid has finished)
-        #pragma unroll 1
+#pragma unroll 1
         for (int x = tid; x < E + n_rep; x += nt) {
             const int r = cspare[x], b0 = rank_base(r), sl = x - b0;
             a.p.slot_expert[(size_t)r * E + sl] = cexp[x];
@@ -1223,14 +1229,14 @@ __device__ void plan_core(const PlanParams &a, int *sm, int seq, const PlanSink 
         }
     } else {
         // the writer: the empty rest of the replica and host tables
-        #pragma unroll 1
+#pragma unroll 1
         for (int q = n_rep + tid; q < E + R; q += nt) {
             a.p.rep_expert[q] = -1;
             a.p.rep_rank[q] = -1;
             a.p.rep_slot[q] = -1;
             a.p.rep_quota[q] = 0;
         }
-        #pragma unroll 1
+#pragma unroll 1
         for (int h = n_hosts + tid; h < nh; h += nt) {
             a.p.host_rank[h] = -1;
             a.p.host_slot[h] = -1;
@@ -1240,7 +1246,7 @@ __device__ void plan_core(const PlanParams &a, int *sm, int seq, const PlanSink 
         }
     }
     // the reduce work list
-    #pragma unroll 1
+#pragma unroll 1
     for (int x = tid; x < E; x += nt) {
         if (flag[x]) a.p.rep_home_list[Z[zf + x] - zf0] = x;
         if (x >= n_rep_experts) a.p.rep_home_list[x] = -1;
@@ -1375,6 +1381,21 @@ __global__ void __launch_bounds__(PLAN_THREADS) hist_plan_kernel(PlanParams a)
 
 // ---------------------------------------------------------- assignment
 
+// The host of rank g among an expert's hosts [h0, hend) (hend > h0): the last
+// h with hstart[h] <= g (hstart[h0] = 0 <= g; starts are non-decreasing in
+// rank order, equal where a host takes no rows), by bisection -- a hot expert
+// has tens of hosts, and a linear walk over them held back its warp.
+__device__ __forceinline__ int host_of(const int *hstart, int h0, int hend, int g)
+{
+    int lo = h0, hi = hend;  // the answer is in [lo, hi)
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (hstart[mid] <= g) lo = mid;
+        else hi = mid;
+    }
+    return lo;
+}
+
 // Pass A, on the ids alone: the calling warp walks its contiguous sub-range
 // [wbeg, wend) of the staged ids in (t, k) order, ranking equal experts with
 // ballots, so loc is the pair's rank among the sub-range's earlier pairs of
@@ -1451,9 +1472,7 @@ __device__ __forceinline__ int assign_pass_b(const int *ids, const int *wb, cons
         const int e = v & PACK_MASK, loc = v >> PACK_BITS;
         if (v < 0 || e >= E) continue;  // cannot happen in a non-empty plan
         const int g = wb[e] + loc;
-        int h = hptr[e];
-        const int hend = hptr[e + 1];
-        while (h + 1 < hend && hstart[h + 1] <= g) ++h;
+        const int h = host_of(hstart, hptr[e], hptr[e + 1], g);
         const int dst = hdst[h] + g;
         const int p = p0 + i;
         if (dst < 0 || dst >= rows) {  // cannot happen for a consistent plan
@@ -1493,11 +1512,9 @@ __device__ __forceinline__ int assign_pass_b_fused(const int *ids, const int *dw
         if (v < 0 || e >= E) continue;  // cannot happen in a non-empty plan
         int dst = dw[e] + loc;
         if (dst >= dlim[e]) {  // past the expert's first host
-            int h = hptr[e];
-            const int hend = hptr[e + 1];
-            const int g = dst - hdst[h];
-            while (h + 1 < hend && hstart[h + 1] <= g) ++h;
-            dst = hdst[h] + g;
+            const int h0 = hptr[e];
+            const int g = dst - hdst[h0];
+            dst = hdst[host_of(hstart, h0, hptr[e + 1], g)] + g;
         }
         const int p = p0 + i;
         if (dst < 0 || dst >= rows) {  // cannot happen for a consistent plan

@@ -158,6 +158,13 @@ class ClockSampler:
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
+    def wait_first(self, timeout: float = 3.0):
+        """Until nvidia-smi has printed a sample: its start-up (driver and
+        NVML initialisation) then lies outside the timed region."""
+        t0 = time.time()
+        while self.proc is not None and not self.lines and time.time() - t0 < timeout:
+            time.sleep(0.01)
+
     def stop(self) -> dict:
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
@@ -367,6 +374,9 @@ class Timer:
     def total_ms(self, name):
         return sum(s.elapsed_time(e) for s, e in self.pairs.get(name, []))
 
+    def times_ms(self, name):
+        return [s.elapsed_time(e) for s, e in self.pairs.get(name, [])]
+
     def count(self, name):
         return len(self.pairs.get(name, []))
 
@@ -496,14 +506,17 @@ def run_ours(args, world, rank, local):
             if tm:
                 ev.record()
 
+    # the clock sampler starts before the warm-up: its start-up once delayed
+    # the first timed plan call by about 45 us
+    sampler = ClockSampler(smi_index(local))
+    sampler.start()
+    sampler.wait_first()
     for _ in range(args.warmup):
         step(None)
     torch.cuda.synchronize()
     info = plan.info()
-    sampler = ClockSampler(smi_index(local))
     barrier(world)
     torch.cuda.synchronize()
-    sampler.start()
     tm = Timer()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
@@ -516,6 +529,20 @@ def run_ours(args, world, rank, local):
     barrier(world)
     step_ms_local = t_start.elapsed_time(t_end) / args.steps
     ms_per_step = max_over_ranks(world, step_ms_local)
+
+    # the same step with the other planner, for comparison (its plan time
+    # only; the data kernels do not depend on which planner made the plan)
+    other = 1 - mp.set_plan_path(1 - args.plan_path)
+    for _ in range(args.warmup):
+        step(None)
+    tm2 = Timer()
+    for _ in range(args.steps):
+        step(tm2)
+    torch.cuda.synchronize()
+    mp.set_plan_path(args.plan_path)
+    other_plan_us = max_over_ranks(world, statistics.median(tm2.times_ms("plan"))) * 1e3
+    plan_steps_us = [round(x * 1e3, 2) for x in tm.times_ms("plan")]
+    plan_median_us = max_over_ranks(world, statistics.median(tm.times_ms("plan"))) * 1e3
 
     k = args.steps
     t = {n: tm.total_ms(n) / k for n in ("plan", "dispatch", "combine", "combine_bwd", "reduce")
@@ -865,7 +892,12 @@ def run_ours(args, world, rank, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic", "config": cfgd,
         "frac_of_peak": round(value / world / peak, 4),
-        "planner_us": kernels["plan"]["us"],
+        # the median over the timed steps (kernels.plan is their mean): a
+        # single slow call, e.g. as the clock sampler starts, moves the mean
+        "planner_us": round(plan_median_us, 2),
+        "planner_us_steps": plan_steps_us,
+        "planner_us_other_path": {"path": "two-kernel" if other == 1 else "one-kernel",
+                                  "us": round(other_plan_us, 2)},
         "roofline": roofline, "kernels": kernels, "sweep": sweep,
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
         "decode": decode, "workloads": workloads, "ep_one_gpu": ep,
@@ -977,7 +1009,13 @@ def main():
     ap.add_argument("--profile-S", type=int, default=0, help="tokens per rank (0: the kernel's case)")
     ap.add_argument("--profile-P", type=int, default=0,
                     help="elements per expert row for reduce / prefetch (0: the kernel's case)")
+    ap.add_argument("--plan-path", type=int, default=0, choices=(0, 1),
+                    help="0: the one-kernel planner where it fits (the library's default); "
+                         "1: the two-kernel planner (moonep_set_plan_path)")
     args = ap.parse_args()
+    if args.impl != "reference" or args.profile:
+        from load_balancing_moonep_b200 import moonep as mp
+        mp.set_plan_path(args.plan_path)
     if args.profile:
         run_profile_case(args)
         return

@@ -232,6 +232,11 @@ def barrier(world):
             dist.barrier()
 
 
+# A device-side sleep of about 50 us before a plan timed alone: the host
+# enqueues the plan meanwhile, so its CUDA events time the device.
+SPACER_CYCLES = 100_000
+
+
 def max_over_ranks(world, x: float) -> float:
     if world <= 1:
         return x
@@ -774,6 +779,10 @@ def run_ours(args, world, rank, local):
                 if e:
                     e.record()
             for k in range(wl.R):
+                if tm and k == 0:
+                    # keep the GPU busy while the host enqueues the plan, so
+                    # the events time the device, not the host's launch path
+                    torch.cuda._sleep(SPACER_CYCLES)
                 e = tm.mark("plan") if tm and k == 0 else None
                 mp.ep_plan(cfg, k, tl[k], counts_all, eplans[k])
                 if e:
@@ -797,6 +806,13 @@ def run_ours(args, world, rank, local):
             ep_layer(et)
         torch.cuda.synchronize()
         it = args.sweep_iters
+        # rank 0's plan with the other expert-parallel planner, timed the same way
+        other_ep = 1 - mp.set_plan_path(1 - args.plan_path)
+        ot = Timer()
+        for _ in range(args.sweep_iters):
+            ep_layer(ot)
+        torch.cuda.synchronize()
+        mp.set_plan_path(args.plan_path)
         pd, pc = et.total_ms("dispatch") / it, et.total_ms("combine") / it
         einf = eplans[0].info()
         gd = bytes_dispatch(wl) / (pd * 1e-3) / 1e9
@@ -818,20 +834,27 @@ def run_ours(args, world, rank, local):
                 for k in range(lwl.R):
                     mp.ep_count(lcfg, ltl[k], lps[k], counts_row=lca[k])
                 lt = Timer()
-                for k in range(lwl.R):
-                    e = lt.mark("plan") if k == 0 else None
-                    mp.ep_plan(lcfg, k, ltl[k], lca, lps[k])
-                    if e:
-                        e.record()
+                for rep_ in range(4):  # the first call warms up; the median of the other three
+                    for k in range(lwl.R):
+                        if k == 0:
+                            torch.cuda._sleep(SPACER_CYCLES)
+                        e = lt.mark("plan") if k == 0 else None
+                        mp.ep_plan(lcfg, k, ltl[k], lca, lps[k])
+                        if e:
+                            e.record()
                 torch.cuda.synchronize()
                 row[key] = round(sum(q.info()["n_remote_pairs"] for q in lps) / lwl.pairs, 4)
-                row["plan_us" + ("_locality" if lflags else "")] = round(lt.total_ms("plan") * 1e3, 2)
+                row["plan_us" + ("_locality" if lflags else "")] = round(
+                    statistics.median(lt.times_ms("plan")[1:]) * 1e3, 2)
                 del lps
             locality.append(row)
         ep = {"what": (f"{wl.R} ranks on one GPU: each rank's ep_count and ep_plan (rank 0 timed), then "
                        f"{wl.R} ep_dispatch and {wl.R} ep_combine launches through per-rank row pointers"),
               "count_us": round(et.total_ms("count") / it * 1e3, 2),
-              "plan_us": round(et.total_ms("plan") / it * 1e3, 2),
+              "plan_us": round(statistics.median(et.times_ms("plan")) * 1e3, 2),
+              "plan_us_other_path": {"path": "two-kernel" if other_ep == 1 else "one-kernel",
+                                     "us": round(statistics.median(ot.times_ms("plan")) * 1e3, 2)},
+              "plan_timing": "rank 0's plan after a device-side sleep that covers the host's launch path",
               "dispatch_GB/s": round(gd, 1), "combine_GB/s": round(gc, 1),
               "dispatch_frac": round(gd / peak, 4), "combine_frac": round(gc / peak, 4),
               "rank0_remote_pair_frac": round(einf["n_remote_pairs"] / (wl.S * wl.K), 4),

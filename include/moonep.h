@@ -330,8 +330,11 @@ MOONEP_API int moonep_ep_count(const moonep_config *cfg, const int32_t *topk_loc
  * a pair's rank within its expert is the lower ranks' counts of that expert
  * plus its rank among this rank's own pairs in (t, k) order, the global
  * order of moonep_plan.  Uses the per-chunk counts moonep_ep_count left in
- * `workspace`: call it with the same workspace and topk_local.  Two
- * launches. */
+ * `workspace`: call it with the same workspace and topk_local.  One launch
+ * in which every CTA plans from the gathered counts and places its own
+ * chunk's pairs (two launches, a planner CTA then the assignment grid, where
+ * that does not fit one CTA's shared memory, or after
+ * moonep_set_plan_path(1)). */
 MOONEP_API int moonep_ep_plan(const moonep_config *cfg, int32_t rank, const int32_t *topk_local,
                               const int32_t *counts_all, const moonep_plan_t *plan, void *workspace,
                               void *stream);
@@ -426,12 +429,13 @@ MOONEP_API const char *moonep_status_string(int status, char *buf, size_t len);
  * already enqueued keep the bound they were launched with. */
 MOONEP_API int moonep_set_wait_limit(int iterations);
 
-/* Which planner moonep_plan / moonep_plan_noalloc launch afterwards in this
- * process: 1 the two-kernel planner always; any other value (0, the
- * default) the one-kernel planner wherever all of its CTAs fit on the device
- * at once, else the two-kernel one.  Both give the same plan; tests use 1 to
- * compare them.  A workspace may pass between the two.  Host-only; returns
- * the previous setting (0 or 1). */
+/* Which planner moonep_plan / moonep_plan_noalloc / moonep_ep_plan launch
+ * afterwards in this process: 1 the two-kernel planner always; any other
+ * value (0, the default) the one-kernel planner wherever it fits (for
+ * moonep_plan: all of its CTAs on the device at once), else the two-kernel
+ * one.  Both give the same plan; tests use 1 to compare them.  A workspace
+ * may pass between the two.  Host-only; returns the previous setting (0 or
+ * 1). */
 MOONEP_API int moonep_set_plan_path(int mode);
 
 /* The replica capacity the relay cascade's guard (MOONEP_FLAG_CASCADE)

@@ -84,6 +84,7 @@ struct PlanSink {
     bool legacy;
     bool writer;
     int *hptr, *hstart, *hdst;  // one-kernel path: [E+1], [2E+R], [2E+R] in shared memory
+    int *hloc = nullptr, *hq = nullptr, *hr = nullptr;  // and, if set, each host's local pairs, quota and rank
 };
 
 // The planner's misc words (16 ints of shared memory): 0 status in, 2
@@ -721,6 +722,11 @@ __device__ void cascade_tail(const PlanParams &a, int *cz, int *dead, int *keep,
             } else {
                 sink.hstart[h] = st;
                 sink.hdst[h] = dst0;
+                if (sink.hloc) {
+                    sink.hloc[h] = loc;
+                    sink.hq[h] = xq[h];
+                    sink.hr[h] = xr[h];
+                }
             }
             st += xq[h] - loc;
         }
@@ -1160,6 +1166,11 @@ __device__ void plan_core(const PlanParams &a, int *sm, int seq, const PlanSink 
         } else {
             sink.hstart[h] = st;
             sink.hdst[h] = dst0;
+            if (sink.hloc) {
+                sink.hloc[h] = loc;
+                sink.hq[h] = quota;
+                sink.hr[h] = r0;
+            }
         }
     }
 #pragma unroll 1
@@ -1281,10 +1292,10 @@ __device__ __forceinline__ void write_table_defaults(const PlanParams &a, int x0
     }
 }
 
-// An empty plan: every table empty, spread over the grid, and dst_pos and
-// row_src -1 for this CTA's pairs [p0, p0 + n) (the rows are as many as the
-// pairs, so the CTAs cover row_src too).
-__device__ __forceinline__ void write_empty_plan(const PlanParams &a, int p0, int n)
+// An empty plan: every table empty, spread over the grid, and dst_pos (and,
+// with rows, row_src) -1 for this CTA's pairs [p0, p0 + n) (the rows are as
+// many as the pairs, so the CTAs cover row_src too).
+__device__ __forceinline__ void write_empty_plan(const PlanParams &a, int p0, int n, bool rows = true)
 {
     const Dims &d = a.d;
     const int E = d.E, R = d.R, nh = 2 * E + R;
@@ -1311,7 +1322,7 @@ __device__ __forceinline__ void write_empty_plan(const PlanParams &a, int p0, in
     for (int x = x0; x < E; x += g) a.p.rep_home_list[x] = -1;
     for (int i = threadIdx.x; i < n; i += blockDim.x) {
         a.p.dst_pos[p0 + i] = -1;
-        a.p.row_src[p0 + i] = -1;
+        if (rows) a.p.row_src[p0 + i] = -1;
     }
 }
 
@@ -1499,10 +1510,12 @@ __device__ __forceinline__ int assign_pass_b(const int *ids, const int *wb, cons
 // and they bound this pass.  (Staging row_src in shared memory in (expert,
 // rank) order, so that its stores coalesce, measured 1.9 µs slower at the
 // large shape than these scattered stores.)
+// src_rank >= 0: the source rank of every pair (one rank's pairs, whose
+// row_src is null); -1 derives it as p / C.
 __device__ __forceinline__ int assign_pass_b_fused(const int *ids, const int *dw, const int *dlim, const int *hptr,
                                                    const int *hstart, const int *hdst, int wbeg, int wend, int p0,
-                                                   int E, int rows, int C, const FastDiv &fC, int *dst_pos,
-                                                   int *row_src, int *status)
+                                                   int E, int rows, int C, const FastDiv &fC, int src_rank,
+                                                   int *dst_pos, int *row_src, int *status)
 {
     const int lane = threadIdx.x & 31;
     int remote = 0;
@@ -1523,8 +1536,9 @@ __device__ __forceinline__ int assign_pass_b_fused(const int *ids, const int *dw
             continue;
         }
         dst_pos[p] = dst;
-        row_src[dst] = p;
-        remote += (uint32_t)dst - fdiv((uint32_t)p, fC) * (uint32_t)C >= (uint32_t)C;
+        if (row_src) row_src[dst] = p;
+        const uint32_t src0 = (src_rank >= 0 ? (uint32_t)src_rank : fdiv((uint32_t)p, fC)) * (uint32_t)C;
+        remote += (uint32_t)dst - src0 >= (uint32_t)C;
     }
     return remote;
 }
@@ -1711,6 +1725,47 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) assign_kernel(PlanParams a)
     pdl_wait();
 }
 
+// The chunk's ids [p0, p0 + n) of topk into shared memory, by the calling
+// CTA: 16-byte loads, all of a thread's in flight together (from pair p0 & ~3
+// on, into ids_raw, so the loads are aligned; the few before p0 belong to the
+// previous chunk and are not used), then the last < 4 one by one; every pair
+// one by one when topk is not 16-byte aligned.  ids = ids_raw + (p0 & 3).
+// Returns whether this thread saw an id outside [0, E).
+__device__ __forceinline__ int stage_ids(const int32_t *topk, int p0, int n, int E, int *ids_raw, int *ids)
+{
+    const int tid = threadIdx.x, nt = blockDim.x;
+    int bad = 0;
+    const int q0 = p0 >> 2, q1 = (p0 + n) >> 2;  // 16-byte words wholly or partly before p0 + n
+    const bool vec = (reinterpret_cast<uintptr_t>(topk) & 15) == 0;
+    const int nv = vec ? q1 - q0 : 0;
+    const int4 *src = reinterpret_cast<const int4 *>(topk) + q0;
+    constexpr int VB = 4;
+    for (int k0 = tid; k0 < nv; k0 += VB * nt) {
+        int4 v[VB];
+#pragma unroll
+        for (int j = 0; j < VB; ++j)
+            if (k0 + j * nt < nv) v[j] = __ldg(src + k0 + j * nt);
+#pragma unroll
+        for (int j = 0; j < VB; ++j) {
+            const int k = k0 + j * nt;
+            if (k < nv) {
+                reinterpret_cast<int4 *>(ids_raw)[k] = v[j];
+                const int q = 4 * (q0 + k);  // pair of v[j].x
+                const int x[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    if (q + c >= p0) bad |= x[c] < 0 || x[c] >= E;
+            }
+        }
+    }
+    for (int i = (vec ? max(4 * q1 - p0, 0) : 0) + tid; i < n; i += nt) {
+        const int e = __ldg(topk + p0 + i);
+        ids[i] = e;
+        bad |= e < 0 || e >= E;
+    }
+    return bad;
+}
+
 // ------------------------------------------------------- one-kernel planner
 //
 // When one CTA per SM can hold a chunk of about tokens / SMs tokens beside
@@ -1776,42 +1831,9 @@ __global__ void __launch_bounds__(PLAN_THREADS, 1) plan_fused_kernel(PlanParams 
         cnt[i] = 0;
         mk[i] = 0;
     }
-    // the chunk's ids: 16-byte loads, all of a thread's in flight together
-    // (from pair p0 & ~3 on, so the loads are aligned; the few before p0 are
-    // the previous chunk's and are not used), then the last < 4 one by one
-    int bad = 0;
-    {
-        const int q0 = p0 >> 2, q1 = (p0 + n) >> 2;  // 16-byte words wholly or partly before p0 + n
-        const bool vec = (reinterpret_cast<uintptr_t>(a.topk) & 15) == 0;
-        const int nv = vec ? q1 - q0 : 0;
-        const int4 *src = reinterpret_cast<const int4 *>(a.topk) + q0;
-        constexpr int VB = 4;
-        for (int k0 = tid; k0 < nv; k0 += VB * nt) {
-            int4 v[VB];
-#pragma unroll
-            for (int j = 0; j < VB; ++j)
-                if (k0 + j * nt < nv) v[j] = __ldg(src + k0 + j * nt);
-#pragma unroll
-            for (int j = 0; j < VB; ++j) {
-                const int k = k0 + j * nt;
-                if (k < nv) {
-                    reinterpret_cast<int4 *>(ids_raw)[k] = v[j];
-                    const int q = 4 * (q0 + k);  // pair of v[j].x
-                    const int x[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
-#pragma unroll
-                    for (int c = 0; c < 4; ++c)
-                        if (q + c >= p0) bad |= x[c] < 0 || x[c] >= E;
-                }
-            }
-        }
-        for (int i = (vec ? max(4 * q1 - p0, 0) : 0) + tid; i < n; i += nt) {
-            const int e = __ldg(a.topk + p0 + i);
-            ids[i] = e;
-            bad |= e < 0 || e >= E;
-        }
-    }
+    const int bad = stage_ids(a.topk, p0, n, E, ids_raw, ids);
     if (tid == 0) s_seq = ld_cg(a.hdr + WS_SEQ);
-    bad = __syncthreads_or(bad);
+    const int any_bad = __syncthreads_or(bad);
     const int seq = s_seq, parity = seq & 1;
     {  // the previous call's group counts are read by nobody now: zero them for the next call
         int *old = a.gs + (size_t)(parity ^ 1) * a.gs_buf;
@@ -1837,7 +1859,7 @@ __global__ void __launch_bounds__(PLAN_THREADS, 1) plan_fused_kernel(PlanParams 
     __syncthreads();
     int mine = 0;
     if (tid == 0) {
-        if (bad) atomicOr(a.hdr + WS_STATUS, MOONEP_ST_EXPERT_ID_RANGE);
+        if (any_bad) atomicOr(a.hdr + WS_STATUS, MOONEP_ST_EXPERT_ID_RANGE);
         __threadfence();
         mine = atomicAdd(a.hdr + WS_TICKET, 1) + 1;
     }
@@ -1967,7 +1989,7 @@ __global__ void __launch_bounds__(PLAN_THREADS, 1) plan_fused_kernel(PlanParams 
         }
         __syncthreads();
         remote = assign_pass_b_fused(ids, dw + warp * E, dlim, hptr, hstart, hdst, wbeg, wend, p0, E, R * C, C, a.fC,
-                                     a.p.dst_pos, a.p.row_src, a.hdr + WS_FLAGS);
+                                     -1, a.p.dst_pos, a.p.row_src, a.hdr + WS_FLAGS);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) remote += __shfl_xor_sync(FULL_MASK, remote, o);
@@ -2019,7 +2041,7 @@ __global__ void __launch_bounds__(PLAN_THREADS, 1) plan_fused_kernel(PlanParams 
 // launch needs more dynamic shared memory than was allowed so far: the
 // driver calls cost host time on every plan of a latency-bound layer.
 constexpr int SMEM_CACHE_DEVICES = 64;
-enum { K_HIST, K_ASSIGN, K_EP_COUNT, K_EP_PLAN, K_EP_ASSIGN, K_FUSED, K_N };
+enum { K_HIST, K_ASSIGN, K_EP_COUNT, K_EP_PLAN, K_EP_ASSIGN, K_FUSED, K_EP_FUSED, K_N };
 static std::atomic<size_t> g_smem_set[SMEM_CACHE_DEVICES][K_N];  // bytes allowed so far, 0 = never set
 
 static bool set_smem(int which, const void *fn, size_t bytes)
@@ -2290,7 +2312,7 @@ __device__ __forceinline__ int assign_pass_b_local(const int *ids, const int *wb
                                                    const int *hstart, const int *hdst, const int *hloc,
                                                    const int *hq, const int *own, const int *before,
                                                    const int *G, int wbeg, int wend, int p0, int E, int rows,
-                                                   int C, int rank, int *dst_pos, int *info)
+                                                   int C, int rank, int *dst_pos, int *status)
 {
     const int lane = threadIdx.x & 31;
     int remote = 0;
@@ -2312,7 +2334,7 @@ __device__ __forceinline__ int assign_pass_b_local(const int *ids, const int *wb
         }
         const int p = p0 + i;
         if (dst < 0 || dst >= rows) {  // cannot happen for a consistent plan
-            atomicOr(info + MOONEP_INFO_STATUS, MOONEP_ST_ROW_RANGE);
+            atomicOr(status, MOONEP_ST_ROW_RANGE);
             dst_pos[p] = -1;
             continue;
         }
@@ -2404,7 +2426,7 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) ep_assign_kernel(PlanParams
         }
         __syncthreads();
         remote = assign_pass_b_local(ids, cnt + warp * E, hptr, hstart, hdst, hloc, hq, own, before, G, wbeg, wend,
-                                     p0, E, R * C, C, rank, a.p.dst_pos, a.p.info);
+                                     p0, E, R * C, C, rank, a.p.dst_pos, a.p.info + MOONEP_INFO_STATUS);
     } else {
         remote = assign_pass_b(ids, cnt + warp * E, hptr, hstart, hdst, wbeg, wend, p0, E, R * C, C, a.fC, rank,
                                a.p.dst_pos, nullptr, a.p.info + MOONEP_INFO_STATUS);
@@ -2417,6 +2439,199 @@ __global__ void __launch_bounds__(ASSIGN_THREADS, 2) ep_assign_kernel(PlanParams
         int s = 0;
         for (int w = 0; w < (nt >> 5); ++w) s += red[w];
         if (s) atomicAdd(a.p.info + MOONEP_INFO_N_REMOTE_PAIRS, s);
+    }
+}
+
+// ------------------------------------------------- expert parallelism, one kernel
+//
+// In expert parallelism the plan's inputs, the gathered counts [R][E+1], are
+// complete before the planner starts, so every CTA can plan at once: one
+// launch over the rank's token chunks (the chunking of moonep_ep_count), each
+// CTA staging its chunk's ids and ranking them (pass A), summing the expert
+// totals and its chunk's base (the lower ranks' counts and this rank's
+// earlier chunks') from the gathered rows, running the planner in its own
+// shared memory and placing its pairs (pass B, or the locality-aware pass B).
+// No CTA waits for another, so none needs the others resident.  One CTA (the
+// last chunk's) writes the small tables, each CTA the slot-table rows of the
+// ranks it owns (r mod chunks), and the CTA that finishes last (EP_DONE) the
+// info block.
+enum { EP_DONE = 9 };
+
+__host__ __device__ inline int ep_fused_smem_ints(int E, int R, int max_pairs, unsigned flags, int B)
+{
+    const int nh = 2 * E + R;
+    return ASSIGN_WARPS * E + (max_pairs + 4) + (E + 1) + 2 * nh + 32 + (E + 1) + 3 * nh + 3 * E +
+           plan_smem_ints(E, R) + ((flags & MOONEP_FLAG_CASCADE) ? cascade_smem_ints(E, R, B) : 0);
+}
+
+__global__ void __launch_bounds__(PLAN_THREADS, 1) ep_fused_kernel(PlanParams a, int rank)
+{
+    extern __shared__ __align__(16) int sm[];
+    const Dims &d = a.d;
+    const int E = d.E, K = d.K, R = d.R, C = d.C;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int nt = PLAN_THREADS;
+    const int chunk = blockIdx.x, nchunk = gridDim.x;
+    const int t0 = chunk * d.chunk_tokens, t1 = min(t0 + d.chunk_tokens, d.S);
+    const int p0 = t0 * K, n = (t1 - t0) * K;
+    const int max_pairs = d.chunk_tokens * K;
+    const int nh = 2 * E + R;
+    const bool locality = (d.flags & MOONEP_FLAG_LOCALITY) != 0;
+
+    int *cnt = sm;                          // ASSIGN_WARPS * E: warp counts, then warp bases
+    int *ids_raw = cnt + ASSIGN_WARPS * E;  // max_pairs + 4
+    int *ids = ids_raw + (p0 & 3);
+    int *hptr = ids_raw + max_pairs + 4;    // E + 1
+    int *hstart = hptr + E + 1;             // nh
+    int *hdst = hstart + nh;                // nh; first each expert's pairs before this chunk
+    int *red = hdst + nh;                   // 32
+    int *dlim = red + 32;                   // E + 1
+    int *hloc = dlim + E + 1;               // nh: each host's local pairs, quota, rank
+    int *hq = hloc + nh;                    // nh
+    int *hr = hq + nh;                      // nh
+    int *own = hr + nh;                     // E: the expert's host on this rank, or -1
+    int *before = own + E;                  // E: local pairs of the hosts on ranks <= rank
+    int *G = before + E;                    // E: the expert's pairs on lower ranks
+    int *psm = G + E;                       // the planner's; first pass A's lane masks
+    unsigned *mk = reinterpret_cast<unsigned *>(psm);
+    int *T = psm;
+    const int *misc = plan_misc(psm, E, R);
+
+    pdl_wait();  // the producer of the ids and of the gathered counts
+    for (int i = tid; i < ASSIGN_WARPS * E; i += nt) {
+        cnt[i] = 0;
+        mk[i] = 0;
+    }
+    stage_ids(a.topk, p0, n, E, ids_raw, ids);  // invalid ids are in the gathered counts' slot E
+    __syncthreads();
+    const int per = (n + ASSIGN_WARPS - 1) / ASSIGN_WARPS;
+    const int wbeg = min(warp * per, n), wend = min(wbeg + per, n);
+    assign_pass_a_mask(ids, cnt + warp * E, mk + warp * E, wbeg, wend, E);
+    __syncthreads();
+
+    // totals, the lower ranks' pairs and this chunk's base, from the gathered
+    // rows and this rank's per-chunk counts
+    int bad = 0, negative = 0;
+    unsigned part = 0;  // <= 2 values < 2^31 each (negative ones are flagged)
+    for (int r = tid; r < R; r += nt) bad |= ld_cg(a.gs + (size_t)r * a.gs_stride + E) != 0;
+    for (int e = tid; e < E; e += nt) {
+        int tot = 0, lower = 0;
+        for (int r0 = 0; r0 < R; r0 += 32) {
+            int v[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = r0 + j < R ? ld_cg(a.gs + (size_t)(r0 + j) * a.gs_stride + e) : 0;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                tot += v[j];
+                lower += r0 + j < rank ? v[j] : 0;
+            }
+        }
+        T[e] = tot;
+        G[e] = lower;
+        hdst[e] = lower + sum_strided<32>(a.cc + e, E, chunk);
+        negative |= tot < 0;
+        part += (unsigned)tot;
+    }
+    {
+        const unsigned lo = __reduce_add_sync(FULL_MASK, part & 0xffffu);
+        const unsigned hi = __reduce_add_sync(FULL_MASK, part >> 16);
+        if (lane == 0) {
+            red[warp] = (int)lo;
+            red[16 + warp] = (int)hi;
+        }
+    }
+    bad = __syncthreads_or(bad);
+    negative = __syncthreads_or(negative);
+    int status_in = bad ? MOONEP_ST_EXPERT_ID_RANGE : 0;
+    {
+        const unsigned lo = __reduce_add_sync(FULL_MASK, lane < ASSIGN_WARPS ? (unsigned)red[lane] : 0u);
+        const unsigned hi = __reduce_add_sync(FULL_MASK, lane < ASSIGN_WARPS ? (unsigned)red[16 + lane] : 0u);
+        const long long total = ((long long)hi << 16) + (long long)lo;
+        if (!bad && (negative || total != (long long)d.pairs)) status_in |= MOONEP_ST_WORKSPACE;
+    }
+    for (int e = tid; e < E; e += nt) {
+        int sb = hdst[e];
+        for (int w = 0; w < ASSIGN_WARPS; ++w) {
+            const int t = cnt[w * E + e];
+            cnt[w * E + e] = sb;
+            sb += t;
+        }
+    }
+    const bool writer = chunk == nchunk - 1;
+    if (writer)
+        for (int e = tid; e < E; e += nt) a.p.expert_count[e] = T[e];
+    __syncthreads();
+
+    const bool empty = (status_in & ST_EMPTY_PLAN) != 0;
+    int remote = 0;
+    if (empty) {
+        write_empty_plan(a, p0, n, false);  // row_src is not this rank's to write
+    } else {
+        PlanSink sink{false, writer, hptr, hstart, hdst};
+        if (locality) {
+            sink.hloc = hloc;
+            sink.hq = hq;
+            sink.hr = hr;
+        }
+        plan_core(a, psm, 0, sink);
+        __syncthreads();
+        if (locality) {
+            for (int e = tid; e < E; e += nt) {
+                int o = -1, b = 0;
+                for (int h = hptr[e]; h < hptr[e + 1]; ++h) {
+                    if (hr[h] <= rank) b += hloc[h];
+                    if (hr[h] == rank) o = h;
+                }
+                own[e] = o;
+                before[e] = b;
+            }
+            __syncthreads();
+            remote = assign_pass_b_local(ids, cnt + warp * E, hptr, hstart, hdst, hloc, hq, own, before, G, wbeg,
+                                         wend, p0, E, R * C, C, rank, a.p.dst_pos, a.hdr + WS_FLAGS);
+        } else {
+            int *dw = cnt;
+            for (int e = tid; e < E; e += nt) {
+                const int h0 = hptr[e], d0 = hdst[h0];
+#pragma unroll 4
+                for (int w = 0; w < ASSIGN_WARPS; ++w) dw[w * E + e] = d0 + cnt[w * E + e];
+                dlim[e] = hptr[e + 1] - h0 > 1 ? d0 + hstart[h0 + 1] : INT_MAX;
+            }
+            __syncthreads();
+            remote = assign_pass_b_fused(ids, dw + warp * E, dlim, hptr, hstart, hdst, wbeg, wend, p0, E, R * C, C,
+                                         a.fC, rank, a.p.dst_pos, nullptr, a.hdr + WS_FLAGS);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) remote += __shfl_xor_sync(FULL_MASK, remote, o);
+    if (lane == 0) red[warp] = remote;
+    __syncthreads();
+    if (tid == 0) {
+        int sr = 0;
+        for (int w = 0; w < ASSIGN_WARPS; ++w) sr += red[w];
+        if (sr) atomicAdd(a.hdr + WS_REMOTE, sr);
+        __threadfence();
+        if (atomicAdd(a.hdr + EP_DONE, 1) == nchunk - 1) {
+            __threadfence();
+            const int late = atomicExch(a.hdr + WS_FLAGS, 0);
+            const int remote_all = atomicExch(a.hdr + WS_REMOTE, 0);
+            int *info = a.p.info;
+            for (int i = 1; i < MOONEP_INFO_LEN; ++i) info[i] = 0;
+            if (empty) {
+                info[MOONEP_INFO_STATUS] = status_in | late;
+            } else {
+                info[MOONEP_INFO_STATUS] = misc[MISC_PLAN_STATUS] | late;
+                info[MOONEP_INFO_N_REP] = misc[MISC_N_REP];
+                info[MOONEP_INFO_N_OVERFLOW] = misc[MISC_N_OVER];
+                info[MOONEP_INFO_N_PIECES] = misc[MISC_N_PIECES];
+                info[MOONEP_INFO_N_RECEIVERS] = misc[MISC_N_RECEIVERS];
+                info[MOONEP_INFO_MAX_REP_PER_RANK] = misc[MISC_MAX_REP];
+                info[MOONEP_INFO_N_REP_EXPERTS] = misc[MISC_N_REP_EXPERTS];
+                info[MOONEP_INFO_N_REMOTE_PAIRS] = remote_all;
+                info[MOONEP_INFO_CASCADE_GUARD_STEPS] = misc[MISC_GUARD_STEPS];
+                info[MOONEP_INFO_CASCADE_GUARD_SLACK] = misc[MISC_GUARD_SLACK];
+            }
+            a.hdr[EP_DONE] = 0;
+        }
     }
 }
 
@@ -2466,15 +2681,32 @@ int launch_ep_plan(const Dims &d, int rank, const int32_t *topk, const int32_t *
     a.spin_limit = 0;
     a.cascade_cap = cascade_cap_for(d);
 
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+
+    // one kernel wherever its shared memory fits (no CTA waits for another,
+    // so residency does not matter)
+    const size_t smemf = sizeof(int) * (size_t)ep_fused_smem_ints(d.E, d.R, d.chunk_tokens * d.K, d.flags, d.B);
+    if (g_plan_path.load(std::memory_order_relaxed) == 0 && smemf <= MAX_BLOCK_SMEM &&
+        set_smem(K_EP_FUSED, (const void *)ep_fused_kernel, smemf)) {
+        cudaLaunchConfig_t cf = {};
+        cf.gridDim = dim3(d.nchunk);
+        cf.blockDim = dim3(PLAN_THREADS);
+        cf.dynamicSmemBytes = smemf;
+        cf.stream = st;
+        cf.attrs = attr;
+        cf.numAttrs = 1;
+        return cudaLaunchKernelEx(&cf, ep_fused_kernel, a, rank) == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
+    }
+    (void)cudaGetLastError();
+
     const size_t smem1 = sizeof(int) * (size_t)(plan_smem_ints(d.E, d.R) +
                                                 ((d.flags & MOONEP_FLAG_CASCADE) ? cascade_smem_ints(d.E, d.R, d.B) : 0));
     if (!set_smem(K_EP_PLAN, (const void *)ep_plan_kernel, smem1)) return MOONEP_ERR_CUDA;
     ep_plan_kernel<<<1, PLAN_THREADS, smem1, st>>>(a);
     if (cudaGetLastError() != cudaSuccess) return MOONEP_ERR_CUDA;
 
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
     const size_t smem2 = sizeof(int) * (size_t)ep_assign_smem_ints(d.E, d.R, d.chunk_tokens * d.K);
     if (!set_smem(K_EP_ASSIGN, (const void *)ep_assign_kernel, smem2)) return MOONEP_ERR_CUDA;
     cudaLaunchConfig_t c = {};

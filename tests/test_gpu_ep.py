@@ -38,6 +38,16 @@ def mp(oracle_lib, cuda_lib_path):
     return moonep
 
 
+@pytest.fixture(autouse=True, params=["one-kernel", "two-kernel"])
+def plan_path(request, mp):
+    """Every test runs under both expert-parallel planners
+    (moonep_set_plan_path): one kernel in which every CTA plans from the
+    gathered counts, and the planner CTA followed by the assignment grid."""
+    prev = mp.set_plan_path(1 if request.param == "two-kernel" else 0)
+    yield request.param
+    mp.set_plan_path(prev)
+
+
 def _ep_plans(mp, cfg, topk):
     """Count, gather (stacking the rows) and plan on every simulated rank."""
     R, S = cfg.R, cfg.S

@@ -118,3 +118,26 @@ def test_ids_not_16_byte_aligned(mp, wname, shift):
     gp = mp.plan(gcfg, view)
     torch.cuda.synchronize()
     _assert_equal(gp, oracle.plan(ocfg, topk.cpu().numpy()), f"{wname} shift {shift}")
+
+
+def test_expert_parallel_plan_launches_the_chosen_planner(mp):
+    # moonep_ep_plan: one kernel by default (every CTA plans from the
+    # gathered counts), the planner CTA then the assignment grid with path 1
+    R, E, K, S = 8, 64, 4, 512
+    cfg = mp.Config(R=R, E=E, K=K, S=S, H=64, B=4)
+    gen = torch.Generator(device="cpu").manual_seed(7)
+    topk = torch.stack([torch.randperm(E, generator=gen)[:K] for _ in range(R * S)]).to(torch.int32).to(DEV)
+    plans = [mp.Plan(cfg, DEV, ep=True) for _ in range(R)]
+    counts = torch.zeros((R, E + 1), dtype=torch.int32, device=DEV)
+    torch.cuda.synchronize()
+    for r in range(R):
+        mp.ep_count(cfg, topk[r * S:(r + 1) * S].contiguous(), plans[r], counts_row=counts[r])
+    prev = mp.set_plan_path(0)
+    try:
+        one = _kernels(lambda: mp.ep_plan(cfg, 0, topk[:S].contiguous(), counts, plans[0]))
+        mp.set_plan_path(1)
+        two = _kernels(lambda: mp.ep_plan(cfg, 0, topk[:S].contiguous(), counts, plans[0]))
+    finally:
+        mp.set_plan_path(prev)
+    assert any("ep_fused_kernel" in k for k in one) and not any("ep_plan_kernel" in k for k in one), one
+    assert any("ep_plan_kernel" in k for k in two) and any("ep_assign_kernel" in k for k in two), two

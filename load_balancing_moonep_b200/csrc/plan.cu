@@ -5,8 +5,19 @@
 // redundant experts") fixes what the plan must achieve -- every rank gets
 // exactly S*K token slots, by replicating a few experts online from the
 // router output -- and calls the planner near-optimal without giving it.
-// This file implements the water-filling plan described in moonep.h in two
-// launches, with no host synchronisation:
+// This file implements the water-filling plan described in moonep.h, with no
+// host synchronisation, in one of two ways that give the same plan:
+//
+//   plan_fused_kernel (the default) one CTA per SM and token chunk: every CTA
+//                     counts its chunk, takes a ticket, sums the totals once
+//                     every chunk's counts are in, runs the planner (plan_core)
+//                     in its own shared memory and places its own pairs from
+//                     its own host tables; ep_fused_kernel is its expert-
+//                     parallel form, which needs no ticket (the gathered
+//                     counts are complete before it starts).
+//
+// or, where the planner's shared memory does not fit beside a chunk, in two
+// launches:
 //
 //   hist_plan_kernel  one CTA per token chunk stages the chunk's ids in
 //                     shared memory and counts them with shared-memory

@@ -237,6 +237,22 @@ def barrier(world):
 SPACER_CYCLES = 100_000
 
 
+def count_library_launches(fn):
+    """Kernels of this library one call of fn launches (a profiler trace of
+    one untimed step): (count, how), or (None, reason)."""
+    try:
+        from torch.profiler import ProfilerActivity, profile
+        torch.cuda.synchronize()
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            fn()
+            torch.cuda.synchronize()
+        n = sum(1 for e in prof.events()
+                if e.device_type == torch.autograd.DeviceType.CUDA and "moonep::" in e.name)
+        return n, "profiler trace of one untimed step: kernels named moonep::"
+    except Exception as exc:  # profiler unavailable
+        return None, f"no profiler trace: {type(exc).__name__}: {str(exc)[:120]}"
+
+
 def max_over_ranks(world, x: float) -> float:
     if world <= 1:
         return x
@@ -907,7 +923,10 @@ def run_ours(args, world, rank, local):
                                      f"elements, rows of 2^18 of the {wl.grad_elems} gradient elements")},
                "gpu_dispatch+combine_tok/s": round(gpu_tok)}
 
-    launches_per_step = 2 + 1 + 1 + 1 + (1 if P else 0)
+    launches_per_step, launches_how = count_library_launches(lambda: step(None))
+    if launches_per_step is None:  # no profiler: the planner's one kernel and the data kernels
+        launches_per_step = 1 + 1 + 1 + 1 + (1 if P else 0)
+        launches_how = "static count (" + launches_how + ")"
     cfgd = workload_config(wl, r, args)
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
@@ -923,6 +942,7 @@ def run_ours(args, world, rank, local):
                                   "us": round(other_plan_us, 2)},
         "roofline": roofline, "kernels": kernels, "sweep": sweep,
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches_how": launches_how,
         "decode": decode, "workloads": workloads, "ep_one_gpu": ep,
         "cascade": cascade, "clocks": clocks, "plan_info": info,
         "reduce": (f"P={P} fp32 ({reduce_note}), {n_pref} prefetched replicas over "

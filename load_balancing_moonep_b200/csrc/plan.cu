@@ -1780,14 +1780,16 @@ __device__ __forceinline__ int stage_ids(const int32_t *topk, int p0, int n, int
 // ------------------------------------------------------- one-kernel planner
 //
 // When one CTA per SM can hold a chunk of about tokens / SMs tokens beside
-// the planner's shared memory, one launch does the whole plan.  Every CTA stages its chunk's ids, ranks them (pass A),
-// adds the chunk's counts to its group's and takes a ticket.  Once every
-// chunk's counts are in, it sums the expert totals and its chunk's base, runs
-// the planner on them in its own shared memory -- every CTA computes the same
-// plan, so no CTA waits for another's tables -- and places its pairs from its
-// own copy of the host tables (pass B).  One CTA (the last chunk's, which has
-// the fewest pairs) stores the plan tables; the CTA that finishes last writes
-// the info block and resets the header for the next call.  One CTA per SM,
+// the planner's shared memory, one launch does the whole plan.  Every CTA
+// stages its chunk's ids, ranks them (pass A), adds the chunk's counts to its
+// group's and takes a ticket.  Once every chunk's counts are in, it sums the
+// expert totals and its chunk's base, runs the planner on them in its own
+// shared memory -- every CTA computes the same plan, so no CTA waits for
+// another's tables -- and places its pairs from its own copy of the host
+// tables (pass B).  Each CTA writes the slot-table rows of the ranks it owns
+// (r mod chunks), one CTA (the last chunk's, which has the fewest pairs) the
+// other tables, and the CTA that finishes last writes the info block and
+// resets the header for the next call.  One CTA per SM,
 // not two with half the tokens each: the planner is a chain of short
 // dependent steps, and two of them on one SM take nearly twice as long.
 // The chunking is this kernel's own (at most one chunk per SM); the group

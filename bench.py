@@ -551,6 +551,12 @@ def run_ours(args, world, rank, local):
     step_ms_local = t_start.elapsed_time(t_end) / args.steps
     ms_per_step = max_over_ranks(world, step_ms_local)
 
+    # this library's kernels in one untimed step
+    launches_per_step, launches_how = count_library_launches(lambda: step(None))
+    if launches_per_step is None:  # no profiler: the planner's one kernel and the data kernels
+        launches_per_step = 1 + 1 + 1 + 1 + (1 if P else 0)
+        launches_how = "static count (" + launches_how + ")"
+
     # the same step with the other planner, for comparison (its plan time
     # only; the data kernels do not depend on which planner made the plan)
     other = 1 - mp.set_plan_path(1 - args.plan_path)
@@ -923,10 +929,6 @@ def run_ours(args, world, rank, local):
                                      f"elements, rows of 2^18 of the {wl.grad_elems} gradient elements")},
                "gpu_dispatch+combine_tok/s": round(gpu_tok)}
 
-    launches_per_step, launches_how = count_library_launches(lambda: step(None))
-    if launches_per_step is None:  # no profiler: the planner's one kernel and the data kernels
-        launches_per_step = 1 + 1 + 1 + 1 + (1 if P else 0)
-        launches_how = "static count (" + launches_how + ")"
     cfgd = workload_config(wl, r, args)
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,

@@ -1052,12 +1052,10 @@ __device__ void plan_core(const PlanParams &a, int *sm, int seq, const PlanSink 
     //        prefetched-replica flag per expert (E) | 0]
     // Rank r's used slots sit at rank_base(r) .. (home slots, then replicas).
     int *Z = hr;     // 4E + R + 2 <= 3 nh ints, free after the sort
-    int *rq_j = scr;  // n_rep <= E + R - 1: piece of each replica (scr is free)
     const int zh = E + n_rep, zf = zh + E + 1, nz = zf + E + 1;
 #pragma unroll 1
     for (int q = tid; q < n_rep; q += nt) {
         const int j = last_le(segb, nP, q);
-        rq_j[q] = j;
         const int i = pilo[j] + (q - segb[j]);
         const int ord = j - jlo[i];
         const int r = qr[i];
@@ -1120,49 +1118,8 @@ __device__ void plan_core(const PlanParams &a, int *sm, int seq, const PlanSink 
     // of e), and its start is in the order of the pairs left over.
     const bool locality = (d.flags & MOONEP_FLAG_LOCALITY) != 0;
     auto own_pairs = [&](int r, int e) { return ld_cg(a.gs + (size_t)r * a.gs_stride + e); };
-#pragma unroll 1
-    for (int x = tid; x < n_hosts; x += nt) {
-        int e, r0, slot, quota, j, pos = 0, st = 0, locsum = 0;
-        if (x < E) {
-            e = x;
-            r0 = (int)fdiv((uint32_t)e, a.fL);
-            slot = e - r0 * L;
-            quota = keep[e];
-            j = pof[e];
-        } else {
-            const int q = x - E;
-            j = rq_j[q];
-            const int i = pilo[j] + (q - segb[j]);
-            e = pe[j];
-            r0 = qr[i];
-            slot = L + (j - jlo[i]);
-            quota = seg_q(j, i);
-            const int home = (int)fdiv((uint32_t)e, a.fL);
-            if (home < r0) {  // the home rank is lower
-                pos = 1;
-                st = keep[e];
-                if (locality) locsum = min(keep[e], own_pairs(home, e));
-            }
-        }
-        if (j >= 0) {
-            // the other hosts of e on lower ranks (a hot expert has tens of
-            // them, and every host walks them all: the loads of four steps
-            // are in flight together)
-            const int ns = segb[j + 1] - segb[j], i0 = pilo[j], ps0 = PS[j], ps1 = PS[j + 1];
-#pragma unroll 4
-            for (int s = 0; s < ns; ++s) {
-                const int i = i0 + s, ri = qr[i];
-                if (ri < r0) {
-                    ++pos;
-                    const int qi = min(ps1, QSr[i + 1] - qbase) - max(ps0, QSr[i] - qbase);
-                    st += qi;
-                    if (locality) locsum += min(qi, own_pairs(ri, e));
-                }
-            }
-        }
-        const int loc = locality ? min(quota, own_pairs(r0, e)) : 0;
-        st -= locsum;
-        const int h = hptr(e) + pos;
+    // host h of e: rank r0, slot, quota, start st, local pairs loc
+    auto put_host = [&](int e, int h, int r0, int slot, int quota, int st, int loc) {
         const int b0 = rank_base(r0);
         if (wr) {
             a.p.host_rank[h] = r0;
@@ -1181,6 +1138,65 @@ __device__ void plan_core(const PlanParams &a, int *sm, int seq, const PlanSink 
                 sink.hloc[h] = loc;
                 sink.hq[h] = quota;
                 sink.hr[h] = r0;
+            }
+        }
+    };
+    // an expert with no replica: its home is its one host, at start 0
+#pragma unroll 1
+    for (int e = tid; e < E; e += nt) {
+        if (pof[e] >= 0) continue;
+        const int r0 = (int)fdiv((uint32_t)e, a.fL);
+        put_host(e, hptr(e), r0, e - r0 * L, keep[e], 0, locality ? min(keep[e], own_pairs(r0, e)) : 0);
+    }
+    // a replicated expert (piece j): one warp, its hosts (the home, then the
+    // piece's receivers) as lanes, 32 at a time; a host's position and start
+    // are the count and the quota sum of the expert's hosts on lower ranks,
+    // broadcast 32 at a time by shuffles (a hot expert has tens of hosts; one
+    // thread per host walking all of them took 6 µs at the decode shape)
+    auto host_of_piece = [&](int j, int e, int home, int k, int &r, int &q) {
+        if (k == 0) {
+            r = home;
+            q = keep[e];
+        } else {
+            const int i = pilo[j] + k - 1;
+            r = qr[i];
+            q = seg_q(j, i);
+        }
+    };
+#pragma unroll 1
+    for (int j = warp; j < nP; j += nwarp) {
+        const int e = pe[j], home = (int)fdiv((uint32_t)e, a.fL);
+        const int nhost = segb[j + 1] - segb[j] + 1;
+#pragma unroll 1
+        for (int k0 = 0; k0 < nhost; k0 += 32) {
+            const int k = k0 + lane;
+            int rk = 0, qk = 0;
+            if (k < nhost) host_of_piece(j, e, home, k, rk, qk);
+            int pos = 0, st = 0, locsum = 0;
+#pragma unroll 1
+            for (int m0 = 0; m0 < nhost; m0 += 32) {
+                const int m = m0 + lane;
+                int rm = INT_MAX, qm = 0, lm = 0;
+                if (m < nhost) {
+                    host_of_piece(j, e, home, m, rm, qm);
+                    if (locality) lm = min(qm, own_pairs(rm, e));
+                }
+                const int tn = min(32, nhost - m0);  // the hosts in this round (warp-uniform)
+#pragma unroll 4
+                for (int t = 0; t < tn; ++t) {
+                    const int r_ = __shfl_sync(FULL_MASK, rm, t), q_ = __shfl_sync(FULL_MASK, qm, t);
+                    const int l_ = locality ? __shfl_sync(FULL_MASK, lm, t) : 0;
+                    if (r_ < rk) {
+                        ++pos;
+                        st += q_;
+                        locsum += l_;
+                    }
+                }
+            }
+            if (k < nhost) {
+                const int slot = k == 0 ? e - home * L : L + (j - jlo[pilo[j] + k - 1]);
+                const int loc = locality ? min(qk, own_pairs(rk, e)) : 0;
+                put_host(e, hptr(e) + pos, rk, slot, qk, st - locsum, loc);
             }
         }
     }

@@ -141,3 +141,48 @@ def test_expert_parallel_plan_launches_the_chosen_planner(mp):
         mp.set_plan_path(prev)
     assert any("ep_fused_kernel" in k for k in one) and not any("ep_plan_kernel" in k for k in one), one
     assert any("ep_plan_kernel" in k for k in two) and any("ep_assign_kernel" in k for k in two), two
+
+
+@pytest.mark.parametrize("path", [0, 1])
+def test_plan_is_exact_while_other_streams_hold_sms(mp, path):
+    # Sleeping one-block kernels on 140 other streams hold SMs (the one-kernel
+    # planner's CTAs each need a whole SM) for about 20 ms while the plan
+    # runs with a short wait bound: CTAs that cannot all be resident take the
+    # fallback (the one kernel counts every pair itself, the two-kernel pass
+    # waits for the histogram grid), and the plan must still be the oracle's
+    # (MOONEP_ST_WAIT_TIMEOUT may be set, nothing else may differ; on a B200
+    # the one-kernel planner's CTAs did time out in this setting).  Every wait
+    # in the library is bounded, and nothing here waits on the plan.
+    wl = W.WORKLOADS["large"]
+    gcfg, ocfg = _cfg(mp, wl)
+    topk = W.routing(wl, 1.0, device=DEV).topk_idx
+    op = oracle.plan(ocfg, topk.cpu().numpy())
+    p = mp.Plan(gcfg)
+    streams = [torch.cuda.Stream() for _ in range(140)]
+    torch.cuda.synchronize()
+    prev_limit = mp.set_wait_limit(2000)
+    prev_path = mp.set_plan_path(path)
+    try:
+        for s in streams:
+            with torch.cuda.stream(s):
+                torch.cuda._sleep(40_000_000)  # about 20 ms at 2 GHz
+        mp.plan(gcfg, topk, out=p)
+        torch.cuda.synchronize()
+    finally:
+        mp.set_wait_limit(prev_limit)
+        mp.set_plan_path(prev_path)
+    g = p.to_numpy()
+    for k, v in op.items():
+        if k == "info":
+            assert g[k][0] & ~mp.ST_WAIT_TIMEOUT == v[0]
+            assert np.array_equal(g[k][1:], v[1:])
+        else:
+            assert np.array_equal(g[k], v), f"plan field {k} differs"
+    # and the next plan, with the SMs free again, is exact without the bit
+    mp.set_plan_path(path)
+    try:
+        mp.plan(gcfg, topk, out=p)
+        torch.cuda.synchronize()
+    finally:
+        mp.set_plan_path(prev_path)
+    assert p.info()["status"] == op["info"][0]

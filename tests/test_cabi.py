@@ -119,3 +119,45 @@ def test_single_gpu_planner_refuses_the_locality_flag(cuda_lib_path):
     c = cfg.c()
     assert moonep._lib.moonep_plan(ctypes.byref(c), 1 << 20, ctypes.byref(cp), 1 << 20, None) == 1
     assert moonep._lib.moonep_plan_noalloc(ctypes.byref(c), 1 << 20, ctypes.byref(cp), None) == 1
+
+
+def test_host_setters_return_the_previous_setting(cuda_lib_path):
+    """The three process-wide settings are host-only: each call returns the
+    setting it replaces, and out-of-range values map as the header states
+    (a negative wait bound restores the default 65536 iterations, a capacity
+    <= 0 the plan's own E + R - 1 (reported as 0), any plan path other than 1
+    the default 0).  The binding refuses plan paths other than 0 and 1."""
+    import ctypes
+    from load_balancing_moonep_b200 import moonep
+    lib = ctypes.CDLL(cuda_lib_path)
+
+    prev = moonep.set_wait_limit(5)
+    try:
+        assert moonep.set_wait_limit(-1) == 5
+        assert moonep.set_wait_limit(0) == 65536
+        assert moonep.set_wait_limit(7) == 0
+        assert moonep.set_wait_limit(7) == 7
+    finally:
+        moonep.set_wait_limit(prev)
+
+    prev = moonep.set_cascade_capacity(10)
+    try:
+        assert moonep.set_cascade_capacity(-3) == 10
+        assert moonep.set_cascade_capacity(4) == 0
+        assert moonep.set_cascade_capacity(0) == 4
+        assert moonep.set_cascade_capacity(0) == 0
+    finally:
+        moonep.set_cascade_capacity(prev)
+
+    prev = moonep.set_plan_path(1)
+    try:
+        assert lib.moonep_set_plan_path(5) == 1  # the C entry maps it to 0
+        assert moonep.set_plan_path(0) == 0
+        assert moonep.set_plan_path(1) == 0
+        assert moonep.set_plan_path(1) == 1
+        for bad in (2, -1):
+            with pytest.raises(ValueError):
+                moonep.set_plan_path(bad)
+        assert moonep.set_plan_path(0) == 1  # the refused calls changed nothing
+    finally:
+        moonep.set_plan_path(prev)

@@ -1533,8 +1533,9 @@ __device__ __forceinline__ int assign_pass_b(const int *ids, const int *wb, cons
 // pair of rank loc in the warp's sub-range thus has row dw + loc, unless that
 // is past the first host, where the host intervals give it: two
 // shared-memory loads per pair on the common path, where the generic pass
-// makes about six.  Their random expert index makes each of them conflict,
-// and they bound this pass.  (Staging row_src in shared memory in (expert,
+// makes about six.  Their random expert index makes them conflict, but
+// halving them did not shorten this pass: the host search and the scattered
+// row_src stores take its time.  (Staging row_src in shared memory in (expert,
 // rank) order, so that its stores coalesce, measured 1.9 µs slower at the
 // large shape than these scattered stores.)
 // src_rank >= 0: the source rank of every pair (one rank's pairs, whose
